@@ -1,0 +1,189 @@
+"""Float64 CPU oracle for the Vision-RWKV spatial-mix core.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may use this package; the product path (the
+CUDA library and its Python binding) never imports, links or loads it, and
+this package imports nothing from the product.
+
+It wraps ``vrwkv_oracle.c`` (plain C, float64, OpenMP over channel columns):
+
+* ``qshift``        -- Q-Shift of "Vision-RWKV Backbone" (Quad-Directional
+                       Token Shift, eq. 9) with the group layout of the
+                       q_shift listing on "LinXin's Blog".
+* ``qshift_f32``    -- the same interpolation in binary32 with a fixed
+                       operation order, optionally rounded to bfloat16; used
+                       for bit-exact comparisons.
+* ``biwkv_direct``  -- Bi-WKV by direct summation of eq. 5 (O(T^2)).
+* ``biwkv_points``  -- eq. 5 at selected (b, t, c) positions.
+* ``biwkv_rnn``     -- Bi-WKV by the RNN form, eq. 6-7 (O(T)).
+* ``biwkv_rnn_literal`` -- eq. 6-7 with the subtract-and-divide update the
+                       page describes (short sequences only).
+* ``gate``          -- sigma(R) (.) wkv of eq. 2.
+* ``spatial_core``  -- gate(QS_R(r), Bi-WKV(QS_K(k), QS_V(v))).
+
+Every array is row-major (B, T, C) with token index t = h*W + w.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "vrwkv_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile vrwkv_oracle.c into liboracle.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        dp = ctypes.POINTER(ctypes.c_double)
+        fp = ctypes.POINTER(ctypes.c_float)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        ci, cd, cl = ctypes.c_int, ctypes.c_double, ctypes.c_long
+        lib.oracle_qshift_f64.argtypes = [dp, dp, dp, ci, ci, ci, ci, ci, cd, ci]
+        lib.oracle_qshift_f32.argtypes = [fp, fp, fp, ci, ci, ci, ci, ci, cd, ci]
+        lib.oracle_round_bf16.argtypes = [fp, fp, cl]
+        for name in ("oracle_biwkv_direct", "oracle_biwkv_rnn",
+                     "oracle_biwkv_rnn_literal"):
+            getattr(lib, name).argtypes = [dp, dp, dp, dp, dp, ci, ci, ci]
+        lib.oracle_biwkv_direct_points.argtypes = [dp, dp, dp, dp, ci, ci, ci,
+                                                   i64p, cl, dp]
+        lib.oracle_gate.argtypes = [dp, dp, dp, cl]
+        lib.oracle_num_threads.restype = ci
+        _lib = lib
+    return _lib
+
+
+def _d(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a: np.ndarray, ctype=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def qshift(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25,
+           mu=None, eq9_order: bool = False) -> np.ndarray:
+    """Q-Shift of x (B, H*W, C): X^dagger, or mu*X + (1-mu)*X^dagger."""
+    x = _d(x)
+    B, T, C = x.shape
+    assert T == H * W
+    out = np.empty_like(x)
+    mu_p = None
+    if mu is not None:
+        mu = _d(mu)
+        assert mu.shape == (C,)
+        mu_p = _ptr(mu)
+    _load().oracle_qshift_f64(_ptr(x), _ptr(out), mu_p, B, H, W, C,
+                              int(shift_pixel), float(gamma), int(eq9_order))
+    return out
+
+
+def qshift_f32(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25,
+               mu=None, round_bf16: bool = False) -> np.ndarray:
+    """Q-Shift in binary32 with the fixed operation order
+    t1 = mu*x, t2 = (1-mu)*x_dagger, out = t1 + t2 (each rounded), then an
+    optional round-to-nearest-even to bfloat16.  Returns float32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    B, T, C = x.shape
+    assert T == H * W
+    out = np.empty_like(x)
+    mu_p = None
+    if mu is not None:
+        mu = np.ascontiguousarray(mu, dtype=np.float32)
+        mu_p = _ptr(mu, ctypes.c_float)
+    _load().oracle_qshift_f32(_ptr(x, ctypes.c_float), _ptr(out, ctypes.c_float),
+                              mu_p, B, H, W, C, int(shift_pixel), float(gamma),
+                              int(round_bf16))
+    return out
+
+
+def round_bf16(a) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even)."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    out = np.empty_like(a)
+    _load().oracle_round_bf16(_ptr(a, ctypes.c_float), _ptr(out, ctypes.c_float),
+                              a.size)
+    return out
+
+
+def _biwkv(fn_name: str, k, v, w, u) -> np.ndarray:
+    k, v, w, u = _d(k), _d(v), _d(w), _d(u)
+    B, T, C = k.shape
+    assert v.shape == k.shape and w.shape == (C,) and u.shape == (C,)
+    out = np.empty_like(k)
+    getattr(_load(), fn_name)(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(out),
+                              B, T, C)
+    return out
+
+
+def biwkv_direct(k, v, w, u) -> np.ndarray:
+    """Bi-WKV by direct evaluation of eq. 5, O(B*C*T^2)."""
+    return _biwkv("oracle_biwkv_direct", k, v, w, u)
+
+
+def biwkv_rnn(k, v, w, u) -> np.ndarray:
+    """Bi-WKV by the RNN form of eq. 6-7, O(B*C*T)."""
+    return _biwkv("oracle_biwkv_rnn", k, v, w, u)
+
+
+def biwkv_rnn_literal(k, v, w, u) -> np.ndarray:
+    """Bi-WKV by eq. 6-7 with subtract-and-divide updates for b and d."""
+    return _biwkv("oracle_biwkv_rnn_literal", k, v, w, u)
+
+
+def biwkv_points(k, v, w, u, flat_idx) -> np.ndarray:
+    """eq. 5 evaluated only at flat indices (b*T + t)*C + c."""
+    k, v, w, u = _d(k), _d(v), _d(w), _d(u)
+    B, T, C = k.shape
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    out = np.empty(idx.shape[0], dtype=np.float64)
+    _load().oracle_biwkv_direct_points(
+        _ptr(k), _ptr(v), _ptr(w), _ptr(u), B, T, C,
+        idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), idx.shape[0],
+        _ptr(out))
+    return out
+
+
+def gate(r, wkv) -> np.ndarray:
+    """sigma(r) * wkv (eq. 2)."""
+    r, wkv = _d(r), _d(wkv)
+    out = np.empty_like(wkv)
+    _load().oracle_gate(_ptr(r), _ptr(wkv), _ptr(out), wkv.size)
+    return out
+
+
+def spatial_core(r, k, v, w, u, H=None, W=None, shift_pixel=1, gamma=0.25,
+                 mu_r=None, mu_k=None, mu_v=None, qshift_on=True,
+                 method: str = "direct") -> np.ndarray:
+    """sigma(QS_R(r)) * Bi-WKV(QS_K(k), QS_V(v)); without Q-Shift when
+    qshift_on is False.  method selects eq. 5 ("direct") or eq. 6-7 ("rnn")."""
+    if qshift_on:
+        r = qshift(r, H, W, shift_pixel, gamma, mu_r)
+        k = qshift(k, H, W, shift_pixel, gamma, mu_k)
+        v = qshift(v, H, W, shift_pixel, gamma, mu_v)
+    f = biwkv_direct if method == "direct" else biwkv_rnn
+    return gate(r, f(k, v, w, u))

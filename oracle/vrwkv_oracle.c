@@ -1,0 +1,332 @@
+/*
+ * Float64 CPU oracle for the Vision-RWKV spatial-mix core.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no code, header, table or constant
+ * with the CUDA library and includes nothing from it.
+ *
+ * Sources (page titles as given in the reference pages):
+ *   [VRWKV]  "OpenGVLab&港中文&复旦&南大&清华提出Vision-RWKV Backbone"
+ *            (cloud.tencent.com article 2395249):
+ *              - Linear Complexity Bidirectional Attention, eq. 5 (summation
+ *                form of Bi-WKV) and eq. 6-7 (RNN form, hidden states a,b,c,d);
+ *              - Quad-Directional Token Shift, eq. 9 (Q-Shift);
+ *              - Overall Architecture, eq. 2 (sigma(R) (.) wkv gate).
+ *   [BLOG]   "LinXin's Blog" (linxin.blog), Vision-RWKV entry: the q_shift
+ *            listing (patch_resolution, shift_pixel, gamma, zero-initialised
+ *            output, four slice assignments, copy of the remaining channels).
+ *
+ * Layout of every token tensor: row-major (B, T, C), channel fastest, token
+ * index t = h*W + w (the listing's transpose/reshape of (B,N,C) to (B,C,H,W)).
+ *
+ * Readings of the pages taken here (each also listed in the design notes):
+ *   - eq. 9 prints "X + (1-mu)X^dagger" but calls it a linear interpolation of
+ *     X and X^dagger; the interpolation mu*X + (1-mu)*X^dagger is computed.
+ *   - channel-group order follows the listing (w-s, w+s, h-s, h+s); eq. 9's
+ *     order (h-1, h+1, w-1, w+1) is available through eq9_order=1.
+ *   - g = int(C*gamma) truncates as Python int() does.
+ *   - a shift_pixel at or beyond the grid extent empties that group (zeros).
+ *   - the garbled "ki" in eq. 5 is k_i; T is the total token count.
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -shared -fPIC (see build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* Q-Shift: the gather X^dagger (eq. 9 and the q_shift listing)        */
+/* ------------------------------------------------------------------ */
+
+/* Source pixel of output pixel (h,w) for channel c, following the listing's
+ * slice assignments.  Returns 0 when the output stays at its zero initial
+ * value (border, or an emptied group), 1 with (*sh,*sw) set otherwise. */
+static int qshift_source(int c, int h, int w, int H, int W, int C, int s,
+                         double gamma, int eq9_order, int* sh, int* sw) {
+    int g = (int)((double)C * gamma); /* Python int(): truncation toward 0 */
+    int grp;
+    if (c < g) grp = 0;
+    else if (c < 2 * g) grp = 1;
+    else if (c < 3 * g) grp = 2;
+    else if (c < 4 * g) grp = 3;
+    else grp = 4; /* output[:, 4g:] = input[:, 4g:] */
+    if (eq9_order && grp < 4) {
+        /* eq. 9 order: h-1, h+1, w-1, w+1  ->  listing groups 2,3,0,1 */
+        static const int perm[4] = {2, 3, 0, 1};
+        grp = perm[grp];
+    }
+    int srch = h, srcw = w;
+    switch (grp) {
+    case 0: /* output[..., s:W] = input[..., 0:W-s]: value comes from w-s */
+        srcw = w - s;
+        break;
+    case 1: /* output[..., 0:W-s] = input[..., s:W]: value comes from w+s */
+        srcw = w + s;
+        break;
+    case 2: /* output[.., s:H, :] = input[.., 0:H-s, :]: from h-s */
+        srch = h - s;
+        break;
+    case 3: /* output[.., 0:H-s, :] = input[.., s:H, :]: from h+s */
+        srch = h + s;
+        break;
+    default:
+        break;
+    }
+    if (srch < 0 || srch >= H || srcw < 0 || srcw >= W) return 0;
+    *sh = srch;
+    *sw = srcw;
+    return 1;
+}
+
+/* out = X^dagger (mu == NULL) or mu*X + (1-mu)*X^dagger, in float64. */
+void oracle_qshift_f64(const double* x, double* out, const double* mu, int B,
+                       int H, int W, int C, int s, double gamma,
+                       int eq9_order) {
+    const long T = (long)H * W;
+#pragma omp parallel for schedule(static)
+    for (long bt = 0; bt < (long)B * T; ++bt) {
+        long b = bt / T, t = bt % T;
+        int h = (int)(t / W), w = (int)(t % W);
+        for (int c = 0; c < C; ++c) {
+            int sh, sw;
+            double xd = 0.0;
+            if (qshift_source(c, h, w, H, W, C, s, gamma, eq9_order, &sh, &sw))
+                xd = x[(b * T + (long)sh * W + sw) * C + c];
+            double xv = x[(b * T + t) * C + c];
+            out[(b * T + t) * C + c] =
+                mu ? mu[c] * xv + (1.0 - mu[c]) * xd : xd;
+        }
+    }
+}
+
+/* Round a float to the nearest bfloat16 (ties to even), returned as float.
+ * bfloat16 keeps the top 16 bits of the IEEE binary32 pattern. */
+static float round_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) { /* inf or nan */
+        if (u & 0x007fffffu) u |= 0x00400000u; /* keep nan quiet */
+        u &= 0xffff0000u;
+    } else {
+        uint32_t lsb = (u >> 16) & 1u;
+        u += 0x7fffu + lsb;
+        u &= 0xffff0000u;
+    }
+    float r;
+    memcpy(&r, &u, 4);
+    return r;
+}
+
+void oracle_round_bf16(const float* in, float* out, long n) {
+    for (long i = 0; i < n; ++i) out[i] = round_to_bf16(in[i]);
+}
+
+/* The interpolation evaluated in binary32 with each operation rounded on its
+ * own (t1 = mu*x, t2 = (1-mu)*x^dagger, out = t1 + t2; no fused multiply-add,
+ * enforced by -ffp-contract=off), then optionally rounded to bfloat16.  This
+ * is the fixed operation order the bit-exact Q-Shift comparison uses. */
+void oracle_qshift_f32(const float* x, float* out, const float* mu, int B,
+                       int H, int W, int C, int s, double gamma,
+                       int round_bf16) {
+    const long T = (long)H * W;
+#pragma omp parallel for schedule(static)
+    for (long bt = 0; bt < (long)B * T; ++bt) {
+        long b = bt / T, t = bt % T;
+        int h = (int)(t / W), w = (int)(t % W);
+        for (int c = 0; c < C; ++c) {
+            int sh, sw;
+            float xd = 0.0f;
+            if (qshift_source(c, h, w, H, W, C, s, gamma, 0, &sh, &sw))
+                xd = x[(b * T + (long)sh * W + sw) * C + c];
+            float r;
+            if (mu) {
+                volatile float t1 = mu[c] * x[(b * T + t) * C + c];
+                volatile float om = 1.0f - mu[c];
+                volatile float t2 = om * xd;
+                r = t1 + t2;
+            } else {
+                r = xd;
+            }
+            out[(b * T + t) * C + c] = round_bf16 ? round_to_bf16(r) : r;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Bi-WKV, summation form (eq. 5)                                      */
+/* ------------------------------------------------------------------ */
+
+/* wkv_t for one channel column, directly from eq. 5:
+ *   num = sum_{i != t} exp(-(|t-i|-1)/T * w + k_i) v_i + exp(u + k_t) v_t
+ *   den = the same sums with v replaced by 1.                          */
+static double biwkv_direct_one(const double* kc, const double* vc, long T,
+                               double w, double u, long t) {
+    double num = 0.0, den = 0.0;
+    for (long i = 0; i < T; ++i) {
+        double e;
+        if (i == t) {
+            e = exp(u + kc[i]);
+        } else {
+            long d = i > t ? i - t : t - i;
+            e = exp(-((double)(d - 1) / (double)T) * w + kc[i]);
+        }
+        num += e * vc[i];
+        den += e;
+    }
+    return num / den;
+}
+
+static void gather_column(const double* src, double* col, long b, long T,
+                          long C, long c) {
+    for (long t = 0; t < T; ++t) col[t] = src[(b * T + t) * C + c];
+}
+
+void oracle_biwkv_direct(const double* k, const double* v, const double* w,
+                         const double* u, double* out, int B, int T, int C) {
+#pragma omp parallel
+    {
+        double* kc = (double*)malloc(sizeof(double) * (size_t)T);
+        double* vc = (double*)malloc(sizeof(double) * (size_t)T);
+#pragma omp for schedule(dynamic, 1)
+        for (long bc = 0; bc < (long)B * C; ++bc) {
+            long b = bc / C, c = bc % C;
+            gather_column(k, kc, b, T, C, c);
+            gather_column(v, vc, b, T, C, c);
+            for (long t = 0; t < T; ++t)
+                out[(b * T + t) * C + c] =
+                    biwkv_direct_one(kc, vc, T, w[c], u[c], t);
+        }
+        free(kc);
+        free(vc);
+    }
+}
+
+/* eq. 5 at selected flat indices idx[j] = (b*T + t)*C + c only. */
+void oracle_biwkv_direct_points(const double* k, const double* v,
+                                const double* w, const double* u, int B, int T,
+                                int C, const int64_t* idx, long n,
+                                double* out) {
+    (void)B;
+#pragma omp parallel
+    {
+        double* kc = (double*)malloc(sizeof(double) * (size_t)T);
+        double* vc = (double*)malloc(sizeof(double) * (size_t)T);
+#pragma omp for schedule(dynamic, 16)
+        for (long j = 0; j < n; ++j) {
+            long f = (long)idx[j];
+            long c = f % C, bt = f / C, t = bt % T, b = bt / T;
+            gather_column(k, kc, b, T, C, c);
+            gather_column(v, vc, b, T, C, c);
+            out[j] = biwkv_direct_one(kc, vc, T, w[c], u[c], t);
+        }
+        free(kc);
+        free(vc);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Bi-WKV, RNN form (eq. 6-7)                                          */
+/* ------------------------------------------------------------------ */
+
+/* Hidden states for output t (eq. 6):
+ *   a_{t-1} = sum_{i<t} e^{-(|t-i|-1)/T w + k_i} v_i,   c_{t-1}: v -> 1
+ *   b_{t-1} = sum_{i>t} e^{-(|t-i|-1)/T w + k_i} v_i,   d_{t-1}: v -> 1
+ * and eq. 7: wkv_t = (a+b+e^{k_t+u} v_t) / (c+d+e^{k_t+u}).
+ * Each step adds one term and multiplies by e^{-w/T}.  The forward pair (a,c)
+ * is run for increasing t; the backward pair (b,d) is run as its own pass for
+ * decreasing t (b_{t-1} = e^{-w/T} b_t + e^{k_{t+1}} v_{t+1}), which is the
+ * same sum built from the other end. */
+void oracle_biwkv_rnn(const double* k, const double* v, const double* w,
+                      const double* u, double* out, int B, int T, int C) {
+#pragma omp parallel
+    {
+        double* bb = (double*)malloc(sizeof(double) * (size_t)T);
+        double* dd = (double*)malloc(sizeof(double) * (size_t)T);
+#pragma omp for schedule(static)
+        for (long bc = 0; bc < (long)B * C; ++bc) {
+            long b = bc / C, c = bc % C;
+            const double decay = exp(-w[c] / (double)T);
+            /* backward pass: bb[t] = b_{t-1}, dd[t] = d_{t-1} */
+            double sb = 0.0, sd = 0.0;
+            for (long t = T - 1; t >= 0; --t) {
+                bb[t] = sb;
+                dd[t] = sd;
+                double e = exp(k[(b * T + t) * C + c]);
+                sb = decay * sb + e * v[(b * T + t) * C + c];
+                sd = decay * sd + e;
+            }
+            /* forward pass and eq. 7 */
+            double sa = 0.0, sc = 0.0;
+            for (long t = 0; t < T; ++t) {
+                double kt = k[(b * T + t) * C + c];
+                double vt = v[(b * T + t) * C + c];
+                double eu = exp(u[c] + kt);
+                out[(b * T + t) * C + c] =
+                    (sa + bb[t] + eu * vt) / (sc + dd[t] + eu);
+                double e = exp(kt);
+                sa = decay * sa + e * vt;
+                sc = decay * sc + e;
+            }
+        }
+        free(bb);
+        free(dd);
+    }
+}
+
+/* The RNN form exactly as the pages phrase it: b and d start as full sums
+ * over i > 0 and each later state is obtained by removing the term that
+ * becomes the current token and dividing by e^{-w/T}.  Subtraction makes it
+ * lose precision for long sequences; it is used on short sequences only. */
+void oracle_biwkv_rnn_literal(const double* k, const double* v,
+                              const double* w, const double* u, double* out,
+                              int B, int T, int C) {
+    for (long b = 0; b < B; ++b)
+        for (long c = 0; c < C; ++c) {
+            const double decay = exp(-w[c] / (double)T);
+            double sa = 0.0, sc = 0.0, sb = 0.0, sd = 0.0;
+            for (long i = 1; i < T; ++i) { /* b_{-1}, d_{-1} for t = 0 */
+                double e = exp(-((double)(i - 1) / (double)T) * w[c] +
+                               k[(b * T + i) * C + c]);
+                sb += e * v[(b * T + i) * C + c];
+                sd += e;
+            }
+            for (long t = 0; t < T; ++t) {
+                double kt = k[(b * T + t) * C + c];
+                double vt = v[(b * T + t) * C + c];
+                double eu = exp(u[c] + kt);
+                out[(b * T + t) * C + c] = (sa + sb + eu * vt) / (sc + sd + eu);
+                /* a,c: add the current term, multiply by e^{-w/T} */
+                double e = exp(kt);
+                sa = decay * sa + e * vt;
+                sc = decay * sc + e;
+                /* b,d: remove the term of token t+1, divide by e^{-w/T} */
+                if (t + 1 < T) {
+                    double e1 = exp(k[(b * T + t + 1) * C + c]);
+                    sb = (sb - e1 * v[(b * T + t + 1) * C + c]) / decay;
+                    sd = (sd - e1) / decay;
+                }
+            }
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Gate (eq. 2): sigma(R) (.) wkv, sigma(z) = 1 / (1 + e^{-z})         */
+/* ------------------------------------------------------------------ */
+void oracle_gate(const double* r, const double* wkv, double* out, long n) {
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; ++i) out[i] = wkv[i] * (1.0 / (1.0 + exp(-r[i])));
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
