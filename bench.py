@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 Vision-RWKV spatial-mix core.
+
+One step = one pass of the whole hot path over one batch: Q-Shift of x into
+r, k and v, Bi-WKV (eq. 5) and the sigma(R) gate, fused in one kernel launch
+(default workload: B=8, 64x64 token grid (T=4096, a 1024^2 image at patch
+16), C=1024, bfloat16 I/O, one x shared by r, k and v).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5]
+                    [--impl ours|reference]
+
+Timing: the K timed launches are replayed from CUDA graphs between a
+barrier + synchronize on each side, timed with CUDA events on the launching
+stream; the max over ranks is taken.  Inputs and outputs rotate over enough
+buffer sets that every launch reads and writes memory not touched for more
+than an L2's worth of traffic.  Multi-GPU runs are replicas (every (b, c)
+column is independent): each rank processes its own batch, no collective
+touches the data path, and the value is the whole-job throughput.
+
+The JSON line also carries the roofline of the fused kernel (algorithmic
+bytes / average launch time against the measured HBM copy bandwidth), an
+end-to-end figure through the C ABI with host buffers, the float64 CPU
+oracle timed on a bounded sample, and SM clocks sampled during the timed
+region.  ``--impl reference`` times the CPU oracle alone on the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from linear_complexity_vision_b200 import synth  # noqa: E402
+
+METRIC = ("Bi-WKV fused fwd tokens·ch/s and HBM GB/s (% of B200 peak) "
+          "at T=196–4096")
+UNIT = "tokens*ch/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["linear_complexity_vision_b200/csrc/common.cuh",
+                  "linear_complexity_vision_b200/csrc/biwkv.cuh",
+                  "linear_complexity_vision_b200/csrc/qshift.cuh",
+                  "linear_complexity_vision_b200/csrc/vrwkv_api.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def algorithmic_bytes(wl) -> dict:
+    """Bytes a launch must move at minimum: inputs read once, output written
+    once, parameter vectors read once.  Returns per-call bytes."""
+    es = 4 if wl.dtype == "f32" else 2
+    N, C = wl.N, wl.C
+    if wl.call == "biwkv":
+        return {"fused": 3 * N * es + 2 * C * 4}
+    if wl.call == "qshift_biwkv":
+        return {"qshift": 2 * N * es + C * 4, "fused": 3 * N * es + 4 * C * 4}
+    if wl.call == "gate_qs":
+        return {"fused": 4 * N * es + 5 * C * 4}
+    return {"fused": 2 * N * es + 5 * C * 4}  # gate_qs_x: x once, out once
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas; used for the barrier and max-over-ranks)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float, device) -> float:
+        if self.pg is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML, read-only queries)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, local_rank: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = local_rank
+            if vis:
+                ids = [v.strip() for v in vis.split(",") if v.strip()]
+                if local_rank < len(ids) and ids[local_rank].isdigit():
+                    idx = int(ids[local_rank])
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reason_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.ok = True
+        except Exception:  # no NVML: report no clocks rather than fail
+            self.ok = False
+
+    def _sample(self):
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            rs = int(self._reason_fn(self.h))
+            self.samples.append(mhz)
+            self.reasons |= rs & ~0x1
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._sample()
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": sorted(n for b, n in self.REASONS.items() if self.reasons & b)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(wl_name: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources and this workload."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+        ent = rec.get(wl_name)
+        if ent and ent.get("kernel_sha") == kernel_source_hash():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def make_inputs(wl, torch, dev, rank):
+    """Device tensors of one input set plus float64 copies for checks."""
+    import dataclasses
+    wlr = dataclasses.replace(wl, seed=wl.seed + 1000003 * rank)
+    inp = wlr.generate()
+    tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    host = {n: torch.from_numpy(inp[n]).to(tdt) for n in wl.tensor_names()}
+    par = {n: torch.from_numpy(inp[n]).to(torch.float32) for n in inp if n not in host}
+    return inp, host, par, tdt
+
+
+class Runner:
+    """Holds the rotating buffer sets and launches one step on set i."""
+
+    def __init__(self, vk, wl, torch, dev, rank):
+        self.vk, self.wl, self.torch = vk, wl, torch
+        self.inp, host, par, tdt = make_inputs(wl, torch, dev, rank)
+        self.host = host
+        self.par = {n: t.to(dev) for n, t in par.items()}
+        per_set = sum(t.numel() * t.element_size() for t in host.values()) * 2
+        self.nsets = max(2, int(np.ceil(3 * L2_BYTES / per_set)) + 1)
+        self.sets = []
+        shape = (wl.B, wl.T, wl.C)
+        for _ in range(self.nsets):
+            d = {n: t.to(dev) for n, t in host.items()}
+            d["out"] = torch.empty(shape, dtype=tdt, device=dev)
+            if wl.call == "qshift_biwkv":
+                d["xs"] = torch.empty(shape, dtype=tdt, device=dev)
+            self.sets.append(d)
+        if wl.call != "biwkv":
+            self.qs = vk.QShift(wl.H, wl.W, wl.shift_pixel, wl.gamma, self.par.get("mu_r"),
+                                self.par.get("mu_k"), self.par.get("mu_v"))
+        self.launches_per_step = 2 if wl.call == "qshift_biwkv" else 1
+
+    def step(self, i: int):
+        d = self.sets[i % self.nsets]
+        vk, p, wl = self.vk, self.par, self.wl
+        if wl.call == "biwkv":
+            vk.biwkv_fwd(d["k"], d["v"], p["w"], p["u"], out=d["out"])
+        elif wl.call == "qshift_biwkv":
+            vk.qshift(d["x"], wl.H, wl.W, wl.shift_pixel, wl.gamma, mu=p["mu_r"], out=d["xs"])
+            vk.biwkv_fwd(d["k"], d["v"], p["w"], p["u"], qs=self.qs, out=d["out"])
+        elif wl.call == "gate_qs":
+            vk.spatial_gate(d["r"], d["k"], d["v"], p["w"], p["u"], qs=self.qs, out=d["out"])
+        else:
+            x = d["x"]
+            vk.spatial_gate(x, x, x, p["w"], p["u"], qs=self.qs, out=d["out"])
+        return d["out"]
+
+    def step_host(self, hin: dict, hout, dbuf: dict):
+        """One end-to-end step: pinned host inputs -> device -> C ABI -> host."""
+        for n, t in hin.items():
+            dbuf[n].copy_(t, non_blocking=True)
+        out = self.step_on(dbuf)
+        hout.copy_(out, non_blocking=True)
+
+    def step_on(self, d):
+        saved = self.sets
+        self.sets = [d]
+        try:
+            return self.step(0)
+        finally:
+            self.sets = saved
+
+
+def parity_sample(runner, out_dev, oracle, npts=128):
+    """Max |GPU - float64 oracle| on a seeded sample of output positions."""
+    wl, inp = runner.wl, runner.inp
+    got = out_dev.to(runner.torch.float64).cpu().numpy().reshape(-1)
+    rng = np.random.default_rng(7)
+    idx = np.sort(rng.choice(got.size, size=npts, replace=False))
+    tdt = runner.torch.float32 if wl.dtype == "f32" else runner.torch.bfloat16
+    r64 = {n: runner.torch.from_numpy(inp[n]).to(tdt).to(runner.torch.float64).numpy()
+           for n in wl.tensor_names()}
+    p64 = {n: runner.torch.from_numpy(inp[n]).to(runner.torch.float32).double().numpy()
+           for n in inp if n not in r64}
+    if wl.call == "gate_qs_x":
+        r = k = v = r64["x"]
+    else:
+        r, k, v = r64.get("r"), r64["k"], r64["v"]
+    want = oracle.spatial_core_points(
+        r, k, v, p64["w"], p64["u"], wl.H, wl.W, idx, wl.shift_pixel, wl.gamma,
+        p64.get("mu_r"), p64.get("mu_k"), p64.get("mu_v"),
+        qshift_on=wl.call != "biwkv", gate_on=wl.call in ("gate_qs", "gate_qs_x"))
+    return float(np.max(np.abs(got[idx] - want)))
+
+
+def oracle_throughput(wl, oracle, target_s: float, max_points: int = 1 << 20):
+    """The float64 oracle (eq. 5 directly, per output position, with Q-Shift
+    and gate) on a seeded sample of output positions of the workload, sized
+    to take about target_s seconds.  Returns (tokens*ch/s, points, seconds)."""
+    inp = wl.generate()
+    if wl.call == "gate_qs_x":
+        r = k = v = inp["x"]
+    else:
+        r, k, v = inp.get("r"), inp["k"], inp["v"]
+    qs_on = wl.call != "biwkv"
+    gate_on = wl.call in ("gate_qs", "gate_qs_x")
+    rng = np.random.default_rng(11)
+
+    def run(n):
+        idx = rng.integers(0, wl.N, size=n)
+        t0 = time.perf_counter()
+        oracle.spatial_core_points(r, k, v, inp["w"], inp["u"], wl.H, wl.W, idx, wl.shift_pixel,
+                                   wl.gamma, inp.get("mu_r"), inp.get("mu_k"), inp.get("mu_v"),
+                                   qshift_on=qs_on, gate_on=gate_on)
+        return time.perf_counter() - t0
+
+    n = 4 * oracle.num_threads()
+    dt = run(n)
+    while dt < 0.5 and n < max_points:
+        n *= 4
+        dt = run(n)
+    n = int(min(max_points, max(n, n * target_s / max(dt, 1e-9))))
+    dt = run(n)
+    return n / dt, n, dt
+
+
+def run_ours(args, dist):
+    import torch
+    import linear_complexity_vision_b200 as vk
+    vk.load_library()  # fail loudly if the CUDA library is missing
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    dist.init("nccl")
+    wl = synth.WORKLOADS[args.workload]
+    runner = Runner(vk, wl, torch, dev, dist.rank)
+    stream = torch.cuda.Stream(device=dev)
+
+    # warm-up (also raises the kernel's shared-memory limit before capture)
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            out = runner.step(i)
+    torch.cuda.synchronize(dev)
+
+    # capture one rotation period of launches (a multiple of nsets) per graph
+    G = runner.nsets * max(1, 64 // runner.nsets)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            runner.step(i)
+    torch.cuda.synchronize(dev)
+    reps, rem = divmod(args.steps, G)
+
+    clocks = ClockSampler(dist.local_rank)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        for i in range(rem):
+            runner.step(i)
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    dist.barrier()
+    ms_local = ev0.elapsed_time(ev1)
+    ms = dist.max(ms_local, dev)
+    del graph
+
+    steps = args.steps
+    units = wl.N
+    value = dist.world * steps * units / (ms / 1e3)
+    ms_per_step = ms / steps
+
+    # roofline of the fused kernel: the timed region holds only our launches
+    # back to back, so the average launch time is (region / launches)
+    ab = algorithmic_bytes(wl)
+    launch_s = (ms_local / 1e3) / (steps * runner.launches_per_step)
+    fused_bytes = ab["fused"]
+    if wl.call == "qshift_biwkv":  # two kernels: attribute by bytes
+        fused_share = ab["fused"] / (ab["fused"] + ab["qshift"])
+        launch_s = (ms_local / 1e3) * fused_share / steps
+    peak, peak_kind = measured_hbm_peak()
+    achieved = fused_bytes / launch_s / 1e9
+    traffic = committed_traffic(wl.name)
+
+    # end to end through the C ABI with pinned host buffers
+    e2e_steps = max(3, min(args.steps, 50))
+    hin = {n: t.pin_memory() for n, t in runner.host.items()}
+    hout = torch.empty((wl.B, wl.T, wl.C), dtype=next(iter(hin.values())).dtype).pin_memory()
+    dbuf = dict(runner.sets[0])
+    with torch.cuda.stream(stream):
+        runner.step_host(hin, hout, dbuf)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            runner.step_host(hin, hout, dbuf)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = dist.max(e0.elapsed_time(e1), dev)
+    h2d = sum(t.numel() * t.element_size() for t in hin.values())
+    d2h = hout.numel() * hout.element_size()
+    e2e = {"value": dist.world * e2e_steps * units / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "W": wl.W, "C": wl.C,
+                   "call": wl.call, "shift_pixel": wl.shift_pixel, "gamma": wl.gamma,
+                   "io_dtype": wl.dtype, "accumulate": "f32",
+                   "l2": f"rotating {runner.nsets} input/output buffer sets "
+                         f"({runner.nsets * 2 * wl.N * (4 if wl.dtype == 'f32' else 2) / 1e6:.0f} MB"
+                         " > 126 MB L2)",
+                   "timing": f"CUDA graphs of {G} launches, events on the launching stream",
+                   "parallelism": f"replicas x{dist.world} (independent batches, no collective)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": "biwkv_fused_kernel",
+                     "algorithmic_bytes_per_launch": fused_bytes,
+                     "avg_launch_us": launch_s * 1e6},
+        "e2e": e2e,
+        "gpu_launches": steps * runner.launches_per_step,
+        "clocks": clocks.summary(),
+    }
+    # correctness guard on the last timed output (first set of the rotation)
+    if dist.rank == 0:
+        import oracle
+        line["parity_sample_max_abs_err"] = parity_sample(runner, runner.sets[0]["out"], oracle)
+        if dist.world == 1 and not args.no_cpu_baseline:
+            v, n, dt = oracle_throughput(wl, oracle, target_s=args.cpu_seconds)
+            line["cpu_baseline"] = {
+                "value": v, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"{n} seeded output positions of the workload; each by direct "
+                          f"eq. 5 summation over its T={wl.T} column with Q-Shift and gate, "
+                          f"float64 ({dt:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 CPU oracle as it stands
+# ---------------------------------------------------------------------------
+def run_reference(args, dist):
+    if dist.rank != 0:
+        return
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    inp = wl.generate()
+    if wl.call == "gate_qs_x":
+        r = k = v = inp["x"]
+    else:
+        r, k, v = inp.get("r"), inp["k"], inp["v"]
+    qs_on, gate_on = wl.call != "biwkv", wl.call in ("gate_qs", "gate_qs_x")
+    rng = np.random.default_rng(13)
+
+    def step(n):
+        idx = rng.integers(0, wl.N, size=n)
+        oracle.spatial_core_points(r, k, v, inp["w"], inp["u"], wl.H, wl.W, idx, wl.shift_pixel,
+                                   wl.gamma, inp.get("mu_r"), inp.get("mu_k"), inp.get("mu_v"),
+                                   qshift_on=qs_on, gate_on=gate_on)
+
+    # size each step so that warm-up + timed steps take about budget seconds
+    t0 = time.perf_counter()
+    step(oracle.num_threads())
+    per_point = (time.perf_counter() - t0) / oracle.num_threads()
+    total = max(1, args.steps + args.warmup)
+    n = max(1, int(args.reference_seconds / total / per_point))
+    for _ in range(args.warmup):
+        step(n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(n)
+    dt = time.perf_counter() - t0
+    value = args.steps * n / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "W": wl.W, "C": wl.C,
+                   "call": wl.call},
+        "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
+                         "cores": oracle.num_threads(),
+                         "sample": f"{n} seeded output positions per step, each by direct eq. 5 "
+                                   f"summation over its T={wl.T} column with Q-Shift and gate"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", type=int, default=5, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-seconds", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+    else:
+        run_ours(args, dist)
+
+
+if __name__ == "__main__":
+    main()

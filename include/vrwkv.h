@@ -1,0 +1,147 @@
+/*
+ * vrwkv.h -- C ABI of the B200 (sm_100a) Vision-RWKV spatial-mix core.
+ *
+ * The operations follow "OpenGVLab&港中文&复旦&南大&清华提出Vision-RWKV
+ * Backbone" (cloud.tencent.com article 2395249) and the q_shift listing on
+ * "LinXin's Blog" (Vision-RWKV entry):
+ *   - Q-Shift, Quad-Directional Token Shift, eq. 9;
+ *   - Bi-WKV, Linear Complexity Bidirectional Attention, eq. 5
+ *     (equivalently the RNN form, eq. 6-7);
+ *   - the receptance gate sigma(R) (.) wkv, Overall Architecture, eq. 2.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  Token tensors are dense row-major (B, T, C): channel fastest, then
+ *   token, then batch.  With a patch grid H x W the token index is
+ *   t = h*W + w (raster order) and T = H*W.  w, u and the mu vectors are
+ *   dense float32 vectors of length C.
+ * Memory.  Every pointer is caller-owned DEVICE memory.  The library keeps
+ *   no state between calls and allocates no device or host memory.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *   default stream).  Work is enqueued asynchronously; the caller
+ *   synchronises.  Calls may be captured into CUDA graphs.
+ * Dtypes.  VRWKV_F32 or VRWKV_BF16 select the storage type of the token
+ *   tensors (inputs and output alike).  Arithmetic is float32 throughout;
+ *   bfloat16 outputs are rounded to nearest even once, at the store.
+ * Aliasing.  Inputs may alias one another (the spatial-mix core commonly
+ *   passes one tensor x as r, k and v).  An output must not overlap any
+ *   input: that is VRWKV_ERR_INVALID_ARG.
+ * Errors.  Every entry point validates its arguments on the host before it
+ *   touches the GPU and returns a status; nothing aborts and no exception
+ *   crosses the ABI.  vrwkv_last_error() gives a one-line reason for the most
+ *   recent non-OK status of the calling thread.  VRWKV_ERR_CUDA reports a
+ *   launch failure (the CUDA error string is in vrwkv_last_error()); errors of
+ *   kernels that already ran asynchronously surface at the caller's next
+ *   synchronisation, as usual in CUDA.
+ */
+#ifndef VRWKV_H
+#define VRWKV_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VRWKV_OK = 0,
+    VRWKV_ERR_INVALID_ARG = 1, /* bad size, pointer, alignment or parameter */
+    VRWKV_ERR_UNSUPPORTED = 2, /* valid problem outside the kernels' limits */
+    VRWKV_ERR_CUDA = 3         /* the CUDA runtime reported an error        */
+} vrwkv_status;
+
+typedef enum {
+    VRWKV_F32 = 0,
+    VRWKV_BF16 = 1
+} vrwkv_dtype;
+
+/*
+ * Q-Shift parameters (eq. 9 and the q_shift listing).
+ *   H, W         patch grid; T must equal H*W.
+ *   shift_pixel  shift distance in patches, >= 0.  A distance at or beyond
+ *                the grid extent leaves that channel group all zero.
+ *   gamma        channel-group fraction, 0 <= gamma <= 1/4; the group size is
+ *                g = (int)(C*gamma) computed in double precision.  Channels
+ *                [0,g) take x[h, w-s], [g,2g) x[h, w+s], [2g,3g) x[h-s, w],
+ *                [3g,4g) x[h+s, w] (zero outside the grid); channels >= 4g
+ *                take x[h, w] unchanged.
+ *   mu_r, mu_k, mu_v  device float32[C] interpolation weights, each nullable.
+ *                With mu the shifted input is mu*x + (1-mu)*x_shift; a NULL
+ *                mu means the shifted tensor x_shift itself.
+ */
+typedef struct {
+    int H;
+    int W;
+    int shift_pixel;
+    double gamma;
+    const float* mu_r;
+    const float* mu_k;
+    const float* mu_v;
+} vrwkv_qshift_params;
+
+/*
+ * vrwkv_qshift -- Q-Shift of one tensor (eq. 9; q_shift listing).
+ *   x    (B, H*W, C) input, dtype `dtype`.
+ *   out  (B, H*W, C) output, same dtype, must not overlap x.
+ *   mu   float32[C] or NULL: out = x_shift (NULL) or mu*x + (1-mu)*x_shift,
+ *        evaluated in float32 as t1 = mu*x, t2 = (1-mu)*x_shift, t1 + t2 with
+ *        each operation rounded separately (no fused multiply-add), then
+ *        stored (rounded to bfloat16 for VRWKV_BF16).  Without mu the result
+ *        is a pure gather and bit-exact in either dtype.
+ * Errors: INVALID_ARG for B, H, W or C <= 0, shift_pixel < 0, gamma outside
+ *   [0, 1/4], NULL x/out, misaligned pointers, or out overlapping x.
+ */
+vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B,
+                          int H, int W, int C, int shift_pixel, double gamma,
+                          vrwkv_dtype dtype, void* stream);
+
+/*
+ * vrwkv_biwkv_fwd -- Bi-WKV forward (eq. 5):
+ *   wkv_t = [ sum_{i!=t} e^{-(|t-i|-1)/T * w + k_i} v_i + e^{u + k_t} v_t ]
+ *         / [ sum_{i!=t} e^{-(|t-i|-1)/T * w + k_i}     + e^{u + k_t}     ]
+ * independently for every batch b and channel c, with w[c] of either sign.
+ *   k, v  (B, T, C) inputs, dtype `dtype`.
+ *   w, u  float32[C] decay and current-token bonus.
+ *   wkv   (B, T, C) output, same dtype, must not overlap k, v, w or u.
+ *   qs    NULL, or Q-Shift parameters applied to k (mu_k) and v (mu_v) on
+ *         load (mu_r is ignored); T must then equal qs->H * qs->W.
+ * Limits: T <= 4096 (UNSUPPORTED above); with qs, a halo of shift_pixel*W
+ *   tokens must fit the kernel's shared-memory tile (UNSUPPORTED otherwise).
+ *   Exponents are renormalised by the running maximum of k, so a constant
+ *   added to every k of a channel leaves wkv unchanged; results stay finite
+ *   while |w| + (spread of k within a channel) stays well below 80.
+ * Errors: INVALID_ARG for B, T or C <= 0, NULL k/v/w/u/wkv, misaligned
+ *   pointers, an overlapping output, or bad qs fields (see the struct).
+ */
+vrwkv_status vrwkv_biwkv_fwd(const void* k, const void* v, const float* w,
+                             const float* u, void* wkv, int B, int T, int C,
+                             vrwkv_dtype dtype, const vrwkv_qshift_params* qs,
+                             void* stream);
+
+/*
+ * vrwkv_spatial_gate -- the spatial-mix core without projections (eq. 2
+ * with identity W_R, W_K, W_V and no W_O):
+ *   out = sigma(QS_R(r)) (.) Bi-WKV(QS_K(k), QS_V(v)),  sigma(z) = 1/(1+e^{-z})
+ * where QS_* is Q-Shift with mu_r, mu_k, mu_v when qs is given and the
+ * identity when qs is NULL.  r, k and v may be the same tensor (eq. 1 shifts
+ * one X three ways); that case reads the tensor once.
+ *   r, k, v  (B, T, C) inputs, dtype `dtype`.
+ *   w, u     float32[C].
+ *   out      (B, T, C) output, same dtype, must not overlap any input.
+ * Limits and errors as vrwkv_biwkv_fwd, with r also required non-NULL.
+ */
+vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
+                                const float* w, const float* u, void* out,
+                                int B, int T, int C, vrwkv_dtype dtype,
+                                const vrwkv_qshift_params* qs, void* stream);
+
+/* Static, never-NULL name of a status code. */
+const char* vrwkv_status_string(vrwkv_status status);
+
+/* One-line reason for the calling thread's most recent non-OK status
+ * ("" if none).  Valid until that thread's next call into the library. */
+const char* vrwkv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VRWKV_H */

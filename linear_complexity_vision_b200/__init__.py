@@ -1,0 +1,162 @@
+"""Python binding of the B200 (sm_100a) Vision-RWKV spatial-mix core.
+
+Thin ctypes marshalling over ``libvrwkv.so`` (the C ABI in include/vrwkv.h):
+every step of Q-Shift, Bi-WKV and the sigma(R) gate runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream only.
+There is no fallback: if the library is missing, the calls raise.
+
+    qshift(x, H, W, shift_pixel=1, gamma=0.25, mu=None)
+    biwkv_fwd(k, v, w, u, qs=None)
+    spatial_gate(r, k, v, w, u, qs=None)
+
+Token tensors are contiguous (B, T, C) CUDA tensors of dtype float32 or
+bfloat16; w, u and mu vectors are contiguous float32 CUDA tensors of
+length C.  ``qs`` is a ``QShift`` (grid, shift, gamma and the three mu
+vectors).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvrwkv.so")
+
+VRWKV_OK = 0
+VRWKV_F32 = 0
+VRWKV_BF16 = 1
+
+_lib = None
+
+
+class VrwkvError(RuntimeError):
+    """A non-OK status returned by the C ABI."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class _QsParams(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int), ("W", ctypes.c_int), ("shift_pixel", ctypes.c_int),
+                ("gamma", ctypes.c_double), ("mu_r", ctypes.c_void_p),
+                ("mu_k", ctypes.c_void_p), ("mu_v", ctypes.c_void_p)]
+
+
+def load_library():
+    """Load libvrwkv.so; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m linear_complexity_vision_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, ci, cd = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        lib.vrwkv_qshift.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cd, ci, vp]
+        lib.vrwkv_qshift.restype = ci
+        for name in ("vrwkv_biwkv_fwd",):
+            getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                           ctypes.POINTER(_QsParams), vp]
+            getattr(lib, name).restype = ci
+        lib.vrwkv_spatial_gate.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                           ctypes.POINTER(_QsParams), vp]
+        lib.vrwkv_spatial_gate.restype = ci
+        lib.vrwkv_status_string.argtypes = [ci]
+        lib.vrwkv_status_string.restype = ctypes.c_char_p
+        lib.vrwkv_last_error.argtypes = []
+        lib.vrwkv_last_error.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != VRWKV_OK:
+        lib = load_library()
+        name = lib.vrwkv_status_string(status).decode()
+        msg = lib.vrwkv_last_error().decode()
+        raise VrwkvError(status, f"{name}: {msg}")
+
+
+@dataclass
+class QShift:
+    """Q-Shift parameters: patch grid H x W, shift_pixel, gamma and the
+    interpolation weights mu_r, mu_k, mu_v (float32 (C,) CUDA tensors or
+    None for the pure shifted tensor)."""
+    H: int
+    W: int
+    shift_pixel: int = 1
+    gamma: float = 0.25
+    mu_r: Optional[object] = None
+    mu_k: Optional[object] = None
+    mu_v: Optional[object] = None
+
+    def _struct(self) -> _QsParams:
+        def ptr(t):
+            return None if t is None else t.data_ptr()
+        return _QsParams(int(self.H), int(self.W), int(self.shift_pixel), float(self.gamma),
+                         ptr(self.mu_r), ptr(self.mu_k), ptr(self.mu_v))
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return VRWKV_F32
+    if t.dtype == torch.bfloat16:
+        return VRWKV_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_ptr(t) -> int:
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _require(t, name: str) -> None:
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def qshift(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25, mu=None, out=None):
+    """Q-Shift of x (B, H*W, C): the shifted tensor, or mu*x + (1-mu)*shifted."""
+    import torch
+    _require(x, "x")
+    B, T, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(load_library().vrwkv_qshift(
+        x.data_ptr(), out.data_ptr(), None if mu is None else mu.data_ptr(), B, H, W, C,
+        shift_pixel, float(gamma), _dtype_code(x), _stream_ptr(x)))
+    return out
+
+
+def biwkv_fwd(k, v, w, u, qs: Optional[QShift] = None, out=None):
+    """Bi-WKV forward of eq. 5 on (B, T, C) tensors; Q-Shift on load if qs."""
+    import torch
+    for t, name in ((k, "k"), (v, "v"), (w, "w"), (u, "u")):
+        _require(t, name)
+    B, T, C = k.shape
+    if out is None:
+        out = torch.empty_like(k)
+    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _check(load_library().vrwkv_biwkv_fwd(
+        k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(), B, T, C,
+        _dtype_code(k), qsp, _stream_ptr(k)))
+    return out
+
+
+def spatial_gate(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
+    """sigma(QS_R(r)) * Bi-WKV(QS_K(k), QS_V(v)); r, k, v may be one tensor."""
+    import torch
+    for t, name in ((r, "r"), (k, "k"), (v, "v"), (w, "w"), (u, "u")):
+        _require(t, name)
+    B, T, C = k.shape
+    if out is None:
+        out = torch.empty_like(k)
+    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _check(load_library().vrwkv_spatial_gate(
+        r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
+        B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
+    return out

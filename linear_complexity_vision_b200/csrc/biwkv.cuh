@@ -1,0 +1,439 @@
+// Fused Q-Shift -> Bi-WKV -> sigma(R) gate kernel for sm_100a.
+//
+// Computes Bi-WKV ("Vision-RWKV Backbone", Linear Complexity Bidirectional
+// Attention, eq. 5), optionally on Q-Shifted inputs (Quad-Directional Token
+// Shift, eq. 9) and optionally gated by sigma(R) (Overall Architecture,
+// eq. 2).  Instead of the page's token-serial RNN form (eq. 6-7) the kernel
+// evaluates the same four sums as a chunked two-sided linear scan:
+//
+//   A_t = sum_{i<t} a^{t-1-i} p_i v_i,   B_t = sum_{i>t} a^{i-t-1} p_i v_i,
+//   C_t, D_t likewise with v = 1,        a = e^{-w/T},  p_i = e^{k_i - M},
+//   wkv_t = (A_t + B_t + e^u p_t v_t) / (C_t + D_t + e^u p_t).
+//
+// Work decomposition.  A CTA owns one batch row b, a slab of 16 channels and
+// a range of at most 512 tokens; longer sequences split across the CTAs of a
+// thread-block cluster (up to 8, so T <= 4096).  A thread owns 2 adjacent
+// channels (packed float2 arithmetic) x 8 consecutive tokens (a chunk); the
+// 32 lanes of a warp are 8 channel pairs x 4 consecutive chunks.
+//
+//   1. the CTA's input tiles (plus a Q-Shift halo) are staged in shared
+//      memory with 16-byte cp.async copies; rows are padded by one row every
+//      eight so the four chunks of a warp hit distinct banks;
+//   2. each thread mixes Q-Shift on load, takes the CTA maximum M of k per
+//      channel, computes p = e^{k-M} once, and runs its chunk forward and
+//      backward to get the chunk-local parts of A..D and the chunk aggregates;
+//   3. chunk aggregates are scanned within the warp (shuffles), across warps
+//      (one shuffle scan over 16 warp aggregates), and across the cluster
+//      (each CTA folds its peers' aggregates read through distributed shared
+//      memory, carrying (exponent, sum) pairs so no power of a is ever formed
+//      by repeated multiplication over more than 8 steps);
+//   4. each thread adds the carries to its chunk-local sums, applies the gate
+//      and stores.
+// Exponents are kept in base 2 (log2(e) is folded into k, u, w and r).
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace vrwkv {
+namespace cg = cooperative_groups;
+
+constexpr int kCS = 16;        // channels per CTA slab
+constexpr int kNP = kCS / 2;   // channel pairs per slab
+constexpr int kL = 8;          // tokens per thread chunk
+constexpr int kTcMax = 512;    // tokens per CTA
+constexpr int kNWMax = 16;     // warps per CTA
+constexpr int kClusterMax = 8; // CTAs per cluster (portable limit)
+constexpr int kMinThreads = 128;
+
+enum Layout { kKV = 0, kRKV = 1, kX = 2 };
+
+struct FusedParams {
+    const char* src[3];  // token tensors in tile order: KV: k,v; RKV: r,k,v; X: x
+    const float* w;
+    const float* u;
+    const float* mu_r;  // nullable
+    const float* mu_k;  // nullable
+    const float* mu_v;  // nullable
+    char* out;
+    int B, T, C;
+    int H, W, s, g;   // Q-Shift grid, shift and group size
+    int Tc;           // tokens per CTA (multiple of 32 when ncl > 1)
+    int ncl;          // CTAs per (b, slab) column = cluster size
+    int halo;         // tile rows before and after the CTA's own tokens
+    int rows;         // tile rows = Tc + 2 * halo
+    int tile_bytes;   // bytes per padded tile
+    int vec_in;       // 16-byte copies allowed
+    int vec_out;      // paired stores allowed
+};
+
+__host__ __device__ constexpr int padded_row(int r) { return r + (r >> 3); }
+
+// Shared-memory scratch that follows the tiles.
+struct Scratch {
+    float2 wmax[kNWMax][kNP];   // per-warp channel maxima
+    float4 waggF[kNWMax][kNP];  // per-warp forward aggregates (A.x, A.y, C.x, C.y)
+    float4 waggB[kNWMax][kNP];  // per-warp backward aggregates
+    float4 wcarF[kNWMax][kNP];  // exclusive forward carry into each warp
+    float4 wcarB[kNWMax][kNP];  // exclusive backward carry into each warp
+    float2 cM[kNP];             // CTA maximum of k (base-2 units)
+    float4 caggF[kNP];          // CTA forward aggregate (read by cluster peers)
+    float4 caggB[kNP];          // CTA backward aggregate (read by cluster peers)
+    float cinfo[kCS][8];        // per channel: sl, ef, eb, Af, Cf, Bf, Df
+};
+
+__device__ __forceinline__ float4 shfl_up4(float4 v, int d, int width = 32) {
+    return make_float4(__shfl_up_sync(0xffffffffu, v.x, d, width),
+                       __shfl_up_sync(0xffffffffu, v.y, d, width),
+                       __shfl_up_sync(0xffffffffu, v.z, d, width),
+                       __shfl_up_sync(0xffffffffu, v.w, d, width));
+}
+__device__ __forceinline__ float4 shfl_down4(float4 v, int d, int width = 32) {
+    return make_float4(__shfl_down_sync(0xffffffffu, v.x, d, width),
+                       __shfl_down_sync(0xffffffffu, v.y, d, width),
+                       __shfl_down_sync(0xffffffffu, v.z, d, width),
+                       __shfl_down_sync(0xffffffffu, v.w, d, width));
+}
+// (A, C) pairs packed as float4 = (A.x, A.y, C.x, C.y); scale both by m.
+__device__ __forceinline__ float4 fma4(float2 m, float4 x, float4 y) {
+    float2 a = fma2(m, make_float2(x.x, x.y), make_float2(y.x, y.y));
+    float2 c = fma2(m, make_float2(x.z, x.w), make_float2(y.z, y.w));
+    return make_float4(a.x, a.y, c.x, c.y);
+}
+__device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float4 pack4(float2 a, float2 c) { return make_float4(a.x, a.y, c.x, c.y); }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
+// Stage rows [t0 - halo, t0 - halo + rows) x channels [c0, c0 + 16) of one
+// (B, T, C) tensor into a padded shared-memory tile.  Rows outside [0, T)
+// are left unwritten: no thread reads them.
+template <typename IO>
+__device__ __forceinline__ void load_tile(char* tile, const char* g, const FusedParams& p,
+                                          int b, int t0, int c0) {
+    constexpr int es = Io<IO>::kBytes;
+    constexpr int pitch = kCS * es;
+    constexpr int upr = pitch / 16;  // 16-byte units per row
+    constexpr int epu = 16 / es;     // elements per unit
+    const int n = p.rows * upr;
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
+        const int r = e / upr, uu = e - (e / upr) * upr;
+        const int t = t0 - p.halo + r;
+        if (t < 0 || t >= p.T) continue;
+        char* dst = tile + padded_row(r) * pitch + uu * 16;
+        const int c = c0 + uu * epu;
+        const char* srcp = g + (((size_t)b * p.T + t) * p.C + c) * es;
+        if (p.vec_in && c + epu <= p.C) {
+            cp_async16(dst, srcp);
+        } else {
+#pragma unroll
+            for (int q = 0; q < epu; ++q) {
+                float v = (c + q < p.C) ? Io<IO>::ld1(srcp + q * es) : 0.0f;
+                Io<IO>::st1(dst + q * es, v);
+            }
+        }
+    }
+}
+
+// Mixed (Q-Shifted, interpolated, scaled) value of one channel pair at tile
+// row r.  cm and cd are the coefficients of x and of the shifted x.
+template <typename IO, bool QS>
+__device__ __forceinline__ float2 mixed_pair(const char* tile, int r, int j, bool split,
+                                             const ShiftRule& ra, const ShiftRule& rb, int h,
+                                             int w, float2 cm, float2 cd) {
+    constexpr int es = Io<IO>::kBytes;
+    constexpr int pitch = kCS * es;
+    const float2 x = Io<IO>::ld_pair(tile + padded_row(r) * pitch + j * 2 * es);
+    if (!QS) return mul2(cm, x);
+    float2 xd;
+    if (!split) {
+        xd = shift_ok(ra, h, w) ? Io<IO>::ld_pair(tile + padded_row(r + ra.off) * pitch + j * 2 * es)
+                                : make_float2(0.0f, 0.0f);
+    } else {
+        xd.x = shift_ok(ra, h, w) ? Io<IO>::ld1(tile + padded_row(r + ra.off) * pitch + (2 * j) * es)
+                                  : 0.0f;
+        xd.y = shift_ok(rb, h, w)
+                   ? Io<IO>::ld1(tile + padded_row(r + rb.off) * pitch + (2 * j + 1) * es)
+                   : 0.0f;
+    }
+    return fma2(cm, x, mul2(cd, xd));
+}
+
+template <typename IO, int LAYOUT, bool QS>
+__global__ void __launch_bounds__(512, 1) biwkv_fused_kernel(const __grid_constant__ FusedParams p) {
+    constexpr bool GATE = (LAYOUT != kKV);
+    constexpr int NT = (LAYOUT == kKV) ? 2 : (LAYOUT == kRKV ? 3 : 1);
+    constexpr int TR = 0;                               // tile of r
+    constexpr int TK = (LAYOUT == kKV) ? 0 : (LAYOUT == kRKV ? 1 : 0);
+    constexpr int TV = (LAYOUT == kKV) ? 1 : (LAYOUT == kRKV ? 2 : 0);
+    constexpr int es = Io<IO>::kBytes;
+
+    extern __shared__ __align__(128) char smem[];
+    Scratch& S = *reinterpret_cast<Scratch*>(smem + NT * p.tile_bytes);
+
+    const int tid = threadIdx.x;
+    const int j = tid & 7;          // channel pair within the slab
+    const int q = tid >> 3;         // chunk within the CTA
+    const int cq = q & 3;           // chunk within the warp
+    const int warp = tid >> 5;
+    const int NW = blockDim.x >> 5;
+    const int rank = blockIdx.x;    // CTA rank along T (= cluster rank)
+    const int c0 = blockIdx.y * kCS;
+    const int b = blockIdx.z;
+    const int t0 = rank * p.Tc;
+    const int tend = min(p.T, t0 + p.Tc);
+
+    // ---- 1. stage the tiles ------------------------------------------------
+#pragma unroll
+    for (int ti = 0; ti < NT; ++ti) load_tile<IO>(smem + ti * p.tile_bytes, p.src[ti], p, b, t0, c0);
+
+    // per-channel constants of this thread's pair (overlaps the copies)
+    const int cA = c0 + 2 * j, cB = cA + 1;
+    const bool okA = cA < p.C, okB = cB < p.C;
+    const float invT = 1.0f / (float)p.T;
+    const float2 wv = make_float2(okA ? __ldg(p.w + cA) : 0.0f, okB ? __ldg(p.w + cB) : 0.0f);
+    const float2 uv = make_float2(okA ? __ldg(p.u + cA) : 0.0f, okB ? __ldg(p.u + cB) : 0.0f);
+    const float2 lam2 = mul2(wv, f2(invT * kLog2e));  // w/T in base-2 units
+    const float2 alpha = ex2(make_float2(-lam2.x, -lam2.y));
+    const float2 eu = ex2(mul2(uv, f2(kLog2e)));
+
+    ShiftRule ra{0, 1, 0, 0x7fffffff}, rb{0, 1, 0, 0x7fffffff};
+    bool split = false;
+    float2 kcm = f2(kLog2e), kcd = f2(0.0f), vcm = f2(1.0f), vcd = f2(0.0f);
+    float2 rcm = f2(-kLog2e), rcd = f2(0.0f);
+    if (QS) {
+        ra = shift_rule(cA, p.g, p.H, p.W, p.s);
+        rb = okB ? shift_rule(cB, p.g, p.H, p.W, p.s) : ra;
+        split = !(ra.off == rb.off && ra.use_w == rb.use_w && ra.lo == rb.lo && ra.hi == rb.hi);
+        auto coef = [&](const float* mu, float scale, float2& cm, float2& cd) {
+            float2 m = make_float2(0.0f, 0.0f);
+            if (mu) m = make_float2(okA ? __ldg(mu + cA) : 0.0f, okB ? __ldg(mu + cB) : 0.0f);
+            cm = mul2(m, f2(scale));
+            cd = mul2(make_float2(1.0f - m.x, 1.0f - m.y), f2(scale));
+        };
+        coef(p.mu_k, kLog2e, kcm, kcd);
+        coef(p.mu_v, 1.0f, vcm, vcd);
+        if (GATE) coef(p.mu_r, -kLog2e, rcm, rcd);
+    }
+
+    const int s_tok = t0 + q * kL;
+    const int nv = max(0, min(kL, tend - s_tok));
+    int h0 = 0, w0 = 0;
+    if (QS) { h0 = s_tok / p.W; w0 = s_tok - h0 * p.W; }
+    const int rbase = q * kL + p.halo;  // tile row of the chunk's first token
+
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- 2. load + Q-Shift + chunk maximum -----------------------------------
+    const char* tk = smem + TK * p.tile_bytes;
+    const char* tv = smem + TV * p.tile_bytes;
+    float2 kk[kL], vv[kL];
+    float2 mx = f2(-INFINITY);
+    {
+        int h = h0, w = w0;
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            if (i < nv) {
+                kk[i] = mixed_pair<IO, QS>(tk, rbase + i, j, split, ra, rb, h, w, kcm, kcd);
+                vv[i] = mixed_pair<IO, QS>(tv, rbase + i, j, split, ra, rb, h, w, vcm, vcd);
+                mx = max2(mx, kk[i]);
+            } else {
+                kk[i] = f2(-INFINITY);
+                vv[i] = f2(0.0f);
+            }
+            if (QS) { if (++w == p.W) { w = 0; ++h; } }
+        }
+    }
+    // CTA maximum per channel: across the 4 chunks of the warp, then warps.
+#pragma unroll
+    for (int d = 8; d <= 16; d <<= 1) {
+        mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
+        mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
+    }
+    if (cq == 0) S.wmax[warp][j] = mx;
+    __syncthreads();
+    if (tid < kNP * 16) {
+        const int jj = tid >> 4, wi = tid & 15;
+        float2 m = (wi < NW) ? S.wmax[wi][jj] : f2(-INFINITY);
+#pragma unroll
+        for (int d = 1; d < 16; d <<= 1) {
+            m.x = fmaxf(m.x, __shfl_xor_sync(0xffffffffu, m.x, d, 16));
+            m.y = fmaxf(m.y, __shfl_xor_sync(0xffffffffu, m.y, d, 16));
+        }
+        if (wi == 0) S.cM[jj] = m;
+    }
+    __syncthreads();
+    const float2 M = S.cM[j];
+
+    // ---- 3. chunk-local two-sided sums -----------------------------------------
+#pragma unroll
+    for (int i = 0; i < kL; ++i) kk[i] = ex2(add2(kk[i], make_float2(-M.x, -M.y)));  // p_i
+    float2 n[kL], dd[kL];
+    float2 fa = f2(0.0f), fc = f2(0.0f);
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        n[i] = fa;
+        dd[i] = fc;
+        const float2 pv = mul2(kk[i], vv[i]);
+        fa = fma2(alpha, fa, pv);
+        fc = fma2(alpha, fc, kk[i]);
+    }
+    float2 ga = f2(0.0f), gc = f2(0.0f);
+#pragma unroll
+    for (int i = kL - 1; i >= 0; --i) {
+        const float2 pv = mul2(kk[i], vv[i]);
+        n[i] = add2(n[i], fma2(eu, pv, ga));
+        dd[i] = add2(dd[i], fma2(eu, kk[i], gc));
+        ga = fma2(alpha, ga, pv);
+        gc = fma2(alpha, gc, kk[i]);
+    }
+
+    // ---- 4. scan of chunk aggregates -------------------------------------------
+    // within the warp: 4 chunks of 8 tokens
+    const float2 a8 = ex2(mul2(lam2, f2(-8.0f)));
+    const float2 a16 = ex2(mul2(lam2, f2(-16.0f)));
+    float4 Fi = pack4(fa, fc), Gi = pack4(ga, gc);
+    {
+        float4 o = shfl_up4(Fi, 8);
+        if (cq >= 1) Fi = fma4(a8, o, Fi);
+        o = shfl_up4(Fi, 16);
+        if (cq >= 2) Fi = fma4(a16, o, Fi);
+        o = shfl_down4(Gi, 8);
+        if (cq <= 2) Gi = fma4(a8, o, Gi);
+        o = shfl_down4(Gi, 16);
+        if (cq <= 1) Gi = fma4(a16, o, Gi);
+    }
+    float4 X = shfl_up4(Fi, 8), Y = shfl_down4(Gi, 8);
+    if (cq == 0) X = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (cq == 3) Y = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (cq == 3) S.waggF[warp][j] = Fi;
+    if (cq == 0) S.waggB[warp][j] = Gi;
+    __syncthreads();
+    // across warps: 16 lanes per channel pair, one lane per warp
+    if (tid < kNP * 16) {
+        const int jj = tid >> 4, wi = tid & 15;
+        const int ca = c0 + 2 * jj;
+        const float2 lw = mul2(make_float2(ca < p.C ? __ldg(p.w + ca) : 0.0f,
+                                           ca + 1 < p.C ? __ldg(p.w + ca + 1) : 0.0f),
+                               f2(invT * kLog2e));
+        float4 f = (wi < NW) ? S.waggF[wi][jj] : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 gb = (wi < NW) ? S.waggB[wi][jj] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int d = 1; d < 16; d <<= 1) {
+            const float2 m = ex2(mul2(lw, f2(-32.0f * d)));
+            float4 o = shfl_up4(f, d, 16);
+            if (wi >= d) f = fma4(m, o, f);
+            o = shfl_down4(gb, d, 16);
+            if (wi + d < 16) gb = fma4(m, o, gb);
+        }
+        float4 xw = shfl_up4(f, 1, 16), yw = shfl_down4(gb, 1, 16);
+        if (wi == 0) xw = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (wi == 15) yw = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (wi < NW) { S.wcarF[wi][jj] = xw; S.wcarB[wi][jj] = yw; }
+        if (wi == NW - 1) S.caggF[jj] = f;
+        if (wi == 0) S.caggB[jj] = gb;
+    }
+    cg::cluster_group cluster = cg::this_cluster();
+    if (p.ncl > 1) cluster.sync(); else __syncthreads();
+
+    // across the cluster: fold the peers' CTA aggregates as (exponent, sum)
+    if (tid < kCS) {
+        const int lc = tid, jj = lc >> 1, comp = lc & 1;
+        const int c = c0 + lc;
+        const float l2 = (c < p.C ? __ldg(p.w + c) : 0.0f) * (invT * kLog2e);
+        const float span = (float)p.Tc * l2;  // decay exponent across one CTA
+        const float Mme = comp ? S.cM[jj].y : S.cM[jj].x;
+        float mf = -INFINITY, af = 0.f, cf = 0.f;
+        for (int rr = 0; rr < rank; ++rr) {
+            const Scratch* P = cluster.map_shared_rank(&S, rr);
+            const float Mr = comp ? P->cM[jj].y : P->cM[jj].x;
+            const float4 F = P->caggF[jj];
+            const float Fa = comp ? F.y : F.x, Fc = comp ? F.w : F.z;
+            const float md = mf - span;
+            const float nm = fmaxf(md, Mr);
+            const float s0 = ex2(md - nm), s1 = ex2(Mr - nm);
+            af = af * s0 + Fa * s1;
+            cf = cf * s0 + Fc * s1;
+            mf = nm;
+        }
+        float mb = -INFINITY, ab = 0.f, cb = 0.f;
+        for (int rr = p.ncl - 1; rr > rank; --rr) {
+            const Scratch* P = cluster.map_shared_rank(&S, rr);
+            const float Mr = comp ? P->cM[jj].y : P->cM[jj].x;
+            const float4 G = P->caggB[jj];
+            const float Ga = comp ? G.y : G.x, Gc = comp ? G.w : G.z;
+            const float md = mb - span;
+            const float nm = fmaxf(md, Mr);
+            const float s0 = ex2(md - nm), s1 = ex2(Mr - nm);
+            ab = ab * s0 + Ga * s1;
+            cb = cb * s0 + Gc * s1;
+            mb = nm;
+        }
+        const float R = fmaxf(Mme, fmaxf(mf, mb));
+        S.cinfo[lc][0] = ex2(Mme - R);
+        S.cinfo[lc][1] = mf - R;
+        S.cinfo[lc][2] = mb - R;
+        S.cinfo[lc][3] = af;
+        S.cinfo[lc][4] = cf;
+        S.cinfo[lc][5] = ab;
+        S.cinfo[lc][6] = cb;
+    }
+    if (p.ncl > 1) cluster.sync(); else __syncthreads();
+
+    // ---- 5. carries -> outputs ---------------------------------------------
+    const float* ci0 = S.cinfo[2 * j];
+    const float* ci1 = S.cinfo[2 * j + 1];
+    const float2 sl = make_float2(ci0[0], ci1[0]);
+    const float2 ef = make_float2(ci0[1], ci1[1]);
+    const float2 eb = make_float2(ci0[2], ci1[2]);
+    const float4 XW = S.wcarF[warp][j], YW = S.wcarB[warp][j];
+    const float2 pwF = ex2(mul2(lam2, f2(-8.0f * cq)));
+    const float2 pwB = ex2(mul2(lam2, f2(-8.0f * (3 - cq))));
+    const float2 kf = ex2(fma2(lam2, f2(-8.0f * q), ef));
+    const float2 kb = ex2(fma2(lam2, f2(-(float)(p.Tc - kL * (q + 1))), eb));
+    const float2 As = fma2(sl, fma2(pwF, lo2(XW), lo2(X)), mul2(kf, make_float2(ci0[3], ci1[3])));
+    const float2 Cs = fma2(sl, fma2(pwF, hi2(XW), hi2(X)), mul2(kf, make_float2(ci0[4], ci1[4])));
+    const float2 Be = fma2(sl, fma2(pwB, lo2(YW), lo2(Y)), mul2(kb, make_float2(ci0[5], ci1[5])));
+    const float2 De = fma2(sl, fma2(pwB, hi2(YW), hi2(Y)), mul2(kb, make_float2(ci0[6], ci1[6])));
+
+    const char* tr = smem + TR * p.tile_bytes;
+    // powers a^0 .. a^7 by running product (they may underflow to 0 for a
+    // very large positive w, which is exact in the limit)
+    float2 pw[kL];
+    pw[0] = f2(1.0f);
+#pragma unroll
+    for (int i = 1; i < kL; ++i) pw[i] = mul2(pw[i - 1], alpha);
+    int h = h0, w = w0;
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        if (i < nv) {
+            const float2 pf = pw[i], pb = pw[kL - 1 - i];
+            const float2 num = fma2(sl, n[i], fma2(pf, As, mul2(pb, Be)));
+            float2 den = fma2(sl, dd[i], fma2(pf, Cs, mul2(pb, De)));
+            if (GATE) {
+                const float2 rn = mixed_pair<IO, QS>(tr, rbase + i, j, split, ra, rb, h, w, rcm, rcd);
+                den = mul2(den, add2(f2(1.0f), ex2(rn)));
+            }
+            const float2 o = mul2(num, rcp(den));
+            char* dst = p.out + (((size_t)b * p.T + s_tok + i) * p.C + cA) * es;
+            if (p.vec_out && okB) {
+                Io<IO>::st_pair(dst, o);
+            } else {
+                if (okA) Io<IO>::st1(dst, o.x);
+                if (okB) Io<IO>::st1(dst + es, o.y);
+            }
+        }
+        if (QS) { if (++w == p.W) { w = 0; ++h; } }
+    }
+}
+
+}  // namespace vrwkv

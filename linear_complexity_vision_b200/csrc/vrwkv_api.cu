@@ -1,0 +1,303 @@
+// C ABI of the Vision-RWKV spatial-mix core (declared in include/vrwkv.h):
+// host-side argument validation, tiling decisions and kernel launches.
+// Validation happens before any CUDA call, so invalid arguments are
+// rejected without touching the device.
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "vrwkv.h"
+#include "biwkv.cuh"
+#include "qshift.cuh"
+
+namespace {
+
+using namespace vrwkv;
+
+thread_local std::string g_last_error;
+
+vrwkv_status fail(vrwkv_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+vrwkv_status ok() {
+    g_last_error.clear();
+    return VRWKV_OK;
+}
+
+vrwkv_status cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return ok();
+    return fail(VRWKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+int elem_bytes(vrwkv_dtype dt) { return dt == VRWKV_F32 ? 4 : 2; }
+
+int group_size(int C, double gamma) { return (int)((double)C * gamma); }
+
+// Raise the dynamic shared-memory limit of a kernel once per size needed.
+template <typename K>
+cudaError_t ensure_smem(K kernel, std::atomic<int>& granted, int bytes) {
+    if (bytes <= 48 * 1024 || bytes <= granted.load(std::memory_order_relaxed)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) {
+        int cur = granted.load();
+        while (bytes > cur && !granted.compare_exchange_weak(cur, bytes)) {
+        }
+    }
+    return e;
+}
+
+struct FusedPlan {
+    FusedParams p;
+    int ntiles;
+    int layout;
+    bool qs;
+    dim3 grid;
+    int threads;
+    int smem;
+};
+
+template <typename IO, int LAYOUT, bool QS>
+vrwkv_status launch_fused(const FusedPlan& pl, cudaStream_t stream) {
+    static std::atomic<int> granted{0};
+    auto kern = biwkv_fused_kernel<IO, LAYOUT, QS>;
+    cudaError_t e = ensure_smem(kern, granted, pl.smem);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = pl.grid;
+    cfg.blockDim = dim3(pl.threads, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.p.ncl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pl.p.ncl > 1 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, pl.p);
+    if (e != cudaSuccess) return cuda_status(e, "biwkv_fused_kernel launch");
+    return ok();
+}
+
+template <typename IO>
+vrwkv_status dispatch_layout(const FusedPlan& pl, cudaStream_t s) {
+    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
+    case kKV * 2 + 0: return launch_fused<IO, kKV, false>(pl, s);
+    case kKV * 2 + 1: return launch_fused<IO, kKV, true>(pl, s);
+    case kRKV * 2 + 0: return launch_fused<IO, kRKV, false>(pl, s);
+    case kRKV * 2 + 1: return launch_fused<IO, kRKV, true>(pl, s);
+    case kX * 2 + 0: return launch_fused<IO, kX, false>(pl, s);
+    default: return launch_fused<IO, kX, true>(pl, s);
+    }
+}
+
+vrwkv_status check_qs(const vrwkv_qshift_params* qs, int T, int C) {
+    if (qs->H <= 0 || qs->W <= 0) return fail(VRWKV_ERR_INVALID_ARG, "qs: H and W must be positive");
+    if ((long long)qs->H * qs->W != T)
+        return fail(VRWKV_ERR_INVALID_ARG, "qs: H*W (%lld) must equal T (%d)",
+                    (long long)qs->H * qs->W, T);
+    if (qs->shift_pixel < 0) return fail(VRWKV_ERR_INVALID_ARG, "qs: shift_pixel must be >= 0");
+    if (!(qs->gamma >= 0.0 && qs->gamma <= 0.25))
+        return fail(VRWKV_ERR_INVALID_ARG, "qs: gamma must lie in [0, 1/4]");
+    const float* mus[3] = {qs->mu_r, qs->mu_k, qs->mu_v};
+    for (const float* m : mus)
+        if (m && !aligned(m, 4)) return fail(VRWKV_ERR_INVALID_ARG, "qs: mu must be 4-byte aligned");
+    (void)C;
+    return VRWKV_OK;
+}
+
+// Shared front end of vrwkv_biwkv_fwd (gate = false) and vrwkv_spatial_gate.
+vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v, const float* w,
+                         const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
+                         const vrwkv_qshift_params* qs, void* stream) {
+    if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
+        return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B <= 0 || T <= 0 || C <= 0)
+        return fail(VRWKV_ERR_INVALID_ARG, "B, T and C must be positive (got %d, %d, %d)", B, T, C);
+    if (!k || !v || !w || !u || !out || (gate && !r))
+        return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
+    const int es = elem_bytes(dtype);
+    const void* toks[3] = {gate ? r : nullptr, k, v};
+    for (const void* t : toks)
+        if (t && !aligned(t, es)) return fail(VRWKV_ERR_INVALID_ARG, "token tensor misaligned");
+    if (!aligned(out, es)) return fail(VRWKV_ERR_INVALID_ARG, "output misaligned");
+    if (!aligned(w, 4) || !aligned(u, 4)) return fail(VRWKV_ERR_INVALID_ARG, "w/u misaligned");
+    if (qs) {
+        vrwkv_status st = check_qs(qs, T, C);
+        if (st != VRWKV_OK) return st;
+    }
+    const size_t nbytes = (size_t)B * T * C * es;
+    for (const void* t : toks)
+        if (overlaps(out, nbytes, t, nbytes)) return fail(VRWKV_ERR_INVALID_ARG, "output overlaps an input");
+    if (overlaps(out, nbytes, w, (size_t)C * 4) || overlaps(out, nbytes, u, (size_t)C * 4))
+        return fail(VRWKV_ERR_INVALID_ARG, "output overlaps w or u");
+    if (qs) {
+        const float* mus[3] = {qs->mu_r, qs->mu_k, qs->mu_v};
+        for (const float* m : mus)
+            if (overlaps(out, nbytes, m, (size_t)C * 4))
+                return fail(VRWKV_ERR_INVALID_ARG, "output overlaps a mu vector");
+    }
+
+    FusedPlan pl{};
+    FusedParams& p = pl.p;
+    const int slabs = (C + kCS - 1) / kCS;
+    if (B > 65535 || slabs > 65535)
+        return fail(VRWKV_ERR_UNSUPPORTED, "B (%d) or C/16 (%d) exceeds the grid limit 65535", B, slabs);
+    if (T <= kTcMax) {
+        p.ncl = 1;
+        p.Tc = T;
+    } else {
+        p.ncl = (T + kTcMax - 1) / kTcMax;
+        if (p.ncl > kClusterMax)
+            return fail(VRWKV_ERR_UNSUPPORTED, "T = %d exceeds the supported maximum %d", T,
+                        kTcMax * kClusterMax);
+        p.Tc = ((T + p.ncl - 1) / p.ncl + 31) / 32 * 32;
+    }
+    pl.qs = qs != nullptr;
+    if (pl.qs && p.ncl > 1) {
+        long long halo = (long long)qs->shift_pixel * qs->W;
+        p.halo = (int)std::min<long long>(halo, T);
+    } else {
+        p.halo = 0;
+    }
+    p.rows = p.Tc + 2 * p.halo;
+    const int pitch = kCS * es;
+    p.tile_bytes = ((padded_row(p.rows - 1) + 1) * pitch + 127) / 128 * 128;
+    if (!gate) {
+        pl.layout = kKV;
+        p.src[0] = static_cast<const char*>(k);
+        p.src[1] = static_cast<const char*>(v);
+        pl.ntiles = 2;
+    } else if (r == k && k == v) {
+        pl.layout = kX;
+        p.src[0] = static_cast<const char*>(r);
+        pl.ntiles = 1;
+    } else {
+        pl.layout = kRKV;
+        p.src[0] = static_cast<const char*>(r);
+        p.src[1] = static_cast<const char*>(k);
+        p.src[2] = static_cast<const char*>(v);
+        pl.ntiles = 3;
+    }
+    pl.smem = pl.ntiles * p.tile_bytes + (int)sizeof(Scratch);
+    if (pl.smem > 227 * 1024)
+        return fail(VRWKV_ERR_UNSUPPORTED,
+                    "Q-Shift halo of %d tokens needs %d bytes of shared memory (limit %d)", p.halo,
+                    pl.smem, 227 * 1024);
+    p.w = w;
+    p.u = u;
+    p.mu_r = qs ? qs->mu_r : nullptr;
+    p.mu_k = qs ? qs->mu_k : nullptr;
+    p.mu_v = qs ? qs->mu_v : nullptr;
+    p.out = static_cast<char*>(out);
+    p.B = B;
+    p.T = T;
+    p.C = C;
+    p.H = qs ? qs->H : 1;
+    p.W = qs ? qs->W : T;
+    p.s = qs ? qs->shift_pixel : 0;
+    p.g = qs ? group_size(C, qs->gamma) : 0;
+    bool vin = ((size_t)C * es) % 16 == 0;
+    for (int i = 0; i < pl.ntiles; ++i) vin = vin && aligned(p.src[i], 16);
+    p.vec_in = vin ? 1 : 0;
+    p.vec_out = (C % 2 == 0 && aligned(out, 2 * es)) ? 1 : 0;
+    const int nch = (p.Tc + kL - 1) / kL;
+    pl.threads = std::max(kMinThreads, (kNP * nch + 31) / 32 * 32);
+    pl.grid = dim3(p.ncl, slabs, B);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dtype == VRWKV_F32 ? dispatch_layout<float>(pl, s) : dispatch_layout<__nv_bfloat16>(pl, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B, int H, int W, int C,
+                          int shift_pixel, double gamma, vrwkv_dtype dtype, void* stream) {
+    if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
+        return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B <= 0 || H <= 0 || W <= 0 || C <= 0)
+        return fail(VRWKV_ERR_INVALID_ARG, "B, H, W and C must be positive");
+    if ((long long)H * W > 0x7fffffffLL) return fail(VRWKV_ERR_UNSUPPORTED, "H*W too large");
+    if (shift_pixel < 0) return fail(VRWKV_ERR_INVALID_ARG, "shift_pixel must be >= 0");
+    if (!(gamma >= 0.0 && gamma <= 0.25)) return fail(VRWKV_ERR_INVALID_ARG, "gamma must lie in [0, 1/4]");
+    if (!x || !out) return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
+    const int es = elem_bytes(dtype);
+    if (!aligned(x, es) || !aligned(out, es) || (mu && !aligned(mu, 4)))
+        return fail(VRWKV_ERR_INVALID_ARG, "pointer misaligned");
+    const long long T = (long long)H * W;
+    const size_t nbytes = (size_t)B * T * C * es;
+    if (overlaps(out, nbytes, x, nbytes)) return fail(VRWKV_ERR_INVALID_ARG, "output overlaps the input");
+    if (mu && overlaps(out, nbytes, mu, (size_t)C * 4))
+        return fail(VRWKV_ERR_INVALID_ARG, "output overlaps mu");
+
+    QshiftParams p;
+    p.x = static_cast<const char*>(x);
+    p.out = static_cast<char*>(out);
+    p.mu = mu;
+    p.BT = (long long)B * T;
+    p.T = (int)T;
+    p.C = C;
+    p.H = H;
+    p.W = W;
+    p.s = shift_pixel;
+    p.g = group_size(C, gamma);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool vec = ((size_t)C * es) % 16 == 0 && aligned(x, 16) && aligned(out, 16);
+    const long long work = vec ? p.BT * (C / (16 / es)) : p.BT * C;
+    const int threads = 256;
+    const long long blocks = std::min<long long>((work + threads - 1) / threads, 148LL * 16);
+    if (vec) {
+        if (dtype == VRWKV_F32) qshift_vec_kernel<float><<<(unsigned)blocks, threads, 0, s>>>(p);
+        else qshift_vec_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(p);
+    } else {
+        if (dtype == VRWKV_F32) qshift_scalar_kernel<float><<<(unsigned)blocks, threads, 0, s>>>(p);
+        else qshift_scalar_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(p);
+    }
+    return cuda_status(cudaGetLastError(), "qshift kernel launch");
+}
+
+vrwkv_status vrwkv_biwkv_fwd(const void* k, const void* v, const float* w, const float* u, void* wkv,
+                             int B, int T, int C, vrwkv_dtype dtype, const vrwkv_qshift_params* qs,
+                             void* stream) {
+    return fused_entry(false, nullptr, k, v, w, u, wkv, B, T, C, dtype, qs, stream);
+}
+
+vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v, const float* w,
+                                const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
+                                const vrwkv_qshift_params* qs, void* stream) {
+    return fused_entry(true, r, k, v, w, u, out, B, T, C, dtype, qs, stream);
+}
+
+const char* vrwkv_status_string(vrwkv_status status) {
+    switch (status) {
+    case VRWKV_OK: return "VRWKV_OK";
+    case VRWKV_ERR_INVALID_ARG: return "VRWKV_ERR_INVALID_ARG";
+    case VRWKV_ERR_UNSUPPORTED: return "VRWKV_ERR_UNSUPPORTED";
+    case VRWKV_ERR_CUDA: return "VRWKV_ERR_CUDA";
+    default: return "VRWKV_ERR_UNKNOWN";
+    }
+}
+
+const char* vrwkv_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -20,6 +20,8 @@ It wraps ``vrwkv_oracle.c`` (plain C, float64, OpenMP over channel columns):
                        page describes (short sequences only).
 * ``gate``          -- sigma(R) (.) wkv of eq. 2.
 * ``spatial_core``  -- gate(QS_R(r), Bi-WKV(QS_K(k), QS_V(v))).
+* ``spatial_core_points`` -- the same at selected output positions only, by
+                       direct summation of eq. 5 over each needed column.
 
 Every array is row-major (B, T, C) with token index t = h*W + w.
 """
@@ -68,6 +70,8 @@ def _load():
         lib.oracle_biwkv_direct_points.argtypes = [dp, dp, dp, dp, ci, ci, ci,
                                                    i64p, cl, dp]
         lib.oracle_gate.argtypes = [dp, dp, dp, cl]
+        lib.oracle_spatial_core_points.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, ci,
+                                                   ci, ci, cd, ci, ci, i64p, cl, dp]
         lib.oracle_num_threads.restype = ci
         _lib = lib
     return _lib
@@ -187,3 +191,23 @@ def spatial_core(r, k, v, w, u, H=None, W=None, shift_pixel=1, gamma=0.25,
         v = qshift(v, H, W, shift_pixel, gamma, mu_v)
     f = biwkv_direct if method == "direct" else biwkv_rnn
     return gate(r, f(k, v, w, u))
+
+
+def spatial_core_points(r, k, v, w, u, H, W, flat_idx, shift_pixel=1, gamma=0.25,
+                        mu_r=None, mu_k=None, mu_v=None, qshift_on=True,
+                        gate_on=True) -> np.ndarray:
+    """spatial_core (or Bi-WKV alone when gate_on is False) at flat indices
+    (b*T + t)*C + c, building each needed Q-Shifted column on the fly."""
+    k, v, w, u = _d(k), _d(v), _d(w), _d(u)
+    r = _d(r) if r is not None else k
+    B, T, C = k.shape
+    assert T == H * W
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    out = np.empty(idx.shape[0], dtype=np.float64)
+    mus = [None if m is None else _d(m) for m in (mu_r, mu_k, mu_v)]
+    mps = [None if m is None else _ptr(m) for m in mus]
+    _load().oracle_spatial_core_points(
+        _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), mps[0], mps[1], mps[2], B, H, W, C,
+        int(shift_pixel), float(gamma), int(qshift_on), int(gate_on),
+        idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), idx.shape[0], _ptr(out))
+    return out

@@ -330,3 +330,61 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------ */
+/* The spatial-mix core at selected output positions                   */
+/* ------------------------------------------------------------------ */
+
+/* Q-Shifted value of tensor x at (b, t, c): mu*x + (1-mu)*x^dagger, or
+ * x^dagger when mu is NULL, or x itself when qshift_on is 0. */
+static double qs_value(const double* x, const double* mu, long b, long t, int c,
+                       int H, int W, int C, int s, double gamma,
+                       int qshift_on) {
+    const long T = (long)H * W;
+    double xv = x[(b * T + t) * C + c];
+    if (!qshift_on) return xv;
+    int sh, sw;
+    double xd = 0.0;
+    if (qshift_source(c, (int)(t / W), (int)(t % W), H, W, C, s, gamma, 0,
+                      &sh, &sw))
+        xd = x[(b * T + (long)sh * W + sw) * C + c];
+    return mu ? mu[c] * xv + (1.0 - mu[c]) * xd : xd;
+}
+
+/* out[j] = sigma(QS_R(r))[p] * Bi-WKV(QS_K(k), QS_V(v))[p] at the flat
+ * position p = idx[j] = (b*T + t)*C + c, evaluating eq. 5 directly over the
+ * (b, c) column (gate_on = 0 drops the sigma factor; r is then unused). */
+void oracle_spatial_core_points(const double* r, const double* k,
+                                const double* v, const double* w,
+                                const double* u, const double* mu_r,
+                                const double* mu_k, const double* mu_v, int B,
+                                int H, int W, int C, int s, double gamma,
+                                int qshift_on, int gate_on,
+                                const int64_t* idx, long n, double* out) {
+    (void)B;
+    const long T = (long)H * W;
+#pragma omp parallel
+    {
+        double* kc = (double*)malloc(sizeof(double) * (size_t)T);
+        double* vc = (double*)malloc(sizeof(double) * (size_t)T);
+#pragma omp for schedule(dynamic, 4)
+        for (long j = 0; j < n; ++j) {
+            long f = (long)idx[j];
+            int c = (int)(f % C);
+            long bt = f / C, t = bt % T, b = bt / T;
+            for (long i = 0; i < T; ++i) {
+                kc[i] = qs_value(k, mu_k, b, i, c, H, W, C, s, gamma, qshift_on);
+                vc[i] = qs_value(v, mu_v, b, i, c, H, W, C, s, gamma, qshift_on);
+            }
+            double y = biwkv_direct_one(kc, vc, T, w[c], u[c], t);
+            if (gate_on) {
+                double rs = qs_value(r, mu_r, b, t, c, H, W, C, s, gamma,
+                                     qshift_on);
+                y = y * (1.0 / (1.0 + exp(-rs)));
+            }
+            out[j] = y;
+        }
+        free(kc);
+        free(vc);
+    }
+}

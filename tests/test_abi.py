@@ -1,0 +1,87 @@
+"""The C ABI library loads, exports every function include/vrwkv.h declares,
+and rejects invalid arguments on the host (no GPU is touched: validation
+precedes every CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vrwkv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_complexity_vision_b200 import build
+    build.build()
+    import linear_complexity_vision_b200 as vk
+    return vk.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vrwkv_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_operations():
+    names = _declared_functions()
+    for n in ("vrwkv_qshift", "vrwkv_biwkv_fwd", "vrwkv_spatial_gate",
+              "vrwkv_status_string", "vrwkv_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert lib.vrwkv_status_string(0) == b"VRWKV_OK"
+    assert lib.vrwkv_status_string(1) == b"VRWKV_ERR_INVALID_ARG"
+    assert lib.vrwkv_status_string(99) == b"VRWKV_ERR_UNKNOWN"
+
+
+FAKE = 1 << 20  # non-null, never dereferenced: validation fails first
+
+
+def _qs(H, W, s=1, gamma=0.25):
+    import linear_complexity_vision_b200 as vk
+    return ctypes.byref(vk._QsParams(H, W, s, gamma, None, None, None))
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(B=0), "positive"),
+    (dict(C=-1), "positive"),
+    (dict(k=None), "NULL"),
+    (dict(dtype=7), "dtype"),
+    (dict(k=FAKE + 1, dtype=1), "misaligned"),
+    (dict(out=FAKE), "overlaps"),
+    (dict(qs=(14, 15)), "H*W"),
+    (dict(qs=(14, 14, -1)), "shift_pixel"),
+    (dict(qs=(14, 14, 1, 0.3)), "gamma"),
+    (dict(T=8192, qs=None), "T = 8192"),
+])
+def test_biwkv_rejects_invalid_arguments(lib, args, frag):
+    a = dict(k=FAKE, v=FAKE + (1 << 24), w=FAKE + (2 << 24), u=FAKE + (3 << 24),
+             out=FAKE + (4 << 24), B=2, T=196, C=32, dtype=0, qs=None)
+    a.update(args)
+    qs = _qs(*a["qs"]) if a["qs"] else None
+    st = lib.vrwkv_biwkv_fwd(a["k"], a["v"], a["w"], a["u"], a["out"], a["B"], a["T"],
+                             a["C"], a["dtype"], qs, None)
+    assert st in (1, 2)
+    assert frag in lib.vrwkv_last_error().decode()
+
+
+def test_spatial_gate_requires_r(lib):
+    st = lib.vrwkv_spatial_gate(None, FAKE, FAKE, FAKE, FAKE, FAKE + (1 << 24), 1, 4, 4, 0,
+                                None, None)
+    assert st == 1
+
+
+def test_qshift_rejects_invalid_arguments(lib):
+    assert lib.vrwkv_qshift(FAKE, FAKE + (1 << 24), None, 1, 0, 4, 8, 1, 0.25, 0, None) == 1
+    assert lib.vrwkv_qshift(FAKE, FAKE + (1 << 24), None, 1, 4, 4, 8, 1, 0.26, 0, None) == 1
+    assert lib.vrwkv_qshift(FAKE, FAKE + 4, None, 1, 4, 4, 8, 1, 0.25, 0, None) == 1
+    assert b"overlaps" in lib.vrwkv_last_error()

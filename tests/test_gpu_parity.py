@@ -1,0 +1,285 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle,
+element by element, on the same seeded inputs.
+
+Q-Shift must be bit-exact.  Bi-WKV and the gated core must stay within a
+scaled error (see helpers.py) of 1e-4 for float32 I/O and 2e-2 for bfloat16
+I/O.  Small cases compare every element with eq. 5 evaluated directly; large
+cases compare every element with the RNN form (eq. 6-7, itself pinned to
+eq. 5 by the CPU tests) and a seeded sample of elements with eq. 5 directly.
+"""
+import zlib
+
+import numpy as np
+import pytest
+
+from linear_complexity_vision_b200 import synth
+from helpers import (TOL, biwkv_scale, scaled_error, to_device, to_numpy, torch_dtype,
+                     vec_f32)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def vk():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import linear_complexity_vision_b200 as vk
+    vk.load_library()
+    return vk
+
+
+# ---------------------------------------------------------------------------
+# Q-Shift: bit-exact
+# ---------------------------------------------------------------------------
+QS_CASES = [
+    (2, 14, 14, 384, 1, 0.25),   # the 224^2 grid
+    (3, 5, 7, 13, 1, 0.25),      # odd C: scalar path
+    (1, 4, 6, 40, 2, 0.25),      # shift 2
+    (2, 3, 3, 16, 3, 0.25),      # shift >= H and >= W: empty groups
+    (1, 1, 9, 24, 1, 0.25),      # H = 1
+    (1, 9, 1, 24, 1, 0.25),      # W = 1
+    (1, 8, 8, 20, 1, 0.2),       # g = 4
+    (1, 8, 8, 24, 1, 0.25),      # g = 6: vectors straddle group boundaries
+    (2, 6, 6, 32, 0, 0.25),      # shift 0
+    (1, 6, 6, 32, 1, 0.0),       # gamma 0: every channel copied
+    (2, 64, 64, 1024, 1, 0.25),  # the 1024^2 grid at C = 1024
+]
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("use_mu", [True, False])
+@pytest.mark.parametrize("B,H,W,C,s,gamma", QS_CASES)
+def test_qshift_bit_exact(vk, oracle_mod, dt, use_mu, B, H, W, C, s, gamma):
+    seed = 1000 + B * 7 + H * 13 + W * 17 + C + s
+    x = synth.draw(seed, "x", (B, H * W, C), ("normal", 1.0))
+    mu = synth.draw(seed, "mu_k", (C,), ("uniform", 0.0, 1.0))
+    xt, xd = to_device(x, dt)
+    mut, mud = vec_f32(mu)
+    out = vk.qshift(xt, H, W, s, gamma, mu=mut if use_mu else None)
+    want = oracle_mod.qshift_f32(xd.astype(np.float32), H, W, s, gamma,
+                                 mu=mud.astype(np.float32) if use_mu else None,
+                                 round_bf16=(dt == "bf16"))
+    np.testing.assert_array_equal(to_numpy(out), want.astype(np.float64))
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_qshift_unaligned_pointers(vk, oracle_mod, dt):
+    import torch
+    B, H, W, C = 2, 5, 6, 32
+    x = synth.draw(5, "x", (B, H * W, C), ("normal", 1.0))
+    mu = synth.draw(5, "mu_k", (C,), ("uniform", 0.0, 1.0))
+    xt, xd = to_device(x, dt)
+    buf = torch.empty(B * H * W * C + 1, dtype=torch_dtype(dt), device="cuda")
+    xs = buf[1:].view(B, H * W, C)
+    xs.copy_(xt)
+    obuf = torch.empty_like(buf)
+    os_ = obuf[1:].view(B, H * W, C)
+    mut, mud = vec_f32(mu)
+    vk.qshift(xs, H, W, 1, 0.25, mu=mut, out=os_)
+    want = oracle_mod.qshift_f32(xd.astype(np.float32), H, W, 1, 0.25, mu=mud.astype(np.float32),
+                                 round_bf16=(dt == "bf16"))
+    np.testing.assert_array_equal(to_numpy(os_), want.astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# Fused Bi-WKV / spatial gate
+# ---------------------------------------------------------------------------
+def _custom(call, B, H, W, C, dt, seed, s=1, gamma=0.25, **d):
+    dists = {"x": ("normal", 1.0), "r": ("normal", 1.0), "k": ("normal", 1.0),
+             "v": ("normal", 1.0), "w": ("uniform", -5.0, 5.0), "u": ("normal", 1.0)}
+    dists.update(d)
+    return synth.Workload(f"{call}_{B}x{H}x{W}x{C}_{dt}", B, H, W, C, dt, call, dists,
+                          shift_pixel=s, gamma=gamma, seed=seed)
+
+
+def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
+    """Run the workload's call on the GPU and compare with the oracle."""
+    inp = wl.generate()
+    dt = wl.dtype
+    dev, ref = {}, {}
+    for name in wl.tensor_names():
+        a = inp[name] + (kshift if name in ("k", "x") and wl.call == "biwkv" else 0.0)
+        dev[name], ref[name] = to_device(a, dt)
+    for name in ("w", "u", "mu_r", "mu_k", "mu_v"):
+        if name in inp:
+            dev[name], ref[name] = vec_f32(inp[name])
+    if mu_none:
+        for name in ("mu_r", "mu_k", "mu_v"):
+            dev[name] = None
+            ref[name] = None
+    H, W, s, g = wl.H, wl.W, wl.shift_pixel, wl.gamma
+    w, u = ref["w"], ref["u"]
+
+    if wl.call == "biwkv":
+        out = vk.biwkv_fwd(dev["k"], dev["v"], dev["w"], dev["u"])
+        ks, vs, rs = ref["k"], ref["v"], None
+    else:
+        qs = vk.QShift(H, W, s, g, dev.get("mu_r"), dev.get("mu_k"), dev.get("mu_v"))
+        if wl.call == "qshift_biwkv":
+            out = vk.biwkv_fwd(dev["k"], dev["v"], dev["w"], dev["u"], qs=qs)
+            kin, vin, rin = ref["k"], ref["v"], None
+        elif wl.call == "gate_qs":
+            out = vk.spatial_gate(dev["r"], dev["k"], dev["v"], dev["w"], dev["u"], qs=qs)
+            kin, vin, rin = ref["k"], ref["v"], ref["r"]
+        else:  # gate_qs_x: one x feeds r, k and v
+            x = dev["x"]
+            out = vk.spatial_gate(x, x, x, dev["w"], dev["u"], qs=qs)
+            kin = vin = rin = ref["x"]
+        ks = oracle.qshift(kin, H, W, s, g, ref["mu_k"])
+        vs = oracle.qshift(vin, H, W, s, g, ref["mu_v"])
+        rs = None if rin is None else oracle.qshift(rin, H, W, s, g, ref["mu_r"])
+    got = to_numpy(out)
+    assert np.isfinite(got).all()
+
+    B, T, C = ks.shape
+    small = B * C * T * T <= 4e8
+    want = oracle.biwkv_direct(ks, vs, w, u) if small else oracle.biwkv_rnn(ks, vs, w, u)
+    scale = biwkv_scale(oracle, ks, vs, w, u)
+    if rs is not None:
+        want = oracle.gate(rs, want)
+        scale = oracle.gate(rs, scale)
+    tol = TOL[dt]
+    err = scaled_error(got, want, scale)
+    assert err <= tol, f"{wl.name}: scaled error {err:.3e} > {tol}"
+    if not small:
+        rng = np.random.default_rng(wl.seed)
+        idx = rng.choice(got.size, size=min(got.size, 3000), replace=False)
+        pts = oracle.biwkv_points(ks, vs, w, u, idx)
+        if rs is not None:
+            pts = oracle.gate(rs.reshape(-1)[idx], pts)
+        perr = scaled_error(got.reshape(-1)[idx], pts, scale.reshape(-1)[idx])
+        assert perr <= tol, f"{wl.name}: sampled eq. 5 error {perr:.3e} > {tol}"
+    return (got, err) if return_out else err
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+def test_workload_full_size(vk, oracle_mod, cfg):
+    wl = synth.WORKLOADS[cfg]
+    run_fused(vk, oracle_mod, wl)
+
+
+def test_workload2_qshift_of_x_full_size(vk, oracle_mod):
+    wl = synth.WORKLOADS[2]
+    inp = wl.generate()
+    xt, xd = to_device(inp["x"], "f32")
+    mut, mud = vec_f32(inp["mu_r"])
+    out = vk.qshift(xt, wl.H, wl.W, 1, 0.25, mu=mut)
+    want = oracle_mod.qshift_f32(xd.astype(np.float32), wl.H, wl.W, 1, 0.25,
+                                 mu=mud.astype(np.float32))
+    np.testing.assert_array_equal(to_numpy(out), want.astype(np.float64))
+
+
+EDGE = [
+    # call, B, H, W, C, dtype
+    ("biwkv", 2, 1, 1, 16, "f32"),          # T = 1
+    ("biwkv", 2, 1, 2, 16, "f32"),          # T = 2
+    ("biwkv", 1, 1, 7, 5, "f32"),           # one ragged chunk, C odd
+    ("biwkv", 3, 3, 11, 17, "f32"),         # T = 33, C = 17
+    ("biwkv", 1, 1, 1, 1, "bf16"),          # smallest problem
+    ("biwkv", 2, 27, 19, 40, "bf16"),       # T = 513: two CTAs, ragged tail
+    ("biwkv", 2, 25, 40, 32, "f32"),        # T = 1000
+    ("biwkv", 1, 64, 64, 32, "f32"),        # T = 4096 in float32
+    ("biwkv", 1, 50, 60, 24, "bf16"),       # T = 3000
+    ("qshift_biwkv", 2, 1, 9, 24, "f32"),   # H = 1
+    ("qshift_biwkv", 2, 9, 1, 24, "f32"),   # W = 1
+    ("qshift_biwkv", 2, 20, 31, 40, "f32"), # T = 620: halo across CTAs
+    ("qshift_biwkv", 1, 64, 64, 48, "f32"), # 8 CTAs, halo 64
+    ("gate_qs", 2, 7, 9, 20, "bf16"),
+    ("gate_qs", 1, 33, 33, 24, "bf16"),     # T = 1089: 3 CTAs
+    ("gate_qs_x", 2, 14, 14, 96, "bf16"),
+    ("gate_qs_x", 1, 40, 40, 64, "f32"),    # T = 1600 in float32
+    ("gate_qs_x", 1, 3, 11, 6, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=lambda c: "_".join(map(str, c)))
+def test_edge_shapes(vk, oracle_mod, case):
+    call, B, H, W, C, dt = case
+    wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000)
+    run_fused(vk, oracle_mod, wl)
+
+
+@pytest.mark.parametrize("s,H,W", [(2, 6, 7), (3, 2, 300), (5, 4, 4)])
+def test_large_shifts(vk, oracle_mod, s, H, W):
+    wl = _custom("gate_qs", 1, H, W, 24, "bf16", seed=77 + s, s=s)
+    run_fused(vk, oracle_mod, wl)
+    wl = _custom("gate_qs_x", 1, H, W, 24, "f32", seed=78 + s, s=s)
+    run_fused(vk, oracle_mod, wl)
+
+
+def test_mu_none_is_pure_shift(vk, oracle_mod):
+    wl = _custom("gate_qs", 2, 10, 10, 32, "f32", seed=91)
+    run_fused(vk, oracle_mod, wl, mu_none=True)
+    wl = _custom("qshift_biwkv", 1, 30, 30, 16, "f32", seed=92)
+    run_fused(vk, oracle_mod, wl, mu_none=True)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_shift_invariance_in_k(vk, oracle_mod, dt):
+    # adding 80 to every k would overflow exp(k) in float32 without the
+    # running-maximum renormalisation; the result must not change
+    wl = _custom("biwkv", 2, 40, 40, 32, dt, seed=93)
+    a, _ = run_fused(vk, oracle_mod, wl, return_out=True)
+    b, _ = run_fused(vk, oracle_mod, wl, kshift=80.0, return_out=True)
+    assert np.max(np.abs(a - b)) <= (1e-5 if dt == "f32" else 2e-2)
+
+
+@pytest.mark.parametrize("w_kind", ["zero", "huge_positive", "strong_negative"])
+def test_decay_extremes(vk, oracle_mod, w_kind):
+    T = 24 * 30
+    d = {"zero": ("uniform", 0.0, 0.0), "huge_positive": ("uniform", 60.0 * T, 60.0 * T),
+         "strong_negative": ("uniform", -20.0, -10.0)}[w_kind]
+    wl = _custom("biwkv", 1, 24, 30, 32, "f32", seed=94, w=d)
+    run_fused(vk, oracle_mod, wl)
+
+
+def test_large_bonus(vk, oracle_mod):
+    wl = _custom("biwkv", 1, 16, 16, 16, "f32", seed=95, u=("uniform", 30.0, 40.0))
+    run_fused(vk, oracle_mod, wl)
+
+
+def test_deterministic(vk):
+    import torch
+    wl = synth.workload(5, B=2, H=64, W=64, C=64)
+    inp = wl.generate()
+    x, _ = to_device(inp["x"], "bf16")
+    f = {k: vec_f32(inp[k])[0] for k in ("w", "u", "mu_r", "mu_k", "mu_v")}
+    qs = vk.QShift(64, 64, 1, 0.25, f["mu_r"], f["mu_k"], f["mu_v"])
+    a = vk.spatial_gate(x, x, x, f["w"], f["u"], qs=qs)
+    b = vk.spatial_gate(x, x, x, f["w"], f["u"], qs=qs)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_unaligned_fused(vk, oracle_mod):
+    import torch
+    wl = _custom("gate_qs_x", 1, 12, 12, 32, "bf16", seed=96)
+    inp = wl.generate()
+    xt, xd = to_device(inp["x"], "bf16")
+    buf = torch.empty(xt.numel() + 1, dtype=torch.bfloat16, device="cuda")
+    xs = buf[1:].view(xt.shape)
+    xs.copy_(xt)
+    obuf = torch.empty_like(buf)
+    os_ = obuf[1:].view(xt.shape)
+    f = {k: vec_f32(inp[k]) for k in ("w", "u", "mu_r", "mu_k", "mu_v")}
+    qs = vk.QShift(12, 12, 1, 0.25, f["mu_r"][0], f["mu_k"][0], f["mu_v"][0])
+    vk.spatial_gate(xs, xs, xs, f["w"][0], f["u"][0], qs=qs, out=os_)
+    ref = {k: v[1] for k, v in f.items()}
+    want = oracle_mod.spatial_core(xd, xd, xd, ref["w"], ref["u"], 12, 12, 1, 0.25,
+                                   ref["mu_r"], ref["mu_k"], ref["mu_v"])
+    ks = oracle_mod.qshift(xd, 12, 12, 1, 0.25, ref["mu_k"])
+    vs = oracle_mod.qshift(xd, 12, 12, 1, 0.25, ref["mu_v"])
+    rs = oracle_mod.qshift(xd, 12, 12, 1, 0.25, ref["mu_r"])
+    scale = oracle_mod.gate(rs, biwkv_scale(oracle_mod, ks, vs, ref["w"], ref["u"]))
+    assert scaled_error(to_numpy(os_), want, scale) <= TOL["bf16"]
+
+
+def test_invalid_arguments_raise(vk):
+    import torch
+    x = torch.zeros(1, 12, 8, device="cuda")
+    w = torch.zeros(8, device="cuda")
+    with pytest.raises(vk.VrwkvError, match="H\\*W"):
+        vk.biwkv_fwd(x, x, w, w, qs=vk.QShift(3, 5))
+    with pytest.raises(vk.VrwkvError, match="overlaps"):
+        vk.biwkv_fwd(x, x, w, w, out=x)

@@ -190,3 +190,22 @@ def test_spatial_core_composition(oracle_mod):
                                   wl.H, wl.W, 1, 0.25, inp["mu_r"], inp["mu_k"], inp["mu_v"],
                                   method="rnn")
     np.testing.assert_allclose(out, rnn, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("qshift_on,gate_on", [(True, True), (True, False), (False, True)])
+def test_spatial_core_points_match_full(oracle_mod, qshift_on, gate_on):
+    wl = synth.workload(3, B=2, H=6, W=7, C=20)
+    inp = wl.generate()
+    r, k, v = inp["r"], inp["k"], inp["v"]
+    args = (wl.H, wl.W, 1, 0.25, inp["mu_r"], inp["mu_k"], inp["mu_v"])
+    if gate_on:
+        full = oracle_mod.spatial_core(r, k, v, inp["w"], inp["u"], *args, qshift_on=qshift_on)
+    else:
+        ks = oracle_mod.qshift(k, wl.H, wl.W, 1, 0.25, inp["mu_k"])
+        vs = oracle_mod.qshift(v, wl.H, wl.W, 1, 0.25, inp["mu_v"])
+        full = oracle_mod.biwkv_direct(ks, vs, inp["w"], inp["u"])
+    idx = np.arange(0, full.size, 7)
+    pts = oracle_mod.spatial_core_points(r, k, v, inp["w"], inp["u"], wl.H, wl.W, idx, 1, 0.25,
+                                         inp["mu_r"], inp["mu_k"], inp["mu_v"],
+                                         qshift_on=qshift_on, gate_on=gate_on)
+    np.testing.assert_allclose(pts, full.reshape(-1)[idx], rtol=1e-13, atol=1e-14)
