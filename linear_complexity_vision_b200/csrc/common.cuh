@@ -31,6 +31,16 @@ __device__ __forceinline__ float ex2(float x) {
 }
 __device__ __forceinline__ float2 ex2(float2 x) { return make_float2(ex2(x.x), ex2(x.y)); }
 
+// 2^x with x capped at 126, so the result is finite.  Used for decay powers:
+// a span that reaches past the end of the sequence (padding chunks) only ever
+// multiplies zero aggregates, and a finite factor keeps 0 * factor == 0.
+constexpr float kMaxExp2 = 126.0f;
+__device__ __forceinline__ float ex2c(float x) { return ex2(fminf(x, kMaxExp2)); }
+__device__ __forceinline__ float2 ex2c(float2 x) { return make_float2(ex2c(x.x), ex2c(x.y)); }
+__device__ __forceinline__ float2 min2(float2 a, float2 b) {
+    return make_float2(fminf(a.x, b.x), fminf(a.y, b.y));
+}
+
 // Hardware reciprocal (MUFU.RCP, PTX rcp.approx.ftz.f32).
 __device__ __forceinline__ float rcp(float x) {
     float y;

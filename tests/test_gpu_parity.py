@@ -222,7 +222,10 @@ def test_shift_invariance_in_k(vk, oracle_mod, dt):
     wl = _custom("biwkv", 2, 40, 40, 32, dt, seed=93)
     a, _ = run_fused(vk, oracle_mod, wl, return_out=True)
     b, _ = run_fused(vk, oracle_mod, wl, kshift=80.0, return_out=True)
-    assert np.max(np.abs(a - b)) <= (1e-5 if dt == "f32" else 2e-2)
+    # each run matched the oracle on its own inputs above; in bfloat16, k + 80
+    # is re-rounded (ulp 0.5 at 80), so only float32 inputs stay comparable
+    if dt == "f32":
+        assert np.max(np.abs(a - b)) <= 1e-5
 
 
 @pytest.mark.parametrize("w_kind", ["zero", "huge_positive", "strong_negative"])
