@@ -45,7 +45,9 @@ typedef enum {
     VRWKV_OK = 0,
     VRWKV_ERR_INVALID_ARG = 1, /* bad size, pointer, alignment or parameter */
     VRWKV_ERR_UNSUPPORTED = 2, /* valid problem outside the kernels' limits */
-    VRWKV_ERR_CUDA = 3         /* the CUDA runtime reported an error        */
+    VRWKV_ERR_CUDA = 3,        /* the CUDA runtime reported an error        */
+    VRWKV_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see
+                                  vrwkv_device_status)                      */
 } vrwkv_status;
 
 typedef enum {
@@ -103,8 +105,13 @@ vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B,
  *   wkv   (B, T, C) output, same dtype, must not overlap k, v, w or u.
  *   qs    NULL, or Q-Shift parameters applied to k (mu_k) and v (mu_v) on
  *         load (mu_r is ignored); T must then equal qs->H * qs->W.
- * Limits: T <= 4096 (UNSUPPORTED above); with qs, a halo of shift_pixel*W
- *   tokens must fit the kernel's shared-memory tile (UNSUPPORTED otherwise).
+ * Kernels: a TMA fast path serves C % 16 == 0 with 16-byte-aligned inputs
+ *   (and, with qs, a channel-group size int(C*gamma) that is a multiple of
+ *   16 and W <= 256); everything else runs a generic kernel with the same
+ *   results up to rounding.  Setting VRWKV_DISABLE_TMA=1 in the environment
+ *   forces the generic kernel (diagnostics).
+ * Limits: T <= 4096 (UNSUPPORTED above); on the generic kernel with qs, a
+ *   halo of shift_pixel*W tokens must fit its shared-memory tile.
  *   Exponents are renormalised by the running maximum of k, so a constant
  *   added to every k of a channel leaves wkv unchanged; results stay finite
  *   while |w| + (spread of k within a channel) stays well below 80.
@@ -132,6 +139,17 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
                                 const float* w, const float* u, void* out,
                                 int B, int T, int C, vrwkv_dtype dtype,
                                 const vrwkv_qshift_params* qs, void* stream);
+
+/*
+ * vrwkv_device_status -- report and clear kernel-side failures on the
+ * current device.  Kernels that wait for their asynchronous (TMA) tile
+ * copies give up after about two seconds, record the failure in a device
+ * error word and finish (their outputs are then undefined) instead of
+ * hanging.  This call synchronises with the current device, reads that
+ * word, clears it and returns VRWKV_ERR_TIMEOUT if it was set, VRWKV_OK
+ * otherwise (VRWKV_ERR_CUDA if the device cannot be read).
+ */
+vrwkv_status vrwkv_device_status(void);
 
 /* Static, never-NULL name of a status code. */
 const char* vrwkv_status_string(vrwkv_status status);

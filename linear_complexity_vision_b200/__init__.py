@@ -8,6 +8,7 @@ There is no fallback: if the library is missing, the calls raise.
     qshift(x, H, W, shift_pixel=1, gamma=0.25, mu=None)
     biwkv_fwd(k, v, w, u, qs=None)
     spatial_gate(r, k, v, w, u, qs=None)
+    device_status()     # synchronise; raise if a kernel's bounded wait ran out
 
 Token tensors are contiguous (B, T, C) CUDA tensors of dtype float32 or
 bfloat16; w, u and mu vectors are contiguous float32 CUDA tensors of
@@ -64,6 +65,8 @@ def load_library():
         lib.vrwkv_spatial_gate.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                            ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_spatial_gate.restype = ci
+        lib.vrwkv_device_status.argtypes = []
+        lib.vrwkv_device_status.restype = ci
         lib.vrwkv_status_string.argtypes = [ci]
         lib.vrwkv_status_string.restype = ctypes.c_char_p
         lib.vrwkv_last_error.argtypes = []
@@ -160,3 +163,9 @@ def spatial_gate(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
         r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
         B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
     return out
+
+
+def device_status() -> None:
+    """Synchronise with the current device and raise VrwkvError if a kernel
+    recorded a timed-out wait since the last check (vrwkv_device_status)."""
+    _check(load_library().vrwkv_device_status())

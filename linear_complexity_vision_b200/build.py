@@ -10,7 +10,6 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libvrwkv.so")
 SOURCES = ["vrwkv_api.cu"]
-HEADERS = ["common.cuh", "qshift.cuh", "biwkv.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
               "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-O2",
@@ -21,7 +20,7 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh"))]
     deps.append(os.path.join(ROOT, "include", "vrwkv.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 

@@ -1,0 +1,516 @@
+// Fused Q-Shift -> Bi-WKV -> sigma(R) gate, TMA fast path for sm_100a.
+//
+// Same chunked two-sided scan as the generic kernel (biwkv.cuh) evaluating
+// Bi-WKV of "Vision-RWKV Backbone", Linear Complexity Bidirectional
+// Attention, eq. 5, on inputs Q-Shifted per Quad-Directional Token Shift,
+// eq. 9, gated per Overall Architecture, eq. 2:
+//
+//   A_t = sum_{i<t} a^{t-1-i} p_i v_i,  B_t = sum_{i>t} a^{i-t-1} p_i v_i,
+//   C_t, D_t with v = 1,  a = e^{-w/T},  p_i = e^{k_i - M},
+//   wkv_t = (A_t + B_t + e^u p_t v_t) / (C_t + D_t + e^u p_t).
+//
+// What makes this path fast:
+//  * Tiles arrive by TMA (cp.async.bulk.tensor, no multicast) with an element
+//    stride of 8 along the token axis: box i (i = 0..7) holds tokens 8q + i,
+//    so sub-tile i, row q is token i of chunk q.  At each step the four
+//    chunks a warp reads are four consecutive rows: conflict-free, and every
+//    address is a compile-time offset from one base register.
+//  * With Q-Shift the (B, T, C) tensor is described as the 4-D image
+//    (C, W, H, B) (W a multiple of 8); the shifted tile x_shift is the same
+//    set of boxes displaced by +-s along w or h.  TMA fills out-of-image
+//    elements with zeros, which is exactly Q-Shift's zero border, so no
+//    per-token shift arithmetic remains: token t of both tiles sits at the
+//    same shared-memory offset.  A CTA's 16 channels lie in one channel
+//    group (the host requires the group size to be a multiple of 16).
+//  * 256 threads and <= 128 registers per thread: two CTAs per SM, so one
+//    CTA's barriers and scans overlap the other's arithmetic.  Sequences
+//    longer than 256 tokens split over a thread-block cluster of up to 16
+//    CTAs along T; CTA aggregates travel through distributed shared memory.
+//  * Decay powers a^(8m) come from a per-CTA table (one exp2 each), the
+//    bf16 unpack is integer arithmetic, and arithmetic is packed float2.
+// Exponents are base 2 (log2 e is folded into k, u, w and r).
+#pragma once
+
+#include <cuda.h>
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace vrwkv {
+namespace fast {
+
+namespace cg = cooperative_groups;
+
+constexpr int kCS = 16;         // channels per CTA
+constexpr int kNP = kCS / 2;    // channel pairs per CTA
+constexpr int kL = 8;           // tokens per thread chunk
+constexpr int kThreads = 256;   // threads per CTA
+constexpr int kNW = kThreads / 32;
+constexpr int kTcMax = kThreads / kNP * kL;  // 256 tokens per CTA
+constexpr int kClusterMax = 16;
+constexpr int kTab = kTcMax / kL;            // a^(8m), m < 32
+constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+
+enum Layout { kKV = 0, kRKV = 1, kX = 2 };
+
+struct alignas(64) Params {
+    CUtensorMap map[3];  // one per distinct source tensor (tile order below)
+    const float* w;
+    const float* u;
+    const float* mu[3];  // mu of r, k, v (each nullable)
+    char* out;
+    unsigned int* err;   // device error word (bounded waits)
+    int B, T, C;
+    int H, W, s, g;      // Q-Shift grid, shift, group size
+    int Tc;              // tokens per CTA (multiple of 32 when ncl > 1)
+    int rows;            // image rows per CTA (Q-Shift path): Tc = rows * W
+    int ncl;             // CTAs per column (cluster size)
+    int tile_bytes;      // bytes per tile: 8 sub-tiles of 32 token rows
+    int box_bytes;       // bytes one strided box delivers (zero fill included)
+};
+
+struct alignas(16) Scratch {
+    float2 tab[kTab][kNP];      // a^(8m) per channel pair
+    float2 wmax[kNP][kNW];      // per-warp maxima of k
+    float4 waggF[kNP][kNW];     // per-warp forward aggregates (A.xy, C.xy)
+    float4 waggB[kNP][kNW];     // per-warp backward aggregates
+    float4 wcarF[kNP][kNW];     // exclusive forward carry into each warp
+    float4 wcarB[kNP][kNW];     // exclusive backward carry into each warp
+    float cM[kCS];              // CTA maximum of k times log2(e), read by peers
+    float4 caggF[kNP];          // CTA forward aggregate, read by peers
+    float4 caggB[kNP];          // CTA backward aggregate, read by peers
+    float4 cscale[kCS];         // per channel: sl (scale of this CTA's own sums)
+    float4 ccarry[kCS];         // per channel: carries Af, Cf, Bb, Db
+    unsigned long long bar;     // TMA completion barrier
+};
+
+// ---- PTX wrappers ----------------------------------------------------------
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+    return (unsigned)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+// try_wait with a suspend-time hint (ns): the thread sleeps in hardware until
+// the phase completes or the hint elapses, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+}
+// Wait for phase 0 of the barrier; give up after ~2 s, record the failure in
+// the device error word and continue (the caller's barriers stay matched).
+__device__ __forceinline__ void mbar_wait_bounded(unsigned long long* bar, unsigned* err) {
+    if (mbar_try_wait(bar, 0)) return;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, 0)) {
+        if (clock64() - t0 > kWaitCycles) {
+            atomicOr(err, 1u);
+            return;
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            unsigned long long* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            int c3, unsigned long long* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Channel pair of one token from a tile, as float2.
+template <typename IO>
+__device__ __forceinline__ float2 lds_pair(const char* tile, int off);
+template <>
+__device__ __forceinline__ float2 lds_pair<__nv_bfloat16>(const char* tile, int off) {
+    const unsigned u = *reinterpret_cast<const unsigned*>(tile + off);
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+template <>
+__device__ __forceinline__ float2 lds_pair<float>(const char* tile, int off) {
+    return *reinterpret_cast<const float2*>(tile + off);
+}
+
+__device__ __forceinline__ float4 shfl_up4(float4 v, int d, int width) {
+    return make_float4(__shfl_up_sync(0xffffffffu, v.x, d, width), __shfl_up_sync(0xffffffffu, v.y, d, width),
+                       __shfl_up_sync(0xffffffffu, v.z, d, width), __shfl_up_sync(0xffffffffu, v.w, d, width));
+}
+__device__ __forceinline__ float4 shfl_down4(float4 v, int d, int width) {
+    return make_float4(__shfl_down_sync(0xffffffffu, v.x, d, width),
+                       __shfl_down_sync(0xffffffffu, v.y, d, width),
+                       __shfl_down_sync(0xffffffffu, v.z, d, width),
+                       __shfl_down_sync(0xffffffffu, v.w, d, width));
+}
+__device__ __forceinline__ float4 fma4(float2 m, float4 x, float4 y) {
+    const float2 a = fma2(m, make_float2(x.x, x.y), make_float2(y.x, y.y));
+    const float2 c = fma2(m, make_float2(x.z, x.w), make_float2(y.z, y.w));
+    return make_float4(a.x, a.y, c.x, c.y);
+}
+__device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float4 zero4() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+
+template <typename IO, int LAYOUT, bool QS>
+__global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_constant__ Params p) {
+    constexpr bool GATE = LAYOUT != kKV;
+    constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
+    constexpr int NTILE = NSRC * (QS ? 2 : 1);
+    constexpr int SR = 0;
+    constexpr int SK = LAYOUT == kRKV ? 1 : 0;
+    constexpr int SV = LAYOUT == kKV ? 1 : (LAYOUT == kRKV ? 2 : 0);
+    constexpr int es = Io<IO>::kBytes;
+    constexpr int RB = kCS * es;  // bytes per token row of a tile
+    constexpr int PB = 2 * es;    // bytes per channel pair
+
+    // dynamic shared memory, re-aligned to 128 bytes for the TMA
+    // destinations; the host adds 128 bytes of slack
+    extern __shared__ __align__(128) char smem_raw[];
+    char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+    Scratch& S = *reinterpret_cast<Scratch*>(smem + NTILE * p.tile_bytes);
+
+    const int tid = threadIdx.x;
+    const int j = tid & 7;       // channel pair
+    const int q = tid >> 3;      // chunk within the CTA
+    const int cq = q & 3;        // chunk within the warp
+    const int warp = tid >> 5;
+    const int rank = blockIdx.x;
+    const int c0 = blockIdx.y * kCS;
+    const int b = blockIdx.z;
+    const int t0 = rank * p.Tc;
+    const int tend = min(p.T, t0 + p.Tc);
+
+    // group of this CTA's channels (Q-Shift): 0..3 shifted, 4 copied
+    int grp = 4;
+    if (QS && p.g > 0) grp = min(c0 / p.g, 4);
+    const bool shifted = QS && grp < 4;
+
+    // ---- issue the tile loads: lane i of warp 0 loads sub-tile i of each tile
+    constexpr int SUB = kTcMax / kL * RB;  // bytes per sub-tile (32 token rows)
+    if (tid == 0) mbar_init(&S.bar, 1);
+    __syncthreads();
+    if (warp == 0) {
+        if (tid == 0) {
+            mbar_expect_tx(&S.bar, (unsigned)p.box_bytes * (unsigned)(kL * NSRC * (shifted ? 2 : 1)));
+        }
+        __syncwarp();
+        if (tid < kL) {
+            const int i = tid;
+            const int h0 = rank * p.rows;
+            for (int s = 0; s < NSRC; ++s) {
+                char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB;
+                if (!QS) {
+                    tma_load_3d(plain, &p.map[s], c0, t0 + i, b, &S.bar);
+                } else {
+                    tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar);
+                    if (shifted) {
+                        const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
+                        const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
+                        tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, h0 + dh, b, &S.bar);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- per-thread constants (overlap the copies) ---------------------------
+    const int cA = c0 + 2 * j;
+    const float invT = 1.0f / (float)p.T;
+    const float2 wv = make_float2(__ldg(p.w + cA), __ldg(p.w + cA + 1));
+    const float2 uv = make_float2(__ldg(p.u + cA), __ldg(p.u + cA + 1));
+    const float2 lam2 = mul2(wv, f2(invT * kLog2e));  // w / T in base-2 units
+    const float2 alpha = ex2c(make_float2(-lam2.x, -lam2.y));
+    const float2 eu = ex2(mul2(uv, f2(kLog2e)));
+    auto mu_of = [&](const float* m) {
+        return m ? make_float2(__ldg(m + cA), __ldg(m + cA + 1)) : f2(0.0f);
+    };
+    const float2 muk = QS ? mu_of(p.mu[1]) : f2(1.0f);
+    const float2 muv = QS ? mu_of(p.mu[2]) : f2(1.0f);
+    const float2 mur = (QS && GATE) ? mu_of(p.mu[0]) : f2(1.0f);
+    // decay table a^(8m): one entry (2 channels) per thread
+    {
+        const int m = tid >> 3, jj = tid & 7;
+        const float2 l = mul2(make_float2(__ldg(p.w + c0 + 2 * jj), __ldg(p.w + c0 + 2 * jj + 1)),
+                              f2(invT * kLog2e));
+        S.tab[m][jj] = ex2c(mul2(l, f2(-8.0f * m)));
+    }
+
+    const int s_tok = t0 + q * kL;
+    const int nv = max(0, min(kL, tend - s_tok));
+    const int rowoff = q * RB + j * PB;  // token i of the chunk: + i * SUB
+
+    // one thread waits for the tiles; the others sleep at the CTA barrier
+    if (tid == 0) mbar_wait_bounded(&S.bar, p.err);
+    __syncthreads();
+
+    // ---- 1. load, Q-Shift mix, chunk maximum -----------------------------------
+    const char* tK = smem + (QS ? 2 * SK : SK) * p.tile_bytes;
+    const char* tV = smem + (QS ? 2 * SV : SV) * p.tile_bytes;
+    const char* tR = smem + (QS ? 2 * SR : SR) * p.tile_bytes;
+    const int dsh = shifted ? p.tile_bytes : 0;  // shifted tile = plain + dsh
+    float2 kk[kL], vv[kL], gg[kL];
+    float2 mx = f2(-INFINITY);
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        const int o = rowoff + i * SUB;
+        float2 k, v, r;
+        if (QS) {
+            if (LAYOUT == kX) {
+                const float2 x = lds_pair<IO>(tK, o), xd = lds_pair<IO>(tK + dsh, o);
+                const float2 d = add2(x, make_float2(-xd.x, -xd.y));
+                k = fma2(muk, d, xd);
+                v = fma2(muv, d, xd);
+                r = fma2(mur, d, xd);
+            } else {
+                const float2 xk = lds_pair<IO>(tK, o), xkd = lds_pair<IO>(tK + dsh, o);
+                const float2 xv = lds_pair<IO>(tV, o), xvd = lds_pair<IO>(tV + dsh, o);
+                k = fma2(muk, add2(xk, make_float2(-xkd.x, -xkd.y)), xkd);
+                v = fma2(muv, add2(xv, make_float2(-xvd.x, -xvd.y)), xvd);
+                if (GATE) {
+                    const float2 xr = lds_pair<IO>(tR, o), xrd = lds_pair<IO>(tR + dsh, o);
+                    r = fma2(mur, add2(xr, make_float2(-xrd.x, -xrd.y)), xrd);
+                }
+            }
+        } else {
+            k = lds_pair<IO>(tK, o);
+            v = lds_pair<IO>(tV, o);
+            if (GATE) r = lds_pair<IO>(tR, o);
+        }
+        if (GATE) gg[i] = ex2(mul2(r, f2(-kLog2e)));
+        // tokens past the sequence end hold zeros (TMA fill) or stale shared
+        // memory (rows beyond a short box): mask both so p = 0 and p*v = 0
+        kk[i] = (i < nv) ? k : f2(-INFINITY);
+        vv[i] = (i < nv) ? v : f2(0.0f);
+        mx = max2(mx, kk[i]);
+    }
+#pragma unroll
+    for (int d = 8; d <= 16; d <<= 1) {
+        mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
+        mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
+    }
+    if (cq == 0) S.wmax[j][warp] = mx;
+    __syncthreads();
+    float2 M = S.wmax[j][0];
+#pragma unroll
+    for (int w = 1; w < kNW; ++w) M = max2(M, S.wmax[j][w]);
+
+    // ---- 2. p = 2^(k - M), chunk-local two-sided sums ---------------------------
+    const float2 negM = mul2(M, f2(-kLog2e));
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        kk[i] = ex2(fma2(kk[i], f2(kLog2e), negM));  // p_i (0 beyond T)
+        vv[i] = mul2(kk[i], vv[i]);                  // p_i v_i
+    }
+    float2 n[kL], dd[kL];
+    float2 fa = f2(0.0f), fc = f2(0.0f);
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        n[i] = fa;
+        dd[i] = fc;
+        fa = fma2(alpha, fa, vv[i]);
+        fc = fma2(alpha, fc, kk[i]);
+    }
+    float2 ga = f2(0.0f), gc = f2(0.0f);
+#pragma unroll
+    for (int i = kL - 1; i >= 0; --i) {
+        n[i] = add2(n[i], fma2(eu, vv[i], ga));
+        dd[i] = add2(dd[i], fma2(eu, kk[i], gc));
+        ga = fma2(alpha, ga, vv[i]);
+        gc = fma2(alpha, gc, kk[i]);
+    }
+
+    // ---- 3. scans: warp, CTA, cluster --------------------------------------------
+    float4 Fi = make_float4(fa.x, fa.y, fc.x, fc.y);
+    float4 Gi = make_float4(ga.x, ga.y, gc.x, gc.y);
+    {
+        const float2 a8 = S.tab[1][j], a16 = S.tab[2][j];
+        float4 o = shfl_up4(Fi, 8, 32);
+        if (cq >= 1) Fi = fma4(a8, o, Fi);
+        o = shfl_up4(Fi, 16, 32);
+        if (cq >= 2) Fi = fma4(a16, o, Fi);
+        o = shfl_down4(Gi, 8, 32);
+        if (cq <= 2) Gi = fma4(a8, o, Gi);
+        o = shfl_down4(Gi, 16, 32);
+        if (cq <= 1) Gi = fma4(a16, o, Gi);
+    }
+    float4 X = shfl_up4(Fi, 8, 32), Y = shfl_down4(Gi, 8, 32);
+    if (cq == 0) X = zero4();
+    if (cq == 3) Y = zero4();
+    if (cq == 3) S.waggF[j][warp] = Fi;
+    if (cq == 0) S.waggB[j][warp] = Gi;
+    __syncthreads();
+    if (tid < kNP * kNW) {  // 64 threads: one per (pair, warp)
+        const int jj = tid >> 3, wi = tid & 7;
+        float4 f = S.waggF[jj][wi], gb = S.waggB[jj][wi];
+#pragma unroll
+        for (int d = 1; d < kNW; d <<= 1) {
+            const float2 m = S.tab[4 * d][jj];  // a^(32 d)
+            float4 o = shfl_up4(f, d, kNW);
+            if (wi >= d) f = fma4(m, o, f);
+            o = shfl_down4(gb, d, kNW);
+            if (wi + d < kNW) gb = fma4(m, o, gb);
+        }
+        float4 xw = shfl_up4(f, 1, kNW), yw = shfl_down4(gb, 1, kNW);
+        if (wi == 0) xw = zero4();
+        if (wi == kNW - 1) yw = zero4();
+        S.wcarF[jj][wi] = xw;
+        S.wcarB[jj][wi] = yw;
+        // the CTA's forward aggregate sits at its last real warp (Tc may be
+        // shorter than 256 tokens; padding warps after it hold zeros)
+        if (wi == p.Tc / 32 - 1) S.caggF[jj] = f;
+        if (wi == 0) {
+            S.caggB[jj] = gb;
+            float2 Mj = S.wmax[jj][0];
+#pragma unroll
+            for (int w = 1; w < kNW; ++w) Mj = max2(Mj, S.wmax[jj][w]);
+            // published in base 2, the unit of the cluster fold's exponents
+            S.cM[2 * jj] = Mj.x * kLog2e;
+            S.cM[2 * jj + 1] = Mj.y * kLog2e;
+        }
+    }
+    if (p.ncl > 1) {
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    } else {
+        __syncthreads();
+    }
+    // Exchange with the other CTAs of the column.  Thread (channel lc, peer
+    // rr) reads peer rr's CTA record for channel lc straight from distributed
+    // shared memory; each 16-lane segment then holds one channel's column.
+    // The segment maximum of the peers' exponents is the common reference;
+    // forward and backward carries are 16-lane shuffle scans with the
+    // one-CTA decay a^Tc, a^(2 Tc), ...
+    float2 cs_sl = f2(1.0f), cs_af = f2(0.0f), cs_cf = f2(0.0f), cs_bb = f2(0.0f), cs_db = f2(0.0f);
+    if (p.ncl > 1) {
+        const int lc = tid >> 4, rr = tid & 15;
+        float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
+        if (rr < p.ncl) {
+            cg::cluster_group cluster = cg::this_cluster();
+            const Scratch* P = cluster.map_shared_rank(&S, rr);
+            const float4 F = P->caggF[lc >> 1], G = P->caggB[lc >> 1];
+            const bool hi = lc & 1;
+            Mr = P->cM[lc];
+            fa2 = hi ? F.y : F.x;
+            fc2 = hi ? F.w : F.z;
+            ga2 = hi ? G.y : G.x;
+            gc2 = hi ? G.w : G.z;
+        }
+        // release: this thread's reads of the peers' shared memory are
+        // complete before any peer can pass its final wait and exit
+        cluster_arrive_release();
+        float Mc = Mr;
+#pragma unroll
+        for (int d = 8; d >= 1; d >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, 16));
+        const float sc = ex2(Mr - Mc);  // 0 for lanes past the cluster
+        fa2 *= sc;
+        fc2 *= sc;
+        ga2 *= sc;
+        gc2 *= sc;
+        const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
+#pragma unroll
+        for (int d = 1; d < kClusterMax; d <<= 1) {
+            const float m = ex2c(-(float)(p.Tc * d) * l2);  // decay across d CTAs
+            const float ua = __shfl_up_sync(0xffffffffu, fa2, d, 16);
+            const float uc = __shfl_up_sync(0xffffffffu, fc2, d, 16);
+            const float da = __shfl_down_sync(0xffffffffu, ga2, d, 16);
+            const float dc = __shfl_down_sync(0xffffffffu, gc2, d, 16);
+            if (rr >= d) {
+                fa2 = fmaf(m, ua, fa2);
+                fc2 = fmaf(m, uc, fc2);
+            }
+            if (rr + d < kClusterMax) {
+                ga2 = fmaf(m, da, ga2);
+                gc2 = fmaf(m, dc, gc2);
+            }
+        }
+        // exclusive carries of this CTA: inclusive forward at rank-1,
+        // inclusive backward at rank+1 (zero past the ends)
+        const float Af = __shfl_sync(0xffffffffu, fa2, max(rank - 1, 0), 16);
+        const float Cf = __shfl_sync(0xffffffffu, fc2, max(rank - 1, 0), 16);
+        const float Bb = __shfl_sync(0xffffffffu, ga2, min(rank + 1, kClusterMax - 1), 16);
+        const float Db = __shfl_sync(0xffffffffu, gc2, min(rank + 1, kClusterMax - 1), 16);
+        const float Mme = __shfl_sync(0xffffffffu, Mr, rank, 16);
+        if (rr == 0) {
+            S.cscale[lc] = make_float4(ex2(Mme - Mc), 0.f, 0.f, 0.f);
+            S.ccarry[lc] = make_float4(rank > 0 ? Af : 0.f, rank > 0 ? Cf : 0.f,
+                                       rank + 1 < p.ncl ? Bb : 0.f, rank + 1 < p.ncl ? Db : 0.f);
+        }
+        __syncthreads();
+        const float4 s0 = S.cscale[2 * j], s1 = S.cscale[2 * j + 1];
+        const float4 k0 = S.ccarry[2 * j], k1 = S.ccarry[2 * j + 1];
+        cs_sl = make_float2(s0.x, s1.x);
+        cs_af = make_float2(k0.x, k1.x);
+        cs_cf = make_float2(k0.y, k1.y);
+        cs_bb = make_float2(k0.z, k1.z);
+        cs_db = make_float2(k0.w, k1.w);
+    }
+
+    // ---- 4. carries -> outputs ---------------------------------------------------
+    const float2 sl = cs_sl;
+    const float4 XW = S.wcarF[j][warp], YW = S.wcarB[j][warp];
+    const float2 pwF = S.tab[cq][j], pwB = S.tab[3 - cq][j];
+    const float2 kf = S.tab[q][j];                              // a^(8q): CTA start -> chunk
+    const float2 kb = S.tab[max(0, p.Tc / kL - 1 - q)][j];      // chunk end -> CTA end
+    const float2 As = fma2(sl, fma2(pwF, lo2(XW), lo2(X)), mul2(kf, cs_af));
+    const float2 Cs = fma2(sl, fma2(pwF, hi2(XW), hi2(X)), mul2(kf, cs_cf));
+    const float2 Be = fma2(sl, fma2(pwB, lo2(YW), lo2(Y)), mul2(kb, cs_bb));
+    const float2 De = fma2(sl, fma2(pwB, hi2(YW), hi2(Y)), mul2(kb, cs_db));
+
+    float2 pw[kL];
+    pw[0] = f2(1.0f);
+#pragma unroll
+    for (int i = 1; i < kL; ++i) pw[i] = min2(mul2(pw[i - 1], alpha), f2(0x1p126f));
+    // results go to the first input tile (dead since the load phase), at the
+    // same conflict-free offsets, then leave as coalesced 16-byte stores
+    char* tout = smem;
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        const float2 num = fma2(sl, n[i], fma2(pw[i], As, mul2(pw[kL - 1 - i], Be)));
+        float2 den = fma2(sl, dd[i], fma2(pw[i], Cs, mul2(pw[kL - 1 - i], De)));
+        if (GATE) den = fma2(den, gg[i], den);
+        Io<IO>::st_pair(tout + rowoff + i * SUB, mul2(num, rcp(den)));
+    }
+    __syncthreads();
+    {
+        constexpr int UPS = SUB / 16;  // 16-byte units per sub-tile
+        char* gout = p.out + ((size_t)b * p.T + t0) * p.C * es + (size_t)c0 * es;
+#pragma unroll
+        for (int u = tid; u < kL * UPS; u += kThreads) {
+            const int i = u / UPS, o = (u - i * UPS) * 16;
+            const int t = (o / RB) * kL + i;  // token within the CTA
+            if (t0 + t < tend)
+                *reinterpret_cast<uint4*>(gout + (size_t)t * p.C * es + (o % RB)) =
+                    *reinterpret_cast<const uint4*>(tout + i * SUB + o);
+        }
+    }
+    if (p.ncl > 1) cluster_wait_acquire();  // peers finished reading this CTA
+}
+
+}  // namespace fast
+}  // namespace vrwkv

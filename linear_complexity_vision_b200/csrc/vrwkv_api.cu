@@ -7,11 +7,19 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
+#include <mutex>
 #include <string>
+
+#include <cuda.h>
 
 #include "vrwkv.h"
 #include "biwkv.cuh"
+#include "biwkv_tma.cuh"
 #include "qshift.cuh"
+
+// Device error word: set by kernels whose bounded waits ran out (bit 0).
+__device__ unsigned int g_vrwkv_device_error;
 
 namespace {
 
@@ -109,6 +117,230 @@ vrwkv_status dispatch_layout(const FusedPlan& pl, cudaStream_t s) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// TMA fast path
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// Device address of the error word on the current device (looked up once per
+// device; the symbol's host-side name is not a device address).
+unsigned int* device_error_word() {
+    static unsigned int* addr[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_vrwkv_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned int*>(a);
+    }
+    return addr[dev];
+}
+
+bool tma_disabled() {
+    const char* e = getenv("VRWKV_DISABLE_TMA");
+    return e && e[0] && e[0] != '0';
+}
+
+struct FastPlan {
+    fast::Params p;
+    int layout;
+    bool qs;
+    dim3 grid;
+    int smem;
+};
+
+template <typename IO, int LAYOUT, bool QS>
+vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
+    auto kern = fast::biwkv_tma_kernel<IO, LAYOUT, QS>;
+    static std::atomic<int> granted{0};
+    static std::atomic<int> nonportable{0};
+    cudaError_t e = ensure_smem(kern, granted, pl.smem);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    if (pl.p.ncl > 8 && !nonportable.load()) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            *fell_back = true;
+            return VRWKV_OK;
+        }
+        nonportable.store(1);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = pl.grid;
+    cfg.blockDim = dim3(fast::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.p.ncl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pl.p.ncl > 1 ? 1 : 0;
+    if (pl.p.ncl > 1) {
+        // a cluster shape the GPU cannot co-schedule falls back to the generic kernel
+        static std::atomic<int> checked[fast::kClusterMax + 1];
+        int v = checked[pl.p.ncl].load();
+        if (v == 0) {
+            int n = 0;
+            cudaError_t oe = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+            v = (oe == cudaSuccess && n > 0) ? 1 : -1;
+            if (oe != cudaSuccess) cudaGetLastError();
+            checked[pl.p.ncl].store(v);
+        }
+        if (v < 0) {
+            *fell_back = true;
+            return VRWKV_OK;
+        }
+    }
+    e = cudaLaunchKernelEx(&cfg, kern, pl.p);
+    if (e != cudaSuccess) return cuda_status(e, "biwkv_tma_kernel launch");
+    return ok();
+}
+
+template <typename IO>
+vrwkv_status dispatch_fast(const FastPlan& pl, cudaStream_t s, bool* fb) {
+    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
+    case fast::kKV * 2 + 0: return launch_fast<IO, fast::kKV, false>(pl, s, fb);
+    case fast::kKV * 2 + 1: return launch_fast<IO, fast::kKV, true>(pl, s, fb);
+    case fast::kRKV * 2 + 0: return launch_fast<IO, fast::kRKV, false>(pl, s, fb);
+    case fast::kRKV * 2 + 1: return launch_fast<IO, fast::kRKV, true>(pl, s, fb);
+    case fast::kX * 2 + 0: return launch_fast<IO, fast::kX, false>(pl, s, fb);
+    default: return launch_fast<IO, fast::kX, true>(pl, s, fb);
+    }
+}
+
+// Plan the TMA path; returns false when the problem is outside its limits
+// (the generic kernel then runs).
+bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void* v, const float* w,
+               const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
+               const vrwkv_qshift_params* qs) {
+    if (tma_disabled()) return false;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const int es = elem_bytes(dtype);
+    if (C % fast::kCS != 0 || !aligned(out, 16)) return false;
+    const void* srcs[3];
+    int nsrc;
+    if (!gate) {
+        pl.layout = fast::kKV;
+        srcs[0] = k;
+        srcs[1] = v;
+        nsrc = 2;
+    } else if (r == k && k == v) {
+        pl.layout = fast::kX;
+        srcs[0] = r;
+        nsrc = 1;
+    } else {
+        pl.layout = fast::kRKV;
+        srcs[0] = r;
+        srcs[1] = k;
+        srcs[2] = v;
+        nsrc = 3;
+    }
+    for (int i = 0; i < nsrc; ++i)
+        if (!aligned(srcs[i], 16)) return false;
+    fast::Params& p = pl.p;
+    pl.qs = qs != nullptr;
+    p.B = B;
+    p.T = T;
+    p.C = C;
+    if (pl.qs) {
+        p.H = qs->H;
+        p.W = qs->W;
+        p.s = qs->shift_pixel;
+        p.g = group_size(C, qs->gamma);
+        if (p.g % fast::kCS != 0 || p.W > 256 || p.W % fast::kL != 0) return false;
+        if (T <= fast::kTcMax) {
+            p.rows = p.H;
+            p.Tc = T;
+            p.ncl = 1;
+        } else {
+            int rows = 0;
+            for (int rr = fast::kTcMax / p.W; rr >= 1; --rr)
+                if ((rr * p.W) % 32 == 0) {
+                    rows = rr;
+                    break;
+                }
+            if (rows == 0 || rows > 256) return false;
+            p.rows = rows;
+            p.Tc = rows * p.W;
+            p.ncl = (p.H + rows - 1) / rows;
+        }
+    } else {
+        p.H = 1;
+        p.W = T;
+        p.s = 0;
+        p.g = 0;
+        p.rows = 1;
+        p.Tc = std::min(T, fast::kTcMax);
+        p.ncl = (T + p.Tc - 1) / p.Tc;
+    }
+    if (p.ncl > fast::kClusterMax) return false;
+    const int RB = fast::kCS * es;
+    // 8 sub-tiles of 32 token rows; every thread reads its row of each, so a
+    // tile always spans 256 tokens even when the boxes deliver fewer
+    p.tile_bytes = fast::kTcMax * RB;
+    // a strided box delivers (W / 8) x rows token rows with Q-Shift, and its
+    // full 256 / 8 = 32 rows without (tokens past T arrive as zeros)
+    p.box_bytes = (pl.qs ? (p.W / fast::kL) * p.rows : fast::kTcMax / fast::kL) * RB;
+    const int ntiles = nsrc * (pl.qs ? 2 : 1);
+    pl.smem = ntiles * p.tile_bytes + (int)sizeof(fast::Scratch) + 128;  // + alignment slack
+    if (pl.smem > 227 * 1024) return false;
+    const CUtensorMapDataType dt =
+        dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    for (int i = 0; i < nsrc; ++i) {
+        CUresult cr;
+        // element stride 8 along the token (w) axis: box i holds tokens 8q + i
+        const cuuint32_t estr[4] = {1, (cuuint32_t)fast::kL, 1, 1};
+        if (pl.qs) {
+            const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)B};
+            const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)p.W * C * es,
+                                           (cuuint64_t)p.H * p.W * C * es};
+            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, (cuuint32_t)p.W, (cuuint32_t)p.rows, 1};
+            cr = enc(&p.map[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        } else {
+            const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+            const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
+            const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, (cuuint32_t)fast::kTcMax, 1};
+            cr = enc(&p.map[i], dt, 3, const_cast<void*>(srcs[i]), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        }
+        if (cr != CUDA_SUCCESS) return false;
+    }
+    p.err = device_error_word();
+    if (!p.err) return false;
+    p.w = w;
+    p.u = u;
+    p.mu[0] = qs ? qs->mu_r : nullptr;
+    p.mu[1] = qs ? qs->mu_k : nullptr;
+    p.mu[2] = qs ? qs->mu_v : nullptr;
+    p.out = static_cast<char*>(out);
+    pl.grid = dim3(p.ncl, C / fast::kCS, B);
+    return true;
+}
+
 vrwkv_status check_qs(const vrwkv_qshift_params* qs, int T, int C) {
     if (qs->H <= 0 || qs->W <= 0) return fail(VRWKV_ERR_INVALID_ARG, "qs: H and W must be positive");
     if ((long long)qs->H * qs->W != T)
@@ -154,6 +386,17 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
         for (const float* m : mus)
             if (overlaps(out, nbytes, m, (size_t)C * 4))
                 return fail(VRWKV_ERR_INVALID_ARG, "output overlaps a mu vector");
+    }
+
+    if (B <= 65535 && C / vrwkv::fast::kCS <= 65535) {
+        FastPlan fp;
+        if (plan_fast(fp, gate, r, k, v, w, u, out, B, T, C, dtype, qs)) {
+            bool fell_back = false;
+            cudaStream_t fs = static_cast<cudaStream_t>(stream);
+            vrwkv_status st = dtype == VRWKV_F32 ? dispatch_fast<float>(fp, fs, &fell_back)
+                                                 : dispatch_fast<__nv_bfloat16>(fp, fs, &fell_back);
+            if (!fell_back) return st;
+        }
     }
 
     FusedPlan pl{};
@@ -294,10 +537,24 @@ const char* vrwkv_status_string(vrwkv_status status) {
     case VRWKV_ERR_INVALID_ARG: return "VRWKV_ERR_INVALID_ARG";
     case VRWKV_ERR_UNSUPPORTED: return "VRWKV_ERR_UNSUPPORTED";
     case VRWKV_ERR_CUDA: return "VRWKV_ERR_CUDA";
+    case VRWKV_ERR_TIMEOUT: return "VRWKV_ERR_TIMEOUT";
     default: return "VRWKV_ERR_UNKNOWN";
     }
 }
 
 const char* vrwkv_last_error(void) { return g_last_error.c_str(); }
+
+vrwkv_status vrwkv_device_status(void) {
+    unsigned int* word = device_error_word();
+    if (!word) return fail(VRWKV_ERR_CUDA, "cannot locate the device error word");
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
+    if (v == 0) return ok();
+    const unsigned int zero = 0;
+    e = cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_status(e, "clearing the device error word");
+    return fail(VRWKV_ERR_TIMEOUT, "a kernel's bounded wait for its TMA tiles ran out (flags 0x%x)", v);
+}
 
 }  // extern "C"

@@ -129,6 +129,7 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
         ks = oracle.qshift(kin, H, W, s, g, ref["mu_k"])
         vs = oracle.qshift(vin, H, W, s, g, ref["mu_v"])
         rs = None if rin is None else oracle.qshift(rin, H, W, s, g, ref["mu_r"])
+    vk.device_status()  # no kernel's bounded wait ran out
     got = to_numpy(out)
     assert np.isfinite(got).all()
 
@@ -153,8 +154,19 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     return (got, err) if return_out else err
 
 
+@pytest.fixture(params=["tma", "generic"])
+def kernel_path(request, monkeypatch):
+    """Run a test on the TMA fast path (when the shape qualifies) and again
+    with the generic kernel forced."""
+    if request.param == "generic":
+        monkeypatch.setenv("VRWKV_DISABLE_TMA", "1")
+    else:
+        monkeypatch.delenv("VRWKV_DISABLE_TMA", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
-def test_workload_full_size(vk, oracle_mod, cfg):
+def test_workload_full_size(vk, oracle_mod, cfg, kernel_path):
     wl = synth.WORKLOADS[cfg]
     run_fused(vk, oracle_mod, wl)
 
@@ -190,21 +202,29 @@ EDGE = [
     ("gate_qs_x", 2, 14, 14, 96, "bf16"),
     ("gate_qs_x", 1, 40, 40, 64, "f32"),    # T = 1600 in float32
     ("gate_qs_x", 1, 3, 11, 6, "bf16"),
+    ("gate_qs_x", 2, 16, 16, 64, "bf16"),   # T = 256: one full CTA
+    ("gate_qs_x", 1, 40, 40, 64, "bf16"),   # W = 40: 10-CTA cluster
+    ("gate_qs", 2, 64, 64, 64, "bf16"),     # 16-CTA cluster, separate r, k, v
+    ("qshift_biwkv", 1, 48, 64, 64, "bf16"),
+    ("qshift_biwkv", 2, 24, 24, 64, "f32"),  # W = 24: 8 rows of 24 per CTA
+    ("biwkv", 2, 1, 4096, 16, "bf16"),      # 16 CTAs without Q-Shift
+    ("biwkv", 3, 1, 257, 32, "f32"),        # one token into a second CTA
 ]
 
 
 @pytest.mark.parametrize("case", EDGE, ids=lambda c: "_".join(map(str, c)))
-def test_edge_shapes(vk, oracle_mod, case):
+def test_edge_shapes(vk, oracle_mod, case, kernel_path):
     call, B, H, W, C, dt = case
     wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000)
     run_fused(vk, oracle_mod, wl)
 
 
-@pytest.mark.parametrize("s,H,W", [(2, 6, 7), (3, 2, 300), (5, 4, 4)])
-def test_large_shifts(vk, oracle_mod, s, H, W):
-    wl = _custom("gate_qs", 1, H, W, 24, "bf16", seed=77 + s, s=s)
+@pytest.mark.parametrize("s,H,W", [(2, 6, 7), (3, 2, 300), (5, 4, 4), (2, 32, 64), (70, 8, 64)])
+def test_large_shifts(vk, oracle_mod, s, H, W, kernel_path):
+    C = 64 if W % 8 == 0 and W <= 256 else 24  # C = 64: the TMA path qualifies
+    wl = _custom("gate_qs", 1, H, W, C, "bf16", seed=77 + s, s=s)
     run_fused(vk, oracle_mod, wl)
-    wl = _custom("gate_qs_x", 1, H, W, 24, "f32", seed=78 + s, s=s)
+    wl = _custom("gate_qs_x", 1, H, W, C, "f32", seed=78 + s, s=s)
     run_fused(vk, oracle_mod, wl)
 
 
@@ -216,7 +236,7 @@ def test_mu_none_is_pure_shift(vk, oracle_mod):
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_shift_invariance_in_k(vk, oracle_mod, dt):
+def test_shift_invariance_in_k(vk, oracle_mod, dt, kernel_path):
     # adding 80 to every k would overflow exp(k) in float32 without the
     # running-maximum renormalisation; the result must not change
     wl = _custom("biwkv", 2, 40, 40, 32, dt, seed=93)
@@ -229,7 +249,7 @@ def test_shift_invariance_in_k(vk, oracle_mod, dt):
 
 
 @pytest.mark.parametrize("w_kind", ["zero", "huge_positive", "strong_negative"])
-def test_decay_extremes(vk, oracle_mod, w_kind):
+def test_decay_extremes(vk, oracle_mod, w_kind, kernel_path):
     T = 24 * 30
     d = {"zero": ("uniform", 0.0, 0.0), "huge_positive": ("uniform", 60.0 * T, 60.0 * T),
          "strong_negative": ("uniform", -20.0, -10.0)}[w_kind]
