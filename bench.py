@@ -47,17 +47,18 @@ METRIC = ("Bi-WKV fused fwd tokens·ch/s and HBM GB/s (% of B200 peak) "
 UNIT = "tokens*ch/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["linear_complexity_vision_b200/csrc/common.cuh",
-                  "linear_complexity_vision_b200/csrc/biwkv.cuh",
-                  "linear_complexity_vision_b200/csrc/qshift.cuh",
-                  "linear_complexity_vision_b200/csrc/vrwkv_api.cu"]
+CSRC = os.path.join(ROOT, "linear_complexity_vision_b200", "csrc")
 
 
 def kernel_source_hash() -> str:
+    """Hash of every CUDA source of the library (the traffic record is only
+    valid for the exact kernels it was measured on)."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+    for f in sorted(os.listdir(CSRC)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(CSRC, f), "rb") as fh:
+                h.update(f.encode())
+                h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -233,6 +234,11 @@ class Runner:
             self.qs = vk.QShift(wl.H, wl.W, wl.shift_pixel, wl.gamma, self.par.get("mu_r"),
                                 self.par.get("mu_k"), self.par.get("mu_v"))
         self.launches_per_step = 2 if wl.call == "qshift_biwkv" else 1
+
+    @property
+    def kernel_name(self) -> str:
+        """Name of the fused kernel the library launched last on this thread."""
+        return self.vk.load_library().vrwkv_last_kernel().decode()
 
     def step(self, i: int):
         d = self.sets[i % self.nsets]
@@ -417,7 +423,7 @@ def run_ours(args, dist):
                    "parallelism": f"replicas x{dist.world} (independent batches, no collective)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "biwkv_fused_kernel",
+                     "kernel": runner.kernel_name,
                      "algorithmic_bytes_per_launch": fused_bytes,
                      "avg_launch_us": launch_s * 1e6},
         "e2e": e2e,

@@ -151,6 +151,11 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
  */
 vrwkv_status vrwkv_device_status(void);
 
+/* Name of the kernel the calling thread's most recent successful
+ * vrwkv_biwkv_fwd / vrwkv_spatial_gate call launched ("" before any), e.g.
+ * "biwkv_tma_kernel" or "biwkv_fused_kernel".  Diagnostics only. */
+const char* vrwkv_last_kernel(void);
+
 /* Static, never-NULL name of a status code. */
 const char* vrwkv_status_string(vrwkv_status status);
 

@@ -69,6 +69,8 @@ def load_library():
         lib.vrwkv_device_status.restype = ci
         lib.vrwkv_status_string.argtypes = [ci]
         lib.vrwkv_status_string.restype = ctypes.c_char_p
+        lib.vrwkv_last_kernel.argtypes = []
+        lib.vrwkv_last_kernel.restype = ctypes.c_char_p
         lib.vrwkv_last_error.argtypes = []
         lib.vrwkv_last_error.restype = ctypes.c_char_p
         _lib = lib

@@ -49,6 +49,7 @@ constexpr int kThreads = 256;   // threads per CTA
 constexpr int kNW = kThreads / 32;
 constexpr int kTcMax = kThreads / kNP * kL;  // 256 tokens per CTA
 constexpr int kClusterMax = 16;
+constexpr int kMinBlocks = 4;   // resident CTAs per SM the register budget targets
 constexpr int kTab = kTcMax / kL;            // a^(8m), m < 32
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 
@@ -63,6 +64,8 @@ struct alignas(64) Params {
     unsigned int* err;   // device error word (bounded waits)
     int B, T, C;
     int H, W, s, g;      // Q-Shift grid, shift, group size
+    int gslab;           // group size in 16-channel slabs (g / 16; 0 if g == 0)
+    float invT;          // 1 / T
     int Tc;              // tokens per CTA (multiple of 32 when ncl > 1)
     int rows;            // image rows per CTA (Q-Shift path): Tc = rows * W
     int ncl;             // CTAs per column (cluster size)
@@ -77,9 +80,10 @@ struct alignas(16) Scratch {
     float4 waggB[kNP][kNW];     // per-warp backward aggregates
     float4 wcarF[kNP][kNW];     // exclusive forward carry into each warp
     float4 wcarB[kNP][kNW];     // exclusive backward carry into each warp
-    float cM[kCS];              // CTA maximum of k times log2(e), read by peers
-    float4 caggF[kNP];          // CTA forward aggregate, read by peers
-    float4 caggB[kNP];          // CTA backward aggregate, read by peers
+    float2 mbM[kClusterMax][kNP];   // mailbox: each CTA's max of k (times log2 e)
+    float4 mbF[kClusterMax][kNP];   // mailbox: each CTA's forward aggregate
+    float4 mbG[kClusterMax][kNP];   // mailbox: each CTA's backward aggregate
+    float2 gpark[kTcMax / kL * kL][kNP];  // gate factors, parked between load and output
     float4 cscale[kCS];         // per channel: sl (scale of this CTA's own sums)
     float4 ccarry[kCS];         // per channel: carries Af, Cf, Bb, Db
     unsigned long long bar;     // TMA completion barrier
@@ -178,7 +182,7 @@ __device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); 
 __device__ __forceinline__ float4 zero4() { return make_float4(0.f, 0.f, 0.f, 0.f); }
 
 template <typename IO, int LAYOUT, bool QS>
-__global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const __grid_constant__ Params p) {
     constexpr bool GATE = LAYOUT != kKV;
     constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
     constexpr int NTILE = NSRC * (QS ? 2 : 1);
@@ -208,7 +212,10 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
 
     // group of this CTA's channels (Q-Shift): 0..3 shifted, 4 copied
     int grp = 4;
-    if (QS && p.g > 0) grp = min(c0 / p.g, 4);
+    if (QS && p.gslab > 0) {
+        const int y = blockIdx.y;
+        grp = (y >= p.gslab) + (y >= 2 * p.gslab) + (y >= 3 * p.gslab) + (y >= 4 * p.gslab);
+    }
     const bool shifted = QS && grp < 4;
 
     // ---- issue the tile loads: lane i of warp 0 loads sub-tile i of each tile
@@ -241,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
 
     // ---- per-thread constants (overlap the copies) ---------------------------
     const int cA = c0 + 2 * j;
-    const float invT = 1.0f / (float)p.T;
+    const float invT = p.invT;
     const float2 wv = make_float2(__ldg(p.w + cA), __ldg(p.w + cA + 1));
     const float2 uv = make_float2(__ldg(p.u + cA), __ldg(p.u + cA + 1));
     const float2 lam2 = mul2(wv, f2(invT * kLog2e));  // w / T in base-2 units
@@ -274,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
     const char* tV = smem + (QS ? 2 * SV : SV) * p.tile_bytes;
     const char* tR = smem + (QS ? 2 * SR : SR) * p.tile_bytes;
     const int dsh = shifted ? p.tile_bytes : 0;  // shifted tile = plain + dsh
-    float2 kk[kL], vv[kL], gg[kL];
+    float2 kk[kL], vv[kL];
     float2 mx = f2(-INFINITY);
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
@@ -302,12 +309,23 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
             v = lds_pair<IO>(tV, o);
             if (GATE) r = lds_pair<IO>(tR, o);
         }
-        if (GATE) gg[i] = ex2(mul2(r, f2(-kLog2e)));
+        // gate factor e^{-r}, parked in shared memory until the output phase
+        if (GATE) S.gpark[i * (kTcMax / kL) + q][j] = ex2(mul2(r, f2(-kLog2e)));
+        kk[i] = k;
+        vv[i] = v;
+    }
+    if (nv == kL) {
+#pragma unroll
+        for (int i = 0; i < kL; ++i) mx = max2(mx, kk[i]);
+    } else {
         // tokens past the sequence end hold zeros (TMA fill) or stale shared
         // memory (rows beyond a short box): mask both so p = 0 and p*v = 0
-        kk[i] = (i < nv) ? k : f2(-INFINITY);
-        vv[i] = (i < nv) ? v : f2(0.0f);
-        mx = max2(mx, kk[i]);
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            kk[i] = (i < nv) ? kk[i] : f2(-INFINITY);
+            vv[i] = (i < nv) ? vv[i] : f2(0.0f);
+            mx = max2(mx, kk[i]);
+        }
     }
 #pragma unroll
     for (int d = 8; d <= 16; d <<= 1) {
@@ -381,17 +399,24 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
         if (wi == kNW - 1) yw = zero4();
         S.wcarF[jj][wi] = xw;
         S.wcarB[jj][wi] = yw;
-        // the CTA's forward aggregate sits at its last real warp (Tc may be
-        // shorter than 256 tokens; padding warps after it hold zeros)
-        if (wi == p.Tc / 32 - 1) S.caggF[jj] = f;
-        if (wi == 0) {
-            S.caggB[jj] = gb;
+        // publish this CTA's record for pair jj into every CTA's mailbox
+        // (its own included) with remote shared-memory stores; the cluster
+        // barrier below makes them visible.  The CTA's forward aggregate sits
+        // at its last real warp (Tc may be shorter than 256 tokens).
+        if (p.ncl > 1 && (wi == p.Tc / 32 - 1 || wi == 0)) {
+            cg::cluster_group cluster = cg::this_cluster();
             float2 Mj = S.wmax[jj][0];
 #pragma unroll
             for (int w = 1; w < kNW; ++w) Mj = max2(Mj, S.wmax[jj][w]);
-            // published in base 2, the unit of the cluster fold's exponents
-            S.cM[2 * jj] = Mj.x * kLog2e;
-            S.cM[2 * jj + 1] = Mj.y * kLog2e;
+            Mj = mul2(Mj, f2(kLog2e));  // base 2, the unit of the exponents below
+            for (int rr = 0; rr < p.ncl; ++rr) {
+                Scratch* P = cluster.map_shared_rank(&S, rr);
+                if (wi == p.Tc / 32 - 1) P->mbF[rank][jj] = f;
+                if (wi == 0) {
+                    P->mbG[rank][jj] = gb;
+                    P->mbM[rank][jj] = Mj;
+                }
+            }
         }
     }
     if (p.ncl > 1) {
@@ -400,30 +425,25 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
     } else {
         __syncthreads();
     }
-    // Exchange with the other CTAs of the column.  Thread (channel lc, peer
-    // rr) reads peer rr's CTA record for channel lc straight from distributed
-    // shared memory; each 16-lane segment then holds one channel's column.
-    // The segment maximum of the peers' exponents is the common reference;
-    // forward and backward carries are 16-lane shuffle scans with the
-    // one-CTA decay a^Tc, a^(2 Tc), ...
+    // Exchange with the other CTAs of the column: thread (channel lc, peer
+    // rr) reads peer rr's record for channel lc from this CTA's mailbox;
+    // each 16-lane segment holds one channel's column.  The segment maximum
+    // of the peers' exponents is the common reference; forward and backward
+    // carries are 16-lane shuffle scans with the one-CTA decay a^Tc.
     float2 cs_sl = f2(1.0f), cs_af = f2(0.0f), cs_cf = f2(0.0f), cs_bb = f2(0.0f), cs_db = f2(0.0f);
     if (p.ncl > 1) {
         const int lc = tid >> 4, rr = tid & 15;
         float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
         if (rr < p.ncl) {
-            cg::cluster_group cluster = cg::this_cluster();
-            const Scratch* P = cluster.map_shared_rank(&S, rr);
-            const float4 F = P->caggF[lc >> 1], G = P->caggB[lc >> 1];
+            const float4 F = S.mbF[rr][lc >> 1], G = S.mbG[rr][lc >> 1];
+            const float2 Mp = S.mbM[rr][lc >> 1];
             const bool hi = lc & 1;
-            Mr = P->cM[lc];
+            Mr = hi ? Mp.y : Mp.x;
             fa2 = hi ? F.y : F.x;
             fc2 = hi ? F.w : F.z;
             ga2 = hi ? G.y : G.x;
             gc2 = hi ? G.w : G.z;
         }
-        // release: this thread's reads of the peers' shared memory are
-        // complete before any peer can pass its final wait and exit
-        cluster_arrive_release();
         float Mc = Mr;
 #pragma unroll
         for (int d = 8; d >= 1; d >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, 16));
@@ -493,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
     for (int i = 0; i < kL; ++i) {
         const float2 num = fma2(sl, n[i], fma2(pw[i], As, mul2(pw[kL - 1 - i], Be)));
         float2 den = fma2(sl, dd[i], fma2(pw[i], Cs, mul2(pw[kL - 1 - i], De)));
-        if (GATE) den = fma2(den, gg[i], den);
+        if (GATE) den = fma2(den, S.gpark[i * (kTcMax / kL) + q][j], den);
         Io<IO>::st_pair(tout + rowoff + i * SUB, mul2(num, rcp(den)));
     }
     __syncthreads();
@@ -509,7 +529,8 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_tma_kernel(const __grid_con
                     *reinterpret_cast<const uint4*>(tout + i * SUB + o);
         }
     }
-    if (p.ncl > 1) cluster_wait_acquire();  // peers finished reading this CTA
+    // no closing cluster barrier: peers wrote into this CTA's mailbox before
+    // the exchange barrier and nobody reads another CTA's memory after it
 }
 
 }  // namespace fast

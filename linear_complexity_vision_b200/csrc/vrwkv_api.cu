@@ -26,6 +26,7 @@ namespace {
 using namespace vrwkv;
 
 thread_local std::string g_last_error;
+thread_local const char* g_last_kernel = "";
 
 vrwkv_status fail(vrwkv_status s, const char* fmt, ...) {
     char buf[512];
@@ -102,6 +103,7 @@ vrwkv_status launch_fused(const FusedPlan& pl, cudaStream_t stream) {
     cfg.numAttrs = pl.p.ncl > 1 ? 1 : 0;
     e = cudaLaunchKernelEx(&cfg, kern, pl.p);
     if (e != cudaSuccess) return cuda_status(e, "biwkv_fused_kernel launch");
+    g_last_kernel = "biwkv_fused_kernel";
     return ok();
 }
 
@@ -213,6 +215,7 @@ vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_bac
     }
     e = cudaLaunchKernelEx(&cfg, kern, pl.p);
     if (e != cudaSuccess) return cuda_status(e, "biwkv_tma_kernel launch");
+    g_last_kernel = "biwkv_tma_kernel";
     return ok();
 }
 
@@ -329,6 +332,8 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         }
         if (cr != CUDA_SUCCESS) return false;
     }
+    p.gslab = pl.qs ? p.g / fast::kCS : 0;
+    p.invT = (float)(1.0 / (double)T);
     p.err = device_error_word();
     if (!p.err) return false;
     p.w = w;
@@ -543,6 +548,8 @@ const char* vrwkv_status_string(vrwkv_status status) {
 }
 
 const char* vrwkv_last_error(void) { return g_last_error.c_str(); }
+
+const char* vrwkv_last_kernel(void) { return g_last_kernel; }
 
 vrwkv_status vrwkv_device_status(void) {
     unsigned int* word = device_error_word();
