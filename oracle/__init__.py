@@ -20,6 +20,8 @@ It wraps ``vrwkv_oracle.c`` (plain C, float64, OpenMP over channel columns):
                        page describes (short sequences only).
 * ``gate``          -- sigma(R) (.) wkv of eq. 2.
 * ``spatial_core``  -- gate(QS_R(r), Bi-WKV(QS_K(k), QS_V(v))).
+* ``channel_mix``   -- sigma(QS_R(x)) * max(QS_K(x), 0)^2, the channel-mix
+                       module of eq. 3-4 without projections.
 * ``spatial_core_points`` -- the same at selected output positions only, by
                        direct summation of eq. 5 over each needed column.
 
@@ -70,6 +72,7 @@ def _load():
         lib.oracle_biwkv_direct_points.argtypes = [dp, dp, dp, dp, ci, ci, ci,
                                                    i64p, cl, dp]
         lib.oracle_gate.argtypes = [dp, dp, dp, cl]
+        lib.oracle_channel_mix.argtypes = [dp, dp, dp, dp, ci, ci, ci, ci, ci, cd]
         lib.oracle_spatial_core_points.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, ci,
                                                    ci, ci, cd, ci, ci, i64p, cl, dp]
         lib.oracle_num_threads.restype = ci
@@ -210,4 +213,17 @@ def spatial_core_points(r, k, v, w, u, H, W, flat_idx, shift_pixel=1, gamma=0.25
         _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), mps[0], mps[1], mps[2], B, H, W, C,
         int(shift_pixel), float(gamma), int(qshift_on), int(gate_on),
         idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), idx.shape[0], _ptr(out))
+    return out
+
+
+def channel_mix(x, H, W, shift_pixel=1, gamma=0.25, mu_r=None, mu_k=None) -> np.ndarray:
+    """sigma(QS_R(x)) * SquaredReLU(QS_K(x)) (eq. 3-4, identity projections)."""
+    x = _d(x)
+    B, T, C = x.shape
+    assert T == H * W
+    out = np.empty_like(x)
+    mus = [None if m is None else _d(m) for m in (mu_r, mu_k)]
+    _load().oracle_channel_mix(_ptr(x), None if mus[0] is None else _ptr(mus[0]),
+                               None if mus[1] is None else _ptr(mus[1]), _ptr(out), B, H, W, C,
+                               int(shift_pixel), float(gamma))
     return out

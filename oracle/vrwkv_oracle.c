@@ -388,3 +388,24 @@ void oracle_spatial_core_points(const double* r, const double* k,
         free(vc);
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* Channel mix without projections (eq. 3-4 with identity W_R, W_K,   */
+/* W_V and no W_O):  out = sigma(QS_R(x)) (.) SquaredReLU(QS_K(x)),   */
+/* SquaredReLU(z) = max(z, 0)^2.                                      */
+/* ------------------------------------------------------------------ */
+void oracle_channel_mix(const double* x, const double* mu_r,
+                        const double* mu_k, double* out, int B, int H, int W,
+                        int C, int s, double gamma) {
+    const long T = (long)H * W;
+#pragma omp parallel for schedule(static)
+    for (long bt = 0; bt < (long)B * T; ++bt) {
+        long b = bt / T, t = bt % T;
+        for (int c = 0; c < C; ++c) {
+            double rs = qs_value(x, mu_r, b, t, c, H, W, C, s, gamma, 1);
+            double ks = qs_value(x, mu_k, b, t, c, H, W, C, s, gamma, 1);
+            double kp = ks > 0.0 ? ks : 0.0;
+            out[bt * C + c] = (1.0 / (1.0 + exp(-rs))) * (kp * kp);
+        }
+    }
+}
