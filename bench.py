@@ -22,6 +22,9 @@ bytes / average launch time against the measured HBM copy bandwidth), an
 end-to-end figure through the C ABI with host buffers, the float64 CPU
 oracle timed on a bounded sample, and SM clocks sampled during the timed
 region.  ``--impl reference`` times the CPU oracle alone on the same metric.
+``rows.channel_mix`` adds the roofline of the channel-mix elementwise path
+(eq. 3-4 with identity projections) on the same x buffers, timed in its own
+region after the main one (``--no-rows`` skips it).
 """
 from __future__ import annotations
 
@@ -271,6 +274,48 @@ class Runner:
             self.sets = saved
 
 
+def time_channel_mix(runner, stream, torch, dev, launches: int, peak: float):
+    """Roofline of the channel-mix elementwise path (eq. 3-4 with identity
+    projections) on the workload's x buffers, outside the main timed region:
+    CUDA graphs over the same rotating buffer sets, events on the stream."""
+    wl, vk = runner.wl, runner.vk
+    if "x" not in runner.sets[0]:
+        return None
+    n = runner.nsets
+    outs = [torch.empty_like(d["x"]) for d in runner.sets]
+
+    def launch(i):
+        vk.channel_mix(runner.sets[i % n]["x"], runner.qs, out=outs[i % n])
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            launch(i)
+    torch.cuda.synchronize(dev)
+    G = n * max(1, 64 // n)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            launch(i)
+    reps = max(1, launches // G)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    del graph
+    us = e0.elapsed_time(e1) * 1e3 / (reps * G)
+    es = 4 if wl.dtype == "f32" else 2
+    nbytes = 2 * wl.N * es + 2 * wl.C * 4  # x once, out once, mu_r and mu_k
+    achieved = nbytes / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "kernel": runner.kernel_name,
+            "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
+            "launches": reps * G}
+
+
 def parity_sample(runner, out_dev, oracle, npts=128):
     """Max |GPU - float64 oracle| on a seeded sample of output positions."""
     wl, inp = runner.wl, runner.inp
@@ -430,6 +475,11 @@ def run_ours(args, dist):
         "gpu_launches": steps * runner.launches_per_step,
         "clocks": clocks.summary(),
     }
+    # the next hot-path row on the same buffers (its own timed region)
+    if args.rows:
+        cm = time_channel_mix(runner, stream, torch, dev, args.row_launches, peak)
+        if cm is not None:
+            line["rows"] = {"channel_mix": cm}
     # correctness guard on the last timed output (first set of the rotation)
     if dist.rank == 0:
         import oracle
@@ -506,6 +556,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", dest="rows", action="store_false",
+                    help="skip the channel-mix row measurement")
+    ap.add_argument("--row-launches", type=int, default=4000)
     args = ap.parse_args(argv)
     dist = Dist()
     if args.impl == "reference":

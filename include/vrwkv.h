@@ -7,7 +7,9 @@
  *   - Q-Shift, Quad-Directional Token Shift, eq. 9;
  *   - Bi-WKV, Linear Complexity Bidirectional Attention, eq. 5
  *     (equivalently the RNN form, eq. 6-7);
- *   - the receptance gate sigma(R) (.) wkv, Overall Architecture, eq. 2.
+ *   - the receptance gate sigma(R) (.) wkv, Overall Architecture, eq. 2;
+ *   - the channel-mix gate sigma(R_c) (.) SquaredReLU(K_c), Overall
+ *     Architecture, eq. 3-4.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -141,6 +143,28 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
                                 const vrwkv_qshift_params* qs, void* stream);
 
 /*
+ * vrwkv_channel_mix -- the elementwise part of the channel-mix module (eq. 3-4
+ * with identity W_R, W_K, W_V and no W_O):
+ *   out = sigma(QS_R(x)) (.) SquaredReLU(QS_K(x)),  SquaredReLU(z) = max(z, 0)^2
+ * where QS_R, QS_K are Q-Shift with qs->mu_r and qs->mu_k (qs->mu_v is
+ * ignored), or the identity when qs is NULL.
+ *   x    (B, T, C) input, dtype `dtype`.
+ *   out  (B, T, C) output, same dtype, must not overlap x, mu_r or mu_k.
+ *   qs   NULL, or Q-Shift parameters; T must then equal qs->H * qs->W.
+ * Arithmetic: float32, with the mix evaluated as x_shift + mu*(x - x_shift)
+ *   (fused multiply-add) and sigma(r) = 1/(1 + 2^(-r*log2 e)) from the hardware
+ *   exp2 and reciprocal; one rounding to bfloat16 at the store for VRWKV_BF16.
+ * Kernels: a vector kernel serves C*sizeof(dtype) % 16 == 0 with 16-byte-
+ *   aligned x and out, 8-byte-aligned mu and a group size int(C*gamma) that is
+ *   a multiple of 16/sizeof(dtype); everything else runs a scalar kernel.
+ * Errors: INVALID_ARG for B, T or C <= 0, NULL x/out, misaligned pointers, an
+ *   overlapping output or bad qs fields; UNSUPPORTED for B*T >= 2^31.
+ */
+vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C,
+                               vrwkv_dtype dtype, const vrwkv_qshift_params* qs,
+                               void* stream);
+
+/*
  * vrwkv_device_status -- report and clear kernel-side failures on the
  * current device.  Kernels that wait for their asynchronous (TMA) tile
  * copies give up after about two seconds, record the failure in a device
@@ -152,8 +176,9 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
 vrwkv_status vrwkv_device_status(void);
 
 /* Name of the kernel the calling thread's most recent successful
- * vrwkv_biwkv_fwd / vrwkv_spatial_gate call launched ("" before any), e.g.
- * "biwkv_tma_kernel" or "biwkv_fused_kernel".  Diagnostics only. */
+ * vrwkv_biwkv_fwd / vrwkv_spatial_gate / vrwkv_channel_mix call launched
+ * ("" before any), e.g. "biwkv_tma_kernel", "biwkv_fused_kernel" or
+ * "channel_mix_vec_kernel".  Diagnostics only. */
 const char* vrwkv_last_kernel(void);
 
 /* Static, never-NULL name of a status code. */

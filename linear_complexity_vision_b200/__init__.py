@@ -8,6 +8,7 @@ There is no fallback: if the library is missing, the calls raise.
     qshift(x, H, W, shift_pixel=1, gamma=0.25, mu=None)
     biwkv_fwd(k, v, w, u, qs=None)
     spatial_gate(r, k, v, w, u, qs=None)
+    channel_mix(x, qs=None)
     device_status()     # synchronise; raise if a kernel's bounded wait ran out
 
 Token tensors are contiguous (B, T, C) CUDA tensors of dtype float32 or
@@ -65,6 +66,8 @@ def load_library():
         lib.vrwkv_spatial_gate.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                            ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_spatial_gate.restype = ci
+        lib.vrwkv_channel_mix.argtypes = [vp, vp, ci, ci, ci, ci, ctypes.POINTER(_QsParams), vp]
+        lib.vrwkv_channel_mix.restype = ci
         lib.vrwkv_device_status.argtypes = []
         lib.vrwkv_device_status.restype = ci
         lib.vrwkv_status_string.argtypes = [ci]
@@ -164,6 +167,20 @@ def spatial_gate(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
     _check(load_library().vrwkv_spatial_gate(
         r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
         B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
+    return out
+
+
+def channel_mix(x, qs: Optional[QShift] = None, out=None):
+    """sigma(QS_R(x)) * max(QS_K(x), 0)^2 on a (B, T, C) tensor (eq. 3-4 with
+    identity projections); QS is the identity if qs is None."""
+    import torch
+    _require(x, "x")
+    B, T, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _check(load_library().vrwkv_channel_mix(
+        x.data_ptr(), out.data_ptr(), B, T, C, _dtype_code(x), qsp, _stream_ptr(x)))
     return out
 
 

@@ -17,6 +17,7 @@
 #include "biwkv.cuh"
 #include "biwkv_tma.cuh"
 #include "qshift.cuh"
+#include "channel_mix.cuh"
 
 // Device error word: set by kernels whose bounded waits ran out (bit 0).
 __device__ unsigned int g_vrwkv_device_error;
@@ -522,6 +523,89 @@ vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B, int 
         else qshift_scalar_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(p);
     }
     return cuda_status(cudaGetLastError(), "qshift kernel launch");
+}
+
+vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vrwkv_dtype dtype,
+                               const vrwkv_qshift_params* qs, void* stream) {
+    if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
+        return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B <= 0 || T <= 0 || C <= 0)
+        return fail(VRWKV_ERR_INVALID_ARG, "B, T and C must be positive (got %d, %d, %d)", B, T, C);
+    if (!x || !out) return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
+    if ((long long)B * T > 0x7fffffffLL) return fail(VRWKV_ERR_UNSUPPORTED, "B*T must be below 2^31");
+    const int es = elem_bytes(dtype);
+    if (!aligned(x, es) || !aligned(out, es)) return fail(VRWKV_ERR_INVALID_ARG, "pointer misaligned");
+    const size_t nbytes = (size_t)B * T * C * es;
+    if (overlaps(out, nbytes, x, nbytes)) return fail(VRWKV_ERR_INVALID_ARG, "output overlaps the input");
+    ChannelMixParams p;
+    p.x = static_cast<const char*>(x);
+    p.out = static_cast<char*>(out);
+    p.mu_r = p.mu_k = nullptr;
+    p.BT = B * T;
+    p.T = T;
+    p.C = C;
+    p.H = 1;
+    p.W = T;
+    p.s = 0;
+    p.g = 0;  // without qs every channel reads its own token: QS is the identity
+    if (qs) {
+        vrwkv_status st = check_qs(qs, T, C);
+        if (st != VRWKV_OK) return st;
+        p.mu_r = qs->mu_r;
+        p.mu_k = qs->mu_k;
+        p.H = qs->H;
+        p.W = qs->W;
+        p.s = qs->shift_pixel;
+        p.g = group_size(C, qs->gamma);
+        for (const float* m : {p.mu_r, p.mu_k})
+            if (m && overlaps(out, nbytes, m, (size_t)C * 4))
+                return fail(VRWKV_ERR_INVALID_ARG, "output overlaps mu");
+    }
+    p.divT = make_fastdiv((unsigned)p.T);
+    p.divW = make_fastdiv((unsigned)p.W);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int nv = 16 / es;  // channels per 16-byte vector
+    const bool vec = (C % nv) == 0 && p.g % nv == 0 && aligned(x, 16) && aligned(out, 16) &&
+                     (!p.mu_r || aligned(p.mu_r, 8)) && (!p.mu_k || aligned(p.mu_k, 8));
+    if (!vec) {
+        const long long n = (long long)p.BT * C;
+        const long long blocks = std::min<long long>((n + 255) / 256, 148LL * 16);
+        if (dtype == VRWKV_F32) channel_mix_scalar_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(p);
+        else channel_mix_scalar_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(p);
+        g_last_kernel = "channel_mix_scalar_kernel";
+        return cuda_status(cudaGetLastError(), "channel_mix kernel launch");
+    }
+    p.UR = C / nv;
+    // Channel chunks of at most 256 vectors, rounded to whole warps when split.
+    const int nchunks = (p.UR + 255) / 256;
+    int tx = (p.UR + nchunks - 1) / nchunks;
+    if (nchunks > 1) tx = (tx + 31) / 32 * 32;
+    const int ty = std::max(1, 256 / tx);
+    // One wave of CTAs, each owning an equal share of the token rows.
+    static std::atomic<int> occ[2] = {{0}, {0}};
+    int o = occ[dtype == VRWKV_F32 ? 0 : 1].load(std::memory_order_relaxed);
+    if (o == 0) {
+        int nb = 0;
+        cudaError_t e = dtype == VRWKV_F32
+            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, channel_mix_vec_kernel<float>, 256, 0)
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, channel_mix_vec_kernel<__nv_bfloat16>, 256, 0);
+        if (e != cudaSuccess) return cuda_status(e, "channel_mix occupancy query");
+        o = std::max(1, nb);
+        occ[dtype == VRWKV_F32 ? 0 : 1].store(o, std::memory_order_relaxed);
+    }
+    int sms = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const long long row_groups = ((long long)p.BT + ty * kCmRows - 1) / (ty * kCmRows);
+    const long long gy = std::max<long long>(1, std::min<long long>(row_groups, (long long)sms * o / nchunks));
+    dim3 grid((unsigned)nchunks, (unsigned)gy), block((unsigned)tx, (unsigned)ty);
+    if (dtype == VRWKV_F32) channel_mix_vec_kernel<float><<<grid, block, 0, s>>>(p);
+    else channel_mix_vec_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(p);
+    g_last_kernel = "channel_mix_vec_kernel";
+    return cuda_status(cudaGetLastError(), "channel_mix kernel launch");
 }
 
 vrwkv_status vrwkv_biwkv_fwd(const void* k, const void* v, const float* w, const float* u, void* wkv,

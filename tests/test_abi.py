@@ -85,3 +85,23 @@ def test_qshift_rejects_invalid_arguments(lib):
     assert lib.vrwkv_qshift(FAKE, FAKE + (1 << 24), None, 1, 4, 4, 8, 1, 0.26, 0, None) == 1
     assert lib.vrwkv_qshift(FAKE, FAKE + 4, None, 1, 4, 4, 8, 1, 0.25, 0, None) == 1
     assert b"overlaps" in lib.vrwkv_last_error()
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(B=0), "positive"),
+    (dict(T=-3), "positive"),
+    (dict(x=None), "NULL"),
+    (dict(dtype=5), "dtype"),
+    (dict(x=FAKE + 1, dtype=1), "misaligned"),
+    (dict(out=FAKE + 64), "overlaps"),
+    (dict(qs=(14, 15)), "H*W"),
+    (dict(qs=(14, 14, 1, -0.1)), "gamma"),
+    (dict(B=1 << 16, T=1 << 15), "2^31"),
+])
+def test_channel_mix_rejects_invalid_arguments(lib, args, frag):
+    a = dict(x=FAKE, out=FAKE + (1 << 24), B=2, T=196, C=32, dtype=0, qs=None)
+    a.update(args)
+    qs = _qs(*a["qs"]) if a["qs"] else None
+    st = lib.vrwkv_channel_mix(a["x"], a["out"], a["B"], a["T"], a["C"], a["dtype"], qs, None)
+    assert st in (1, 2)
+    assert frag in lib.vrwkv_last_error().decode()
