@@ -83,6 +83,9 @@ struct alignas(16) Scratch {
     float2 mbM[kClusterMax][kNP];   // mailbox: each CTA's max of k (times log2 e)
     float4 mbF[kClusterMax][kNP];   // mailbox: each CTA's forward aggregate
     float4 mbG[kClusterMax][kNP];   // mailbox: each CTA's backward aggregate
+    float4 ownF[kNP];           // this CTA's inclusive forward aggregate, staged for the push
+    float4 ownG[kNP];           // this CTA's inclusive backward aggregate
+    float2 ownM[kNP];           // this CTA's max of k (times log2 e)
     float2 gpark[kTcMax / kL * kL][kNP];  // gate factors, parked between load and output
     float4 cscale[kCS];         // per channel: sl (scale of this CTA's own sums)
     float4 ccarry[kCS];         // per channel: carries Af, Cf, Bb, Db
@@ -399,23 +402,40 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
         if (wi == kNW - 1) yw = zero4();
         S.wcarF[jj][wi] = xw;
         S.wcarB[jj][wi] = yw;
-        // publish this CTA's record for pair jj into every CTA's mailbox
-        // (its own included) with remote shared-memory stores; the cluster
-        // barrier below makes them visible.  The CTA's forward aggregate sits
-        // at its last real warp (Tc may be shorter than 256 tokens).
-        if (p.ncl > 1 && (wi == p.Tc / 32 - 1 || wi == 0)) {
-            cg::cluster_group cluster = cg::this_cluster();
-            float2 Mj = S.wmax[jj][0];
+        // stage this CTA's record; the CTA's forward aggregate sits at its last
+        // real warp (Tc may be shorter than 256 tokens)
+        if (p.ncl > 1) {
+            if (wi == p.Tc / 32 - 1) S.ownF[jj] = f;
+            if (wi == 0) {
+                float2 Mj = S.wmax[jj][0];
 #pragma unroll
-            for (int w = 1; w < kNW; ++w) Mj = max2(Mj, S.wmax[jj][w]);
-            Mj = mul2(Mj, f2(kLog2e));  // base 2, the unit of the exponents below
-            for (int rr = 0; rr < p.ncl; ++rr) {
-                Scratch* P = cluster.map_shared_rank(&S, rr);
-                if (wi == p.Tc / 32 - 1) P->mbF[rank][jj] = f;
-                if (wi == 0) {
-                    P->mbG[rank][jj] = gb;
-                    P->mbM[rank][jj] = Mj;
-                }
+                for (int w = 1; w < kNW; ++w) Mj = max2(Mj, S.wmax[jj][w]);
+                S.ownG[jj] = gb;
+                S.ownM[jj] = mul2(Mj, f2(kLog2e));  // base 2, the unit of the exponents below
+            }
+        }
+    }
+    // Thread (peer rr, channel lc) of the exchange below: decay powers across
+    // d = 1, 2, 4, 8 CTAs, computed before the cluster barrier.
+    const int lc = tid >> 4, rr = tid & 15;
+    float mdec[4];
+    if (p.ncl > 1) {
+        const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
+        __syncthreads();
+        // publish the record into every CTA's mailbox (its own included) with
+        // remote shared-memory stores, one (peer, pair, half) per thread; the
+        // cluster barrier below makes them visible
+        const int peer = tid >> 4, jj = (tid >> 1) & 7;
+        if (peer < p.ncl) {
+            cg::cluster_group cluster = cg::this_cluster();
+            Scratch* P = cluster.map_shared_rank(&S, peer);
+            if ((tid & 1) == 0) {
+                P->mbF[rank][jj] = S.ownF[jj];
+            } else {
+                P->mbG[rank][jj] = S.ownG[jj];
+                P->mbM[rank][jj] = S.ownM[jj];
             }
         }
     }
@@ -432,7 +452,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
     // carries are 16-lane shuffle scans with the one-CTA decay a^Tc.
     float2 cs_sl = f2(1.0f), cs_af = f2(0.0f), cs_cf = f2(0.0f), cs_bb = f2(0.0f), cs_db = f2(0.0f);
     if (p.ncl > 1) {
-        const int lc = tid >> 4, rr = tid & 15;
         float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
         if (rr < p.ncl) {
             const float4 F = S.mbF[rr][lc >> 1], G = S.mbG[rr][lc >> 1];
@@ -452,10 +471,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
         fc2 *= sc;
         ga2 *= sc;
         gc2 *= sc;
-        const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
 #pragma unroll
-        for (int d = 1; d < kClusterMax; d <<= 1) {
-            const float m = ex2c(-(float)(p.Tc * d) * l2);  // decay across d CTAs
+        for (int e = 0, d = 1; d < kClusterMax; ++e, d <<= 1) {
+            const float m = mdec[e];  // decay across d CTAs
             const float ua = __shfl_up_sync(0xffffffffu, fa2, d, 16);
             const float uc = __shfl_up_sync(0xffffffffu, fc2, d, 16);
             const float da = __shfl_down_sync(0xffffffffu, ga2, d, 16);

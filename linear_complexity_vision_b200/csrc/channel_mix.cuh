@@ -10,7 +10,8 @@
 // run at the same time).  Shared memory and L1 deliver 128 B/clk/SM, too
 // little to fetch mu_r and mu_k for every element, so each thread owns ONE
 // fixed 16-byte vector of channels, keeps its mu values in registers and walks
-// a contiguous range of token rows, four rows in flight at a time.
+// a contiguous range of token rows, four rows in flight at a time (two
+// batches of two, software-pipelined).
 #pragma once
 
 #include "common.cuh"
@@ -55,41 +56,22 @@ struct ChannelMixParams {
     FastDiv divT, divW;
 };
 
-constexpr int kCmRows = 4;  // token rows in flight per thread
+constexpr int kCmRows = 2;  // token rows per load batch; two batches in flight
 
-// Vector path: C*sizeof(IO) is a multiple of 16, x and out are 16-byte aligned
-// and no vector straddles a channel-group boundary (g is a multiple of the
-// vector width, or g == 0).  blockDim = (tx, ty): threadIdx.x picks the
-// vector within a channel chunk of tx vectors (blockIdx.x), threadIdx.y the
-// row within a group of ty consecutive rows.  blockIdx.y owns the contiguous
-// token-row range [BT*by/Gy, BT*(by+1)/Gy), so every CTA moves the same bytes.
 template <typename IO>
-__global__ void __launch_bounds__(256, 3) channel_mix_vec_kernel(const ChannelMixParams p) {
+struct CmColumn {
     using V = Vec16<IO>;
-    constexpr int N = V::N;
-    const int v = blockIdx.x * blockDim.x + threadIdx.x;
-    if (v >= p.UR) return;
-    const int c0 = v * N;
-
+    static constexpr int N = V::N;
+    const ChannelMixParams& p;
+    ShiftRule rule;
     float2 mur[N / 2], muk[N / 2];
-#pragma unroll
-    for (int e = 0; e < N / 2; ++e) {
-        mur[e] = p.mu_r ? __ldg(reinterpret_cast<const float2*>(p.mu_r + c0) + e) : f2(0.0f);
-        muk[e] = p.mu_k ? __ldg(reinterpret_cast<const float2*>(p.mu_k + c0) + e) : f2(0.0f);
-    }
-    // Without mu the mix below, xd + mu*(x - xd), is xd itself.
-    const ShiftRule rule = shift_rule(c0, p.g, p.H, p.W, p.s);
+    const char* xcol;
+    char* ocol;
+    size_t rowb;
+    int r1, ty;
 
-    const long long Gy = gridDim.y;
-    const int r0 = (int)((long long)p.BT * blockIdx.y / Gy);
-    const int r1 = (int)((long long)p.BT * (blockIdx.y + 1) / Gy);
-    const int ty = blockDim.y;
-    const size_t rowb = (size_t)p.C * sizeof(IO);
-    const char* xcol = p.x + (size_t)c0 * sizeof(IO);
-    char* ocol = p.out + (size_t)c0 * sizeof(IO);
-
-    for (int base = r0 + threadIdx.y; base < r1; base += ty * kCmRows) {
-        uint4 rx[kCmRows], rd[kCmRows];
+    // Loads x and x_shift of rows base, base+ty, ... (rows >= r1 read nothing).
+    __device__ __forceinline__ void load(int base, uint4 (&rx)[kCmRows], uint4 (&rd)[kCmRows]) const {
 #pragma unroll
         for (int j = 0; j < kCmRows; ++j) {
             const int r = base + j * ty;
@@ -101,10 +83,13 @@ __global__ void __launch_bounds__(256, 3) channel_mix_vec_kernel(const ChannelMi
                 const int w = (int)t - h * p.W;
                 rx[j] = __ldg(reinterpret_cast<const uint4*>(xcol + (size_t)r * rowb));
                 if (shift_ok(rule, h, w))
-                    rd[j] = __ldg(reinterpret_cast<const uint4*>(
-                        xcol + (size_t)(r + rule.off) * rowb));
+                    rd[j] = __ldg(reinterpret_cast<const uint4*>(xcol + (size_t)(r + rule.off) * rowb));
             }
         }
+    }
+
+    __device__ __forceinline__ void compute(int base, const uint4 (&rx)[kCmRows],
+                                            const uint4 (&rd)[kCmRows]) const {
 #pragma unroll
         for (int j = 0; j < kCmRows; ++j) {
             const int r = base + j * ty;
@@ -128,6 +113,50 @@ __global__ void __launch_bounds__(256, 3) channel_mix_vec_kernel(const ChannelMi
             }
             __stcs(reinterpret_cast<uint4*>(ocol + (size_t)r * rowb), V::pack(o));
         }
+    }
+};
+
+// Vector path: C*sizeof(IO) is a multiple of 16, x and out are 16-byte aligned
+// and no vector straddles a channel-group boundary (g is a multiple of the
+// vector width, or g == 0).  blockDim = (tx, ty): threadIdx.x picks the
+// vector within a channel chunk of tx vectors (blockIdx.x), threadIdx.y the
+// row within a group of ty consecutive rows.  blockIdx.y owns the contiguous
+// token-row range [BT*by/Gy, BT*(by+1)/Gy), so every CTA moves the same bytes.
+// The loads of the next batch of rows are issued before the current batch is
+// computed (two register sets), keeping four row loads per thread in flight.
+template <typename IO>
+__global__ void __launch_bounds__(256, 3) channel_mix_vec_kernel(const ChannelMixParams p) {
+    constexpr int N = Vec16<IO>::N;
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= p.UR) return;
+    const int c0 = v * N;
+
+    CmColumn<IO> col{p};
+#pragma unroll
+    for (int e = 0; e < N / 2; ++e) {
+        col.mur[e] = p.mu_r ? __ldg(reinterpret_cast<const float2*>(p.mu_r + c0) + e) : f2(0.0f);
+        col.muk[e] = p.mu_k ? __ldg(reinterpret_cast<const float2*>(p.mu_k + c0) + e) : f2(0.0f);
+    }
+    // Without mu the mix, xd + mu*(x - xd), is xd itself.
+    col.rule = shift_rule(c0, p.g, p.H, p.W, p.s);
+    const long long Gy = gridDim.y;
+    const int r0 = (int)((long long)p.BT * blockIdx.y / Gy);
+    col.r1 = (int)((long long)p.BT * (blockIdx.y + 1) / Gy);
+    col.ty = blockDim.y;
+    col.rowb = (size_t)p.C * sizeof(IO);
+    col.xcol = p.x + (size_t)c0 * sizeof(IO);
+    col.ocol = p.out + (size_t)c0 * sizeof(IO);
+
+    const int step = col.ty * kCmRows;
+    uint4 ax[kCmRows], ad[kCmRows], bx[kCmRows], bd[kCmRows];
+    int base = r0 + threadIdx.y;
+    col.load(base, ax, ad);
+    for (; base < col.r1; base += 2 * step) {
+        col.load(base + step, bx, bd);
+        col.compute(base, ax, ad);
+        if (base + step >= col.r1) break;
+        col.load(base + 2 * step, ax, ad);
+        col.compute(base + step, bx, bd);
     }
 }
 
