@@ -311,7 +311,8 @@ def time_channel_mix(runner, stream, torch, dev, launches: int, peak: float):
     nbytes = 2 * wl.N * es + 2 * wl.C * 4  # x once, out once, mu_r and mu_k
     achieved = nbytes / (us * 1e-6) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "kernel": runner.kernel_name,
+            "frac": achieved / peak, "traffic": committed_traffic("channel_mix/" + wl.name),
+            "kernel": runner.kernel_name,
             "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
             "launches": reps * G}
 

@@ -22,10 +22,12 @@
 //    per-token shift arithmetic remains: token t of both tiles sits at the
 //    same shared-memory offset.  A CTA's 16 channels lie in one channel
 //    group (the host requires the group size to be a multiple of 16).
-//  * 256 threads and <= 128 registers per thread: two CTAs per SM, so one
-//    CTA's barriers and scans overlap the other's arithmetic.  Sequences
+//  * 256-thread CTAs at 64 registers per thread: four CTAs per SM, so one
+//    CTA's barriers and scans overlap another's arithmetic.  Sequences
 //    longer than 256 tokens split over a thread-block cluster of up to 16
 //    CTAs along T; CTA aggregates travel through distributed shared memory.
+//  * Arrays that a warp reads down a column ([pair][warp], [peer][pair])
+//    have one element of row padding, so those reads are bank-conflict free.
 //  * Decay powers a^(8m) come from a per-CTA table (one exp2 each), the
 //    bf16 unpack is integer arithmetic, and arithmetic is packed float2.
 // Exponents are base 2 (log2 e is folded into k, u, w and r).
@@ -45,13 +47,21 @@ namespace cg = cooperative_groups;
 constexpr int kCS = 16;         // channels per CTA
 constexpr int kNP = kCS / 2;    // channel pairs per CTA
 constexpr int kL = 8;           // tokens per thread chunk
-constexpr int kThreads = 256;   // threads per CTA
-constexpr int kNW = kThreads / 32;
-constexpr int kTcMax = kThreads / kNP * kL;  // 256 tokens per CTA
 constexpr int kClusterMax = 16;
-constexpr int kMinBlocks = 4;   // resident CTAs per SM the register budget targets
-constexpr int kTab = kTcMax / kL;            // a^(8m), m < 32
+constexpr int kExThreads = kCS * kClusterMax;  // threads of the cross-CTA exchange
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+
+// CTA shape: NT threads = 8 channel pairs x NT/8 chunks of 8 tokens, so a
+// CTA spans NT tokens, at 64 registers per thread (1024/NT CTAs per SM).  The
+// library launches NT = 256 (four CTAs per SM, clusters of up to 16 along T).
+template <int NT>
+struct Cfg {
+    static constexpr int kThreads = NT;
+    static constexpr int kNW = NT / 32;             // warps
+    static constexpr int kTcMax = NT / kNP * kL;    // tokens per CTA (= NT)
+    static constexpr int kTab = kTcMax / kL;        // a^(8m), m < kTab
+    static constexpr int kMinBlocks = 1024 / NT;    // resident CTAs per SM (64 registers)
+};
 
 enum Layout { kKV = 0, kRKV = 1, kX = 2 };
 
@@ -73,20 +83,25 @@ struct alignas(64) Params {
     int box_bytes;       // bytes one strided box delivers (zero fill included)
 };
 
+template <int NT>
 struct alignas(16) Scratch {
-    float2 tab[kTab][kNP];      // a^(8m) per channel pair
-    float2 wmax[kNP][kNW];      // per-warp maxima of k
-    float4 waggF[kNP][kNW];     // per-warp forward aggregates (A.xy, C.xy)
-    float4 waggB[kNP][kNW];     // per-warp backward aggregates
-    float4 wcarF[kNP][kNW];     // exclusive forward carry into each warp
-    float4 wcarB[kNP][kNW];     // exclusive backward carry into each warp
-    float2 mbM[kClusterMax][kNP];   // mailbox: each CTA's max of k (times log2 e)
-    float4 mbF[kClusterMax][kNP];   // mailbox: each CTA's forward aggregate
-    float4 mbG[kClusterMax][kNP];   // mailbox: each CTA's backward aggregate
+    static constexpr int kNW = Cfg<NT>::kNW;
+    float2 tab[Cfg<NT>::kTab][kNP];  // a^(8m) per channel pair
+    // Rows of the [pair][warp] and [peer][pair] arrays carry one element of
+    // padding: a warp reads one column across eight (or sixteen) rows, and
+    // the odd row stride spreads those reads over all 32 banks.
+    float2 wmax[kNP][kNW + 1];      // per-warp maxima of k
+    float4 waggF[kNP][kNW + 1];     // per-warp forward aggregates (A.xy, C.xy)
+    float4 waggB[kNP][kNW + 1];     // per-warp backward aggregates
+    float4 wcarF[kNP][kNW + 1];     // exclusive forward carry into each warp
+    float4 wcarB[kNP][kNW + 1];     // exclusive backward carry into each warp
+    float2 mbM[kClusterMax][kNP + 1];   // mailbox: each CTA's max of k (times log2 e)
+    float4 mbF[kClusterMax][kNP + 1];   // mailbox: each CTA's forward aggregate
+    float4 mbG[kClusterMax][kNP + 1];   // mailbox: each CTA's backward aggregate
     float4 ownF[kNP];           // this CTA's inclusive forward aggregate, staged for the push
     float4 ownG[kNP];           // this CTA's inclusive backward aggregate
     float2 ownM[kNP];           // this CTA's max of k (times log2 e)
-    float2 gpark[kTcMax / kL * kL][kNP];  // gate factors, parked between load and output
+    float2 gpark[Cfg<NT>::kTcMax][kNP];  // gate factors, parked between load and output
     float4 cscale[kCS];         // per channel: sl (scale of this CTA's own sums)
     float4 ccarry[kCS];         // per channel: carries Af, Cf, Bb, Db
     unsigned long long bar;     // TMA completion barrier
@@ -184,8 +199,12 @@ __device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); 
 __device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); }
 __device__ __forceinline__ float4 zero4() { return make_float4(0.f, 0.f, 0.f, 0.f); }
 
-template <typename IO, int LAYOUT, bool QS>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const __grid_constant__ Params p) {
+template <typename IO, int LAYOUT, bool QS, int NT>
+__global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(const __grid_constant__ Params p) {
+    constexpr int kThreads = Cfg<NT>::kThreads;
+    constexpr int kNW = Cfg<NT>::kNW;
+    constexpr int kTcMax = Cfg<NT>::kTcMax;
+    using Scratch = fast::Scratch<NT>;
     constexpr bool GATE = LAYOUT != kKV;
     constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
     constexpr int NTILE = NSRC * (QS ? 2 : 1);
@@ -222,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
     const bool shifted = QS && grp < 4;
 
     // ---- issue the tile loads: lane i of warp 0 loads sub-tile i of each tile
-    constexpr int SUB = kTcMax / kL * RB;  // bytes per sub-tile (32 token rows)
+    constexpr int SUB = kTcMax / kL * RB;  // bytes per sub-tile (kTcMax / 8 token rows)
     if (tid == 0) mbar_init(&S.bar, 1);
     __syncthreads();
     if (warp == 0) {
@@ -236,7 +255,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
             for (int s = 0; s < NSRC; ++s) {
                 char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB;
                 if (!QS) {
-                    tma_load_3d(plain, &p.map[s], c0, t0 + i, b, &S.bar);
+                    // boxes of 256 strided tokens (32 rows); a box wholly past T
+                    // still delivers its zero-filled bytes
+#pragma unroll
+                    for (int h = 0; h < kTcMax / 256; ++h)
+                        tma_load_3d(plain + h * 32 * RB, &p.map[s], c0, t0 + i + 256 * h, b, &S.bar);
                 } else {
                     tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar);
                     if (shifted) {
@@ -386,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
     if (cq == 3) S.waggF[j][warp] = Fi;
     if (cq == 0) S.waggB[j][warp] = Gi;
     __syncthreads();
-    if (tid < kNP * kNW) {  // 64 threads: one per (pair, warp)
-        const int jj = tid >> 3, wi = tid & 7;
+    if (tid < kNP * kNW) {  // one thread per (pair, warp)
+        const int jj = tid / kNW, wi = tid % kNW;
         float4 f = S.waggF[jj][wi], gb = S.waggB[jj][wi];
 #pragma unroll
         for (int d = 1; d < kNW; d <<= 1) {
@@ -415,14 +438,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
             }
         }
     }
-    // Thread (peer rr, channel lc) of the exchange below: decay powers across
-    // d = 1, 2, 4, 8 CTAs, computed before the cluster barrier.
+    // Thread (peer rr, channel lc) of the exchange below (the first 256
+    // threads): decay powers across d = 1, 2, 4, 8 CTAs, computed before the
+    // cluster barrier.
     const int lc = tid >> 4, rr = tid & 15;
     float mdec[4];
     if (p.ncl > 1) {
-        const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
+        if (tid < kExThreads) {
+            const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
+            for (int e = 0; e < 4; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
+        }
         __syncthreads();
         // publish the record into every CTA's mailbox (its own included) with
         // remote shared-memory stores, one (peer, pair, half) per thread; the
@@ -452,52 +478,54 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) biwkv_tma_kernel(const _
     // carries are 16-lane shuffle scans with the one-CTA decay a^Tc.
     float2 cs_sl = f2(1.0f), cs_af = f2(0.0f), cs_cf = f2(0.0f), cs_bb = f2(0.0f), cs_db = f2(0.0f);
     if (p.ncl > 1) {
-        float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
-        if (rr < p.ncl) {
-            const float4 F = S.mbF[rr][lc >> 1], G = S.mbG[rr][lc >> 1];
-            const float2 Mp = S.mbM[rr][lc >> 1];
-            const bool hi = lc & 1;
-            Mr = hi ? Mp.y : Mp.x;
-            fa2 = hi ? F.y : F.x;
-            fc2 = hi ? F.w : F.z;
-            ga2 = hi ? G.y : G.x;
-            gc2 = hi ? G.w : G.z;
-        }
-        float Mc = Mr;
-#pragma unroll
-        for (int d = 8; d >= 1; d >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, 16));
-        const float sc = ex2(Mr - Mc);  // 0 for lanes past the cluster
-        fa2 *= sc;
-        fc2 *= sc;
-        ga2 *= sc;
-        gc2 *= sc;
-#pragma unroll
-        for (int e = 0, d = 1; d < kClusterMax; ++e, d <<= 1) {
-            const float m = mdec[e];  // decay across d CTAs
-            const float ua = __shfl_up_sync(0xffffffffu, fa2, d, 16);
-            const float uc = __shfl_up_sync(0xffffffffu, fc2, d, 16);
-            const float da = __shfl_down_sync(0xffffffffu, ga2, d, 16);
-            const float dc = __shfl_down_sync(0xffffffffu, gc2, d, 16);
-            if (rr >= d) {
-                fa2 = fmaf(m, ua, fa2);
-                fc2 = fmaf(m, uc, fc2);
+        if (tid < kExThreads) {  // warp-uniform
+            float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
+            if (rr < p.ncl) {
+                const float4 F = S.mbF[rr][lc >> 1], G = S.mbG[rr][lc >> 1];
+                const float2 Mp = S.mbM[rr][lc >> 1];
+                const bool hi = lc & 1;
+                Mr = hi ? Mp.y : Mp.x;
+                fa2 = hi ? F.y : F.x;
+                fc2 = hi ? F.w : F.z;
+                ga2 = hi ? G.y : G.x;
+                gc2 = hi ? G.w : G.z;
             }
-            if (rr + d < kClusterMax) {
-                ga2 = fmaf(m, da, ga2);
-                gc2 = fmaf(m, dc, gc2);
+            float Mc = Mr;
+#pragma unroll
+            for (int d = 8; d >= 1; d >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, 16));
+            const float sc = ex2(Mr - Mc);  // 0 for lanes past the cluster
+            fa2 *= sc;
+            fc2 *= sc;
+            ga2 *= sc;
+            gc2 *= sc;
+#pragma unroll
+            for (int e = 0, d = 1; d < kClusterMax; ++e, d <<= 1) {
+                const float m = mdec[e];  // decay across d CTAs
+                const float ua = __shfl_up_sync(0xffffffffu, fa2, d, 16);
+                const float uc = __shfl_up_sync(0xffffffffu, fc2, d, 16);
+                const float da = __shfl_down_sync(0xffffffffu, ga2, d, 16);
+                const float dc = __shfl_down_sync(0xffffffffu, gc2, d, 16);
+                if (rr >= d) {
+                    fa2 = fmaf(m, ua, fa2);
+                    fc2 = fmaf(m, uc, fc2);
+                }
+                if (rr + d < kClusterMax) {
+                    ga2 = fmaf(m, da, ga2);
+                    gc2 = fmaf(m, dc, gc2);
+                }
             }
-        }
-        // exclusive carries of this CTA: inclusive forward at rank-1,
-        // inclusive backward at rank+1 (zero past the ends)
-        const float Af = __shfl_sync(0xffffffffu, fa2, max(rank - 1, 0), 16);
-        const float Cf = __shfl_sync(0xffffffffu, fc2, max(rank - 1, 0), 16);
-        const float Bb = __shfl_sync(0xffffffffu, ga2, min(rank + 1, kClusterMax - 1), 16);
-        const float Db = __shfl_sync(0xffffffffu, gc2, min(rank + 1, kClusterMax - 1), 16);
-        const float Mme = __shfl_sync(0xffffffffu, Mr, rank, 16);
-        if (rr == 0) {
-            S.cscale[lc] = make_float4(ex2(Mme - Mc), 0.f, 0.f, 0.f);
-            S.ccarry[lc] = make_float4(rank > 0 ? Af : 0.f, rank > 0 ? Cf : 0.f,
-                                       rank + 1 < p.ncl ? Bb : 0.f, rank + 1 < p.ncl ? Db : 0.f);
+            // exclusive carries of this CTA: inclusive forward at rank-1,
+            // inclusive backward at rank+1 (zero past the ends)
+            const float Af = __shfl_sync(0xffffffffu, fa2, max(rank - 1, 0), 16);
+            const float Cf = __shfl_sync(0xffffffffu, fc2, max(rank - 1, 0), 16);
+            const float Bb = __shfl_sync(0xffffffffu, ga2, min(rank + 1, kClusterMax - 1), 16);
+            const float Db = __shfl_sync(0xffffffffu, gc2, min(rank + 1, kClusterMax - 1), 16);
+            const float Mme = __shfl_sync(0xffffffffu, Mr, rank, 16);
+            if (rr == 0) {
+                S.cscale[lc] = make_float4(ex2(Mme - Mc), 0.f, 0.f, 0.f);
+                S.ccarry[lc] = make_float4(rank > 0 ? Af : 0.f, rank > 0 ? Cf : 0.f,
+                                           rank + 1 < p.ncl ? Bb : 0.f, rank + 1 < p.ncl ? Db : 0.f);
+            }
         }
         __syncthreads();
         const float4 s0 = S.cscale[2 * j], s1 = S.cscale[2 * j + 1];

@@ -166,13 +166,14 @@ struct FastPlan {
     fast::Params p;
     int layout;
     bool qs;
+    int nt;  // threads (= tokens) per CTA
     dim3 grid;
     int smem;
 };
 
-template <typename IO, int LAYOUT, bool QS>
+template <typename IO, int LAYOUT, bool QS, int NT>
 vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
-    auto kern = fast::biwkv_tma_kernel<IO, LAYOUT, QS>;
+    auto kern = fast::biwkv_tma_kernel<IO, LAYOUT, QS, NT>;
     static std::atomic<int> granted{0};
     static std::atomic<int> nonportable{0};
     cudaError_t e = ensure_smem(kern, granted, pl.smem);
@@ -188,7 +189,7 @@ vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_bac
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = pl.grid;
-    cfg.blockDim = dim3(fast::kThreads, 1, 1);
+    cfg.blockDim = dim3(NT, 1, 1);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -220,16 +221,31 @@ vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_bac
     return ok();
 }
 
+template <typename IO, int NT>
+vrwkv_status dispatch_fast_nt(const FastPlan& pl, cudaStream_t s, bool* fb) {
+    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
+    case fast::kKV * 2 + 0: return launch_fast<IO, fast::kKV, false, NT>(pl, s, fb);
+    case fast::kKV * 2 + 1: return launch_fast<IO, fast::kKV, true, NT>(pl, s, fb);
+    case fast::kRKV * 2 + 0: return launch_fast<IO, fast::kRKV, false, NT>(pl, s, fb);
+    case fast::kRKV * 2 + 1: return launch_fast<IO, fast::kRKV, true, NT>(pl, s, fb);
+    case fast::kX * 2 + 0: return launch_fast<IO, fast::kX, false, NT>(pl, s, fb);
+    default: return launch_fast<IO, fast::kX, true, NT>(pl, s, fb);
+    }
+}
+
+// CTA size of the fast path.  512-thread CTAs (8-CTA clusters at T = 4096)
+// measured slower than 256-thread CTAs (16-CTA clusters): fewer independent
+// CTAs per SM hide less of each other's barrier and exchange latency.
+constexpr int kFastThreads = 256;
+
 template <typename IO>
 vrwkv_status dispatch_fast(const FastPlan& pl, cudaStream_t s, bool* fb) {
-    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
-    case fast::kKV * 2 + 0: return launch_fast<IO, fast::kKV, false>(pl, s, fb);
-    case fast::kKV * 2 + 1: return launch_fast<IO, fast::kKV, true>(pl, s, fb);
-    case fast::kRKV * 2 + 0: return launch_fast<IO, fast::kRKV, false>(pl, s, fb);
-    case fast::kRKV * 2 + 1: return launch_fast<IO, fast::kRKV, true>(pl, s, fb);
-    case fast::kX * 2 + 0: return launch_fast<IO, fast::kX, false>(pl, s, fb);
-    default: return launch_fast<IO, fast::kX, true>(pl, s, fb);
-    }
+    return dispatch_fast_nt<IO, kFastThreads>(pl, s, fb);
+}
+
+// Shared memory of a fast-path CTA: the tiles plus the scratch block.
+int fast_smem(int ntiles, int tile_bytes) {
+    return ntiles * tile_bytes + (int)sizeof(fast::Scratch<kFastThreads>) + 128;  // + alignment slack
 }
 
 // Plan the TMA path; returns false when the problem is outside its limits
@@ -267,19 +283,23 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     p.B = B;
     p.T = T;
     p.C = C;
+    const int RB = fast::kCS * es;
+    const int ntiles = nsrc * (pl.qs ? 2 : 1);
+    pl.nt = kFastThreads;
+    const int TcMax = fast::Cfg<kFastThreads>::kTcMax;
     if (pl.qs) {
         p.H = qs->H;
         p.W = qs->W;
         p.s = qs->shift_pixel;
         p.g = group_size(C, qs->gamma);
         if (p.g % fast::kCS != 0 || p.W > 256 || p.W % fast::kL != 0) return false;
-        if (T <= fast::kTcMax) {
+        if (T <= TcMax) {
             p.rows = p.H;
             p.Tc = T;
             p.ncl = 1;
         } else {
             int rows = 0;
-            for (int rr = fast::kTcMax / p.W; rr >= 1; --rr)
+            for (int rr = TcMax / p.W; rr >= 1; --rr)
                 if ((rr * p.W) % 32 == 0) {
                     rows = rr;
                     break;
@@ -295,19 +315,19 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         p.s = 0;
         p.g = 0;
         p.rows = 1;
-        p.Tc = std::min(T, fast::kTcMax);
+        p.Tc = std::min(T, TcMax);
         p.ncl = (T + p.Tc - 1) / p.Tc;
     }
     if (p.ncl > fast::kClusterMax) return false;
-    const int RB = fast::kCS * es;
-    // 8 sub-tiles of 32 token rows; every thread reads its row of each, so a
-    // tile always spans 256 tokens even when the boxes deliver fewer
-    p.tile_bytes = fast::kTcMax * RB;
-    // a strided box delivers (W / 8) x rows token rows with Q-Shift, and its
-    // full 256 / 8 = 32 rows without (tokens past T arrive as zeros)
-    p.box_bytes = (pl.qs ? (p.W / fast::kL) * p.rows : fast::kTcMax / fast::kL) * RB;
-    const int ntiles = nsrc * (pl.qs ? 2 : 1);
-    pl.smem = ntiles * p.tile_bytes + (int)sizeof(fast::Scratch) + 128;  // + alignment slack
+    // 8 sub-tiles of TcMax / 8 token rows; every thread reads its row of
+    // each, so a tile always spans TcMax tokens even when the boxes deliver
+    // fewer
+    p.tile_bytes = TcMax * RB;
+    // a sub-tile receives (W / 8) x rows token rows with Q-Shift (one box),
+    // and its full TcMax / 8 rows without (boxes of 32 rows; tokens past T
+    // arrive as zeros)
+    p.box_bytes = (pl.qs ? (p.W / fast::kL) * p.rows : TcMax / fast::kL) * RB;
+    pl.smem = fast_smem(ntiles, p.tile_bytes);
     if (pl.smem > 227 * 1024) return false;
     const CUtensorMapDataType dt =
         dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -326,7 +346,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         } else {
             const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
             const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
-            const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, (cuuint32_t)fast::kTcMax, 1};
+            const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, 256u, 1};  // 32 strided rows
             cr = enc(&p.map[i], dt, 3, const_cast<void*>(srcs[i]), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
