@@ -20,6 +20,9 @@ It wraps ``vrwkv_oracle.c`` (plain C, float64, OpenMP over channel columns):
                        page describes (short sequences only).
 * ``gate``          -- sigma(R) (.) wkv of eq. 2.
 * ``spatial_core``  -- gate(QS_R(r), Bi-WKV(QS_K(k), QS_V(v))).
+* ``biwkv_bwd``     -- gradients of eq. 5 (dk, dv and per-batch dw, du) for
+                       an upstream gradient gy, by the chain rule, O(T^2).
+* ``biwkv_bwd_columns`` -- the same for selected (b, c) columns only.
 * ``channel_mix``   -- sigma(QS_R(x)) * max(QS_K(x), 0)^2, the channel-mix
                        module of eq. 3-4 without projections.
 * ``spatial_core_points`` -- the same at selected output positions only, by
@@ -72,6 +75,9 @@ def _load():
         lib.oracle_biwkv_direct_points.argtypes = [dp, dp, dp, dp, ci, ci, ci,
                                                    i64p, cl, dp]
         lib.oracle_gate.argtypes = [dp, dp, dp, cl]
+        lib.oracle_biwkv_bwd_direct.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, dp, dp, dp, dp]
+        lib.oracle_biwkv_bwd_columns.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ctypes.c_void_p,
+                                                 ctypes.c_long, dp, dp, dp, dp]
         lib.oracle_channel_mix.argtypes = [dp, dp, dp, dp, ci, ci, ci, ci, ci, cd]
         lib.oracle_spatial_core_points.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, ci,
                                                    ci, ci, cd, ci, ci, i64p, cl, dp]
@@ -227,3 +233,31 @@ def channel_mix(x, H, W, shift_pixel=1, gamma=0.25, mu_r=None, mu_k=None) -> np.
                                None if mus[1] is None else _ptr(mus[1]), _ptr(out), B, H, W, C,
                                int(shift_pixel), float(gamma))
     return out
+
+
+def biwkv_bwd(k, v, w, u, gy):
+    """Gradients of eq. 5: (gk, gv) of shape (B, T, C) and (gw, gu) of shape
+    (B, C), the per-batch contributions to dL/dw and dL/du."""
+    k, v, gy = _d(k), _d(v), _d(gy)
+    w, u = _d(w), _d(u)
+    B, T, C = k.shape
+    gk, gv = np.empty_like(k), np.empty_like(k)
+    gw, gu = np.empty((B, C)), np.empty((B, C))
+    _load().oracle_biwkv_bwd_direct(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(gy), B, T, C,
+                                    _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu))
+    return gk, gv, gw, gu
+
+
+def biwkv_bwd_columns(k, v, w, u, gy, cols):
+    """biwkv_bwd restricted to the flat columns cols[j] = b*C + c: gk, gv of
+    shape (n, T); gw, gu of shape (n,)."""
+    k, v, gy = _d(k), _d(v), _d(gy)
+    w, u = _d(w), _d(u)
+    B, T, C = k.shape
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    n = cols.size
+    gk, gv = np.empty((n, T)), np.empty((n, T))
+    gw, gu = np.empty(n), np.empty(n)
+    _load().oracle_biwkv_bwd_columns(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(gy), B, T, C,
+                                     cols.ctypes.data, n, _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu))
+    return gk, gv, gw, gu

@@ -12,7 +12,11 @@
  *              - Linear Complexity Bidirectional Attention, eq. 5 (summation
  *                form of Bi-WKV) and eq. 6-7 (RNN form, hidden states a,b,c,d);
  *              - Quad-Directional Token Shift, eq. 9 (Q-Shift);
- *              - Overall Architecture, eq. 2 (sigma(R) (.) wkv gate).
+ *              - Overall Architecture, eq. 2 (sigma(R) (.) wkv gate) and
+ *                eq. 3-4 (channel mix);
+ *              - the Bi-WKV backward pass, which the pages place in an
+ *                appendix they do not reproduce: here it is the plain
+ *                derivative of eq. 5, written out below.
  *   [BLOG]   "LinXin's Blog" (linxin.blog), Vision-RWKV entry: the q_shift
  *            listing (patch_resolution, shift_pixel, gamma, zero-initialised
  *            output, four slice assignments, copy of the remaining channels).
@@ -407,5 +411,119 @@ void oracle_channel_mix(const double* x, const double* mu_r,
             double kp = ks > 0.0 ? ks : 0.0;
             out[bt * C + c] = (1.0 / (1.0 + exp(-rs))) * (kp * kp);
         }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Bi-WKV backward: derivatives of eq. 5                               */
+/* ------------------------------------------------------------------ */
+/* For one (b, c) column with weights
+ *   W_ti = exp(-(|t-i|-1)/T * w)  (i != t),   W_tt = exp(u),
+ *   N_t = sum_i W_ti e^{k_i} v_i,  D_t = sum_i W_ti e^{k_i},  y_t = N_t / D_t,
+ * and the upstream gradient g_t = dL/dy_t, the chain rule gives
+ *   dL/dv_i = e^{k_i} sum_t W_ti g_t / D_t
+ *   dL/dk_i = e^{k_i} sum_t W_ti g_t (v_i - y_t) / D_t
+ *   dL/du   = sum_t e^{u + k_t} g_t (v_t - y_t) / D_t
+ *   dL/dw   = -(1/T) sum_t sum_{i != t} (|t-i|-1) W_ti e^{k_i} g_t (v_i - y_t) / D_t
+ * Every term is a ratio e^{k_i} / D_t, so e^{k} is evaluated as e^{k - max k}
+ * (the factor cancels) to keep the exponentials in range.  O(T^2) per column. */
+static void biwkv_bwd_column(const double* kc, const double* vc,
+                             const double* gc, long T, double w, double u,
+                             double* gk, double* gv, double* gw, double* gu,
+                             double* y, double* q) {
+    double M = kc[0];
+    for (long i = 1; i < T; ++i)
+        if (kc[i] > M) M = kc[i];
+    /* forward values: y_t and q_t = g_t / D_t (D_t scaled by e^{-M}) */
+    for (long t = 0; t < T; ++t) {
+        double num = 0.0, den = 0.0;
+        for (long i = 0; i < T; ++i) {
+            double e;
+            if (i == t) {
+                e = exp(u + kc[i] - M);
+            } else {
+                long d = i > t ? i - t : t - i;
+                e = exp(-((double)(d - 1) / (double)T) * w + kc[i] - M);
+            }
+            num += e * vc[i];
+            den += e;
+        }
+        y[t] = num / den;
+        q[t] = gc[t] / den;
+    }
+    double sgu = 0.0, sgw = 0.0;
+    for (long i = 0; i < T; ++i) {
+        double sv = 0.0, sk = 0.0;
+        for (long t = 0; t < T; ++t) {
+            double e;  /* W_ti e^{k_i - M} */
+            if (t == i) {
+                e = exp(u + kc[i] - M);
+                sgu += e * q[t] * (vc[i] - y[t]);
+            } else {
+                long d = i > t ? i - t : t - i;
+                e = exp(-((double)(d - 1) / (double)T) * w + kc[i] - M);
+                sgw += (double)(d - 1) * e * q[t] * (vc[i] - y[t]);
+            }
+            sv += e * q[t];
+            sk += e * q[t] * (vc[i] - y[t]);
+        }
+        gv[i] = sv;
+        gk[i] = sk;
+    }
+    *gu = sgu;
+    *gw = -sgw / (double)T;
+}
+
+/* Gradients of every column.  gk, gv: (B, T, C); gw, gu: (B, C), the
+ * contribution of each batch element (the batch gradient is their sum). */
+void oracle_biwkv_bwd_direct(const double* k, const double* v, const double* w,
+                             const double* u, const double* gy, int B, int T,
+                             int C, double* gk, double* gv, double* gw,
+                             double* gu) {
+#pragma omp parallel
+    {
+        double* buf = (double*)malloc(sizeof(double) * (size_t)T * 7);
+        double *kc = buf, *vc = buf + T, *gc = buf + 2 * T, *ok = buf + 3 * T,
+               *ov = buf + 4 * T, *y = buf + 5 * T, *q = buf + 6 * T;
+#pragma omp for schedule(dynamic, 1)
+        for (long bc = 0; bc < (long)B * C; ++bc) {
+            long b = bc / C, c = bc % C;
+            gather_column(k, kc, b, T, C, c);
+            gather_column(v, vc, b, T, C, c);
+            gather_column(gy, gc, b, T, C, c);
+            biwkv_bwd_column(kc, vc, gc, T, w[c], u[c], ok, ov, &gw[bc], &gu[bc],
+                             y, q);
+            for (long t = 0; t < T; ++t) {
+                gk[(b * T + t) * C + c] = ok[t];
+                gv[(b * T + t) * C + c] = ov[t];
+            }
+        }
+        free(buf);
+    }
+}
+
+/* The same for selected columns cols[j] = b*C + c only: gk, gv are (n, T),
+ * gw, gu are (n). */
+void oracle_biwkv_bwd_columns(const double* k, const double* v,
+                              const double* w, const double* u,
+                              const double* gy, int B, int T, int C,
+                              const int64_t* cols, long n, double* gk,
+                              double* gv, double* gw, double* gu) {
+    (void)B;
+#pragma omp parallel
+    {
+        double* buf = (double*)malloc(sizeof(double) * (size_t)T * 5);
+        double *kc = buf, *vc = buf + T, *gc = buf + 2 * T, *y = buf + 3 * T,
+               *q = buf + 4 * T;
+#pragma omp for schedule(dynamic, 1)
+        for (long j = 0; j < n; ++j) {
+            long b = (long)cols[j] / C, c = (long)cols[j] % C;
+            gather_column(k, kc, b, T, C, c);
+            gather_column(v, vc, b, T, C, c);
+            gather_column(gy, gc, b, T, C, c);
+            biwkv_bwd_column(kc, vc, gc, T, w[c], u[c], gk + j * (long)T,
+                             gv + j * (long)T, &gw[j], &gu[j], y, q);
+        }
+        free(buf);
     }
 }
