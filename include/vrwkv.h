@@ -9,7 +9,10 @@
  *     (equivalently the RNN form, eq. 6-7);
  *   - the receptance gate sigma(R) (.) wkv, Overall Architecture, eq. 2;
  *   - the channel-mix gate sigma(R_c) (.) SquaredReLU(K_c), Overall
- *     Architecture, eq. 3-4.
+ *     Architecture, eq. 3-4;
+ *   - the Bi-WKV backward pass: the pages state that one exists (in an
+ *     appendix they do not reproduce), so vrwkv_biwkv_bwd computes the plain
+ *     derivatives of eq. 5.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -143,6 +146,38 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
                                 const vrwkv_qshift_params* qs, void* stream);
 
 /*
+ * vrwkv_biwkv_bwd -- gradients of Bi-WKV (eq. 5) for an upstream gradient gy
+ * = dL/dwkv, by the chain rule.  For each (b, c) column, with
+ * W_ti = e^{-(|t-i|-1)/T * w} (i != t), W_tt = e^u, D_t = sum_i W_ti e^{k_i}
+ * and wkv_t the forward output:
+ *   gk_i = e^{k_i} sum_t W_ti gy_t (v_i - wkv_t) / D_t
+ *   gv_i = e^{k_i} sum_t W_ti gy_t / D_t
+ *   gu   = sum_t e^{u + k_t} gy_t (v_t - wkv_t) / D_t
+ *   gw   = -(1/T) sum_t sum_{i != t} (|t-i|-1) W_ti e^{k_i} gy_t (v_i - wkv_t) / D_t
+ * The forward sums are recomputed from k, v, w, u (nothing is saved from the
+ * forward call).
+ *   k, v, gy  (B, T, C) inputs, dtype `dtype`.
+ *   w, u      float32[C].
+ *   gk, gv    (B, T, C) outputs, dtype `dtype` (rounded once for VRWKV_BF16).
+ *   gw, gu    float32[B*C] outputs: row b holds batch element b's share; the
+ *             gradient of the shared w and u is their sum over b.
+ *   gw_total, gu_total  float32[C] or NULL: if given, that sum over b, taken
+ *             in order b = 0..B-1 by a second kernel on the same stream.
+ * Arithmetic is float32; dw and du are summed in a fixed order, so repeated
+ * calls give identical bits.
+ * Limits: T <= 4096 (UNSUPPORTED above, or when the GPU cannot co-schedule
+ *   the thread-block cluster a column needs); the exponent range is that of
+ *   vrwkv_biwkv_fwd.
+ * Errors: INVALID_ARG for B, T or C <= 0, NULL required pointers, misaligned
+ *   pointers, or an output that overlaps an input or another output.
+ */
+vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w,
+                             const float* u, const void* gy, void* gk, void* gv,
+                             float* gw, float* gu, float* gw_total,
+                             float* gu_total, int B, int T, int C,
+                             vrwkv_dtype dtype, void* stream);
+
+/*
  * vrwkv_channel_mix -- the elementwise part of the channel-mix module (eq. 3-4
  * with identity W_R, W_K, W_V and no W_O):
  *   out = sigma(QS_R(x)) (.) SquaredReLU(QS_K(x)),  SquaredReLU(z) = max(z, 0)^2
@@ -175,10 +210,11 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C,
  */
 vrwkv_status vrwkv_device_status(void);
 
-/* Name of the kernel the calling thread's most recent successful
- * vrwkv_biwkv_fwd / vrwkv_spatial_gate / vrwkv_channel_mix call launched
- * ("" before any), e.g. "biwkv_tma_kernel", "biwkv_fused_kernel" or
- * "channel_mix_vec_kernel".  Diagnostics only. */
+/* Name of the main kernel the calling thread's most recent successful
+ * vrwkv_biwkv_fwd / vrwkv_spatial_gate / vrwkv_channel_mix / vrwkv_biwkv_bwd
+ * call launched ("" before any), e.g. "biwkv_tma_kernel",
+ * "biwkv_fused_kernel", "channel_mix_vec_kernel" or "biwkv_bwd_kernel".
+ * Diagnostics only. */
 const char* vrwkv_last_kernel(void);
 
 /* Static, never-NULL name of a status code. */

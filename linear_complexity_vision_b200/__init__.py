@@ -9,6 +9,7 @@ There is no fallback: if the library is missing, the calls raise.
     biwkv_fwd(k, v, w, u, qs=None)
     spatial_gate(r, k, v, w, u, qs=None)
     channel_mix(x, qs=None)
+    biwkv_bwd(k, v, w, u, gy)  # -> gk, gv, gw (B, C), gu (B, C), gw_total, gu_total
     device_status()     # synchronise; raise if a kernel's bounded wait ran out
 
 Token tensors are contiguous (B, T, C) CUDA tensors of dtype float32 or
@@ -66,6 +67,8 @@ def load_library():
         lib.vrwkv_spatial_gate.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                            ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_spatial_gate.restype = ci
+        lib.vrwkv_biwkv_bwd.argtypes = [vp] * 11 + [ci] * 4 + [vp]
+        lib.vrwkv_biwkv_bwd.restype = ci
         lib.vrwkv_channel_mix.argtypes = [vp, vp, ci, ci, ci, ci, ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_channel_mix.restype = ci
         lib.vrwkv_device_status.argtypes = []
@@ -182,6 +185,26 @@ def channel_mix(x, qs: Optional[QShift] = None, out=None):
     _check(load_library().vrwkv_channel_mix(
         x.data_ptr(), out.data_ptr(), B, T, C, _dtype_code(x), qsp, _stream_ptr(x)))
     return out
+
+
+def biwkv_bwd(k, v, w, u, gy, totals: bool = True):
+    """Gradients of eq. 5 for the upstream gradient gy: gk, gv (B, T, C) in
+    the input dtype, gw, gu float32 (B, C) per batch row and, if totals, their
+    sums over the batch (float32 (C,)); otherwise those two are None."""
+    import torch
+    for t, name in ((k, "k"), (v, "v"), (w, "w"), (u, "u"), (gy, "gy")):
+        _require(t, name)
+    B, T, C = k.shape
+    gk, gv = torch.empty_like(k), torch.empty_like(k)
+    gw = torch.empty((B, C), dtype=torch.float32, device=k.device)
+    gu = torch.empty((B, C), dtype=torch.float32, device=k.device)
+    gwt = torch.empty(C, dtype=torch.float32, device=k.device) if totals else None
+    gut = torch.empty(C, dtype=torch.float32, device=k.device) if totals else None
+    _check(load_library().vrwkv_biwkv_bwd(
+        k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), gy.data_ptr(), gk.data_ptr(),
+        gv.data_ptr(), gw.data_ptr(), gu.data_ptr(), None if gwt is None else gwt.data_ptr(),
+        None if gut is None else gut.data_ptr(), B, T, C, _dtype_code(k), _stream_ptr(k)))
+    return gk, gv, gw, gu, gwt, gut
 
 
 def device_status() -> None:

@@ -1,0 +1,557 @@
+// Bi-WKV backward for sm_100a: gradients of eq. 5 ("Vision-RWKV Backbone",
+// Linear Complexity Bidirectional Attention) with respect to k, v, w and u.
+//
+// For one (b, c) column, with p_i = e^{k_i - M}, a = e^{-w/T}, E = e^u and the
+// two-sided decayed sum  S(x)_t = sum_{i != t} a^{|t-i|-1} x_i:
+//
+//   N = S(p v) + E p v,   D = S(p) + E p,   y = N / D        (eq. 5)
+//   q = g / D,   r = q y                                     (g = dL/dy)
+//   dL/dv = p (S(q) + E q)
+//   dL/dk = v dL/dv - p (S(r) + E r)
+//   dL/du = E sum_t p_t (q_t v_t - r_t)
+//   dL/dw = -(1/T) sum_t (q_t H(p v)_t - r_t H(p)_t)
+//
+// where H(x)_t = sum_{i != t} (|t-i|-1) a^{|t-i|-1} x_i is the distance-
+// weighted sum (S differentiated by w, times -T).  The factor e^{-M} cancels
+// from every product, so M can be any common reference; the kernel uses the
+// column maximum of k.
+//
+// S and H are two-sided linear scans.  In each direction a pair (A, H) is
+// carried across a segment of L tokens whose own contribution is (a, h):
+//   A' = a^L A + a,   H' = a^L (H + L A) + h,
+// an associative composition, so both scans run as in the forward kernel:
+// walks over a thread's 4 tokens, shuffle scans over the 4 chunks of a warp,
+// a CTA scan over its 16 warps and an exchange across the CTAs of a cluster.
+// Round 1 scans (p v, p) with their H parts and yields y, q, r and the dw, du
+// terms; round 2 scans (q, r) and yields dk and dv.
+//
+// Work decomposition.  A CTA owns batch row b, a slab of 16 channels and 256
+// tokens; T > 256 splits over a cluster of up to 16 CTAs (T <= 4096).  Thread
+// = 2 adjacent channels (packed float2) x 4 consecutive tokens; the 32 lanes
+// of a warp are 8 channel pairs x 4 consecutive chunks.  Inputs come straight
+// from global memory: at each token step a warp reads four 16-channel rows.
+// Exponents are base 2 (log2 e is folded into k, u and w).
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace vrwkv {
+namespace bwd {
+
+namespace cg = cooperative_groups;
+
+constexpr int kCS = 16;                    // channels per CTA
+constexpr int kNP = kCS / 2;               // channel pairs
+constexpr int kL = 4;                      // tokens per thread
+constexpr int kThreads = 512;
+constexpr int kNW = kThreads / 32;         // 16 warps
+constexpr int kTc = kThreads / kNP * kL;   // 256 tokens per CTA
+constexpr int kWarpTok = 4 * kL;           // 16 tokens per warp
+constexpr int kClusterMax = 16;
+
+struct Params {
+    const char* k;
+    const char* v;
+    const char* g;  // upstream gradient dL/dy
+    const float* w;
+    const float* u;
+    char* gk;
+    char* gv;
+    float* gw;      // (B, C): per batch row
+    float* gu;      // (B, C)
+    int B, T, C;
+    int Tc;         // tokens per CTA (kTc when the column spans several CTAs)
+    int ncl;        // CTAs per column = cluster size
+    int vec;        // channel-pair loads and stores allowed
+    float invT;
+};
+
+// Round-1 record of one channel pair: sums of p v and p with their
+// distance-weighted parts.
+struct R1 {
+    float2 apv, ap, hpv, hp;
+};
+// Round-2 record: sums of q and r.
+struct R2 {
+    float2 aq, ar;
+};
+
+__device__ __forceinline__ R1 r1_zero() { return {f2(0.f), f2(0.f), f2(0.f), f2(0.f)}; }
+__device__ __forceinline__ R2 r2_zero() { return {f2(0.f), f2(0.f)}; }
+
+// Carry `x` across a segment of L tokens (decay aL = a^L) and add the
+// segment's own part `in`.
+__device__ __forceinline__ R1 r1_cross(const R1& x, float2 aL, float L, const R1& in) {
+    R1 o;
+    o.apv = fma2(aL, x.apv, in.apv);
+    o.ap = fma2(aL, x.ap, in.ap);
+    o.hpv = fma2(aL, fma2(f2(L), x.apv, x.hpv), in.hpv);
+    o.hp = fma2(aL, fma2(f2(L), x.ap, x.hp), in.hp);
+    return o;
+}
+__device__ __forceinline__ R2 r2_cross(const R2& x, float2 aL, const R2& in) {
+    return {fma2(aL, x.aq, in.aq), fma2(aL, x.ar, in.ar)};
+}
+__device__ __forceinline__ R1 r1_scale(const R1& x, float2 s) {
+    return {mul2(s, x.apv), mul2(s, x.ap), mul2(s, x.hpv), mul2(s, x.hp)};
+}
+
+__device__ __forceinline__ float2 shfl_up2(float2 v, int d, int width) {
+    return make_float2(__shfl_up_sync(0xffffffffu, v.x, d, width), __shfl_up_sync(0xffffffffu, v.y, d, width));
+}
+__device__ __forceinline__ float2 shfl_down2(float2 v, int d, int width) {
+    return make_float2(__shfl_down_sync(0xffffffffu, v.x, d, width),
+                       __shfl_down_sync(0xffffffffu, v.y, d, width));
+}
+__device__ __forceinline__ R1 shfl_up(const R1& x, int d, int width) {
+    return {shfl_up2(x.apv, d, width), shfl_up2(x.ap, d, width), shfl_up2(x.hpv, d, width),
+            shfl_up2(x.hp, d, width)};
+}
+__device__ __forceinline__ R1 shfl_down(const R1& x, int d, int width) {
+    return {shfl_down2(x.apv, d, width), shfl_down2(x.ap, d, width), shfl_down2(x.hpv, d, width),
+            shfl_down2(x.hp, d, width)};
+}
+__device__ __forceinline__ R2 shfl_up(const R2& x, int d, int width) {
+    return {shfl_up2(x.aq, d, width), shfl_up2(x.ar, d, width)};
+}
+__device__ __forceinline__ R2 shfl_down(const R2& x, int d, int width) {
+    return {shfl_down2(x.aq, d, width), shfl_down2(x.ar, d, width)};
+}
+
+// a^L for both channels of a pair: lam2 = w/T in base-2 units.
+__device__ __forceinline__ float2 decay(float2 lam2, float L) {
+    return ex2c(make_float2(-L * lam2.x, -L * lam2.y));
+}
+
+// Scalar component `hi` (0: .x, 1: .y) of a float2.
+__device__ __forceinline__ float comp(float2 v, int hi) { return hi ? v.y : v.x; }
+__device__ __forceinline__ void set_comp(float2& v, int hi, float x) {
+    if (hi) v.y = x; else v.x = x;
+}
+
+struct alignas(16) Scratch {
+    float2 wmax[kNW][kNP];       // per-warp maxima of k (base 2)
+    // per-warp aggregates and exclusive carries, [pair][warp] with one element
+    // of row padding against bank conflicts
+    R1 w1F[kNP][kNW + 1], w1B[kNP][kNW + 1];
+    R1 c1F[kNP][kNW + 1], c1B[kNP][kNW + 1];
+    R2 w2F[kNP][kNW + 1], w2B[kNP][kNW + 1];
+    R2 c2F[kNP][kNW + 1], c2B[kNP][kNW + 1];
+    float2 wgw[kNW][kNP], wgu[kNW][kNP];  // per-warp dw, du partial sums
+    // this CTA's records, staged for the pushes
+    R1 own1F[kNP], own1B[kNP];
+    float2 ownM[kNP];
+    R2 own2F[kNP], own2B[kNP];
+    float2 ownW[kNP], ownU[kNP];
+    // mailboxes: each peer's records, written by the peers
+    R1 mb1F[kClusterMax][kNP + 1], mb1B[kClusterMax][kNP + 1];
+    float2 mbM[kClusterMax][kNP + 1];
+    R2 mb2F[kClusterMax][kNP + 1], mb2B[kClusterMax][kNP + 1];
+    float2 mbW[kClusterMax][kNP + 1], mbU[kClusterMax][kNP + 1];
+    // carries into this CTA (common exponent Mc) and Mc itself
+    R1 k1F[kNP], k1B[kNP];
+    R2 k2F[kNP], k2B[kNP];
+    float2 kMc[kNP];
+};
+
+template <typename IO>
+__device__ __forceinline__ float2 load_pair(const char* base, size_t row_elem, int cA, int C, bool ok_t,
+                                            bool vec) {
+    constexpr int es = Io<IO>::kBytes;
+    if (!ok_t) return f2(0.0f);
+    const char* p = base + (row_elem + cA) * es;
+    if (vec && cA + 1 < C) return Io<IO>::ld_pair(p);
+    return make_float2(cA < C ? Io<IO>::ld1(p) : 0.0f, cA + 1 < C ? Io<IO>::ld1(p + es) : 0.0f);
+}
+
+template <typename IO>
+__device__ __forceinline__ void store_pair(char* base, size_t row_elem, int cA, int C, bool ok_t, bool vec,
+                                           float2 val) {
+    constexpr int es = Io<IO>::kBytes;
+    if (!ok_t) return;
+    char* p = base + (row_elem + cA) * es;
+    if (vec && cA + 1 < C) {
+        Io<IO>::st_pair(p, val);
+    } else {
+        if (cA < C) Io<IO>::st1(p, val.x);
+        if (cA + 1 < C) Io<IO>::st1(p + es, val.y);
+    }
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) {
+    __shared__ Scratch S;
+
+    const int tid = threadIdx.x;
+    const int j = tid & 7;    // channel pair
+    const int q = tid >> 3;   // chunk within the CTA (0..63)
+    const int cq = q & 3;     // chunk within the warp
+    const int warp = tid >> 5;
+    const int rank = blockIdx.x;
+    const int c0 = blockIdx.y * kCS;
+    const int b = blockIdx.z;
+    const int t0 = rank * p.Tc;
+    const int tend = min(p.T, t0 + p.Tc);
+    const int cA = c0 + 2 * j;
+    const bool vec = p.vec != 0;
+    const bool multi = p.ncl > 1;
+
+    // ---- per-channel constants -----------------------------------------------
+    const float2 wv = make_float2(cA < p.C ? __ldg(p.w + cA) : 0.f, cA + 1 < p.C ? __ldg(p.w + cA + 1) : 0.f);
+    const float2 uv = make_float2(cA < p.C ? __ldg(p.u + cA) : 0.f, cA + 1 < p.C ? __ldg(p.u + cA + 1) : 0.f);
+    const float2 lam2 = mul2(wv, f2(p.invT * kLog2e));  // w/T, base 2
+    const float2 alpha = decay(lam2, 1.0f);
+    const float2 eu = ex2(mul2(uv, f2(kLog2e)));
+
+    // ---- load k, v, g of the thread's 4 tokens -------------------------------
+    const int s_tok = t0 + q * kL;
+    float2 kk[kL], vv[kL], gg[kL];
+    float2 mx = f2(-INFINITY);
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        const int t = s_tok + i;
+        const bool ok = t < tend;
+        const size_t row = ((size_t)b * p.T + t) * p.C;
+        kk[i] = load_pair<IO>(p.k, row, cA, p.C, ok, vec);
+        vv[i] = load_pair<IO>(p.v, row, cA, p.C, ok, vec);
+        gg[i] = load_pair<IO>(p.g, row, cA, p.C, ok, vec);
+        kk[i] = ok ? mul2(kk[i], f2(kLog2e)) : f2(-INFINITY);  // base 2; -inf => p = 0
+        mx = max2(mx, kk[i]);
+    }
+    // CTA maximum of k per channel
+#pragma unroll
+    for (int d = 8; d <= 16; d <<= 1) {
+        mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
+        mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
+    }
+    if (cq == 0) S.wmax[warp][j] = mx;
+    __syncthreads();
+    float2 Mcta = S.wmax[0][j];
+#pragma unroll
+    for (int w = 1; w < kNW; ++w) Mcta = max2(Mcta, S.wmax[w][j]);
+    // a column chunk may hold no token of a padded channel: keep M finite
+    Mcta = make_float2(Mcta.x == -INFINITY ? 0.f : Mcta.x, Mcta.y == -INFINITY ? 0.f : Mcta.y);
+
+    // ---- round 1: p, p v, thread-local sums ------------------------------------
+    float2 pp[kL], pv[kL];
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        pp[i] = ex2(add2(kk[i], make_float2(-Mcta.x, -Mcta.y)));
+        pv[i] = mul2(pp[i], vv[i]);
+    }
+    R1 lf = r1_zero(), lb = r1_zero();
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {  // forward: segment grows to the right
+        lf.hpv = mul2(alpha, add2(lf.hpv, lf.apv));
+        lf.hp = mul2(alpha, add2(lf.hp, lf.ap));
+        lf.apv = fma2(alpha, lf.apv, pv[i]);
+        lf.ap = fma2(alpha, lf.ap, pp[i]);
+    }
+#pragma unroll
+    for (int i = kL - 1; i >= 0; --i) {  // backward: segment grows to the left
+        lb.hpv = mul2(alpha, add2(lb.hpv, lb.apv));
+        lb.hp = mul2(alpha, add2(lb.hp, lb.ap));
+        lb.apv = fma2(alpha, lb.apv, pv[i]);
+        lb.ap = fma2(alpha, lb.ap, pp[i]);
+    }
+    // warp scan over the 4 chunks (lanes 8 apart)
+    R1 fI = lf, bI = lb;
+#pragma unroll
+    for (int d = 1; d < 4; d <<= 1) {
+        const float L = (float)(kL * d);
+        const float2 aL = decay(lam2, L);
+        const R1 o = shfl_up(fI, 8 * d, 32);
+        if (cq >= d) fI = r1_cross(o, aL, L, fI);
+        const R1 o2 = shfl_down(bI, 8 * d, 32);
+        if (cq + d < 4) bI = r1_cross(o2, aL, L, bI);
+    }
+    R1 X1 = shfl_up(fI, 8, 32), Y1 = shfl_down(bI, 8, 32);  // lane-exclusive
+    if (cq == 0) X1 = r1_zero();
+    if (cq == 3) Y1 = r1_zero();
+    if (cq == 3) S.w1F[j][warp] = fI;
+    if (cq == 0) S.w1B[j][warp] = bI;
+    __syncthreads();
+    // CTA scan over the 16 warps: thread (pair jj, warp wi)
+    if (tid < kNP * kNW) {
+        const int jj = tid / kNW, wi = tid % kNW;
+        const float2 wjw = make_float2(c0 + 2 * jj < p.C ? __ldg(p.w + c0 + 2 * jj) : 0.f,
+                                       c0 + 2 * jj + 1 < p.C ? __ldg(p.w + c0 + 2 * jj + 1) : 0.f);
+        const float2 lj = mul2(wjw, f2(p.invT * kLog2e));
+        R1 f = S.w1F[jj][wi], g = S.w1B[jj][wi];
+#pragma unroll
+        for (int d = 1; d < kNW; d <<= 1) {
+            const float L = (float)(kWarpTok * d);
+            const float2 aL = decay(lj, L);
+            const R1 o = shfl_up(f, d, kNW);
+            if (wi >= d) f = r1_cross(o, aL, L, f);
+            const R1 o2 = shfl_down(g, d, kNW);
+            if (wi + d < kNW) g = r1_cross(o2, aL, L, g);
+        }
+        R1 xw = shfl_up(f, 1, kNW), yw = shfl_down(g, 1, kNW);
+        if (wi == 0) xw = r1_zero();
+        if (wi == kNW - 1) yw = r1_zero();
+        S.c1F[jj][wi] = xw;
+        S.c1B[jj][wi] = yw;
+        if (wi == kNW - 1) S.own1F[jj] = f;  // the CTA spans kTc tokens when multi
+        if (wi == 0) {
+            S.own1B[jj] = g;
+            float2 M = S.wmax[0][jj];
+            for (int w = 1; w < kNW; ++w) M = max2(M, S.wmax[w][jj]);
+            S.ownM[jj] = make_float2(M.x == -INFINITY ? 0.f : M.x, M.y == -INFINITY ? 0.f : M.y);
+        }
+    }
+    __syncthreads();
+    // cluster exchange 1: push the records into every peer's mailbox (one
+    // (peer, pair, part) per thread), then one cluster barrier
+    if (multi) {
+        const int peer = tid >> 5, jj = (tid >> 2) & 7, part = tid & 3;
+        if (peer < p.ncl && part < 3) {
+            cg::cluster_group cluster = cg::this_cluster();
+            Scratch* P = cluster.map_shared_rank(&S, peer);
+            if (part == 0) P->mb1F[rank][jj] = S.own1F[jj];
+            else if (part == 1) P->mb1B[rank][jj] = S.own1B[jj];
+            else P->mbM[rank][jj] = S.ownM[jj];
+        }
+        cg::this_cluster().sync();
+    }
+    // carries into this CTA: one thread per (channel, direction), a fixed-order
+    // fold over the peers in the common exponent frame Mc
+    if (tid < 2 * kCS) {
+        const int lc = tid & 15, dir = tid >> 4, jj = lc >> 1, hi = lc & 1;
+        const float lw = (c0 + lc < p.C ? __ldg(p.w + c0 + lc) : 0.f) * (p.invT * kLog2e);
+        float Mc = comp(S.ownM[jj], hi);
+        float kapv = 0.f, kap = 0.f, khpv = 0.f, khp = 0.f;
+        if (multi) {
+            for (int r = 0; r < p.ncl; ++r) Mc = fmaxf(Mc, comp(S.mbM[r][jj], hi));
+            const float aT = ex2c(-(float)p.Tc * lw), LT = (float)p.Tc;
+            const int rs = dir == 0 ? 0 : p.ncl - 1, re = rank, st = dir == 0 ? 1 : -1;
+            for (int r = rs; r != re; r += st) {
+                const R1& m = dir == 0 ? S.mb1F[r][jj] : S.mb1B[r][jj];
+                const float sc = ex2(comp(S.mbM[r][jj], hi) - Mc);
+                khpv = aT * fmaf(LT, kapv, khpv) + sc * comp(m.hpv, hi);
+                khp = aT * fmaf(LT, kap, khp) + sc * comp(m.hp, hi);
+                kapv = fmaf(aT, kapv, sc * comp(m.apv, hi));
+                kap = fmaf(aT, kap, sc * comp(m.ap, hi));
+            }
+        }
+        R1& K = dir == 0 ? S.k1F[jj] : S.k1B[jj];
+        set_comp(K.apv, hi, kapv);
+        set_comp(K.ap, hi, kap);
+        set_comp(K.hpv, hi, khpv);
+        set_comp(K.hp, hi, khp);
+        if (dir == 0) set_comp(S.kMc[jj], hi, Mc);
+    }
+    __syncthreads();
+
+    // ---- round 1: carries into the thread's chunk, then y, q, r ----------------
+    const float2 Mc = S.kMc[j];
+    const float2 sl = ex2(add2(Mcta, make_float2(-Mc.x, -Mc.y)));  // CTA frame -> common frame
+    R1 KF, KB;
+    {
+        const float Lw = (float)(kWarpTok * warp), Ll = (float)(kL * cq);
+        KF = r1_cross(S.k1F[j], decay(lam2, Lw), Lw, r1_scale(S.c1F[j][warp], sl));
+        KF = r1_cross(KF, decay(lam2, Ll), Ll, r1_scale(X1, sl));
+        const float Lw2 = (float)(kWarpTok * (kNW - 1 - warp)), Ll2 = (float)(kL * (3 - cq));
+        KB = r1_cross(S.k1B[j], decay(lam2, Lw2), Lw2, r1_scale(S.c1B[j][warp], sl));
+        KB = r1_cross(KB, decay(lam2, Ll2), Ll2, r1_scale(Y1, sl));
+    }
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {  // p, p v in the common frame
+        pp[i] = mul2(pp[i], sl);
+        pv[i] = mul2(pv[i], sl);
+    }
+    R1 fw[kL];  // forward sums at each token (over tokens before it)
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        fw[i] = KF;
+        KF.hpv = mul2(alpha, add2(KF.hpv, KF.apv));
+        KF.hp = mul2(alpha, add2(KF.hp, KF.ap));
+        KF.apv = fma2(alpha, KF.apv, pv[i]);
+        KF.ap = fma2(alpha, KF.ap, pp[i]);
+    }
+    float2 qq[kL], rr[kL];
+    float2 gwa = f2(0.f), gua = f2(0.f);
+#pragma unroll
+    for (int i = kL - 1; i >= 0; --i) {
+        const float2 N = add2(add2(fw[i].apv, KB.apv), mul2(eu, pv[i]));
+        const float2 D = add2(add2(fw[i].ap, KB.ap), mul2(eu, pp[i]));
+        const float2 HN = add2(fw[i].hpv, KB.hpv);
+        const float2 HD = add2(fw[i].hp, KB.hp);
+        const float2 rD = rcp(D);
+        const float2 y = mul2(N, rD);
+        // Tokens past T (padding of the last CTA) take no part: their forward
+        // sums are real sums carried over up to 255 positions, which can
+        // overflow for w < 0, so they are selected away, not multiplied by 0.
+        const bool real = s_tok + i < tend;
+        qq[i] = real ? mul2(gg[i], rD) : f2(0.f);
+        rr[i] = real ? mul2(qq[i], y) : f2(0.f);
+        if (real) {
+            gwa = add2(gwa, fma2(qq[i], HN, mul2(make_float2(-rr[i].x, -rr[i].y), HD)));
+            gua = fma2(mul2(eu, pp[i]), fma2(qq[i], vv[i], make_float2(-rr[i].x, -rr[i].y)), gua);
+        }
+        KB.hpv = mul2(alpha, add2(KB.hpv, KB.apv));
+        KB.hp = mul2(alpha, add2(KB.hp, KB.ap));
+        KB.apv = fma2(alpha, KB.apv, pv[i]);
+        KB.ap = fma2(alpha, KB.ap, pp[i]);
+    }
+
+    // ---- round 2: sums of q and r ---------------------------------------------
+    R2 mf = r2_zero(), mb = r2_zero();
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        mf.aq = fma2(alpha, mf.aq, qq[i]);
+        mf.ar = fma2(alpha, mf.ar, rr[i]);
+    }
+#pragma unroll
+    for (int i = kL - 1; i >= 0; --i) {
+        mb.aq = fma2(alpha, mb.aq, qq[i]);
+        mb.ar = fma2(alpha, mb.ar, rr[i]);
+    }
+    R2 fJ = mf, bJ = mb;
+#pragma unroll
+    for (int d = 1; d < 4; d <<= 1) {
+        const float2 aL = decay(lam2, (float)(kL * d));
+        const R2 o = shfl_up(fJ, 8 * d, 32);
+        if (cq >= d) fJ = r2_cross(o, aL, fJ);
+        const R2 o2 = shfl_down(bJ, 8 * d, 32);
+        if (cq + d < 4) bJ = r2_cross(o2, aL, bJ);
+    }
+    R2 X2 = shfl_up(fJ, 8, 32), Y2 = shfl_down(bJ, 8, 32);
+    if (cq == 0) X2 = r2_zero();
+    if (cq == 3) Y2 = r2_zero();
+    if (cq == 3) S.w2F[j][warp] = fJ;
+    if (cq == 0) S.w2B[j][warp] = bJ;
+    // dw, du partial sums: over the warp's 4 chunks, then over the warps
+#pragma unroll
+    for (int d = 8; d <= 16; d <<= 1) {
+        gwa = add2(gwa, make_float2(__shfl_xor_sync(0xffffffffu, gwa.x, d), __shfl_xor_sync(0xffffffffu, gwa.y, d)));
+        gua = add2(gua, make_float2(__shfl_xor_sync(0xffffffffu, gua.x, d), __shfl_xor_sync(0xffffffffu, gua.y, d)));
+    }
+    if (cq == 0) {
+        S.wgw[warp][j] = gwa;
+        S.wgu[warp][j] = gua;
+    }
+    __syncthreads();
+    if (tid < kNP * kNW) {
+        const int jj = tid / kNW, wi = tid % kNW;
+        const float2 wjw = make_float2(c0 + 2 * jj < p.C ? __ldg(p.w + c0 + 2 * jj) : 0.f,
+                                       c0 + 2 * jj + 1 < p.C ? __ldg(p.w + c0 + 2 * jj + 1) : 0.f);
+        const float2 lj = mul2(wjw, f2(p.invT * kLog2e));
+        R2 f = S.w2F[jj][wi], g = S.w2B[jj][wi];
+#pragma unroll
+        for (int d = 1; d < kNW; d <<= 1) {
+            const float2 aL = decay(lj, (float)(kWarpTok * d));
+            const R2 o = shfl_up(f, d, kNW);
+            if (wi >= d) f = r2_cross(o, aL, f);
+            const R2 o2 = shfl_down(g, d, kNW);
+            if (wi + d < kNW) g = r2_cross(o2, aL, g);
+        }
+        R2 xw = shfl_up(f, 1, kNW), yw = shfl_down(g, 1, kNW);
+        if (wi == 0) xw = r2_zero();
+        if (wi == kNW - 1) yw = r2_zero();
+        S.c2F[jj][wi] = xw;
+        S.c2B[jj][wi] = yw;
+        if (wi == kNW - 1) S.own2F[jj] = f;
+        if (wi == 0) {
+            S.own2B[jj] = g;
+            float2 sw = S.wgw[0][jj], su = S.wgu[0][jj];
+            for (int w = 1; w < kNW; ++w) {  // fixed order: deterministic
+                sw = add2(sw, S.wgw[w][jj]);
+                su = add2(su, S.wgu[w][jj]);
+            }
+            S.ownW[jj] = sw;
+            S.ownU[jj] = su;
+        }
+    }
+    __syncthreads();
+    if (multi) {
+        const int peer = tid >> 5, jj = (tid >> 2) & 7, part = tid & 3;
+        if (peer < p.ncl) {
+            cg::cluster_group cluster = cg::this_cluster();
+            Scratch* P = cluster.map_shared_rank(&S, peer);
+            if (part == 0) P->mb2F[rank][jj] = S.own2F[jj];
+            else if (part == 1) P->mb2B[rank][jj] = S.own2B[jj];
+            else if (part == 2) P->mbW[rank][jj] = S.ownW[jj];
+            else P->mbU[rank][jj] = S.ownU[jj];
+        }
+        cg::this_cluster().sync();
+    }
+    if (tid < 2 * kCS) {
+        const int lc = tid & 15, dir = tid >> 4, jj = lc >> 1, hi = lc & 1;
+        float kq = 0.f, kr = 0.f;
+        if (multi) {
+            const float lw = (c0 + lc < p.C ? __ldg(p.w + c0 + lc) : 0.f) * (p.invT * kLog2e);
+            const float aT = ex2c(-(float)p.Tc * lw);
+            const int rs = dir == 0 ? 0 : p.ncl - 1, re = rank, st = dir == 0 ? 1 : -1;
+            for (int r = rs; r != re; r += st) {
+                const R2& m = dir == 0 ? S.mb2F[r][jj] : S.mb2B[r][jj];
+                kq = fmaf(aT, kq, comp(m.aq, hi));
+                kr = fmaf(aT, kr, comp(m.ar, hi));
+            }
+        }
+        R2& K = dir == 0 ? S.k2F[jj] : S.k2B[jj];
+        set_comp(K.aq, hi, kq);
+        set_comp(K.ar, hi, kr);
+        // dw, du of the column: rank 0 folds the CTAs' partials in rank order
+        if (rank == 0 && dir == 0 && c0 + lc < p.C) {
+            float sw = comp(S.ownW[jj], hi), su = comp(S.ownU[jj], hi);
+            if (multi) {
+                sw = 0.f;
+                su = 0.f;
+                for (int r = 0; r < p.ncl; ++r) {
+                    sw += comp(S.mbW[r][jj], hi);
+                    su += comp(S.mbU[r][jj], hi);
+                }
+            }
+            p.gw[(size_t)b * p.C + c0 + lc] = -sw * p.invT;
+            p.gu[(size_t)b * p.C + c0 + lc] = su;
+        }
+    }
+    __syncthreads();
+
+    // ---- round 2: carries, then dv and dk ------------------------------------------
+    R2 QF, QB;
+    {
+        const float2 aW = decay(lam2, (float)(kWarpTok * warp)), aLn = decay(lam2, (float)(kL * cq));
+        QF = r2_cross(r2_cross(S.k2F[j], aW, S.c2F[j][warp]), aLn, X2);
+        const float2 aW2 = decay(lam2, (float)(kWarpTok * (kNW - 1 - warp)));
+        const float2 aLn2 = decay(lam2, (float)(kL * (3 - cq)));
+        QB = r2_cross(r2_cross(S.k2B[j], aW2, S.c2B[j][warp]), aLn2, Y2);
+    }
+    R2 fq[kL];
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        fq[i] = QF;
+        QF.aq = fma2(alpha, QF.aq, qq[i]);
+        QF.ar = fma2(alpha, QF.ar, rr[i]);
+    }
+#pragma unroll
+    for (int i = kL - 1; i >= 0; --i) {
+        const float2 Sq = fma2(eu, qq[i], add2(fq[i].aq, QB.aq));
+        const float2 Sr = fma2(eu, rr[i], add2(fq[i].ar, QB.ar));
+        const float2 dv = mul2(pp[i], Sq);
+        const float2 dk = fma2(vv[i], dv, mul2(make_float2(-pp[i].x, -pp[i].y), Sr));
+        const int t = s_tok + i;
+        const size_t row = ((size_t)b * p.T + t) * p.C;
+        store_pair<IO>(p.gv, row, cA, p.C, t < tend, vec, dv);
+        store_pair<IO>(p.gk, row, cA, p.C, t < tend, vec, dk);
+        QB.aq = fma2(alpha, QB.aq, qq[i]);
+        QB.ar = fma2(alpha, QB.ar, rr[i]);
+    }
+    // no closing cluster barrier: the last remote writes precede the second
+    // exchange barrier and no CTA touches another's memory after it
+}
+
+// dw, du of the batch: the per-row parts summed over b in order.
+__global__ void __launch_bounds__(256) batch_sum_kernel(const float* in, float* out, int B, int C) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s += in[(size_t)b * C + c];
+    out[c] = s;
+}
+
+}  // namespace bwd
+}  // namespace vrwkv

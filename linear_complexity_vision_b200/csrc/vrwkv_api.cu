@@ -18,6 +18,7 @@
 #include "biwkv_tma.cuh"
 #include "qshift.cuh"
 #include "channel_mix.cuh"
+#include "biwkv_bwd.cuh"
 
 // Device error word: set by kernels whose bounded waits ran out (bit 0).
 __device__ unsigned int g_vrwkv_device_error;
@@ -626,6 +627,97 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
     else channel_mix_vec_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(p);
     g_last_kernel = "channel_mix_vec_kernel";
     return cuda_status(cudaGetLastError(), "channel_mix kernel launch");
+}
+
+vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const float* u,
+                             const void* gy, void* gk, void* gv, float* gw, float* gu, float* gw_total,
+                             float* gu_total, int B, int T, int C, vrwkv_dtype dtype, void* stream) {
+    if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
+        return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B <= 0 || T <= 0 || C <= 0)
+        return fail(VRWKV_ERR_INVALID_ARG, "B, T and C must be positive (got %d, %d, %d)", B, T, C);
+    if (!k || !v || !w || !u || !gy || !gk || !gv || !gw || !gu)
+        return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
+    if (T > bwd::kTc * bwd::kClusterMax)
+        return fail(VRWKV_ERR_UNSUPPORTED, "T = %d exceeds %d", T, bwd::kTc * bwd::kClusterMax);
+    const int es = elem_bytes(dtype);
+    const void* toks[5] = {k, v, gy, gk, gv};
+    for (const void* t : toks)
+        if (!aligned(t, es)) return fail(VRWKV_ERR_INVALID_ARG, "token tensor misaligned");
+    const float* vecs[6] = {w, u, gw, gu, gw_total, gu_total};
+    for (const float* f : vecs)
+        if (f && !aligned(f, 4)) return fail(VRWKV_ERR_INVALID_ARG, "float32 vector misaligned");
+    const size_t nb = (size_t)B * T * C * es, nbc = (size_t)B * C * 4, nc = (size_t)C * 4;
+    struct Span { const void* p; size_t n; };
+    const Span ins[5] = {{k, nb}, {v, nb}, {gy, nb}, {w, nc}, {u, nc}};
+    const Span outs[6] = {{gk, nb}, {gv, nb}, {gw, nbc}, {gu, nbc}, {gw_total, nc}, {gu_total, nc}};
+    for (int i = 0; i < 6; ++i) {
+        for (const Span& in : ins)
+            if (overlaps(outs[i].p, outs[i].n, in.p, in.n))
+                return fail(VRWKV_ERR_INVALID_ARG, "an output overlaps an input");
+        for (int j2 = i + 1; j2 < 6; ++j2)
+            if (overlaps(outs[i].p, outs[i].n, outs[j2].p, outs[j2].n))
+                return fail(VRWKV_ERR_INVALID_ARG, "outputs overlap");
+    }
+    bwd::Params p;
+    p.k = static_cast<const char*>(k);
+    p.v = static_cast<const char*>(v);
+    p.g = static_cast<const char*>(gy);
+    p.w = w;
+    p.u = u;
+    p.gk = static_cast<char*>(gk);
+    p.gv = static_cast<char*>(gv);
+    p.gw = gw;
+    p.gu = gu;
+    p.B = B;
+    p.T = T;
+    p.C = C;
+    p.Tc = std::min(T, bwd::kTc);
+    p.ncl = (T + p.Tc - 1) / p.Tc;
+    p.invT = (float)(1.0 / (double)T);
+    p.vec = (C % 2 == 0);
+    for (const void* t : toks) p.vec = p.vec && aligned(t, 2 * es);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto kern = dtype == VRWKV_F32 ? bwd::biwkv_bwd_kernel<float> : bwd::biwkv_bwd_kernel<__nv_bfloat16>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.ncl, (C + bwd::kCS - 1) / bwd::kCS, B);
+    cfg.blockDim = dim3(bwd::kThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.ncl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.ncl > 1 ? 1 : 0;
+    if (p.ncl > 1) {
+        static std::atomic<int> nonportable[2] = {{0}, {0}};
+        static std::atomic<int> checked[2][bwd::kClusterMax + 1];
+        const int di = dtype == VRWKV_F32 ? 0 : 1;
+        cudaError_t e;
+        if (p.ncl > 8 && !nonportable[di].load()) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return cuda_status(e, "cluster size attribute");
+            nonportable[di].store(1);
+        }
+        int v2 = checked[di][p.ncl].load();
+        if (v2 == 0) {
+            int n = 0;
+            e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+            v2 = (e == cudaSuccess && n > 0) ? 1 : -1;
+            if (e != cudaSuccess) cudaGetLastError();
+            checked[di][p.ncl].store(v2);
+        }
+        if (v2 < 0)
+            return fail(VRWKV_ERR_UNSUPPORTED, "a cluster of %d backward CTAs cannot be scheduled", p.ncl);
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return cuda_status(e, "biwkv_bwd_kernel launch");
+    g_last_kernel = "biwkv_bwd_kernel";
+    const int blocks = (C + 255) / 256;
+    if (gw_total) bwd::batch_sum_kernel<<<blocks, 256, 0, s>>>(gw, gw_total, B, C);
+    if (gu_total) bwd::batch_sum_kernel<<<blocks, 256, 0, s>>>(gu, gu_total, B, C);
+    return cuda_status(cudaGetLastError(), "batch_sum_kernel launch");
 }
 
 vrwkv_status vrwkv_biwkv_fwd(const void* k, const void* v, const float* w, const float* u, void* wkv,

@@ -77,7 +77,7 @@ def _load():
         lib.oracle_gate.argtypes = [dp, dp, dp, cl]
         lib.oracle_biwkv_bwd_direct.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, dp, dp, dp, dp]
         lib.oracle_biwkv_bwd_columns.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ctypes.c_void_p,
-                                                 ctypes.c_long, dp, dp, dp, dp]
+                                                 ctypes.c_long, dp, dp, dp, dp, dp]
         lib.oracle_channel_mix.argtypes = [dp, dp, dp, dp, ci, ci, ci, ci, ci, cd]
         lib.oracle_spatial_core_points.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, ci,
                                                    ci, ci, cd, ci, ci, i64p, cl, dp]
@@ -248,9 +248,11 @@ def biwkv_bwd(k, v, w, u, gy):
     return gk, gv, gw, gu
 
 
-def biwkv_bwd_columns(k, v, w, u, gy, cols):
+def biwkv_bwd_columns(k, v, w, u, gy, cols, with_scale: bool = False):
     """biwkv_bwd restricted to the flat columns cols[j] = b*C + c: gk, gv of
-    shape (n, T); gw, gu of shape (n,)."""
+    shape (n, T); gw, gu of shape (n,).  With with_scale, also the sums of
+    the absolute values of each gradient's terms: (sk, sv) of shape (n, T)
+    and (sw, su) of shape (n,)."""
     k, v, gy = _d(k), _d(v), _d(gy)
     w, u = _d(w), _d(u)
     B, T, C = k.shape
@@ -258,6 +260,10 @@ def biwkv_bwd_columns(k, v, w, u, gy, cols):
     n = cols.size
     gk, gv = np.empty((n, T)), np.empty((n, T))
     gw, gu = np.empty(n), np.empty(n)
+    sc = np.empty((n, 2 * T + 2)) if with_scale else None
     _load().oracle_biwkv_bwd_columns(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(gy), B, T, C,
-                                     cols.ctypes.data, n, _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu))
+                                     cols.ctypes.data, n, _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu),
+                                     None if sc is None else _ptr(sc))
+    if with_scale:
+        return gk, gv, gw, gu, (sc[:, :T], sc[:, T:2 * T], sc[:, 2 * T], sc[:, 2 * T + 1])
     return gk, gv, gw, gu

@@ -430,7 +430,7 @@ void oracle_channel_mix(const double* x, const double* mu_r,
 static void biwkv_bwd_column(const double* kc, const double* vc,
                              const double* gc, long T, double w, double u,
                              double* gk, double* gv, double* gw, double* gu,
-                             double* y, double* q) {
+                             double* y, double* q, double* scale) {
     double M = kc[0];
     for (long i = 1; i < T; ++i)
         if (kc[i] > M) M = kc[i];
@@ -451,27 +451,40 @@ static void biwkv_bwd_column(const double* kc, const double* vc,
         y[t] = num / den;
         q[t] = gc[t] / den;
     }
-    double sgu = 0.0, sgw = 0.0;
+    double sgu = 0.0, sgw = 0.0, agu = 0.0, agw = 0.0;
     for (long i = 0; i < T; ++i) {
-        double sv = 0.0, sk = 0.0;
+        double sv = 0.0, sk = 0.0, av = 0.0, ak = 0.0;
         for (long t = 0; t < T; ++t) {
             double e;  /* W_ti e^{k_i - M} */
+            const double m = fabs(q[t]) * (fabs(vc[i]) + fabs(y[t]));
             if (t == i) {
                 e = exp(u + kc[i] - M);
                 sgu += e * q[t] * (vc[i] - y[t]);
+                agu += e * m;
             } else {
                 long d = i > t ? i - t : t - i;
                 e = exp(-((double)(d - 1) / (double)T) * w + kc[i] - M);
                 sgw += (double)(d - 1) * e * q[t] * (vc[i] - y[t]);
+                agw += (double)(d - 1) * e * m;
             }
             sv += e * q[t];
             sk += e * q[t] * (vc[i] - y[t]);
+            av += e * fabs(q[t]);
+            ak += e * m;
         }
         gv[i] = sv;
         gk[i] = sk;
+        if (scale) {  /* sums of the absolute values of the terms */
+            scale[i] = ak;
+            scale[T + i] = av;
+        }
     }
     *gu = sgu;
     *gw = -sgw / (double)T;
+    if (scale) {
+        scale[2 * T] = agw / (double)T;
+        scale[2 * T + 1] = agu;
+    }
 }
 
 /* Gradients of every column.  gk, gv: (B, T, C); gw, gu: (B, C), the
@@ -492,7 +505,7 @@ void oracle_biwkv_bwd_direct(const double* k, const double* v, const double* w,
             gather_column(v, vc, b, T, C, c);
             gather_column(gy, gc, b, T, C, c);
             biwkv_bwd_column(kc, vc, gc, T, w[c], u[c], ok, ov, &gw[bc], &gu[bc],
-                             y, q);
+                             y, q, NULL);
             for (long t = 0; t < T; ++t) {
                 gk[(b * T + t) * C + c] = ok[t];
                 gv[(b * T + t) * C + c] = ov[t];
@@ -503,12 +516,15 @@ void oracle_biwkv_bwd_direct(const double* k, const double* v, const double* w,
 }
 
 /* The same for selected columns cols[j] = b*C + c only: gk, gv are (n, T),
- * gw, gu are (n). */
+ * gw, gu are (n).  If scale is not NULL it receives, per column, the sums of
+ * the absolute values of the terms of each gradient (an error scale for
+ * comparisons), laid out as (n, 2T + 2): gk's T, gv's T, then gw, gu. */
 void oracle_biwkv_bwd_columns(const double* k, const double* v,
                               const double* w, const double* u,
                               const double* gy, int B, int T, int C,
                               const int64_t* cols, long n, double* gk,
-                              double* gv, double* gw, double* gu) {
+                              double* gv, double* gw, double* gu,
+                              double* scale) {
     (void)B;
 #pragma omp parallel
     {
@@ -522,7 +538,8 @@ void oracle_biwkv_bwd_columns(const double* k, const double* v,
             gather_column(v, vc, b, T, C, c);
             gather_column(gy, gc, b, T, C, c);
             biwkv_bwd_column(kc, vc, gc, T, w[c], u[c], gk + j * (long)T,
-                             gv + j * (long)T, &gw[j], &gu[j], y, q);
+                             gv + j * (long)T, &gw[j], &gu[j], y, q,
+                             scale ? scale + j * (2 * (long)T + 2) : NULL);
         }
         free(buf);
     }

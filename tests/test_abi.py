@@ -105,3 +105,26 @@ def test_channel_mix_rejects_invalid_arguments(lib, args, frag):
     st = lib.vrwkv_channel_mix(a["x"], a["out"], a["B"], a["T"], a["C"], a["dtype"], qs, None)
     assert st in (1, 2)
     assert frag in lib.vrwkv_last_error().decode()
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(B=0), "positive"),
+    (dict(gy=None), "NULL"),
+    (dict(gw=None), "NULL"),
+    (dict(dtype=9), "dtype"),
+    (dict(T=4097), "exceeds"),
+    (dict(k=FAKE + 1, dtype=1), "misaligned"),
+    (dict(gk=FAKE + 64), "overlaps"),
+    (dict(gw_total=FAKE + (6 << 24) + 4, gu_total=FAKE + (6 << 24)), "overlap"),
+])
+def test_biwkv_bwd_rejects_invalid_arguments(lib, args, frag):
+    a = dict(k=FAKE, v=FAKE + (1 << 24), w=FAKE + (2 << 24), u=FAKE + (3 << 24), gy=FAKE + (4 << 24),
+             gk=FAKE + (5 << 24), gv=FAKE + (5 << 24) + (1 << 22), gw=FAKE + (6 << 24) + (1 << 20),
+             gu=FAKE + (6 << 24) + (2 << 20), gw_total=None, gu_total=None,
+             B=2, T=196, C=32, dtype=0)
+    a.update(args)
+    st = lib.vrwkv_biwkv_bwd(a["k"], a["v"], a["w"], a["u"], a["gy"], a["gk"], a["gv"], a["gw"],
+                             a["gu"], a["gw_total"], a["gu_total"], a["B"], a["T"], a["C"],
+                             a["dtype"], None)
+    assert st in (1, 2)
+    assert frag in lib.vrwkv_last_error().decode()
