@@ -23,8 +23,9 @@ end-to-end figure through the C ABI with host buffers, the float64 CPU
 oracle timed on a bounded sample, and SM clocks sampled during the timed
 region.  ``--impl reference`` times the CPU oracle alone on the same metric.
 ``rows.channel_mix`` adds the roofline of the channel-mix elementwise path
-(eq. 3-4 with identity projections) on the same x buffers, timed in its own
-region after the main one (``--no-rows`` skips it).
+(eq. 3-4 with identity projections) on the same x buffers and
+``rows.biwkv_bwd`` that of the Bi-WKV backward at the workload's shape, each
+timed in its own region after the main one (``--no-rows`` skips them).
 """
 from __future__ import annotations
 
@@ -317,6 +318,51 @@ def time_channel_mix(runner, stream, torch, dev, launches: int, peak: float):
             "launches": reps * G}
 
 
+def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float):
+    """Roofline of the Bi-WKV backward (vrwkv_biwkv_bwd) at the workload's
+    (B, T, C) and dtype, timed in its own region: k, v and gy read once, gk
+    and gv written once, w, u read and the per-row dw, du written."""
+    wl, vk = runner.wl, runner.vk
+    if wl.T > 4096:
+        return None
+    tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    shape = (wl.B, wl.T, wl.C)
+    per_set = 5 * wl.N * (4 if wl.dtype == "f32" else 2)
+    nsets = max(2, int(np.ceil(2 * L2_BYTES / per_set)))
+    g = torch.Generator(device=dev).manual_seed(20260101)
+    sets = []
+    for _ in range(nsets):
+        d = {n: torch.randn(shape, generator=g, device=dev).to(tdt) for n in ("k", "v", "gy")}
+        sets.append(d)
+    w = torch.rand(wl.C, generator=g, device=dev) * 10 - 5
+    u = torch.randn(wl.C, generator=g, device=dev)
+
+    def launch(i):
+        d = sets[i % nsets]
+        vk.biwkv_bwd(d["k"], d["v"], w, u, d["gy"], totals=False)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            launch(i)
+    torch.cuda.synchronize(dev)
+    kname = runner.kernel_name
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(launches):
+            launch(i)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / launches
+    es = 4 if wl.dtype == "f32" else 2
+    nbytes = 5 * wl.N * es + 2 * wl.C * 4 + 2 * wl.B * wl.C * 4
+    achieved = nbytes / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": committed_traffic("biwkv_bwd/" + wl.name),
+            "kernel": kname, "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
+            "launches": launches, "timing": "back-to-back launches (each allocates its outputs)"}
+
+
 def parity_sample(runner, out_dev, oracle, npts=128):
     """Max |GPU - float64 oracle| on a seeded sample of output positions."""
     wl, inp = runner.wl, runner.inp
@@ -479,8 +525,14 @@ def run_ours(args, dist):
     # the next hot-path row on the same buffers (its own timed region)
     if args.rows:
         cm = time_channel_mix(runner, stream, torch, dev, args.row_launches, peak)
+        rows = {}
         if cm is not None:
-            line["rows"] = {"channel_mix": cm}
+            rows["channel_mix"] = cm
+        bw = time_biwkv_bwd(runner, stream, torch, dev, max(20, args.row_launches // 20), peak)
+        if bw is not None:
+            rows["biwkv_bwd"] = bw
+        if rows:
+            line["rows"] = rows
     # correctness guard on the last timed output (first set of the rotation)
     if dist.rank == 0:
         import oracle
@@ -558,7 +610,7 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", dest="rows", action="store_false",
-                    help="skip the channel-mix row measurement")
+                    help="skip the channel-mix and backward row measurements")
     ap.add_argument("--row-launches", type=int, default=4000)
     args = ap.parse_args(argv)
     dist = Dist()
