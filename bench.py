@@ -54,15 +54,23 @@ FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "linear_complexity_vision_b200", "csrc")
 
 
-def kernel_source_hash() -> str:
-    """Hash of every CUDA source of the library (the traffic record is only
-    valid for the exact kernels it was measured on)."""
+# CUDA sources each kernel is compiled from; a traffic record holds only while
+# they are unchanged (a change of launch shape comes with a new capture).
+KERNEL_SOURCES = {
+    "biwkv_tma_kernel": ("common.cuh", "biwkv_tma.cuh"),
+    "biwkv_fused_kernel": ("common.cuh", "qshift.cuh", "biwkv.cuh"),
+    "channel_mix_vec_kernel": ("common.cuh", "qshift.cuh", "channel_mix.cuh"),
+    "biwkv_bwd_kernel": ("common.cuh", "biwkv_bwd.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the CUDA sources `kernel` is built from."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(CSRC, f), "rb") as fh:
-                h.update(f.encode())
-                h.update(fh.read())
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -190,15 +198,15 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def committed_traffic(wl_name: str):
+def committed_traffic(key: str, kernel: str):
     """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources and this workload."""
+    on `kernel` as currently written and on this workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)
-        ent = rec.get(wl_name)
-        if ent and ent.get("kernel_sha") == kernel_source_hash():
+        ent = rec.get(key)
+        if ent and ent.get("kernel") == kernel and ent.get("kernel_sha") == kernel_source_hash(kernel):
             return float(ent["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -312,7 +320,8 @@ def time_channel_mix(runner, stream, torch, dev, launches: int, peak: float):
     nbytes = 2 * wl.N * es + 2 * wl.C * 4  # x once, out once, mu_r and mu_k
     achieved = nbytes / (us * 1e-6) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": committed_traffic("channel_mix/" + wl.name),
+            "frac": achieved / peak,
+            "traffic": committed_traffic("channel_mix/" + wl.name, runner.kernel_name),
             "kernel": runner.kernel_name,
             "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
             "launches": reps * G}
@@ -358,7 +367,7 @@ def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float):
     nbytes = 5 * wl.N * es + 2 * wl.C * 4 + 2 * wl.B * wl.C * 4
     achieved = nbytes / (us * 1e-6) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": committed_traffic("biwkv_bwd/" + wl.name),
+            "frac": achieved / peak, "traffic": committed_traffic("biwkv_bwd/" + wl.name, kname),
             "kernel": kname, "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
             "launches": launches, "timing": "back-to-back launches (each allocates its outputs)"}
 
@@ -476,7 +485,7 @@ def run_ours(args, dist):
         launch_s = (ms_local / 1e3) * fused_share / steps
     peak, peak_kind = measured_hbm_peak()
     achieved = fused_bytes / launch_s / 1e9
-    traffic = committed_traffic(wl.name)
+    traffic = committed_traffic(wl.name, runner.kernel_name)
 
     # end to end through the C ABI with pinned host buffers
     e2e_steps = max(3, min(args.steps, 50))

@@ -83,5 +83,7 @@ def test_algorithmic_bytes():
 def test_kernel_source_hash_is_stable():
     sys.path.insert(0, ROOT)
     import bench
-    assert bench.kernel_source_hash() == bench.kernel_source_hash()
-    assert len(bench.kernel_source_hash()) == 16
+    for kern in bench.KERNEL_SOURCES:
+        assert bench.kernel_source_hash(kern) == bench.kernel_source_hash(kern)
+        assert len(bench.kernel_source_hash(kern)) == 16
+    assert bench.kernel_source_hash("biwkv_tma_kernel") != bench.kernel_source_hash("biwkv_bwd_kernel")
