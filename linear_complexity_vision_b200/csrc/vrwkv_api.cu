@@ -193,13 +193,17 @@ vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_bac
     cfg.blockDim = dim3(NT, 1, 1);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = pl.p.ncl;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // let the hardware balance a cluster's CTAs over the SMs: 33 instead of 31
+    // co-resident 16-CTA clusters on the B200, 3 % faster at T = 4096
+    attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
-    cfg.numAttrs = pl.p.ncl > 1 ? 1 : 0;
+    cfg.numAttrs = pl.p.ncl > 1 ? 2 : 0;
     if (pl.p.ncl > 1) {
         // a cluster shape the GPU cannot co-schedule falls back to the generic kernel
         static std::atomic<int> checked[fast::kClusterMax + 1];
@@ -683,13 +687,15 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
     cfg.gridDim = dim3(p.ncl, (C + bwd::kCS - 1) / bwd::kCS, B);
     cfg.blockDim = dim3(bwd::kThreads, 1, 1);
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = p.ncl;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
-    cfg.numAttrs = p.ncl > 1 ? 1 : 0;
+    cfg.numAttrs = p.ncl > 1 ? 2 : 0;
     if (p.ncl > 1) {
         static std::atomic<int> nonportable[2] = {{0}, {0}};
         static std::atomic<int> checked[2][bwd::kClusterMax + 1];
