@@ -24,8 +24,10 @@ oracle timed on a bounded sample, and SM clocks sampled during the timed
 region.  ``--impl reference`` times the CPU oracle alone on the same metric.
 ``rows.channel_mix`` adds the roofline of the channel-mix elementwise path
 (eq. 3-4 with identity projections) on the same x buffers and
-``rows.biwkv_bwd`` that of the Bi-WKV backward at the workload's shape, each
-timed in its own region after the main one (``--no-rows`` skips them).
+``rows.biwkv_bwd`` that of the Bi-WKV backward at the workload's shape;
+``rows.fused_workspace`` times the main step through the workspace entry
+points (global-memory exchange instead of clusters).  Each is timed in its
+own region after the main one (``--no-rows`` skips them).
 """
 from __future__ import annotations
 
@@ -327,6 +329,58 @@ def time_channel_mix(runner, stream, torch, dev, launches: int, peak: float):
             "launches": reps * G}
 
 
+def time_fused_ws(runner, stream, torch, dev, launches: int, peak: float):
+    """The main step through the workspace entry points (the CTAs of a column
+    exchange their sums through global memory instead of a cluster), graph-
+    replayed over the same rotating buffer sets."""
+    wl, vk = runner.wl, runner.vk
+    if wl.T <= 256:
+        return None
+    ws = vk.fwd_workspace(wl.B, wl.T, wl.C, device=dev)
+    n = runner.nsets
+
+    def launch(i):
+        d, p = runner.sets[i % n], runner.par
+        if wl.call == "biwkv":
+            vk.biwkv_fwd(d["k"], d["v"], p["w"], p["u"], out=d["out"], workspace=ws)
+        elif wl.call == "qshift_biwkv":
+            vk.biwkv_fwd(d["k"], d["v"], p["w"], p["u"], qs=runner.qs, out=d["out"], workspace=ws)
+        elif wl.call == "gate_qs":
+            vk.spatial_gate(d["r"], d["k"], d["v"], p["w"], p["u"], qs=runner.qs, out=d["out"],
+                            workspace=ws)
+        else:
+            x = d["x"]
+            vk.spatial_gate(x, x, x, p["w"], p["u"], qs=runner.qs, out=d["out"], workspace=ws)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            launch(i)
+    torch.cuda.synchronize(dev)
+    G = n * max(1, 64 // n)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            launch(i)
+    reps = max(1, launches // G)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    del graph
+    vk.device_status()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * G)
+    nbytes = algorithmic_bytes(wl)["fused"]
+    achieved = nbytes / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "kernel": runner.kernel_name,
+            "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us, "launches": reps * G,
+            "exchange": "global-memory workspace (no clusters)"}
+
+
 def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float):
     """Roofline of the Bi-WKV backward (vrwkv_biwkv_bwd) at the workload's
     (B, T, C) and dtype, timed in its own region: k, v and gy read once, gk
@@ -537,6 +591,9 @@ def run_ours(args, dist):
         rows = {}
         if cm is not None:
             rows["channel_mix"] = cm
+        gx = time_fused_ws(runner, stream, torch, dev, args.row_launches, peak)
+        if gx is not None:
+            rows["fused_workspace"] = gx
         bw = time_biwkv_bwd(runner, stream, torch, dev, max(20, args.row_launches // 20), peak)
         if bw is not None:
             rows["biwkv_bwd"] = bw

@@ -42,6 +42,8 @@
 #ifndef VRWKV_H
 #define VRWKV_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -146,6 +148,41 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
                                 const vrwkv_qshift_params* qs, void* stream);
 
 /*
+ * Workspace variants of vrwkv_biwkv_fwd and vrwkv_spatial_gate.  Same
+ * operations, arguments, results and limits; for sequences that span several
+ * CTAs the CTAs of one (b, 16-channel) column exchange their partial sums
+ * through the caller's workspace instead of a thread-block cluster, which
+ * frees the kernel from cluster co-scheduling (every SM can hold its full
+ * share of CTAs).
+ *   workspace        device memory of at least vrwkv_fwd_workspace_bytes(B,
+ *                    T, C) bytes, 256-byte aligned, owned by the caller.  It
+ *                    must be zero-filled once before its first use; the
+ *                    kernels leave it ready for the next call (counters reset,
+ *                    a generation number advanced).  Calls that may run at
+ *                    the same time (other streams) need separate workspaces;
+ *                    calls queued on one stream may share one.
+ *   workspace_bytes  its size.
+ * The CTAs of a column wait for one another with a bounded spin (~2 s); a
+ * timeout is recorded in the device error word (see vrwkv_device_status).
+ * Errors: as the plain entry points, plus INVALID_ARG for a NULL, misaligned,
+ *   too small or overlapping workspace.
+ */
+size_t vrwkv_fwd_workspace_bytes(int B, int T, int C);
+
+vrwkv_status vrwkv_biwkv_fwd_ws(const void* k, const void* v, const float* w,
+                                const float* u, void* wkv, int B, int T, int C,
+                                vrwkv_dtype dtype,
+                                const vrwkv_qshift_params* qs, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+vrwkv_status vrwkv_spatial_gate_ws(const void* r, const void* k, const void* v,
+                                   const float* w, const float* u, void* out,
+                                   int B, int T, int C, vrwkv_dtype dtype,
+                                   const vrwkv_qshift_params* qs,
+                                   void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
  * vrwkv_biwkv_bwd -- gradients of Bi-WKV (eq. 5) for an upstream gradient gy
  * = dL/dwkv, by the chain rule.  For each (b, c) column, with
  * W_ti = e^{-(|t-i|-1)/T * w} (i != t), W_tt = e^u, D_t = sum_i W_ti e^{k_i}
@@ -202,11 +239,15 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C,
 /*
  * vrwkv_device_status -- report and clear kernel-side failures on the
  * current device.  Kernels that wait for their asynchronous (TMA) tile
- * copies give up after about two seconds, record the failure in a device
- * error word and finish (their outputs are then undefined) instead of
- * hanging.  This call synchronises with the current device, reads that
+ * copies (bit 0) or, in the workspace variants, for the records of the other
+ * CTAs of a column (bit 1) give up after about two seconds; a workspace
+ * variant that finds its workspace in an invalid state (not zero-filled
+ * before first use; bit 2) stops at once.  Each records the failure in a
+ * device error word and finishes (its outputs are then undefined) instead
+ * of hanging.  This call synchronises with the current device, reads that
  * word, clears it and returns VRWKV_ERR_TIMEOUT if it was set, VRWKV_OK
- * otherwise (VRWKV_ERR_CUDA if the device cannot be read).
+ * otherwise (VRWKV_ERR_CUDA if the device cannot be read); the bits are in
+ * vrwkv_last_error().
  */
 vrwkv_status vrwkv_device_status(void);
 

@@ -6,8 +6,9 @@ CUDA kernels.  PyTorch provides device memory and the current stream only.
 There is no fallback: if the library is missing, the calls raise.
 
     qshift(x, H, W, shift_pixel=1, gamma=0.25, mu=None)
-    biwkv_fwd(k, v, w, u, qs=None)
-    spatial_gate(r, k, v, w, u, qs=None)
+    biwkv_fwd(k, v, w, u, qs=None, workspace=None)
+    spatial_gate(r, k, v, w, u, qs=None, workspace=None)
+    fwd_workspace(B, T, C, device)  # a zeroed workspace for the two calls above
     channel_mix(x, qs=None)
     biwkv_bwd(k, v, w, u, gy)  # -> gk, gv, gw (B, C), gu (B, C), gw_total, gu_total
     device_status()     # synchronise; raise if a kernel's bounded wait ran out
@@ -67,6 +68,14 @@ def load_library():
         lib.vrwkv_spatial_gate.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                            ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_spatial_gate.restype = ci
+        lib.vrwkv_fwd_workspace_bytes.argtypes = [ci, ci, ci]
+        lib.vrwkv_fwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.vrwkv_biwkv_fwd_ws.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                           ctypes.POINTER(_QsParams), vp, ctypes.c_size_t, vp]
+        lib.vrwkv_biwkv_fwd_ws.restype = ci
+        lib.vrwkv_spatial_gate_ws.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                              ctypes.POINTER(_QsParams), vp, ctypes.c_size_t, vp]
+        lib.vrwkv_spatial_gate_ws.restype = ci
         lib.vrwkv_biwkv_bwd.argtypes = [vp] * 11 + [ci] * 4 + [vp]
         lib.vrwkv_biwkv_bwd.restype = ci
         lib.vrwkv_channel_mix.argtypes = [vp, vp, ci, ci, ci, ci, ctypes.POINTER(_QsParams), vp]
@@ -143,8 +152,22 @@ def qshift(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25, mu=None
     return out
 
 
-def biwkv_fwd(k, v, w, u, qs: Optional[QShift] = None, out=None):
-    """Bi-WKV forward of eq. 5 on (B, T, C) tensors; Q-Shift on load if qs."""
+def fwd_workspace_bytes(B: int, T: int, C: int) -> int:
+    """Bytes of workspace the *_ws forward entry points need."""
+    return int(load_library().vrwkv_fwd_workspace_bytes(B, T, C))
+
+
+def fwd_workspace(B: int, T: int, C: int, device="cuda"):
+    """A zero-filled uint8 CUDA tensor usable as the forward workspace of
+    (B, T, C) problems (and smaller ones) on one stream at a time."""
+    import torch
+    return torch.zeros(fwd_workspace_bytes(B, T, C), dtype=torch.uint8, device=device)
+
+
+def biwkv_fwd(k, v, w, u, qs: Optional[QShift] = None, out=None, workspace=None):
+    """Bi-WKV forward of eq. 5 on (B, T, C) tensors; Q-Shift on load if qs.
+    With a workspace (see fwd_workspace) the CTAs of long sequences exchange
+    their sums through it instead of a thread-block cluster."""
     import torch
     for t, name in ((k, "k"), (v, "v"), (w, "w"), (u, "u")):
         _require(t, name)
@@ -152,14 +175,23 @@ def biwkv_fwd(k, v, w, u, qs: Optional[QShift] = None, out=None):
     if out is None:
         out = torch.empty_like(k)
     qsp = ctypes.byref(qs._struct()) if qs is not None else None
-    _check(load_library().vrwkv_biwkv_fwd(
-        k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(), B, T, C,
-        _dtype_code(k), qsp, _stream_ptr(k)))
+    lib = load_library()
+    if workspace is None:
+        _check(lib.vrwkv_biwkv_fwd(
+            k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(), B, T, C,
+            _dtype_code(k), qsp, _stream_ptr(k)))
+    else:
+        _require(workspace, "workspace")
+        _check(lib.vrwkv_biwkv_fwd_ws(
+            k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(), B, T, C,
+            _dtype_code(k), qsp, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+            _stream_ptr(k)))
     return out
 
 
-def spatial_gate(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
-    """sigma(QS_R(r)) * Bi-WKV(QS_K(k), QS_V(v)); r, k, v may be one tensor."""
+def spatial_gate(r, k, v, w, u, qs: Optional[QShift] = None, out=None, workspace=None):
+    """sigma(QS_R(r)) * Bi-WKV(QS_K(k), QS_V(v)); r, k, v may be one tensor.
+    workspace: as for biwkv_fwd."""
     import torch
     for t, name in ((r, "r"), (k, "k"), (v, "v"), (w, "w"), (u, "u")):
         _require(t, name)
@@ -167,9 +199,17 @@ def spatial_gate(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
     if out is None:
         out = torch.empty_like(k)
     qsp = ctypes.byref(qs._struct()) if qs is not None else None
-    _check(load_library().vrwkv_spatial_gate(
-        r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
-        B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
+    lib = load_library()
+    if workspace is None:
+        _check(lib.vrwkv_spatial_gate(
+            r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
+            B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
+    else:
+        _require(workspace, "workspace")
+        _check(lib.vrwkv_spatial_gate_ws(
+            r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
+            B, T, C, _dtype_code(k), qsp, workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), _stream_ptr(k)))
     return out
 
 

@@ -81,7 +81,26 @@ struct alignas(64) Params {
     int ncl;             // CTAs per column (cluster size)
     int tile_bytes;      // bytes per tile: 8 sub-tiles of 32 token rows
     int box_bytes;       // bytes one strided box delivers (zero fill included)
+    // global-memory exchange (GX kernels only): see the workspace layout below
+    unsigned int* ws_ctl;   // [0] ticket counter, [1] finished CTAs, [2] generation
+    unsigned int* ws_flag;  // per (column, rank): generation + 1 once its record is out
+    float4* ws_rec;         // per (column, rank): kRecF4 float4 record
+    int nslab;           // channel slabs (C / 16)
+    int total;           // CTAs in the grid
 };
+
+// Global-memory exchange.  Without clusters, the CTAs of one column find
+// each other through a workspace: every CTA takes a ticket from a counter,
+// tickets map column by column onto (rank, slab, b), so the <= 16 CTAs of a
+// column hold consecutive tickets; a CTA publishes its aggregates (a record
+// and a flag tagged with the launch's generation) and waits, with a bounded
+// spin, for the flags of its column's peers.  Tickets are taken in start
+// order, so the peers a CTA waits for have either started or start as soon
+// as any CTA of an earlier, complete column exits: waiting can only stall a
+// column that has not been fully started, and a GPU that holds 16 CTAs at once
+// always starts it.  The last CTA to finish resets the counters and advances
+// the generation, so stale flags of earlier launches never match.
+constexpr int kRecF4 = 20;  // float4 per record: F[8], G[8], M[8] (two pairs per float4)
 
 template <int NT>
 struct alignas(16) Scratch {
@@ -103,6 +122,8 @@ struct alignas(16) Scratch {
     float2 ownM[kNP];           // this CTA's max of k (times log2 e)
     float2 gpark[Cfg<NT>::kTcMax][kNP];  // gate factors, parked between load and output
     float4 cscale[kCS];         // per channel: sl (scale of this CTA's own sums)
+    int tk;                     // GX: this CTA's ticket
+    unsigned int gen;           // GX: the launch's generation
     float4 ccarry[kCS];         // per channel: carries Af, Cf, Bb, Db
     unsigned long long bar;     // TMA completion barrier
 };
@@ -199,7 +220,27 @@ __device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); 
 __device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); }
 __device__ __forceinline__ float4 zero4() { return make_float4(0.f, 0.f, 0.f, 0.f); }
 
-template <typename IO, int LAYOUT, bool QS, int NT>
+// Bounded wait for a peer's flag (acquire); records a timeout in the device
+// error word (bit 1) and gives up instead of hanging.
+__device__ __forceinline__ void wait_flag(const unsigned int* f, unsigned int want, unsigned int* err) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    if (v == want) return;
+    const long long t0 = clock64();
+    unsigned int ns = 32;
+    for (;;) {
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+        if (v == want) return;
+        if (clock64() - t0 > kWaitCycles) {
+            atomicOr(err, 2u);
+            return;
+        }
+    }
+}
+
+template <typename IO, int LAYOUT, bool QS, int NT, bool GX>
 __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(const __grid_constant__ Params p) {
     constexpr int kThreads = Cfg<NT>::kThreads;
     constexpr int kNW = Cfg<NT>::kNW;
@@ -226,24 +267,41 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     const int q = tid >> 3;      // chunk within the CTA
     const int cq = q & 3;        // chunk within the warp
     const int warp = tid >> 5;
-    const int rank = blockIdx.x;
-    const int c0 = blockIdx.y * kCS;
-    const int b = blockIdx.z;
+    if (tid == 0) {
+        mbar_init(&S.bar, 1);
+        if (GX) {
+            S.tk = (int)atomicAdd(p.ws_ctl, 1u);
+            S.gen = *reinterpret_cast<volatile unsigned int*>(p.ws_ctl + 2);
+        }
+    }
+    __syncthreads();
+    // this CTA's column chunk: the block index, or (GX) the ticket
+    int rank = blockIdx.x, slab = blockIdx.y, b = blockIdx.z;
+    unsigned int gen = 0;
+    if (GX) {
+        const int t = S.tk;
+        if (t < 0 || t >= p.total) {  // a workspace that was not zero-filled
+            if (tid == 0) atomicOr(p.err, 4u);
+            return;
+        }
+        gen = S.gen;
+        rank = t % p.ncl;
+        slab = (t / p.ncl) % p.nslab;
+        b = t / p.ncl / p.nslab;
+    }
+    const int col = b * p.nslab + slab;  // GX: the column's records and flags
+    const int c0 = slab * kCS;
     const int t0 = rank * p.Tc;
     const int tend = min(p.T, t0 + p.Tc);
 
     // group of this CTA's channels (Q-Shift): 0..3 shifted, 4 copied
     int grp = 4;
-    if (QS && p.gslab > 0) {
-        const int y = blockIdx.y;
-        grp = (y >= p.gslab) + (y >= 2 * p.gslab) + (y >= 3 * p.gslab) + (y >= 4 * p.gslab);
-    }
+    if (QS && p.gslab > 0)
+        grp = (slab >= p.gslab) + (slab >= 2 * p.gslab) + (slab >= 3 * p.gslab) + (slab >= 4 * p.gslab);
     const bool shifted = QS && grp < 4;
 
     // ---- issue the tile loads: lane i of warp 0 loads sub-tile i of each tile
     constexpr int SUB = kTcMax / kL * RB;  // bytes per sub-tile (kTcMax / 8 token rows)
-    if (tid == 0) mbar_init(&S.bar, 1);
-    __syncthreads();
     if (warp == 0) {
         if (tid == 0) {
             mbar_expect_tx(&S.bar, (unsigned)p.box_bytes * (unsigned)(kL * NSRC * (shifted ? 2 : 1)));
@@ -450,22 +508,62 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
             for (int e = 0; e < 4; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
         }
         __syncthreads();
-        // publish the record into every CTA's mailbox (its own included) with
-        // remote shared-memory stores, one (peer, pair, half) per thread; the
-        // cluster barrier below makes them visible
-        const int peer = tid >> 4, jj = (tid >> 1) & 7;
-        if (peer < p.ncl) {
-            cg::cluster_group cluster = cg::this_cluster();
-            Scratch* P = cluster.map_shared_rank(&S, peer);
-            if ((tid & 1) == 0) {
-                P->mbF[rank][jj] = S.ownF[jj];
-            } else {
-                P->mbG[rank][jj] = S.ownG[jj];
-                P->mbM[rank][jj] = S.ownM[jj];
+        if (GX) {
+            // publish the record to the workspace, then the flag (release
+            // after every writer's fence), then wait for the column's flags
+            // and copy the records into the mailbox
+            float4* rec = p.ws_rec + ((size_t)col * kClusterMax + rank) * kRecF4;
+            if (tid < kRecF4) {
+                float4 v;
+                if (tid < kNP) {
+                    v = S.ownF[tid];
+                } else if (tid < 2 * kNP) {
+                    v = S.ownG[tid - kNP];
+                } else {
+                    const int m = 2 * (tid - 2 * kNP);
+                    v = make_float4(S.ownM[m].x, S.ownM[m].y, S.ownM[m + 1].x, S.ownM[m + 1].y);
+                }
+                __stcg(rec + tid, v);
+                __threadfence();
+            }
+            __syncthreads();
+            unsigned int* flags = p.ws_flag + (size_t)col * kClusterMax;
+            if (tid == 0)
+                asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flags + rank), "r"(gen + 1u) : "memory");
+            if (tid < p.ncl) wait_flag(flags + tid, gen + 1u, p.err);
+            __syncthreads();
+            const float4* peers = p.ws_rec + (size_t)col * kClusterMax * kRecF4;
+            for (int e = tid; e < p.ncl * kRecF4; e += kThreads) {
+                const int r = e / kRecF4, k = e - r * kRecF4;
+                const float4 v = __ldcg(peers + e);
+                if (k < kNP) {
+                    S.mbF[r][k] = v;
+                } else if (k < 2 * kNP) {
+                    S.mbG[r][k - kNP] = v;
+                } else {
+                    const int m = 2 * (k - 2 * kNP);
+                    S.mbM[r][m] = make_float2(v.x, v.y);
+                    S.mbM[r][m + 1] = make_float2(v.z, v.w);
+                }
+            }
+        } else {
+            // publish the record into every CTA's mailbox (its own included)
+            // with remote shared-memory stores, one (peer, pair, half) per
+            // thread; the cluster barrier below makes them visible
+            const int peer = tid >> 4, jj = (tid >> 1) & 7;
+            if (peer < p.ncl) {
+                cg::cluster_group cluster = cg::this_cluster();
+                Scratch* P = cluster.map_shared_rank(&S, peer);
+                if ((tid & 1) == 0) {
+                    P->mbF[rank][jj] = S.ownF[jj];
+                } else {
+                    P->mbG[rank][jj] = S.ownG[jj];
+                    P->mbM[rank][jj] = S.ownM[jj];
+                }
             }
         }
     }
-    if (p.ncl > 1) {
+    if (p.ncl > 1 && !GX) {
         cluster_arrive_release();
         cluster_wait_acquire();
     } else {
@@ -577,6 +675,20 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     }
     // no closing cluster barrier: peers wrote into this CTA's mailbox before
     // the exchange barrier and nobody reads another CTA's memory after it
+    if (GX) {
+        // count the CTA out; the last one resets the counters for the next
+        // launch and advances the generation
+        if (tid == 0) {
+            __threadfence();
+            const unsigned int d = atomicAdd(p.ws_ctl + 1, 1u);
+            if (d == (unsigned int)p.total - 1u) {
+                atomicExch(p.ws_ctl + 0, 0u);
+                atomicExch(p.ws_ctl + 1, 0u);
+                __threadfence();
+                atomicExch(p.ws_ctl + 2, gen + 1u);
+            }
+        }
+    }
 }
 
 }  // namespace fast

@@ -167,18 +167,45 @@ struct FastPlan {
     fast::Params p;
     int layout;
     bool qs;
-    int nt;  // threads (= tokens) per CTA
+    bool gx;  // exchange through the caller's workspace instead of a cluster
+    int nt;   // threads (= tokens) per CTA
     dim3 grid;
     int smem;
 };
 
-template <typename IO, int LAYOUT, bool QS, int NT>
+// Workspace of the global-exchange path: 16 bytes of counters, then a flag
+// per (column, rank), then a record per (column, rank); a column is one
+// (batch row, 16-channel slab).
+struct WsLayout {
+    size_t flags_off, recs_off, bytes;
+};
+WsLayout ws_layout(int B, int C) {
+    const size_t cols = (size_t)B * (size_t)((C + fast::kCS - 1) / fast::kCS);
+    WsLayout L;
+    L.flags_off = 16;
+    L.recs_off = (L.flags_off + cols * fast::kClusterMax * sizeof(unsigned int) + 255) / 256 * 256;
+    L.bytes = L.recs_off + cols * fast::kClusterMax * fast::kRecF4 * sizeof(float4);
+    return L;
+}
+
+template <typename IO, int LAYOUT, bool QS, int NT, bool GX>
 vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
-    auto kern = fast::biwkv_tma_kernel<IO, LAYOUT, QS, NT>;
+    auto kern = fast::biwkv_tma_kernel<IO, LAYOUT, QS, NT, GX>;
     static std::atomic<int> granted{0};
     static std::atomic<int> nonportable{0};
     cudaError_t e = ensure_smem(kern, granted, pl.smem);
     if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    if (GX) {  // a plain 1-D grid: the CTAs of a column meet through the workspace
+        cudaLaunchConfig_t gcfg = {};
+        gcfg.gridDim = pl.grid;
+        gcfg.blockDim = dim3(NT, 1, 1);
+        gcfg.dynamicSmemBytes = pl.smem;
+        gcfg.stream = stream;
+        e = cudaLaunchKernelEx(&gcfg, kern, pl.p);
+        if (e != cudaSuccess) return cuda_status(e, "biwkv_tma_kernel launch");
+        g_last_kernel = "biwkv_tma_kernel";
+        return ok();
+    }
     if (pl.p.ncl > 8 && !nonportable.load()) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) {
@@ -226,15 +253,15 @@ vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_bac
     return ok();
 }
 
-template <typename IO, int NT>
+template <typename IO, int NT, bool GX>
 vrwkv_status dispatch_fast_nt(const FastPlan& pl, cudaStream_t s, bool* fb) {
     switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
-    case fast::kKV * 2 + 0: return launch_fast<IO, fast::kKV, false, NT>(pl, s, fb);
-    case fast::kKV * 2 + 1: return launch_fast<IO, fast::kKV, true, NT>(pl, s, fb);
-    case fast::kRKV * 2 + 0: return launch_fast<IO, fast::kRKV, false, NT>(pl, s, fb);
-    case fast::kRKV * 2 + 1: return launch_fast<IO, fast::kRKV, true, NT>(pl, s, fb);
-    case fast::kX * 2 + 0: return launch_fast<IO, fast::kX, false, NT>(pl, s, fb);
-    default: return launch_fast<IO, fast::kX, true, NT>(pl, s, fb);
+    case fast::kKV * 2 + 0: return launch_fast<IO, fast::kKV, false, NT, GX>(pl, s, fb);
+    case fast::kKV * 2 + 1: return launch_fast<IO, fast::kKV, true, NT, GX>(pl, s, fb);
+    case fast::kRKV * 2 + 0: return launch_fast<IO, fast::kRKV, false, NT, GX>(pl, s, fb);
+    case fast::kRKV * 2 + 1: return launch_fast<IO, fast::kRKV, true, NT, GX>(pl, s, fb);
+    case fast::kX * 2 + 0: return launch_fast<IO, fast::kX, false, NT, GX>(pl, s, fb);
+    default: return launch_fast<IO, fast::kX, true, NT, GX>(pl, s, fb);
     }
 }
 
@@ -245,7 +272,8 @@ constexpr int kFastThreads = 256;
 
 template <typename IO>
 vrwkv_status dispatch_fast(const FastPlan& pl, cudaStream_t s, bool* fb) {
-    return dispatch_fast_nt<IO, kFastThreads>(pl, s, fb);
+    return pl.gx ? dispatch_fast_nt<IO, kFastThreads, true>(pl, s, fb)
+                 : dispatch_fast_nt<IO, kFastThreads, false>(pl, s, fb);
 }
 
 // Shared memory of a fast-path CTA: the tiles plus the scratch block.
@@ -257,7 +285,7 @@ int fast_smem(int ntiles, int tile_bytes) {
 // (the generic kernel then runs).
 bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void* v, const float* w,
                const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
-               const vrwkv_qshift_params* qs) {
+               const vrwkv_qshift_params* qs, void* ws) {
     if (tma_disabled()) return false;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
@@ -369,6 +397,20 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     p.mu[2] = qs ? qs->mu_v : nullptr;
     p.out = static_cast<char*>(out);
     pl.grid = dim3(p.ncl, C / fast::kCS, B);
+    p.nslab = C / fast::kCS;
+    p.total = p.ncl * p.nslab * B;
+    pl.gx = ws != nullptr && p.ncl > 1;
+    if (pl.gx) {
+        const WsLayout L = ws_layout(B, C);
+        char* base = static_cast<char*>(ws);
+        p.ws_ctl = reinterpret_cast<unsigned int*>(base);
+        p.ws_flag = reinterpret_cast<unsigned int*>(base + L.flags_off);
+        p.ws_rec = reinterpret_cast<float4*>(base + L.recs_off);
+        pl.grid = dim3((unsigned)p.total, 1, 1);
+    } else {
+        p.ws_ctl = p.ws_flag = nullptr;
+        p.ws_rec = nullptr;
+    }
     return true;
 }
 
@@ -390,7 +432,8 @@ vrwkv_status check_qs(const vrwkv_qshift_params* qs, int T, int C) {
 // Shared front end of vrwkv_biwkv_fwd (gate = false) and vrwkv_spatial_gate.
 vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v, const float* w,
                          const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
-                         const vrwkv_qshift_params* qs, void* stream) {
+                         const vrwkv_qshift_params* qs, void* stream, bool with_ws = false,
+                         void* ws = nullptr, size_t ws_bytes = 0) {
     if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
         return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     if (B <= 0 || T <= 0 || C <= 0)
@@ -419,9 +462,20 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
                 return fail(VRWKV_ERR_INVALID_ARG, "output overlaps a mu vector");
     }
 
+    if (with_ws) {
+        if (!ws) return fail(VRWKV_ERR_INVALID_ARG, "workspace is NULL");
+        if (!aligned(ws, 256)) return fail(VRWKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+        const size_t need = ws_layout(B, C).bytes;
+        if (ws_bytes < need)
+            return fail(VRWKV_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes,
+                        need);
+        for (const void* t : toks)
+            if (overlaps(ws, need, t, nbytes)) return fail(VRWKV_ERR_INVALID_ARG, "workspace overlaps an input");
+        if (overlaps(ws, need, out, nbytes)) return fail(VRWKV_ERR_INVALID_ARG, "workspace overlaps the output");
+    }
     if (B <= 65535 && C / vrwkv::fast::kCS <= 65535) {
         FastPlan fp;
-        if (plan_fast(fp, gate, r, k, v, w, u, out, B, T, C, dtype, qs)) {
+        if (plan_fast(fp, gate, r, k, v, w, u, out, B, T, C, dtype, qs, with_ws ? ws : nullptr)) {
             bool fell_back = false;
             cudaStream_t fs = static_cast<cudaStream_t>(stream);
             vrwkv_status st = dtype == VRWKV_F32 ? dispatch_fast<float>(fp, fs, &fell_back)
@@ -738,6 +792,27 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v, con
     return fused_entry(true, r, k, v, w, u, out, B, T, C, dtype, qs, stream);
 }
 
+size_t vrwkv_fwd_workspace_bytes(int B, int T, int C) {
+    (void)T;
+    if (B <= 0 || C <= 0) return 0;
+    return ws_layout(B, C).bytes;
+}
+
+vrwkv_status vrwkv_biwkv_fwd_ws(const void* k, const void* v, const float* w, const float* u, void* wkv,
+                                int B, int T, int C, vrwkv_dtype dtype, const vrwkv_qshift_params* qs,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    return fused_entry(false, nullptr, k, v, w, u, wkv, B, T, C, dtype, qs, stream, true, workspace,
+                       workspace_bytes);
+}
+
+vrwkv_status vrwkv_spatial_gate_ws(const void* r, const void* k, const void* v, const float* w,
+                                   const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
+                                   const vrwkv_qshift_params* qs, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+    return fused_entry(true, r, k, v, w, u, out, B, T, C, dtype, qs, stream, true, workspace,
+                       workspace_bytes);
+}
+
 const char* vrwkv_status_string(vrwkv_status status) {
     switch (status) {
     case VRWKV_OK: return "VRWKV_OK";
@@ -763,7 +838,10 @@ vrwkv_status vrwkv_device_status(void) {
     const unsigned int zero = 0;
     e = cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_status(e, "clearing the device error word");
-    return fail(VRWKV_ERR_TIMEOUT, "a kernel's bounded wait for its TMA tiles ran out (flags 0x%x)", v);
+    return fail(VRWKV_ERR_TIMEOUT,
+                "kernel-side failure (flags 0x%x: 1 = TMA tile wait ran out, 2 = wait for a column "
+                "peer's record ran out, 4 = workspace not zero-filled)",
+                v);
 }
 
 }  // extern "C"

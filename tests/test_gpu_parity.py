@@ -93,6 +93,19 @@ def _custom(call, B, H, W, C, dt, seed, s=1, gamma=0.25, **d):
                           shift_pixel=s, gamma=gamma, seed=seed)
 
 
+# Workspace of the global-exchange kernels, shared by every "gx" test on the
+# one stream (the kernels leave it ready for the next call).
+_GX = {"on": False, "ws": None}
+
+
+def _workspace(vk, B, T, C):
+    need = vk.fwd_workspace_bytes(B, T, C)
+    if _GX["ws"] is None or _GX["ws"].numel() < need:
+        import torch
+        _GX["ws"] = torch.zeros(max(need, 64 << 20), dtype=torch.uint8, device="cuda")
+    return _GX["ws"]
+
+
 def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     """Run the workload's call on the GPU and compare with the oracle."""
     inp = wl.generate()
@@ -111,20 +124,22 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     H, W, s, g = wl.H, wl.W, wl.shift_pixel, wl.gamma
     w, u = ref["w"], ref["u"]
 
+    ws = _workspace(vk, wl.B, wl.T, wl.C) if _GX["on"] else None
     if wl.call == "biwkv":
-        out = vk.biwkv_fwd(dev["k"], dev["v"], dev["w"], dev["u"])
+        out = vk.biwkv_fwd(dev["k"], dev["v"], dev["w"], dev["u"], workspace=ws)
         ks, vs, rs = ref["k"], ref["v"], None
     else:
         qs = vk.QShift(H, W, s, g, dev.get("mu_r"), dev.get("mu_k"), dev.get("mu_v"))
         if wl.call == "qshift_biwkv":
-            out = vk.biwkv_fwd(dev["k"], dev["v"], dev["w"], dev["u"], qs=qs)
+            out = vk.biwkv_fwd(dev["k"], dev["v"], dev["w"], dev["u"], qs=qs, workspace=ws)
             kin, vin, rin = ref["k"], ref["v"], None
         elif wl.call == "gate_qs":
-            out = vk.spatial_gate(dev["r"], dev["k"], dev["v"], dev["w"], dev["u"], qs=qs)
+            out = vk.spatial_gate(dev["r"], dev["k"], dev["v"], dev["w"], dev["u"], qs=qs,
+                                  workspace=ws)
             kin, vin, rin = ref["k"], ref["v"], ref["r"]
         else:  # gate_qs_x: one x feeds r, k and v
             x = dev["x"]
-            out = vk.spatial_gate(x, x, x, dev["w"], dev["u"], qs=qs)
+            out = vk.spatial_gate(x, x, x, dev["w"], dev["u"], qs=qs, workspace=ws)
             kin = vin = rin = ref["x"]
         ks = oracle.qshift(kin, H, W, s, g, ref["mu_k"])
         vs = oracle.qshift(vin, H, W, s, g, ref["mu_v"])
@@ -154,15 +169,18 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     return (got, err) if return_out else err
 
 
-@pytest.fixture(params=["tma", "generic"])
+@pytest.fixture(params=["tma", "gx", "generic"])
 def kernel_path(request, monkeypatch):
-    """Run a test on the TMA fast path (when the shape qualifies) and again
-    with the generic kernel forced."""
+    """Run a test on the TMA fast path (when the shape qualifies), on its
+    workspace variant (global-memory exchange instead of clusters) and with
+    the generic kernel forced."""
     if request.param == "generic":
         monkeypatch.setenv("VRWKV_DISABLE_TMA", "1")
     else:
         monkeypatch.delenv("VRWKV_DISABLE_TMA", raising=False)
-    return request.param
+    _GX["on"] = request.param == "gx"
+    yield request.param
+    _GX["on"] = False
 
 
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
@@ -306,3 +324,40 @@ def test_invalid_arguments_raise(vk):
         vk.biwkv_fwd(x, x, w, w, qs=vk.QShift(3, 5))
     with pytest.raises(vk.VrwkvError, match="overlaps"):
         vk.biwkv_fwd(x, x, w, w, out=x)
+
+
+def test_workspace_reuse_across_launches(vk, oracle_mod):
+    # the global-exchange kernel resets its counters and advances a
+    # generation at the end of every launch: back-to-back launches on one
+    # workspace (different shapes, then the same one again) stay exact
+    import torch
+    ws = torch.zeros(vk.fwd_workspace_bytes(8, 4096, 1024), dtype=torch.uint8, device="cuda")
+    outs = []
+    for B, H, W, C in [(2, 64, 64, 64), (1, 40, 40, 64), (2, 64, 64, 64), (2, 64, 64, 64)]:
+        wl = _custom("gate_qs_x", B, H, W, C, "bf16", seed=4242)
+        inp = wl.generate()
+        x, _ = to_device(inp["x"], "bf16")
+        w, _ = vec_f32(inp["w"])
+        u, _ = vec_f32(inp["u"])
+        mus = [vec_f32(inp[n])[0] for n in ("mu_r", "mu_k", "mu_v")]
+        qs = vk.QShift(H, W, 1, 0.25, *mus)
+        a = vk.spatial_gate(x, x, x, w, u, qs=qs, workspace=ws)
+        b = vk.spatial_gate(x, x, x, w, u, qs=qs)  # cluster exchange
+        vk.device_status()
+        assert torch.equal(a, b)
+        outs.append(a)
+    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[2], outs[3])
+    ctl = ws[:12].view(torch.int32).cpu().tolist()
+    assert ctl[0] == 0 and ctl[1] == 0 and ctl[2] >= 4  # counters reset, 4+ generations
+
+
+def test_workspace_rejects_bad_arguments(vk):
+    import torch
+    x = torch.zeros(1, 512, 64, device="cuda", dtype=torch.bfloat16)
+    w = torch.zeros(64, device="cuda")
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(vk.VrwkvError):
+        vk.spatial_gate(x, x, x, w, w, workspace=small)
+    big = torch.zeros(vk.fwd_workspace_bytes(1, 512, 64) + 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(vk.VrwkvError):
+        vk.spatial_gate(x, x, x, w, w, workspace=big[1:])  # misaligned
