@@ -183,6 +183,29 @@ vrwkv_status vrwkv_spatial_gate_ws(const void* r, const void* k, const void* v,
                                    void* stream);
 
 /*
+ * vrwkv_spatial_gate_static -- vrwkv_spatial_gate_ws on a workspace the
+ * library owns, for callers that cannot allocate device memory (a fixed
+ * memory budget, an allocator they may not call at this point): the call
+ * allocates nothing.  The pages have no counterpart of this entry point; it
+ * exists only for such callers.
+ * The workspace is one 4 MiB array per device, reserved when the library is
+ * loaded, which holds the exchange state of B * ceil(C / 16) <= ~800 columns;
+ * larger problems return VRWKV_ERR_UNSUPPORTED.  Each call first clears the
+ * array's counters and flags on `stream` (cudaMemsetAsync), then runs the
+ * workspace kernel; results equal vrwkv_spatial_gate's.
+ * Calls that overlap in time (other streams, other host threads) share the
+ * one array and race: serialise them, or use vrwkv_spatial_gate_ws with a
+ * workspace per stream.
+ * Arguments, results, limits and errors otherwise as vrwkv_spatial_gate.
+ */
+vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k,
+                                       const void* v, const float* w,
+                                       const float* u, void* out, int B, int T,
+                                       int C, vrwkv_dtype dtype,
+                                       const vrwkv_qshift_params* qs,
+                                       void* stream);
+
+/*
  * vrwkv_biwkv_bwd -- gradients of Bi-WKV (eq. 5) for an upstream gradient gy
  * = dL/dwkv, by the chain rule.  For each (b, c) column, with
  * W_ti = e^{-(|t-i|-1)/T * w} (i != t), W_tt = e^u, D_t = sum_i W_ti e^{k_i}

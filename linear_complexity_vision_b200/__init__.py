@@ -76,6 +76,9 @@ def load_library():
         lib.vrwkv_spatial_gate_ws.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                               ctypes.POINTER(_QsParams), vp, ctypes.c_size_t, vp]
         lib.vrwkv_spatial_gate_ws.restype = ci
+        lib.vrwkv_spatial_gate_static.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                                  ctypes.POINTER(_QsParams), vp]
+        lib.vrwkv_spatial_gate_static.restype = ci
         lib.vrwkv_biwkv_bwd.argtypes = [vp] * 11 + [ci] * 4 + [vp]
         lib.vrwkv_biwkv_bwd.restype = ci
         lib.vrwkv_channel_mix.argtypes = [vp, vp, ci, ci, ci, ci, ctypes.POINTER(_QsParams), vp]
@@ -224,6 +227,24 @@ def channel_mix(x, qs: Optional[QShift] = None, out=None):
     qsp = ctypes.byref(qs._struct()) if qs is not None else None
     _check(load_library().vrwkv_channel_mix(
         x.data_ptr(), out.data_ptr(), B, T, C, _dtype_code(x), qsp, _stream_ptr(x)))
+    return out
+
+
+def spatial_gate_static(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
+    """spatial_gate for callers that cannot allocate device memory: the
+    column exchange runs in a fixed workspace the library reserved at load
+    time (up to ~800 (batch row, 16-channel) columns).  Calls overlapping in
+    time on other streams share that workspace and race."""
+    import torch
+    for t, name in ((r, "r"), (k, "k"), (v, "v"), (w, "w"), (u, "u")):
+        _require(t, name)
+    B, T, C = k.shape
+    if out is None:
+        out = torch.empty_like(k)
+    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _check(load_library().vrwkv_spatial_gate_static(
+        r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
+        B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
     return out
 
 

@@ -158,6 +158,29 @@ unsigned int* device_error_word() {
     return addr[dev];
 }
 
+// Fixed device workspace of vrwkv_spatial_gate_static, for callers that
+// cannot allocate device memory: it is reserved when the module loads, so a
+// call allocates nothing.  4 MiB holds the exchange state of about 800
+// (batch row, 16-channel) columns.  One array per device, shared by every
+// caller of that entry point.
+constexpr size_t kStaticWsBytes = 4u << 20;
+static __device__ __align__(256) unsigned char g_vrwkv_static_ws[kStaticWsBytes];
+
+// Address of the current device's static workspace (nullptr if unknown).
+unsigned char* static_workspace() {
+    static std::mutex mu;
+    static unsigned char* addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_vrwkv_static_ws) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned char*>(a);
+    }
+    return addr[dev];
+}
+
 bool tma_disabled() {
     const char* e = getenv("VRWKV_DISABLE_TMA");
     return e && e[0] && e[0] != '0';
@@ -685,6 +708,36 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
     else channel_mix_vec_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(p);
     g_last_kernel = "channel_mix_vec_kernel";
     return cuda_status(cudaGetLastError(), "channel_mix kernel launch");
+}
+
+vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k, const void* v, const float* w,
+                                       const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
+                                       const vrwkv_qshift_params* qs, void* stream) {
+    // the argument checks that need no device come first, so an invalid call
+    // leaves the device untouched (the launch path repeats them all)
+    if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
+        return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B <= 0 || T <= 0 || C <= 0)
+        return fail(VRWKV_ERR_INVALID_ARG, "B, T and C must be positive (got %d, %d, %d)", B, T, C);
+    if (!r || !k || !v || !w || !u || !out) return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
+    if (qs) {
+        vrwkv_status st = check_qs(qs, T, C);
+        if (st != VRWKV_OK) return st;
+    }
+    const WsLayout L = ws_layout(B, C);
+    if (L.bytes > kStaticWsBytes)
+        return fail(VRWKV_ERR_UNSUPPORTED,
+                    "B*ceil(C/16) = %lld columns need %zu bytes of exchange state; the static workspace "
+                    "holds %zu",
+                    (long long)B * ((C + fast::kCS - 1) / fast::kCS), L.bytes, kStaticWsBytes);
+    unsigned char* ws = static_workspace();
+    if (!ws) return fail(VRWKV_ERR_CUDA, "cannot locate the static workspace");
+    // counters and flags start at zero for every call (a previous call that
+    // stopped on an error may have left them set); the records need no reset
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, L.recs_off, s);
+    if (e != cudaSuccess) return cuda_status(e, "clearing the static workspace");
+    return fused_entry(true, r, k, v, w, u, out, B, T, C, dtype, qs, stream, true, ws, kStaticWsBytes);
 }
 
 vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const float* u,

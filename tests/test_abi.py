@@ -128,3 +128,14 @@ def test_biwkv_bwd_rejects_invalid_arguments(lib, args, frag):
                              a["dtype"], None)
     assert st in (1, 2)
     assert frag in lib.vrwkv_last_error().decode()
+
+
+def test_static_entry_rejects_on_the_host(lib):
+    # validation and the size limit come before any device work
+    assert lib.vrwkv_spatial_gate_static(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + (1 << 24), 0, 4, 16, 1,
+                                         None, None) == 1
+    assert lib.vrwkv_spatial_gate_static(None, FAKE, FAKE, FAKE, FAKE, FAKE + (1 << 24), 1, 4, 16, 1,
+                                         None, None) == 1
+    st = lib.vrwkv_spatial_gate_static(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + (1 << 24), 64, 4, 16384,
+                                       1, None, None)
+    assert st == 2 and b"static workspace" in lib.vrwkv_last_error()
