@@ -20,8 +20,10 @@
  *   token, then batch.  With a patch grid H x W the token index is
  *   t = h*W + w (raster order) and T = H*W.  w, u and the mu vectors are
  *   dense float32 vectors of length C.
- * Memory.  Every pointer is caller-owned DEVICE memory.  The library keeps
- *   no state between calls and allocates no device or host memory.
+ * Memory.  Every pointer is caller-owned DEVICE memory.  No call allocates
+ *   device or host memory.  The only device memory the library owns is
+ *   reserved when it loads: a device error word and the fixed workspace of
+ *   vrwkv_spatial_gate_static.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *   default stream).  Work is enqueued asynchronously; the caller
  *   synchronises.  Calls may be captured into CUDA graphs.
