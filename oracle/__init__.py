@@ -23,6 +23,10 @@ It wraps ``vrwkv_oracle.c`` (plain C, float64, OpenMP over channel columns):
 * ``biwkv_bwd``     -- gradients of eq. 5 (dk, dv and per-batch dw, du) for
                        an upstream gradient gy, by the chain rule, O(T^2).
 * ``biwkv_bwd_columns`` -- the same for selected (b, c) columns only.
+* ``layer_norm``    -- LayerNorm over channels (biased variance).
+* ``spatial_mix_block`` -- the spatial-mix block with projections: Q-Shift,
+                       R/K/V projections (eq. 1), Bi-WKV and the sigma gate
+                       (eq. 5, eq. 2), output projection W_O and LayerNorm.
 * ``channel_mix``   -- sigma(QS_R(x)) * max(QS_K(x), 0)^2, the channel-mix
                        module of eq. 3-4 without projections.
 * ``spatial_core_points`` -- the same at selected output positions only, by
@@ -267,3 +271,43 @@ def biwkv_bwd_columns(k, v, w, u, gy, cols, with_scale: bool = False):
     if with_scale:
         return gk, gv, gw, gu, (sc[:, :T], sc[:, T:2 * T], sc[:, 2 * T], sc[:, 2 * T + 1])
     return gk, gv, gw, gu
+
+
+def layer_norm(y, g, b, eps: float = 1e-5) -> np.ndarray:
+    """LayerNorm over the last (channel) axis: g * (y - mean) / sqrt(var + eps)
+    + b, with the biased variance, in float64."""
+    y = _d(y)
+    mean = y.mean(axis=-1, keepdims=True)
+    var = ((y - mean) ** 2).mean(axis=-1, keepdims=True)
+    return _d(g) * (y - mean) / np.sqrt(var + eps) + _d(b)
+
+
+def _bf16(a):
+    """Round float64 values to bfloat16 (nearest even), back to float64."""
+    a32 = np.ascontiguousarray(a, dtype=np.float32)
+    return round_bf16(a32).astype(np.float64)
+
+
+def spatial_mix_block(x, w_r, w_k, w_v, w_o, w, u, mu_r, mu_k, mu_v, ln_g, ln_b, H, W,
+                      shift_pixel=1, gamma=0.25, eps=1e-5, method="rnn",
+                      round_like_bf16: bool = False) -> np.ndarray:
+    """The spatial-mix block of "Vision-RWKV Backbone", Overall Architecture:
+    R = QS_R(x) W_R, K = QS_K(x) W_K, V = QS_V(x) W_V (eq. 1, Q-Shift of eq. 9),
+    O = (sigma(R) (.) Bi-WKV(K, V)) W_O (eq. 2, eq. 5), then LayerNorm of O over
+    channels (the pages normalise after the output projection).  Weights are
+    (C_in, C_out): row vectors times W.  With round_like_bf16 the stored
+    intermediates (the three shifted inputs, R, K, V, the gated core and O)
+    are rounded to bfloat16, as a bfloat16 implementation stores them."""
+    x = _d(x)
+    B, T, C = x.shape
+    rnd = _bf16 if round_like_bf16 else (lambda a: a)
+    xr = rnd(qshift(x, H, W, shift_pixel, gamma, mu_r))
+    xk = rnd(qshift(x, H, W, shift_pixel, gamma, mu_k))
+    xv = rnd(qshift(x, H, W, shift_pixel, gamma, mu_v))
+    R = rnd(xr @ _d(w_r))
+    K = rnd(xk @ _d(w_k))
+    V = rnd(xv @ _d(w_v))
+    f = biwkv_direct if method == "direct" else biwkv_rnn
+    core = rnd(gate(R, f(K, V, w, u)))
+    O = rnd(core @ _d(w_o))
+    return layer_norm(O, ln_g, ln_b, eps)
