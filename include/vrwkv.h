@@ -10,6 +10,7 @@
  *   - the receptance gate sigma(R) (.) wkv, Overall Architecture, eq. 2;
  *   - the channel-mix gate sigma(R_c) (.) SquaredReLU(K_c), Overall
  *     Architecture, eq. 3-4;
+ *   - the spatial-mix block with its projections and LayerNorm, eq. 1-2;
  *   - the Bi-WKV backward pass: the pages state that one exists (in an
  *     appendix they do not reproduce), so vrwkv_biwkv_bwd computes the plain
  *     derivatives of eq. 5.
@@ -21,7 +22,8 @@
  *   t = h*W + w (raster order) and T = H*W.  w, u and the mu vectors are
  *   dense float32 vectors of length C.
  * Memory.  Every pointer is caller-owned DEVICE memory.  No call allocates
- *   device or host memory.  The only device memory the library owns is
+ *   device memory; vrwkv_spatial_mix_block creates a cuBLASLt handle (host
+ *   state) once per device.  The only device memory the library owns is
  *   reserved when it loads: a device error word and the fixed workspace of
  *   vrwkv_spatial_gate_static.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
@@ -206,6 +208,45 @@ vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k,
                                        int C, vrwkv_dtype dtype,
                                        const vrwkv_qshift_params* qs,
                                        void* stream);
+
+/*
+ * vrwkv_spatial_mix_block -- the spatial-mix block with its projections
+ * (Overall Architecture, eq. 1-2, with Q-Shift of eq. 9 and Bi-WKV of eq. 5):
+ *   R = QS_R(x) W_R,  K = QS_K(x) W_K,  V = QS_V(x) W_V             (eq. 1)
+ *   O = (sigma(R) (.) Bi-WKV(K, V)) W_O                              (eq. 2)
+ *   out = LayerNorm(O) = ln_gamma * (O - mean) / sqrt(var + ln_eps) + ln_beta
+ * (LayerNorm over channels, biased variance; the pages normalise after the
+ * output projection).  Residual connections are left to the caller.
+ *   x          (B, T, C) input, dtype `dtype`, 16-byte aligned.
+ *   w_r, w_k, w_v, w_o  (C, C) weights, dtype `dtype`, row-major (C_in,
+ *              C_out): a token row times the matrix; 16-byte aligned.
+ *   w, u       float32[C] Bi-WKV decay and bonus of the projected channels.
+ *   ln_gamma, ln_beta  float32[C]; ln_eps >= 0.
+ *   out        (B, T, C) output, dtype `dtype`, 16-byte aligned.
+ *   qs         required: grid, shift, gamma and mu_r, mu_k, mu_v.
+ *   workspace  device memory of at least vrwkv_block_workspace_bytes(B, T,
+ *              C, dtype) bytes, 256-byte aligned: four (B, T, C) staging
+ *              buffers and the GEMM workspace.
+ * Steps (all on `stream`): three vrwkv_qshift calls each followed by a
+ * cuBLASLt GEMM (float32 accumulation, results stored in `dtype`), the fused
+ * vrwkv_spatial_gate core on the projected R, K, V, the W_O GEMM and a
+ * LayerNorm kernel.  The cuBLASLt handle is created once per device.
+ * Errors: INVALID_ARG for bad sizes, NULL or misaligned pointers, overlaps,
+ *   bad qs fields or a small workspace; UNSUPPORTED for B*T >= 2^31 or the
+ *   core's limits; CUDA if cuBLASLt fails.
+ */
+size_t vrwkv_block_workspace_bytes(int B, int T, int C, vrwkv_dtype dtype);
+
+vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r,
+                                     const void* w_k, const void* w_v,
+                                     const void* w_o, const float* w,
+                                     const float* u, const float* ln_gamma,
+                                     const float* ln_beta, float ln_eps,
+                                     void* out, int B, int T, int C,
+                                     vrwkv_dtype dtype,
+                                     const vrwkv_qshift_params* qs,
+                                     void* workspace, size_t workspace_bytes,
+                                     void* stream);
 
 /*
  * vrwkv_biwkv_bwd -- gradients of Bi-WKV (eq. 5) for an upstream gradient gy

@@ -11,6 +11,7 @@ There is no fallback: if the library is missing, the calls raise.
     fwd_workspace(B, T, C, device)  # a zeroed workspace for the two calls above
     channel_mix(x, qs=None)
     biwkv_bwd(k, v, w, u, gy)  # -> gk, gv, gw (B, C), gu (B, C), gw_total, gu_total
+    spatial_mix_block(x, weights, w, u, ln_gamma, ln_beta, qs, workspace=None)
     device_status()     # synchronise; raise if a kernel's bounded wait ran out
 
 Token tensors are contiguous (B, T, C) CUDA tensors of dtype float32 or
@@ -76,6 +77,11 @@ def load_library():
         lib.vrwkv_spatial_gate_ws.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                               ctypes.POINTER(_QsParams), vp, ctypes.c_size_t, vp]
         lib.vrwkv_spatial_gate_ws.restype = ci
+        lib.vrwkv_block_workspace_bytes.argtypes = [ci, ci, ci, ci]
+        lib.vrwkv_block_workspace_bytes.restype = ctypes.c_size_t
+        lib.vrwkv_spatial_mix_block.argtypes = [vp] * 9 + [ctypes.c_float, vp, ci, ci, ci, ci,
+                                                ctypes.POINTER(_QsParams), vp, ctypes.c_size_t, vp]
+        lib.vrwkv_spatial_mix_block.restype = ci
         lib.vrwkv_spatial_gate_static.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                                   ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_spatial_gate_static.restype = ci
@@ -245,6 +251,39 @@ def spatial_gate_static(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
     _check(load_library().vrwkv_spatial_gate_static(
         r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
         B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
+    return out
+
+
+def block_workspace(B: int, T: int, C: int, dtype, device="cuda"):
+    """A uint8 CUDA tensor large enough for spatial_mix_block on (B, T, C)."""
+    import torch
+    code = VRWKV_F32 if dtype == torch.float32 else VRWKV_BF16
+    n = int(load_library().vrwkv_block_workspace_bytes(B, T, C, code))
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def spatial_mix_block(x, weights, w, u, ln_gamma, ln_beta, qs: QShift, ln_eps: float = 1e-5,
+                      workspace=None, out=None):
+    """LayerNorm((sigma(R) * Bi-WKV(K, V)) W_O) with R, K, V = QS_*(x) W_*
+    (eq. 1-2).  weights = (W_R, W_K, W_V, W_O), each (C, C) in x's dtype,
+    row-major (C_in, C_out).  workspace: see block_workspace."""
+    import torch
+    _require(x, "x")
+    for i, t in enumerate(weights):
+        _require(t, f"weights[{i}]")
+    for t, name in ((w, "w"), (u, "u"), (ln_gamma, "ln_gamma"), (ln_beta, "ln_beta")):
+        _require(t, name)
+    B, T, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = block_workspace(B, T, C, x.dtype, device=x.device)
+    wr, wk, wv, wo = weights
+    _check(load_library().vrwkv_spatial_mix_block(
+        x.data_ptr(), wr.data_ptr(), wk.data_ptr(), wv.data_ptr(), wo.data_ptr(), w.data_ptr(),
+        u.data_ptr(), ln_gamma.data_ptr(), ln_beta.data_ptr(), float(ln_eps), out.data_ptr(),
+        B, T, C, _dtype_code(x), ctypes.byref(qs._struct()), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_ptr(x)))
     return out
 
 

@@ -14,6 +14,8 @@ SOURCES = ["vrwkv_api.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
               "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-O2",
               "-I" + os.path.join(ROOT, "include"), "-I" + CSRC]
+# cuBLASLt serves the dense projections of the spatial-mix block
+LIBS = ["-lcublasLt"]
 
 
 def _stale() -> bool:
@@ -31,7 +33,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp] + [os.path.join(CSRC, f) for f in SOURCES]
+    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp] + [os.path.join(CSRC, f) for f in SOURCES] + LIBS
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)

@@ -1,0 +1,85 @@
+// LayerNorm over channels for sm_100a: y = g * (x - mean) / sqrt(var + eps) + b
+// per token row, with the biased variance, as applied after the output
+// projection of the spatial-mix module ("Vision-RWKV Backbone", Overall
+// Architecture).  One warp per row: the row (a few KB) stays in L1 across the
+// three passes (mean, centred variance, normalise), so the variance has no
+// E[x^2] - E[x]^2 cancellation; HBM sees one read and one write per element.
+#pragma once
+
+#include "common.cuh"
+#include "qshift.cuh"
+
+namespace vrwkv {
+
+struct LayerNormParams {
+    const char* x;
+    char* y;
+    const float* g;
+    const float* b;
+    long long rows;
+    int C;
+    float eps;
+    int vec;  // 16-byte vectors (C * sizeof(IO) % 16 == 0, aligned pointers)
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    return v;
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(256) layer_norm_kernel(const LayerNormParams p) {
+    using V = Vec16<IO>;
+    constexpr int N = V::N;
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= p.rows) return;
+    const char* xr = p.x + (size_t)row * p.C * sizeof(IO);
+    char* yr = p.y + (size_t)row * p.C * sizeof(IO);
+    const float invC = 1.0f / (float)p.C;
+    float s = 0.f;
+    if (p.vec) {
+        const int nv = p.C / N;
+        for (int v = lane; v < nv; v += 32) {
+            float f[N];
+            V::unpack(*reinterpret_cast<const uint4*>(xr + (size_t)v * 16), f);
+#pragma unroll
+            for (int e = 0; e < N; ++e) s += f[e];
+        }
+        const float mean = warp_sum(s) * invC;
+        float q = 0.f;
+        for (int v = lane; v < nv; v += 32) {
+            float f[N];
+            V::unpack(*reinterpret_cast<const uint4*>(xr + (size_t)v * 16), f);
+#pragma unroll
+            for (int e = 0; e < N; ++e) q = fmaf(f[e] - mean, f[e] - mean, q);
+        }
+        const float rstd = rsqrtf(warp_sum(q) * invC + p.eps);
+        for (int v = lane; v < nv; v += 32) {
+            float f[N], o[N];
+            V::unpack(*reinterpret_cast<const uint4*>(xr + (size_t)v * 16), f);
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+                const int c = v * N + e;
+                o[e] = fmaf(__ldg(p.g + c), (f[e] - mean) * rstd, __ldg(p.b + c));
+            }
+            *reinterpret_cast<uint4*>(yr + (size_t)v * 16) = V::pack(o);
+        }
+    } else {
+        for (int c = lane; c < p.C; c += 32) s += Io<IO>::ld1(xr + (size_t)c * sizeof(IO));
+        const float mean = warp_sum(s) * invC;
+        float q = 0.f;
+        for (int c = lane; c < p.C; c += 32) {
+            const float d = Io<IO>::ld1(xr + (size_t)c * sizeof(IO)) - mean;
+            q = fmaf(d, d, q);
+        }
+        const float rstd = rsqrtf(warp_sum(q) * invC + p.eps);
+        for (int c = lane; c < p.C; c += 32) {
+            const float d = Io<IO>::ld1(xr + (size_t)c * sizeof(IO)) - mean;
+            Io<IO>::st1(yr + (size_t)c * sizeof(IO), fmaf(__ldg(p.g + c), d * rstd, __ldg(p.b + c)));
+        }
+    }
+}
+
+}  // namespace vrwkv

@@ -12,6 +12,7 @@
 #include <string>
 
 #include <cuda.h>
+#include <cublasLt.h>
 
 #include "vrwkv.h"
 #include "biwkv.cuh"
@@ -19,6 +20,7 @@
 #include "qshift.cuh"
 #include "channel_mix.cuh"
 #include "biwkv_bwd.cuh"
+#include "layer_norm.cuh"
 
 // Device error word: set by kernels whose bounded waits ran out (bit 0).
 __device__ unsigned int g_vrwkv_device_error;
@@ -179,6 +181,64 @@ unsigned char* static_workspace() {
         addr[dev] = static_cast<unsigned char*>(a);
     }
     return addr[dev];
+}
+
+// ---- dense projections (cuBLASLt) --------------------------------------------
+// One cuBLASLt handle per device, created on first use.
+cublasLtHandle_t lt_handle() {
+    static std::mutex mu;
+    static cublasLtHandle_t h[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!h[dev] && cublasLtCreate(&h[dev]) != CUBLAS_STATUS_SUCCESS) h[dev] = nullptr;
+    return h[dev];
+}
+
+// D (M x N) = X (M x K) * Wt (K x N), all row-major, float32 accumulation.
+// In cuBLASLt's column-major terms: D^T (N x M) = Wt^T (N x K) * X^T (K x M),
+// where each row-major matrix read column-major is its transpose.
+vrwkv_status gemm_rowmajor(const void* X, const void* Wt, void* D, int M, int N, int K,
+                           vrwkv_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t s) {
+    cublasLtHandle_t h = lt_handle();
+    if (!h) return fail(VRWKV_ERR_CUDA, "cuBLASLt handle could not be created");
+    const cudaDataType_t dt = dtype == VRWKV_F32 ? CUDA_R_32F : CUDA_R_16BF;
+    cublasLtMatmulDesc_t op = nullptr;
+    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
+    cublasLtMatmulPreference_t pref = nullptr;
+    vrwkv_status st = VRWKV_OK;
+    cublasLtMatmulHeuristicResult_t res = {};
+    int nres = 0;
+    const float one = 1.0f, zero = 0.0f;
+    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatrixLayoutCreate(&la, dt, N, K, N) != CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatrixLayoutCreate(&lb, dt, K, M, K) != CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatrixLayoutCreate(&ld, dt, N, M, N) != CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
+                                             sizeof(ws_bytes)) != CUBLAS_STATUS_SUCCESS) {
+        st = fail(VRWKV_ERR_CUDA, "cuBLASLt descriptor setup failed");
+    } else if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, ld, ld, pref, 1, &res, &nres) !=
+                   CUBLAS_STATUS_SUCCESS ||
+               nres == 0) {
+        st = fail(VRWKV_ERR_UNSUPPORTED, "no cuBLASLt algorithm for a %d x %d x %d GEMM", M, N, K);
+    } else if (cublasLtMatmul(h, op, &one, Wt, la, X, lb, &zero, D, ld, D, ld, &res.algo, ws, ws_bytes,
+                              s) != CUBLAS_STATUS_SUCCESS) {
+        st = fail(VRWKV_ERR_CUDA, "cuBLASLt matmul failed");
+    }
+    if (pref) cublasLtMatmulPreferenceDestroy(pref);
+    if (ld) cublasLtMatrixLayoutDestroy(ld);
+    if (lb) cublasLtMatrixLayoutDestroy(lb);
+    if (la) cublasLtMatrixLayoutDestroy(la);
+    if (op) cublasLtMatmulDescDestroy(op);
+    return st;
+}
+
+// Workspace of vrwkv_spatial_mix_block: four (B, T, C) token buffers and the
+// GEMM workspace, each 256-byte aligned.
+constexpr size_t kGemmWsBytes = 32u << 20;
+size_t block_ws_slot(int B, int T, int C, vrwkv_dtype dtype) {
+    return ((size_t)B * T * C * elem_bytes(dtype) + 255) / 256 * 256;
 }
 
 bool tma_disabled() {
@@ -708,6 +768,98 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
     else channel_mix_vec_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(p);
     g_last_kernel = "channel_mix_vec_kernel";
     return cuda_status(cudaGetLastError(), "channel_mix kernel launch");
+}
+
+size_t vrwkv_block_workspace_bytes(int B, int T, int C, vrwkv_dtype dtype) {
+    if (B <= 0 || T <= 0 || C <= 0 || (dtype != VRWKV_F32 && dtype != VRWKV_BF16)) return 0;
+    return 4 * block_ws_slot(B, T, C, dtype) + kGemmWsBytes;
+}
+
+vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void* w_k, const void* w_v,
+                                     const void* w_o, const float* w, const float* u, const float* ln_gamma,
+                                     const float* ln_beta, float ln_eps, void* out, int B, int T, int C,
+                                     vrwkv_dtype dtype, const vrwkv_qshift_params* qs, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
+        return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B <= 0 || T <= 0 || C <= 0)
+        return fail(VRWKV_ERR_INVALID_ARG, "B, T and C must be positive (got %d, %d, %d)", B, T, C);
+    if (!x || !w_r || !w_k || !w_v || !w_o || !w || !u || !ln_gamma || !ln_beta || !out || !qs || !workspace)
+        return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
+    if (!(ln_eps >= 0.0f)) return fail(VRWKV_ERR_INVALID_ARG, "ln_eps must be >= 0");
+    if ((long long)B * T > 0x7fffffffLL) return fail(VRWKV_ERR_UNSUPPORTED, "B*T must be below 2^31");
+    {
+        vrwkv_status st = check_qs(qs, T, C);
+        if (st != VRWKV_OK) return st;
+    }
+    const void* mats[6] = {x, w_r, w_k, w_v, w_o, out};
+    for (const void* m : mats)
+        if (!aligned(m, 16)) return fail(VRWKV_ERR_INVALID_ARG, "token and weight tensors must be 16-byte aligned");
+    const float* vecs[4] = {w, u, ln_gamma, ln_beta};
+    for (const float* f : vecs)
+        if (!aligned(f, 4)) return fail(VRWKV_ERR_INVALID_ARG, "float32 vector misaligned");
+    if (!aligned(workspace, 256)) return fail(VRWKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const size_t need = vrwkv_block_workspace_bytes(B, T, C, dtype);
+    if (workspace_bytes < need)
+        return fail(VRWKV_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed",
+                    workspace_bytes, need);
+    const int es = elem_bytes(dtype);
+    const size_t nb = (size_t)B * T * C * es, wb = (size_t)C * C * es;
+    struct Span { const void* p; size_t n; };
+    const Span ins[11] = {{x, nb}, {w_r, wb}, {w_k, wb}, {w_v, wb}, {w_o, wb}, {w, (size_t)C * 4},
+                          {u, (size_t)C * 4}, {ln_gamma, (size_t)C * 4}, {ln_beta, (size_t)C * 4},
+                          {qs->mu_r, (size_t)C * 4}, {qs->mu_k, (size_t)C * 4}};
+    for (const Span& in : ins) {
+        if (overlaps(out, nb, in.p, in.n)) return fail(VRWKV_ERR_INVALID_ARG, "output overlaps an input");
+        if (overlaps(workspace, need, in.p, in.n))
+            return fail(VRWKV_ERR_INVALID_ARG, "workspace overlaps an input");
+    }
+    if (overlaps(workspace, need, out, nb) || overlaps(workspace, need, qs->mu_v, (size_t)C * 4) ||
+        overlaps(out, nb, qs->mu_v, (size_t)C * 4))
+        return fail(VRWKV_ERR_INVALID_ARG, "workspace or output overlaps");
+
+    // Q-Shift -> projection, three times; the shifted input is staged in t0
+    const size_t slot = block_ws_slot(B, T, C, dtype);
+    char* base = static_cast<char*>(workspace);
+    void* t0 = base;
+    void* bR = base + slot;
+    void* bK = base + 2 * slot;
+    void* bV = base + 3 * slot;
+    void* gws = base + 4 * slot;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int M = B * T;
+    const float* mus[3] = {qs->mu_r, qs->mu_k, qs->mu_v};
+    const void* wts[3] = {w_r, w_k, w_v};
+    void* dst[3] = {bR, bK, bV};
+    for (int i = 0; i < 3; ++i) {
+        vrwkv_status st = vrwkv_qshift(x, t0, mus[i], B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma, dtype,
+                                       stream);
+        if (st != VRWKV_OK) return st;
+        st = gemm_rowmajor(t0, wts[i], dst[i], M, C, C, dtype, gws, kGemmWsBytes, s);
+        if (st != VRWKV_OK) return st;
+    }
+    // sigma(R) (.) Bi-WKV(K, V) on the projected channels (Q-Shift already
+    // applied before the projections), into t0
+    vrwkv_status st = vrwkv_spatial_gate(bR, bK, bV, w, u, t0, B, T, C, dtype, nullptr, stream);
+    if (st != VRWKV_OK) return st;
+    // W_O into the R buffer (dead after the gate), then LayerNorm into out
+    st = gemm_rowmajor(t0, w_o, bR, M, C, C, dtype, gws, kGemmWsBytes, s);
+    if (st != VRWKV_OK) return st;
+    LayerNormParams lp;
+    lp.x = static_cast<const char*>(bR);
+    lp.y = static_cast<char*>(out);
+    lp.g = ln_gamma;
+    lp.b = ln_beta;
+    lp.rows = M;
+    lp.C = C;
+    lp.eps = ln_eps;
+    lp.vec = ((size_t)C * es) % 16 == 0;
+    const unsigned blocks = (unsigned)((M + 7) / 8);
+    if (dtype == VRWKV_F32) layer_norm_kernel<float><<<blocks, 256, 0, s>>>(lp);
+    else layer_norm_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(lp);
+    st = cuda_status(cudaGetLastError(), "layer_norm_kernel launch");
+    if (st == VRWKV_OK) g_last_kernel = "spatial_mix_block";
+    return st;
 }
 
 vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k, const void* v, const float* w,

@@ -1,0 +1,110 @@
+"""GPU parity of the spatial-mix block (vrwkv_spatial_mix_block: Q-Shift,
+R/K/V projections, Bi-WKV, sigma gate, W_O, LayerNorm; "Vision-RWKV
+Backbone", Overall Architecture, eq. 1-2) against the float64 oracle.
+
+The oracle rounds the intermediates the bfloat16 path stores (the shifted
+inputs, R, K, V, the gated core, O) to bfloat16 at the same points; what is
+left are float32-versus-float64 differences, which can flip a bfloat16
+rounding (2^-8 relative) of an intermediate, and the core's own error.  The
+output is LayerNorm-scaled (unit variance before ln_gamma) and stored in the
+I/O dtype, whose last place grows with the value (one bfloat16 ulp is 0.03 at
+|out| = 4), so each element's error is divided by max(|ln_gamma|, |ref|):
+max <= 3e-2 and mean <= 3e-3 for bfloat16 I/O, 1e-3 / 1e-4 for float32 I/O.
+"""
+import zlib
+
+import numpy as np
+import pytest
+
+from linear_complexity_vision_b200 import synth
+from helpers import to_device, to_numpy, vec_f32
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": (3e-2, 3e-3), "f32": (1e-3, 1e-4)}
+
+
+@pytest.fixture(scope="module")
+def vk():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import linear_complexity_vision_b200 as vk
+    vk.load_library()
+    return vk
+
+
+def _case(B, H, W, C, dt):
+    seed = 20290000 + zlib.crc32(repr((B, H, W, C, dt)).encode()) % 100000
+    x = synth.draw(seed, "x", (B, H * W, C), ("normal", 1.0))
+    mats = [synth.draw(seed + 1 + i, "r", (C, C), ("normal", 1.0 / np.sqrt(C))) for i in range(4)]
+    w = synth.draw(seed, "w", (C,), ("uniform", -5.0, 5.0))
+    u = synth.draw(seed, "u", (C,), ("normal", 1.0))
+    mus = [synth.draw(seed, n, (C,), ("uniform", 0.0, 1.0)) for n in ("mu_r", "mu_k", "mu_v")]
+    g = 1.0 + 0.1 * synth.draw(seed, "k", (C,), ("normal", 1.0))
+    b = 0.1 * synth.draw(seed, "v", (C,), ("normal", 1.0))
+    return x, mats, w, u, mus, g, b
+
+
+@pytest.mark.parametrize("dt,B,H,W,C", [
+    ("bf16", 2, 14, 14, 64),     # the 224^2 grid
+    ("bf16", 1, 16, 32, 128),    # two CTAs per column in the core
+    ("f32", 1, 14, 14, 64),
+    ("bf16", 8, 64, 64, 1024),   # the full-size 1024^2 grid at C = 1024
+])
+def test_block_parity(vk, oracle_mod, dt, B, H, W, C):
+    x, mats, w, u, mus, g, b = _case(B, H, W, C, dt)
+    xt, xd = to_device(x, dt)
+    mt, md = zip(*[to_device(m, dt) for m in mats])
+    wt, wd = vec_f32(w)
+    ut, ud = vec_f32(u)
+    mut, mud = zip(*[vec_f32(m) for m in mus])
+    gt, gd = vec_f32(g)
+    bt, bd = vec_f32(b)
+    qs = vk.QShift(H, W, 1, 0.25, *mut)
+    out = vk.spatial_mix_block(xt, mt, wt, ut, gt, bt, qs)
+    vk.device_status()
+    got = to_numpy(out)
+    want = oracle_mod.spatial_mix_block(xd, *md, wd, ud, *mud, gd, bd, H, W,
+                                        round_like_bf16=(dt == "bf16"),
+                                        method="rnn" if H * W > 600 else "direct")
+    if dt == "bf16":
+        want = oracle_mod._bf16(want)
+    err = np.abs(got - want) / np.maximum(np.abs(gd), np.abs(want))
+    tmax, tmean = TOL[dt]
+    assert np.all(np.isfinite(got))
+    assert err.max() <= tmax, f"max error {err.max():.3e}"
+    assert err.mean() <= tmean, f"mean error {err.mean():.3e}"
+    assert vk.load_library().vrwkv_last_kernel().decode() == "spatial_mix_block"
+
+
+def test_block_identity_weights_equal_layer_norm_of_core(vk):
+    # W = I everywhere: the block is LayerNorm of vrwkv_spatial_gate's output
+    import torch
+    B, H, W, C = 2, 16, 16, 64
+    x, _, w, u, mus, g, b = _case(B, H, W, C, "f32")
+    xt, _ = to_device(x, "f32")
+    eye = torch.eye(C, device="cuda")
+    wt, _ = vec_f32(w)
+    ut, _ = vec_f32(u)
+    mut = [vec_f32(m)[0] for m in mus]
+    gt, _ = vec_f32(g)
+    bt, _ = vec_f32(b)
+    qs = vk.QShift(H, W, 1, 0.25, *mut)
+    got = vk.spatial_mix_block(xt, (eye, eye, eye, eye), wt, ut, gt, bt, qs)
+    core = vk.spatial_gate(xt, xt, xt, wt, ut, qs=qs)
+    want = torch.nn.functional.layer_norm(core, (C,), gt, bt, eps=1e-5)
+    # the block's core runs on the projected (here shifted, unmixed-again)
+    # inputs without Q-Shift, so it reads the same mixes as spatial_gate
+    torch.testing.assert_close(got, want, rtol=1e-4, atol=1e-4)
+
+
+def test_block_rejects_small_workspace(vk):
+    import torch
+    x = torch.zeros(1, 16, 64, device="cuda", dtype=torch.bfloat16)
+    m = torch.zeros(64, 64, device="cuda", dtype=torch.bfloat16)
+    v = torch.zeros(64, device="cuda")
+    qs = vk.QShift(4, 4, 1, 0.25, v, v, v)
+    with pytest.raises(vk.VrwkvError):
+        vk.spatial_mix_block(x, (m, m, m, m), v, v, v, v, qs,
+                             workspace=torch.empty(1024, dtype=torch.uint8, device="cuda"))
