@@ -26,7 +26,8 @@ region.  ``--impl reference`` times the CPU oracle alone on the same metric.
 (eq. 3-4 with identity projections) on the same x buffers and
 ``rows.biwkv_bwd`` that of the Bi-WKV backward at the workload's shape;
 ``rows.fused_workspace`` times the main step through the workspace entry
-points (global-memory exchange instead of clusters).  Each is timed in its
+points (global-memory exchange instead of clusters), and
+``rows.spatial_mix_block`` the block with projections and LayerNorm.  Each is timed in its
 own region after the main one (``--no-rows`` skips them).
 """
 from __future__ import annotations
@@ -381,6 +382,62 @@ def time_fused_ws(runner, stream, torch, dev, launches: int, peak: float):
             "exchange": "global-memory workspace (no clusters)"}
 
 
+def measured_tensor_peak():
+    """Measured dense bf16 GEMM throughput (burst), TFLOP/s."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def time_block(runner, stream, torch, dev, launches: int):
+    """The spatial-mix block with projections (vrwkv_spatial_mix_block) at the
+    workload's (B, T, C): Q-Shift, four cuBLASLt GEMMs, the fused core and a
+    LayerNorm per launch.  Roofline against the dense bf16 peak with the four
+    GEMMs' 8*B*T*C^2 FLOPs; random weights of scale 1/sqrt(C)."""
+    wl, vk = runner.wl, runner.vk
+    if wl.call == "biwkv" or wl.dtype != "bf16":
+        return None
+    g = torch.Generator(device=dev).manual_seed(20260202)
+    C = wl.C
+    mats = tuple((torch.randn(C, C, generator=g, device=dev) / C ** 0.5).to(torch.bfloat16)
+                 for _ in range(4))
+    lg = 1 + 0.1 * torch.randn(C, generator=g, device=dev)
+    lb = 0.1 * torch.randn(C, generator=g, device=dev)
+    p = runner.par
+    ws = vk.block_workspace(wl.B, wl.T, C, torch.bfloat16, device=dev)
+    n = runner.nsets
+    key = "x" if "x" in runner.sets[0] else "k"
+
+    def launch(i):
+        d = runner.sets[i % n]
+        vk.spatial_mix_block(d[key], mats, p["w"], p["u"], lg, lb, runner.qs, workspace=ws,
+                             out=d["out"])
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            launch(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(launches):
+            launch(i)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    vk.device_status()
+    us = e0.elapsed_time(e1) * 1e3 / launches
+    flops = 8.0 * wl.B * wl.T * C * C
+    peak, kind = measured_tensor_peak()
+    achieved = flops / (us * 1e-6) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "peak_source": kind, "kernel": "spatial_mix_block",
+            "flops_per_launch": flops, "avg_launch_us": us, "launches": launches,
+            "gemm": "cuBLASLt bf16, float32 accumulation",
+            "timing": "back-to-back launches"}
+
+
 def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float):
     """Roofline of the Bi-WKV backward (vrwkv_biwkv_bwd) at the workload's
     (B, T, C) and dtype, timed in its own region: k, v and gy read once, gk
@@ -594,6 +651,9 @@ def run_ours(args, dist):
         gx = time_fused_ws(runner, stream, torch, dev, args.row_launches, peak)
         if gx is not None:
             rows["fused_workspace"] = gx
+        blk = time_block(runner, stream, torch, dev, max(20, args.row_launches // 20))
+        if blk is not None:
+            rows["spatial_mix_block"] = blk
         bw = time_biwkv_bwd(runner, stream, torch, dev, max(20, args.row_launches // 20), peak)
         if bw is not None:
             rows["biwkv_bwd"] = bw

@@ -3,6 +3,7 @@
 // Validation happens before any CUDA call, so invalid arguments are
 // rejected without touching the device.
 #include <algorithm>
+#include <array>
 #include <atomic>
 #include <cstdarg>
 #include <cstdint>
@@ -10,6 +11,8 @@
 #include <cstdlib>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include <cuda.h>
 #include <cublasLt.h>
@@ -197,41 +200,61 @@ cublasLtHandle_t lt_handle() {
 
 // D (M x N) = X (M x K) * Wt (K x N), all row-major, float32 accumulation.
 // In cuBLASLt's column-major terms: D^T (N x M) = Wt^T (N x K) * X^T (K x M),
-// where each row-major matrix read column-major is its transpose.
+// where each row-major matrix read column-major is its transpose.  The
+// descriptors and the algorithm the heuristic picks are built once per
+// (device, shape, dtype) and kept: they are host-side objects, and rebuilding
+// them for every call costs more host time than the GEMM takes on the GPU.
+struct GemmPlan {
+    cublasLtMatmulDesc_t op = nullptr;
+    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
+    cublasLtMatmulAlgo_t algo;
+    bool ok = false;
+};
+
+const GemmPlan* gemm_plan(cublasLtHandle_t h, int dev, int M, int N, int K, vrwkv_dtype dtype,
+                          size_t ws_bytes) {
+    static std::mutex mu;
+    static std::vector<std::pair<std::array<long long, 6>, GemmPlan*>> cache;
+    const std::array<long long, 6> key = {dev, M, N, K, (long long)dtype, (long long)ws_bytes};
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto& e : cache)
+        if (e.first == key) return e.second->ok ? e.second : nullptr;
+    GemmPlan* g = new GemmPlan();  // kept for the life of the process
+    const cudaDataType_t dt = dtype == VRWKV_F32 ? CUDA_R_32F : CUDA_R_16BF;
+    cublasLtMatmulPreference_t pref = nullptr;
+    cublasLtMatmulHeuristicResult_t res = {};
+    int nres = 0;
+    if (cublasLtMatmulDescCreate(&g->op, CUBLAS_COMPUTE_32F, CUDA_R_32F) == CUBLAS_STATUS_SUCCESS &&
+        cublasLtMatrixLayoutCreate(&g->la, dt, N, K, N) == CUBLAS_STATUS_SUCCESS &&
+        cublasLtMatrixLayoutCreate(&g->lb, dt, K, M, K) == CUBLAS_STATUS_SUCCESS &&
+        cublasLtMatrixLayoutCreate(&g->ld, dt, N, M, N) == CUBLAS_STATUS_SUCCESS &&
+        cublasLtMatmulPreferenceCreate(&pref) == CUBLAS_STATUS_SUCCESS &&
+        cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
+                                             sizeof(ws_bytes)) == CUBLAS_STATUS_SUCCESS &&
+        cublasLtMatmulAlgoGetHeuristic(h, g->op, g->la, g->lb, g->ld, g->ld, pref, 1, &res, &nres) ==
+            CUBLAS_STATUS_SUCCESS &&
+        nres > 0) {
+        g->algo = res.algo;
+        g->ok = true;
+    }
+    if (pref) cublasLtMatmulPreferenceDestroy(pref);
+    cache.emplace_back(key, g);
+    return g->ok ? g : nullptr;
+}
+
 vrwkv_status gemm_rowmajor(const void* X, const void* Wt, void* D, int M, int N, int K,
                            vrwkv_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t s) {
     cublasLtHandle_t h = lt_handle();
     if (!h) return fail(VRWKV_ERR_CUDA, "cuBLASLt handle could not be created");
-    const cudaDataType_t dt = dtype == VRWKV_F32 ? CUDA_R_32F : CUDA_R_16BF;
-    cublasLtMatmulDesc_t op = nullptr;
-    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
-    cublasLtMatmulPreference_t pref = nullptr;
-    vrwkv_status st = VRWKV_OK;
-    cublasLtMatmulHeuristicResult_t res = {};
-    int nres = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(VRWKV_ERR_CUDA, "cudaGetDevice failed");
+    const GemmPlan* g = gemm_plan(h, dev, M, N, K, dtype, ws_bytes);
+    if (!g) return fail(VRWKV_ERR_UNSUPPORTED, "no cuBLASLt algorithm for a %d x %d x %d GEMM", M, N, K);
     const float one = 1.0f, zero = 0.0f;
-    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutCreate(&la, dt, N, K, N) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutCreate(&lb, dt, K, M, K) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutCreate(&ld, dt, N, M, N) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
-                                             sizeof(ws_bytes)) != CUBLAS_STATUS_SUCCESS) {
-        st = fail(VRWKV_ERR_CUDA, "cuBLASLt descriptor setup failed");
-    } else if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, ld, ld, pref, 1, &res, &nres) !=
-                   CUBLAS_STATUS_SUCCESS ||
-               nres == 0) {
-        st = fail(VRWKV_ERR_UNSUPPORTED, "no cuBLASLt algorithm for a %d x %d x %d GEMM", M, N, K);
-    } else if (cublasLtMatmul(h, op, &one, Wt, la, X, lb, &zero, D, ld, D, ld, &res.algo, ws, ws_bytes,
-                              s) != CUBLAS_STATUS_SUCCESS) {
-        st = fail(VRWKV_ERR_CUDA, "cuBLASLt matmul failed");
-    }
-    if (pref) cublasLtMatmulPreferenceDestroy(pref);
-    if (ld) cublasLtMatrixLayoutDestroy(ld);
-    if (lb) cublasLtMatrixLayoutDestroy(lb);
-    if (la) cublasLtMatrixLayoutDestroy(la);
-    if (op) cublasLtMatmulDescDestroy(op);
-    return st;
+    if (cublasLtMatmul(h, g->op, &one, Wt, g->la, X, g->lb, &zero, D, g->ld, D, g->ld, &g->algo, ws,
+                       ws_bytes, s) != CUBLAS_STATUS_SUCCESS)
+        return fail(VRWKV_ERR_CUDA, "cuBLASLt matmul failed");
+    return ok();
 }
 
 // Workspace of vrwkv_spatial_mix_block: four (B, T, C) token buffers and the
