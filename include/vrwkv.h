@@ -225,12 +225,13 @@ vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k,
  *   out        (B, T, C) output, dtype `dtype`, 16-byte aligned.
  *   qs         required: grid, shift, gamma and mu_r, mu_k, mu_v.
  *   workspace  device memory of at least vrwkv_block_workspace_bytes(B, T,
- *              C, dtype) bytes, 256-byte aligned: four (B, T, C) staging
+ *              C, dtype) bytes, 256-byte aligned: six (B, T, C) staging
  *              buffers and the GEMM workspace.
- * Steps (all on `stream`): three vrwkv_qshift calls each followed by a
- * cuBLASLt GEMM (float32 accumulation, results stored in `dtype`), the fused
- * vrwkv_spatial_gate core on the projected R, K, V, the W_O GEMM and a
- * LayerNorm kernel.  The cuBLASLt handle is created once per device.
+ * Steps (all on `stream`): the three Q-Shift mixes (one pass over x; each
+ * bit-identical to vrwkv_qshift's), three cuBLASLt GEMMs (float32
+ * accumulation, results stored in `dtype`), the fused vrwkv_spatial_gate core
+ * on the projected R, K, V, the W_O GEMM and a LayerNorm kernel.  The
+ * cuBLASLt handle and each GEMM shape's plan are created once per device.
  * Errors: INVALID_ARG for bad sizes, NULL or misaligned pointers, overlaps,
  *   bad qs fields or a small workspace; UNSUPPORTED for B*T >= 2^31 or the
  *   core's limits; CUDA if cuBLASLt fails.

@@ -257,7 +257,7 @@ vrwkv_status gemm_rowmajor(const void* X, const void* Wt, void* D, int M, int N,
     return ok();
 }
 
-// Workspace of vrwkv_spatial_mix_block: four (B, T, C) token buffers and the
+// Workspace of vrwkv_spatial_mix_block: six (B, T, C) token buffers and the
 // GEMM workspace, each 256-byte aligned.
 constexpr size_t kGemmWsBytes = 32u << 20;
 size_t block_ws_slot(int B, int T, int C, vrwkv_dtype dtype) {
@@ -795,7 +795,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
 
 size_t vrwkv_block_workspace_bytes(int B, int T, int C, vrwkv_dtype dtype) {
     if (B <= 0 || T <= 0 || C <= 0 || (dtype != VRWKV_F32 && dtype != VRWKV_BF16)) return 0;
-    return 4 * block_ws_slot(B, T, C, dtype) + kGemmWsBytes;
+    return 6 * block_ws_slot(B, T, C, dtype) + kGemmWsBytes;
 }
 
 vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void* w_k, const void* w_v,
@@ -841,24 +841,54 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
         overlaps(out, nb, qs->mu_v, (size_t)C * 4))
         return fail(VRWKV_ERR_INVALID_ARG, "workspace or output overlaps");
 
-    // Q-Shift -> projection, three times; the shifted input is staged in t0
+    // the three Q-Shift mixes (one pass over x when the vector kernel
+    // applies, else three), then the three projections
     const size_t slot = block_ws_slot(B, T, C, dtype);
     char* base = static_cast<char*>(workspace);
-    void* t0 = base;
-    void* bR = base + slot;
-    void* bK = base + 2 * slot;
-    void* bV = base + 3 * slot;
-    void* gws = base + 4 * slot;
+    void* sh[3] = {base, base + slot, base + 2 * slot};
+    void* bR = base + 3 * slot;
+    void* bK = base + 4 * slot;
+    void* bV = base + 5 * slot;
+    void* gws = base + 6 * slot;
+    void* t0 = sh[0];
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int M = B * T;
     const float* mus[3] = {qs->mu_r, qs->mu_k, qs->mu_v};
     const void* wts[3] = {w_r, w_k, w_v};
     void* dst[3] = {bR, bK, bV};
-    for (int i = 0; i < 3; ++i) {
-        vrwkv_status st = vrwkv_qshift(x, t0, mus[i], B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma, dtype,
-                                       stream);
+    const int g = group_size(C, qs->gamma);
+    const int nvec = 16 / es;
+    if (mus[0] && mus[1] && mus[2] && C % nvec == 0 && (long long)qs->H * qs->W <= 0x7fffffffLL) {
+        Qshift3Params q3;
+        q3.base.x = static_cast<const char*>(x);
+        q3.base.out = nullptr;
+        q3.base.mu = nullptr;
+        q3.base.BT = (long long)B * T;
+        q3.base.T = T;
+        q3.base.C = C;
+        q3.base.H = qs->H;
+        q3.base.W = qs->W;
+        q3.base.s = qs->shift_pixel;
+        q3.base.g = g;
+        for (int i = 0; i < 3; ++i) {
+            q3.out[i] = static_cast<char*>(sh[i]);
+            q3.mu[i] = mus[i];
+        }
+        const long long work = q3.base.BT * (C / nvec);
+        const long long blocks = std::min<long long>((work + 255) / 256, 148LL * 16);
+        if (dtype == VRWKV_F32) qshift3_vec_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(q3);
+        else qshift3_vec_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(q3);
+        vrwkv_status st = cuda_status(cudaGetLastError(), "qshift3 kernel launch");
         if (st != VRWKV_OK) return st;
-        st = gemm_rowmajor(t0, wts[i], dst[i], M, C, C, dtype, gws, kGemmWsBytes, s);
+    } else {
+        for (int i = 0; i < 3; ++i) {
+            vrwkv_status st = vrwkv_qshift(x, sh[i], mus[i], B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
+                                           dtype, stream);
+            if (st != VRWKV_OK) return st;
+        }
+    }
+    for (int i = 0; i < 3; ++i) {
+        vrwkv_status st = gemm_rowmajor(sh[i], wts[i], dst[i], M, C, C, dtype, gws, kGemmWsBytes, s);
         if (st != VRWKV_OK) return st;
     }
     // sigma(R) (.) Bi-WKV(K, V) on the projected channels (Q-Shift already
