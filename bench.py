@@ -409,11 +409,12 @@ def time_block(runner, stream, torch, dev, launches: int):
     ws = vk.block_workspace(wl.B, wl.T, C, torch.bfloat16, device=dev)
     n = runner.nsets
     key = "x" if "x" in runner.sets[0] else "k"
+    outs = [torch.empty_like(d[key]) for d in runner.sets]  # the main step's outputs stay intact
 
     def launch(i):
         d = runner.sets[i % n]
         vk.spatial_mix_block(d[key], mats, p["w"], p["u"], lg, lb, runner.qs, workspace=ws,
-                             out=d["out"])
+                             out=outs[i % n])
 
     with torch.cuda.stream(stream):
         for i in range(3):
@@ -653,7 +654,13 @@ def run_ours(args, dist):
         "gpu_launches": steps * runner.launches_per_step,
         "clocks": clocks.summary(),
     }
-    # the next hot-path row on the same buffers (its own timed region)
+    # correctness guard on the main step's last output (first set of the
+    # rotation), taken before the rows below reuse the device
+    parity_err = None
+    if dist.rank == 0:
+        import oracle
+        parity_err = parity_sample(runner, runner.sets[0]["out"], oracle)
+    # the next hot-path rows on the same shape (each its own timed region)
     if args.rows:
         cm = time_channel_mix(runner, stream, torch, dev, args.row_launches, peak)
         rows = {}
@@ -670,10 +677,10 @@ def run_ours(args, dist):
             rows["biwkv_bwd"] = bw
         if rows:
             line["rows"] = rows
-    # correctness guard on the last timed output (first set of the rotation)
+    # the guard's result and, on one GPU, the CPU oracle baseline (rank 0)
     if dist.rank == 0:
         import oracle
-        line["parity_sample_max_abs_err"] = parity_sample(runner, runner.sets[0]["out"], oracle)
+        line["parity_sample_max_abs_err"] = parity_err
         if dist.world == 1 and not args.no_cpu_baseline:
             v, n, dt = oracle_throughput(wl, oracle, target_s=args.cpu_seconds)
             line["cpu_baseline"] = {

@@ -160,6 +160,73 @@ __global__ void __launch_bounds__(256, 3) channel_mix_vec_kernel(const ChannelMi
     }
 }
 
+// Q-Shift mixes on the same column walk: NMIX outputs out[m] = mu_m*x +
+// (1-mu_m)*x_shift (t1 = mu*x, t2 = (1-mu)*x_shift, t1 + t2, each rounded, as
+// qshift_vec_kernel), or x_shift itself when mu[0] is null (NMIX = 1).  One
+// load of x and of its neighbour feeds every output.  Requires the vector
+// conditions of channel_mix_vec_kernel (no vector straddles a channel group).
+template <int NMIX>
+struct QsMixParams {
+    ChannelMixParams base;  // x, BT, T, C, H, W, s, g, UR, divT, divW
+    char* out[NMIX];
+    const float* mu[NMIX];
+};
+
+template <typename IO, int NMIX>
+__global__ void __launch_bounds__(256) qs_mix_vec_kernel(const QsMixParams<NMIX> q) {
+    using V = Vec16<IO>;
+    constexpr int N = V::N;
+    const ChannelMixParams& p = q.base;
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= p.UR) return;
+    const int c0 = v * N;
+    const bool with_mu = q.mu[0] != nullptr;
+    float mu[NMIX][N];
+#pragma unroll
+    for (int m = 0; m < NMIX; ++m)
+#pragma unroll
+        for (int e = 0; e < N; ++e) mu[m][e] = with_mu ? __ldg(q.mu[m] + c0 + e) : 0.0f;
+    const ShiftRule rule = shift_rule(c0, p.g, p.H, p.W, p.s);
+    const long long Gy = gridDim.y;
+    const int r0 = (int)((long long)p.BT * blockIdx.y / Gy);
+    const int r1 = (int)((long long)p.BT * (blockIdx.y + 1) / Gy);
+    const int ty = blockDim.y;
+    const size_t rowb = (size_t)p.C * sizeof(IO);
+    const char* xcol = p.x + (size_t)c0 * sizeof(IO);
+    for (int base = r0 + threadIdx.y; base < r1; base += ty * kCmRows) {
+        uint4 rx[kCmRows], rd[kCmRows];
+#pragma unroll
+        for (int j = 0; j < kCmRows; ++j) {
+            const int r = base + j * ty;
+            rx[j] = make_uint4(0u, 0u, 0u, 0u);
+            rd[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < r1) {
+                const unsigned int t = (unsigned int)r - fdiv((unsigned int)r, p.divT) * (unsigned int)p.T;
+                const int h = (int)fdiv(t, p.divW);
+                const int w = (int)t - h * p.W;
+                rx[j] = __ldg(reinterpret_cast<const uint4*>(xcol + (size_t)r * rowb));
+                if (shift_ok(rule, h, w))
+                    rd[j] = __ldg(reinterpret_cast<const uint4*>(xcol + (size_t)(r + rule.off) * rowb));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kCmRows; ++j) {
+            const int r = base + j * ty;
+            if (r >= r1) break;
+            float xv[N], xd[N];
+            V::unpack(rx[j], xv);
+            V::unpack(rd[j], xd);
+#pragma unroll
+            for (int m = 0; m < NMIX; ++m) {
+                float o[N];
+#pragma unroll
+                for (int e = 0; e < N; ++e) o[e] = with_mu ? qs_mix(mu[m][e], xv[e], xd[e]) : xd[e];
+                *reinterpret_cast<uint4*>(q.out[m] + (size_t)r * rowb + (size_t)c0 * sizeof(IO)) = V::pack(o);
+            }
+        }
+    }
+}
+
 // Scalar path for any C, group size and element-aligned pointers.
 template <typename IO>
 __global__ void __launch_bounds__(256) channel_mix_scalar_kernel(const ChannelMixParams p) {

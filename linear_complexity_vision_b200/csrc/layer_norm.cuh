@@ -28,6 +28,56 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Rows of at most 32 * VPL 16-byte vectors: the warp holds its row in
+// registers, so each element is read once; mean and centred variance come
+// from the registers.
+template <typename IO, int VPL>
+__global__ void __launch_bounds__(256) layer_norm_reg_kernel(const LayerNormParams p) {
+    using V = Vec16<IO>;
+    constexpr int N = V::N;
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= p.rows) return;
+    const char* xr = p.x + (size_t)row * p.C * sizeof(IO);
+    char* yr = p.y + (size_t)row * p.C * sizeof(IO);
+    const int nv = p.C / N;
+    float f[VPL][N];
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+        const int v = lane + 32 * k;
+        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+        if (v < nv) raw = *reinterpret_cast<const uint4*>(xr + (size_t)v * 16);
+        V::unpack(raw, f[k]);
+#pragma unroll
+        for (int e = 0; e < N; ++e) s += f[k][e];
+    }
+    const float invC = 1.0f / (float)p.C;
+    const float mean = warp_sum(s) * invC;
+    float q = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+        if (lane + 32 * k < nv) {
+#pragma unroll
+            for (int e = 0; e < N; ++e) q = fmaf(f[k][e] - mean, f[k][e] - mean, q);
+        }
+    }
+    const float rstd = rsqrtf(warp_sum(q) * invC + p.eps);
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+        const int v = lane + 32 * k;
+        if (v < nv) {
+            float o[N];
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+                const int c = v * N + e;
+                o[e] = fmaf(__ldg(p.g + c), (f[k][e] - mean) * rstd, __ldg(p.b + c));
+            }
+            *reinterpret_cast<uint4*>(yr + (size_t)v * 16) = V::pack(o);
+        }
+    }
+}
+
 template <typename IO>
 __global__ void __launch_bounds__(256) layer_norm_kernel(const LayerNormParams p) {
     using V = Vec16<IO>;

@@ -113,63 +113,6 @@ __global__ void __launch_bounds__(256) qshift_vec_kernel(const QshiftParams p) {
     }
 }
 
-// Three Q-Shift mixes of one x (mu_r, mu_k, mu_v, as the projections of the
-// spatial-mix block need them) from one load of x and of its neighbour, into
-// three outputs; each output is bit-identical to qshift_vec_kernel's with the
-// same mu.  Same vector conditions as qshift_vec_kernel, and every mu
-// non-null.
-struct Qshift3Params {
-    QshiftParams base;  // x, BT, T, C, H, W, s, g (out and mu unused)
-    char* out[3];
-    const float* mu[3];
-};
-
-template <typename IO>
-__global__ void __launch_bounds__(256) qshift3_vec_kernel(const Qshift3Params q) {
-    using V = Vec16<IO>;
-    constexpr int N = V::N;
-    const QshiftParams& p = q.base;
-    const int UR = p.C / N;
-    const long long units = p.BT * UR;
-    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < units;
-         idx += (long long)gridDim.x * blockDim.x) {
-        const long long bt = idx / UR;
-        const int c = (int)(idx - bt * UR) * N;
-        const int t = (int)(bt % p.T);
-        const int h = t / p.W, w = t - (t / p.W) * p.W;
-        const size_t row = (size_t)bt * p.C;
-        float xv[N], xd[N];
-        V::unpack(__ldg(reinterpret_cast<const uint4*>(p.x + (row + c) * sizeof(IO))), xv);
-        const ShiftRule r0 = shift_rule(c, p.g, p.H, p.W, p.s);
-        const ShiftRule r1 = shift_rule(c + N - 1, p.g, p.H, p.W, p.s);
-        if (r0.off == r1.off && r0.use_w == r1.use_w && r0.lo == r1.lo && r0.hi == r1.hi) {
-            if (shift_ok(r0, h, w)) {
-                V::unpack(__ldg(reinterpret_cast<const uint4*>(
-                              p.x + (row + (long long)r0.off * p.C + c) * sizeof(IO))),
-                          xd);
-            } else {
-#pragma unroll
-                for (int e = 0; e < N; ++e) xd[e] = 0.0f;
-            }
-        } else {  // the vector straddles a channel-group boundary
-#pragma unroll
-            for (int e = 0; e < N; ++e) {
-                const ShiftRule re = shift_rule(c + e, p.g, p.H, p.W, p.s);
-                xd[e] = shift_ok(re, h, w)
-                            ? Io<IO>::ld1(p.x + (row + (long long)re.off * p.C + c + e) * sizeof(IO))
-                            : 0.0f;
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < 3; ++m) {
-            float o[N];
-#pragma unroll
-            for (int e = 0; e < N; ++e) o[e] = qs_mix(__ldg(q.mu[m] + c + e), xv[e], xd[e]);
-            *reinterpret_cast<uint4*>(q.out[m] + (row + c) * sizeof(IO)) = V::pack(o);
-        }
-    }
-}
-
 // Scalar path for any C and any element-aligned pointers.
 template <typename IO>
 __global__ void __launch_bounds__(256) qshift_scalar_kernel(const QshiftParams p) {

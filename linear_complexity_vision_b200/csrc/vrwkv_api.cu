@@ -264,6 +264,76 @@ size_t block_ws_slot(int B, int T, int C, vrwkv_dtype dtype) {
     return ((size_t)B * T * C * elem_bytes(dtype) + 255) / 256 * 256;
 }
 
+// Launch shape of the column-walking kernels (channel mix, Q-Shift mixes):
+// blocks of (tx vectors) x (ty rows), channel chunks of at most 256 vectors
+// along x, and along y one wave of CTAs (SMs x resident CTAs per SM, from the
+// occupancy of `kern`), each owning an equal share of the BT token rows.
+template <typename K>
+vrwkv_status column_launch(K kern, std::atomic<int>& occ, int UR, long long BT, dim3* grid, dim3* block) {
+    const int nchunks = (UR + 255) / 256;
+    int tx = (UR + nchunks - 1) / nchunks;
+    if (nchunks > 1) tx = (tx + 31) / 32 * 32;
+    const int ty = std::max(1, 256 / tx);
+    int o = occ.load(std::memory_order_relaxed);
+    if (o == 0) {
+        int nb = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, tx * ty, 0);
+        if (e != cudaSuccess) return cuda_status(e, "occupancy query");
+        o = std::max(1, nb);
+        occ.store(o, std::memory_order_relaxed);
+    }
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long row_groups = (BT + ty * kCmRows - 1) / (ty * kCmRows);
+    const long long gy = std::max<long long>(1, std::min<long long>(row_groups, (long long)sms * o / nchunks));
+    *grid = dim3((unsigned)nchunks, (unsigned)gy);
+    *block = dim3((unsigned)tx, (unsigned)ty);
+    return VRWKV_OK;
+}
+
+// Q-Shift mixes of one x into NMIX outputs by the column walker; false when
+// the vector conditions do not hold (the caller then takes another path).
+template <int NMIX>
+bool launch_qs_mix(const void* x, void* const* outs, const float* const* mus, int B, int H, int W, int C,
+                   int shift, double gamma, vrwkv_dtype dtype, cudaStream_t s, vrwkv_status* st) {
+    const int es = elem_bytes(dtype), nv = 16 / es;
+    const long long BT = (long long)B * H * W;
+    const int g = group_size(C, gamma);
+    if (C % nv != 0 || g % nv != 0 || BT > 0x7fffffffLL || !aligned(x, 16)) return false;
+    for (int m = 0; m < NMIX; ++m)
+        if (!aligned(outs[m], 16) || (mus[0] && !mus[m])) return false;
+    QsMixParams<NMIX> q;
+    ChannelMixParams& p = q.base;
+    p.x = static_cast<const char*>(x);
+    p.out = nullptr;
+    p.mu_r = p.mu_k = nullptr;
+    p.BT = (int)BT;
+    p.T = H * W;
+    p.C = C;
+    p.H = H;
+    p.W = W;
+    p.s = shift;
+    p.g = g;
+    p.UR = C / nv;
+    p.divT = make_fastdiv((unsigned)p.T);
+    p.divW = make_fastdiv((unsigned)W);
+    for (int m = 0; m < NMIX; ++m) {
+        q.out[m] = static_cast<char*>(outs[m]);
+        q.mu[m] = mus[0] ? mus[m] : nullptr;
+    }
+    static std::atomic<int> occ[2] = {{0}, {0}};
+    dim3 grid, block;
+    const int di = dtype == VRWKV_F32 ? 0 : 1;
+    *st = dtype == VRWKV_F32 ? column_launch(qs_mix_vec_kernel<float, NMIX>, occ[di], p.UR, BT, &grid, &block)
+                             : column_launch(qs_mix_vec_kernel<__nv_bfloat16, NMIX>, occ[di], p.UR, BT, &grid,
+                                             &block);
+    if (*st != VRWKV_OK) return true;
+    if (dtype == VRWKV_F32) qs_mix_vec_kernel<float, NMIX><<<grid, block, 0, s>>>(q);
+    else qs_mix_vec_kernel<__nv_bfloat16, NMIX><<<grid, block, 0, s>>>(q);
+    *st = cuda_status(cudaGetLastError(), "qs_mix kernel launch");
+    return true;
+}
+
 bool tma_disabled() {
     const char* e = getenv("VRWKV_DISABLE_TMA");
     return e && e[0] && e[0] != '0';
@@ -696,6 +766,12 @@ vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B, int 
     p.s = shift_pixel;
     p.g = group_size(C, gamma);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        vrwkv_status st = VRWKV_OK;
+        void* outs[1] = {out};
+        const float* mus[1] = {mu};
+        if (launch_qs_mix<1>(x, outs, mus, B, H, W, C, shift_pixel, gamma, dtype, s, &st)) return st;
+    }
     const bool vec = ((size_t)C * es) % 16 == 0 && aligned(x, 16) && aligned(out, 16);
     const long long work = vec ? p.BT * (C / (16 / es)) : p.BT * C;
     const int threads = 256;
@@ -761,32 +837,13 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
         return cuda_status(cudaGetLastError(), "channel_mix kernel launch");
     }
     p.UR = C / nv;
-    // Channel chunks of at most 256 vectors, rounded to whole warps when split.
-    const int nchunks = (p.UR + 255) / 256;
-    int tx = (p.UR + nchunks - 1) / nchunks;
-    if (nchunks > 1) tx = (tx + 31) / 32 * 32;
-    const int ty = std::max(1, 256 / tx);
-    // One wave of CTAs, each owning an equal share of the token rows.
     static std::atomic<int> occ[2] = {{0}, {0}};
-    int o = occ[dtype == VRWKV_F32 ? 0 : 1].load(std::memory_order_relaxed);
-    if (o == 0) {
-        int nb = 0;
-        cudaError_t e = dtype == VRWKV_F32
-            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, channel_mix_vec_kernel<float>, 256, 0)
-            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, channel_mix_vec_kernel<__nv_bfloat16>, 256, 0);
-        if (e != cudaSuccess) return cuda_status(e, "channel_mix occupancy query");
-        o = std::max(1, nb);
-        occ[dtype == VRWKV_F32 ? 0 : 1].store(o, std::memory_order_relaxed);
-    }
-    int sms = 148;
-    {
-        int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    const long long row_groups = ((long long)p.BT + ty * kCmRows - 1) / (ty * kCmRows);
-    const long long gy = std::max<long long>(1, std::min<long long>(row_groups, (long long)sms * o / nchunks));
-    dim3 grid((unsigned)nchunks, (unsigned)gy), block((unsigned)tx, (unsigned)ty);
+    dim3 grid, block;
+    const int di = dtype == VRWKV_F32 ? 0 : 1;
+    vrwkv_status st = dtype == VRWKV_F32
+        ? column_launch(channel_mix_vec_kernel<float>, occ[di], p.UR, p.BT, &grid, &block)
+        : column_launch(channel_mix_vec_kernel<__nv_bfloat16>, occ[di], p.UR, p.BT, &grid, &block);
+    if (st != VRWKV_OK) return st;
     if (dtype == VRWKV_F32) channel_mix_vec_kernel<float><<<grid, block, 0, s>>>(p);
     else channel_mix_vec_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(p);
     g_last_kernel = "channel_mix_vec_kernel";
@@ -856,31 +913,12 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     const float* mus[3] = {qs->mu_r, qs->mu_k, qs->mu_v};
     const void* wts[3] = {w_r, w_k, w_v};
     void* dst[3] = {bR, bK, bV};
-    const int g = group_size(C, qs->gamma);
-    const int nvec = 16 / es;
-    if (mus[0] && mus[1] && mus[2] && C % nvec == 0 && (long long)qs->H * qs->W <= 0x7fffffffLL) {
-        Qshift3Params q3;
-        q3.base.x = static_cast<const char*>(x);
-        q3.base.out = nullptr;
-        q3.base.mu = nullptr;
-        q3.base.BT = (long long)B * T;
-        q3.base.T = T;
-        q3.base.C = C;
-        q3.base.H = qs->H;
-        q3.base.W = qs->W;
-        q3.base.s = qs->shift_pixel;
-        q3.base.g = g;
-        for (int i = 0; i < 3; ++i) {
-            q3.out[i] = static_cast<char*>(sh[i]);
-            q3.mu[i] = mus[i];
-        }
-        const long long work = q3.base.BT * (C / nvec);
-        const long long blocks = std::min<long long>((work + 255) / 256, 148LL * 16);
-        if (dtype == VRWKV_F32) qshift3_vec_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(q3);
-        else qshift3_vec_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(q3);
-        vrwkv_status st = cuda_status(cudaGetLastError(), "qshift3 kernel launch");
-        if (st != VRWKV_OK) return st;
-    } else {
+    vrwkv_status qst = VRWKV_OK;
+    const bool walked = mus[0] && mus[1] && mus[2] &&
+                        launch_qs_mix<3>(x, sh, mus, B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma, dtype, s,
+                                         &qst);
+    if (walked && qst != VRWKV_OK) return qst;
+    if (!walked) {
         for (int i = 0; i < 3; ++i) {
             vrwkv_status st = vrwkv_qshift(x, sh[i], mus[i], B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
                                            dtype, stream);
@@ -908,8 +946,17 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     lp.eps = ln_eps;
     lp.vec = ((size_t)C * es) % 16 == 0;
     const unsigned blocks = (unsigned)((M + 7) / 8);
-    if (dtype == VRWKV_F32) layer_norm_kernel<float><<<blocks, 256, 0, s>>>(lp);
-    else layer_norm_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(lp);
+    const int vpl = lp.vec ? (int)(((size_t)C * es / 16 + 31) / 32) : 0;  // 16-byte vectors per lane
+    auto launch_ln = [&](auto io) {
+        using IO = decltype(io);
+        if (vpl >= 1 && vpl <= 1) layer_norm_reg_kernel<IO, 1><<<blocks, 256, 0, s>>>(lp);
+        else if (vpl == 2) layer_norm_reg_kernel<IO, 2><<<blocks, 256, 0, s>>>(lp);
+        else if (vpl >= 3 && vpl <= 4) layer_norm_reg_kernel<IO, 4><<<blocks, 256, 0, s>>>(lp);
+        else if (vpl >= 5 && vpl <= 8) layer_norm_reg_kernel<IO, 8><<<blocks, 256, 0, s>>>(lp);
+        else layer_norm_kernel<IO><<<blocks, 256, 0, s>>>(lp);
+    };
+    if (dtype == VRWKV_F32) launch_ln(float{});
+    else launch_ln(__nv_bfloat16{});
     st = cuda_status(cudaGetLastError(), "layer_norm_kernel launch");
     if (st == VRWKV_OK) g_last_kernel = "spatial_mix_block";
     return st;
