@@ -27,8 +27,11 @@
 //
 // Work decomposition.  A CTA owns batch row b, a slab of 16 channels and 256
 // tokens; T > 256 splits over a cluster of up to 16 CTAs (T <= 4096).  Thread
-// = 2 adjacent channels (packed float2) x 4 consecutive tokens; the 32 lanes
-// of a warp are 8 channel pairs x 4 consecutive chunks.  Inputs come straight
+// = 2 adjacent channels (packed float2) x 8 consecutive tokens; the 32 lanes
+// of a warp are 8 channel pairs x 4 consecutive chunks; 256 threads, two CTAs
+// per SM within 128 registers: the per-token forward states (round 1) and
+// prefix sums (round 2) wait in shared memory between the two walks, and p v
+// is recomputed from p and v instead of being kept.  Inputs come straight
 // from global memory: at each token step a warp reads four 16-channel rows.
 // Exponents are base 2 (log2 e is folded into k, u and w).
 #pragma once
@@ -44,9 +47,9 @@ namespace cg = cooperative_groups;
 
 constexpr int kCS = 16;                    // channels per CTA
 constexpr int kNP = kCS / 2;               // channel pairs
-constexpr int kL = 4;                      // tokens per thread
-constexpr int kThreads = 512;
-constexpr int kNW = kThreads / 32;         // 16 warps
+constexpr int kL = 8;                      // tokens per thread
+constexpr int kThreads = 256;
+constexpr int kNW = kThreads / 32;         // 8 warps
 constexpr int kTc = kThreads / kNP * kL;   // 256 tokens per CTA
 constexpr int kWarpTok = 4 * kL;           // 16 tokens per warp
 constexpr int kClusterMax = 16;
@@ -156,6 +159,11 @@ struct alignas(16) Scratch {
     float2 kMc[kNP];
 };
 
+// Per-token state between the two walks of a round, [token][thread]: R1 in
+// round 1, R2 (the first half of each slot) in round 2.
+constexpr size_t kStashBytes = sizeof(R1) * kL * kThreads;
+constexpr size_t kSmemBytes = sizeof(Scratch) + kStashBytes;
+
 template <typename IO>
 __device__ __forceinline__ float2 load_pair(const char* base, size_t row_elem, int cA, int C, bool ok_t,
                                             bool vec) {
@@ -181,12 +189,15 @@ __device__ __forceinline__ void store_pair(char* base, size_t row_elem, int cA, 
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) {
-    __shared__ Scratch S;
+__global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) {
+    extern __shared__ __align__(16) char smem_raw[];
+    Scratch& S = *reinterpret_cast<Scratch*>(smem_raw);
+    R1* stash1 = reinterpret_cast<R1*>(smem_raw + sizeof(Scratch));  // [kL][kThreads]
+    R2* stash2 = reinterpret_cast<R2*>(stash1);                      // [kL][kThreads], round 2
 
     const int tid = threadIdx.x;
     const int j = tid & 7;    // channel pair
-    const int q = tid >> 3;   // chunk within the CTA (0..63)
+    const int q = tid >> 3;   // chunk within the CTA (0..31)
     const int cq = q & 3;     // chunk within the warp
     const int warp = tid >> 5;
     const int rank = blockIdx.x;
@@ -205,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) 
     const float2 alpha = decay(lam2, 1.0f);
     const float2 eu = ex2(mul2(uv, f2(kLog2e)));
 
-    // ---- load k, v, g of the thread's 4 tokens -------------------------------
+    // ---- load k, v, g of the thread's 8 tokens -------------------------------
     const int s_tok = t0 + q * kL;
     float2 kk[kL], vv[kL], gg[kL];
     float2 mx = f2(-INFINITY);
@@ -234,26 +245,23 @@ __global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) 
     // a column chunk may hold no token of a padded channel: keep M finite
     Mcta = make_float2(Mcta.x == -INFINITY ? 0.f : Mcta.x, Mcta.y == -INFINITY ? 0.f : Mcta.y);
 
-    // ---- round 1: p, p v, thread-local sums ------------------------------------
-    float2 pp[kL], pv[kL];
+    // ---- round 1: p, thread-local sums (p v recomputed where needed) ----------
+    float2 pp[kL];
 #pragma unroll
-    for (int i = 0; i < kL; ++i) {
-        pp[i] = ex2(add2(kk[i], make_float2(-Mcta.x, -Mcta.y)));
-        pv[i] = mul2(pp[i], vv[i]);
-    }
+    for (int i = 0; i < kL; ++i) pp[i] = ex2(add2(kk[i], make_float2(-Mcta.x, -Mcta.y)));
     R1 lf = r1_zero(), lb = r1_zero();
 #pragma unroll
     for (int i = 0; i < kL; ++i) {  // forward: segment grows to the right
         lf.hpv = mul2(alpha, add2(lf.hpv, lf.apv));
         lf.hp = mul2(alpha, add2(lf.hp, lf.ap));
-        lf.apv = fma2(alpha, lf.apv, pv[i]);
+        lf.apv = fma2(alpha, lf.apv, mul2(pp[i], vv[i]));
         lf.ap = fma2(alpha, lf.ap, pp[i]);
     }
 #pragma unroll
     for (int i = kL - 1; i >= 0; --i) {  // backward: segment grows to the left
         lb.hpv = mul2(alpha, add2(lb.hpv, lb.apv));
         lb.hp = mul2(alpha, add2(lb.hp, lb.ap));
-        lb.apv = fma2(alpha, lb.apv, pv[i]);
+        lb.apv = fma2(alpha, lb.apv, mul2(pp[i], vv[i]));
         lb.ap = fma2(alpha, lb.ap, pp[i]);
     }
     // warp scan over the 4 chunks (lanes 8 apart)
@@ -306,15 +314,15 @@ __global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) 
     // cluster exchange 1: push the records into every peer's mailbox (one
     // (peer, pair, part) per thread), then one cluster barrier
     if (multi) {
-        const int peer = tid >> 5, jj = (tid >> 2) & 7, part = tid & 3;
-        if (peer < p.ncl && part < 3) {
-            cg::cluster_group cluster = cg::this_cluster();
+        cg::cluster_group cluster = cg::this_cluster();
+        for (int e = tid; e < p.ncl * kNP * 3; e += kThreads) {  // (peer, pair, part)
+            const int peer = e / (kNP * 3), jj = (e / 3) % kNP, part = e % 3;
             Scratch* P = cluster.map_shared_rank(&S, peer);
             if (part == 0) P->mb1F[rank][jj] = S.own1F[jj];
             else if (part == 1) P->mb1B[rank][jj] = S.own1B[jj];
             else P->mbM[rank][jj] = S.ownM[jj];
         }
-        cg::this_cluster().sync();
+        cluster.sync();
     }
     // carries into this CTA: one thread per (channel, direction), a fixed-order
     // fold over the peers in the common exponent frame Mc
@@ -358,27 +366,26 @@ __global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) 
         KB = r1_cross(KB, decay(lam2, Ll2), Ll2, r1_scale(Y1, sl));
     }
 #pragma unroll
-    for (int i = 0; i < kL; ++i) {  // p, p v in the common frame
-        pp[i] = mul2(pp[i], sl);
-        pv[i] = mul2(pv[i], sl);
-    }
-    R1 fw[kL];  // forward sums at each token (over tokens before it)
+    for (int i = 0; i < kL; ++i) pp[i] = mul2(pp[i], sl);  // p in the common frame
+    // forward sums at each token (over the tokens before it), kept in the stash
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
-        fw[i] = KF;
+        stash1[i * kThreads + tid] = KF;
         KF.hpv = mul2(alpha, add2(KF.hpv, KF.apv));
         KF.hp = mul2(alpha, add2(KF.hp, KF.ap));
-        KF.apv = fma2(alpha, KF.apv, pv[i]);
+        KF.apv = fma2(alpha, KF.apv, mul2(pp[i], vv[i]));
         KF.ap = fma2(alpha, KF.ap, pp[i]);
     }
     float2 qq[kL], rr[kL];
     float2 gwa = f2(0.f), gua = f2(0.f);
 #pragma unroll
     for (int i = kL - 1; i >= 0; --i) {
-        const float2 N = add2(add2(fw[i].apv, KB.apv), mul2(eu, pv[i]));
-        const float2 D = add2(add2(fw[i].ap, KB.ap), mul2(eu, pp[i]));
-        const float2 HN = add2(fw[i].hpv, KB.hpv);
-        const float2 HD = add2(fw[i].hp, KB.hp);
+        const R1 fw = stash1[i * kThreads + tid];
+        const float2 pvi = mul2(pp[i], vv[i]);
+        const float2 N = add2(add2(fw.apv, KB.apv), mul2(eu, pvi));
+        const float2 D = add2(add2(fw.ap, KB.ap), mul2(eu, pp[i]));
+        const float2 HN = add2(fw.hpv, KB.hpv);
+        const float2 HD = add2(fw.hp, KB.hp);
         const float2 rD = rcp(D);
         const float2 y = mul2(N, rD);
         // Tokens past T (padding of the last CTA) take no part: their forward
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) 
         }
         KB.hpv = mul2(alpha, add2(KB.hpv, KB.apv));
         KB.hp = mul2(alpha, add2(KB.hp, KB.ap));
-        KB.apv = fma2(alpha, KB.apv, pv[i]);
+        KB.apv = fma2(alpha, KB.apv, pvi);
         KB.ap = fma2(alpha, KB.ap, pp[i]);
     }
 
@@ -467,16 +474,16 @@ __global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) 
     }
     __syncthreads();
     if (multi) {
-        const int peer = tid >> 5, jj = (tid >> 2) & 7, part = tid & 3;
-        if (peer < p.ncl) {
-            cg::cluster_group cluster = cg::this_cluster();
+        cg::cluster_group cluster = cg::this_cluster();
+        for (int e = tid; e < p.ncl * kNP * 4; e += kThreads) {  // (peer, pair, part)
+            const int peer = e / (kNP * 4), jj = (e / 4) % kNP, part = e % 4;
             Scratch* P = cluster.map_shared_rank(&S, peer);
             if (part == 0) P->mb2F[rank][jj] = S.own2F[jj];
             else if (part == 1) P->mb2B[rank][jj] = S.own2B[jj];
             else if (part == 2) P->mbW[rank][jj] = S.ownW[jj];
             else P->mbU[rank][jj] = S.ownU[jj];
         }
-        cg::this_cluster().sync();
+        cluster.sync();
     }
     if (tid < 2 * kCS) {
         const int lc = tid & 15, dir = tid >> 4, jj = lc >> 1, hi = lc & 1;
@@ -520,17 +527,17 @@ __global__ void __launch_bounds__(kThreads, 1) biwkv_bwd_kernel(const Params p) 
         const float2 aLn2 = decay(lam2, (float)(kL * (3 - cq)));
         QB = r2_cross(r2_cross(S.k2B[j], aW2, S.c2B[j][warp]), aLn2, Y2);
     }
-    R2 fq[kL];
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
-        fq[i] = QF;
+        stash2[i * kThreads + tid] = QF;
         QF.aq = fma2(alpha, QF.aq, qq[i]);
         QF.ar = fma2(alpha, QF.ar, rr[i]);
     }
 #pragma unroll
     for (int i = kL - 1; i >= 0; --i) {
-        const float2 Sq = fma2(eu, qq[i], add2(fq[i].aq, QB.aq));
-        const float2 Sr = fma2(eu, rr[i], add2(fq[i].ar, QB.ar));
+        const R2 fq = stash2[i * kThreads + tid];
+        const float2 Sq = fma2(eu, qq[i], add2(fq.aq, QB.aq));
+        const float2 Sr = fma2(eu, rr[i], add2(fq.ar, QB.ar));
         const float2 dv = mul2(pp[i], Sq);
         const float2 dk = fma2(vv[i], dv, mul2(make_float2(-pp[i].x, -pp[i].y), Sr));
         const int t = s_tok + i;

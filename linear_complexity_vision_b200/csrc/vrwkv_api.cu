@@ -1042,9 +1042,15 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
     for (const void* t : toks) p.vec = p.vec && aligned(t, 2 * es);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto kern = dtype == VRWKV_F32 ? bwd::biwkv_bwd_kernel<float> : bwd::biwkv_bwd_kernel<__nv_bfloat16>;
+    {
+        static std::atomic<int> granted[2] = {{0}, {0}};
+        cudaError_t e = ensure_smem(kern, granted[dtype == VRWKV_F32 ? 0 : 1], (int)bwd::kSmemBytes);
+        if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.ncl, (C + bwd::kCS - 1) / bwd::kCS, B);
     cfg.blockDim = dim3(bwd::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = bwd::kSmemBytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
