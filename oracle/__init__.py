@@ -27,6 +27,9 @@ It wraps ``vrwkv_oracle.c`` (plain C, float64, OpenMP over channel columns):
 * ``spatial_mix_block`` -- the spatial-mix block with projections: Q-Shift,
                        R/K/V projections (eq. 1), Bi-WKV and the sigma gate
                        (eq. 5, eq. 2), output projection W_O and LayerNorm.
+* ``bishift``, ``bishift_f32`` -- the bidirectional shift for sparse (MAE)
+                       inputs: Q-Shift's two row groups only, other channels
+                       unchanged (a reading; see the C source).
 * ``channel_mix``   -- sigma(QS_R(x)) * max(QS_K(x), 0)^2, the channel-mix
                        module of eq. 3-4 without projections.
 * ``spatial_core_points`` -- the same at selected output positions only, by
@@ -82,6 +85,8 @@ def _load():
         lib.oracle_biwkv_bwd_direct.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, dp, dp, dp, dp]
         lib.oracle_biwkv_bwd_columns.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ctypes.c_void_p,
                                                  ctypes.c_long, dp, dp, dp, dp, dp]
+        lib.oracle_bishift_f64.argtypes = [dp, dp, dp, ci, ci, ci, ci, ci, cd]
+        lib.oracle_bishift_f32.argtypes = [ctypes.POINTER(ctypes.c_float)] * 3 + [ci, ci, ci, ci, ci, cd, ci]
         lib.oracle_channel_mix.argtypes = [dp, dp, dp, dp, ci, ci, ci, ci, ci, cd]
         lib.oracle_spatial_core_points.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, ci,
                                                    ci, ci, cd, ci, ci, i64p, cl, dp]
@@ -311,3 +316,29 @@ def spatial_mix_block(x, w_r, w_k, w_v, w_o, w, u, mu_r, mu_k, mu_v, ln_g, ln_b,
     core = rnd(gate(R, f(K, V, w, u)))
     O = rnd(core @ _d(w_o))
     return layer_norm(O, ln_g, ln_b, eps)
+
+
+def bishift(x, H, W, shift_pixel=1, gamma=0.25, mu=None) -> np.ndarray:
+    """Bidirectional shift (sparse-input Q-Shift): [0, g) from w - s,
+    [g, 2g) from w + s (zero past the row), other channels unchanged; or the
+    mu interpolation with x, in float64."""
+    x = _d(x)
+    B, T, C = x.shape
+    assert T == H * W
+    out = np.empty_like(x)
+    _load().oracle_bishift_f64(_ptr(x), _ptr(out), None if mu is None else _ptr(_d(mu)), B, H, W, C,
+                               int(shift_pixel), float(gamma))
+    return out
+
+
+def bishift_f32(x, H, W, shift_pixel=1, gamma=0.25, mu=None, round_bf16=False) -> np.ndarray:
+    """bishift in binary32 with the fixed operation order of qshift_f32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    B, T, C = x.shape
+    out = np.empty_like(x)
+    fp = ctypes.POINTER(ctypes.c_float)
+    m = None if mu is None else np.ascontiguousarray(mu, dtype=np.float32)
+    _load().oracle_bishift_f32(_ptr(x, ctypes.c_float), _ptr(out, ctypes.c_float),
+                               None if m is None else _ptr(m, ctypes.c_float), B, H, W, C,
+                               int(shift_pixel), float(gamma), int(round_bf16))
+    return out

@@ -544,3 +544,70 @@ void oracle_biwkv_bwd_columns(const double* k, const double* v,
         free(buf);
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* Bidirectional shift for sparse (MAE) inputs                          */
+/* ------------------------------------------------------------------ */
+/* The pages pre-train with MAE after changing Q-Shift into a bidirectional
+ * shift, and say no more.  Reading taken: of Q-Shift's four channel groups
+ * only the two that shift along the token row remain -- [0, g) from token
+ * w-s, [g, 2g) from token w+s, zero past the row's ends -- and every other
+ * channel, the two vertical groups included, passes through unchanged.  A
+ * sparse input is one row of its visible tokens (H = 1, W = their count). */
+static int bishift_source(int c, int h, int w, int W, int C, int s,
+                          double gamma, int* sh, int* sw) {
+    int g = (int)((double)C * gamma);
+    int srcw = w;
+    if (c < g) srcw = w - s;
+    else if (c < 2 * g) srcw = w + s;
+    if (srcw < 0 || srcw >= W) return 0;
+    *sh = h;
+    *sw = srcw;
+    return 1;
+}
+
+void oracle_bishift_f64(const double* x, double* out, const double* mu, int B,
+                        int H, int W, int C, int s, double gamma) {
+    const long T = (long)H * W;
+#pragma omp parallel for schedule(static)
+    for (long bt = 0; bt < (long)B * T; ++bt) {
+        long b = bt / T, t = bt % T;
+        int h = (int)(t / W), w = (int)(t % W);
+        for (int c = 0; c < C; ++c) {
+            int sh, sw;
+            double xd = 0.0;
+            if (bishift_source(c, h, w, W, C, s, gamma, &sh, &sw))
+                xd = x[(b * T + (long)sh * W + sw) * C + c];
+            double xv = x[(b * T + t) * C + c];
+            out[(b * T + t) * C + c] = mu ? mu[c] * xv + (1.0 - mu[c]) * xd : xd;
+        }
+    }
+}
+
+/* The same with the binary32 operation order of oracle_qshift_f32. */
+void oracle_bishift_f32(const float* x, float* out, const float* mu, int B,
+                        int H, int W, int C, int s, double gamma,
+                        int round_bf16) {
+    const long T = (long)H * W;
+#pragma omp parallel for schedule(static)
+    for (long bt = 0; bt < (long)B * T; ++bt) {
+        long b = bt / T, t = bt % T;
+        int h = (int)(t / W), w = (int)(t % W);
+        for (int c = 0; c < C; ++c) {
+            int sh, sw;
+            float xd = 0.0f;
+            if (bishift_source(c, h, w, W, C, s, gamma, &sh, &sw))
+                xd = x[(b * T + (long)sh * W + sw) * C + c];
+            float r;
+            if (mu) {
+                volatile float t1 = mu[c] * x[(b * T + t) * C + c];
+                volatile float om = 1.0f - mu[c];
+                volatile float t2 = om * xd;
+                r = t1 + t2;
+            } else {
+                r = xd;
+            }
+            out[(b * T + t) * C + c] = round_bf16 ? round_to_bf16(r) : r;
+        }
+    }
+}
