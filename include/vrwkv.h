@@ -79,7 +79,19 @@ typedef enum {
  *   mu_r, mu_k, mu_v  device float32[C] interpolation weights, each nullable.
  *                With mu the shifted input is mu*x + (1-mu)*x_shift; a NULL
  *                mu means the shifted tensor x_shift itself.
+ *   mode         VRWKV_QSHIFT_QUAD, or VRWKV_QSHIFT_BIDIR for sparse inputs:
+ *                the pages pre-train with MAE after turning Q-Shift into a
+ *                bidirectional shift and say no more; this mode keeps the two
+ *                row groups ([0,g) from x[h, w-s], [g,2g) from x[h, w+s], zero
+ *                past the row) and passes every other channel through.  A
+ *                sparse input is one row of its visible tokens (H = 1).
  */
+typedef enum {
+    VRWKV_QSHIFT_QUAD = 0,  /* Q-Shift, eq. 9: four shifted channel groups   */
+    VRWKV_QSHIFT_BIDIR = 1  /* bidirectional shift for sparse (MAE) inputs: */
+                            /* the two row groups only                      */
+} vrwkv_qshift_mode;
+
 typedef struct {
     int H;
     int W;
@@ -88,6 +100,7 @@ typedef struct {
     const float* mu_r;
     const float* mu_k;
     const float* mu_v;
+    int mode;  /* vrwkv_qshift_mode */
 } vrwkv_qshift_params;
 
 /*
@@ -105,6 +118,15 @@ typedef struct {
 vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B,
                           int H, int W, int C, int shift_pixel, double gamma,
                           vrwkv_dtype dtype, void* stream);
+
+/*
+ * vrwkv_bishift -- the VRWKV_QSHIFT_BIDIR shift of one tensor (see
+ * vrwkv_qshift_params.mode); arguments, mix, exactness and errors as
+ * vrwkv_qshift.
+ */
+vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
+                           int H, int W, int C, int shift_pixel, double gamma,
+                           vrwkv_dtype dtype, void* stream);
 
 /*
  * vrwkv_biwkv_fwd -- Bi-WKV forward (eq. 5):

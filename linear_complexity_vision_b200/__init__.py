@@ -6,6 +6,7 @@ CUDA kernels.  PyTorch provides device memory and the current stream only.
 There is no fallback: if the library is missing, the calls raise.
 
     qshift(x, H, W, shift_pixel=1, gamma=0.25, mu=None)
+    bishift(x, H, W, shift_pixel=1, gamma=0.25, mu=None)  # sparse (MAE) inputs
     biwkv_fwd(k, v, w, u, qs=None, workspace=None)
     spatial_gate(r, k, v, w, u, qs=None, workspace=None)
     fwd_workspace(B, T, C, device)  # a zeroed workspace for the two calls above
@@ -47,7 +48,7 @@ class VrwkvError(RuntimeError):
 class _QsParams(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int), ("W", ctypes.c_int), ("shift_pixel", ctypes.c_int),
                 ("gamma", ctypes.c_double), ("mu_r", ctypes.c_void_p),
-                ("mu_k", ctypes.c_void_p), ("mu_v", ctypes.c_void_p)]
+                ("mu_k", ctypes.c_void_p), ("mu_v", ctypes.c_void_p), ("mode", ctypes.c_int)]
 
 
 def load_library():
@@ -62,6 +63,8 @@ def load_library():
         vp, ci, cd = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         lib.vrwkv_qshift.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cd, ci, vp]
         lib.vrwkv_qshift.restype = ci
+        lib.vrwkv_bishift.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cd, ci, vp]
+        lib.vrwkv_bishift.restype = ci
         for name in ("vrwkv_biwkv_fwd",):
             getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                            ctypes.POINTER(_QsParams), vp]
@@ -121,12 +124,13 @@ class QShift:
     mu_r: Optional[object] = None
     mu_k: Optional[object] = None
     mu_v: Optional[object] = None
+    mode: int = 0  # 0: Q-Shift (eq. 9); 1: bidirectional shift for sparse (MAE) inputs
 
     def _struct(self) -> _QsParams:
         def ptr(t):
             return None if t is None else t.data_ptr()
         return _QsParams(int(self.H), int(self.W), int(self.shift_pixel), float(self.gamma),
-                         ptr(self.mu_r), ptr(self.mu_k), ptr(self.mu_v))
+                         ptr(self.mu_r), ptr(self.mu_k), ptr(self.mu_v), int(self.mode))
 
 
 def _dtype_code(t) -> int:
@@ -156,6 +160,20 @@ def qshift(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25, mu=None
     if out is None:
         out = torch.empty_like(x)
     _check(load_library().vrwkv_qshift(
+        x.data_ptr(), out.data_ptr(), None if mu is None else mu.data_ptr(), B, H, W, C,
+        shift_pixel, float(gamma), _dtype_code(x), _stream_ptr(x)))
+    return out
+
+
+def bishift(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25, mu=None, out=None):
+    """The bidirectional shift of sparse (MAE) inputs (QShift mode 1) of x
+    (B, H*W, C): the shifted tensor, or mu*x + (1-mu)*shifted."""
+    import torch
+    _require(x, "x")
+    B, T, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(load_library().vrwkv_bishift(
         x.data_ptr(), out.data_ptr(), None if mu is None else mu.data_ptr(), B, H, W, C,
         shift_pixel, float(gamma), _dtype_code(x), _stream_ptr(x)))
     return out

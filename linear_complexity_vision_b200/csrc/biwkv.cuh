@@ -59,6 +59,7 @@ struct FusedParams {
     char* out;
     int B, T, C;
     int H, W, s, g;   // Q-Shift grid, shift and group size
+    int ng;           // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
     int Tc;           // tokens per CTA (multiple of 32 when ncl > 1)
     int ncl;          // CTAs per (b, slab) column = cluster size
     int halo;         // tile rows before and after the CTA's own tokens
@@ -210,8 +211,8 @@ __global__ void __launch_bounds__(512, 1) biwkv_fused_kernel(const __grid_consta
     float2 kcm = f2(kLog2e), kcd = f2(0.0f), vcm = f2(1.0f), vcd = f2(0.0f);
     float2 rcm = f2(-kLog2e), rcd = f2(0.0f);
     if (QS) {
-        ra = shift_rule(cA, p.g, p.H, p.W, p.s);
-        rb = okB ? shift_rule(cB, p.g, p.H, p.W, p.s) : ra;
+        ra = shift_rule(cA, p.g, p.ng, p.H, p.W, p.s);
+        rb = okB ? shift_rule(cB, p.g, p.ng, p.H, p.W, p.s) : ra;
         split = !(ra.off == rb.off && ra.use_w == rb.use_w && ra.lo == rb.lo && ra.hi == rb.hi);
         auto coef = [&](const float* mu, float scale, float2& cm, float2& cd) {
             float2 m = make_float2(0.0f, 0.0f);

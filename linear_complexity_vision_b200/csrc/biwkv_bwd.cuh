@@ -159,9 +159,11 @@ struct alignas(16) Scratch {
     float2 kMc[kNP];
 };
 
-// Per-token state between the two walks of a round, [token][thread]: R1 in
-// round 1, R2 (the first half of each slot) in round 2.
-constexpr size_t kStashBytes = sizeof(R1) * kL * kThreads;
+// Per-token state between the two walks of a round, as two 16-byte planes
+// [token][thread] (a thread's accesses are 16 bytes at a 16-byte stride:
+// bank-conflict free): round 1 keeps (apv, ap) in plane 0 and (hpv, hp) in
+// plane 1; round 2 keeps (aq, ar) in plane 0.
+constexpr size_t kStashBytes = 2 * sizeof(float4) * kL * kThreads;
 constexpr size_t kSmemBytes = sizeof(Scratch) + kStashBytes;
 
 template <typename IO>
@@ -192,8 +194,8 @@ template <typename IO>
 __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) {
     extern __shared__ __align__(16) char smem_raw[];
     Scratch& S = *reinterpret_cast<Scratch*>(smem_raw);
-    R1* stash1 = reinterpret_cast<R1*>(smem_raw + sizeof(Scratch));  // [kL][kThreads]
-    R2* stash2 = reinterpret_cast<R2*>(stash1);                      // [kL][kThreads], round 2
+    float4* plane0 = reinterpret_cast<float4*>(smem_raw + sizeof(Scratch));  // [kL][kThreads]
+    float4* plane1 = plane0 + kL * kThreads;
 
     const int tid = threadIdx.x;
     const int j = tid & 7;    // channel pair
@@ -370,7 +372,8 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) 
     // forward sums at each token (over the tokens before it), kept in the stash
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
-        stash1[i * kThreads + tid] = KF;
+        plane0[i * kThreads + tid] = make_float4(KF.apv.x, KF.apv.y, KF.ap.x, KF.ap.y);
+        plane1[i * kThreads + tid] = make_float4(KF.hpv.x, KF.hpv.y, KF.hp.x, KF.hp.y);
         KF.hpv = mul2(alpha, add2(KF.hpv, KF.apv));
         KF.hp = mul2(alpha, add2(KF.hp, KF.ap));
         KF.apv = fma2(alpha, KF.apv, mul2(pp[i], vv[i]));
@@ -380,7 +383,12 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) 
     float2 gwa = f2(0.f), gua = f2(0.f);
 #pragma unroll
     for (int i = kL - 1; i >= 0; --i) {
-        const R1 fw = stash1[i * kThreads + tid];
+        const float4 s0 = plane0[i * kThreads + tid], s1 = plane1[i * kThreads + tid];
+        R1 fw;
+        fw.apv = make_float2(s0.x, s0.y);
+        fw.ap = make_float2(s0.z, s0.w);
+        fw.hpv = make_float2(s1.x, s1.y);
+        fw.hp = make_float2(s1.z, s1.w);
         const float2 pvi = mul2(pp[i], vv[i]);
         const float2 N = add2(add2(fw.apv, KB.apv), mul2(eu, pvi));
         const float2 D = add2(add2(fw.ap, KB.ap), mul2(eu, pp[i]));
@@ -529,13 +537,16 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) 
     }
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
-        stash2[i * kThreads + tid] = QF;
+        plane0[i * kThreads + tid] = make_float4(QF.aq.x, QF.aq.y, QF.ar.x, QF.ar.y);
         QF.aq = fma2(alpha, QF.aq, qq[i]);
         QF.ar = fma2(alpha, QF.ar, rr[i]);
     }
 #pragma unroll
     for (int i = kL - 1; i >= 0; --i) {
-        const R2 fq = stash2[i * kThreads + tid];
+        const float4 s0 = plane0[i * kThreads + tid];
+        R2 fq;
+        fq.aq = make_float2(s0.x, s0.y);
+        fq.ar = make_float2(s0.z, s0.w);
         const float2 Sq = fma2(eu, qq[i], add2(fq.aq, QB.aq));
         const float2 Sr = fma2(eu, rr[i], add2(fq.ar, QB.ar));
         const float2 dv = mul2(pp[i], Sq);

@@ -75,6 +75,7 @@ struct alignas(64) Params {
     int B, T, C;
     int H, W, s, g;      // Q-Shift grid, shift, group size
     int gslab;           // group size in 16-channel slabs (g / 16; 0 if g == 0)
+    int ng;              // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
     float invT;          // 1 / T
     int Tc;              // tokens per CTA (multiple of 32 when ncl > 1)
     int rows;            // image rows per CTA (Q-Shift path): Tc = rows * W
@@ -298,6 +299,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     int grp = 4;
     if (QS && p.gslab > 0)
         grp = (slab >= p.gslab) + (slab >= 2 * p.gslab) + (slab >= 3 * p.gslab) + (slab >= 4 * p.gslab);
+    if (grp >= p.ng) grp = 4;
     const bool shifted = QS && grp < 4;
 
     // ---- issue the tile loads: lane i of warp 0 loads sub-tile i of each tile

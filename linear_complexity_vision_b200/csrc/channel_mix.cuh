@@ -52,6 +52,7 @@ struct ChannelMixParams {
     const float* mu_k;  // nullable: QS_K(x) = x_shift
     int BT;             // B*T token rows, < 2^31
     int T, C, H, W, s, g;
+    int ng;             // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
     int UR;             // 16-byte vectors per token row
     FastDiv divT, divW;
 };
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(256, 3) channel_mix_vec_kernel(const ChannelMi
         col.muk[e] = p.mu_k ? __ldg(reinterpret_cast<const float2*>(p.mu_k + c0) + e) : f2(0.0f);
     }
     // Without mu the mix, xd + mu*(x - xd), is xd itself.
-    col.rule = shift_rule(c0, p.g, p.H, p.W, p.s);
+    col.rule = shift_rule(c0, p.g, p.ng, p.H, p.W, p.s);
     const long long Gy = gridDim.y;
     const int r0 = (int)((long long)p.BT * blockIdx.y / Gy);
     col.r1 = (int)((long long)p.BT * (blockIdx.y + 1) / Gy);
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(256) qs_mix_vec_kernel(const QsMixParams<NMIX>
     for (int m = 0; m < NMIX; ++m)
 #pragma unroll
         for (int e = 0; e < N; ++e) mu[m][e] = with_mu ? __ldg(q.mu[m] + c0 + e) : 0.0f;
-    const ShiftRule rule = shift_rule(c0, p.g, p.H, p.W, p.s);
+    const ShiftRule rule = shift_rule(c0, p.g, p.ng, p.H, p.W, p.s);
     const long long Gy = gridDim.y;
     const int r0 = (int)((long long)p.BT * blockIdx.y / Gy);
     const int r1 = (int)((long long)p.BT * (blockIdx.y + 1) / Gy);
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(256) channel_mix_scalar_kernel(const ChannelMi
         const int c = (int)(idx - bt * p.C);
         const int t = (int)(bt % p.T);
         const int h = t / p.W, w = t - h * p.W;
-        const ShiftRule rule = shift_rule(c, p.g, p.H, p.W, p.s);
+        const ShiftRule rule = shift_rule(c, p.g, p.ng, p.H, p.W, p.s);
         const float X = Io<IO>::ld1(p.x + idx * sizeof(IO));
         const float D = shift_ok(rule, h, w)
                             ? Io<IO>::ld1(p.x + (idx + (long long)rule.off * p.C) * sizeof(IO))

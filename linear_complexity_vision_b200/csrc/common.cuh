@@ -105,8 +105,12 @@ struct ShiftRule {
     int lo, hi;   // admissible [lo, hi) for the tested coordinate
 };
 
-__device__ __forceinline__ ShiftRule shift_rule(int c, int g, int H, int W, int s) {
+// ng = number of shifted groups: 4 for Q-Shift (eq. 9), 2 for the
+// bidirectional shift of sparse (MAE) inputs, whose vertical groups pass
+// their channels through unchanged.
+__device__ __forceinline__ ShiftRule shift_rule(int c, int g, int ng, int H, int W, int s) {
     int grp = (g > 0) ? min(c / g, 4) : 4;
+    if (grp >= ng) grp = 4;
     ShiftRule r;
     switch (grp) {
     case 0: r = {-s, 1, s, W}; break;          // from w - s

@@ -30,7 +30,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Rows of at most 32 * VPL 16-byte vectors: the warp holds its row in
 // registers, so each element is read once; mean and centred variance come
-// from the registers.
+// from the registers.  gamma and beta must be 16-byte aligned.
 template <typename IO, int VPL>
 __global__ void __launch_bounds__(256) layer_norm_reg_kernel(const LayerNormParams p) {
     using V = Vec16<IO>;
@@ -67,12 +67,18 @@ __global__ void __launch_bounds__(256) layer_norm_reg_kernel(const LayerNormPara
     for (int k = 0; k < VPL; ++k) {
         const int v = lane + 32 * k;
         if (v < nv) {
-            float o[N];
+            // gamma and beta of the vector's N channels as float4 loads
+            const float4* g4 = reinterpret_cast<const float4*>(p.g + v * N);
+            const float4* b4 = reinterpret_cast<const float4*>(p.b + v * N);
+            float gg[N], bb[N], o[N];
 #pragma unroll
-            for (int e = 0; e < N; ++e) {
-                const int c = v * N + e;
-                o[e] = fmaf(__ldg(p.g + c), (f[k][e] - mean) * rstd, __ldg(p.b + c));
+            for (int e = 0; e < N / 4; ++e) {
+                const float4 a = __ldg(g4 + e), c = __ldg(b4 + e);
+                gg[4 * e] = a.x; gg[4 * e + 1] = a.y; gg[4 * e + 2] = a.z; gg[4 * e + 3] = a.w;
+                bb[4 * e] = c.x; bb[4 * e + 1] = c.y; bb[4 * e + 2] = c.z; bb[4 * e + 3] = c.w;
             }
+#pragma unroll
+            for (int e = 0; e < N; ++e) o[e] = fmaf(gg[e], (f[k][e] - mean) * rstd, bb[e]);
             *reinterpret_cast<uint4*>(yr + (size_t)v * 16) = V::pack(o);
         }
     }

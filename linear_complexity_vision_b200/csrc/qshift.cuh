@@ -61,6 +61,7 @@ struct QshiftParams {
     const float* mu;  // nullable
     long long BT;     // B*T
     int T, C, H, W, s, g;
+    int ng;           // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
 };
 
 // Vector path: C*sizeof(IO) is a multiple of 16 and both pointers are
@@ -81,8 +82,8 @@ __global__ void __launch_bounds__(256) qshift_vec_kernel(const QshiftParams p) {
         const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.x + (row + c) * sizeof(IO)));
         float xv[N], xd[N];
         V::unpack(raw, xv);
-        const ShiftRule r0 = shift_rule(c, p.g, p.H, p.W, p.s);
-        const ShiftRule r1 = shift_rule(c + N - 1, p.g, p.H, p.W, p.s);
+        const ShiftRule r0 = shift_rule(c, p.g, p.ng, p.H, p.W, p.s);
+        const ShiftRule r1 = shift_rule(c + N - 1, p.g, p.ng, p.H, p.W, p.s);
         if (r0.off == r1.off && r0.use_w == r1.use_w && r0.lo == r1.lo && r0.hi == r1.hi) {
             if (shift_ok(r0, h, w)) {
                 const uint4 rd = __ldg(reinterpret_cast<const uint4*>(
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(256) qshift_vec_kernel(const QshiftParams p) {
         } else {  // the vector straddles a channel-group boundary
 #pragma unroll
             for (int e = 0; e < N; ++e) {
-                const ShiftRule re = shift_rule(c + e, p.g, p.H, p.W, p.s);
+                const ShiftRule re = shift_rule(c + e, p.g, p.ng, p.H, p.W, p.s);
                 xd[e] = shift_ok(re, h, w)
                             ? Io<IO>::ld1(p.x + (row + (long long)re.off * p.C + c + e) * sizeof(IO))
                             : 0.0f;
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(256) qshift_scalar_kernel(const QshiftParams p
         const int c = (int)(idx - bt * p.C);
         const int t = (int)(bt % p.T);
         const int h = t / p.W, w = t - (t / p.W) * p.W;
-        const ShiftRule r = shift_rule(c, p.g, p.H, p.W, p.s);
+        const ShiftRule r = shift_rule(c, p.g, p.ng, p.H, p.W, p.s);
         const float xd = shift_ok(r, h, w)
                              ? Io<IO>::ld1(p.x + (idx + (long long)r.off * p.C) * sizeof(IO))
                              : 0.0f;

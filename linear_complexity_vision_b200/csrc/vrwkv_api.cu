@@ -67,6 +67,11 @@ int elem_bytes(vrwkv_dtype dt) { return dt == VRWKV_F32 ? 4 : 2; }
 
 int group_size(int C, double gamma) { return (int)((double)C * gamma); }
 
+// Shifted channel groups of a Q-Shift mode: all four (eq. 9) or the two
+// row groups (bidirectional shift of sparse inputs).
+int shifted_groups(const vrwkv_qshift_params* qs) { return qs && qs->mode == VRWKV_QSHIFT_BIDIR ? 2 : 4; }
+
+
 // Raise the dynamic shared-memory limit of a kernel once per size needed.
 template <typename K>
 cudaError_t ensure_smem(K kernel, std::atomic<int>& granted, int bytes) {
@@ -295,7 +300,7 @@ vrwkv_status column_launch(K kern, std::atomic<int>& occ, int UR, long long BT, 
 // the vector conditions do not hold (the caller then takes another path).
 template <int NMIX>
 bool launch_qs_mix(const void* x, void* const* outs, const float* const* mus, int B, int H, int W, int C,
-                   int shift, double gamma, vrwkv_dtype dtype, cudaStream_t s, vrwkv_status* st) {
+                   int shift, double gamma, int ng, vrwkv_dtype dtype, cudaStream_t s, vrwkv_status* st) {
     const int es = elem_bytes(dtype), nv = 16 / es;
     const long long BT = (long long)B * H * W;
     const int g = group_size(C, gamma);
@@ -314,6 +319,7 @@ bool launch_qs_mix(const void* x, void* const* outs, const float* const* mus, in
     p.W = W;
     p.s = shift;
     p.g = g;
+    p.ng = ng;
     p.UR = C / nv;
     p.divT = make_fastdiv((unsigned)p.T);
     p.divW = make_fastdiv((unsigned)W);
@@ -501,6 +507,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         p.W = qs->W;
         p.s = qs->shift_pixel;
         p.g = group_size(C, qs->gamma);
+        p.ng = shifted_groups(qs);
         if (p.g % fast::kCS != 0 || p.W > 256 || p.W % fast::kL != 0) return false;
         if (T <= TcMax) {
             p.rows = p.H;
@@ -523,6 +530,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         p.W = T;
         p.s = 0;
         p.g = 0;
+        p.ng = 4;
         p.rows = 1;
         p.Tc = std::min(T, TcMax);
         p.ncl = (T + p.Tc - 1) / p.Tc;
@@ -591,6 +599,8 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
 }
 
 vrwkv_status check_qs(const vrwkv_qshift_params* qs, int T, int C) {
+    if (qs->mode != VRWKV_QSHIFT_QUAD && qs->mode != VRWKV_QSHIFT_BIDIR)
+        return fail(VRWKV_ERR_INVALID_ARG, "qs: unknown mode %d", qs->mode);
     if (qs->H <= 0 || qs->W <= 0) return fail(VRWKV_ERR_INVALID_ARG, "qs: H and W must be positive");
     if ((long long)qs->H * qs->W != T)
         return fail(VRWKV_ERR_INVALID_ARG, "qs: H*W (%lld) must equal T (%d)",
@@ -719,6 +729,7 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
     p.W = qs ? qs->W : T;
     p.s = qs ? qs->shift_pixel : 0;
     p.g = qs ? group_size(C, qs->gamma) : 0;
+    p.ng = shifted_groups(qs);
     bool vin = ((size_t)C * es) % 16 == 0;
     for (int i = 0; i < pl.ntiles; ++i) vin = vin && aligned(p.src[i], 16);
     p.vec_in = vin ? 1 : 0;
@@ -735,8 +746,8 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
 
 extern "C" {
 
-vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B, int H, int W, int C,
-                          int shift_pixel, double gamma, vrwkv_dtype dtype, void* stream) {
+vrwkv_status shift_entry(const void* x, void* out, const float* mu, int B, int H, int W, int C,
+                         int shift_pixel, double gamma, int ng, vrwkv_dtype dtype, void* stream) {
     if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
         return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     if (B <= 0 || H <= 0 || W <= 0 || C <= 0)
@@ -765,12 +776,13 @@ vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B, int 
     p.W = W;
     p.s = shift_pixel;
     p.g = group_size(C, gamma);
+    p.ng = ng;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     {
         vrwkv_status st = VRWKV_OK;
         void* outs[1] = {out};
         const float* mus[1] = {mu};
-        if (launch_qs_mix<1>(x, outs, mus, B, H, W, C, shift_pixel, gamma, dtype, s, &st)) return st;
+        if (launch_qs_mix<1>(x, outs, mus, B, H, W, C, shift_pixel, gamma, ng, dtype, s, &st)) return st;
     }
     const bool vec = ((size_t)C * es) % 16 == 0 && aligned(x, 16) && aligned(out, 16);
     const long long work = vec ? p.BT * (C / (16 / es)) : p.BT * C;
@@ -784,6 +796,16 @@ vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B, int 
         else qshift_scalar_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(p);
     }
     return cuda_status(cudaGetLastError(), "qshift kernel launch");
+}
+
+vrwkv_status vrwkv_qshift(const void* x, void* out, const float* mu, int B, int H, int W, int C,
+                          int shift_pixel, double gamma, vrwkv_dtype dtype, void* stream) {
+    return shift_entry(x, out, mu, B, H, W, C, shift_pixel, gamma, 4, dtype, stream);
+}
+
+vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B, int H, int W, int C,
+                           int shift_pixel, double gamma, vrwkv_dtype dtype, void* stream) {
+    return shift_entry(x, out, mu, B, H, W, C, shift_pixel, gamma, 2, dtype, stream);
 }
 
 vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vrwkv_dtype dtype,
@@ -809,6 +831,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
     p.W = T;
     p.s = 0;
     p.g = 0;  // without qs every channel reads its own token: QS is the identity
+    p.ng = 4;
     if (qs) {
         vrwkv_status st = check_qs(qs, T, C);
         if (st != VRWKV_OK) return st;
@@ -818,6 +841,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
         p.W = qs->W;
         p.s = qs->shift_pixel;
         p.g = group_size(C, qs->gamma);
+        p.ng = shifted_groups(qs);
         for (const float* m : {p.mu_r, p.mu_k})
             if (m && overlaps(out, nbytes, m, (size_t)C * 4))
                 return fail(VRWKV_ERR_INVALID_ARG, "output overlaps mu");
@@ -915,13 +939,13 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     void* dst[3] = {bR, bK, bV};
     vrwkv_status qst = VRWKV_OK;
     const bool walked = mus[0] && mus[1] && mus[2] &&
-                        launch_qs_mix<3>(x, sh, mus, B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma, dtype, s,
-                                         &qst);
+                        launch_qs_mix<3>(x, sh, mus, B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
+                                         shifted_groups(qs), dtype, s, &qst);
     if (walked && qst != VRWKV_OK) return qst;
     if (!walked) {
         for (int i = 0; i < 3; ++i) {
-            vrwkv_status st = vrwkv_qshift(x, sh[i], mus[i], B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
-                                           dtype, stream);
+            vrwkv_status st = shift_entry(x, sh[i], mus[i], B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
+                                          shifted_groups(qs), dtype, stream);
             if (st != VRWKV_OK) return st;
         }
     }
@@ -946,7 +970,9 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     lp.eps = ln_eps;
     lp.vec = ((size_t)C * es) % 16 == 0;
     const unsigned blocks = (unsigned)((M + 7) / 8);
-    const int vpl = lp.vec ? (int)(((size_t)C * es / 16 + 31) / 32) : 0;  // 16-byte vectors per lane
+    // 16-byte vectors per lane of the register-resident kernel (0: three-pass)
+    const int vpl = (lp.vec && aligned(ln_gamma, 16) && aligned(ln_beta, 16))
+                        ? (int)(((size_t)C * es / 16 + 31) / 32) : 0;
     auto launch_ln = [&](auto io) {
         using IO = decltype(io);
         if (vpl >= 1 && vpl <= 1) layer_norm_reg_kernel<IO, 1><<<blocks, 256, 0, s>>>(lp);
