@@ -33,11 +33,19 @@
 // prefix sums (round 2) wait in shared memory between the two walks, and p v
 // is recomputed from p and v instead of being kept.  Inputs come straight
 // from global memory: at each token step a warp reads four 16-channel rows.
+// Inputs of 16-byte-aligned tensors with C % 16 == 0 arrive by TMA in the
+// forward kernel's tile layout (element stride 8 along T: sub-tile i, row q is
+// token i of chunk q, so a warp's four chunks read four consecutive rows),
+// into shared memory that the per-token stash reuses afterwards; other
+// tensors load straight from global memory.
 // Exponents are base 2 (log2 e is folded into k, u and w).
 #pragma once
 
+#include <cuda.h>
+
 #include <cooperative_groups.h>
 
+#include "biwkv_tma.cuh"
 #include "common.cuh"
 
 namespace vrwkv {
@@ -54,7 +62,10 @@ constexpr int kTc = kThreads / kNP * kL;   // 256 tokens per CTA
 constexpr int kWarpTok = 4 * kL;           // 16 tokens per warp
 constexpr int kClusterMax = 16;
 
-struct Params {
+struct alignas(64) Params {
+    CUtensorMap map[3];  // k, v, g (TMA path)
+    unsigned int* err;   // device error word (bounded TMA wait)
+    int tma;             // inputs arrive by TMA
     const char* k;
     const char* v;
     const char* g;  // upstream gradient dL/dy
@@ -164,7 +175,10 @@ struct alignas(16) Scratch {
 // bank-conflict free): round 1 keeps (apv, ap) in plane 0 and (hpv, hp) in
 // plane 1; round 2 keeps (aq, ar) in plane 0.
 constexpr size_t kStashBytes = 2 * sizeof(float4) * kL * kThreads;
-constexpr size_t kSmemBytes = sizeof(Scratch) + kStashBytes;
+// the stash starts 128-byte aligned (it also receives the TMA tiles)
+constexpr size_t kStashOff = (sizeof(Scratch) + 127) / 128 * 128;
+constexpr size_t kSmemBytes = kStashOff + kStashBytes + 128;  // + re-alignment slack
+constexpr int kTileRows = kTc / kL;  // rows of one sub-tile (32)
 
 template <typename IO>
 __device__ __forceinline__ float2 load_pair(const char* base, size_t row_elem, int cA, int C, bool ok_t,
@@ -191,11 +205,13 @@ __device__ __forceinline__ void store_pair(char* base, size_t row_elem, int cA, 
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) {
-    extern __shared__ __align__(16) char smem_raw[];
-    Scratch& S = *reinterpret_cast<Scratch*>(smem_raw);
-    float4* plane0 = reinterpret_cast<float4*>(smem_raw + sizeof(Scratch));  // [kL][kThreads]
+__global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(128) char smem_raw[];
+    char* smem = smem_raw + ((128u - (fast::smem_u32(smem_raw) & 127u)) & 127u);
+    Scratch& S = *reinterpret_cast<Scratch*>(smem);
+    float4* plane0 = reinterpret_cast<float4*>(smem + kStashOff);  // [kL][kThreads]
     float4* plane1 = plane0 + kL * kThreads;
+    __shared__ unsigned long long tma_bar;
 
     const int tid = threadIdx.x;
     const int j = tid & 7;    // channel pair
@@ -211,6 +227,26 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) 
     const bool vec = p.vec != 0;
     const bool multi = p.ncl > 1;
 
+    // ---- TMA: lanes 0..7 of warp 0 load sub-tile i of k, v and g --------------
+    constexpr int es = Io<IO>::kBytes;
+    constexpr int RB = kCS * es;           // bytes per token row of a tile
+    constexpr int SUB = kTileRows * RB;    // bytes per sub-tile
+    constexpr int TILE = kL * SUB;         // bytes per tile
+    char* tiles = smem + kStashOff;        // k, v, g tiles (the stash later)
+    if (p.tma) {
+        if (tid == 0) fast::mbar_init(&tma_bar, 1);
+        __syncthreads();
+        if (warp == 0) {
+            if (tid == 0) fast::mbar_expect_tx(&tma_bar, (unsigned)(3 * TILE));
+            __syncwarp();
+            if (tid < kL) {
+#pragma unroll
+                for (int s3 = 0; s3 < 3; ++s3)
+                    fast::tma_load_3d(tiles + s3 * TILE + tid * SUB, &p.map[s3], c0, t0 + tid, b, &tma_bar);
+            }
+        }
+    }
+
     // ---- per-channel constants -----------------------------------------------
     const float2 wv = make_float2(cA < p.C ? __ldg(p.w + cA) : 0.f, cA + 1 < p.C ? __ldg(p.w + cA + 1) : 0.f);
     const float2 uv = make_float2(cA < p.C ? __ldg(p.u + cA) : 0.f, cA + 1 < p.C ? __ldg(p.u + cA + 1) : 0.f);
@@ -222,15 +258,36 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const Params p) 
     const int s_tok = t0 + q * kL;
     float2 kk[kL], vv[kL], gg[kL];
     float2 mx = f2(-INFINITY);
+    if (p.tma) {
+        if (tid == 0) fast::mbar_wait_bounded(&tma_bar, p.err);
+        __syncthreads();
+        const int rowoff = q * RB + j * 2 * es;  // token i of chunk q: + i * SUB
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            const int o = rowoff + i * SUB;
+            kk[i] = fast::lds_pair<IO>(tiles, o);
+            vv[i] = fast::lds_pair<IO>(tiles + TILE, o);
+            gg[i] = fast::lds_pair<IO>(tiles + 2 * TILE, o);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            const int t = s_tok + i;
+            const bool ok = t < tend;
+            const size_t row = ((size_t)b * p.T + t) * p.C;
+            kk[i] = load_pair<IO>(p.k, row, cA, p.C, ok, vec);
+            vv[i] = load_pair<IO>(p.v, row, cA, p.C, ok, vec);
+            gg[i] = load_pair<IO>(p.g, row, cA, p.C, ok, vec);
+        }
+    }
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
-        const int t = s_tok + i;
-        const bool ok = t < tend;
-        const size_t row = ((size_t)b * p.T + t) * p.C;
-        kk[i] = load_pair<IO>(p.k, row, cA, p.C, ok, vec);
-        vv[i] = load_pair<IO>(p.v, row, cA, p.C, ok, vec);
-        gg[i] = load_pair<IO>(p.g, row, cA, p.C, ok, vec);
+        // tokens past T: k = -inf makes p = 0; v and g are zero (TMA fill or
+        // the masked loads), except stale tile rows, hence the explicit masks
+        const bool ok = s_tok + i < tend;
         kk[i] = ok ? mul2(kk[i], f2(kLog2e)) : f2(-INFINITY);  // base 2; -inf => p = 0
+        vv[i] = ok ? vv[i] : f2(0.0f);
+        gg[i] = ok ? gg[i] : f2(0.0f);
         mx = max2(mx, kk[i]);
     }
     // CTA maximum of k per channel

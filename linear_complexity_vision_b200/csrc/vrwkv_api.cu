@@ -1066,6 +1066,28 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
     p.invT = (float)(1.0 / (double)T);
     p.vec = (C % 2 == 0);
     for (const void* t : toks) p.vec = p.vec && aligned(t, 2 * es);
+    // k, v and gy by TMA (tiles of 16 channels x 256 tokens, element stride 8
+    // along T, as the forward kernel's) when the shape and alignment allow
+    p.tma = 0;
+    p.err = device_error_word();
+    if (!tma_disabled() && C % bwd::kCS == 0 && p.err && aligned(k, 16) && aligned(v, 16) && aligned(gy, 16)) {
+        EncodeTiledFn enc = encode_fn();
+        if (enc) {
+            const void* srcs[3] = {k, v, gy};
+            const CUtensorMapDataType tdt =
+                dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+            const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+            const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
+            const cuuint32_t box[3] = {(cuuint32_t)bwd::kCS, (cuuint32_t)bwd::kTc, 1};
+            const cuuint32_t estr[3] = {1, (cuuint32_t)bwd::kL, 1};
+            bool okm = true;
+            for (int i = 0; i < 3 && okm; ++i)
+                okm = enc(&p.map[i], tdt, 3, const_cast<void*>(srcs[i]), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            p.tma = okm ? 1 : 0;
+        }
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto kern = dtype == VRWKV_F32 ? bwd::biwkv_bwd_kernel<float> : bwd::biwkv_bwd_kernel<__nv_bfloat16>;
     {
