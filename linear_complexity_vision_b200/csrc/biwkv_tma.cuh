@@ -127,6 +127,7 @@ struct alignas(16) Scratch {
     unsigned int gen;           // GX: the launch's generation
     float4 ccarry[kCS];         // per channel: carries Af, Cf, Bb, Db
     unsigned long long bar;     // TMA completion barrier
+    unsigned long long xbar;    // mailbox barrier: completes when every peer's record is in
 };
 
 // ---- PTX wrappers ----------------------------------------------------------
@@ -184,6 +185,44 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
 }
 __device__ __forceinline__ void cluster_arrive_release() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ unsigned mapa_u32(unsigned a, unsigned rank) {
+    unsigned r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+// Asynchronous store into another CTA's shared memory that completes its
+// bytes on that CTA's mbarrier (no fence, no cluster barrier).
+__device__ __forceinline__ void st_async4(unsigned raddr, float4 v, unsigned rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(raddr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rbar) : "memory");
+}
+__device__ __forceinline__ void st_async2(unsigned raddr, float2 v, unsigned rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+                 ::"r"(raddr), "f"(v.x), "f"(v.y), "r"(rbar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(unsigned long long* bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void mbar_wait_cluster_bounded(unsigned long long* bar, unsigned* err) {
+    if (mbar_try_wait_cluster(bar, 0)) return;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, 0)) {
+        if (clock64() - t0 > kWaitCycles) {
+            atomicOr(err, 1u);
+            return;
+        }
+    }
 }
 __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -270,12 +309,20 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     const int warp = tid >> 5;
     if (tid == 0) {
         mbar_init(&S.bar, 1);
+        if (!GX && p.ncl > 1) {
+            // the mailbox barrier: one arrival (here) plus every peer's bytes
+            mbar_init(&S.xbar, 1);
+            mbar_expect_tx(&S.xbar, (unsigned)(p.ncl * kNP * (sizeof(float4) * 2 + sizeof(float2))));
+        }
         if (GX) {
             S.tk = (int)atomicAdd(p.ws_ctl, 1u);
             S.gen = *reinterpret_cast<volatile unsigned int*>(p.ws_ctl + 2);
         }
     }
     __syncthreads();
+    // mailbox barriers initialised cluster-wide before anyone pushes: arrive
+    // now, wait just before the first push
+    if (!GX && p.ncl > 1) cluster_arrive_relaxed();
     // this CTA's column chunk: the block index, or (GX) the ticket
     int rank = blockIdx.x, slab = blockIdx.y, b = blockIdx.z;
     unsigned int gen = 0;
@@ -549,25 +596,25 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
                 }
             }
         } else {
-            // publish the record into every CTA's mailbox (its own included)
-            // with remote shared-memory stores, one (peer, pair, half) per
-            // thread; the cluster barrier below makes them visible
+            // asynchronous stores of the record into every CTA's mailbox (its
+            // own included), one (peer, pair, half) per thread, completing on
+            // the receiver's mailbox barrier
+            cluster_wait_acquire();  // every mailbox barrier is initialised
             const int peer = tid >> 4, jj = (tid >> 1) & 7;
             if (peer < p.ncl) {
-                cg::cluster_group cluster = cg::this_cluster();
-                Scratch* P = cluster.map_shared_rank(&S, peer);
+                const unsigned rbar = mapa_u32(smem_u32(&S.xbar), peer);
                 if ((tid & 1) == 0) {
-                    P->mbF[rank][jj] = S.ownF[jj];
+                    st_async4(mapa_u32(smem_u32(&S.mbF[rank][jj]), peer), S.ownF[jj], rbar);
                 } else {
-                    P->mbG[rank][jj] = S.ownG[jj];
-                    P->mbM[rank][jj] = S.ownM[jj];
+                    st_async4(mapa_u32(smem_u32(&S.mbG[rank][jj]), peer), S.ownG[jj], rbar);
+                    st_async2(mapa_u32(smem_u32(&S.mbM[rank][jj]), peer), S.ownM[jj], rbar);
                 }
             }
         }
     }
     if (p.ncl > 1 && !GX) {
-        cluster_arrive_release();
-        cluster_wait_acquire();
+        if (tid == 0) mbar_wait_cluster_bounded(&S.xbar, p.err);
+        __syncthreads();
     } else {
         __syncthreads();
     }
