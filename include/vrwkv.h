@@ -138,9 +138,9 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *   wkv   (B, T, C) output, same dtype, must not overlap k, v, w or u.
  *   qs    NULL, or Q-Shift parameters applied to k (mu_k) and v (mu_v) on
  *         load (mu_r is ignored); T must then equal qs->H * qs->W.
- * Kernels: a TMA fast path serves C % 16 == 0 with 16-byte-aligned inputs
+ * Kernels: a TMA fast path serves C % 8 == 0 with 16-byte-aligned inputs
  *   (and, with qs, a channel-group size int(C*gamma) that is a multiple of
- *   16 and W <= 256); everything else runs a generic kernel with the same
+ *   8 and W <= 256); everything else runs a generic kernel with the same
  *   results up to rounding.  Setting VRWKV_DISABLE_TMA=1 in the environment
  *   forces the generic kernel (diagnostics).
  * Limits: T <= 4096 (UNSUPPORTED above); on the generic kernel with qs, a
@@ -176,7 +176,7 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
 /*
  * Workspace variants of vrwkv_biwkv_fwd and vrwkv_spatial_gate.  Same
  * operations, arguments, results and limits; for sequences that span several
- * CTAs the CTAs of one (b, 16-channel) column exchange their partial sums
+ * CTAs the CTAs of one (b, 8-channel) column exchange their partial sums
  * through the caller's workspace instead of a thread-block cluster, which
  * frees the kernel from cluster co-scheduling (every SM can hold its full
  * share of CTAs).
@@ -215,7 +215,7 @@ vrwkv_status vrwkv_spatial_gate_ws(const void* r, const void* k, const void* v,
  * allocates nothing.  The pages have no counterpart of this entry point; it
  * exists only for such callers.
  * The workspace is one 4 MiB array per device, reserved when the library is
- * loaded, which holds the exchange state of B * ceil(C / 16) <= ~800 columns;
+ * loaded, which holds the exchange state of B * ceil(C / 8) <= ~1600 columns;
  * larger problems return VRWKV_ERR_UNSUPPORTED.  Each call first clears the
  * array's counters and flags on `stream` (cudaMemsetAsync), then runs the
  * workspace kernel; results equal vrwkv_spatial_gate's.

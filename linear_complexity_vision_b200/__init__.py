@@ -257,7 +257,7 @@ def channel_mix(x, qs: Optional[QShift] = None, out=None):
 def spatial_gate_static(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
     """spatial_gate for callers that cannot allocate device memory: the
     column exchange runs in a fixed workspace the library reserved at load
-    time (up to ~800 (batch row, 16-channel) columns).  Calls overlapping in
+    time (up to ~1600 (batch row, 8-channel) columns).  Calls overlapping in
     time on other streams share that workspace and race."""
     import torch
     for t, name in ((r, "r"), (k, "k"), (v, "v"), (w, "w"), (u, "u")):

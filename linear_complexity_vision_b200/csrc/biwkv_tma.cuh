@@ -20,12 +20,13 @@
 //    set of boxes displaced by +-s along w or h.  TMA fills out-of-image
 //    elements with zeros, which is exactly Q-Shift's zero border, so no
 //    per-token shift arithmetic remains: token t of both tiles sits at the
-//    same shared-memory offset.  A CTA's 16 channels lie in one channel
-//    group (the host requires the group size to be a multiple of 16).
+//    same shared-memory offset.  A CTA's kCS channels lie in one channel
+//    group (the host requires the group size to be a multiple of kCS).
 //  * 256-thread CTAs at 64 registers per thread: four CTAs per SM, so one
 //    CTA's barriers and scans overlap another's arithmetic.  Sequences
-//    longer than 256 tokens split over a thread-block cluster of up to 16
-//    CTAs along T; CTA aggregates travel through distributed shared memory.
+//    longer than one CTA's span (256 kL / kNP tokens) split over a
+//    thread-block cluster of up to 16 CTAs along T; CTA aggregates travel
+//    through distributed shared memory.
 //  * Arrays that a warp reads down a column ([pair][warp], [peer][pair])
 //    have one element of row padding, so those reads are bank-conflict free.
 //  * Decay powers a^(8m) come from a per-CTA table (one exp2 each), the
@@ -44,21 +45,23 @@ namespace fast {
 
 namespace cg = cooperative_groups;
 
-constexpr int kCS = 16;         // channels per CTA
+constexpr int kCS = 8;          // channels per CTA (a column slab)
 constexpr int kNP = kCS / 2;    // channel pairs per CTA
 constexpr int kL = 8;           // tokens per thread chunk
+constexpr int kCPW = 32 / kNP;  // chunks per warp
+constexpr int kWarpTok = kCPW * kL;  // tokens per warp
 constexpr int kClusterMax = 16;
 constexpr int kExThreads = kCS * kClusterMax;  // threads of the cross-CTA exchange
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 
-// CTA shape: NT threads = 8 channel pairs x NT/8 chunks of 8 tokens, so a
-// CTA spans NT tokens, at 64 registers per thread (1024/NT CTAs per SM).  The
-// library launches NT = 256 (four CTAs per SM, clusters of up to 16 along T).
+// CTA shape: NT threads = kNP channel pairs x NT/kNP chunks of 8 tokens, at
+// 64 registers per thread (1024/NT CTAs per SM).  The library launches
+// NT = 256 (four CTAs per SM; clusters of up to 16 CTAs along T).
 template <int NT>
 struct Cfg {
     static constexpr int kThreads = NT;
     static constexpr int kNW = NT / 32;             // warps
-    static constexpr int kTcMax = NT / kNP * kL;    // tokens per CTA (= NT)
+    static constexpr int kTcMax = NT / kNP * kL;    // tokens per CTA
     static constexpr int kTab = kTcMax / kL;        // a^(8m), m < kTab
     static constexpr int kMinBlocks = 1024 / NT;    // resident CTAs per SM (64 registers)
 };
@@ -77,7 +80,7 @@ struct alignas(64) Params {
     int gslab;           // group size in 16-channel slabs (g / 16; 0 if g == 0)
     int ng;              // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
     float invT;          // 1 / T
-    int Tc;              // tokens per CTA (multiple of 32 when ncl > 1)
+    int Tc;              // tokens per CTA (multiple of kWarpTok when ncl > 1)
     int rows;            // image rows per CTA (Q-Shift path): Tc = rows * W
     int ncl;             // CTAs per column (cluster size)
     int tile_bytes;      // bytes per tile: 8 sub-tiles of 32 token rows
@@ -101,7 +104,7 @@ struct alignas(64) Params {
 // column that has not been fully started, and a GPU that holds 16 CTAs at once
 // always starts it.  The last CTA to finish resets the counters and advances
 // the generation, so stale flags of earlier launches never match.
-constexpr int kRecF4 = 20;  // float4 per record: F[8], G[8], M[8] (two pairs per float4)
+constexpr int kRecF4 = 2 * kNP + kNP / 2;  // float4 per record: F, G per pair; M two pairs per float4
 
 template <int NT>
 struct alignas(16) Scratch {
@@ -303,9 +306,9 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     Scratch& S = *reinterpret_cast<Scratch*>(smem + NTILE * p.tile_bytes);
 
     const int tid = threadIdx.x;
-    const int j = tid & 7;       // channel pair
-    const int q = tid >> 3;      // chunk within the CTA
-    const int cq = q & 3;        // chunk within the warp
+    const int j = tid % kNP;     // channel pair
+    const int q = tid / kNP;     // chunk within the CTA
+    const int cq = q % kCPW;     // chunk within the warp
     const int warp = tid >> 5;
     if (tid == 0) {
         mbar_init(&S.bar, 1);
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     const float2 mur = (QS && GATE) ? mu_of(p.mu[0]) : f2(1.0f);
     // decay table a^(8m): one entry (2 channels) per thread
     {
-        const int m = tid >> 3, jj = tid & 7;
+        const int m = tid / kNP, jj = tid % kNP;
         const float2 l = mul2(make_float2(__ldg(p.w + c0 + 2 * jj), __ldg(p.w + c0 + 2 * jj + 1)),
                               f2(invT * kLog2e));
         S.tab[m][jj] = ex2c(mul2(l, f2(-8.0f * m)));
@@ -461,7 +464,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
         }
     }
 #pragma unroll
-    for (int d = 8; d <= 16; d <<= 1) {
+    for (int d = kNP; d < 32; d <<= 1) {
         mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
         mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
     }
@@ -499,21 +502,19 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     // ---- 3. scans: warp, CTA, cluster --------------------------------------------
     float4 Fi = make_float4(fa.x, fa.y, fc.x, fc.y);
     float4 Gi = make_float4(ga.x, ga.y, gc.x, gc.y);
-    {
-        const float2 a8 = S.tab[1][j], a16 = S.tab[2][j];
-        float4 o = shfl_up4(Fi, 8, 32);
-        if (cq >= 1) Fi = fma4(a8, o, Fi);
-        o = shfl_up4(Fi, 16, 32);
-        if (cq >= 2) Fi = fma4(a16, o, Fi);
-        o = shfl_down4(Gi, 8, 32);
-        if (cq <= 2) Gi = fma4(a8, o, Gi);
-        o = shfl_down4(Gi, 16, 32);
-        if (cq <= 1) Gi = fma4(a16, o, Gi);
+    // warp scan across the kCPW chunks of a warp: step e spans 2^e chunks
+#pragma unroll
+    for (int e = 0; (kNP << e) < 32; ++e) {
+        const float2 m = S.tab[1 << e][j];  // a^(8 * 2^e)
+        float4 o = shfl_up4(Fi, kNP << e, 32);
+        if (cq >= (1 << e)) Fi = fma4(m, o, Fi);
+        o = shfl_down4(Gi, kNP << e, 32);
+        if (cq + (1 << e) < kCPW) Gi = fma4(m, o, Gi);
     }
-    float4 X = shfl_up4(Fi, 8, 32), Y = shfl_down4(Gi, 8, 32);
+    float4 X = shfl_up4(Fi, kNP, 32), Y = shfl_down4(Gi, kNP, 32);
     if (cq == 0) X = zero4();
-    if (cq == 3) Y = zero4();
-    if (cq == 3) S.waggF[j][warp] = Fi;
+    if (cq == kCPW - 1) Y = zero4();
+    if (cq == kCPW - 1) S.waggF[j][warp] = Fi;
     if (cq == 0) S.waggB[j][warp] = Gi;
     __syncthreads();
     if (tid < kNP * kNW) {  // one thread per (pair, warp)
@@ -521,7 +522,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
         float4 f = S.waggF[jj][wi], gb = S.waggB[jj][wi];
 #pragma unroll
         for (int d = 1; d < kNW; d <<= 1) {
-            const float2 m = S.tab[4 * d][jj];  // a^(32 d)
+            const float2 m = S.tab[kCPW * d][jj];  // a^(8 kCPW d): across d warps
             float4 o = shfl_up4(f, d, kNW);
             if (wi >= d) f = fma4(m, o, f);
             o = shfl_down4(gb, d, kNW);
@@ -533,9 +534,9 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
         S.wcarF[jj][wi] = xw;
         S.wcarB[jj][wi] = yw;
         // stage this CTA's record; the CTA's forward aggregate sits at its last
-        // real warp (Tc may be shorter than 256 tokens)
+        // real warp (Tc may be shorter than the CTA's capacity)
         if (p.ncl > 1) {
-            if (wi == p.Tc / 32 - 1) S.ownF[jj] = f;
+            if (wi == p.Tc / kWarpTok - 1) S.ownF[jj] = f;
             if (wi == 0) {
                 float2 Mj = S.wmax[jj][0];
 #pragma unroll
@@ -600,7 +601,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
             // own included), one (peer, pair, half) per thread, completing on
             // the receiver's mailbox barrier
             cluster_wait_acquire();  // every mailbox barrier is initialised
-            const int peer = tid >> 4, jj = (tid >> 1) & 7;
+            const int peer = tid / (2 * kNP), jj = (tid >> 1) % kNP;
             if (peer < p.ncl) {
                 const unsigned rbar = mapa_u32(smem_u32(&S.xbar), peer);
                 if ((tid & 1) == 0) {
@@ -687,7 +688,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     // ---- 4. carries -> outputs ---------------------------------------------------
     const float2 sl = cs_sl;
     const float4 XW = S.wcarF[j][warp], YW = S.wcarB[j][warp];
-    const float2 pwF = S.tab[cq][j], pwB = S.tab[3 - cq][j];
+    const float2 pwF = S.tab[cq][j], pwB = S.tab[kCPW - 1 - cq][j];
     const float2 kf = S.tab[q][j];                              // a^(8q): CTA start -> chunk
     const float2 kb = S.tab[max(0, p.Tc / kL - 1 - q)][j];      // chunk end -> CTA end
     const float2 As = fma2(sl, fma2(pwF, lo2(XW), lo2(X)), mul2(kf, cs_af));

@@ -516,7 +516,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         } else {
             int rows = 0;
             for (int rr = TcMax / p.W; rr >= 1; --rr)
-                if ((rr * p.W) % 32 == 0) {
+                if ((rr * p.W) % fast::kWarpTok == 0) {
                     rows = rr;
                     break;
                 }

@@ -33,7 +33,7 @@ def _inputs(B, H, W, C, dt, seed):
 @pytest.mark.parametrize("dt,B,H,W,C", [
     ("bf16", 2, 64, 64, 64),    # 16 CTAs per column: the exchange runs in the static workspace
     ("f32", 1, 40, 40, 64),     # 10 CTAs per column
-    ("bf16", 8, 64, 64, 1024),  # 512 columns: the full-size workload
+    ("bf16", 8, 64, 64, 1024),  # 1024 columns: the full-size workload
     ("bf16", 2, 14, 14, 96),    # one CTA per column: no exchange
 ])
 def test_static_matches_spatial_gate_twice(vk, dt, B, H, W, C):
@@ -49,7 +49,7 @@ def test_static_matches_spatial_gate_twice(vk, dt, B, H, W, C):
 
 def test_static_rejects_oversize(vk):
     import torch
-    # 8 x ceil(16384/16) = 8192 columns exceed the fixed workspace
+    # 8 x ceil(16384/8) = 16384 columns exceed the fixed workspace
     x = torch.zeros(8, 512, 16384, dtype=torch.bfloat16, device="cuda")
     w = torch.zeros(16384, device="cuda")
     with pytest.raises(vk.VrwkvError) as ei:
