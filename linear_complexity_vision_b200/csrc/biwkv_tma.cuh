@@ -51,7 +51,6 @@ constexpr int kL = 8;           // tokens per thread chunk
 constexpr int kCPW = 32 / kNP;  // chunks per warp
 constexpr int kWarpTok = kCPW * kL;  // tokens per warp
 constexpr int kClusterMax = 16;
-constexpr int kExThreads = kCS * kClusterMax;  // threads of the cross-CTA exchange
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 
 // CTA shape: NT threads = kNP channel pairs x NT/kNP chunks of 8 tokens, at
@@ -113,7 +112,8 @@ struct alignas(16) Scratch {
     // Rows of the [pair][warp] and [peer][pair] arrays carry one element of
     // padding: a warp reads one column across eight (or sixteen) rows, and
     // the odd row stride spreads those reads over all 32 banks.
-    float2 wmax[kNP][kNW + 1];      // per-warp maxima of k
+    float2 wmax[kNP][kNW + 1];      // per-warp maxima of k (-inf for a warp wholly past T)
+    float2 wsc[kNP][kNW + 1];       // per-warp scale 2^(M_warp - M_cta) onto the CTA reference
     float4 waggF[kNP][kNW + 1];     // per-warp forward aggregates (A.xy, C.xy)
     float4 waggB[kNP][kNW + 1];     // per-warp backward aggregates
     float4 wcarF[kNP][kNW + 1];     // exclusive forward carry into each warp
@@ -468,11 +468,11 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
         mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
         mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
     }
+    // The warp's own maximum is the exponent reference of its sums (no CTA
+    // barrier here); the CTA scan below rescales warp aggregates onto the CTA
+    // maximum.  A warp wholly past T keeps p = 0 with the reference 0.
     if (cq == 0) S.wmax[j][warp] = mx;
-    __syncthreads();
-    float2 M = S.wmax[j][0];
-#pragma unroll
-    for (int w = 1; w < kNW; ++w) M = max2(M, S.wmax[j][w]);
+    const float2 M = make_float2(mx.x == -INFINITY ? 0.0f : mx.x, mx.y == -INFINITY ? 0.0f : mx.y);
 
     // ---- 2. p = 2^(k - M), chunk-local two-sided sums ---------------------------
     const float2 negM = mul2(M, f2(-kLog2e));
@@ -519,7 +519,20 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     __syncthreads();
     if (tid < kNP * kNW) {  // one thread per (pair, warp)
         const int jj = tid / kNW, wi = tid % kNW;
-        float4 f = S.waggF[jj][wi], gb = S.waggB[jj][wi];
+        // CTA maximum; warp wi's sums move onto it by 2^(M_wi - M_cta) <= 1
+        // (0 for a warp wholly past T)
+        const float2 mw = S.wmax[jj][wi];
+        float2 mc = mw;
+#pragma unroll
+        for (int d = 1; d < kNW; d <<= 1) {
+            mc.x = fmaxf(mc.x, __shfl_xor_sync(0xffffffffu, mc.x, d, kNW));
+            mc.y = fmaxf(mc.y, __shfl_xor_sync(0xffffffffu, mc.y, d, kNW));
+        }
+        const float2 ws = ex2(mul2(add2(mw, make_float2(-mc.x, -mc.y)), f2(kLog2e)));
+        S.wsc[jj][wi] = ws;
+        const float4 f0 = S.waggF[jj][wi], g0 = S.waggB[jj][wi];
+        float4 f = make_float4(f0.x * ws.x, f0.y * ws.y, f0.z * ws.x, f0.w * ws.y);
+        float4 gb = make_float4(g0.x * ws.x, g0.y * ws.y, g0.z * ws.x, g0.w * ws.y);
 #pragma unroll
         for (int d = 1; d < kNW; d <<= 1) {
             const float2 m = S.tab[kCPW * d][jj];  // a^(8 kCPW d): across d warps
@@ -538,24 +551,25 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
         if (p.ncl > 1) {
             if (wi == p.Tc / kWarpTok - 1) S.ownF[jj] = f;
             if (wi == 0) {
-                float2 Mj = S.wmax[jj][0];
-#pragma unroll
-                for (int w = 1; w < kNW; ++w) Mj = max2(Mj, S.wmax[jj][w]);
                 S.ownG[jj] = gb;
-                S.ownM[jj] = mul2(Mj, f2(kLog2e));  // base 2, the unit of the exponents below
+                S.ownM[jj] = mul2(mc, f2(kLog2e));  // base 2, the unit of the exponents below
             }
         }
     }
-    // Thread (peer rr, channel lc) of the exchange below (the first 256
-    // threads): decay powers across d = 1, 2, 4, 8 CTAs, computed before the
-    // cluster barrier.
-    const int lc = tid >> 4, rr = tid & 15;
+    // Thread (peer rr, channel lc) of the exchange below: segments of sw
+    // lanes, one per channel (8 lanes when the column has at most 8 CTAs, else
+    // 16), so the first kCS * sw threads take part.  Decay powers across
+    // d = 1, 2, 4 (, 8) CTAs are computed before the wait for the peers.
+    const bool narrow = p.ncl <= 8;
+    const int sw = narrow ? 8 : 16;
+    const int lc = narrow ? tid >> 3 : tid >> 4, rr = tid & (sw - 1);
+    const int nex = kCS * sw;  // a multiple of 32: warp-uniform
     float mdec[4];
     if (p.ncl > 1) {
-        if (tid < kExThreads) {
+        if (tid < nex) {
             const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
+            for (int e = 0; e < 4; ++e) mdec[e] = (1 << e) < sw ? ex2c(-(float)(p.Tc << e) * l2) : 0.0f;
         }
         __syncthreads();
         if (GX) {
@@ -621,12 +635,12 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     }
     // Exchange with the other CTAs of the column: thread (channel lc, peer
     // rr) reads peer rr's record for channel lc from this CTA's mailbox;
-    // each 16-lane segment holds one channel's column.  The segment maximum
+    // each sw-lane segment holds one channel's column.  The segment maximum
     // of the peers' exponents is the common reference; forward and backward
-    // carries are 16-lane shuffle scans with the one-CTA decay a^Tc.
+    // carries are sw-lane shuffle scans with the one-CTA decay a^Tc.
     float2 cs_sl = f2(1.0f), cs_af = f2(0.0f), cs_cf = f2(0.0f), cs_bb = f2(0.0f), cs_db = f2(0.0f);
     if (p.ncl > 1) {
-        if (tid < kExThreads) {  // warp-uniform
+        if (tid < nex) {  // warp-uniform
             float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
             if (rr < p.ncl) {
                 const float4 F = S.mbF[rr][lc >> 1], G = S.mbG[rr][lc >> 1];
@@ -640,7 +654,8 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
             }
             float Mc = Mr;
 #pragma unroll
-            for (int d = 8; d >= 1; d >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, 16));
+            for (int d = 8; d >= 1; d >>= 1)
+                if (d < sw) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, sw));
             const float sc = ex2(Mr - Mc);  // 0 for lanes past the cluster
             fa2 *= sc;
             fc2 *= sc;
@@ -648,27 +663,28 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
             gc2 *= sc;
 #pragma unroll
             for (int e = 0, d = 1; d < kClusterMax; ++e, d <<= 1) {
+                if (d >= sw) break;
                 const float m = mdec[e];  // decay across d CTAs
-                const float ua = __shfl_up_sync(0xffffffffu, fa2, d, 16);
-                const float uc = __shfl_up_sync(0xffffffffu, fc2, d, 16);
-                const float da = __shfl_down_sync(0xffffffffu, ga2, d, 16);
-                const float dc = __shfl_down_sync(0xffffffffu, gc2, d, 16);
+                const float ua = __shfl_up_sync(0xffffffffu, fa2, d, sw);
+                const float uc = __shfl_up_sync(0xffffffffu, fc2, d, sw);
+                const float da = __shfl_down_sync(0xffffffffu, ga2, d, sw);
+                const float dc = __shfl_down_sync(0xffffffffu, gc2, d, sw);
                 if (rr >= d) {
                     fa2 = fmaf(m, ua, fa2);
                     fc2 = fmaf(m, uc, fc2);
                 }
-                if (rr + d < kClusterMax) {
+                if (rr + d < sw) {
                     ga2 = fmaf(m, da, ga2);
                     gc2 = fmaf(m, dc, gc2);
                 }
             }
             // exclusive carries of this CTA: inclusive forward at rank-1,
             // inclusive backward at rank+1 (zero past the ends)
-            const float Af = __shfl_sync(0xffffffffu, fa2, max(rank - 1, 0), 16);
-            const float Cf = __shfl_sync(0xffffffffu, fc2, max(rank - 1, 0), 16);
-            const float Bb = __shfl_sync(0xffffffffu, ga2, min(rank + 1, kClusterMax - 1), 16);
-            const float Db = __shfl_sync(0xffffffffu, gc2, min(rank + 1, kClusterMax - 1), 16);
-            const float Mme = __shfl_sync(0xffffffffu, Mr, rank, 16);
+            const float Af = __shfl_sync(0xffffffffu, fa2, max(rank - 1, 0), sw);
+            const float Cf = __shfl_sync(0xffffffffu, fc2, max(rank - 1, 0), sw);
+            const float Bb = __shfl_sync(0xffffffffu, ga2, min(rank + 1, sw - 1), sw);
+            const float Db = __shfl_sync(0xffffffffu, gc2, min(rank + 1, sw - 1), sw);
+            const float Mme = __shfl_sync(0xffffffffu, Mr, rank, sw);
             if (rr == 0) {
                 S.cscale[lc] = make_float4(ex2(Mme - Mc), 0.f, 0.f, 0.f);
                 S.ccarry[lc] = make_float4(rank > 0 ? Af : 0.f, rank > 0 ? Cf : 0.f,
@@ -686,15 +702,18 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     }
 
     // ---- 4. carries -> outputs ---------------------------------------------------
+    // sl: CTA reference -> column reference; slw: this warp's reference ->
+    // column reference (the warp-local sums n, dd, X, Y use the warp's own)
     const float2 sl = cs_sl;
+    const float2 slw = mul2(sl, S.wsc[j][warp]);
     const float4 XW = S.wcarF[j][warp], YW = S.wcarB[j][warp];
-    const float2 pwF = S.tab[cq][j], pwB = S.tab[kCPW - 1 - cq][j];
+    const float2 slF = mul2(sl, S.tab[cq][j]), slB = mul2(sl, S.tab[kCPW - 1 - cq][j]);
     const float2 kf = S.tab[q][j];                              // a^(8q): CTA start -> chunk
     const float2 kb = S.tab[max(0, p.Tc / kL - 1 - q)][j];      // chunk end -> CTA end
-    const float2 As = fma2(sl, fma2(pwF, lo2(XW), lo2(X)), mul2(kf, cs_af));
-    const float2 Cs = fma2(sl, fma2(pwF, hi2(XW), hi2(X)), mul2(kf, cs_cf));
-    const float2 Be = fma2(sl, fma2(pwB, lo2(YW), lo2(Y)), mul2(kb, cs_bb));
-    const float2 De = fma2(sl, fma2(pwB, hi2(YW), hi2(Y)), mul2(kb, cs_db));
+    const float2 As = fma2(slw, lo2(X), fma2(slF, lo2(XW), mul2(kf, cs_af)));
+    const float2 Cs = fma2(slw, hi2(X), fma2(slF, hi2(XW), mul2(kf, cs_cf)));
+    const float2 Be = fma2(slw, lo2(Y), fma2(slB, lo2(YW), mul2(kb, cs_bb)));
+    const float2 De = fma2(slw, hi2(Y), fma2(slB, hi2(YW), mul2(kb, cs_db)));
 
     float2 pw[kL];
     pw[0] = f2(1.0f);
@@ -705,8 +724,8 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     char* tout = smem;
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
-        const float2 num = fma2(sl, n[i], fma2(pw[i], As, mul2(pw[kL - 1 - i], Be)));
-        float2 den = fma2(sl, dd[i], fma2(pw[i], Cs, mul2(pw[kL - 1 - i], De)));
+        const float2 num = fma2(slw, n[i], fma2(pw[i], As, mul2(pw[kL - 1 - i], Be)));
+        float2 den = fma2(slw, dd[i], fma2(pw[i], Cs, mul2(pw[kL - 1 - i], De)));
         if (GATE) den = fma2(den, S.gpark[i * (kTcMax / kL) + q][j], den);
         Io<IO>::st_pair(tout + rowoff + i * SUB, mul2(num, rcp(den)));
     }
