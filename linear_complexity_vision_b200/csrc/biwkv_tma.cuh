@@ -47,22 +47,26 @@ namespace cg = cooperative_groups;
 
 constexpr int kCS = 8;          // channels per CTA (a column slab)
 constexpr int kNP = kCS / 2;    // channel pairs per CTA
-constexpr int kL = 8;           // tokens per thread chunk
+constexpr int kL = 8;           // tokens per sub-chunk (= the TMA element stride)
 constexpr int kCPW = 32 / kNP;  // chunks per warp
-constexpr int kWarpTok = kCPW * kL;  // tokens per warp
 constexpr int kClusterMax = 16;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 
-// CTA shape: NT threads = kNP channel pairs x NT/kNP chunks of 8 tokens, at
-// 64 registers per thread (1024/NT CTAs per SM).  The library launches
-// NT = 256 (four CTAs per SM; clusters of up to 16 CTAs along T).
-template <int NT>
+// CTA shape: NT threads = kNP channel pairs x NT/kNP chunks of KL tokens
+// (KL = 8: one sub-chunk, 64 registers per thread; KL = 16: two sub-chunks
+// of 8, 128 registers).  The library launches NT = 256 with KL = 8 and
+// NT = 128 with KL = 16: both span 512 tokens, four CTAs per SM, clusters of
+// up to 16 CTAs along T.
+template <int NT, int KL>
 struct Cfg {
+    static_assert(KL == 8 || KL == 16, "8 or 16 tokens per thread chunk");
     static constexpr int kThreads = NT;
     static constexpr int kNW = NT / 32;             // warps
-    static constexpr int kTcMax = NT / kNP * kL;    // tokens per CTA
-    static constexpr int kTab = kTcMax / kL;        // a^(8m), m < kTab
-    static constexpr int kMinBlocks = 1024 / NT;    // resident CTAs per SM (64 registers)
+    static constexpr int kH = KL / kL;              // sub-chunks per chunk
+    static constexpr int kTcMax = NT / kNP * KL;    // tokens per CTA
+    static constexpr int kTab = kTcMax / KL;        // chunks per CTA: a^(KL m), m < kTab
+    static constexpr int kWarpTok = kCPW * KL;      // tokens per warp
+    static constexpr int kMinBlocks = 65536 / (NT * 16 * KL / 2);  // 64 or 128 registers per thread
 };
 
 enum Layout { kKV = 0, kRKV = 1, kX = 2 };
@@ -105,10 +109,10 @@ struct alignas(64) Params {
 // the generation, so stale flags of earlier launches never match.
 constexpr int kRecF4 = 2 * kNP + kNP / 2;  // float4 per record: F, G per pair; M two pairs per float4
 
-template <int NT>
+template <int NT, int KL>
 struct alignas(16) Scratch {
-    static constexpr int kNW = Cfg<NT>::kNW;
-    float2 tab[Cfg<NT>::kTab][kNP];  // a^(8m) per channel pair
+    static constexpr int kNW = Cfg<NT, KL>::kNW;
+    float2 tab[Cfg<NT, KL>::kTab][kNP];  // a^(KL m) per channel pair
     // Rows of the [pair][warp] and [peer][pair] arrays carry one element of
     // padding: a warp reads one column across eight (or sixteen) rows, and
     // the odd row stride spreads those reads over all 32 banks.
@@ -124,7 +128,7 @@ struct alignas(16) Scratch {
     float4 ownF[kNP];           // this CTA's inclusive forward aggregate, staged for the push
     float4 ownG[kNP];           // this CTA's inclusive backward aggregate
     float2 ownM[kNP];           // this CTA's max of k (times log2 e)
-    float2 gpark[Cfg<NT>::kTcMax][kNP];  // gate factors, parked between load and output
+    float2 gpark[Cfg<NT, KL>::kTcMax][kNP];  // gate factors, parked between load and output
     float4 cscale[kCS];         // per channel: sl (scale of this CTA's own sums)
     int tk;                     // GX: this CTA's ticket
     unsigned int gen;           // GX: the launch's generation
@@ -283,12 +287,16 @@ __device__ __forceinline__ void wait_flag(const unsigned int* f, unsigned int wa
     }
 }
 
-template <typename IO, int LAYOUT, bool QS, int NT, bool GX>
-__global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(const __grid_constant__ Params p) {
-    constexpr int kThreads = Cfg<NT>::kThreads;
-    constexpr int kNW = Cfg<NT>::kNW;
-    constexpr int kTcMax = Cfg<NT>::kTcMax;
-    using Scratch = fast::Scratch<NT>;
+template <typename IO, int LAYOUT, bool QS, int NT, int KL, bool GX>
+__global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
+    biwkv_tma_kernel(const __grid_constant__ Params p) {
+    using C_ = Cfg<NT, KL>;
+    constexpr int kThreads = C_::kThreads;
+    constexpr int kNW = C_::kNW;
+    constexpr int kTcMax = C_::kTcMax;
+    constexpr int kH = C_::kH;          // sub-chunks of 8 tokens per thread chunk
+    constexpr int kChunks = C_::kTab;   // chunks per CTA
+    using Scratch = fast::Scratch<NT, KL>;
     constexpr bool GATE = LAYOUT != kKV;
     constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
     constexpr int NTILE = NSRC * (QS ? 2 : 1);
@@ -390,122 +398,153 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     const float2 lam2 = mul2(wv, f2(invT * kLog2e));  // w / T in base-2 units
     const float2 alpha = ex2c(make_float2(-lam2.x, -lam2.y));
     const float2 eu = ex2(mul2(uv, f2(kLog2e)));
+    const float2 a8 = ex2c(mul2(lam2, f2(-(float)kL)));  // a^8: across one sub-chunk (KL = 16)
     auto mu_of = [&](const float* m) {
         return m ? make_float2(__ldg(m + cA), __ldg(m + cA + 1)) : f2(0.0f);
     };
     const float2 muk = QS ? mu_of(p.mu[1]) : f2(1.0f);
     const float2 muv = QS ? mu_of(p.mu[2]) : f2(1.0f);
     const float2 mur = (QS && GATE) ? mu_of(p.mu[0]) : f2(1.0f);
-    // decay table a^(8m): one entry (2 channels) per thread
+    // decay table a^(KL m), one per chunk distance m: one entry (2 channels)
+    // per thread
     {
         const int m = tid / kNP, jj = tid % kNP;
         const float2 l = mul2(make_float2(__ldg(p.w + c0 + 2 * jj), __ldg(p.w + c0 + 2 * jj + 1)),
                               f2(invT * kLog2e));
-        S.tab[m][jj] = ex2c(mul2(l, f2(-8.0f * m)));
+        S.tab[m][jj] = ex2c(mul2(l, f2(-(float)KL * m)));
     }
 
-    const int s_tok = t0 + q * kL;
-    const int nv = max(0, min(kL, tend - s_tok));
-    const int rowoff = q * RB + j * PB;  // token i of the chunk: + i * SUB
+    const int s_tok = t0 + q * KL;
+    const int nvt = max(0, min(KL, tend - s_tok));  // valid tokens of this chunk
 
     // one thread waits for the tiles; the others sleep at the CTA barrier
     if (tid == 0) mbar_wait_bounded(&S.bar, p.err);
     __syncthreads();
 
-    // ---- 1. load, Q-Shift mix, chunk maximum -----------------------------------
+    // ---- 1-2. per 8-token sub-chunk: load, Q-Shift mix, gate factor, local
+    // maximum, p = 2^(k - M_h), two-sided sums inside the sub-chunk ----------
+    // Token 8 (q kH + h) + i of the CTA is sub-tile i, row q kH + h.  Each
+    // sub-chunk works relative to its own maximum M_h (0 if it lies wholly past
+    // T); the thread combine below rescales by 2^(M_h - M_warp) <= 1.
     const char* tK = smem + (QS ? 2 * SK : SK) * p.tile_bytes;
     const char* tV = smem + (QS ? 2 * SV : SV) * p.tile_bytes;
     const char* tR = smem + (QS ? 2 * SR : SR) * p.tile_bytes;
     const int dsh = shifted ? p.tile_bytes : 0;  // shifted tile = plain + dsh
-    float2 kk[kL], vv[kL];
-    float2 mx = f2(-INFINITY);
+    float2 n[kH][kL], dd[kH][kL];
+    float4 Fh[kH], Gh[kH];  // per sub-chunk: forward (A.xy, C.xy) and backward totals
+    float2 Mh[kH];          // per sub-chunk maximum of k (-inf if wholly past T)
 #pragma unroll
-    for (int i = 0; i < kL; ++i) {
-        const int o = rowoff + i * SUB;
-        float2 k, v, r;
-        if (QS) {
-            if (LAYOUT == kX) {
-                const float2 x = lds_pair<IO>(tK, o), xd = lds_pair<IO>(tK + dsh, o);
-                const float2 d = add2(x, make_float2(-xd.x, -xd.y));
-                k = fma2(muk, d, xd);
-                v = fma2(muv, d, xd);
-                r = fma2(mur, d, xd);
-            } else {
-                const float2 xk = lds_pair<IO>(tK, o), xkd = lds_pair<IO>(tK + dsh, o);
-                const float2 xv = lds_pair<IO>(tV, o), xvd = lds_pair<IO>(tV + dsh, o);
-                k = fma2(muk, add2(xk, make_float2(-xkd.x, -xkd.y)), xkd);
-                v = fma2(muv, add2(xv, make_float2(-xvd.x, -xvd.y)), xvd);
-                if (GATE) {
-                    const float2 xr = lds_pair<IO>(tR, o), xrd = lds_pair<IO>(tR + dsh, o);
-                    r = fma2(mur, add2(xr, make_float2(-xrd.x, -xrd.y)), xrd);
-                }
-            }
-        } else {
-            k = lds_pair<IO>(tK, o);
-            v = lds_pair<IO>(tV, o);
-            if (GATE) r = lds_pair<IO>(tR, o);
-        }
-        // gate factor e^{-r}, parked in shared memory until the output phase
-        if (GATE) S.gpark[i * (kTcMax / kL) + q][j] = ex2(mul2(r, f2(-kLog2e)));
-        kk[i] = k;
-        vv[i] = v;
-    }
-    if (nv == kL) {
-#pragma unroll
-        for (int i = 0; i < kL; ++i) mx = max2(mx, kk[i]);
-    } else {
-        // tokens past the sequence end hold zeros (TMA fill) or stale shared
-        // memory (rows beyond a short box): mask both so p = 0 and p*v = 0
+    for (int h = 0; h < kH; ++h) {
+        const int rowoff = (q * kH + h) * RB + j * PB;
+        const int nv = max(0, min(kL, nvt - h * kL));
+        float2 kk[kL], vv[kL];
 #pragma unroll
         for (int i = 0; i < kL; ++i) {
-            kk[i] = (i < nv) ? kk[i] : f2(-INFINITY);
-            vv[i] = (i < nv) ? vv[i] : f2(0.0f);
-            mx = max2(mx, kk[i]);
+            const int o = rowoff + i * SUB;
+            float2 k, v, r;
+            if (QS) {
+                if (LAYOUT == kX) {
+                    const float2 x = lds_pair<IO>(tK, o), xd = lds_pair<IO>(tK + dsh, o);
+                    const float2 d = add2(x, make_float2(-xd.x, -xd.y));
+                    k = fma2(muk, d, xd);
+                    v = fma2(muv, d, xd);
+                    r = fma2(mur, d, xd);
+                } else {
+                    const float2 xk = lds_pair<IO>(tK, o), xkd = lds_pair<IO>(tK + dsh, o);
+                    const float2 xv = lds_pair<IO>(tV, o), xvd = lds_pair<IO>(tV + dsh, o);
+                    k = fma2(muk, add2(xk, make_float2(-xkd.x, -xkd.y)), xkd);
+                    v = fma2(muv, add2(xv, make_float2(-xvd.x, -xvd.y)), xvd);
+                    if (GATE) {
+                        const float2 xr = lds_pair<IO>(tR, o), xrd = lds_pair<IO>(tR + dsh, o);
+                        r = fma2(mur, add2(xr, make_float2(-xrd.x, -xrd.y)), xrd);
+                    }
+                }
+            } else {
+                k = lds_pair<IO>(tK, o);
+                v = lds_pair<IO>(tV, o);
+                if (GATE) r = lds_pair<IO>(tR, o);
+            }
+            // gate factor e^{-r}, parked in shared memory until the output phase
+            if (GATE) S.gpark[(h * kL + i) * kChunks + q][j] = ex2(mul2(r, f2(-kLog2e)));
+            kk[i] = k;
+            vv[i] = v;
         }
+        float2 mx = f2(-INFINITY);
+        if (nv == kL) {
+#pragma unroll
+            for (int i = 0; i < kL; ++i) mx = max2(mx, kk[i]);
+        } else {
+            // tokens past the sequence end hold zeros (TMA fill) or stale shared
+            // memory (rows beyond a short box): mask both so p = 0 and p*v = 0
+#pragma unroll
+            for (int i = 0; i < kL; ++i) {
+                kk[i] = (i < nv) ? kk[i] : f2(-INFINITY);
+                vv[i] = (i < nv) ? vv[i] : f2(0.0f);
+                mx = max2(mx, kk[i]);
+            }
+        }
+        Mh[h] = mx;
+        const float2 negM = make_float2(mx.x == -INFINITY ? 0.0f : -mx.x * kLog2e,
+                                        mx.y == -INFINITY ? 0.0f : -mx.y * kLog2e);
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            kk[i] = ex2(fma2(kk[i], f2(kLog2e), negM));  // p_i (0 beyond T)
+            vv[i] = mul2(kk[i], vv[i]);                  // p_i v_i
+        }
+        float2 fa = f2(0.0f), fc = f2(0.0f);
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            n[h][i] = fa;
+            dd[h][i] = fc;
+            fa = fma2(alpha, fa, vv[i]);
+            fc = fma2(alpha, fc, kk[i]);
+        }
+        float2 ga = f2(0.0f), gc = f2(0.0f);
+#pragma unroll
+        for (int i = kL - 1; i >= 0; --i) {
+            n[h][i] = add2(n[h][i], fma2(eu, vv[i], ga));
+            dd[h][i] = add2(dd[h][i], fma2(eu, kk[i], gc));
+            ga = fma2(alpha, ga, vv[i]);
+            gc = fma2(alpha, gc, kk[i]);
+        }
+        Fh[h] = make_float4(fa.x, fa.y, fc.x, fc.y);
+        Gh[h] = make_float4(ga.x, ga.y, gc.x, gc.y);
     }
+
+    // ---- 3a. warp maximum (the reference of the warp's sums) and the chunk's
+    // totals on it ---------------------------------------------------------------
+    float2 mx = Mh[0];
+#pragma unroll
+    for (int h = 1; h < kH; ++h) mx = max2(mx, Mh[h]);
 #pragma unroll
     for (int d = kNP; d < 32; d <<= 1) {
         mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
         mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
     }
-    // The warp's own maximum is the exponent reference of its sums (no CTA
-    // barrier here); the CTA scan below rescales warp aggregates onto the CTA
-    // maximum.  A warp wholly past T keeps p = 0 with the reference 0.
-    if (cq == 0) S.wmax[j][warp] = mx;
-    const float2 M = make_float2(mx.x == -INFINITY ? 0.0f : mx.x, mx.y == -INFINITY ? 0.0f : mx.y);
-
-    // ---- 2. p = 2^(k - M), chunk-local two-sided sums ---------------------------
-    const float2 negM = mul2(M, f2(-kLog2e));
+    if (cq == 0) S.wmax[j][warp] = mx;  // -inf for a warp wholly past T
+    // sub-chunk h -> warp reference: 2^(M_h - M_warp), 0 for an empty sub-chunk
+    const float2 mref = make_float2(mx.x == -INFINITY ? 0.0f : mx.x, mx.y == -INFINITY ? 0.0f : mx.y);
+    float2 eh[kH];
 #pragma unroll
-    for (int i = 0; i < kL; ++i) {
-        kk[i] = ex2(fma2(kk[i], f2(kLog2e), negM));  // p_i (0 beyond T)
-        vv[i] = mul2(kk[i], vv[i]);                  // p_i v_i
-    }
-    float2 n[kL], dd[kL];
-    float2 fa = f2(0.0f), fc = f2(0.0f);
-#pragma unroll
-    for (int i = 0; i < kL; ++i) {
-        n[i] = fa;
-        dd[i] = fc;
-        fa = fma2(alpha, fa, vv[i]);
-        fc = fma2(alpha, fc, kk[i]);
-    }
-    float2 ga = f2(0.0f), gc = f2(0.0f);
-#pragma unroll
-    for (int i = kL - 1; i >= 0; --i) {
-        n[i] = add2(n[i], fma2(eu, vv[i], ga));
-        dd[i] = add2(dd[i], fma2(eu, kk[i], gc));
-        ga = fma2(alpha, ga, vv[i]);
-        gc = fma2(alpha, gc, kk[i]);
+    for (int h = 0; h < kH; ++h) eh[h] = ex2(mul2(add2(Mh[h], make_float2(-mref.x, -mref.y)), f2(kLog2e)));
+    auto scale4 = [](float2 e, float4 v) { return make_float4(v.x * e.x, v.y * e.y, v.z * e.x, v.w * e.y); };
+    float4 Fi, Gi;
+    float4 F0s = zero4(), G1s = zero4();  // KL = 16: sub-chunk 0's forward, sub-chunk 1's backward total
+    if (kH == 1) {
+        Fi = scale4(eh[0], Fh[0]);
+        Gi = scale4(eh[0], Gh[0]);
+    } else {
+        F0s = scale4(eh[0], Fh[0]);
+        G1s = scale4(eh[kH - 1], Gh[kH - 1]);
+        Fi = fma4(a8, F0s, scale4(eh[kH - 1], Fh[kH - 1]));
+        Gi = fma4(a8, G1s, scale4(eh[0], Gh[0]));
     }
 
-    // ---- 3. scans: warp, CTA, cluster --------------------------------------------
-    float4 Fi = make_float4(fa.x, fa.y, fc.x, fc.y);
-    float4 Gi = make_float4(ga.x, ga.y, gc.x, gc.y);
+    // ---- 3b. scans: warp, CTA, cluster -----------------------------------------
     // warp scan across the kCPW chunks of a warp: step e spans 2^e chunks
 #pragma unroll
     for (int e = 0; (kNP << e) < 32; ++e) {
-        const float2 m = S.tab[1 << e][j];  // a^(8 * 2^e)
+        const float2 m = S.tab[1 << e][j];  // a^(KL * 2^e)
         float4 o = shfl_up4(Fi, kNP << e, 32);
         if (cq >= (1 << e)) Fi = fma4(m, o, Fi);
         o = shfl_down4(Gi, kNP << e, 32);
@@ -517,8 +556,9 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     if (cq == kCPW - 1) S.waggF[j][warp] = Fi;
     if (cq == 0) S.waggB[j][warp] = Gi;
     __syncthreads();
-    if (tid < kNP * kNW) {  // one thread per (pair, warp)
-        const int jj = tid / kNW, wi = tid % kNW;
+    if (warp == 0) {  // lanes (pair, warp) < kNP * kNW; the rest idle along
+        const bool act = tid < kNP * kNW;
+        const int jj = act ? tid / kNW : 0, wi = act ? tid % kNW : 0;
         // CTA maximum; warp wi's sums move onto it by 2^(M_wi - M_cta) <= 1
         // (0 for a warp wholly past T)
         const float2 mw = S.wmax[jj][wi];
@@ -529,13 +569,11 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
             mc.y = fmaxf(mc.y, __shfl_xor_sync(0xffffffffu, mc.y, d, kNW));
         }
         const float2 ws = ex2(mul2(add2(mw, make_float2(-mc.x, -mc.y)), f2(kLog2e)));
-        S.wsc[jj][wi] = ws;
-        const float4 f0 = S.waggF[jj][wi], g0 = S.waggB[jj][wi];
-        float4 f = make_float4(f0.x * ws.x, f0.y * ws.y, f0.z * ws.x, f0.w * ws.y);
-        float4 gb = make_float4(g0.x * ws.x, g0.y * ws.y, g0.z * ws.x, g0.w * ws.y);
+        float4 f = scale4(ws, S.waggF[jj][wi]);
+        float4 gb = scale4(ws, S.waggB[jj][wi]);
 #pragma unroll
         for (int d = 1; d < kNW; d <<= 1) {
-            const float2 m = S.tab[kCPW * d][jj];  // a^(8 kCPW d): across d warps
+            const float2 m = S.tab[kCPW * d][jj];  // a^(KL kCPW d): across d warps
             float4 o = shfl_up4(f, d, kNW);
             if (wi >= d) f = fma4(m, o, f);
             o = shfl_down4(gb, d, kNW);
@@ -544,15 +582,18 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
         float4 xw = shfl_up4(f, 1, kNW), yw = shfl_down4(gb, 1, kNW);
         if (wi == 0) xw = zero4();
         if (wi == kNW - 1) yw = zero4();
-        S.wcarF[jj][wi] = xw;
-        S.wcarB[jj][wi] = yw;
-        // stage this CTA's record; the CTA's forward aggregate sits at its last
-        // real warp (Tc may be shorter than the CTA's capacity)
-        if (p.ncl > 1) {
-            if (wi == p.Tc / kWarpTok - 1) S.ownF[jj] = f;
-            if (wi == 0) {
-                S.ownG[jj] = gb;
-                S.ownM[jj] = mul2(mc, f2(kLog2e));  // base 2, the unit of the exponents below
+        if (act) {
+            S.wsc[jj][wi] = ws;
+            S.wcarF[jj][wi] = xw;
+            S.wcarB[jj][wi] = yw;
+            // stage this CTA's record; the CTA's forward aggregate sits at its
+            // last real warp (Tc may be shorter than the CTA's capacity)
+            if (p.ncl > 1) {
+                if (wi == p.Tc / C_::kWarpTok - 1) S.ownF[jj] = f;
+                if (wi == 0) {
+                    S.ownG[jj] = gb;
+                    S.ownM[jj] = mul2(mc, f2(kLog2e));  // base 2, the unit of the exponents below
+                }
             }
         }
     }
@@ -703,13 +744,15 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
 
     // ---- 4. carries -> outputs ---------------------------------------------------
     // sl: CTA reference -> column reference; slw: this warp's reference ->
-    // column reference (the warp-local sums n, dd, X, Y use the warp's own)
+    // column reference (the warp-local sums X, Y and the sub-chunk totals use
+    // the warp's own; n, dd use their sub-chunk's, hence the extra eh)
     const float2 sl = cs_sl;
     const float2 slw = mul2(sl, S.wsc[j][warp]);
     const float4 XW = S.wcarF[j][warp], YW = S.wcarB[j][warp];
     const float2 slF = mul2(sl, S.tab[cq][j]), slB = mul2(sl, S.tab[kCPW - 1 - cq][j]);
-    const float2 kf = S.tab[q][j];                              // a^(8q): CTA start -> chunk
-    const float2 kb = S.tab[max(0, p.Tc / kL - 1 - q)][j];      // chunk end -> CTA end
+    const float2 kf = S.tab[q][j];                              // a^(KL q): CTA start -> chunk
+    const float2 kb = S.tab[max(0, p.Tc / KL - 1 - q)][j];      // chunk end -> CTA end
+    // carries into the chunk: from the left at its start, from the right at its end
     const float2 As = fma2(slw, lo2(X), fma2(slF, lo2(XW), mul2(kf, cs_af)));
     const float2 Cs = fma2(slw, hi2(X), fma2(slF, hi2(XW), mul2(kf, cs_cf)));
     const float2 Be = fma2(slw, lo2(Y), fma2(slB, lo2(YW), mul2(kb, cs_bb)));
@@ -723,11 +766,26 @@ __global__ void __launch_bounds__(NT, Cfg<NT>::kMinBlocks) biwkv_tma_kernel(cons
     // same conflict-free offsets, then leave as coalesced 16-byte stores
     char* tout = smem;
 #pragma unroll
-    for (int i = 0; i < kL; ++i) {
-        const float2 num = fma2(slw, n[i], fma2(pw[i], As, mul2(pw[kL - 1 - i], Be)));
-        float2 den = fma2(slw, dd[i], fma2(pw[i], Cs, mul2(pw[kL - 1 - i], De)));
-        if (GATE) den = fma2(den, S.gpark[i * (kTcMax / kL) + q][j], den);
-        Io<IO>::st_pair(tout + rowoff + i * SUB, mul2(num, rcp(den)));
+    for (int h = 0; h < kH; ++h) {
+        // carries into sub-chunk h: the other sub-chunk's total joins them
+        float2 Ah = As, Ch = Cs, Bh = Be, Dh = De;
+        if (kH == 2 && h == 0) {
+            Bh = fma2(slw, lo2(G1s), mul2(a8, Be));
+            Dh = fma2(slw, hi2(G1s), mul2(a8, De));
+        }
+        if (kH == 2 && h == 1) {
+            Ah = fma2(slw, lo2(F0s), mul2(a8, As));
+            Ch = fma2(slw, hi2(F0s), mul2(a8, Cs));
+        }
+        const float2 sh = mul2(slw, eh[h]);
+        const int rowoff = (q * kH + h) * RB + j * PB;
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            const float2 num = fma2(sh, n[h][i], fma2(pw[i], Ah, mul2(pw[kL - 1 - i], Bh)));
+            float2 den = fma2(sh, dd[h][i], fma2(pw[i], Ch, mul2(pw[kL - 1 - i], Dh)));
+            if (GATE) den = fma2(den, S.gpark[(h * kL + i) * kChunks + q][j], den);
+            Io<IO>::st_pair(tout + rowoff + i * SUB, mul2(num, rcp(den)));
+        }
     }
     __syncthreads();
     {

@@ -345,12 +345,20 @@ bool tma_disabled() {
     return e && e[0] && e[0] != '0';
 }
 
+// VRWKV_TMA_CHUNK=8 keeps the forward TMA path on 8-token thread chunks even
+// where the 16-token kernel qualifies (diagnostics and tests).
+bool tma_chunk8_forced() {
+    const char* e = getenv("VRWKV_TMA_CHUNK");
+    return e && e[0] == '8' && e[1] == 0;
+}
+
 struct FastPlan {
     fast::Params p;
     int layout;
     bool qs;
     bool gx;  // exchange through the caller's workspace instead of a cluster
-    int nt;   // threads (= tokens) per CTA
+    int nt;   // threads per CTA
+    int kl;   // tokens per thread chunk (8 or 16)
     dim3 grid;
     int smem;
 };
@@ -370,9 +378,9 @@ WsLayout ws_layout(int B, int C) {
     return L;
 }
 
-template <typename IO, int LAYOUT, bool QS, int NT, bool GX>
+template <typename IO, int LAYOUT, bool QS, int NT, int KL, bool GX>
 vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
-    auto kern = fast::biwkv_tma_kernel<IO, LAYOUT, QS, NT, GX>;
+    auto kern = fast::biwkv_tma_kernel<IO, LAYOUT, QS, NT, KL, GX>;
     static std::atomic<int> granted{0};
     static std::atomic<int> nonportable{0};
     cudaError_t e = ensure_smem(kern, granted, pl.smem);
@@ -435,32 +443,41 @@ vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_bac
     return ok();
 }
 
-template <typename IO, int NT, bool GX>
+template <typename IO, int NT, int KL, bool GX>
 vrwkv_status dispatch_fast_nt(const FastPlan& pl, cudaStream_t s, bool* fb) {
     switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
-    case fast::kKV * 2 + 0: return launch_fast<IO, fast::kKV, false, NT, GX>(pl, s, fb);
-    case fast::kKV * 2 + 1: return launch_fast<IO, fast::kKV, true, NT, GX>(pl, s, fb);
-    case fast::kRKV * 2 + 0: return launch_fast<IO, fast::kRKV, false, NT, GX>(pl, s, fb);
-    case fast::kRKV * 2 + 1: return launch_fast<IO, fast::kRKV, true, NT, GX>(pl, s, fb);
-    case fast::kX * 2 + 0: return launch_fast<IO, fast::kX, false, NT, GX>(pl, s, fb);
-    default: return launch_fast<IO, fast::kX, true, NT, GX>(pl, s, fb);
+    case fast::kKV * 2 + 0: return launch_fast<IO, fast::kKV, false, NT, KL, GX>(pl, s, fb);
+    case fast::kKV * 2 + 1: return launch_fast<IO, fast::kKV, true, NT, KL, GX>(pl, s, fb);
+    case fast::kRKV * 2 + 0: return launch_fast<IO, fast::kRKV, false, NT, KL, GX>(pl, s, fb);
+    case fast::kRKV * 2 + 1: return launch_fast<IO, fast::kRKV, true, NT, KL, GX>(pl, s, fb);
+    case fast::kX * 2 + 0: return launch_fast<IO, fast::kX, false, NT, KL, GX>(pl, s, fb);
+    default: return launch_fast<IO, fast::kX, true, NT, KL, GX>(pl, s, fb);
     }
 }
 
-// CTA size of the fast path.  512-thread CTAs (8-CTA clusters at T = 4096)
-// measured slower than 256-thread CTAs (16-CTA clusters): fewer independent
-// CTAs per SM hide less of each other's barrier and exchange latency.
-constexpr int kFastThreads = 256;
+// CTA shapes of the fast path, both 512 tokens x 8 channels at four CTAs per
+// SM: 128 threads with 16-token chunks (the default: half the per-thread
+// scan and exchange work per token), or 256 threads with 8-token chunks where
+// a cluster's CTAs cannot hold whole 128-token warps.
+constexpr int kFastThreads16 = 128;
+constexpr int kFastThreads8 = 256;
+constexpr int kFastTcMax = fast::Cfg<kFastThreads16, 16>::kTcMax;
+static_assert(kFastTcMax == fast::Cfg<kFastThreads8, 8>::kTcMax, "one tile geometry for both shapes");
 
 template <typename IO>
 vrwkv_status dispatch_fast(const FastPlan& pl, cudaStream_t s, bool* fb) {
-    return pl.gx ? dispatch_fast_nt<IO, kFastThreads, true>(pl, s, fb)
-                 : dispatch_fast_nt<IO, kFastThreads, false>(pl, s, fb);
+    if (pl.kl == 16)
+        return pl.gx ? dispatch_fast_nt<IO, kFastThreads16, 16, true>(pl, s, fb)
+                     : dispatch_fast_nt<IO, kFastThreads16, 16, false>(pl, s, fb);
+    return pl.gx ? dispatch_fast_nt<IO, kFastThreads8, 8, true>(pl, s, fb)
+                 : dispatch_fast_nt<IO, kFastThreads8, 8, false>(pl, s, fb);
 }
 
 // Shared memory of a fast-path CTA: the tiles plus the scratch block.
-int fast_smem(int ntiles, int tile_bytes) {
-    return ntiles * tile_bytes + (int)sizeof(fast::Scratch<kFastThreads>) + 128;  // + alignment slack
+int fast_smem(int ntiles, int tile_bytes, int kl) {
+    const int scratch = kl == 16 ? (int)sizeof(fast::Scratch<kFastThreads16, 16>)
+                                 : (int)sizeof(fast::Scratch<kFastThreads8, 8>);
+    return ntiles * tile_bytes + scratch + 128;  // + alignment slack
 }
 
 // Plan the TMA path; returns false when the problem is outside its limits
@@ -500,8 +517,8 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     p.C = C;
     const int RB = fast::kCS * es;
     const int ntiles = nsrc * (pl.qs ? 2 : 1);
-    pl.nt = kFastThreads;
-    const int TcMax = fast::Cfg<kFastThreads>::kTcMax;
+    const int TcMax = kFastTcMax;
+    pl.kl = tma_chunk8_forced() ? 8 : 16;
     if (pl.qs) {
         p.H = qs->H;
         p.W = qs->W;
@@ -514,12 +531,19 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
             p.Tc = T;
             p.ncl = 1;
         } else {
+            // whole image rows per CTA, a whole number of warps' tokens:
+            // 16-token chunks where possible, else 8-token chunks
             int rows = 0;
-            for (int rr = TcMax / p.W; rr >= 1; --rr)
-                if ((rr * p.W) % fast::kWarpTok == 0) {
-                    rows = rr;
-                    break;
-                }
+            for (int kl = pl.kl; kl >= 8 && rows == 0; kl /= 2) {
+                const int warp_tok = kl == 16 ? fast::Cfg<kFastThreads16, 16>::kWarpTok
+                                              : fast::Cfg<kFastThreads8, 8>::kWarpTok;
+                for (int rr = TcMax / p.W; rr >= 1; --rr)
+                    if ((rr * p.W) % warp_tok == 0) {
+                        rows = rr;
+                        pl.kl = kl;
+                        break;
+                    }
+            }
             if (rows == 0 || rows > 256) return false;
             p.rows = rows;
             p.Tc = rows * p.W;
@@ -544,7 +568,8 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     // and its full TcMax / 8 rows without (boxes of 32 rows; tokens past T
     // arrive as zeros)
     p.box_bytes = (pl.qs ? (p.W / fast::kL) * p.rows : TcMax / fast::kL) * RB;
-    pl.smem = fast_smem(ntiles, p.tile_bytes);
+    pl.nt = pl.kl == 16 ? kFastThreads16 : kFastThreads8;
+    pl.smem = fast_smem(ntiles, p.tile_bytes, pl.kl);
     if (pl.smem > 227 * 1024) return false;
     const CUtensorMapDataType dt =
         dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;

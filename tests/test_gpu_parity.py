@@ -169,15 +169,20 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     return (got, err) if return_out else err
 
 
-@pytest.fixture(params=["tma", "gx", "generic"])
+@pytest.fixture(params=["tma", "tma8", "gx", "generic"])
 def kernel_path(request, monkeypatch):
-    """Run a test on the TMA fast path (when the shape qualifies), on its
-    workspace variant (global-memory exchange instead of clusters) and with
-    the generic kernel forced."""
+    """Run a test on the TMA fast path (when the shape qualifies; 16-token
+    thread chunks where the cluster geometry allows), on the same path held to
+    8-token chunks, on its workspace variant (global-memory exchange instead
+    of clusters) and with the generic kernel forced."""
     if request.param == "generic":
         monkeypatch.setenv("VRWKV_DISABLE_TMA", "1")
     else:
         monkeypatch.delenv("VRWKV_DISABLE_TMA", raising=False)
+    if request.param == "tma8":
+        monkeypatch.setenv("VRWKV_TMA_CHUNK", "8")
+    else:
+        monkeypatch.delenv("VRWKV_TMA_CHUNK", raising=False)
     _GX["on"] = request.param == "gx"
     yield request.param
     _GX["on"] = False
@@ -220,12 +225,12 @@ EDGE = [
     ("gate_qs_x", 2, 14, 14, 96, "bf16"),
     ("gate_qs_x", 1, 40, 40, 64, "f32"),    # T = 1600 in float32
     ("gate_qs_x", 1, 3, 11, 6, "bf16"),
-    ("gate_qs_x", 2, 16, 16, 64, "bf16"),   # T = 256: one full CTA
-    ("gate_qs_x", 1, 40, 40, 64, "bf16"),   # W = 40: 10-CTA cluster
-    ("gate_qs", 2, 64, 64, 64, "bf16"),     # 16-CTA cluster, separate r, k, v
+    ("gate_qs_x", 2, 16, 16, 64, "bf16"),   # T = 256: half a CTA
+    ("gate_qs_x", 1, 40, 40, 64, "bf16"),   # W = 40: 8-token chunks, 5-CTA cluster
+    ("gate_qs", 2, 64, 64, 64, "bf16"),     # 8-CTA cluster, separate r, k, v
     ("qshift_biwkv", 1, 48, 64, 64, "bf16"),
     ("qshift_biwkv", 2, 24, 24, 64, "f32"),  # W = 24: 8 rows of 24 per CTA
-    ("biwkv", 2, 1, 4096, 16, "bf16"),      # 16 CTAs without Q-Shift
+    ("biwkv", 2, 1, 4096, 16, "bf16"),      # 8 CTAs without Q-Shift
     ("biwkv", 3, 1, 257, 32, "f32"),        # one token into a second CTA
 ]
 
