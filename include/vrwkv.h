@@ -291,7 +291,7 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r,
  *   gw_total, gu_total  float32[C] or NULL: if given, that sum over b, taken
  *             in order b = 0..B-1 by a second kernel on the same stream.
  * Arithmetic is float32; dw and du are summed in a fixed order, so repeated
- * calls give identical bits.  With C % 16 == 0 and 16-byte-aligned k, v, gy
+ * calls give identical bits.  With C % 8 == 0 and 16-byte-aligned k, v, gy
  * the inputs arrive by TMA, else by direct loads (VRWKV_DISABLE_TMA=1 forces
  * the direct loads; same results).
  * Limits: T <= 4096 (UNSUPPORTED above, or when the GPU cannot co-schedule

@@ -20,30 +20,31 @@
 // carried across a segment of L tokens whose own contribution is (a, h):
 //   A' = a^L A + a,   H' = a^L (H + L A) + h,
 // an associative composition, so both scans run as in the forward kernel:
-// walks over a thread's 4 tokens, shuffle scans over the 4 chunks of a warp,
-// a CTA scan over its 16 warps and an exchange across the CTAs of a cluster.
+// walks over a thread's 8 tokens, shuffle scans over the 8 chunks of a warp,
+// a CTA scan over its 8 warps and an exchange across the CTAs of a cluster.
 // Round 1 scans (p v, p) with their H parts and yields y, q, r and the dw, du
 // terms; round 2 scans (q, r) and yields dk and dv.
 //
-// Work decomposition.  A CTA owns batch row b, a slab of 16 channels and 256
-// tokens; T > 256 splits over a cluster of up to 16 CTAs (T <= 4096).  Thread
-// = 2 adjacent channels (packed float2) x 8 consecutive tokens; the 32 lanes
-// of a warp are 8 channel pairs x 4 consecutive chunks; 256 threads, two CTAs
-// per SM within 128 registers: the per-token forward states (round 1) and
-// prefix sums (round 2) wait in shared memory between the two walks, and p v
-// is recomputed from p and v instead of being kept.  Inputs come straight
-// from global memory: at each token step a warp reads four 16-channel rows.
-// Inputs of 16-byte-aligned tensors with C % 16 == 0 arrive by TMA in the
-// forward kernel's tile layout (element stride 8 along T: sub-tile i, row q is
-// token i of chunk q, so a warp's four chunks read four consecutive rows),
-// into shared memory that the per-token stash reuses afterwards; other
-// tensors load straight from global memory.
+// Work decomposition.  A CTA owns batch row b, a slab of 8 channels and 512
+// tokens; T > 512 splits over a cluster of up to 8 CTAs (T <= 4096), which
+// at two CTAs per SM spans four SMs and packs onto the GPCs far better than
+// 16-CTA clusters.  Thread = 2 adjacent channels (packed float2) x 8
+// consecutive tokens; the 32 lanes of a warp are 4 channel pairs x 8
+// consecutive chunks; 256 threads, two CTAs per SM within 128 registers: the
+// per-token forward states (round 1) and prefix sums (round 2) wait in shared
+// memory between the two walks, and p v is recomputed from p and v instead of
+// being kept.  Inputs of 16-byte-aligned tensors with C % 8 == 0 arrive by
+// TMA in the forward kernel's tile layout (element stride 8 along T: sub-tile
+// i, row q is token i of chunk q, so a warp's eight chunks read eight
+// consecutive rows), into shared memory that the per-token stash reuses
+// afterwards; other tensors load straight from global memory.
+// The CTAs of a column exchange their records with asynchronous stores into
+// each other's shared memory that complete on the receiver's mailbox
+// mbarrier (one per exchange round), so no cluster-wide barrier is waited on.
 // Exponents are base 2 (log2 e is folded into k, u and w).
 #pragma once
 
 #include <cuda.h>
-
-#include <cooperative_groups.h>
 
 #include "biwkv_tma.cuh"
 #include "common.cuh"
@@ -51,16 +52,16 @@
 namespace vrwkv {
 namespace bwd {
 
-namespace cg = cooperative_groups;
-
-constexpr int kCS = 16;                    // channels per CTA
+constexpr int kCS = 8;                     // channels per CTA (a column slab)
 constexpr int kNP = kCS / 2;               // channel pairs
 constexpr int kL = 8;                      // tokens per thread
 constexpr int kThreads = 256;
 constexpr int kNW = kThreads / 32;         // 8 warps
-constexpr int kTc = kThreads / kNP * kL;   // 256 tokens per CTA
-constexpr int kWarpTok = 4 * kL;           // 16 tokens per warp
-constexpr int kClusterMax = 16;
+constexpr int kCPW = 32 / kNP;             // chunks per warp (8)
+constexpr int kTc = kThreads / kNP * kL;   // 512 tokens per CTA
+constexpr int kWarpTok = kCPW * kL;        // 64 tokens per warp
+constexpr int kMaxT = 4096;
+constexpr int kClusterMax = kMaxT / kTc;   // 8
 
 struct alignas(64) Params {
     CUtensorMap map[3];  // k, v, g (TMA path)
@@ -84,11 +85,11 @@ struct alignas(64) Params {
 
 // Round-1 record of one channel pair: sums of p v and p with their
 // distance-weighted parts.
-struct R1 {
+struct alignas(16) R1 {
     float2 apv, ap, hpv, hp;
 };
 // Round-2 record: sums of q and r.
-struct R2 {
+struct alignas(16) R2 {
     float2 aq, ar;
 };
 
@@ -168,7 +169,26 @@ struct alignas(16) Scratch {
     R1 k1F[kNP], k1B[kNP];
     R2 k2F[kNP], k2B[kNP];
     float2 kMc[kNP];
+    unsigned long long xbar[2];  // mailbox barriers of the two exchange rounds
 };
+
+// Bytes one peer stores into a mailbox per channel pair: round 1 two R1 and
+// the maximum; round 2 two R2, dw and du.
+constexpr unsigned kRec1Bytes = 2 * sizeof(R1) + sizeof(float2);
+constexpr unsigned kRec2Bytes = 2 * sizeof(R2) + 2 * sizeof(float2);
+
+// Asynchronous store of one record into a peer's shared memory, completing
+// its bytes on the peer's mailbox barrier.
+__device__ __forceinline__ void st_async(unsigned raddr, const R1& x, unsigned rbar) {
+    fast::st_async4(raddr, make_float4(x.apv.x, x.apv.y, x.ap.x, x.ap.y), rbar);
+    fast::st_async4(raddr + 16, make_float4(x.hpv.x, x.hpv.y, x.hp.x, x.hp.y), rbar);
+}
+__device__ __forceinline__ void st_async(unsigned raddr, const R2& x, unsigned rbar) {
+    fast::st_async4(raddr, make_float4(x.aq.x, x.aq.y, x.ar.x, x.ar.y), rbar);
+}
+__device__ __forceinline__ unsigned peer_addr(const void* local, int peer) {
+    return fast::mapa_u32(fast::smem_u32(local), (unsigned)peer);
+}
 
 // Per-token state between the two walks of a round, as two 16-byte planes
 // [token][thread] (a thread's accesses are 16 bytes at a 16-byte stride:
@@ -178,7 +198,7 @@ constexpr size_t kStashBytes = 2 * sizeof(float4) * kL * kThreads;
 // the stash starts 128-byte aligned (it also receives the TMA tiles)
 constexpr size_t kStashOff = (sizeof(Scratch) + 127) / 128 * 128;
 constexpr size_t kSmemBytes = kStashOff + kStashBytes + 128;  // + re-alignment slack
-constexpr int kTileRows = kTc / kL;  // rows of one sub-tile (32)
+constexpr int kTileRows = kTc / kL;  // rows of one sub-tile (64)
 
 template <typename IO>
 __device__ __forceinline__ float2 load_pair(const char* base, size_t row_elem, int cA, int C, bool ok_t,
@@ -214,9 +234,9 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
     __shared__ unsigned long long tma_bar;
 
     const int tid = threadIdx.x;
-    const int j = tid & 7;    // channel pair
-    const int q = tid >> 3;   // chunk within the CTA (0..31)
-    const int cq = q & 3;     // chunk within the warp
+    const int j = tid % kNP;  // channel pair
+    const int q = tid / kNP;  // chunk within the CTA (0..63)
+    const int cq = q % kCPW;  // chunk within the warp
     const int warp = tid >> 5;
     const int rank = blockIdx.x;
     const int c0 = blockIdx.y * kCS;
@@ -233,16 +253,32 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
     constexpr int SUB = kTileRows * RB;    // bytes per sub-tile
     constexpr int TILE = kL * SUB;         // bytes per tile
     char* tiles = smem + kStashOff;        // k, v, g tiles (the stash later)
+    if (tid == 0) {
+        if (p.tma) fast::mbar_init(&tma_bar, 1);
+        if (multi) {
+            // mailbox barriers: one arrival (here) plus every peer's bytes
+            fast::mbar_init(&S.xbar[0], 1);
+            fast::mbar_expect_tx(&S.xbar[0], (unsigned)p.ncl * kNP * kRec1Bytes);
+            fast::mbar_init(&S.xbar[1], 1);
+            fast::mbar_expect_tx(&S.xbar[1], (unsigned)p.ncl * kNP * kRec2Bytes);
+        }
+    }
+    __syncthreads();
+    // every CTA's mailbox barriers exist before a peer stores: arrive now,
+    // wait just before the first store
+    if (multi) fast::cluster_arrive_relaxed();
     if (p.tma) {
-        if (tid == 0) fast::mbar_init(&tma_bar, 1);
-        __syncthreads();
         if (warp == 0) {
             if (tid == 0) fast::mbar_expect_tx(&tma_bar, (unsigned)(3 * TILE));
             __syncwarp();
             if (tid < kL) {
+                // two boxes of 256 strided tokens (32 rows) per sub-tile
 #pragma unroll
                 for (int s3 = 0; s3 < 3; ++s3)
-                    fast::tma_load_3d(tiles + s3 * TILE + tid * SUB, &p.map[s3], c0, t0 + tid, b, &tma_bar);
+#pragma unroll
+                    for (int h = 0; h < kTc / 256; ++h)
+                        fast::tma_load_3d(tiles + s3 * TILE + tid * SUB + h * 32 * RB, &p.map[s3], c0,
+                                          t0 + tid + 256 * h, b, &tma_bar);
             }
         }
     }
@@ -292,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
     }
     // CTA maximum of k per channel
 #pragma unroll
-    for (int d = 8; d <= 16; d <<= 1) {
+    for (int d = kNP; d < 32; d <<= 1) {
         mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
         mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
     }
@@ -323,24 +359,24 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         lb.apv = fma2(alpha, lb.apv, mul2(pp[i], vv[i]));
         lb.ap = fma2(alpha, lb.ap, pp[i]);
     }
-    // warp scan over the 4 chunks (lanes 8 apart)
+    // warp scan over the kCPW chunks (lanes kNP apart)
     R1 fI = lf, bI = lb;
 #pragma unroll
-    for (int d = 1; d < 4; d <<= 1) {
+    for (int d = 1; d < kCPW; d <<= 1) {
         const float L = (float)(kL * d);
         const float2 aL = decay(lam2, L);
-        const R1 o = shfl_up(fI, 8 * d, 32);
+        const R1 o = shfl_up(fI, kNP * d, 32);
         if (cq >= d) fI = r1_cross(o, aL, L, fI);
-        const R1 o2 = shfl_down(bI, 8 * d, 32);
-        if (cq + d < 4) bI = r1_cross(o2, aL, L, bI);
+        const R1 o2 = shfl_down(bI, kNP * d, 32);
+        if (cq + d < kCPW) bI = r1_cross(o2, aL, L, bI);
     }
-    R1 X1 = shfl_up(fI, 8, 32), Y1 = shfl_down(bI, 8, 32);  // lane-exclusive
+    R1 X1 = shfl_up(fI, kNP, 32), Y1 = shfl_down(bI, kNP, 32);  // lane-exclusive
     if (cq == 0) X1 = r1_zero();
-    if (cq == 3) Y1 = r1_zero();
-    if (cq == 3) S.w1F[j][warp] = fI;
+    if (cq == kCPW - 1) Y1 = r1_zero();
+    if (cq == kCPW - 1) S.w1F[j][warp] = fI;
     if (cq == 0) S.w1B[j][warp] = bI;
     __syncthreads();
-    // CTA scan over the 16 warps: thread (pair jj, warp wi)
+    // CTA scan over the warps: thread (pair jj, warp wi)
     if (tid < kNP * kNW) {
         const int jj = tid / kNW, wi = tid % kNW;
         const float2 wjw = make_float2(c0 + 2 * jj < p.C ? __ldg(p.w + c0 + 2 * jj) : 0.f,
@@ -370,23 +406,25 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         }
     }
     __syncthreads();
-    // cluster exchange 1: push the records into every peer's mailbox (one
-    // (peer, pair, part) per thread), then one cluster barrier
+    // cluster exchange 1: asynchronous stores of the records into every
+    // peer's mailbox (one (peer, pair, part) per thread), then a bounded wait
+    // until this CTA's own mailbox is full
     if (multi) {
-        cg::cluster_group cluster = cg::this_cluster();
+        fast::cluster_wait_acquire();  // every mailbox barrier is initialised
         for (int e = tid; e < p.ncl * kNP * 3; e += kThreads) {  // (peer, pair, part)
             const int peer = e / (kNP * 3), jj = (e / 3) % kNP, part = e % 3;
-            Scratch* P = cluster.map_shared_rank(&S, peer);
-            if (part == 0) P->mb1F[rank][jj] = S.own1F[jj];
-            else if (part == 1) P->mb1B[rank][jj] = S.own1B[jj];
-            else P->mbM[rank][jj] = S.ownM[jj];
+            const unsigned rbar = peer_addr(&S.xbar[0], peer);
+            if (part == 0) st_async(peer_addr(&S.mb1F[rank][jj], peer), S.own1F[jj], rbar);
+            else if (part == 1) st_async(peer_addr(&S.mb1B[rank][jj], peer), S.own1B[jj], rbar);
+            else fast::st_async2(peer_addr(&S.mbM[rank][jj], peer), S.ownM[jj], rbar);
         }
-        cluster.sync();
+        if (tid == 0) fast::mbar_wait_cluster_bounded(&S.xbar[0], p.err);
+        __syncthreads();
     }
     // carries into this CTA: one thread per (channel, direction), a fixed-order
     // fold over the peers in the common exponent frame Mc
     if (tid < 2 * kCS) {
-        const int lc = tid & 15, dir = tid >> 4, jj = lc >> 1, hi = lc & 1;
+        const int lc = tid % kCS, dir = tid / kCS, jj = lc >> 1, hi = lc & 1;
         const float lw = (c0 + lc < p.C ? __ldg(p.w + c0 + lc) : 0.f) * (p.invT * kLog2e);
         float Mc = comp(S.ownM[jj], hi);
         float kapv = 0.f, kap = 0.f, khpv = 0.f, khp = 0.f;
@@ -420,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         const float Lw = (float)(kWarpTok * warp), Ll = (float)(kL * cq);
         KF = r1_cross(S.k1F[j], decay(lam2, Lw), Lw, r1_scale(S.c1F[j][warp], sl));
         KF = r1_cross(KF, decay(lam2, Ll), Ll, r1_scale(X1, sl));
-        const float Lw2 = (float)(kWarpTok * (kNW - 1 - warp)), Ll2 = (float)(kL * (3 - cq));
+        const float Lw2 = (float)(kWarpTok * (kNW - 1 - warp)), Ll2 = (float)(kL * (kCPW - 1 - cq));
         KB = r1_cross(S.k1B[j], decay(lam2, Lw2), Lw2, r1_scale(S.c1B[j][warp], sl));
         KB = r1_cross(KB, decay(lam2, Ll2), Ll2, r1_scale(Y1, sl));
     }
@@ -483,21 +521,21 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
     }
     R2 fJ = mf, bJ = mb;
 #pragma unroll
-    for (int d = 1; d < 4; d <<= 1) {
+    for (int d = 1; d < kCPW; d <<= 1) {
         const float2 aL = decay(lam2, (float)(kL * d));
-        const R2 o = shfl_up(fJ, 8 * d, 32);
+        const R2 o = shfl_up(fJ, kNP * d, 32);
         if (cq >= d) fJ = r2_cross(o, aL, fJ);
-        const R2 o2 = shfl_down(bJ, 8 * d, 32);
-        if (cq + d < 4) bJ = r2_cross(o2, aL, bJ);
+        const R2 o2 = shfl_down(bJ, kNP * d, 32);
+        if (cq + d < kCPW) bJ = r2_cross(o2, aL, bJ);
     }
-    R2 X2 = shfl_up(fJ, 8, 32), Y2 = shfl_down(bJ, 8, 32);
+    R2 X2 = shfl_up(fJ, kNP, 32), Y2 = shfl_down(bJ, kNP, 32);
     if (cq == 0) X2 = r2_zero();
-    if (cq == 3) Y2 = r2_zero();
-    if (cq == 3) S.w2F[j][warp] = fJ;
+    if (cq == kCPW - 1) Y2 = r2_zero();
+    if (cq == kCPW - 1) S.w2F[j][warp] = fJ;
     if (cq == 0) S.w2B[j][warp] = bJ;
-    // dw, du partial sums: over the warp's 4 chunks, then over the warps
+    // dw, du partial sums: over the warp's chunks, then over the warps
 #pragma unroll
-    for (int d = 8; d <= 16; d <<= 1) {
+    for (int d = kNP; d < 32; d <<= 1) {
         gwa = add2(gwa, make_float2(__shfl_xor_sync(0xffffffffu, gwa.x, d), __shfl_xor_sync(0xffffffffu, gwa.y, d)));
         gua = add2(gua, make_float2(__shfl_xor_sync(0xffffffffu, gua.x, d), __shfl_xor_sync(0xffffffffu, gua.y, d)));
     }
@@ -538,20 +576,20 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         }
     }
     __syncthreads();
-    if (multi) {
-        cg::cluster_group cluster = cg::this_cluster();
+    if (multi) {  // cluster exchange 2, as exchange 1 on the second mailbox barrier
         for (int e = tid; e < p.ncl * kNP * 4; e += kThreads) {  // (peer, pair, part)
             const int peer = e / (kNP * 4), jj = (e / 4) % kNP, part = e % 4;
-            Scratch* P = cluster.map_shared_rank(&S, peer);
-            if (part == 0) P->mb2F[rank][jj] = S.own2F[jj];
-            else if (part == 1) P->mb2B[rank][jj] = S.own2B[jj];
-            else if (part == 2) P->mbW[rank][jj] = S.ownW[jj];
-            else P->mbU[rank][jj] = S.ownU[jj];
+            const unsigned rbar = peer_addr(&S.xbar[1], peer);
+            if (part == 0) st_async(peer_addr(&S.mb2F[rank][jj], peer), S.own2F[jj], rbar);
+            else if (part == 1) st_async(peer_addr(&S.mb2B[rank][jj], peer), S.own2B[jj], rbar);
+            else if (part == 2) fast::st_async2(peer_addr(&S.mbW[rank][jj], peer), S.ownW[jj], rbar);
+            else fast::st_async2(peer_addr(&S.mbU[rank][jj], peer), S.ownU[jj], rbar);
         }
-        cluster.sync();
+        if (tid == 0) fast::mbar_wait_cluster_bounded(&S.xbar[1], p.err);
+        __syncthreads();
     }
     if (tid < 2 * kCS) {
-        const int lc = tid & 15, dir = tid >> 4, jj = lc >> 1, hi = lc & 1;
+        const int lc = tid % kCS, dir = tid / kCS, jj = lc >> 1, hi = lc & 1;
         float kq = 0.f, kr = 0.f;
         if (multi) {
             const float lw = (c0 + lc < p.C ? __ldg(p.w + c0 + lc) : 0.f) * (p.invT * kLog2e);
@@ -589,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         const float2 aW = decay(lam2, (float)(kWarpTok * warp)), aLn = decay(lam2, (float)(kL * cq));
         QF = r2_cross(r2_cross(S.k2F[j], aW, S.c2F[j][warp]), aLn, X2);
         const float2 aW2 = decay(lam2, (float)(kWarpTok * (kNW - 1 - warp)));
-        const float2 aLn2 = decay(lam2, (float)(kL * (3 - cq)));
+        const float2 aLn2 = decay(lam2, (float)(kL * (kCPW - 1 - cq)));
         QB = r2_cross(r2_cross(S.k2B[j], aW2, S.c2B[j][warp]), aLn2, Y2);
     }
 #pragma unroll
@@ -615,8 +653,9 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         QB.aq = fma2(alpha, QB.aq, qq[i]);
         QB.ar = fma2(alpha, QB.ar, rr[i]);
     }
-    // no closing cluster barrier: the last remote writes precede the second
-    // exchange barrier and no CTA touches another's memory after it
+    // no closing cluster barrier: every peer's stores into this CTA completed
+    // before its second mailbox wait, and no CTA touches another's memory
+    // after that
 }
 
 // dw, du of the batch: the per-row parts summed over b in order.

@@ -36,14 +36,10 @@
 
 #include <cuda.h>
 
-#include <cooperative_groups.h>
-
 #include "common.cuh"
 
 namespace vrwkv {
 namespace fast {
-
-namespace cg = cooperative_groups;
 
 constexpr int kCS = 8;          // channels per CTA (a column slab)
 constexpr int kNP = kCS / 2;    // channel pairs per CTA

@@ -1052,8 +1052,7 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
         return fail(VRWKV_ERR_INVALID_ARG, "B, T and C must be positive (got %d, %d, %d)", B, T, C);
     if (!k || !v || !w || !u || !gy || !gk || !gv || !gw || !gu)
         return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
-    if (T > bwd::kTc * bwd::kClusterMax)
-        return fail(VRWKV_ERR_UNSUPPORTED, "T = %d exceeds %d", T, bwd::kTc * bwd::kClusterMax);
+    if (T > bwd::kMaxT) return fail(VRWKV_ERR_UNSUPPORTED, "T = %d exceeds %d", T, bwd::kMaxT);
     const int es = elem_bytes(dtype);
     const void* toks[5] = {k, v, gy, gk, gv};
     for (const void* t : toks)
@@ -1091,8 +1090,9 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
     p.invT = (float)(1.0 / (double)T);
     p.vec = (C % 2 == 0);
     for (const void* t : toks) p.vec = p.vec && aligned(t, 2 * es);
-    // k, v and gy by TMA (tiles of 16 channels x 256 tokens, element stride 8
-    // along T, as the forward kernel's) when the shape and alignment allow
+    // k, v and gy by TMA (tiles of 8 channels x 512 tokens as two boxes of 256
+    // strided tokens, element stride 8 along T, as the forward kernel's) when
+    // the shape and alignment allow
     p.tma = 0;
     p.err = device_error_word();
     if (!tma_disabled() && C % bwd::kCS == 0 && p.err && aligned(k, 16) && aligned(v, 16) && aligned(gy, 16)) {
@@ -1103,7 +1103,7 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
                 dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
             const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
             const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
-            const cuuint32_t box[3] = {(cuuint32_t)bwd::kCS, (cuuint32_t)bwd::kTc, 1};
+            const cuuint32_t box[3] = {(cuuint32_t)bwd::kCS, 256u, 1};  // 32 strided rows
             const cuuint32_t estr[3] = {1, (cuuint32_t)bwd::kL, 1};
             bool okm = true;
             for (int i = 0; i < 3 && okm; ++i)
@@ -1135,15 +1135,11 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
     cfg.attrs = attr;
     cfg.numAttrs = p.ncl > 1 ? 2 : 0;
     if (p.ncl > 1) {
-        static std::atomic<int> nonportable[2] = {{0}, {0}};
+        // clusters of at most 8 CTAs (T <= 4096): a portable size
+        static_assert(bwd::kClusterMax <= 8, "portable cluster size");
         static std::atomic<int> checked[2][bwd::kClusterMax + 1];
         const int di = dtype == VRWKV_F32 ? 0 : 1;
         cudaError_t e;
-        if (p.ncl > 8 && !nonportable[di].load()) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-            if (e != cudaSuccess) return cuda_status(e, "cluster size attribute");
-            nonportable[di].store(1);
-        }
         int v2 = checked[di][p.ncl].load();
         if (v2 == 0) {
             int n = 0;
