@@ -18,7 +18,10 @@ column is independent): each rank processes its own batch, no collective
 touches the data path, and the value is the whole-job throughput.
 
 The JSON line also carries the roofline of the fused kernel (algorithmic
-bytes / average launch time against the measured HBM copy bandwidth), an
+bytes / average launch time against the measured HBM copy bandwidth), its
+instruction-issue roofline (``issue_roofline``: ncu's warp-instruction count
+per launch over the launch time, against 4 per SM per clock; the kernel is
+bound by issue, not by HBM), an
 end-to-end figure through the C ABI with host buffers, the float64 CPU
 oracle timed on a bounded sample, and SM clocks sampled during the timed
 region.  ``--impl reference`` times the CPU oracle alone on the same metric.
@@ -201,19 +204,43 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def committed_traffic(key: str, kernel: str):
-    """dram bytes per launch from the committed ncu summary, if it was taken
-    on `kernel` as currently written and on this workload."""
+def committed_record(key: str, kernel: str):
+    """The committed ncu record of `kernel` on this workload, if it was taken
+    on the kernel as currently written (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)
         ent = rec.get(key)
         if ent and ent.get("kernel") == kernel and ent.get("kernel_sha") == kernel_source_hash(kernel):
-            return float(ent["dram_bytes_per_launch"])
+            return ent
     except Exception:
         pass
     return None
+
+
+def committed_traffic(key: str, kernel: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on `kernel` as currently written and on this workload."""
+    ent = committed_record(key, kernel)
+    return float(ent["dram_bytes_per_launch"]) if ent else None
+
+
+WARP_SCHEDULERS_PER_SM = 4  # one warp-instruction issued per scheduler per clock
+
+
+def issue_roofline(warp_inst_per_launch, launch_s, sms, sm_mhz):
+    """Instruction-issue roofline of a kernel bound by its arithmetic rather
+    than by HBM: warp-instructions per launch (ncu smsp__inst_executed.sum)
+    over the launch time, against SMs x 4 schedulers x 1 per clock at the SM
+    clock sampled during the run."""
+    if not warp_inst_per_launch or not launch_s or not sms or not sm_mhz:
+        return None
+    achieved = warp_inst_per_launch / launch_s / 1e9
+    peak = sms * WARP_SCHEDULERS_PER_SM * sm_mhz / 1e3
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "G warp-instructions/s",
+            "frac": achieved / peak, "warp_inst_per_launch": warp_inst_per_launch,
+            "peak_basis": f"{sms} SMs x {WARP_SCHEDULERS_PER_SM} schedulers x 1/clock x {sm_mhz:.0f} MHz"}
 
 
 def make_inputs(wl, torch, dev, rank):
@@ -450,7 +477,7 @@ def time_block(runner, stream, torch, dev, launches: int):
             "timing": "CUDA graphs over the rotating buffer sets"}
 
 
-def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float):
+def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float, sm_mhz=None):
     """Roofline of the Bi-WKV backward (vrwkv_biwkv_bwd) at the workload's
     (B, T, C) and dtype, timed in its own region: k, v and gy read once, gk
     and gv written once, w, u read and the per-row dw, du written."""
@@ -489,9 +516,13 @@ def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float):
     es = 4 if wl.dtype == "f32" else 2
     nbytes = 5 * wl.N * es + 2 * wl.C * 4 + 2 * wl.B * wl.C * 4
     achieved = nbytes / (us * 1e-6) / 1e9
+    rec = committed_record("biwkv_bwd/" + wl.name, kname)
+    issue = issue_roofline(rec.get("warp_inst_per_launch") if rec else None, us * 1e-6,
+                           torch.cuda.get_device_properties(dev).multi_processor_count, sm_mhz)
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": committed_traffic("biwkv_bwd/" + wl.name, kname),
             "kernel": kname, "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
+            "issue_roofline": issue,
             "launches": launches, "timing": "back-to-back launches (each allocates its outputs)"}
 
 
@@ -609,6 +640,11 @@ def run_ours(args, dist):
     peak, peak_kind = measured_hbm_peak()
     achieved = fused_bytes / launch_s / 1e9
     traffic = committed_traffic(wl.name, runner.kernel_name)
+    rec = committed_record(wl.name, runner.kernel_name)
+    clk = clocks.summary()
+    issue = issue_roofline(rec.get("warp_inst_per_launch") if rec else None, launch_s,
+                           torch.cuda.get_device_properties(dev).multi_processor_count,
+                           (clk or {}).get("sm_mhz") or (clk or {}).get("sm_max_mhz"))
 
     # end to end through the C ABI with pinned host buffers
     e2e_steps = max(3, min(args.steps, 50))
@@ -650,9 +686,10 @@ def run_ours(args, dist):
                      "kernel": runner.kernel_name,
                      "algorithmic_bytes_per_launch": fused_bytes,
                      "avg_launch_us": launch_s * 1e6},
+        "issue_roofline": issue,
         "e2e": e2e,
         "gpu_launches": steps * runner.launches_per_step,
-        "clocks": clocks.summary(),
+        "clocks": clk,
     }
     # correctness guard on the main step's last output (first set of the
     # rotation), taken before the rows below reuse the device
@@ -672,7 +709,8 @@ def run_ours(args, dist):
         blk = time_block(runner, stream, torch, dev, max(20, args.row_launches // 20))
         if blk is not None:
             rows["spatial_mix_block"] = blk
-        bw = time_biwkv_bwd(runner, stream, torch, dev, max(20, args.row_launches // 20), peak)
+        bw = time_biwkv_bwd(runner, stream, torch, dev, max(20, args.row_launches // 20), peak,
+                            sm_mhz=(clk or {}).get("sm_mhz"))
         if bw is not None:
             rows["biwkv_bwd"] = bw
         if rows:

@@ -87,3 +87,16 @@ def test_kernel_source_hash_is_stable():
         assert bench.kernel_source_hash(kern) == bench.kernel_source_hash(kern)
         assert len(bench.kernel_source_hash(kern)) == 16
     assert bench.kernel_source_hash("biwkv_tma_kernel") != bench.kernel_source_hash("biwkv_bwd_kernel")
+
+
+def test_issue_roofline_arithmetic():
+    import bench
+    # 45.7 M warp-instructions in 100 us on 148 SMs at 2000 MHz:
+    # 457 G/s of 148 * 4 * 2 = 1184 G/s
+    r = bench.issue_roofline(45.7e6, 100e-6, 148, 2000.0)
+    assert r["bound"] == "alu"
+    assert abs(r["achieved"] - 457.0) < 1e-9
+    assert abs(r["peak"] - 1184.0) < 1e-9
+    assert abs(r["frac"] - 457.0 / 1184.0) < 1e-12
+    assert bench.issue_roofline(None, 100e-6, 148, 2000.0) is None
+    assert bench.issue_roofline(45.7e6, 100e-6, 148, None) is None
