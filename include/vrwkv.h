@@ -142,8 +142,9 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *   (and, with qs, a channel-group size int(C*gamma) that is a multiple of
  *   8 and W <= 256); everything else runs a generic kernel with the same
  *   results up to rounding.  Setting VRWKV_DISABLE_TMA=1 in the environment
- *   forces the generic kernel, and VRWKV_TMA_CHUNK=8 holds the fast path to
- *   8-token thread chunks (diagnostics).
+ *   forces the generic kernel, VRWKV_TMA_CHUNK=8 holds the fast path to
+ *   8-token thread chunks and VRWKV_NO_TMA_STORE=1 to per-thread stores of
+ *   its results (diagnostics).
  * Limits: T <= 4096 (UNSUPPORTED above); on the generic kernel with qs, a
  *   halo of shift_pixel*W tokens must fit its shared-memory tile.
  *   Exponents are renormalised by the running maximum of k, so a constant

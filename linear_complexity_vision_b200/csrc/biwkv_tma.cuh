@@ -69,6 +69,7 @@ enum Layout { kKV = 0, kRKV = 1, kX = 2 };
 
 struct alignas(64) Params {
     CUtensorMap map[3];  // one per distinct source tensor (tile order below)
+    CUtensorMap omap;    // the output, in the tiles' layout (stores by TMA)
     const float* w;
     const float* u;
     const float* mu[3];  // mu of r, k, v (each nullable)
@@ -84,6 +85,7 @@ struct alignas(64) Params {
     int ncl;             // CTAs per column (cluster size)
     int tile_bytes;      // bytes per tile: 8 sub-tiles of 32 token rows
     int box_bytes;       // bytes one strided box delivers (zero fill included)
+    int tma_store;       // results leave by TMA stores (the CTA's span is whole boxes, or the column's end)
     // global-memory exchange (GX kernels only): see the workspace layout below
     unsigned int* ws_ctl;   // [0] ticket counter, [1] finished CTAs, [2] generation
     unsigned int* ws_flag;  // per (column, rank): generation + 1 once its record is out
@@ -185,6 +187,23 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
         "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
         "r"(smem_u32(bar))
         : "memory");
+}
+// Store a box of a shared-memory tile to global memory (bulk async group);
+// elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<unsigned long long>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Generic-proxy writes to shared memory become visible to the async proxy
+// (TMA) of this CTA.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_arrive_release() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
@@ -783,8 +802,19 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
             Io<IO>::st_pair(tout + rowoff + i * SUB, mul2(num, rcp(den)));
         }
     }
-    __syncthreads();
-    {
+    if (p.tma_store) {
+        // lane i of warp 0 stores sub-tile i: boxes of 256 strided tokens,
+        // clipped at T by the tensor map
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid < kL) {
+            const int nbox = (tend - t0 + 255) / 256;
+            for (int hb = 0; hb < nbox; ++hb)
+                tma_store_3d(&p.omap, tout + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
+            bulk_commit_and_wait_read();
+        }
+    } else {
+        __syncthreads();
         constexpr int UPS = SUB / 16;  // 16-byte units per sub-tile
         char* gout = p.out + ((size_t)b * p.T + t0) * p.C * es + (size_t)c0 * es;
 #pragma unroll

@@ -345,6 +345,13 @@ bool tma_disabled() {
     return e && e[0] && e[0] != '0';
 }
 
+// VRWKV_NO_TMA_STORE=1 makes the forward TMA path write its results with
+// plain 16-byte stores instead of TMA stores (diagnostics).
+bool tma_store_disabled() {
+    const char* e = getenv("VRWKV_NO_TMA_STORE");
+    return e && e[0] && e[0] != '0';
+}
+
 // VRWKV_TMA_CHUNK=8 keeps the forward TMA path on 8-token thread chunks even
 // where the 16-token kernel qualifies (diagnostics and tests).
 bool tma_chunk8_forced() {
@@ -594,6 +601,19 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         }
         if (cr != CUDA_SUCCESS) return false;
+    }
+    {
+        // the output in the tiles' layout: boxes of 256 strided tokens; a CTA
+        // stores by TMA when its span is whole boxes or ends the column, so no
+        // box reaches another CTA's tokens (the tensor bound clips at T)
+        const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+        const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
+        const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, 256u, 1};
+        const cuuint32_t estr[3] = {1, (cuuint32_t)fast::kL, 1};
+        const CUresult cr = enc(&p.omap, dt, 3, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        p.tma_store = (cr == CUDA_SUCCESS && (p.Tc % 256 == 0 || p.ncl == 1) && !tma_store_disabled()) ? 1 : 0;
     }
     p.gslab = pl.qs ? p.g / fast::kCS : 0;
     p.invT = (float)(1.0 / (double)T);
