@@ -65,8 +65,10 @@ constexpr int kClusterMax = kMaxT / kTc;   // 8
 
 struct alignas(64) Params {
     CUtensorMap map[3];  // k, v, g (TMA path)
+    CUtensorMap omap[2]; // gk, gv in the same layout (TMA stores)
     unsigned int* err;   // device error word (bounded TMA wait)
     int tma;             // inputs arrive by TMA
+    int tma_store;       // gk, gv leave by TMA stores from shared memory
     const char* k;
     const char* v;
     const char* g;  // upstream gradient dL/dy
@@ -636,6 +638,10 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         QF.aq = fma2(alpha, QF.aq, qq[i]);
         QF.ar = fma2(alpha, QF.ar, rr[i]);
     }
+    // with TMA stores the results gather in two tiles in the stash's second
+    // plane (free since round 1), at the input tiles' offsets
+    char* otile = reinterpret_cast<char*>(plane1);
+    const int orow = q * RB + j * 2 * es;  // token i of chunk q: + i * SUB
 #pragma unroll
     for (int i = kL - 1; i >= 0; --i) {
         const float4 s0 = plane0[i * kThreads + tid];
@@ -646,12 +652,32 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         const float2 Sr = fma2(eu, rr[i], add2(fq.ar, QB.ar));
         const float2 dv = mul2(pp[i], Sq);
         const float2 dk = fma2(vv[i], dv, mul2(make_float2(-pp[i].x, -pp[i].y), Sr));
-        const int t = s_tok + i;
-        const size_t row = ((size_t)b * p.T + t) * p.C;
-        store_pair<IO>(p.gv, row, cA, p.C, t < tend, vec, dv);
-        store_pair<IO>(p.gk, row, cA, p.C, t < tend, vec, dk);
+        if (p.tma_store) {
+            Io<IO>::st_pair(otile + orow + i * SUB, dk);
+            Io<IO>::st_pair(otile + TILE + orow + i * SUB, dv);
+        } else {
+            const int t = s_tok + i;
+            const size_t row = ((size_t)b * p.T + t) * p.C;
+            store_pair<IO>(p.gv, row, cA, p.C, t < tend, vec, dv);
+            store_pair<IO>(p.gk, row, cA, p.C, t < tend, vec, dk);
+        }
         QB.aq = fma2(alpha, QB.aq, qq[i]);
         QB.ar = fma2(alpha, QB.ar, rr[i]);
+    }
+    if (p.tma_store) {
+        // lane i of warp 0 stores sub-tile i of gk and gv: boxes of 256
+        // strided tokens, clipped at T by the tensor maps
+        fast::fence_proxy_async_smem();
+        __syncthreads();
+        if (tid < kL) {
+            const int nbox = (tend - t0 + 255) / 256;
+#pragma unroll
+            for (int o2 = 0; o2 < 2; ++o2)
+                for (int hb = 0; hb < nbox; ++hb)
+                    fast::tma_store_3d(&p.omap[o2], otile + o2 * TILE + tid * SUB + hb * 32 * RB, c0,
+                                       t0 + tid + 256 * hb, b);
+            fast::bulk_commit_and_wait_read();
+        }
     }
     // no closing cluster barrier: every peer's stores into this CTA completed
     // before its second mailbox wait, and no CTA touches another's memory

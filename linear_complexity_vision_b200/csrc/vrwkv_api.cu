@@ -352,6 +352,14 @@ bool tma_store_disabled() {
     return e && e[0] && e[0] != '0';
 }
 
+// VRWKV_BWD_TMA_STORE=1 makes the backward kernel store gk, gv by TMA from
+// shared memory; off by default: at two CTAs per SM, waiting for the bulk
+// store to drain delays the next CTA more than the per-thread stores cost.
+bool bwd_tma_store_enabled() {
+    const char* e = getenv("VRWKV_BWD_TMA_STORE");
+    return e && e[0] == '1' && e[1] == 0;
+}
+
 // VRWKV_TMA_CHUNK=8 keeps the forward TMA path on 8-token thread chunks even
 // where the 16-token kernel qualifies (diagnostics and tests).
 bool tma_chunk8_forced() {
@@ -1114,6 +1122,7 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
     // strided tokens, element stride 8 along T, as the forward kernel's) when
     // the shape and alignment allow
     p.tma = 0;
+    p.tma_store = 0;
     p.err = device_error_word();
     if (!tma_disabled() && C % bwd::kCS == 0 && p.err && aligned(k, 16) && aligned(v, 16) && aligned(gy, 16)) {
         EncodeTiledFn enc = encode_fn();
@@ -1131,6 +1140,16 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
             p.tma = okm ? 1 : 0;
+            // optionally, gk, gv leave by TMA stores in the same layout (a CTA
+            // spans 512 tokens or ends the column, so no box reaches another
+            // CTA's tokens)
+            void* dsts[2] = {gk, gv};
+            bool oks = okm && aligned(gk, 16) && aligned(gv, 16) && bwd_tma_store_enabled();
+            for (int i = 0; i < 2 && oks; ++i)
+                oks = enc(&p.omap[i], tdt, 3, dsts[i], dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            p.tma_store = oks ? 1 : 0;
         }
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);

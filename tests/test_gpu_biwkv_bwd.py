@@ -149,6 +149,16 @@ def test_bwd_unaligned(vk, oracle_mod, dt):
     _check(vk, oracle_mod, k, v, g, w, u, dt, offset=1)
 
 
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("B,T,C", [(2, 1000, 16), (1, 4096, 24), (2, 257, 8)])
+def test_bwd_tma_store_path(vk, oracle_mod, monkeypatch, dt, B, T, C):
+    # the optional TMA-store output path (VRWKV_BWD_TMA_STORE=1) against the
+    # oracle: full CTAs, a ragged last CTA and a single short column
+    monkeypatch.setenv("VRWKV_BWD_TMA_STORE", "1")
+    k, v, g, w, u = _inputs(B, T, C, dt, "tma_store")
+    _check(vk, oracle_mod, k, v, g, w, u, dt)
+
+
 def test_bwd_deterministic(vk, oracle_mod):
     k, v, g, w, u = _inputs(2, 1024, 64, "bf16", "det")
     a, _, _, _ = _run(vk, k, v, g, w, u, "bf16")
