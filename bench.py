@@ -70,13 +70,25 @@ KERNEL_SOURCES = {
 }
 
 
+def code_only(text: str) -> str:
+    """CUDA/C++ source without comments, trailing blanks or empty lines: the
+    part that decides what the kernel does (the sources hold no string that
+    contains a comment marker)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the CUDA sources `kernel` is built from."""
+    """Hash of the code (comments and blank lines left out) of the CUDA
+    sources `kernel` is built from: a traffic record stays valid across
+    comment edits and is dropped by any change to the code."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(CSRC, f), "rb") as fh:
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
             h.update(f.encode())
-            h.update(fh.read())
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

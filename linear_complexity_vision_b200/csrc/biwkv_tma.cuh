@@ -9,12 +9,20 @@
 //   C_t, D_t with v = 1,  a = e^{-w/T},  p_i = e^{k_i - M},
 //   wkv_t = (A_t + B_t + e^u p_t v_t) / (C_t + D_t + e^u p_t).
 //
+// Work decomposition: a CTA owns batch row b, a slab of kCS = 8 channels
+// and 512 tokens; a thread owns one channel pair and a chunk of KL tokens
+// (16 by default: two 8-token sub-chunks walked one after the other; 8
+// where a cluster's CTAs cannot hold whole 128-token warps).  Each sub-chunk
+// works relative to its own maximum of k, and the thread, warp, CTA and
+// cluster steps rescale by 2^(M_lower - M_upper) <= 1 on the way up.
+//
 // What makes this path fast:
 //  * Tiles arrive by TMA (cp.async.bulk.tensor, no multicast) with an element
-//    stride of 8 along the token axis: box i (i = 0..7) holds tokens 8q + i,
-//    so sub-tile i, row q is token i of chunk q.  At each step the four
-//    chunks a warp reads are four consecutive rows: conflict-free, and every
-//    address is a compile-time offset from one base register.
+//    stride of 8 along the token axis: box i (i = 0..7) holds tokens 8m + i,
+//    so sub-tile i, row m is token i of sub-chunk m.  At each step the
+//    sub-chunks a warp reads are consecutive rows (every other row with
+//    16-token chunks), and every address is a compile-time offset from one
+//    base register.
 //  * With Q-Shift the (B, T, C) tensor is described as the 4-D image
 //    (C, W, H, B) (W a multiple of 8); the shifted tile x_shift is the same
 //    set of boxes displaced by +-s along w or h.  TMA fills out-of-image
@@ -22,14 +30,17 @@
 //    per-token shift arithmetic remains: token t of both tiles sits at the
 //    same shared-memory offset.  A CTA's kCS channels lie in one channel
 //    group (the host requires the group size to be a multiple of kCS).
-//  * 256-thread CTAs at 64 registers per thread: four CTAs per SM, so one
-//    CTA's barriers and scans overlap another's arithmetic.  Sequences
-//    longer than one CTA's span (256 kL / kNP tokens) split over a
-//    thread-block cluster of up to 16 CTAs along T; CTA aggregates travel
-//    through distributed shared memory.
+//  * Four CTAs per SM (128 threads at <= 128 registers, or 256 at 64), so
+//    one CTA's barriers and scans overlap another's arithmetic.  Sequences
+//    longer than 512 tokens split over a thread-block cluster along T (8
+//    CTAs at T = 4096: two SMs per cluster, so clusters fill every SM); CTA
+//    aggregates travel by asynchronous stores into the peers' shared-memory
+//    mailboxes that complete on the receiver's mbarrier.
+//  * Results go back into the first input tile and leave by TMA tensor
+//    stores in the same strided layout.
 //  * Arrays that a warp reads down a column ([pair][warp], [peer][pair])
 //    have one element of row padding, so those reads are bank-conflict free.
-//  * Decay powers a^(8m) come from a per-CTA table (one exp2 each), the
+//  * Decay powers a^(KL m) come from a per-CTA table (one exp2 each), the
 //    bf16 unpack is integer arithmetic, and arithmetic is packed float2.
 // Exponents are base 2 (log2 e is folded into k, u, w and r).
 #pragma once
@@ -826,8 +837,9 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
                     *reinterpret_cast<const uint4*>(tout + i * SUB + o);
         }
     }
-    // no closing cluster barrier: peers wrote into this CTA's mailbox before
-    // the exchange barrier and nobody reads another CTA's memory after it
+    // no closing cluster barrier: every peer's store into this CTA's mailbox
+    // completed before its mailbox wait, and nobody touches another CTA's
+    // memory after that
     if (GX) {
         // count the CTA out; the last one resets the counters for the next
         // launch and advances the generation

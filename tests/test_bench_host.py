@@ -100,3 +100,19 @@ def test_issue_roofline_arithmetic():
     assert abs(r["frac"] - 457.0 / 1184.0) < 1e-12
     assert bench.issue_roofline(None, 100e-6, 148, 2000.0) is None
     assert bench.issue_roofline(45.7e6, 100e-6, 148, None) is None
+
+
+def test_kernel_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    import shutil
+    import bench
+    for f in bench.KERNEL_SOURCES["biwkv_tma_kernel"]:
+        shutil.copy(os.path.join(bench.CSRC, f), tmp_path / f)
+    monkeypatch.setattr(bench, "CSRC", str(tmp_path))
+    h0 = bench.kernel_source_hash("biwkv_tma_kernel")
+    src = tmp_path / "biwkv_tma.cuh"
+    text = src.read_text()
+    src.write_text("// a new comment line\n" + text.replace("#pragma once", "#pragma once  // trailing", 1)
+                   + "\n/* block\n comment */\n\n")
+    assert bench.kernel_source_hash("biwkv_tma_kernel") == h0
+    src.write_text(text.replace("constexpr int kL = 8;", "constexpr int kL = 9;", 1))
+    assert bench.kernel_source_hash("biwkv_tma_kernel") != h0
