@@ -139,3 +139,77 @@ def test_static_entry_rejects_on_the_host(lib):
     st = lib.vrwkv_spatial_gate_static(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + (1 << 24), 64, 4, 16384,
                                        1, None, None)
     assert st == 2 and b"static workspace" in lib.vrwkv_last_error()
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(B=0), "positive"),
+    (dict(x=None), "NULL"),
+    (dict(dtype=4), "dtype"),
+    (dict(s=-1), "shift_pixel"),
+    (dict(gamma=0.3), "gamma"),
+    (dict(x=FAKE + 1, dtype=1), "misaligned"),
+    (dict(out=FAKE + 64), "overlaps"),
+])
+def test_bishift_rejects_invalid_arguments(lib, args, frag):
+    a = dict(x=FAKE, out=FAKE + (1 << 24), mu=None, B=2, H=14, W=14, C=32, s=1, gamma=0.25, dtype=0)
+    a.update(args)
+    st = lib.vrwkv_bishift(a["x"], a["out"], a["mu"], a["B"], a["H"], a["W"], a["C"], a["s"],
+                           a["gamma"], a["dtype"], None)
+    assert st in (1, 2)
+    assert frag in lib.vrwkv_last_error().decode()
+
+
+def test_qshift_params_mode_is_checked(lib):
+    import linear_complexity_vision_b200 as vk
+    qs = vk._QsParams(14, 14, 1, 0.25, None, None, None, 7)
+    st = lib.vrwkv_biwkv_fwd(FAKE, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24),
+                             FAKE + (4 << 24), 2, 196, 32, 0, ctypes.byref(qs), None)
+    assert st == 1 and b"mode" in lib.vrwkv_last_error()
+
+
+def test_workspace_variants_reject_bad_workspaces(lib):
+    B, T, C = 2, 1024, 32
+    need = lib.vrwkv_fwd_workspace_bytes(B, T, C)
+    assert need > 0
+    base = dict(k=FAKE, v=FAKE + (1 << 24), w=FAKE + (2 << 24), u=FAKE + (3 << 24), out=FAKE + (4 << 24))
+    ws_ok = FAKE + (8 << 24)
+
+    def call(ws, nbytes):
+        return lib.vrwkv_biwkv_fwd_ws(base["k"], base["v"], base["w"], base["u"], base["out"], B, T, C,
+                                      0, None, ws, nbytes, None)
+    assert call(None, need) == 1 and b"NULL" in lib.vrwkv_last_error()
+    assert call(ws_ok + 128, need) == 1 and b"256-byte" in lib.vrwkv_last_error()
+    assert call(ws_ok, need - 1) == 1 and b"smaller" in lib.vrwkv_last_error()
+    assert call(base["k"], need) == 1 and b"overlaps" in lib.vrwkv_last_error()
+    st = lib.vrwkv_spatial_gate_ws(FAKE, FAKE, FAKE, base["w"], base["u"], base["out"], B, T, C, 0,
+                                   None, None, need, None)
+    assert st == 1 and b"NULL" in lib.vrwkv_last_error()
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(B=0), "positive"),
+    (dict(x=None), "NULL"),
+    (dict(w_o=None), "NULL"),
+    (dict(ws=None), "NULL"),
+    (dict(dtype=3), "dtype"),
+    (dict(eps=-1.0), "ln_eps"),
+    (dict(x=FAKE + 8), "16-byte"),
+    (dict(ws=FAKE + (9 << 24) + 64), "256-byte"),
+    (dict(ws_bytes=16), "smaller"),
+    (dict(out=FAKE), "overlaps"),
+])
+def test_block_rejects_invalid_arguments(lib, args, frag):
+    B, T, C = 2, 196, 64
+    a = dict(x=FAKE, w_r=FAKE + (1 << 24), w_k=FAKE + (2 << 24), w_v=FAKE + (3 << 24),
+             w_o=FAKE + (4 << 24), w=FAKE + (5 << 24), u=FAKE + (5 << 24) + 4096,
+             g=FAKE + (5 << 24) + 8192, be=FAKE + (5 << 24) + 12288, eps=1e-5, out=FAKE + (6 << 24),
+             B=B, T=T, C=C, dtype=1, ws=FAKE + (9 << 24), ws_bytes=None)
+    a.update(args)
+    need = lib.vrwkv_block_workspace_bytes(B, T, C, 1)
+    assert need > 0
+    nb = need if a["ws_bytes"] is None else a["ws_bytes"]
+    st = lib.vrwkv_spatial_mix_block(a["x"], a["w_r"], a["w_k"], a["w_v"], a["w_o"], a["w"], a["u"],
+                                     a["g"], a["be"], a["eps"], a["out"], a["B"], a["T"], a["C"],
+                                     a["dtype"], _qs(14, 14), a["ws"], nb, None)
+    assert st in (1, 2)
+    assert frag in lib.vrwkv_last_error().decode()
