@@ -22,8 +22,8 @@
 // an associative composition, so both scans run as in the forward kernel:
 // walks over a thread's 8 tokens, shuffle scans over the 8 chunks of a warp,
 // a CTA scan over its 8 warps and an exchange across the CTAs of a cluster.
-// Round 1 scans (p v, p) with their H parts and yields y, q, r and the dw, du
-// terms; round 2 scans (q, r) and yields dk and dv.
+// Pass 1 scans (p v, p) with their H parts and yields y, q, r and the dw, du
+// terms; pass 2 scans (q, r) and yields dk and dv.
 //
 // Work decomposition.  A CTA owns batch row b, a slab of 8 channels and 512
 // tokens; T > 512 splits over a cluster of up to 8 CTAs (T <= 4096), which
@@ -31,7 +31,7 @@
 // 16-CTA clusters.  Thread = 2 adjacent channels (packed float2) x 8
 // consecutive tokens; the 32 lanes of a warp are 4 channel pairs x 8
 // consecutive chunks; 256 threads, two CTAs per SM within 128 registers: the
-// per-token forward states (round 1) and prefix sums (round 2) wait in shared
+// per-token forward states (pass 1) and prefix sums (pass 2) wait in shared
 // memory between the two walks, and p v is recomputed from p and v instead of
 // being kept.  Inputs of 16-byte-aligned tensors with C % 8 == 0 arrive by
 // TMA in the forward kernel's tile layout (element stride 8 along T: sub-tile
@@ -40,7 +40,7 @@
 // afterwards; other tensors load straight from global memory.
 // The CTAs of a column exchange their records with asynchronous stores into
 // each other's shared memory that complete on the receiver's mailbox
-// mbarrier (one per exchange round), so no cluster-wide barrier is waited on.
+// mbarrier (one per exchange pass), so no cluster-wide barrier is waited on.
 // Exponents are base 2 (log2 e is folded into k, u and w).
 #pragma once
 
@@ -85,12 +85,12 @@ struct alignas(64) Params {
     float invT;
 };
 
-// Round-1 record of one channel pair: sums of p v and p with their
+// Pass-1 record of one channel pair: sums of p v and p with their
 // distance-weighted parts.
 struct alignas(16) R1 {
     float2 apv, ap, hpv, hp;
 };
-// Round-2 record: sums of q and r.
+// Pass-2 record: sums of q and r.
 struct alignas(16) R2 {
     float2 aq, ar;
 };
@@ -171,11 +171,11 @@ struct alignas(16) Scratch {
     R1 k1F[kNP], k1B[kNP];
     R2 k2F[kNP], k2B[kNP];
     float2 kMc[kNP];
-    unsigned long long xbar[2];  // mailbox barriers of the two exchange rounds
+    unsigned long long xbar[2];  // mailbox barriers of the two exchange passes
 };
 
-// Bytes one peer stores into a mailbox per channel pair: round 1 two R1 and
-// the maximum; round 2 two R2, dw and du.
+// Bytes one peer stores into a mailbox per channel pair: pass 1 two R1 and
+// the maximum; pass 2 two R2, dw and du.
 constexpr unsigned kRec1Bytes = 2 * sizeof(R1) + sizeof(float2);
 constexpr unsigned kRec2Bytes = 2 * sizeof(R2) + 2 * sizeof(float2);
 
@@ -192,10 +192,10 @@ __device__ __forceinline__ unsigned peer_addr(const void* local, int peer) {
     return fast::mapa_u32(fast::smem_u32(local), (unsigned)peer);
 }
 
-// Per-token state between the two walks of a round, as two 16-byte planes
+// Per-token state between the two walks of a pass, as two 16-byte planes
 // [token][thread] (a thread's accesses are 16 bytes at a 16-byte stride:
-// bank-conflict free): round 1 keeps (apv, ap) in plane 0 and (hpv, hp) in
-// plane 1; round 2 keeps (aq, ar) in plane 0.
+// bank-conflict free): pass 1 keeps (apv, ap) in plane 0 and (hpv, hp) in
+// plane 1; pass 2 keeps (aq, ar) in plane 0.
 constexpr size_t kStashBytes = 2 * sizeof(float4) * kL * kThreads;
 // the stash starts 128-byte aligned (it also receives the TMA tiles)
 constexpr size_t kStashOff = (sizeof(Scratch) + 127) / 128 * 128;
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
     // a column chunk may hold no token of a padded channel: keep M finite
     Mcta = make_float2(Mcta.x == -INFINITY ? 0.f : Mcta.x, Mcta.y == -INFINITY ? 0.f : Mcta.y);
 
-    // ---- round 1: p, thread-local sums (p v recomputed where needed) ----------
+    // ---- pass 1: p, thread-local sums (p v recomputed where needed) ----------
     float2 pp[kL];
 #pragma unroll
     for (int i = 0; i < kL; ++i) pp[i] = ex2(add2(kk[i], make_float2(-Mcta.x, -Mcta.y)));
@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
     }
     __syncthreads();
 
-    // ---- round 1: carries into the thread's chunk, then y, q, r ----------------
+    // ---- pass 1: carries into the thread's chunk, then y, q, r ----------------
     const float2 Mc = S.kMc[j];
     const float2 sl = ex2(add2(Mcta, make_float2(-Mc.x, -Mc.y)));  // CTA frame -> common frame
     R1 KF, KB;
@@ -509,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         KB.ap = fma2(alpha, KB.ap, pp[i]);
     }
 
-    // ---- round 2: sums of q and r ---------------------------------------------
+    // ---- pass 2: sums of q and r ---------------------------------------------
     R2 mf = r2_zero(), mb = r2_zero();
 #pragma unroll
     for (int i = 0; i < kL; ++i) {
@@ -623,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
     }
     __syncthreads();
 
-    // ---- round 2: carries, then dv and dk ------------------------------------------
+    // ---- pass 2: carries, then dv and dk ------------------------------------------
     R2 QF, QB;
     {
         const float2 aW = decay(lam2, (float)(kWarpTok * warp)), aLn = decay(lam2, (float)(kL * cq));
@@ -639,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_bwd_kernel(const __grid_con
         QF.ar = fma2(alpha, QF.ar, rr[i]);
     }
     // with TMA stores the results gather in two tiles in the stash's second
-    // plane (free since round 1), at the input tiles' offsets
+    // plane (free since pass 1), at the input tiles' offsets
     char* otile = reinterpret_cast<char*>(plane1);
     const int orow = q * RB + j * 2 * es;  // token i of chunk q: + i * SUB
 #pragma unroll
