@@ -152,13 +152,50 @@ def _require(t, name: str) -> None:
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
+def _require_tokens(*named) -> None:
+    """(name, tensor) pairs of token tensors: contiguous CUDA (B, T, C)
+    tensors of one shape, dtype and device (the C ABI cannot see sizes, so a
+    mismatched output would be written past its end)."""
+    ref_name, ref = named[0]
+    for name, t in named:
+        _require(t, name)
+        if t.dim() != 3:
+            raise ValueError(f"{name} must be a (B, T, C) tensor")
+        if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError(f"{name} must match {ref_name} in shape, dtype and device")
+
+
+def _require_vec(t, C: int, device, name: str) -> None:
+    """A per-channel parameter: a contiguous float32 CUDA tensor of C
+    elements on `device` (read as float32[C] by the kernels)."""
+    import torch
+    _require(t, name)
+    if t.dtype != torch.float32 or t.numel() != C or t.device != device:
+        raise ValueError(f"{name} must be a float32 tensor of {C} elements on {device}")
+
+
+def _qs_ptr(qs, C: int, device):
+    """ctypes pointer to the Q-Shift parameters (None without Q-Shift), after
+    checking the mu vectors."""
+    if qs is None:
+        return None
+    for name in ("mu_r", "mu_k", "mu_v"):
+        t = getattr(qs, name)
+        if t is not None:
+            _require_vec(t, C, device, f"qs.{name}")
+    return ctypes.byref(qs._struct())
+
+
 def qshift(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25, mu=None, out=None):
     """Q-Shift of x (B, H*W, C): the shifted tensor, or mu*x + (1-mu)*shifted."""
     import torch
-    _require(x, "x")
+    _require_tokens(("x", x))
     B, T, C = x.shape
+    if mu is not None:
+        _require_vec(mu, C, x.device, "mu")
     if out is None:
         out = torch.empty_like(x)
+    _require_tokens(("x", x), ("out", out))
     _check(load_library().vrwkv_qshift(
         x.data_ptr(), out.data_ptr(), None if mu is None else mu.data_ptr(), B, H, W, C,
         shift_pixel, float(gamma), _dtype_code(x), _stream_ptr(x)))
@@ -169,10 +206,13 @@ def bishift(x, H: int, W: int, shift_pixel: int = 1, gamma: float = 0.25, mu=Non
     """The bidirectional shift of sparse (MAE) inputs (QShift mode 1) of x
     (B, H*W, C): the shifted tensor, or mu*x + (1-mu)*shifted."""
     import torch
-    _require(x, "x")
+    _require_tokens(("x", x))
     B, T, C = x.shape
+    if mu is not None:
+        _require_vec(mu, C, x.device, "mu")
     if out is None:
         out = torch.empty_like(x)
+    _require_tokens(("x", x), ("out", out))
     _check(load_library().vrwkv_bishift(
         x.data_ptr(), out.data_ptr(), None if mu is None else mu.data_ptr(), B, H, W, C,
         shift_pixel, float(gamma), _dtype_code(x), _stream_ptr(x)))
@@ -196,12 +236,14 @@ def biwkv_fwd(k, v, w, u, qs: Optional[QShift] = None, out=None, workspace=None)
     With a workspace (see fwd_workspace) the CTAs of long sequences exchange
     their sums through it instead of a thread-block cluster."""
     import torch
-    for t, name in ((k, "k"), (v, "v"), (w, "w"), (u, "u")):
-        _require(t, name)
+    _require_tokens(("k", k), ("v", v))
     B, T, C = k.shape
+    for t, name in ((w, "w"), (u, "u")):
+        _require_vec(t, C, k.device, name)
     if out is None:
         out = torch.empty_like(k)
-    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _require_tokens(("k", k), ("out", out))
+    qsp = _qs_ptr(qs, C, k.device)
     lib = load_library()
     if workspace is None:
         _check(lib.vrwkv_biwkv_fwd(
@@ -220,12 +262,14 @@ def spatial_gate(r, k, v, w, u, qs: Optional[QShift] = None, out=None, workspace
     """sigma(QS_R(r)) * Bi-WKV(QS_K(k), QS_V(v)); r, k, v may be one tensor.
     workspace: as for biwkv_fwd."""
     import torch
-    for t, name in ((r, "r"), (k, "k"), (v, "v"), (w, "w"), (u, "u")):
-        _require(t, name)
+    _require_tokens(("k", k), ("r", r), ("v", v))
     B, T, C = k.shape
+    for t, name in ((w, "w"), (u, "u")):
+        _require_vec(t, C, k.device, name)
     if out is None:
         out = torch.empty_like(k)
-    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _require_tokens(("k", k), ("out", out))
+    qsp = _qs_ptr(qs, C, k.device)
     lib = load_library()
     if workspace is None:
         _check(lib.vrwkv_spatial_gate(
@@ -244,11 +288,12 @@ def channel_mix(x, qs: Optional[QShift] = None, out=None):
     """sigma(QS_R(x)) * max(QS_K(x), 0)^2 on a (B, T, C) tensor (eq. 3-4 with
     identity projections); QS is the identity if qs is None."""
     import torch
-    _require(x, "x")
+    _require_tokens(("x", x))
     B, T, C = x.shape
     if out is None:
         out = torch.empty_like(x)
-    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _require_tokens(("x", x), ("out", out))
+    qsp = _qs_ptr(qs, C, x.device)
     _check(load_library().vrwkv_channel_mix(
         x.data_ptr(), out.data_ptr(), B, T, C, _dtype_code(x), qsp, _stream_ptr(x)))
     return out
@@ -260,12 +305,14 @@ def spatial_gate_static(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
     time (up to ~1600 (batch row, 8-channel) columns).  Calls overlapping in
     time on other streams share that workspace and race."""
     import torch
-    for t, name in ((r, "r"), (k, "k"), (v, "v"), (w, "w"), (u, "u")):
-        _require(t, name)
+    _require_tokens(("k", k), ("r", r), ("v", v))
     B, T, C = k.shape
+    for t, name in ((w, "w"), (u, "u")):
+        _require_vec(t, C, k.device, name)
     if out is None:
         out = torch.empty_like(k)
-    qsp = ctypes.byref(qs._struct()) if qs is not None else None
+    _require_tokens(("k", k), ("out", out))
+    qsp = _qs_ptr(qs, C, k.device)
     _check(load_library().vrwkv_spatial_gate_static(
         r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
         B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
@@ -286,14 +333,25 @@ def spatial_mix_block(x, weights, w, u, ln_gamma, ln_beta, qs: QShift, ln_eps: f
     (eq. 1-2).  weights = (W_R, W_K, W_V, W_O), each (C, C) in x's dtype,
     row-major (C_in, C_out).  workspace: see block_workspace."""
     import torch
-    _require(x, "x")
+    _require_tokens(("x", x))
+    B, T, C = x.shape
+    if len(weights) != 4:
+        raise ValueError("weights must be (W_R, W_K, W_V, W_O)")
     for i, t in enumerate(weights):
         _require(t, f"weights[{i}]")
+        if tuple(t.shape) != (C, C) or t.dtype != x.dtype or t.device != x.device:
+            raise ValueError(f"weights[{i}] must be a ({C}, {C}) tensor in x's dtype on x's device")
     for t, name in ((w, "w"), (u, "u"), (ln_gamma, "ln_gamma"), (ln_beta, "ln_beta")):
-        _require(t, name)
-    B, T, C = x.shape
+        _require_vec(t, C, x.device, name)
+    if qs is None:
+        raise ValueError("spatial_mix_block needs the Q-Shift parameters")
+    for name in ("mu_r", "mu_k", "mu_v"):
+        t = getattr(qs, name)
+        if t is not None:
+            _require_vec(t, C, x.device, f"qs.{name}")
     if out is None:
         out = torch.empty_like(x)
+    _require_tokens(("x", x), ("out", out))
     if workspace is None:
         workspace = block_workspace(B, T, C, x.dtype, device=x.device)
     wr, wk, wv, wo = weights
@@ -310,9 +368,10 @@ def biwkv_bwd(k, v, w, u, gy, totals: bool = True):
     the input dtype, gw, gu float32 (B, C) per batch row and, if totals, their
     sums over the batch (float32 (C,)); otherwise those two are None."""
     import torch
-    for t, name in ((k, "k"), (v, "v"), (w, "w"), (u, "u"), (gy, "gy")):
-        _require(t, name)
+    _require_tokens(("k", k), ("v", v), ("gy", gy))
     B, T, C = k.shape
+    for t, name in ((w, "w"), (u, "u")):
+        _require_vec(t, C, k.device, name)
     gk, gv = torch.empty_like(k), torch.empty_like(k)
     gw = torch.empty((B, C), dtype=torch.float32, device=k.device)
     gu = torch.empty((B, C), dtype=torch.float32, device=k.device)
