@@ -3,24 +3,27 @@ of "Vision-RWKV Backbone" (Linear Complexity Bidirectional Attention),
 checked against the oracle's direct summation of eq. 5.
 
 The model follows the kernel's structure, not its code: a column of T tokens
-splits into CTAs of 512 tokens, a CTA into 4 warps, a warp into 8 chunks of
-16 tokens, a chunk into two 8-token sub-chunks.
+splits into CTAs of 512 tokens, a CTA into warps of 8 chunks of KL tokens,
+a chunk into KL/8 sub-chunks of 8 tokens.  The kernel runs KL = 16 (4 warps)
+and KL = 8 (8 warps); KL = 32 is a candidate for fewer instructions per
+element.
 - Each sub-chunk sums relative to its own maximum of k.
 - Going up, the chunk fold, the warp scan, the CTA scan and the cross-CTA
   exchange rescale by 2^(M_lower - M_upper) <= 1 and decay by a^distance.
 - At the output, each token combines its sub-chunk's local sums with the
   carries from the left and the right.
 
-What this pins (independently of CUDA): the fold F = a^8 e0 F0 + e1 F1,
-G = e0 G0 + a^8 e1 G1, the carries each sub-chunk takes from the other, the
-distances behind every decay power, and the choice of references that keeps
-every scale factor <= 1 (k shifted by +80 and spreads of k across CTAs).
+What this pins (independently of CUDA): the fold
+F = sum_h a^{8(KH-1-h)} e_h F_h and G = sum_h a^{8h} e_h G_h (KL = 16:
+F = a^8 e0 F0 + e1 F1, G = e0 G0 + a^8 e1 G1), the carries each sub-chunk
+takes from the others, the distances behind every decay power, and the
+choice of references that keeps every scale factor <= 1 (k shifted by +80
+and spreads of k across CTAs).
 """
 import numpy as np
 import pytest
 
-SUB, KL, CPW, NW = 8, 16, 8, 4          # sub-chunk, chunk, chunks per warp, warps per CTA
-TC = KL * CPW * NW                       # tokens per CTA (512)
+SUB, CPW, TC = 8, 8, 512   # sub-chunk (the TMA element stride), chunks per warp, tokens per CTA
 
 
 def _exp(x):
@@ -28,16 +31,19 @@ def _exp(x):
         return np.exp(x)
 
 
-def model_column(k, v, w, u):
-    """wkv of one (b, c) column by the kernel's decomposition.  Carries that
-    cross the padding past T may overflow (as in the kernel, they only reach
-    tokens past T, which are dropped); the tests compare the real tokens."""
+def model_column(k, v, w, u, KL=16):
+    """wkv of one (b, c) column by the kernel's decomposition with chunks of
+    KL tokens (8 and 16 are the kernel's two shapes; 32 a candidate).  Carries
+    that cross the padding past T may overflow (as in the kernel, they only
+    reach tokens past T, which are dropped); the tests compare real tokens."""
     with np.errstate(over="ignore", invalid="ignore"):
-        return _model_column(k, v, w, u)
+        return _model_column(k, v, w, u, KL)
 
 
-def _model_column(k, v, w, u):
+def _model_column(k, v, w, u, KL):
     T = k.shape[0]
+    KH = KL // SUB                   # sub-chunks per chunk
+    NW = TC // (KL * CPW)            # warps per CTA
     lam = w / T
     cap = 126.0 * np.log(2.0)  # the kernel caps decay exponents at 2^126
 
@@ -68,19 +74,19 @@ def _model_column(k, v, w, u):
     F = np.stack([pv @ ap(SUB - 1 - i), p @ ap(SUB - 1 - i)], -1)   # to the sub-chunk's end
     G = np.stack([pv @ ap(i), p @ ap(i)], -1)                       # from its start
 
-    # chunks (two sub-chunks) and the warp maximum
-    nch = nsub // 2
-    Mh2 = Mh.reshape(nch, 2)
-    Mw = Mh2.reshape(-1, CPW, 2).max(axis=(1, 2))        # per warp
+    # chunks of KH sub-chunks and the warp maximum
+    nch = nsub // KH
+    MhK = Mh.reshape(nch, KH)
+    Mw = MhK.reshape(-1, CPW, KH).max(axis=(1, 2))       # per warp
     mref = np.where(np.isfinite(Mw), Mw, 0.0)
-    e = _exp(Mh2 - np.repeat(mref, CPW)[:, None])        # 2^(M_h - M_warp), 0 if empty
-    F2, G2 = F.reshape(nch, 2, 2), G.reshape(nch, 2, 2)
-    a8 = ap(SUB)
-    F0s, G1s = e[:, 0, None] * F2[:, 0], e[:, 1, None] * G2[:, 1]
-    Fc = a8 * F0s + e[:, 1, None] * F2[:, 1]
-    Gc = e[:, 0, None] * G2[:, 0] + a8 * G1s
+    e = _exp(MhK - np.repeat(mref, CPW)[:, None])        # 2^(M_h - M_warp), 0 if empty
+    Fs = e[..., None] * F.reshape(nch, KH, 2)            # sub-chunk totals, warp reference
+    Gs = e[..., None] * G.reshape(nch, KH, 2)
+    h_ = np.arange(KH)
+    Fc = np.einsum("h,chx->cx", ap(SUB * (KH - 1 - h_)), Fs)   # the chunk fold
+    Gc = np.einsum("h,chx->cx", ap(SUB * h_), Gs)
 
-    # warp scans over 8 chunks (decay a^16 per chunk)
+    # warp scans over 8 chunks (decay a^KL per chunk)
     nw = nch // CPW
     Fw, Gw = Fc.reshape(nw, CPW, 2), Gc.reshape(nw, CPW, 2)
     X, Y = np.zeros_like(Fw), np.zeros_like(Gw)
@@ -97,10 +103,10 @@ def _model_column(k, v, w, u):
             acc = ap(KL) * acc + Gw[wi, q]
             GI[wi, q] = acc
 
-    # CTA scans over 4 warps (decay a^128 per warp), rescaled to the CTA maximum
-    Mw4 = Mw.reshape(ncl, NW)
-    Mcta = Mw4.max(axis=1)
-    ws = _exp(Mw4 - Mcta[:, None])
+    # CTA scans over the warps (decay a^(KL CPW) per warp), rescaled to the CTA maximum
+    MwN = Mw.reshape(ncl, NW)
+    Mcta = MwN.max(axis=1)
+    ws = _exp(MwN - Mcta[:, None])
     fagg = ws[..., None] * FI.reshape(ncl, NW, CPW, 2)[:, :, -1]
     gagg = ws[..., None] * GI.reshape(ncl, NW, CPW, 2)[:, :, 0]
     XW, YW = np.zeros_like(fagg), np.zeros_like(gagg)
@@ -130,7 +136,7 @@ def _model_column(k, v, w, u):
         Bb[r] = acc
         acc = ap(TC) * acc + sc[r] * own_G[r]
 
-    # outputs
+    # outputs: each sub-chunk's carries take the totals of the other sub-chunks
     out = np.empty(Tp)
     pw = ap(i)
     for r in range(ncl):
@@ -144,28 +150,30 @@ def _model_column(k, v, w, u):
                 kf, kb = ap(KL * qc), ap(KL * (TC // KL - 1 - qc))
                 As = slw * X[W_, cq] + slF * XW[r, wi] + kf * Af[r]
                 Be = slw * Y[W_, cq] + slB * YW[r, wi] + kb * Bb[r]
-                for h in range(2):
-                    Ah, Bh = As, Be
-                    if h == 0:
-                        Bh = slw * G1s[ch] + a8 * Be
-                    else:
-                        Ah = slw * F0s[ch] + a8 * As
+                for h in range(KH):
+                    Ah = ap(SUB * h) * As
+                    for hh in range(h):
+                        Ah = Ah + slw * ap(SUB * (h - 1 - hh)) * Fs[ch, hh]
+                    Bh = ap(SUB * (KH - 1 - h)) * Be
+                    for hh in range(h + 1, KH):
+                        Bh = Bh + slw * ap(SUB * (hh - h - 1)) * Gs[ch, hh]
                     sh = slw * e[ch, h]
-                    s = 2 * ch + h
+                    s = KH * ch + h
                     num = sh * n[s] + pw * Ah[0] + pw[::-1] * Bh[0]
                     den = sh * dd[s] + pw * Ah[1] + pw[::-1] * Bh[1]
                     out[s * SUB:(s + 1) * SUB] = num / den
     return out[:T]
 
 
+@pytest.mark.parametrize("KL", [8, 16, 32])
 @pytest.mark.parametrize("T", [1, 7, 33, 512, 513, 1000, 2048, 4096])
 @pytest.mark.parametrize("w", [-8.0, -0.5, 0.0, 3.0, 8.0])
-def test_model_equals_eq5(oracle_mod, T, w):
+def test_model_equals_eq5(oracle_mod, T, w, KL):
     rng = np.random.default_rng(T * 31 + int(w * 10) + 1000)
     k = rng.normal(0.0, 2.0, T)
     v = rng.normal(0.0, 1.0, T)
     u = 0.7
-    got = model_column(k, v, w, u)
+    got = model_column(k, v, w, u, KL)
     want = oracle_mod.biwkv_direct(k[None, :, None], v[None, :, None], np.array([w]),
                                    np.array([u]))[0, :, 0]
     scale = np.abs(v).max()
