@@ -29,7 +29,11 @@
  *     X and X^dagger; the interpolation mu*X + (1-mu)*X^dagger is computed.
  *   - channel-group order follows the listing (w-s, w+s, h-s, h+s); eq. 9's
  *     order (h-1, h+1, w-1, w+1) is available through eq9_order=1.
- *   - g = int(C*gamma) truncates as Python int() does.
+ *   - the channel groups end where the listing's slices end: at
+ *     b_j = int(C*gamma*j), j = 1..4, with C*gamma formed first, then times
+ *     j, in double precision (Python's left-to-right order), and truncated
+ *     as Python int() does; channels >= b_4 are copied.  Eq. 9's C/4, C/2,
+ *     3C/4, C are the same bounds at gamma = 1/4.
  *   - a shift_pixel at or beyond the grid extent empties that group (zeros).
  *   - the garbled "ki" in eq. 5 is k_i; T is the total token count.
  *
@@ -48,18 +52,29 @@
 /* Q-Shift: the gather X^dagger (eq. 9 and the q_shift listing)        */
 /* ------------------------------------------------------------------ */
 
+/* End of channel group j-1 (j = 1..4): the listing's slice bound
+ * int(C*gamma*j).  Python evaluates C*gamma first and then multiplies by j,
+ * both in double precision, and int() truncates toward zero. */
+static int qshift_bound(int C, double gamma, int j) {
+    double cg = (double)C * gamma;
+    return (int)(cg * (double)j);
+}
+
+/* Channel group of channel c: 0..3 for the four slices
+ * [b_{j}, b_{j+1}) (b_0 = 0), 4 for the copied channels c >= b_4
+ * (output[:, int(C*gamma*4):] = input[:, int(C*gamma*4):]). */
+static int qshift_group(int c, int C, double gamma) {
+    for (int j = 1; j <= 4; ++j)
+        if (c < qshift_bound(C, gamma, j)) return j - 1;
+    return 4;
+}
+
 /* Source pixel of output pixel (h,w) for channel c, following the listing's
  * slice assignments.  Returns 0 when the output stays at its zero initial
  * value (border, or an emptied group), 1 with (*sh,*sw) set otherwise. */
 static int qshift_source(int c, int h, int w, int H, int W, int C, int s,
                          double gamma, int eq9_order, int* sh, int* sw) {
-    int g = (int)((double)C * gamma); /* Python int(): truncation toward 0 */
-    int grp;
-    if (c < g) grp = 0;
-    else if (c < 2 * g) grp = 1;
-    else if (c < 3 * g) grp = 2;
-    else if (c < 4 * g) grp = 3;
-    else grp = 4; /* output[:, 4g:] = input[:, 4g:] */
+    int grp = qshift_group(c, C, gamma);
     if (eq9_order && grp < 4) {
         /* eq. 9 order: h-1, h+1, w-1, w+1  ->  listing groups 2,3,0,1 */
         static const int perm[4] = {2, 3, 0, 1};
@@ -550,16 +565,17 @@ void oracle_biwkv_bwd_columns(const double* k, const double* v,
 /* ------------------------------------------------------------------ */
 /* The pages pre-train with MAE after changing Q-Shift into a bidirectional
  * shift, and say no more.  Reading taken: of Q-Shift's four channel groups
- * only the two that shift along the token row remain -- [0, g) from token
- * w-s, [g, 2g) from token w+s, zero past the row's ends -- and every other
- * channel, the two vertical groups included, passes through unchanged.  A
- * sparse input is one row of its visible tokens (H = 1, W = their count). */
+ * only the two that shift along the token row remain -- [0, b_1) from token
+ * w-s, [b_1, b_2) from token w+s (b_j the listing's int(C*gamma*j)), zero
+ * past the row's ends -- and every other channel, the two vertical groups
+ * included, passes through unchanged.  A sparse input is one row of its
+ * visible tokens (H = 1, W = their count). */
 static int bishift_source(int c, int h, int w, int W, int C, int s,
                           double gamma, int* sh, int* sw) {
-    int g = (int)((double)C * gamma);
+    int grp = qshift_group(c, C, gamma);
     int srcw = w;
-    if (c < g) srcw = w - s;
-    else if (c < 2 * g) srcw = w + s;
+    if (grp == 0) srcw = w - s;
+    else if (grp == 1) srcw = w + s;
     if (srcw < 0 || srcw >= W) return 0;
     *sh = h;
     *sw = srcw;

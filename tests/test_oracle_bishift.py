@@ -45,3 +45,17 @@ def test_mu_interpolation_and_f32_order(oracle_mod):
     np.testing.assert_allclose(f32, mu * x + (1 - mu) * xs, rtol=1e-6, atol=1e-6)
     # the rows of a 2 x 6 grid shift independently
     np.testing.assert_array_equal(xs[0, 6, :4], np.zeros(4))  # row 1, w = 0: [0, g) from w-1
+
+
+def test_hand_worked_row_listing_bounds(oracle_mod):
+    # C = 6, gamma = 1/4: the listing's first two bounds are int(1.5) = 1 and
+    # int(3.0) = 3, so channel 0 comes from t-1, channels 1-2 from t+1, and
+    # channels 3-5 pass through.  Token t, channel c = 10 t + c.
+    x = np.array([[[10 * t + c for c in range(6)] for t in range(3)]], dtype=np.float64)
+    out = oracle_mod.bishift(x, 1, 3, 1, 0.25)[0]
+    want = np.array([
+        [0, 11, 12, 3, 4, 5],
+        [0, 21, 22, 13, 14, 15],
+        [10, 0, 0, 23, 24, 25],
+    ], dtype=np.float64)
+    np.testing.assert_array_equal(out, want)

@@ -10,12 +10,13 @@ import numpy as np
 
 def test_hand_worked_single_token_grid(oracle_mod):
     # a 1x1 grid: every shifted group reads outside the grid (zero), so with
-    # mu the mixes are mu * x; channels >= 4g (here g = 1, C = 6 -> 4, 5)
+    # mu the mixes are mu * x.  gamma = 0.2, C = 6: the listing's bounds are
+    # int(1.2) = 1, int(2.4) = 2, int(3.6) = 3, int(4.8) = 4, so channels 4, 5
     # copy x.  x = [2, -1, 3, 0.5, -2, 1.5]
     x = np.array([[[2.0, -1.0, 3.0, 0.5, -2.0, 1.5]]])
     mu_r = np.array([0.5, 0.5, 0.0, 1.0, 0.3, 0.9])
     mu_k = np.array([1.0, 1.0, 0.5, 0.25, 0.7, 0.1])
-    out = oracle_mod.channel_mix(x, 1, 1, 1, 0.25, mu_r, mu_k)[0, 0]
+    out = oracle_mod.channel_mix(x, 1, 1, 1, 0.2, mu_r, mu_k)[0, 0]
     sig = lambda z: 1.0 / (1.0 + np.exp(-z))
     want = [
         sig(1.0) * 2.0 ** 2,      # r = 0.5*2,   k = 1.0*2
@@ -26,6 +27,11 @@ def test_hand_worked_single_token_grid(oracle_mod):
         sig(1.5) * 1.5 ** 2,      # copied channel: r = k = 1.5
     ]
     np.testing.assert_allclose(out, want, rtol=1e-14)
+    # at gamma = 1/4 the bounds are 1, 3, 4, 6: channels 4, 5 move (from h+1,
+    # outside the grid), so r = mu_r x and k = mu_k x there as well
+    out = oracle_mod.channel_mix(x, 1, 1, 1, 0.25, mu_r, mu_k)[0, 0]
+    np.testing.assert_allclose(out[:4], want[:4], rtol=1e-14)
+    np.testing.assert_allclose(out[4:], [0.0, sig(0.9 * 1.5) * (0.1 * 1.5) ** 2], rtol=1e-14)
 
 
 def test_negative_inputs_give_zero(oracle_mod):
