@@ -74,19 +74,23 @@ typedef enum {
  *   H, W         patch grid; T must equal H*W.
  *   shift_pixel  shift distance in patches, >= 0.  A distance at or beyond
  *                the grid extent leaves that channel group all zero.
- *   gamma        channel-group fraction, 0 <= gamma <= 1/4; the group size is
- *                g = (int)(C*gamma) computed in double precision.  Channels
- *                [0,g) take x[h, w-s], [g,2g) x[h, w+s], [2g,3g) x[h-s, w],
- *                [3g,4g) x[h+s, w] (zero outside the grid); channels >= 4g
- *                take x[h, w] unchanged.
+ *   gamma        channel-group fraction, 0 <= gamma <= 1/4.  The groups end
+ *                at the listing's slice bounds b_j = int(C*gamma*j), j = 1..4,
+ *                evaluated as Python does (C*gamma in double, then times j,
+ *                then truncated).  Channels [0,b_1) take x[h, w-s], [b_1,b_2)
+ *                x[h, w+s], [b_2,b_3) x[h-s, w], [b_3,b_4) x[h+s, w] (zero
+ *                outside the grid); channels >= b_4 take x[h, w] unchanged
+ *                (none at gamma = 1/4, where the bounds are eq. 9's C/4, C/2,
+ *                3C/4, C).  Groups differ in size when C*gamma is not an
+ *                integer: C = 10, gamma = 1/4 gives [0,2) [2,5) [5,7) [7,10).
  *   mu_r, mu_k, mu_v  device float32[C] interpolation weights, each nullable.
  *                With mu the shifted input is mu*x + (1-mu)*x_shift; a NULL
  *                mu means the shifted tensor x_shift itself.
  *   mode         VRWKV_QSHIFT_QUAD, or VRWKV_QSHIFT_BIDIR for sparse inputs:
  *                the pages pre-train with MAE after turning Q-Shift into a
  *                bidirectional shift and say no more; this mode keeps the two
- *                row groups ([0,g) from x[h, w-s], [g,2g) from x[h, w+s], zero
- *                past the row) and passes every other channel through.  A
+ *                row groups ([0,b_1) from x[h, w-s], [b_1,b_2) from x[h, w+s],
+ *                zero past the row) and passes every other channel through.  A
  *                sparse input is one row of its visible tokens (H = 1).
  */
 typedef enum {
@@ -142,8 +146,8 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *   qs    NULL, or Q-Shift parameters applied to k (mu_k) and v (mu_v) on
  *         load (mu_r is ignored); T must then equal qs->H * qs->W.
  * Kernels: a TMA fast path serves C % 8 == 0 with 16-byte-aligned inputs
- *   (and, with qs, a channel-group size int(C*gamma) that is a multiple of
- *   8 and W <= 256); everything else runs a generic kernel with the same
+ *   (and, with qs, channel-group bounds int(C*gamma*j) that are all
+ *   multiples of 8, and W <= 256); everything else runs a generic kernel with the same
  *   results up to rounding.  Setting VRWKV_DISABLE_TMA=1 in the environment
  *   forces the generic kernel, VRWKV_TMA_CHUNK=8 holds the fast path to
  *   8-token thread chunks and VRWKV_NO_TMA_STORE=1 to per-thread stores of
@@ -325,8 +329,8 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w,
  *   (fused multiply-add) and sigma(r) = 1/(1 + 2^(-r*log2 e)) from the hardware
  *   exp2 and reciprocal; one rounding to bfloat16 at the store for VRWKV_BF16.
  * Kernels: a vector kernel serves C*sizeof(dtype) % 16 == 0 with 16-byte-
- *   aligned x and out, 8-byte-aligned mu and a group size int(C*gamma) that is
- *   a multiple of 16/sizeof(dtype); everything else runs a scalar kernel.
+ *   aligned x and out, 8-byte-aligned mu and group bounds int(C*gamma*j) that
+ *   are multiples of 16/sizeof(dtype); everything else runs a scalar kernel.
  * Errors: INVALID_ARG for B, T or C <= 0, NULL x/out, misaligned pointers, an
  *   overlapping output or bad qs fields; UNSUPPORTED for B*T >= 2^31.
  */
@@ -348,6 +352,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C,
  * vrwkv_last_error().
  */
 vrwkv_status vrwkv_device_status(void);
+
 
 /* Name of the main kernel the calling thread's most recent successful
  * vrwkv_biwkv_fwd / vrwkv_spatial_gate / vrwkv_channel_mix / vrwkv_biwkv_bwd

@@ -58,7 +58,8 @@ struct FusedParams {
     const float* mu_v;  // nullable
     char* out;
     int B, T, C;
-    int H, W, s, g;   // Q-Shift grid, shift and group size
+    int H, W, s;      // Q-Shift grid and shift
+    QsBounds g;       // Q-Shift channel-group bounds
     int ng;           // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
     int Tc;           // tokens per CTA (multiple of 32 when ncl > 1)
     int ncl;          // CTAs per (b, slab) column = cluster size

@@ -87,8 +87,8 @@ struct alignas(64) Params {
     char* out;
     unsigned int* err;   // device error word (bounded waits)
     int B, T, C;
-    int H, W, s, g;      // Q-Shift grid, shift, group size
-    int gslab;           // group size in 16-channel slabs (g / 16; 0 if g == 0)
+    int H, W, s;         // Q-Shift grid, shift
+    QsBounds g;          // Q-Shift channel-group bounds (multiples of kCS on this path)
     int ng;              // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
     float invT;          // 1 / T
     int Tc;              // tokens per CTA (multiple of kWarpTok when ncl > 1)
@@ -380,9 +380,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     const int tend = min(p.T, t0 + p.Tc);
 
     // group of this CTA's channels (Q-Shift): 0..3 shifted, 4 copied
-    int grp = 4;
-    if (QS && p.gslab > 0)
-        grp = (slab >= p.gslab) + (slab >= 2 * p.gslab) + (slab >= 3 * p.gslab) + (slab >= 4 * p.gslab);
+    int grp = QS ? qs_group(c0, p.g) : 4;
     if (grp >= p.ng) grp = 4;
     const bool shifted = QS && grp < 4;
 

@@ -51,7 +51,8 @@ struct ChannelMixParams {
     const float* mu_r;  // nullable: QS_R(x) = x_shift
     const float* mu_k;  // nullable: QS_K(x) = x_shift
     int BT;             // B*T token rows, < 2^31
-    int T, C, H, W, s, g;
+    int T, C, H, W, s;
+    QsBounds g;         // Q-Shift channel-group bounds
     int ng;             // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
     int UR;             // 16-byte vectors per token row
     FastDiv divT, divW;

@@ -94,11 +94,22 @@ struct Io<__nv_bfloat16> {
 };
 
 // ---------------------------------------------------------------------------
-// Q-Shift source of one channel (eq. 9; q_shift listing).  The group of a
-// channel fixes a token offset and an admissible coordinate range: groups
-// 0/1 test the column w, groups 2/3 the row h, group 4 (channels >= 4g)
-// always reads the token itself.
+// Q-Shift source of one channel (eq. 9; q_shift listing).  The channel
+// groups end at the listing's slice bounds b[j-1] = int(C*gamma*j), j = 1..4
+// (C*gamma formed in double, times j, truncated; computed on the host):
+// group j covers [b[j-1], b[j]) with b[-1] = 0, and channels >= b[3] are
+// copied.  All-zero bounds make every channel a copy (no shift).  The group
+// fixes a token offset and an admissible coordinate range: groups 0/1 test
+// the column w, groups 2/3 the row h, group 4 always reads the token itself.
 // ---------------------------------------------------------------------------
+struct QsBounds {
+    int b[4];
+};
+
+__host__ __device__ __forceinline__ int qs_group(int c, const QsBounds& g) {
+    return (c >= g.b[0]) + (c >= g.b[1]) + (c >= g.b[2]) + (c >= g.b[3]);
+}
+
 struct ShiftRule {
     int off;      // token offset of the source
     int use_w;    // 1: test w, 0: test h
@@ -108,8 +119,8 @@ struct ShiftRule {
 // ng = number of shifted groups: 4 for Q-Shift (eq. 9), 2 for the
 // bidirectional shift of sparse (MAE) inputs, whose vertical groups pass
 // their channels through unchanged.
-__device__ __forceinline__ ShiftRule shift_rule(int c, int g, int ng, int H, int W, int s) {
-    int grp = (g > 0) ? min(c / g, 4) : 4;
+__device__ __forceinline__ ShiftRule shift_rule(int c, const QsBounds& g, int ng, int H, int W, int s) {
+    int grp = qs_group(c, g);
     if (grp >= ng) grp = 4;
     ShiftRule r;
     switch (grp) {

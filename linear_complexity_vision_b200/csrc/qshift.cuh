@@ -60,7 +60,8 @@ struct QshiftParams {
     char* out;
     const float* mu;  // nullable
     long long BT;     // B*T
-    int T, C, H, W, s, g;
+    int T, C, H, W, s;
+    QsBounds g;       // channel-group bounds
     int ng;           // shifted groups: 4 (Q-Shift) or 2 (bidirectional shift)
 };
 

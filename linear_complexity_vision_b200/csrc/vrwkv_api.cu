@@ -65,7 +65,24 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 int elem_bytes(vrwkv_dtype dt) { return dt == VRWKV_F32 ? 4 : 2; }
 
-int group_size(int C, double gamma) { return (int)((double)C * gamma); }
+// Q-Shift channel-group bounds of the q_shift listing: int(C*gamma*j),
+// j = 1..4, with C*gamma formed first and then multiplied by j, both in
+// double precision (the listing's Python evaluation order), truncated.
+QsBounds qs_bounds(int C, double gamma) {
+    QsBounds g;
+    const double cg = (double)C * gamma;
+    for (int j = 0; j < 4; ++j) g.b[j] = (int)(cg * (double)(j + 1));
+    return g;
+}
+QsBounds no_shift_bounds() { return QsBounds{{0, 0, 0, 0}}; }
+
+// Every bound a multiple of n: vectors (or slabs) of n channels never
+// straddle two groups.
+bool bounds_multiple_of(const QsBounds& g, int n) {
+    for (int j = 0; j < 4; ++j)
+        if (g.b[j] % n != 0) return false;
+    return true;
+}
 
 // Shifted channel groups of a Q-Shift mode: all four (eq. 9) or the two
 // row groups (bidirectional shift of sparse inputs).
@@ -170,8 +187,8 @@ unsigned int* device_error_word() {
 
 // Fixed device workspace of vrwkv_spatial_gate_static, for callers that
 // cannot allocate device memory: it is reserved when the module loads, so a
-// call allocates nothing.  4 MiB holds the exchange state of about 800
-// (batch row, 16-channel) columns.  One array per device, shared by every
+// call allocates nothing.  4 MiB holds the exchange state of about 1600
+// (batch row, 8-channel slab) columns (2624 bytes each).  One array per device, shared by every
 // caller of that entry point.
 constexpr size_t kStaticWsBytes = 4u << 20;
 static __device__ __align__(256) unsigned char g_vrwkv_static_ws[kStaticWsBytes];
@@ -303,8 +320,8 @@ bool launch_qs_mix(const void* x, void* const* outs, const float* const* mus, in
                    int shift, double gamma, int ng, vrwkv_dtype dtype, cudaStream_t s, vrwkv_status* st) {
     const int es = elem_bytes(dtype), nv = 16 / es;
     const long long BT = (long long)B * H * W;
-    const int g = group_size(C, gamma);
-    if (C % nv != 0 || g % nv != 0 || BT > 0x7fffffffLL || !aligned(x, 16)) return false;
+    const QsBounds g = qs_bounds(C, gamma);
+    if (C % nv != 0 || !bounds_multiple_of(g, nv) || BT > 0x7fffffffLL || !aligned(x, 16)) return false;
     for (int m = 0; m < NMIX; ++m)
         if (!aligned(outs[m], 16) || (mus[0] && !mus[m])) return false;
     QsMixParams<NMIX> q;
@@ -380,7 +397,7 @@ struct FastPlan {
 
 // Workspace of the global-exchange path: 16 bytes of counters, then a flag
 // per (column, rank), then a record per (column, rank); a column is one
-// (batch row, 16-channel slab).
+// (batch row, 8-channel slab).
 struct WsLayout {
     size_t flags_off, recs_off, bytes;
 };
@@ -538,9 +555,9 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         p.H = qs->H;
         p.W = qs->W;
         p.s = qs->shift_pixel;
-        p.g = group_size(C, qs->gamma);
+        p.g = qs_bounds(C, qs->gamma);
         p.ng = shifted_groups(qs);
-        if (p.g % fast::kCS != 0 || p.W > 256 || p.W % fast::kL != 0) return false;
+        if (!bounds_multiple_of(p.g, fast::kCS) || p.W > 256 || p.W % fast::kL != 0) return false;
         if (T <= TcMax) {
             p.rows = p.H;
             p.Tc = T;
@@ -568,7 +585,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         p.H = 1;
         p.W = T;
         p.s = 0;
-        p.g = 0;
+        p.g = no_shift_bounds();
         p.ng = 4;
         p.rows = 1;
         p.Tc = std::min(T, TcMax);
@@ -623,7 +640,6 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         p.tma_store = (cr == CUDA_SUCCESS && (p.Tc % 256 == 0 || p.ncl == 1) && !tma_store_disabled()) ? 1 : 0;
     }
-    p.gslab = pl.qs ? p.g / fast::kCS : 0;
     p.invT = (float)(1.0 / (double)T);
     p.err = device_error_word();
     if (!p.err) return false;
@@ -781,7 +797,7 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
     p.H = qs ? qs->H : 1;
     p.W = qs ? qs->W : T;
     p.s = qs ? qs->shift_pixel : 0;
-    p.g = qs ? group_size(C, qs->gamma) : 0;
+    p.g = qs ? qs_bounds(C, qs->gamma) : no_shift_bounds();
     p.ng = shifted_groups(qs);
     bool vin = ((size_t)C * es) % 16 == 0;
     for (int i = 0; i < pl.ntiles; ++i) vin = vin && aligned(p.src[i], 16);
@@ -828,7 +844,7 @@ vrwkv_status shift_entry(const void* x, void* out, const float* mu, int B, int H
     p.H = H;
     p.W = W;
     p.s = shift_pixel;
-    p.g = group_size(C, gamma);
+    p.g = qs_bounds(C, gamma);
     p.ng = ng;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     {
@@ -883,7 +899,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
     p.H = 1;
     p.W = T;
     p.s = 0;
-    p.g = 0;  // without qs every channel reads its own token: QS is the identity
+    p.g = no_shift_bounds();  // without qs every channel reads its own token: QS is the identity
     p.ng = 4;
     if (qs) {
         vrwkv_status st = check_qs(qs, T, C);
@@ -893,7 +909,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
         p.H = qs->H;
         p.W = qs->W;
         p.s = qs->shift_pixel;
-        p.g = group_size(C, qs->gamma);
+        p.g = qs_bounds(C, qs->gamma);
         p.ng = shifted_groups(qs);
         for (const float* m : {p.mu_r, p.mu_k})
             if (m && overlaps(out, nbytes, m, (size_t)C * 4))
@@ -903,7 +919,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
     p.divW = make_fastdiv((unsigned)p.W);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int nv = 16 / es;  // channels per 16-byte vector
-    const bool vec = (C % nv) == 0 && p.g % nv == 0 && aligned(x, 16) && aligned(out, 16) &&
+    const bool vec = (C % nv) == 0 && bounds_multiple_of(p.g, nv) && aligned(x, 16) && aligned(out, 16) &&
                      (!p.mu_r || aligned(p.mu_r, 8)) && (!p.mu_k || aligned(p.mu_k, 8));
     if (!vec) {
         const long long n = (long long)p.BT * C;
@@ -1058,7 +1074,7 @@ vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k, const void*
     const WsLayout L = ws_layout(B, C);
     if (L.bytes > kStaticWsBytes)
         return fail(VRWKV_ERR_UNSUPPORTED,
-                    "B*ceil(C/16) = %lld columns need %zu bytes of exchange state; the static workspace "
+                    "B*ceil(C/8) = %lld columns need %zu bytes of exchange state; the static workspace "
                     "holds %zu",
                     (long long)B * ((C + fast::kCS - 1) / fast::kCS), L.bytes, kStaticWsBytes);
     unsigned char* ws = static_workspace();

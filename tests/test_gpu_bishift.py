@@ -100,3 +100,20 @@ def test_mode_is_validated(vk):
     x = torch.zeros(1, 16, 16, device="cuda")
     with pytest.raises(vk.VrwkvError):
         vk.spatial_gate(x, x, x, x[0, 0], x[0, 0], qs=vk.QShift(4, 4, mode=7))
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("B,H,W,C,s,gamma", [
+    (2, 1, 11, 10, 1, 0.25),   # bounds 2, 5: channel groups [0,2) [2,5)
+    (1, 1, 20, 26, 2, 0.25),   # bounds 6, 13
+    (1, 2, 16, 64, 1, 0.125),  # bounds 8, 16 (vector kernel)
+])
+def test_bishift_listing_bounds(vk, oracle_mod, dt, B, H, W, C, s, gamma):
+    seed, x = _x(B, H, W, C, "bounds")
+    mu = synth.draw(seed, "mu_k", (C,), ("uniform", 0.0, 1.0))
+    xt, xd = to_device(x, dt)
+    mut, mud = vec_f32(mu)
+    got = vk.bishift(xt, H, W, s, gamma, mu=mut)
+    want = oracle_mod.bishift_f32(xd.astype(np.float32), H, W, s, gamma,
+                                  mu=mud.astype(np.float32), round_bf16=(dt == "bf16"))
+    np.testing.assert_array_equal(to_numpy(got), want.astype(np.float64))

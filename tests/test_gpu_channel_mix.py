@@ -105,6 +105,10 @@ CASES = [
     (1, 8, 8, 40, 1, 0.25),       # g = 10: vectors straddle groups (scalar kernel)
     (1, 4, 4, 4160, 1, 0.25),     # 520 bf16 / 1040 f32 vectors: split channel chunks
     (8, 64, 64, 1024, 1, 0.25),   # the 1024^2 grid at C = 1024 (full size)
+    # the listing's bounds int(C*gamma*j) where C*gamma is not an integer
+    (2, 5, 6, 10, 1, 0.25),       # bounds 2, 5, 7, 10 (scalar kernel)
+    (1, 8, 8, 64, 1, 0.125),      # bounds 8, 16, 24, 32: vector kernel, 32.. copied
+    (1, 6, 6, 50, 2, 0.145),      # double rounding: last bound 28
 ]
 
 

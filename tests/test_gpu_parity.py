@@ -44,6 +44,12 @@ QS_CASES = [
     (2, 6, 6, 32, 0, 0.25),      # shift 0
     (1, 6, 6, 32, 1, 0.0),       # gamma 0: every channel copied
     (2, 64, 64, 1024, 1, 0.25),  # the 1024^2 grid at C = 1024
+    # the listing's bounds int(C*gamma*j) where C*gamma is not an integer
+    (2, 3, 4, 10, 2, 0.25),      # bounds 2, 5, 7, 10
+    (1, 5, 6, 50, 1, 0.145),     # double rounding: last bound 28, channels 28.. copied
+    (2, 8, 8, 48, 1, 0.125),     # bounds 6, 12, 18, 24: vectors straddle, 24.. copied
+    (1, 8, 8, 64, 1, 0.125),     # bounds 8, 16, 24, 32: half the channels copied
+    (2, 4, 5, 26, 1, 0.25),      # bounds 6, 13, 19, 26
 ]
 
 
@@ -248,6 +254,27 @@ def test_large_shifts(vk, oracle_mod, s, H, W, kernel_path):
     wl = _custom("gate_qs", 1, H, W, C, "bf16", seed=77 + s, s=s)
     run_fused(vk, oracle_mod, wl)
     wl = _custom("gate_qs_x", 1, H, W, C, "f32", seed=78 + s, s=s)
+    run_fused(vk, oracle_mod, wl)
+
+
+# Channel groups at the listing's bounds int(C*gamma*j): unequal groups when
+# C*gamma is not an integer, copied channels when gamma < 1/4, on the generic
+# kernel and (bounds all multiples of 8) on the TMA path.
+LISTING_BOUNDS = [
+    # call, B, H, W, C, dtype, gamma
+    ("gate_qs_x", 1, 8, 16, 10, "bf16", 0.25),       # bounds 2, 5, 7, 10
+    ("gate_qs", 2, 12, 16, 26, "f32", 0.25),         # bounds 6, 13, 19, 26
+    ("qshift_biwkv", 1, 16, 16, 50, "f32", 0.145),   # bounds 7, 14, 21, 28
+    ("gate_qs_x", 2, 32, 32, 96, "bf16", 0.125),     # bounds 12, 24, 36, 48
+    ("gate_qs_x", 1, 64, 64, 64, "bf16", 0.125),     # TMA path: 8, 16, 24, 32
+    ("gate_qs", 2, 16, 64, 192, "bf16", 0.125),      # TMA path: 24, 48, 72, 96
+]
+
+
+@pytest.mark.parametrize("case", LISTING_BOUNDS, ids=lambda c: "_".join(map(str, c)))
+def test_listing_group_bounds(vk, oracle_mod, case, kernel_path):
+    call, B, H, W, C, dt, gamma = case
+    wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000, gamma=gamma)
     run_fused(vk, oracle_mod, wl)
 
 
