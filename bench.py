@@ -9,9 +9,13 @@ r, k and v, Bi-WKV (eq. 5) and the sigma(R) gate, fused in one kernel launch
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5]
                     [--impl ours|reference]
 
-Timing: the K timed launches are replayed from CUDA graphs between a
-barrier + synchronize on each side, timed with CUDA events on the launching
-stream; the max over ranks is taken.  Inputs and outputs rotate over enough
+Timing: the K timed launches are replayed from CUDA graphs (one graph of
+min(K, 64-ish) launches replayed, one more for any remainder, so every timed
+launch is graph-replayed at any K) between a barrier + synchronize on each
+side, timed with CUDA events on the launching stream; the max over ranks is
+taken.  SM clocks are sampled from a short pre-roll of the same launches
+(about 0.3 s, just before the timed region) through the end of the timed
+region, so a short region still gets many samples.  Inputs and outputs rotate over enough
 buffer sets that every launch reads and writes memory not touched for more
 than an L2's worth of traffic.  Multi-GPU runs are replicas (every (b, c)
 column is independent): each rank processes its own batch, no collective
@@ -57,6 +61,7 @@ METRIC = ("Bi-WKV fused fwd tokens·ch/s and HBM GB/s (% of B200 peak) "
 UNIT = "tokens*ch/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (~8 TB/s)
 CSRC = os.path.join(ROOT, "linear_complexity_vision_b200", "csrc")
 
 
@@ -201,6 +206,7 @@ class ClockSampler:
             return None
         return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "samples": len(self.samples),
+                "window": "pre-roll of the same launches (~0.3 s) + the timed region",
                 "reasons": sorted(n for b, n in self.REASONS.items() if self.reasons & b)}
 
 
@@ -266,6 +272,27 @@ def make_inputs(wl, torch, dev, rank):
     return inp, host, par, tdt
 
 
+def rotation_sets(wl) -> int:
+    """Input/output buffer sets the timed launches rotate over: enough that
+    every launch reads and writes memory untouched for over 3x the L2."""
+    es = 4 if wl.dtype == "f32" else 2
+    per_set = (len(wl.tensor_names()) + 1) * wl.N * es
+    return max(2, int(np.ceil(3 * L2_BYTES / per_set)) + 1)
+
+
+def bench_config(wl, world: int) -> dict:
+    """The workload as both arms report it."""
+    n = rotation_sets(wl)
+    es = 4 if wl.dtype == "f32" else 2
+    mb = n * (len(wl.tensor_names()) + 1) * wl.N * es / 1e6
+    return {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "W": wl.W, "C": wl.C,
+            "call": wl.call, "shift_pixel": wl.shift_pixel, "gamma": wl.gamma,
+            "io_dtype": wl.dtype, "accumulate": "f32",
+            "l2": f"inputs larger than L2: rotating {n} input/output buffer sets "
+                  f"({mb:.0f} MB > 126 MB L2)",
+            "parallelism": f"replicas x{world} (independent batches, no collective)"}
+
+
 class Runner:
     """Holds the rotating buffer sets and launches one step on set i."""
 
@@ -274,8 +301,7 @@ class Runner:
         self.inp, host, par, tdt = make_inputs(wl, torch, dev, rank)
         self.host = host
         self.par = {n: t.to(dev) for n, t in par.items()}
-        per_set = sum(t.numel() * t.element_size() for t in host.values()) * 2
-        self.nsets = max(2, int(np.ceil(3 * L2_BYTES / per_set)) + 1)
+        self.nsets = rotation_sets(wl)
         self.sets = []
         shape = (wl.B, wl.T, wl.C)
         for _ in range(self.nsets):
@@ -539,7 +565,9 @@ def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float, sm_mh
 
 
 def parity_sample(runner, out_dev, oracle, npts=128):
-    """Max |GPU - float64 oracle| on a seeded sample of output positions."""
+    """GPU against the float64 oracle on a seeded sample of output positions:
+    (max |GPU - oracle|, max |GPU - oracle| / max(|oracle|, 1e-6)); the second,
+    a plain relative error, is for information (outputs near zero inflate it)."""
     wl, inp = runner.wl, runner.inp
     got = out_dev.to(runner.torch.float64).cpu().numpy().reshape(-1)
     rng = np.random.default_rng(7)
@@ -557,7 +585,8 @@ def parity_sample(runner, out_dev, oracle, npts=128):
         r, k, v, p64["w"], p64["u"], wl.H, wl.W, idx, wl.shift_pixel, wl.gamma,
         p64.get("mu_r"), p64.get("mu_k"), p64.get("mu_v"),
         qshift_on=wl.call != "biwkv", gate_on=wl.call in ("gate_qs", "gate_qs_x"))
-    return float(np.max(np.abs(got[idx] - want)))
+    d = np.abs(got[idx] - want)
+    return float(np.max(d)), float(np.max(d / np.maximum(np.abs(want), 1e-6)))
 
 
 def oracle_throughput(wl, oracle, target_s: float, max_points: int = 1 << 20):
@@ -608,33 +637,51 @@ def run_ours(args, dist):
             out = runner.step(i)
     torch.cuda.synchronize(dev)
 
-    # capture one rotation period of launches (a multiple of nsets) per graph
-    G = runner.nsets * max(1, 64 // runner.nsets)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for i in range(G):
-            runner.step(i)
-    torch.cuda.synchronize(dev)
+    # The timed launches as CUDA graphs: G = min(K, one rotation period of
+    # about 64 launches) replayed reps times, then a graph of the remaining
+    # launches, so every timed launch is graph-replayed whatever K is.
+    # Launch i uses buffer set i mod nsets; G is a multiple of nsets whenever
+    # it repeats, so no set is used twice in a row.
+    Gmax = runner.nsets * max(1, 64 // runner.nsets)
+    G = min(args.steps, Gmax)
     reps, rem = divmod(args.steps, G)
 
-    clocks = ClockSampler(dist.local_rank)
+    def capture(n, first):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for i in range(first, first + n):
+                runner.step(i)
+        return gr
+
+    graph = capture(G, 0)
+    graph_rem = capture(rem, reps * G) if rem else None
+    torch.cuda.synchronize(dev)
+
+    # clocks: sampled from a pre-roll of the same launches (untimed, about
+    # 0.3 s) right before the timed region through its end
+    clocks = ClockSampler(dist.local_rank, period_s=0.005)
+    clocks.start()
+    t_pre = time.perf_counter()
+    with torch.cuda.stream(stream):
+        while time.perf_counter() - t_pre < 0.3:
+            graph.replay()
+            torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
     with torch.cuda.stream(stream):
         ev0.record(stream)
         for _ in range(reps):
             graph.replay()
-        for i in range(rem):
-            runner.step(i)
+        if graph_rem is not None:
+            graph_rem.replay()
         ev1.record(stream)
     torch.cuda.synchronize(dev)
     clocks.stop()
     dist.barrier()
     ms_local = ev0.elapsed_time(ev1)
     ms = dist.max(ms_local, dev)
-    del graph
+    del graph, graph_rem
 
     steps = args.steps
     units = wl.N
@@ -685,16 +732,13 @@ def run_ours(args, dist):
         "steps": steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "W": wl.W, "C": wl.C,
-                   "call": wl.call, "shift_pixel": wl.shift_pixel, "gamma": wl.gamma,
-                   "io_dtype": wl.dtype, "accumulate": "f32",
-                   "l2": f"rotating {runner.nsets} input/output buffer sets "
-                         f"({runner.nsets * 2 * wl.N * (4 if wl.dtype == 'f32' else 2) / 1e6:.0f} MB"
-                         " > 126 MB L2)",
-                   "timing": f"CUDA graphs of {G} launches, events on the launching stream",
-                   "parallelism": f"replicas x{dist.world} (independent batches, no collective)"},
+        "config": bench_config(wl, dist.world),
+        "timing": (f"{reps} replay(s) of a CUDA graph of {G} launches"
+                   + (f" + a graph of {rem}" if rem else "")
+                   + ", events on the launching stream"),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "kernel": runner.kernel_name,
                      "algorithmic_bytes_per_launch": fused_bytes,
                      "avg_launch_us": launch_s * 1e6},
@@ -705,7 +749,7 @@ def run_ours(args, dist):
     }
     # correctness guard on the main step's last output (first set of the
     # rotation), taken before the rows below reuse the device
-    parity_err = None
+    parity_err = (None, None)
     if dist.rank == 0:
         import oracle
         parity_err = parity_sample(runner, runner.sets[0]["out"], oracle)
@@ -730,7 +774,8 @@ def run_ours(args, dist):
     # the guard's result and, on one GPU, the CPU oracle baseline (rank 0)
     if dist.rank == 0:
         import oracle
-        line["parity_sample_max_abs_err"] = parity_err
+        line["parity_sample_max_abs_err"] = parity_err[0]
+        line["parity_sample_max_rel_err_plain"] = parity_err[1]
         if dist.world == 1 and not args.no_cpu_baseline:
             v, n, dt = oracle_throughput(wl, oracle, target_s=args.cpu_seconds)
             line["cpu_baseline"] = {
@@ -782,8 +827,7 @@ def run_reference(args, dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "W": wl.W, "C": wl.C,
-                   "call": wl.call},
+        "config": bench_config(wl, dist.world),
         "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
                          "cores": oracle.num_threads(),
                          "sample": f"{n} seeded output positions per step, each by direct eq. 5 "
