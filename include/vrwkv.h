@@ -21,9 +21,11 @@
  *   token, then batch.  With a patch grid H x W the token index is
  *   t = h*W + w (raster order) and T = H*W.  w, u and the mu vectors are
  *   dense float32 vectors of length C.
- * Memory.  Every pointer is caller-owned DEVICE memory.  No call allocates
- *   device memory; vrwkv_spatial_mix_block creates a cuBLASLt handle (host
- *   state) once per device.  The only device memory the library owns is
+ * Memory.  Every pointer is caller-owned DEVICE memory, except the token
+ *   buffers of vrwkv_spatial_gate_host (page-locked host memory).  No call
+ *   allocates device memory; vrwkv_spatial_mix_block creates a cuBLASLt
+ *   handle (host state) once per device, vrwkv_spatial_gate_host two copy
+ *   streams and a few events once per device.  The only device memory the library owns is
  *   reserved when it loads: a device error word and the fixed workspace of
  *   vrwkv_spatial_gate_static.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
@@ -181,6 +183,48 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
                                 const float* w, const float* u, void* out,
                                 int B, int T, int C, vrwkv_dtype dtype,
                                 const vrwkv_qshift_params* qs, void* stream);
+
+/*
+ * vrwkv_spatial_gate_host -- vrwkv_spatial_gate on HOST buffers, for callers
+ * whose tokens live in host memory: the same operation (eq. 2, eq. 5, eq. 9),
+ * with the host <-> device traffic overlapped with the computation.  The
+ * batch is cut into slices of slice_b rows (each (b, c) column is
+ * independent and Q-Shift mixes tokens of one batch row only, so a slice is
+ * an exact sub-problem); slice i is copied host -> device into slot i % 2 of
+ * dev_buf on a library copy stream, computed on `stream`, and copied back on
+ * a second copy stream, so both copy directions and the kernels overlap.
+ * Results equal vrwkv_spatial_gate's bit for bit.
+ *   r, k, v   (B, T, C) inputs in page-locked host memory (cudaHostAlloc or
+ *             cudaHostRegister); they may be the same buffer, copied once.
+ *   w, u      float32[C] in device memory; qs as for vrwkv_spatial_gate (its
+ *             mu vectors in device memory).
+ *   out       (B, T, C) page-locked host output, must not overlap an input.
+ *   slice_b   batch rows per slice, 1 <= slice_b <= B.
+ *   dev_buf   caller-owned device staging, 256-byte aligned, of at least
+ *             vrwkv_spatial_gate_host_buffer_bytes(slice_b, T, C, dtype,
+ *             number of distinct input buffers) bytes.
+ * Asynchronous on `stream`: work already queued there runs first, and the
+ * stream (so a synchronisation on it) completes after the last copy back;
+ * the host buffers must stay valid until then.  The library creates its two
+ * copy streams and a few events once per device and keeps them; calls from
+ * several host threads are serialised while they enqueue.
+ * Errors: INVALID_ARG for bad sizes, NULL pointers, an out-of-range slice_b,
+ *   a small or misaligned dev_buf, pageable host memory or an overlapping
+ *   output; the rest as vrwkv_spatial_gate.
+ */
+vrwkv_status vrwkv_spatial_gate_host(const void* r, const void* k,
+                                     const void* v, const float* w,
+                                     const float* u, void* out, int B, int T,
+                                     int C, vrwkv_dtype dtype,
+                                     const vrwkv_qshift_params* qs,
+                                     int slice_b, void* dev_buf,
+                                     size_t dev_buf_bytes, void* stream);
+
+/* Device staging bytes vrwkv_spatial_gate_host needs for slices of slice_b
+ * batch rows with `inputs` (1 to 3) distinct input buffers; 0 for invalid
+ * arguments. */
+size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C,
+                                            vrwkv_dtype dtype, int inputs);
 
 /*
  * Workspace variants of vrwkv_biwkv_fwd and vrwkv_spatial_gate.  Same
@@ -342,7 +386,8 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C,
  * vrwkv_device_status -- report and clear kernel-side failures on the
  * current device.  Kernels that wait for their asynchronous (TMA) tile
  * copies (bit 0) or, in the workspace variants, for the records of the other
- * CTAs of a column (bit 1) give up after about two seconds; a workspace
+ * CTAs of a column (bit 1) give up after the wait limit (two seconds unless
+ * vrwkv_set_wait_limit changes it); a workspace
  * variant that finds its workspace in an invalid state (not zero-filled
  * before first use; bit 2) stops at once.  Each records the failure in a
  * device error word and finishes (its outputs are then undefined) instead
@@ -353,6 +398,22 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C,
  */
 vrwkv_status vrwkv_device_status(void);
 
+/*
+ * vrwkv_set_wait_limit -- how long every bounded wait in the library's
+ * kernels (TMA tile completion, a cluster peer's mailbox record, a column
+ * peer's workspace record) may last before it gives up, records its bit in
+ * the device error word and lets the kernel finish.  The pages have no
+ * counterpart: this bounds the damage of a lost peer or copy.
+ *   seconds  0 < seconds <= 60 (default 2), measured on the GPU's global
+ *            timer.
+ * Applies to the current device, for every later launch on it.  It is a
+ * synchronous copy into device memory: call it outside stream capture and
+ * while no kernel of this library runs on the device.  A limit far below
+ * the kernels' normal run time makes healthy launches report timeouts.
+ * Errors: INVALID_ARG for a limit outside (0, 60]; VRWKV_ERR_CUDA if the
+ * device cannot be written.
+ */
+vrwkv_status vrwkv_set_wait_limit(double seconds);
 
 /* Name of the main kernel the calling thread's most recent successful
  * vrwkv_biwkv_fwd / vrwkv_spatial_gate / vrwkv_channel_mix / vrwkv_biwkv_bwd

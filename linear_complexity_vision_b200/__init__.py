@@ -10,6 +10,7 @@ There is no fallback: if the library is missing, the calls raise.
     biwkv_fwd(k, v, w, u, qs=None, workspace=None)
     spatial_gate(r, k, v, w, u, qs=None, workspace=None)
     fwd_workspace(B, T, C, device)  # a zeroed workspace for the two calls above
+    spatial_gate_host(r, k, v, w, u, qs=None, out=None, slice_b=1)  # host tensors, copies overlapped
     channel_mix(x, qs=None)
     biwkv_bwd(k, v, w, u, gy)  # -> gk, gv, gw (B, C), gu (B, C), gw_total, gu_total
     spatial_mix_block(x, weights, w, u, ln_gamma, ln_beta, qs, workspace=None)
@@ -88,12 +89,19 @@ def load_library():
         lib.vrwkv_spatial_gate_static.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                                   ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_spatial_gate_static.restype = ci
+        lib.vrwkv_spatial_gate_host.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                                ctypes.POINTER(_QsParams), ci, vp, ctypes.c_size_t, vp]
+        lib.vrwkv_spatial_gate_host.restype = ci
+        lib.vrwkv_spatial_gate_host_buffer_bytes.argtypes = [ci, ci, ci, ci, ci]
+        lib.vrwkv_spatial_gate_host_buffer_bytes.restype = ctypes.c_size_t
         lib.vrwkv_biwkv_bwd.argtypes = [vp] * 11 + [ci] * 4 + [vp]
         lib.vrwkv_biwkv_bwd.restype = ci
         lib.vrwkv_channel_mix.argtypes = [vp, vp, ci, ci, ci, ci, ctypes.POINTER(_QsParams), vp]
         lib.vrwkv_channel_mix.restype = ci
         lib.vrwkv_device_status.argtypes = []
         lib.vrwkv_device_status.restype = ci
+        lib.vrwkv_set_wait_limit.argtypes = [ctypes.c_double]
+        lib.vrwkv_set_wait_limit.restype = ci
         lib.vrwkv_status_string.argtypes = [ci]
         lib.vrwkv_status_string.restype = ctypes.c_char_p
         lib.vrwkv_last_kernel.argtypes = []
@@ -303,7 +311,11 @@ def spatial_gate_static(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
     """spatial_gate for callers that cannot allocate device memory: the
     column exchange runs in a fixed workspace the library reserved at load
     time (up to ~1600 (batch row, 8-channel) columns).  Calls overlapping in
-    time on other streams share that workspace and race."""
+    time on other streams share that workspace and race.
+
+    The C entry point allocates nothing.  Pass ``out`` (a preallocated
+    tensor like ``k``) to allocate nothing here either; without it this
+    wrapper allocates the output with torch."""
     import torch
     _require_tokens(("k", k), ("r", r), ("v", v))
     B, T, C = k.shape
@@ -316,6 +328,53 @@ def spatial_gate_static(r, k, v, w, u, qs: Optional[QShift] = None, out=None):
     _check(load_library().vrwkv_spatial_gate_static(
         r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
         B, T, C, _dtype_code(k), qsp, _stream_ptr(k)))
+    return out
+
+
+def spatial_gate_host_buffer(r, k, v, slice_b: int = 1, device="cuda"):
+    """A device staging buffer for spatial_gate_host on host tensors r, k, v
+    (the number of distinct buffers among them decides its size)."""
+    import torch
+    B, T, C = k.shape
+    inputs = len({t.data_ptr() for t in (r, k, v)})
+    n = int(load_library().vrwkv_spatial_gate_host_buffer_bytes(
+        int(slice_b), T, C, _dtype_code(k), inputs))
+    if n == 0:
+        raise ValueError("invalid arguments for the host staging buffer")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def spatial_gate_host(r, k, v, w, u, qs: Optional[QShift] = None, out=None, slice_b: int = 1,
+                      dev_buf=None, stream=None):
+    """spatial_gate on page-locked HOST tensors r, k, v (may be one tensor)
+    with the result written to the page-locked host tensor ``out``: batch
+    slices of ``slice_b`` rows stream through ``dev_buf`` (see
+    spatial_gate_host_buffer) with both copy directions overlapping the
+    kernels.  w, u and the QShift mu vectors are CUDA tensors.  Asynchronous
+    on ``stream`` (default: the current stream of w's device)."""
+    import torch
+    for t, name in ((k, "k"), (r, "r"), (v, "v")):
+        if t.device.type != "cpu" or not t.is_pinned() or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous page-locked CPU tensor")
+        if t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError(f"{name} must match k in shape and dtype")
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    for t, name in ((w, "w"), (u, "u")):
+        _require_vec(t, C, w.device, name)
+    if out is None:
+        out = torch.empty_like(k).pin_memory()
+    if out.shape != k.shape or out.dtype != k.dtype or not out.is_pinned() or not out.is_contiguous():
+        raise ValueError("out must be a contiguous page-locked CPU tensor like k")
+    if dev_buf is None:
+        dev_buf = spatial_gate_host_buffer(r, k, v, slice_b, device=w.device)
+    qsp = _qs_ptr(qs, C, w.device)
+    s = stream if stream is not None else torch.cuda.current_stream(w.device)
+    _check(load_library().vrwkv_spatial_gate_host(
+        r.data_ptr(), k.data_ptr(), v.data_ptr(), w.data_ptr(), u.data_ptr(), out.data_ptr(),
+        B, T, C, _dtype_code(k), qsp, int(slice_b), dev_buf.data_ptr(),
+        dev_buf.numel() * dev_buf.element_size(), s.cuda_stream))
     return out
 
 
@@ -382,6 +441,12 @@ def biwkv_bwd(k, v, w, u, gy, totals: bool = True):
         gv.data_ptr(), gw.data_ptr(), gu.data_ptr(), None if gwt is None else gwt.data_ptr(),
         None if gut is None else gut.data_ptr(), B, T, C, _dtype_code(k), _stream_ptr(k)))
     return gk, gv, gw, gu, gwt, gut
+
+
+def set_wait_limit(seconds: float) -> None:
+    """Limit of every bounded wait in the kernels on the current device
+    (vrwkv_set_wait_limit; default 2 s).  Call outside stream capture."""
+    _check(load_library().vrwkv_set_wait_limit(float(seconds)))
 
 
 def device_status() -> None:

@@ -57,7 +57,17 @@ constexpr int kNP = kCS / 2;    // channel pairs per CTA
 constexpr int kL = 8;           // tokens per sub-chunk (= the TMA element stride)
 constexpr int kCPW = 32 / kNP;  // chunks per warp
 constexpr int kClusterMax = 16;
-constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+
+// Limit of every bounded wait in the library's kernels, in nanoseconds of the
+// GPU's global timer: 2 s unless vrwkv_set_wait_limit changes it (per device).
+// A wait that runs out records a flag in the device error word and lets the
+// kernel finish, so the context stays usable.
+__device__ unsigned long long g_vrwkv_wait_ns = 2000000000ull;
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 // CTA shape: NT threads = kNP channel pairs x NT/kNP chunks of KL tokens
 // (KL = 8: one sub-chunk, 64 registers per thread; KL = 16: two sub-chunks
@@ -101,7 +111,7 @@ struct alignas(64) Params {
     unsigned int* ws_ctl;   // [0] ticket counter, [1] finished CTAs, [2] generation
     unsigned int* ws_flag;  // per (column, rank): generation + 1 once its record is out
     float4* ws_rec;         // per (column, rank): kRecF4 float4 record
-    int nslab;           // channel slabs (C / 16)
+    int nslab;           // channel slabs (C / 8)
     int total;           // CTAs in the grid
 };
 
@@ -170,13 +180,14 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned 
         : "memory");
     return ok != 0;
 }
-// Wait for phase 0 of the barrier; give up after ~2 s, record the failure in
-// the device error word and continue (the caller's barriers stay matched).
+// Wait for phase 0 of the barrier; give up after the wait limit, record the
+// failure in the device error word and continue (the caller's barriers stay
+// matched).
 __device__ __forceinline__ void mbar_wait_bounded(unsigned long long* bar, unsigned* err) {
     if (mbar_try_wait(bar, 0)) return;
-    const long long t0 = clock64();
+    const unsigned long long t0 = global_ns(), lim = g_vrwkv_wait_ns;
     while (!mbar_try_wait(bar, 0)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (global_ns() - t0 > lim) {
             atomicOr(err, 1u);
             return;
         }
@@ -249,9 +260,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(unsigned long long* bar, u
 }
 __device__ __forceinline__ void mbar_wait_cluster_bounded(unsigned long long* bar, unsigned* err) {
     if (mbar_try_wait_cluster(bar, 0)) return;
-    const long long t0 = clock64();
+    const unsigned long long t0 = global_ns(), lim = g_vrwkv_wait_ns;
     while (!mbar_try_wait_cluster(bar, 0)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (global_ns() - t0 > lim) {
             atomicOr(err, 1u);
             return;
         }
@@ -299,14 +310,14 @@ __device__ __forceinline__ void wait_flag(const unsigned int* f, unsigned int wa
     unsigned int v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
     if (v == want) return;
-    const long long t0 = clock64();
+    const unsigned long long t0 = global_ns(), lim = g_vrwkv_wait_ns;
     unsigned int ns = 32;
     for (;;) {
         __nanosleep(ns);
         if (ns < 1024) ns <<= 1;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
         if (v == want) return;
-        if (clock64() - t0 > kWaitCycles) {
+        if (global_ns() - t0 > lim) {
             atomicOr(err, 2u);
             return;
         }

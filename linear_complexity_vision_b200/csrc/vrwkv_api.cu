@@ -811,6 +811,155 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
     return dtype == VRWKV_F32 ? dispatch_layout<float>(pl, s) : dispatch_layout<__nv_bfloat16>(pl, s);
 }
 
+// ---------------------------------------------------------------------------
+// Host-buffer front end of vrwkv_spatial_gate: the batch is cut into slices
+// of slice_b rows (every (b, c) column is independent and Q-Shift mixes
+// tokens of one batch row only, so a slice is an exact sub-problem); slice i
+// is copied host -> device into slot i % 2 of the caller's device buffer on a
+// copy-in stream, computed on the caller's stream and copied back on a
+// copy-out stream, so the two copy directions and the kernels overlap.
+// ---------------------------------------------------------------------------
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+size_t host_slot_bytes(int slice_b, int T, int C, int es, int inputs) {
+    const size_t tensor = (size_t)slice_b * T * C * es;
+    return (size_t)(inputs + 1) * round256(tensor);
+}
+
+// Streams and events of the pipeline, created once per device (never freed:
+// they live as long as the process, like the library's other per-device
+// state).  A mutex serialises the enqueueing of calls from different host
+// threads onto them.
+struct HostPipe {
+    cudaStream_t in = nullptr, outs = nullptr;
+    cudaEvent_t start = nullptr, loaded[2] = {}, done[2] = {}, freed[2] = {};
+    bool ok = false;
+};
+
+HostPipe* host_pipe(int dev) {
+    static std::mutex mu;
+    static HostPipe pipes[64];
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 0 || dev >= 64) return nullptr;
+    HostPipe& p = pipes[dev];
+    if (!p.ok) {
+        bool good = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&p.outs, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; i < 2 && good; ++i)
+            good = cudaEventCreateWithFlags(&p.loaded[i], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&p.done[i], cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&p.freed[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!good) return nullptr;
+        p.ok = true;
+    }
+    return &p;
+}
+
+std::mutex& host_pipe_enqueue_mutex() {
+    static std::mutex mu;
+    return mu;
+}
+
+bool host_pinned(const void* p) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+
+vrwkv_status host_pipeline(const void* r, const void* k, const void* v, const float* w, const float* u,
+                           void* out, int B, int T, int C, vrwkv_dtype dtype, const vrwkv_qshift_params* qs,
+                           int slice_b, void* dev_buf, size_t dev_buf_bytes, cudaStream_t s) {
+    if (dtype != VRWKV_F32 && dtype != VRWKV_BF16)
+        return fail(VRWKV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B <= 0 || T <= 0 || C <= 0)
+        return fail(VRWKV_ERR_INVALID_ARG, "B, T and C must be positive (got %d, %d, %d)", B, T, C);
+    if (!r || !k || !v || !w || !u || !out || !dev_buf)
+        return fail(VRWKV_ERR_INVALID_ARG, "required pointer is NULL");
+    if (slice_b <= 0 || slice_b > B)
+        return fail(VRWKV_ERR_INVALID_ARG, "slice_b must lie in [1, B] (got %d)", slice_b);
+    const int es = elem_bytes(dtype);
+    // distinct host inputs: r, k, v may be one buffer (copied once)
+    const void* srcs[3] = {k, v, r};
+    int slot_of[3] = {0, 0, 0};
+    int inputs = 0;
+    for (int i = 0; i < 3; ++i) {
+        int found = -1;
+        for (int j = 0; j < i; ++j)
+            if (srcs[j] == srcs[i]) found = slot_of[j];
+        slot_of[i] = found >= 0 ? found : inputs++;
+    }
+    const size_t tensor_full = (size_t)B * T * C * es;
+    for (int i = 0; i < 3; ++i)
+        if (overlaps(out, tensor_full, srcs[i], tensor_full))
+            return fail(VRWKV_ERR_INVALID_ARG, "out overlaps an input");
+    const size_t slot = host_slot_bytes(slice_b, T, C, es, inputs);
+    if (dev_buf_bytes < 2 * slot)
+        return fail(VRWKV_ERR_INVALID_ARG, "device buffer holds %zu bytes; slices of %d rows need %zu",
+                    dev_buf_bytes, slice_b, 2 * slot);
+    if (!aligned(dev_buf, 256)) return fail(VRWKV_ERR_INVALID_ARG, "device buffer must be 256-byte aligned");
+    for (const void* p : {r, k, v, (const void*)out})
+        if (!host_pinned(p))
+            return fail(VRWKV_ERR_INVALID_ARG, "host buffers must be page-locked (cudaHostAlloc / cudaHostRegister)");
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaGetLastError(), "cudaGetDevice");
+    HostPipe* hp = host_pipe(dev);
+    if (!hp) return fail(VRWKV_ERR_CUDA, "cannot create the copy streams");
+    std::lock_guard<std::mutex> guard(host_pipe_enqueue_mutex());
+
+    const size_t row = (size_t)T * C * es;  // bytes of one batch row
+    const size_t part = round256((size_t)slice_b * row);
+    char* base = static_cast<char*>(dev_buf);
+    auto in_ptr = [&](int sl, int i) { return base + sl * slot + (size_t)slot_of[i] * part; };
+    auto out_ptr = [&](int sl) { return base + sl * slot + (size_t)inputs * part; };
+    auto check = [&](cudaError_t e, const char* what) -> bool {
+        if (e == cudaSuccess) return true;
+        cuda_status(e, what);
+        return false;
+    };
+    // the pipeline starts after the work already queued on the caller's stream
+    if (!check(cudaEventRecord(hp->start, s), "event record") ||
+        !check(cudaStreamWaitEvent(hp->in, hp->start, 0), "stream wait") ||
+        !check(cudaStreamWaitEvent(hp->outs, hp->start, 0), "stream wait"))
+        return VRWKV_ERR_CUDA;
+    const int nslices = (B + slice_b - 1) / slice_b;
+    for (int i = 0; i < nslices; ++i) {
+        const int sl = i & 1;
+        const int b0 = i * slice_b, nb = std::min(slice_b, B - b0);
+        const size_t off = (size_t)b0 * row, n = (size_t)nb * row;
+        if (i >= 2 && !check(cudaStreamWaitEvent(hp->in, hp->freed[sl], 0), "stream wait")) return VRWKV_ERR_CUDA;
+        for (int j = 0; j < inputs; ++j) {
+            int src = 0;
+            while (slot_of[src] != j) ++src;
+            if (!check(cudaMemcpyAsync(in_ptr(sl, src), static_cast<const char*>(srcs[src]) + off, n,
+                                       cudaMemcpyHostToDevice, hp->in),
+                       "host-to-device copy"))
+                return VRWKV_ERR_CUDA;
+        }
+        if (!check(cudaEventRecord(hp->loaded[sl], hp->in), "event record") ||
+            !check(cudaStreamWaitEvent(s, hp->loaded[sl], 0), "stream wait"))
+            return VRWKV_ERR_CUDA;
+        const vrwkv_status st = fused_entry(true, in_ptr(sl, 2), in_ptr(sl, 0), in_ptr(sl, 1), w, u, out_ptr(sl),
+                                            nb, T, C, dtype, qs, s);
+        if (st != VRWKV_OK) return st;
+        if (!check(cudaEventRecord(hp->done[sl], s), "event record") ||
+            !check(cudaStreamWaitEvent(hp->outs, hp->done[sl], 0), "stream wait") ||
+            !check(cudaMemcpyAsync(static_cast<char*>(out) + off, out_ptr(sl), n, cudaMemcpyDeviceToHost,
+                                   hp->outs),
+                   "device-to-host copy") ||
+            !check(cudaEventRecord(hp->freed[sl], hp->outs), "event record"))
+            return VRWKV_ERR_CUDA;
+    }
+    // the caller's stream completes after the last copy back
+    if (!check(cudaEventRecord(hp->freed[0], hp->outs), "event record") ||
+        !check(cudaStreamWaitEvent(s, hp->freed[0], 0), "stream wait"))
+        return VRWKV_ERR_CUDA;
+    return ok();
+}
+
 }  // namespace
 
 extern "C" {
@@ -1227,6 +1376,21 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v, con
     return fused_entry(true, r, k, v, w, u, out, B, T, C, dtype, qs, stream);
 }
 
+size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C, vrwkv_dtype dtype, int inputs) {
+    if (slice_b <= 0 || T <= 0 || C <= 0 || inputs < 1 || inputs > 3 ||
+        (dtype != VRWKV_F32 && dtype != VRWKV_BF16))
+        return 0;
+    return 2 * host_slot_bytes(slice_b, T, C, elem_bytes(dtype), inputs);
+}
+
+vrwkv_status vrwkv_spatial_gate_host(const void* r, const void* k, const void* v, const float* w,
+                                     const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
+                                     const vrwkv_qshift_params* qs, int slice_b, void* dev_buf,
+                                     size_t dev_buf_bytes, void* stream) {
+    return host_pipeline(r, k, v, w, u, out, B, T, C, dtype, qs, slice_b, dev_buf, dev_buf_bytes,
+                         static_cast<cudaStream_t>(stream));
+}
+
 size_t vrwkv_fwd_workspace_bytes(int B, int T, int C) {
     (void)T;
     if (B <= 0 || C <= 0) return 0;
@@ -1262,6 +1426,13 @@ const char* vrwkv_status_string(vrwkv_status status) {
 const char* vrwkv_last_error(void) { return g_last_error.c_str(); }
 
 const char* vrwkv_last_kernel(void) { return g_last_kernel; }
+
+vrwkv_status vrwkv_set_wait_limit(double seconds) {
+    if (!(seconds > 0.0 && seconds <= 60.0))
+        return fail(VRWKV_ERR_INVALID_ARG, "wait limit must lie in (0, 60] seconds");
+    const unsigned long long ns = (unsigned long long)(seconds * 1e9);
+    return cuda_status(cudaMemcpyToSymbol(fast::g_vrwkv_wait_ns, &ns, sizeof(ns)), "setting the wait limit");
+}
 
 vrwkv_status vrwkv_device_status(void) {
     unsigned int* word = device_error_word();

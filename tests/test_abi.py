@@ -213,3 +213,44 @@ def test_block_rejects_invalid_arguments(lib, args, frag):
                                      a["dtype"], _qs(14, 14), a["ws"], nb, None)
     assert st in (1, 2)
     assert frag in lib.vrwkv_last_error().decode()
+
+
+@pytest.mark.parametrize("seconds", [0.0, -1.0, 61.0, float("nan")])
+def test_wait_limit_outside_range_is_rejected_on_the_host(lib, seconds):
+    lib.vrwkv_set_wait_limit.argtypes = [ctypes.c_double]
+    assert lib.vrwkv_set_wait_limit(seconds) == 1  # VRWKV_ERR_INVALID_ARG
+    assert b"wait limit" in lib.vrwkv_last_error()
+
+
+def test_host_buffer_bytes(lib):
+    f = lib.vrwkv_spatial_gate_host_buffer_bytes
+    f.argtypes = [ctypes.c_int] * 5
+    f.restype = ctypes.c_size_t
+    # two slots of (inputs + 1) tensors of slice_b * T * C elements, 256-byte rounded
+    assert f(1, 4096, 1024, 1, 1) == 2 * 2 * 4096 * 1024 * 2
+    assert f(2, 196, 768, 0, 3) == 2 * 4 * ((2 * 196 * 768 * 4 + 255) // 256 * 256)
+    assert f(1, 3, 5, 1, 1) == 2 * 2 * 256
+    for bad in ((0, 16, 16, 1, 1), (1, 16, 16, 1, 0), (1, 16, 16, 1, 4), (1, 16, 16, 7, 1)):
+        assert f(*bad) == 0
+
+
+@pytest.mark.parametrize("args,frag", [
+    (dict(B=0), "positive"),
+    (dict(slice_b=0), "slice_b"),
+    (dict(slice_b=9), "slice_b"),
+    (dict(dev_buf=None), "NULL"),
+    (dict(dtype=7), "dtype"),
+    (dict(dev_bytes=100), "device buffer"),
+    (dict(dev_buf=FAKE + 16), "aligned"),
+])
+def test_host_pipeline_rejects_bad_arguments_on_the_host(lib, args, frag):
+    a = dict(r=FAKE, k=FAKE, v=FAKE, w=FAKE, u=FAKE, out=2 * FAKE, B=8, T=64, C=32, dtype=1,
+             slice_b=1, dev_buf=4 * FAKE, dev_bytes=1 << 30)
+    a.update(args)
+    vp, ci = ctypes.c_void_p, ctypes.c_int
+    fn = lib.vrwkv_spatial_gate_host
+    fn.argtypes = [vp] * 6 + [ci] * 4 + [vp, ci, vp, ctypes.c_size_t, vp]
+    st = fn(a["r"], a["k"], a["v"], a["w"], a["u"], a["out"], a["B"], a["T"], a["C"], a["dtype"],
+            None, a["slice_b"], a["dev_buf"], a["dev_bytes"], None)
+    assert st == 1, lib.vrwkv_last_error()
+    assert frag in lib.vrwkv_last_error().decode()
