@@ -459,7 +459,7 @@ def measured_tensor_peak():
 
 def time_block(runner, stream, torch, dev, launches: int):
     """The spatial-mix block with projections (vrwkv_spatial_mix_block) at the
-    workload's (B, T, C): Q-Shift, four cuBLASLt GEMMs, the fused core and a
+    workload's (B, T, C): Q-Shift, four tcgen05 GEMMs, the fused core and a
     LayerNorm per launch.  Roofline against the dense bf16 peak with the four
     GEMMs' 8*B*T*C^2 FLOPs; random weights of scale 1/sqrt(C)."""
     wl, vk = runner.wl, runner.vk
@@ -486,8 +486,9 @@ def time_block(runner, stream, torch, dev, launches: int):
         for i in range(3):
             launch(i)
     torch.cuda.synchronize(dev)
-    # replayed from a CUDA graph (the block issues ~9 launches and cuBLASLt
-    # calls per step; the graph keeps host time out of the measurement)
+    # replayed from a CUDA graph (the block issues about 13 launches per step:
+    # weight transposes, GEMMs, mixes, the core, LayerNorm; the graph keeps
+    # host time out of the measurement)
     G = n * max(1, 8 // n)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
@@ -512,7 +513,7 @@ def time_block(runner, stream, torch, dev, launches: int):
     return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "peak_source": kind, "kernel": "spatial_mix_block",
             "flops_per_launch": flops, "avg_launch_us": us, "launches": launches,
-            "gemm": "cuBLASLt bf16, float32 accumulation",
+            "gemm": "library tcgen05 kernel (gemm_tc_kernel), bf16, float32 accumulation in tensor memory",
             "timing": "CUDA graphs over the rotating buffer sets"}
 
 

@@ -23,9 +23,9 @@
  *   dense float32 vectors of length C.
  * Memory.  Every pointer is caller-owned DEVICE memory, except the token
  *   buffers of vrwkv_spatial_gate_host (page-locked host memory).  No call
- *   allocates device memory; vrwkv_spatial_mix_block creates a cuBLASLt
- *   handle (host state) once per device, vrwkv_spatial_gate_host two copy
- *   streams and a few events once per device.  The only device memory the library owns is
+ *   allocates device memory; vrwkv_spatial_gate_host creates two copy
+ *   streams and a few events once per device.  The only device memory the
+ *   library owns is
  *   reserved when it loads: a device error word and the fixed workspace of
  *   vrwkv_spatial_gate_static.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
@@ -147,15 +147,25 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *   wkv   (B, T, C) output, same dtype, must not overlap k, v, w or u.
  *   qs    NULL, or Q-Shift parameters applied to k (mu_k) and v (mu_v) on
  *         load (mu_r is ignored); T must then equal qs->H * qs->W.
- * Kernels: a TMA fast path serves C % 8 == 0 with 16-byte-aligned inputs
- *   (and, with qs, channel-group bounds int(C*gamma*j) that are all
- *   multiples of 8, and W <= 256); everything else runs a generic kernel with the same
- *   results up to rounding.  Setting VRWKV_DISABLE_TMA=1 in the environment
- *   forces the generic kernel, VRWKV_TMA_CHUNK=8 holds the fast path to
- *   8-token thread chunks and VRWKV_NO_TMA_STORE=1 to per-thread stores of
- *   its results (diagnostics).
- * Limits: T <= 4096 (UNSUPPORTED above); on the generic kernel with qs, a
- *   halo of shift_pixel*W tokens must fit its shared-memory tile.
+ * Kernels (the same results up to rounding):
+ *   - the 8-channel TMA kernel, the default: C % 8 == 0, 16-byte-aligned
+ *     inputs and, with qs, group bounds int(C*gamma*j) that are multiples of
+ *     8 and W <= 256, T <= 8192;
+ *   - the 16-channel slab kernel, with VRWKV_FORWARD=wide in the
+ *     environment (and for long sequences through the workspace variants):
+ *     C % 16 == 0, T % 16 == 0, T <= 4096, 16-byte-aligned tensors and,
+ *     with qs, bounds that are multiples of 16, W % 16 == 0, shift_pixel 1
+ *     where a horizontal group exists and shift_pixel*W <= 256 for the
+ *     vertical ones;
+ *   - a generic kernel for everything else (T <= 4096).
+ *   Setting VRWKV_DISABLE_TMA=1 in the environment forces the generic
+ *   kernel, VRWKV_DISABLE_WIDE=1 keeps the 16-channel one off, VRWKV_TMA_CHUNK=8 holds
+ *   the 8-channel kernel to 8-token thread chunks and VRWKV_NO_TMA_STORE=1
+ *   to per-thread stores of its results (diagnostics).
+ * Limits: T <= 8192 on the 8-channel kernel, 4096 on the others
+ *   (UNSUPPORTED above; the workspace variants below reach 32768); on the
+ *   generic kernel with qs, a halo of shift_pixel*W tokens must fit its
+ *   shared-memory tile.
  *   Exponents are renormalised by the running maximum of k, so a constant
  *   added to every k of a channel leaves wkv unchanged; results stay finite
  *   while |w| + (spread of k within a channel) stays well below 80.
@@ -228,11 +238,15 @@ size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C,
 
 /*
  * Workspace variants of vrwkv_biwkv_fwd and vrwkv_spatial_gate.  Same
- * operations, arguments, results and limits; for sequences that span several
- * CTAs the CTAs of one (b, 8-channel) column exchange their partial sums
- * through the caller's workspace instead of a thread-block cluster, which
- * frees the kernel from cluster co-scheduling (every SM can hold its full
- * share of CTAs).
+ * operations, arguments and results.  Up to 4096 tokens, the CTAs of one
+ * (b, 8-channel) column exchange their partial sums through the caller's
+ * workspace instead of a thread-block cluster, which frees the kernel from
+ * cluster co-scheduling.  Longer sequences (up to T = 32768, e.g. the
+ * 16384 tokens of a 2048^2 image at patch 16) run on the 16-channel kernel
+ * when the shape qualifies for it: a column splits into segments of one
+ * 8-CTA cluster (4096 tokens); segments take tickets from a counter in the
+ * workspace, publish their totals there and wait, bounded, for the other
+ * segments of their column.
  *   workspace        device memory of at least vrwkv_fwd_workspace_bytes(B,
  *                    T, C) bytes, 256-byte aligned, owned by the caller.  It
  *                    must be zero-filled once before its first use; the
@@ -241,7 +255,8 @@ size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C,
  *                    the same time (other streams) need separate workspaces;
  *                    calls queued on one stream may share one.
  *   workspace_bytes  its size.
- * The CTAs of a column wait for one another with a bounded spin (~2 s); a
+ * The CTAs of a column wait for one another with a bounded spin (the wait
+ * limit, 2 s by default; see vrwkv_set_wait_limit); a
  * timeout is recorded in the device error word (see vrwkv_device_status).
  * Errors: as the plain entry points, plus INVALID_ARG for a NULL, misaligned,
  *   too small or overlapping workspace.
@@ -301,15 +316,20 @@ vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k,
  *   qs         required: grid, shift, gamma and mu_r, mu_k, mu_v.
  *   workspace  device memory of at least vrwkv_block_workspace_bytes(B, T,
  *              C, dtype) bytes, 256-byte aligned: six (B, T, C) staging
- *              buffers and the GEMM workspace.
+ *              buffers and the four weights transposed to (C_out, C_in).
  * Steps (all on `stream`): the three Q-Shift mixes (one pass over x; each
- * bit-identical to vrwkv_qshift's), three cuBLASLt GEMMs (float32
- * accumulation, results stored in `dtype`), the fused vrwkv_spatial_gate core
- * on the projected R, K, V, the W_O GEMM and a LayerNorm kernel.  The
- * cuBLASLt handle and each GEMM shape's plan are created once per device.
+ * bit-identical to vrwkv_qshift's), three projection GEMMs, the fused
+ * vrwkv_spatial_gate core on the projected R, K, V, the W_O GEMM and a
+ * LayerNorm kernel.  The GEMMs are the library's own: for bfloat16 a
+ * tcgen05 tensor-core kernel (TMA tiles with the 128-byte swizzle, float32
+ * accumulators in tensor memory, results rounded to bfloat16 once) after a
+ * transpose of each weight into the workspace; for float32 a kernel on the
+ * FP32 pipes.  bfloat16 needs C % 8 == 0.
  * Errors: INVALID_ARG for bad sizes, NULL or misaligned pointers, overlaps,
- *   bad qs fields or a small workspace; UNSUPPORTED for B*T >= 2^31 or the
- *   core's limits; CUDA if cuBLASLt fails.
+ *   bad qs fields or a small workspace; UNSUPPORTED for B*T >= 2^31, a
+ *   bfloat16 C that is not a multiple of 8, or the core's limits; CUDA for a
+ *   failed launch.  A GEMM wait that runs out sets flag 8 of the device
+ *   error word (vrwkv_device_status).
  */
 size_t vrwkv_block_workspace_bytes(int B, int T, int C, vrwkv_dtype dtype);
 

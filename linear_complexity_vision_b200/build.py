@@ -14,8 +14,7 @@ SOURCES = ["vrwkv_api.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
               "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-O2",
               "-I" + os.path.join(ROOT, "include"), "-I" + CSRC]
-# cuBLASLt serves the dense projections of the spatial-mix block
-LIBS = ["-lcublasLt"]
+LIBS: list = []
 
 
 def _stale() -> bool:

@@ -1,0 +1,372 @@
+// Dense projections of the spatial-mix block ("Vision-RWKV Backbone",
+// Overall Architecture, eq. 1-2: R, K, V = Q-Shift(X) W_R, W_K, W_V and the
+// output projection W_O) on the 5th-generation tensor cores, sm_100a:
+//
+//   D[M, N] = A[M, K] * Bt[N, K]^T     A, Bt, D row-major bfloat16,
+//                                      float32 accumulation in tensor memory.
+//
+// Persistent kernel, one CTA per SM, 192 threads in three roles:
+//  * warp 0, one lane: TMA producer.  A (128 x 64) and Bt (256 x 64) tiles
+//    arrive with the 128-byte swizzle into a ring of 4 shared-memory stages,
+//    completing on the stage's "full" mbarrier.
+//  * warp 1: allocates 512 tensor-memory columns (two 128 x 256 float32
+//    accumulators); one lane issues tcgen05.mma kind::f16 (K = 16 per
+//    instruction, four per stage) and frees each stage with tcgen05.commit
+//    onto its "empty" mbarrier; after a tile's last stage it commits onto
+//    the accumulator's "full" barrier.
+//  * warps 2-5: epilogue.  Warp w reads tensor-memory lanes 32 (w mod 4) ..
+//    +31 (rows of the tile) with tcgen05.ld, 32 columns at a time, converts
+//    to bfloat16 and stores the rows; then releases the accumulator, so the
+//    MMAs of the next tile overlap this epilogue.
+// Output tiles are taken round-robin, N fastest, so the CTAs working at one
+// time share A rows in L2 (Bt, the weights, stays resident in L2).
+// Every mbarrier wait is bounded (the library's wait limit): a wait that runs
+// out records flag 8 in the device error word, makes every role leave its
+// loop, waits (bounded) for the copies and MMAs already issued and frees the
+// tensor memory before the CTA exits.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "biwkv_tma.cuh"
+
+namespace vrwkv {
+namespace tcgemm {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kStages = 4;
+constexpr int kAcc = 2;                       // accumulator buffers in tensor memory
+constexpr int kTmemCols = kAcc * BN;          // 512: all of an SM's tensor memory
+constexpr int kThreads = 192;
+constexpr int A_BYTES = BM * BK * 2;          // 16 KB
+constexpr int B_BYTES = BN * BK * 2;          // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr unsigned kErrFlag = 8u;
+
+struct Params {
+    CUtensorMap ma;  // A as (K, M): box (64, 128), 128-byte swizzle
+    CUtensorMap mb;  // Bt as (K, N): box (64, 256), 128-byte swizzle
+    __nv_bfloat16* d;
+    int M, N, K;
+    unsigned int* err;
+};
+
+struct alignas(1024) Smem {
+    uint8_t a[kStages][A_BYTES];
+    uint8_t b[kStages][B_BYTES];
+    unsigned long long full[kStages], empty[kStages];
+    unsigned long long tfull[kAcc], tempty[kAcc];
+    unsigned long long drain;  // completion of every issued MMA (abort path)
+    unsigned tmem_base;
+    int abort;
+};
+
+// Shared-memory matrix descriptor of a K-major tile with the 128-byte
+// swizzle: 8-row groups 1024 bytes apart (stride byte offset 64 x 16 B),
+// leading byte offset 1 (unused by the swizzled K-major layout), descriptor
+// version 1, layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)64 << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f16: float32 accumulator, bfloat16 A and
+// B, both K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            unsigned long long* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(fast::smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(fast::smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(unsigned long long* bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(fast::smem_u32(bar)), "r"(parity), "r"(100000u)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase of parity `parity`; false if it ran out or the
+// CTA is aborting (the first to run out records the failure).
+__device__ __forceinline__ bool wait_phase(unsigned long long* bar, unsigned parity, volatile int* abort,
+                                           unsigned* err) {
+    if (mbar_test(bar, parity)) return true;
+    const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+    while (!mbar_test(bar, parity)) {
+        if (*abort) return false;
+        if (fast::global_ns() - t0 > lim) {
+            atomicOr(err, kErrFlag);
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(fast::smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(unsigned long long* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     fast::smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive float32 columns of one tensor-memory lane per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+          "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+          "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(1024) char smem_raw[];
+    Smem& S = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (fast::smem_u32(smem_raw) & 1023u)) & 1023u));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nt = (p.N + BN - 1) / BN, mt = (p.M + BM - 1) / BM;
+    const int ntiles = nt * mt, nk = (p.K + BK - 1) / BK;
+    volatile int* abort = &S.abort;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            fast::mbar_init(&S.full[s], 1);
+            fast::mbar_init(&S.empty[s], 1);
+        }
+        for (int a = 0; a < kAcc; ++a) {
+            fast::mbar_init(&S.tfull[a], 1);
+            fast::mbar_init(&S.tempty[a], 4);  // one arrival per epilogue warp
+        }
+        fast::mbar_init(&S.drain, 1);
+        S.abort = 0;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         fast::smem_u32(&S.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer: one A and one Bt tile per stage
+            int it = 0;
+            int last_par[kStages];
+            for (int s = 0; s < kStages; ++s) last_par[s] = -1;
+            for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+                const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const unsigned ph = (it / kStages) & 1;
+                    if (!wait_phase(&S.empty[s], ph ^ 1u, abort, p.err)) break;
+                    fast::mbar_expect_tx(&S.full[s], STAGE_BYTES);
+                    tma_load_2d(S.a[s], &p.ma, kb * BK, m0, &S.full[s]);
+                    tma_load_2d(S.b[s], &p.mb, kb * BK, n0, &S.full[s]);
+                    last_par[s] = (int)ph;
+                }
+            }
+            if (*abort) {
+                // let the copies already issued land before the CTA exits
+                for (int s = 0; s < kStages; ++s) {
+                    if (last_par[s] < 0) continue;
+                    const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+                    while (!mbar_test(&S.full[s], (unsigned)last_par[s]) && fast::global_ns() - t0 <= lim) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // MMA issuer
+            int it = 0, lt = 0;
+            bool issued = false;
+            for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++lt) {
+                const int acc = lt & 1;
+                const unsigned aph = (lt >> 1) & 1;
+                if (!wait_phase(&S.tempty[acc], aph ^ 1u, abort, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const unsigned ph = (it / kStages) & 1;
+                    if (!wait_phase(&S.full[s], ph, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(fast::smem_u32(S.a[s]));
+                    const uint64_t bd = sw128_desc(fast::smem_u32(S.b[s]));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)  // 32 bytes of K per instruction
+                        tc_mma(d_tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), kIdesc,
+                               (kb > 0 || k > 0) ? 1u : 0u);
+                    issued = true;
+                    tc_commit(&S.empty[s]);
+                }
+                if (!ok) break;
+                tc_commit(&S.tfull[acc]);
+            }
+            if (*abort && issued) {
+                // every MMA issued so far completes before the memory is freed
+                tc_commit(&S.drain);
+                const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+                while (!mbar_test(&S.drain, 0) && fast::global_ns() - t0 <= lim) {
+                }
+            }
+        }
+    } else {
+        // epilogue: warp w reads tensor-memory lanes 32 (w mod 4) .. + 31
+        const int quad = warp & 3;
+        int lt = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            const unsigned aph = (lt >> 1) & 1;
+            if (!wait_phase(&S.tfull[acc], aph, abort, p.err)) break;
+            tc_fence_after();
+            const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
+            const int row = m0 + quad * 32 + lane;
+            const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tbase + (uint32_t)(c * 32), v);
+                const int col = n0 + c * 32;
+                if (row < p.M && col < p.N) {
+                    uint32_t w16[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]),
+                                                                       __uint_as_float(v[2 * e + 1]));
+                        w16[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    __nv_bfloat16* dst = p.d + (size_t)row * p.N + col;
+                    if (col + 32 <= p.N && (p.N % 8) == 0) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            d4[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+                    } else {
+                        for (int e = 0; e < 32 && col + e < p.N; ++e) {
+                            const uint32_t wv = w16[e >> 1];
+                            const unsigned short hv = (e & 1) ? (unsigned short)(wv >> 16) : (unsigned short)(wv & 0xffffu);
+                            dst[e] = __ushort_as_bfloat16(hv);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tempty[acc]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
+// W (K x N, row-major) -> Wt (N x K, row-major), 32 x 32 tiles through
+// shared memory; the GEMM reads its B operand K-major.
+template <typename T>
+__global__ void __launch_bounds__(256) transpose_kernel(const T* __restrict__ w, T* __restrict__ wt, int K, int N) {
+    __shared__ T tile[32][33];
+    const int k0 = blockIdx.y * 32, n0 = blockIdx.x * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    for (int r = ty; r < 32; r += 8) {
+        const int k = k0 + r, n = n0 + tx;
+        if (k < K && n < N) tile[r][tx] = w[(size_t)k * N + n];
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int n = n0 + r, k = k0 + tx;
+        if (n < N && k < K) wt[(size_t)n * K + k] = tile[tx][r];
+    }
+}
+
+// float32 projections on the FP32 pipes (the bfloat16 path above is the
+// tensor-core one): D = A W with W (K x N) row-major, 64 x 64 tiles, 4 x 4
+// results per thread.
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ a, const float* __restrict__ w,
+                                                      float* __restrict__ d, int M, int N, int K) {
+    __shared__ float As[16][64 + 4];
+    __shared__ float Ws[16][64];
+    const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+            const int kk = i & 15, mm = i >> 4;  // A tile, transposed into As[k][m]
+            const int m = m0 + mm, k = k0 + kk;
+            As[kk][mm] = (m < M && k < K) ? a[(size_t)m * K + k] : 0.f;
+            const int nn = i & 63, kw = i >> 6;
+            const int n = n0 + nn, kq = k0 + kw;
+            Ws[kw][nn] = (n < N && kq < K) ? w[(size_t)kq * N + n] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float av[4], wv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) wv[j] = Ws[kk][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + ty * 4 + i;
+        if (m >= M) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tx * 4 + j;
+            if (n < N) d[(size_t)m * N + n] = acc[i][j];
+        }
+    }
+}
+
+}  // namespace tcgemm
+}  // namespace vrwkv

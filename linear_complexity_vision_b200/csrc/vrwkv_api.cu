@@ -15,15 +15,16 @@
 #include <vector>
 
 #include <cuda.h>
-#include <cublasLt.h>
 
 #include "vrwkv.h"
 #include "biwkv.cuh"
 #include "biwkv_tma.cuh"
+#include "biwkv_wide.cuh"
 #include "qshift.cuh"
 #include "channel_mix.cuh"
 #include "biwkv_bwd.cuh"
 #include "layer_norm.cuh"
+#include "gemm_tc.cuh"
 
 // Device error word: set by kernels whose bounded waits ran out (bit 0).
 __device__ unsigned int g_vrwkv_device_error;
@@ -208,80 +209,81 @@ unsigned char* static_workspace() {
     return addr[dev];
 }
 
-// ---- dense projections (cuBLASLt) --------------------------------------------
-// One cuBLASLt handle per device, created on first use.
-cublasLtHandle_t lt_handle() {
-    static std::mutex mu;
-    static cublasLtHandle_t h[64] = {};
+// ---- dense projections (tcgen05 GEMM for bfloat16, FP32 pipes for float32) ----
+int sm_count() {
+    static int n[64] = {};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!h[dev] && cublasLtCreate(&h[dev]) != CUBLAS_STATUS_SUCCESS) h[dev] = nullptr;
-    return h[dev];
-}
-
-// D (M x N) = X (M x K) * Wt (K x N), all row-major, float32 accumulation.
-// In cuBLASLt's column-major terms: D^T (N x M) = Wt^T (N x K) * X^T (K x M),
-// where each row-major matrix read column-major is its transpose.  The
-// descriptors and the algorithm the heuristic picks are built once per
-// (device, shape, dtype) and kept: they are host-side objects, and rebuilding
-// them for every call costs more host time than the GEMM takes on the GPU.
-struct GemmPlan {
-    cublasLtMatmulDesc_t op = nullptr;
-    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
-    cublasLtMatmulAlgo_t algo;
-    bool ok = false;
-};
-
-const GemmPlan* gemm_plan(cublasLtHandle_t h, int dev, int M, int N, int K, vrwkv_dtype dtype,
-                          size_t ws_bytes) {
-    static std::mutex mu;
-    static std::vector<std::pair<std::array<long long, 6>, GemmPlan*>> cache;
-    const std::array<long long, 6> key = {dev, M, N, K, (long long)dtype, (long long)ws_bytes};
-    std::lock_guard<std::mutex> lock(mu);
-    for (auto& e : cache)
-        if (e.first == key) return e.second->ok ? e.second : nullptr;
-    GemmPlan* g = new GemmPlan();  // kept for the life of the process
-    const cudaDataType_t dt = dtype == VRWKV_F32 ? CUDA_R_32F : CUDA_R_16BF;
-    cublasLtMatmulPreference_t pref = nullptr;
-    cublasLtMatmulHeuristicResult_t res = {};
-    int nres = 0;
-    if (cublasLtMatmulDescCreate(&g->op, CUBLAS_COMPUTE_32F, CUDA_R_32F) == CUBLAS_STATUS_SUCCESS &&
-        cublasLtMatrixLayoutCreate(&g->la, dt, N, K, N) == CUBLAS_STATUS_SUCCESS &&
-        cublasLtMatrixLayoutCreate(&g->lb, dt, K, M, K) == CUBLAS_STATUS_SUCCESS &&
-        cublasLtMatrixLayoutCreate(&g->ld, dt, N, M, N) == CUBLAS_STATUS_SUCCESS &&
-        cublasLtMatmulPreferenceCreate(&pref) == CUBLAS_STATUS_SUCCESS &&
-        cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
-                                             sizeof(ws_bytes)) == CUBLAS_STATUS_SUCCESS &&
-        cublasLtMatmulAlgoGetHeuristic(h, g->op, g->la, g->lb, g->ld, g->ld, pref, 1, &res, &nres) ==
-            CUBLAS_STATUS_SUCCESS &&
-        nres > 0) {
-        g->algo = res.algo;
-        g->ok = true;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!n[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        n[dev] = v;
     }
-    if (pref) cublasLtMatmulPreferenceDestroy(pref);
-    cache.emplace_back(key, g);
-    return g->ok ? g : nullptr;
+    return n[dev];
 }
 
-vrwkv_status gemm_rowmajor(const void* X, const void* Wt, void* D, int M, int N, int K,
-                           vrwkv_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t s) {
-    cublasLtHandle_t h = lt_handle();
-    if (!h) return fail(VRWKV_ERR_CUDA, "cuBLASLt handle could not be created");
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return fail(VRWKV_ERR_CUDA, "cudaGetDevice failed");
-    const GemmPlan* g = gemm_plan(h, dev, M, N, K, dtype, ws_bytes);
-    if (!g) return fail(VRWKV_ERR_UNSUPPORTED, "no cuBLASLt algorithm for a %d x %d x %d GEMM", M, N, K);
-    const float one = 1.0f, zero = 0.0f;
-    if (cublasLtMatmul(h, g->op, &one, Wt, g->la, X, g->lb, &zero, D, g->ld, D, g->ld, &g->algo, ws,
-                       ws_bytes, s) != CUBLAS_STATUS_SUCCESS)
-        return fail(VRWKV_ERR_CUDA, "cuBLASLt matmul failed");
-    return ok();
+// D (M x N) = X (M x K) * W (K x N), all row-major.  bfloat16: W is first
+// transposed into wt (N x K, the K-major B operand) and the product runs on
+// the tensor cores with float32 accumulation; float32: on the FP32 pipes.
+vrwkv_status gemm_project(const void* X, const void* W, void* D, int M, int N, int K, vrwkv_dtype dtype,
+                          void* wt, cudaStream_t s) {
+    if (dtype == VRWKV_F32) {
+        const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64));
+        tcgemm::gemm_f32_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(X), static_cast<const float*>(W),
+                                                     static_cast<float*>(D), M, N, K);
+        return cuda_status(cudaGetLastError(), "gemm_f32_kernel launch");
+    }
+    if (K % 8 != 0) return fail(VRWKV_ERR_UNSUPPORTED, "bfloat16 projections need C %% 8 == 0");
+    {
+        const dim3 grid((unsigned)((N + 31) / 32), (unsigned)((K + 31) / 32));
+        tcgemm::transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(W),
+                                                                      static_cast<__nv_bfloat16*>(wt), K, N);
+        vrwkv_status st = cuda_status(cudaGetLastError(), "transpose_kernel launch");
+        if (st != VRWKV_OK) return st;
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(VRWKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    tcgemm::Params p;
+    const cuuint32_t estr[2] = {1, 1};
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)tcgemm::BK, (cuuint32_t)tcgemm::BM};
+        if (enc(&p.ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return fail(VRWKV_ERR_UNSUPPORTED, "tensor map of the GEMM's A operand could not be encoded");
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)tcgemm::BK, (cuuint32_t)tcgemm::BN};
+        if (enc(&p.mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wt, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return fail(VRWKV_ERR_UNSUPPORTED, "tensor map of the GEMM's B operand could not be encoded");
+    }
+    p.d = static_cast<__nv_bfloat16*>(D);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.err = device_error_word();
+    if (!p.err) return fail(VRWKV_ERR_CUDA, "cannot locate the device error word");
+    const int smem = (int)sizeof(tcgemm::Smem) + 1024;
+    static std::atomic<int> granted{0};
+    cudaError_t e = ensure_smem(tcgemm::gemm_tc_kernel, granted, smem);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    const int tiles = ((M + tcgemm::BM - 1) / tcgemm::BM) * ((N + tcgemm::BN - 1) / tcgemm::BN);
+    const int grid = std::min(tiles, sm_count());
+    tcgemm::gemm_tc_kernel<<<grid, tcgemm::kThreads, smem, s>>>(p);
+    return cuda_status(cudaGetLastError(), "gemm_tc_kernel launch");
 }
 
 // Workspace of vrwkv_spatial_mix_block: six (B, T, C) token buffers and the
-// GEMM workspace, each 256-byte aligned.
-constexpr size_t kGemmWsBytes = 32u << 20;
+// four transposed weight matrices, each 256-byte aligned.
+size_t block_wt_slot(int C, vrwkv_dtype dtype) {
+    return ((size_t)C * C * elem_bytes(dtype) + 255) / 256 * 256;
+}
 size_t block_ws_slot(int B, int T, int C, vrwkv_dtype dtype) {
     return ((size_t)B * T * C * elem_bytes(dtype) + 255) / 256 * 256;
 }
@@ -667,6 +669,213 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     return true;
 }
 
+// ---------------------------------------------------------------------------
+// 16-channel slab path (biwkv_wide_kernel): the default where it qualifies
+// ---------------------------------------------------------------------------
+bool wide_disabled() {
+    const char* e = getenv("VRWKV_DISABLE_WIDE");
+    return e && e[0] == '1';
+}
+
+// Which kernel serves sequences of up to 4096 tokens when both qualify:
+// the 8-channel kernel unless VRWKV_FORWARD=wide.
+bool wide_preferred() {
+    const char* e = getenv("VRWKV_FORWARD");
+    return e && e[0] == 'w';
+}
+
+struct WidePlan {
+    wide::Params p;
+    int layout;
+    bool qs;
+    bool seg;  // segmented columns: clusters meet through the workspace
+    dim3 grid;
+    int smem;
+};
+
+// Workspace of the segmented 16-channel path: 16 bytes of counters, a flag
+// per (column, segment), then a record (three float4) per (column, segment,
+// channel pair); a column is one (batch row, 16-channel slab).
+constexpr int kWideSegTokens = wide::kTc * wide::kClusterMax;  // tokens per segment (one cluster)
+constexpr int kWideSegMax = 8;                                  // segments per column (T <= 32768)
+WsLayout wide_ws_layout(int B, int T, int C) {
+    const size_t cols = (size_t)B * (size_t)(C / wide::kCW);
+    const size_t nseg = (size_t)((T + kWideSegTokens - 1) / kWideSegTokens);
+    WsLayout L;
+    L.flags_off = 16;
+    L.recs_off = (L.flags_off + cols * nseg * sizeof(unsigned int) + 255) / 256 * 256;
+    L.bytes = L.recs_off + cols * nseg * wide::kNP * 3 * sizeof(float4);
+    return L;
+}
+
+// Plan the 16-channel slab kernel; false when the shape does not qualify
+// (the caller then takes another path).
+bool plan_wide(WidePlan& pl, bool gate, const void* r, const void* k, const void* v, const float* w,
+               const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype, const vrwkv_qshift_params* qs,
+               void* ws = nullptr, size_t ws_bytes = 0) {
+    if (tma_disabled() || wide_disabled() || tma_chunk8_forced()) return false;
+    const int es = elem_bytes(dtype);
+    if (C % wide::kCW != 0 || T % wide::kL != 0 || B > 65535 || C / wide::kCW > 65535) return false;
+    // one cluster per column up to 4096 tokens; longer columns split into
+    // segments of one cluster each, which meet through the workspace
+    pl.seg = T > kWideSegTokens;
+    const int ncl = pl.seg ? wide::kClusterMax : (T + wide::kTc - 1) / wide::kTc;
+    const int nseg = pl.seg ? (T + kWideSegTokens - 1) / kWideSegTokens : 1;
+    if (nseg > kWideSegMax) return false;
+    if (pl.seg && (!ws || ws_bytes < wide_ws_layout(B, T, C).bytes)) return false;
+    if ((long long)B * (C / wide::kCW) * nseg > 65535) return false;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    wide::Params& p = pl.p;
+    p = wide::Params{};
+    pl.qs = qs != nullptr;
+    p.qs = pl.qs ? 1 : 0;
+    p.W = pl.qs ? qs->W : T;
+    p.s = pl.qs ? qs->shift_pixel : 0;
+    p.g = pl.qs ? qs_bounds(C, qs->gamma) : no_shift_bounds();
+    p.ng = shifted_groups(qs);
+    p.hv = 0;
+    if (pl.qs && p.s > 0) {
+        if (!bounds_multiple_of(p.g, wide::kCW) || p.W % wide::kL != 0) return false;
+        // horizontal groups need shift 1 (the neighbour is the adjacent
+        // token); vertical groups read a halo of s*W tokens
+        const bool horiz = p.g.b[0] > 0 || p.g.b[1] > p.g.b[0];
+        const bool vert = p.ng > 2 && (p.g.b[2] > p.g.b[1] || p.g.b[3] > p.g.b[2]);
+        if (horiz && p.s != 1) return false;
+        if (vert) {
+            const long long hv = (long long)p.s * p.W / wide::kL;
+            if (hv > wide::kHaloMax) return false;
+            p.hv = (int)hv;
+        }
+    }
+    const void* srcs[3];
+    int nsrc;
+    if (!gate) {
+        pl.layout = wide::kKV;
+        srcs[0] = k;
+        srcs[1] = v;
+        nsrc = 2;
+    } else if (r == k && k == v) {
+        pl.layout = wide::kX;
+        srcs[0] = r;
+        nsrc = 1;
+    } else {
+        pl.layout = wide::kRKV;
+        srcs[0] = r;
+        srcs[1] = k;
+        srcs[2] = v;
+        nsrc = 3;
+    }
+    for (int i = 0; i < nsrc; ++i)
+        if (!aligned(srcs[i], 16)) return false;
+    if (!aligned(out, 16) || ((size_t)C * es) % 16 != 0) return false;
+    const CUtensorMapDataType dt = dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    for (int i = 0; i < nsrc; ++i) {
+        // (C, 16, T/16, B): channel, token within a 16-token chunk, chunk,
+        // batch row; a box of 17 rows per chunk (the 17th outside the view,
+        // zero-filled) spaces the chunks in shared memory
+        const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)wide::kL, (cuuint64_t)(T / wide::kL), (cuuint64_t)B};
+        const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)C * es * wide::kL, (cuuint64_t)T * C * es};
+        const cuuint32_t box[4] = {(cuuint32_t)wide::kCW, (cuuint32_t)wide::kRows, (cuuint32_t)wide::kBoxChunks, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        const CUresult cr = enc(&p.map[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (cr != CUDA_SUCCESS) return false;
+    }
+    p.err = device_error_word();
+    if (!p.err) return false;
+    p.w = w;
+    p.u = u;
+    p.mu[0] = qs ? qs->mu_r : nullptr;
+    p.mu[1] = qs ? qs->mu_k : nullptr;
+    p.mu[2] = qs ? qs->mu_v : nullptr;
+    p.out = static_cast<char*>(out);
+    p.B = B;
+    p.T = T;
+    p.C = C;
+    p.invT = (float)(1.0 / (double)T);
+    p.nchunkT = T / wide::kL;
+    p.ncl = ncl;
+    p.nseg = nseg;
+    p.nslab = C / wide::kCW;
+    p.total = ncl * nseg * B * p.nslab;
+    if (pl.seg) {
+        const WsLayout L = wide_ws_layout(B, T, C);
+        char* base = static_cast<char*>(ws);
+        p.ws_ctl = reinterpret_cast<unsigned int*>(base);
+        p.ws_flag = reinterpret_cast<unsigned int*>(base + L.flags_off);
+        p.ws_rec = reinterpret_cast<float4*>(base + L.recs_off);
+    }
+    // shared memory: scratch, the widest tile (main chunks + halo boxes) per
+    // source, the parked gate factors
+    const int halo4 = pl.qs ? (std::max(p.hv, 1) + wide::kBoxChunks - 1) / wide::kBoxChunks * wide::kBoxChunks : 0;
+    const int tile = (wide::kChunks + halo4) * wide::kRows * wide::kCW * es;
+    const int park = gate ? wide::kTc * wide::kNP * (int)sizeof(float2) : 0;
+    pl.smem = (int)((sizeof(wide::Scratch) + 127) / 128 * 128) + nsrc * tile + park + 128;
+    if (pl.smem > 227 * 1024) return false;
+    pl.grid = pl.seg ? dim3(ncl, (unsigned)(nseg * B * p.nslab), 1) : dim3(ncl, C / wide::kCW, B);
+    return true;
+}
+
+template <typename IO, int LAYOUT, bool QS, bool SEG>
+vrwkv_status launch_wide(const WidePlan& pl, cudaStream_t stream, bool* fell_back) {
+    auto kern = wide::biwkv_wide_kernel<IO, LAYOUT, QS, SEG>;
+    static std::atomic<int> granted{0};
+    cudaError_t e = ensure_smem(kern, granted, pl.smem);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = pl.grid;
+    cfg.blockDim = dim3(wide::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.p.ncl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+    cfg.attrs = attr;
+    cfg.numAttrs = pl.p.ncl > 1 ? 2 : 0;
+    if (pl.p.ncl > 1) {
+        static std::atomic<int> checked[wide::kClusterMax + 1];
+        int v = checked[pl.p.ncl].load();
+        if (v == 0) {
+            int n = 0;
+            cudaError_t oe = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+            v = (oe == cudaSuccess && n > 0) ? 1 : -1;
+            if (oe != cudaSuccess) cudaGetLastError();
+            checked[pl.p.ncl].store(v);
+        }
+        if (v < 0) {
+            *fell_back = true;
+            return VRWKV_OK;
+        }
+    }
+    e = cudaLaunchKernelEx(&cfg, kern, pl.p);
+    if (e != cudaSuccess) return cuda_status(e, "biwkv_wide_kernel launch");
+    g_last_kernel = "biwkv_wide_kernel";
+    return ok();
+}
+
+template <typename IO, bool SEG>
+vrwkv_status dispatch_wide_seg(const WidePlan& pl, cudaStream_t s, bool* fb) {
+    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
+    case wide::kKV * 2 + 0: return launch_wide<IO, wide::kKV, false, SEG>(pl, s, fb);
+    case wide::kKV * 2 + 1: return launch_wide<IO, wide::kKV, true, SEG>(pl, s, fb);
+    case wide::kRKV * 2 + 0: return launch_wide<IO, wide::kRKV, false, SEG>(pl, s, fb);
+    case wide::kRKV * 2 + 1: return launch_wide<IO, wide::kRKV, true, SEG>(pl, s, fb);
+    case wide::kX * 2 + 0: return launch_wide<IO, wide::kX, false, SEG>(pl, s, fb);
+    default: return launch_wide<IO, wide::kX, true, SEG>(pl, s, fb);
+    }
+}
+
+template <typename IO>
+vrwkv_status dispatch_wide(const WidePlan& pl, cudaStream_t s, bool* fb) {
+    return pl.seg ? dispatch_wide_seg<IO, true>(pl, s, fb) : dispatch_wide_seg<IO, false>(pl, s, fb);
+}
+
 vrwkv_status check_qs(const vrwkv_qshift_params* qs, int T, int C) {
     if (qs->mode != VRWKV_QSHIFT_QUAD && qs->mode != VRWKV_QSHIFT_BIDIR)
         return fail(VRWKV_ERR_INVALID_ARG, "qs: unknown mode %d", qs->mode);
@@ -727,6 +936,19 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
         for (const void* t : toks)
             if (overlaps(ws, need, t, nbytes)) return fail(VRWKV_ERR_INVALID_ARG, "workspace overlaps an input");
         if (overlaps(ws, need, out, nbytes)) return fail(VRWKV_ERR_INVALID_ARG, "workspace overlaps the output");
+    }
+    // the 16-channel kernel: one cluster per column up to 4096 tokens; with
+    // a workspace, longer columns in segments that meet through it (shorter
+    // ones keep the 8-channel global-exchange path the workspace names)
+    if (with_ws ? T > kWideSegTokens : (T <= kWideSegTokens && wide_preferred())) {
+        WidePlan wp;
+        if (plan_wide(wp, gate, r, k, v, w, u, out, B, T, C, dtype, qs, with_ws ? ws : nullptr, ws_bytes)) {
+            bool fell_back = false;
+            cudaStream_t ws_ = static_cast<cudaStream_t>(stream);
+            vrwkv_status st = dtype == VRWKV_F32 ? dispatch_wide<float>(wp, ws_, &fell_back)
+                                                 : dispatch_wide<__nv_bfloat16>(wp, ws_, &fell_back);
+            if (!fell_back) return st;
+        }
     }
     if (B <= 65535 && C / vrwkv::fast::kCS <= 65535) {
         FastPlan fp;
@@ -1094,7 +1316,7 @@ vrwkv_status vrwkv_channel_mix(const void* x, void* out, int B, int T, int C, vr
 
 size_t vrwkv_block_workspace_bytes(int B, int T, int C, vrwkv_dtype dtype) {
     if (B <= 0 || T <= 0 || C <= 0 || (dtype != VRWKV_F32 && dtype != VRWKV_BF16)) return 0;
-    return 6 * block_ws_slot(B, T, C, dtype) + kGemmWsBytes;
+    return 6 * block_ws_slot(B, T, C, dtype) + 4 * block_wt_slot(C, dtype);
 }
 
 vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void* w_k, const void* w_v,
@@ -1148,7 +1370,8 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     void* bR = base + 3 * slot;
     void* bK = base + 4 * slot;
     void* bV = base + 5 * slot;
-    void* gws = base + 6 * slot;
+    char* wts_t = base + 6 * slot;  // transposed weights (bfloat16 GEMM operands)
+    const size_t wslot = block_wt_slot(C, dtype);
     void* t0 = sh[0];
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int M = B * T;
@@ -1168,7 +1391,7 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
         }
     }
     for (int i = 0; i < 3; ++i) {
-        vrwkv_status st = gemm_rowmajor(sh[i], wts[i], dst[i], M, C, C, dtype, gws, kGemmWsBytes, s);
+        vrwkv_status st = gemm_project(sh[i], wts[i], dst[i], M, C, C, dtype, wts_t + i * wslot, s);
         if (st != VRWKV_OK) return st;
     }
     // sigma(R) (.) Bi-WKV(K, V) on the projected channels (Q-Shift already
@@ -1176,7 +1399,7 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     vrwkv_status st = vrwkv_spatial_gate(bR, bK, bV, w, u, t0, B, T, C, dtype, nullptr, stream);
     if (st != VRWKV_OK) return st;
     // W_O into the R buffer (dead after the gate), then LayerNorm into out
-    st = gemm_rowmajor(t0, w_o, bR, M, C, C, dtype, gws, kGemmWsBytes, s);
+    st = gemm_project(t0, w_o, bR, M, C, C, dtype, wts_t + 3 * wslot, s);
     if (st != VRWKV_OK) return st;
     LayerNormParams lp;
     lp.x = static_cast<const char*>(bR);
@@ -1226,12 +1449,19 @@ vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k, const void*
                     "B*ceil(C/8) = %lld columns need %zu bytes of exchange state; the static workspace "
                     "holds %zu",
                     (long long)B * ((C + fast::kCS - 1) / fast::kCS), L.bytes, kStaticWsBytes);
+    const WsLayout LW = wide_ws_layout(B, T, C);
+    if (T > kWideSegTokens && LW.bytes > kStaticWsBytes)
+        return fail(VRWKV_ERR_UNSUPPORTED,
+                    "B*C/16*ceil(T/4096) = %lld column segments need %zu bytes of exchange state; the static "
+                    "workspace holds %zu",
+                    (long long)B * (C / wide::kCW) * ((T + kWideSegTokens - 1) / kWideSegTokens), LW.bytes,
+                    kStaticWsBytes);
     unsigned char* ws = static_workspace();
     if (!ws) return fail(VRWKV_ERR_CUDA, "cannot locate the static workspace");
     // counters and flags start at zero for every call (a previous call that
     // stopped on an error may have left them set); the records need no reset
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(ws, 0, L.recs_off, s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, std::max(L.recs_off, LW.recs_off), s);
     if (e != cudaSuccess) return cuda_status(e, "clearing the static workspace");
     return fused_entry(true, r, k, v, w, u, out, B, T, C, dtype, qs, stream, true, ws, kStaticWsBytes);
 }
@@ -1392,9 +1622,8 @@ vrwkv_status vrwkv_spatial_gate_host(const void* r, const void* k, const void* v
 }
 
 size_t vrwkv_fwd_workspace_bytes(int B, int T, int C) {
-    (void)T;
-    if (B <= 0 || C <= 0) return 0;
-    return ws_layout(B, C).bytes;
+    if (B <= 0 || T <= 0 || C <= 0) return 0;
+    return std::max(ws_layout(B, C).bytes, wide_ws_layout(B, T, C).bytes);
 }
 
 vrwkv_status vrwkv_biwkv_fwd_ws(const void* k, const void* v, const float* w, const float* u, void* wkv,

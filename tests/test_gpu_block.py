@@ -51,6 +51,9 @@ def _case(B, H, W, C, dt):
     ("bf16", 1, 16, 32, 128),    # two CTAs per column in the core
     ("f32", 1, 14, 14, 64),
     ("bf16", 8, 64, 64, 1024),   # the full-size 1024^2 grid at C = 1024
+    ("bf16", 1, 10, 10, 320),    # GEMM tiles: M = 100 (one partial row tile), N = K = 320
+                                 # (a partial 64-column tile, five K steps)
+    ("bf16", 3, 4, 4, 8),        # K = 8 inside one zero-filled K step, N = 8 (scalar stores)
 ])
 def test_block_parity(vk, oracle_mod, dt, B, H, W, C):
     x, mats, w, u, mus, g, b = _case(B, H, W, C, dt)

@@ -175,12 +175,14 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     return (got, err) if return_out else err
 
 
-@pytest.fixture(params=["tma", "tma8", "gx", "generic"])
+@pytest.fixture(params=["tma", "wide", "tma8", "gx", "generic"])
 def kernel_path(request, monkeypatch):
-    """Run a test on the TMA fast path (when the shape qualifies; 16-token
-    thread chunks where the cluster geometry allows), on the same path held to
-    8-token chunks, on its workspace variant (global-memory exchange instead
-    of clusters) and with the generic kernel forced."""
+    """Run a test on the default path (the 8-channel TMA kernel with 16-token
+    thread chunks where the shape and cluster geometry allow), on the
+    16-channel slab kernel where the shape qualifies ("wide"), on the
+    8-channel kernel held to 8-token chunks, on its workspace variant
+    (global-memory exchange instead of clusters) and with the generic kernel
+    forced."""
     if request.param == "generic":
         monkeypatch.setenv("VRWKV_DISABLE_TMA", "1")
     else:
@@ -189,6 +191,10 @@ def kernel_path(request, monkeypatch):
         monkeypatch.setenv("VRWKV_TMA_CHUNK", "8")
     else:
         monkeypatch.delenv("VRWKV_TMA_CHUNK", raising=False)
+    if request.param == "wide":
+        monkeypatch.setenv("VRWKV_FORWARD", "wide")
+    else:
+        monkeypatch.delenv("VRWKV_FORWARD", raising=False)
     _GX["on"] = request.param == "gx"
     yield request.param
     _GX["on"] = False
@@ -198,6 +204,78 @@ def kernel_path(request, monkeypatch):
 def test_workload_full_size(vk, oracle_mod, cfg, kernel_path):
     wl = synth.WORKLOADS[cfg]
     run_fused(vk, oracle_mod, wl)
+
+
+@pytest.mark.parametrize("cfg", [4, 5])
+def test_forward_selection_takes_the_16_channel_kernel(vk, oracle_mod, cfg, monkeypatch):
+    monkeypatch.setenv("VRWKV_FORWARD", "wide")
+    wl = synth.WORKLOADS[cfg]
+    run_fused(vk, oracle_mod, wl)
+    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_wide_kernel"
+
+
+# Shapes aimed at the 16-channel slab kernel's geometry: rows of 16 to 64
+# tokens (vertical halo of 1 to 4 chunks), a last CTA holding one chunk, 1 to
+# 8 CTAs per column, copied channels (gamma = 1/8) and the three source
+# layouts; `wide` says whether the shape qualifies for it.
+WIDE_CASES = [
+    # call, B, H, W, C, dtype, gamma, shift, wide
+    ("gate_qs_x", 1, 32, 16, 64, "bf16", 0.25, 1, True),     # W = 16: one chunk per image row
+    ("gate_qs", 2, 33, 16, 64, "f32", 0.25, 1, True),        # T = 528: the second CTA holds one chunk
+    ("qshift_biwkv", 1, 64, 48, 64, "bf16", 0.25, 1, True),  # W = 48: halo of 3 chunks, 6 CTAs
+    ("gate_qs_x", 2, 16, 32, 128, "f32", 0.125, 1, True),    # copied channels 64..127
+    ("gate_qs_x", 1, 64, 64, 64, "bf16", 0.25, 2, False),    # shift 2 on the horizontal groups
+    ("gate_qs", 1, 8, 64, 128, "bf16", 0.25, 1, True),       # one CTA
+    ("biwkv", 3, 1, 2048, 32, "bf16", 0.25, 1, True),        # 4 CTAs, no Q-Shift
+    ("biwkv", 1, 1, 1000, 32, "bf16", 0.25, 1, False),       # T not a multiple of 16
+]
+
+
+@pytest.mark.parametrize("case", WIDE_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_wide_kernel_shapes(vk, oracle_mod, case, monkeypatch):
+    monkeypatch.setenv("VRWKV_FORWARD", "wide")
+    call, B, H, W, C, dt, gamma, shift, wide = case
+    wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000, gamma=gamma, s=shift)
+    run_fused(vk, oracle_mod, wl)
+    got = vk.load_library().vrwkv_last_kernel().decode()
+    assert (got == "biwkv_wide_kernel") == wide, got
+
+
+# Sequences past 4096 tokens: the pages' efficiency comparison runs 2048^2
+# images at patch 16, T = 16384 ("Vision-RWKV Backbone", Ablation /
+# efficiency analysis, Fig. 3(b)).  With a workspace the 16-channel kernel
+# splits a column into segments of one 8-CTA cluster (4096 tokens) that meet
+# through it; checked against the RNN form over every output and eq. 5 at
+# sampled positions.
+LONG_CASES = [
+    # call, B, H, W, C, dtype
+    ("gate_qs_x", 1, 128, 128, 64, "bf16"),   # T = 16384: four segments
+    ("gate_qs", 1, 128, 64, 64, "f32"),       # T = 8192: two segments
+    ("biwkv", 2, 1, 12288, 16, "bf16"),       # T = 12288: three segments, no Q-Shift
+    ("gate_qs_x", 1, 72, 64, 64, "bf16"),     # T = 4608: the last segment holds one CTA's tokens
+    ("qshift_biwkv", 1, 256, 128, 64, "bf16"),  # T = 32768: eight segments
+]
+
+
+@pytest.mark.parametrize("case", LONG_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_long_sequences_with_workspace(vk, oracle_mod, case):
+    call, B, H, W, C, dt = case
+    wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000)
+    _GX["on"] = True
+    try:
+        run_fused(vk, oracle_mod, wl)
+    finally:
+        _GX["on"] = False
+    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_wide_kernel"
+
+
+def test_long_sequence_without_workspace_is_refused(vk):
+    import torch
+    x = torch.zeros(1, 16384, 64, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(64, device="cuda")
+    with pytest.raises(vk.VrwkvError) as ei:
+        vk.spatial_gate(x, x, x, w, w)
+    assert ei.value.status == 2  # VRWKV_ERR_UNSUPPORTED
 
 
 def test_workload2_qshift_of_x_full_size(vk, oracle_mod):
@@ -358,7 +436,7 @@ def test_invalid_arguments_raise(vk):
         vk.biwkv_fwd(x, x, w, w, out=x)
 
 
-def test_workspace_reuse_across_launches(vk, oracle_mod):
+def test_workspace_reuse_across_launches(vk, oracle_mod, monkeypatch):
     # the global-exchange kernel resets its counters and advances a
     # generation at the end of every launch: back-to-back launches on one
     # workspace (different shapes, then the same one again) stay exact
@@ -374,7 +452,9 @@ def test_workspace_reuse_across_launches(vk, oracle_mod):
         mus = [vec_f32(inp[n])[0] for n in ("mu_r", "mu_k", "mu_v")]
         qs = vk.QShift(H, W, 1, 0.25, *mus)
         a = vk.spatial_gate(x, x, x, w, u, qs=qs, workspace=ws)
-        b = vk.spatial_gate(x, x, x, w, u, qs=qs)  # cluster exchange
+        monkeypatch.setenv("VRWKV_DISABLE_WIDE", "1")
+        b = vk.spatial_gate(x, x, x, w, u, qs=qs)  # the same kernel's cluster exchange
+        monkeypatch.delenv("VRWKV_DISABLE_WIDE")
         vk.device_status()
         assert torch.equal(a, b)
         outs.append(a)

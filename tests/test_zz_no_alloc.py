@@ -1,13 +1,15 @@
 """vrwkv_spatial_gate_static: the fused forward on the library's fixed
 workspace (for callers that cannot allocate device memory).  Collected last
-on purpose: it must give the same bits as vrwkv_spatial_gate on two calls in
-a row whether it runs alone or after every other test has used the library
-(and the workspace kernels) on this device."""
+on purpose: on two calls in a row, whether it runs alone or after every
+other test has used the library (and the workspace kernels) on this device,
+it must give the same bits as vrwkv_spatial_gate_ws with a caller's
+workspace (the same kernels, the exchange state in another array) and agree
+within the parity tolerance with vrwkv_spatial_gate."""
 import numpy as np
 import pytest
 
 from linear_complexity_vision_b200 import synth
-from helpers import to_device, vec_f32
+from helpers import TOL, scaled_error, to_device, vec_f32
 
 pytestmark = pytest.mark.gpu
 
@@ -27,22 +29,45 @@ def _inputs(B, H, W, C, dt, seed):
     w = synth.draw(seed, "w", (C,), ("uniform", -5.0, 5.0))
     u = synth.draw(seed, "u", (C,), ("normal", 1.0))
     mus = [synth.draw(seed, n, (C,), ("uniform", 0.0, 1.0)) for n in ("mu_r", "mu_k", "mu_v")]
-    return (to_device(x, dt)[0], vec_f32(w)[0], vec_f32(u)[0], [vec_f32(m)[0] for m in mus])
+    xt, xd = to_device(x, dt)
+    dev = [vec_f32(a) for a in (w, u, *mus)]
+    return xt, xd, [d[0] for d in dev], [d[1] for d in dev]
 
 
 @pytest.mark.parametrize("dt,B,H,W,C", [
-    ("bf16", 2, 64, 64, 64),    # 16 CTAs per column: the exchange runs in the static workspace
-    ("f32", 1, 40, 40, 64),     # 10 CTAs per column
+    ("bf16", 2, 64, 64, 64),    # 8 CTAs of 512 tokens per column: the exchange runs in the static workspace
+    ("f32", 1, 40, 40, 64),     # 8-token chunks, 8 rows of 40 per CTA: 5 CTAs per column
+    ("bf16", 1, 128, 64, 64),   # 16 CTAs per column: every flag and record slot of a column
     ("bf16", 8, 64, 64, 1024),  # 1024 columns: the full-size workload
     ("bf16", 2, 14, 14, 96),    # one CTA per column: no exchange
 ])
-def test_static_matches_spatial_gate_twice(vk, dt, B, H, W, C):
+def test_static_matches_spatial_gate_twice(vk, oracle_mod, dt, B, H, W, C):
     import torch
-    x, w, u, mus = _inputs(B, H, W, C, dt, seed=777 + C)
+    x, xd, (w, u, *mus), (wd, ud, *musd) = _inputs(B, H, W, C, dt, seed=777 + C)
     qs = vk.QShift(H, W, 1, 0.25, *mus)
-    want = vk.spatial_gate(x, x, x, w, u, qs=qs)
+    want_default = vk.spatial_gate(x, x, x, w, u, qs=qs)
+    want = vk.spatial_gate(x, x, x, w, u, qs=qs, workspace=vk.fwd_workspace(B, H * W, C))
+    r, k, v = (oracle_mod.qshift(xd, H, W, 1, 0.25, m) for m in musd)
+    scale = oracle_mod.gate(r, oracle_mod.biwkv_rnn(k, np.abs(v), wd, ud))
     for _ in range(2):  # two calls in a row on the same workspace
-        got = vk.spatial_gate_static(x, x, x, w, u, qs=qs)
+        got = vk.spatial_gate_static(x, x, x, w, u, qs=qs, out=torch.empty_like(x))
+        vk.device_status()
+        assert torch.equal(got, want)
+        err = scaled_error(got.double().cpu().numpy(), want_default.double().cpu().numpy(), scale)
+        assert err <= TOL[dt], err
+
+
+def test_static_long_sequence_matches_workspace_call(vk):
+    # T = 16384 (a 2048^2 image at patch 16): the 16-channel kernel's
+    # segments meet through the static array as they do through a caller's
+    # workspace
+    import torch
+    B, H, W, C = 1, 128, 128, 64
+    x, _, (w, u, *mus), _ = _inputs(B, H, W, C, "bf16", seed=4242)
+    qs = vk.QShift(H, W, 1, 0.25, *mus)
+    want = vk.spatial_gate(x, x, x, w, u, qs=qs, workspace=vk.fwd_workspace(B, H * W, C))
+    for _ in range(2):
+        got = vk.spatial_gate_static(x, x, x, w, u, qs=qs, out=torch.empty_like(x))
         vk.device_status()
         assert torch.equal(got, want)
 
