@@ -124,8 +124,11 @@ struct alignas(16) Scratch {
     int tk;                      // SEG: this cluster's ticket
     unsigned int gen;            // SEG: the launch's generation
     int mkey[kCW];               // CTA maximum of k per channel (ordered-int encoding)
-    float4 aggF[kChunks][kNP];   // chunk forward totals, then forward carries into each chunk
-    float4 aggG[kChunks][kNP];   // chunk backward totals, then backward carries
+    // chunk forward / backward totals, then the carries into each chunk; one
+    // float4 of row padding: the scan warps read down a column (32 chunks of
+    // one pair), which without it would hit the same four banks
+    float4 aggF[kChunks][kNP + 1];
+    float4 aggG[kChunks][kNP + 1];
     Rec own[kNP];                // this CTA's record
     Rec mb[kClusterMax][kNP];    // mailbox: every peer's record (own included)
     unsigned long long bar;      // TMA completion barrier
@@ -174,6 +177,12 @@ __device__ __forceinline__ void st2<float>(char* p, float2 v) {
 }
 
 __device__ __forceinline__ float4 f4(float2 a, float2 b) { return make_float4(a.x, a.y, b.x, b.y); }
+// three-input maximum (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 __device__ __forceinline__ float4 fma4(float2 m, float4 x, float4 y) {
     return f4(fma2(m, fast::lo2(x), fast::lo2(y)), fma2(m, fast::hi2(x), fast::hi2(y)));
 }
@@ -190,7 +199,7 @@ __device__ __forceinline__ float4 shfl_idx4(float4 v, int src) {
 template <typename IO, int LAYOUT, bool QS, int MODE>
 __device__ __forceinline__ void load_chunk(const char* const* tb, int hoff, bool left_ok, bool right_ok,
                                            float2 muk, float2 muv, float2 mur, float2* park, int park_stride,
-                                           float2 (&kk)[kL], float2 (&vv)[kL], bool valid) {
+                                           float2 (&kk)[kL], float2 (&vv)[kL]) {
     constexpr int es = Io<IO>::kBytes;
     constexpr int RB = kCW * es;  // bytes per token row
     constexpr int CB = kRows * RB;
@@ -241,8 +250,8 @@ __device__ __forceinline__ void load_chunk(const char* const* tb, int hoff, bool
             r = cur[SR];
         }
         if (GATE) park[i * park_stride] = ex2(mul2(r, f2(-kLog2e)));
-        kk[i] = valid ? k : f2(-INFINITY);
-        vv[i] = valid ? v : f2(0.0f);
+        kk[i] = k;
+        vv[i] = v;
         // advance the sliding neighbours
 #pragma unroll
         for (int s = 0; s < NSRC; ++s) {
@@ -418,23 +427,29 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_wide_kernel(const __grid_co
     float2 kk[kL], vv[kL];
     switch (mode) {
     case kFromLeft:
-        load_chunk<IO, LAYOUT, QS, kFromLeft>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv, valid);
+        load_chunk<IO, LAYOUT, QS, kFromLeft>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv);
         break;
     case kFromRight:
-        load_chunk<IO, LAYOUT, QS, kFromRight>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv, valid);
+        load_chunk<IO, LAYOUT, QS, kFromRight>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv);
         break;
     case kFromUp:
     case kFromDown:
-        load_chunk<IO, LAYOUT, QS, kFromUp>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv, valid);
+        load_chunk<IO, LAYOUT, QS, kFromUp>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv);
         break;
     default:
-        load_chunk<IO, LAYOUT, QS, kSelf>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv, valid);
+        load_chunk<IO, LAYOUT, QS, kSelf>(tb, hoff, left_ok, right_ok, muk, muv, mur, mypark, park_stride, kk, vv);
         break;
     }
-    // CTA maximum of k per channel: warp lanes of one pair, then one atomic
-    float2 mx = kk[0];
+    // CTA maximum of k per channel: warp lanes of one pair, then one atomic.
+    // A chunk past T (zero-filled by the TMA) takes no part in the maximum,
+    // and its p and p v are zeroed below.
+    float2 mx = f2(-INFINITY);
 #pragma unroll
-    for (int i = 1; i < kL; ++i) mx = max2(mx, kk[i]);
+    for (int i = 0; i < kL; i += 2) {
+        mx.x = fmax3(mx.x, kk[i].x, kk[i + 1].x);
+        mx.y = fmax3(mx.y, kk[i].y, kk[i + 1].y);
+    }
+    if (!valid) mx = f2(-INFINITY);
 #pragma unroll
     for (int d = 8; d < 32; d <<= 1) {
         mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
@@ -449,8 +464,10 @@ __global__ void __launch_bounds__(kThreads, 2) biwkv_wide_kernel(const __grid_co
     // ---- 3. p, p v (in place) and sub-chunk totals --------------------------
     const float2 Mcta = make_float2(fkey_inv(S.mkey[2 * j]), fkey_inv(S.mkey[2 * j + 1]));
     // a CTA whose tokens all lie past T has M = -inf: reference 0 (p = 0 there)
-    const float2 negM = make_float2(Mcta.x == -INFINITY ? 0.0f : -Mcta.x * kLog2e,
-                                    Mcta.y == -INFINITY ? 0.0f : -Mcta.y * kLog2e);
+    // a chunk past T gets p = 2^-inf = 0 (its k are the zero fill)
+    const float2 negM = !valid ? f2(-INFINITY)
+                               : make_float2(Mcta.x == -INFINITY ? 0.0f : -Mcta.x * kLog2e,
+                                             Mcta.y == -INFINITY ? 0.0f : -Mcta.y * kLog2e);
     const float2 alpha = S.alpha[j], a8 = S.a8[j];
     float4 Fs[2], Gs[2];  // per sub-chunk: forward and backward totals (num.xy, den.xy)
 #pragma unroll

@@ -304,6 +304,240 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                      : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// The same product on CTA pairs (cta_group::2): a cluster of two CTAs on two
+// SMs computes a 256 x 256 output tile.  CTA r of the pair loads rows
+// 128 r .. of the A tile and rows 128 r .. of the Bt tile (128 x 64 each,
+// 32 KB per stage instead of 48: a 6-stage ring fits), and both copies
+// complete on the leader's "full" barrier; the leader issues tcgen05.mma
+// cta_group::2 (M = 256, N = 256, K = 16), which reads A and B from both
+// CTAs' shared memory and accumulates each CTA's 128 rows in its own tensor
+// memory; tcgen05.commit with a CTA mask frees the stage (and later hands
+// the accumulator to the epilogue) in both CTAs.  No load is multicast:
+// each CTA fetches only its own halves.
+// ---------------------------------------------------------------------------
+namespace pair {
+
+constexpr int BM = 256, BN = 256, BK = 64;   // per cluster
+constexpr int kHalf = 128;                   // rows of A and of Bt per CTA
+constexpr int kStages = 6;
+constexpr int A_BYTES = kHalf * BK * 2;      // 16 KB
+constexpr int B_BYTES = kHalf * BK * 2;      // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+
+struct alignas(1024) Smem {
+    uint8_t a[kStages][A_BYTES];
+    uint8_t b[kStages][B_BYTES];
+    unsigned long long full[kStages], empty[kStages];
+    unsigned long long tfull[kAcc], tempty[kAcc];
+    unsigned long long drain;
+    unsigned tmem_base;
+    int abort;
+};
+
+// kind::f16, float32 accumulator, bfloat16 A and B, both K-major, N = 256,
+// M = 256 (the pair).
+constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                             ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory that completes on the leader's
+// barrier (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int c0, int c1,
+                                                 uint32_t leader_bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(fast::smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(leader_bar)
+        : "memory");
+}
+__device__ __forceinline__ void commit_pair(unsigned long long* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            fast::smem_u32(bar)),
+        "h"((unsigned short)0x3)
+        : "memory");
+}
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(1024) char smem_raw[];
+    Smem& S = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (fast::smem_u32(smem_raw) & 1023u)) & 1023u));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int nt = (p.N + BN - 1) / BN, mt = (p.M + BM - 1) / BM;
+    const int ntiles = nt * mt, nk = (p.K + BK - 1) / BK;
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    volatile int* abort = &S.abort;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            fast::mbar_init(&S.full[s], 1);
+            fast::mbar_init(&S.empty[s], 1);
+        }
+        for (int a = 0; a < kAcc; ++a) {
+            fast::mbar_init(&S.tfull[a], 1);
+            fast::mbar_init(&S.tempty[a], 8);  // the epilogue warps of both CTAs
+        }
+        fast::mbar_init(&S.drain, 1);
+        S.abort = 0;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         fast::smem_u32(&S.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers exist before any remote signal
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer: this CTA's halves of A and Bt, completing on the leader's barrier
+            int it = 0;
+            int last_par[kStages];
+            for (int s = 0; s < kStages; ++s) last_par[s] = -1;
+            for (int t = cid; t < ntiles && !*abort; t += ncl) {
+                const int m0 = (t / nt) * BM + (int)rank * kHalf, n0 = (t % nt) * BN + (int)rank * kHalf;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const unsigned ph = (it / kStages) & 1;
+                    if (!wait_phase(&S.empty[s], ph ^ 1u, abort, p.err)) break;
+                    const uint32_t lbar = fast::mapa_u32(fast::smem_u32(&S.full[s]), 0);
+                    if (leader) fast::mbar_expect_tx(&S.full[s], 2 * STAGE_BYTES);
+                    tma_load_2d_pair(S.a[s], &p.ma, kb * BK, m0, lbar);
+                    tma_load_2d_pair(S.b[s], &p.mb, kb * BK, n0, lbar);
+                    last_par[s] = (int)ph;
+                }
+            }
+            if (*abort && leader) {
+                for (int s = 0; s < kStages; ++s) {
+                    if (last_par[s] < 0) continue;
+                    const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+                    while (!mbar_test(&S.full[s], (unsigned)last_par[s]) && fast::global_ns() - t0 <= lim) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // MMA issuer (the pair's leader)
+            int it = 0, lt = 0;
+            bool issued = false;
+            for (int t = cid; t < ntiles && !*abort; t += ncl, ++lt) {
+                const int acc = lt & 1;
+                const unsigned aph = (lt >> 1) & 1;
+                if (!wait_phase(&S.tempty[acc], aph ^ 1u, abort, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const unsigned ph = (it / kStages) & 1;
+                    if (!wait_phase(&S.full[s], ph, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(fast::smem_u32(S.a[s]));
+                    const uint64_t bd = sw128_desc(fast::smem_u32(S.b[s]));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_pair(d_tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), (kb > 0 || k > 0) ? 1u : 0u);
+                    issued = true;
+                    commit_pair(&S.empty[s]);
+                }
+                if (!ok) break;
+                commit_pair(&S.tfull[acc]);
+            }
+            if (*abort && issued) {
+                tc_commit(&S.drain);
+                const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+                while (!mbar_test(&S.drain, 0) && fast::global_ns() - t0 <= lim) {
+                }
+            }
+        }
+    } else {
+        // epilogue: this CTA's 128 rows of the pair's tile
+        const int quad = warp & 3;
+        const uint32_t leader_tempty[2] = {fast::mapa_u32(fast::smem_u32(&S.tempty[0]), 0),
+                                           fast::mapa_u32(fast::smem_u32(&S.tempty[1]), 0)};
+        int lt = 0;
+        for (int t = cid; t < ntiles; t += ncl, ++lt) {
+            const int acc = lt & 1;
+            const unsigned aph = (lt >> 1) & 1;
+            if (!wait_phase(&S.tfull[acc], aph, abort, p.err)) break;
+            tc_fence_after();
+            const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
+            const int row = m0 + (int)rank * kHalf + quad * 32 + lane;
+            const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tbase + (uint32_t)(c * 32), v);
+                const int col = n0 + c * 32;
+                if (row < p.M && col < p.N) {
+                    uint32_t w16[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]),
+                                                                       __uint_as_float(v[2 * e + 1]));
+                        w16[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    __nv_bfloat16* dst = p.d + (size_t)row * p.N + col;
+                    if (col + 32 <= p.N && (p.N % 8) == 0) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            d4[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+                    } else {
+                        for (int e = 0; e < 32 && col + e < p.N; ++e) {
+                            const uint32_t wv = w16[e >> 1];
+                            const unsigned short hv = (e & 1) ? (unsigned short)(wv >> 16) : (unsigned short)(wv & 0xffffu);
+                            dst[e] = __ushort_as_bfloat16(hv);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_remote(leader_tempty[acc]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its pair may still signal it
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
+}  // namespace pair
+
 // W (K x N, row-major) -> Wt (N x K, row-major), 32 x 32 tiles through
 // shared memory; the GEMM reads its B operand K-major.
 template <typename T>

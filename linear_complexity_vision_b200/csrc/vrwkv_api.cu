@@ -210,6 +210,12 @@ unsigned char* static_workspace() {
 }
 
 // ---- dense projections (tcgen05 GEMM for bfloat16, FP32 pipes for float32) ----
+// VRWKV_GEMM_1CTA=1 keeps the projections on single-CTA tiles (diagnostics).
+bool gemm_single_cta_forced() {
+    const char* e = getenv("VRWKV_GEMM_1CTA");
+    return e && e[0] == '1';
+}
+
 int sm_count() {
     static int n[64] = {};
     int dev = 0;
@@ -269,6 +275,29 @@ vrwkv_status gemm_project(const void* X, const void* W, void* D, int M, int N, i
     p.K = K;
     p.err = device_error_word();
     if (!p.err) return fail(VRWKV_ERR_CUDA, "cannot locate the device error word");
+    if (!gemm_single_cta_forced()) {
+        // CTA pairs (cta_group::2): the B map's box holds one CTA's 128 rows
+        tcgemm::Params p2 = p;
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)tcgemm::BK, (cuuint32_t)tcgemm::pair::kHalf};
+        if (enc(&p2.mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wt, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS) {
+            const int smem2 = (int)sizeof(tcgemm::pair::Smem) + 1024;
+            static std::atomic<int> granted2{0};
+            cudaError_t e2 = ensure_smem(tcgemm::pair::gemm_tc2_kernel, granted2, smem2);
+            if (e2 == cudaSuccess) {
+                const int tiles2 = ((M + tcgemm::pair::BM - 1) / tcgemm::pair::BM) *
+                                   ((N + tcgemm::pair::BN - 1) / tcgemm::pair::BN);
+                const int pairs = std::max(1, std::min(tiles2, sm_count() / 2));
+                tcgemm::pair::gemm_tc2_kernel<<<2 * pairs, tcgemm::kThreads, smem2, s>>>(p2);
+                e2 = cudaGetLastError();
+                if (e2 == cudaSuccess) return ok();
+            }
+            cudaGetLastError();  // fall back to single CTAs
+        }
+    }
     const int smem = (int)sizeof(tcgemm::Smem) + 1024;
     static std::atomic<int> granted{0};
     cudaError_t e = ensure_smem(tcgemm::gemm_tc_kernel, granted, smem);

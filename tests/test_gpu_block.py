@@ -46,6 +46,17 @@ def _case(B, H, W, C, dt):
     return x, mats, w, u, mus, g, b
 
 
+@pytest.fixture(params=["pair", "single"])
+def gemm_path(request, monkeypatch):
+    """The projections on CTA pairs (cta_group::2, the default) or on single
+    CTAs (VRWKV_GEMM_1CTA=1)."""
+    if request.param == "single":
+        monkeypatch.setenv("VRWKV_GEMM_1CTA", "1")
+    else:
+        monkeypatch.delenv("VRWKV_GEMM_1CTA", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("dt,B,H,W,C", [
     ("bf16", 2, 14, 14, 64),     # the 224^2 grid
     ("bf16", 1, 16, 32, 128),    # two CTAs per column in the core
@@ -55,7 +66,7 @@ def _case(B, H, W, C, dt):
                                  # (a partial 64-column tile, five K steps)
     ("bf16", 3, 4, 4, 8),        # K = 8 inside one zero-filled K step, N = 8 (scalar stores)
 ])
-def test_block_parity(vk, oracle_mod, dt, B, H, W, C):
+def test_block_parity(vk, oracle_mod, dt, B, H, W, C, gemm_path):
     x, mats, w, u, mus, g, b = _case(B, H, W, C, dt)
     xt, xd = to_device(x, dt)
     mt, md = zip(*[to_device(m, dt) for m in mats])
