@@ -72,7 +72,7 @@ KERNEL_SOURCES = {
     "biwkv_wide_kernel": ("common.cuh", "biwkv_tma.cuh", "biwkv_wide.cuh"),
     "biwkv_fused_kernel": ("common.cuh", "qshift.cuh", "biwkv.cuh"),
     "channel_mix_vec_kernel": ("common.cuh", "qshift.cuh", "channel_mix.cuh"),
-    "biwkv_bwd_kernel": ("common.cuh", "biwkv_bwd.cuh"),
+    "biwkv_bwd_kernel": ("common.cuh", "biwkv_tma.cuh", "biwkv_bwd.cuh"),
 }
 
 
@@ -230,9 +230,13 @@ def committed_record(key: str, kernel: str):
     try:
         with open(p) as f:
             rec = json.load(f)
-        ent = rec.get(key)
-        if ent and ent.get("kernel") == kernel and ent.get("kernel_sha") == kernel_source_hash(kernel):
-            return ent
+        # the workload's record, or one kept for another kernel of the same
+        # workload (e.g. "wide/<workload>")
+        for k, ent in rec.items():
+            if not isinstance(ent, dict) or not (k == key or k.endswith("/" + key)):
+                continue
+            if ent.get("kernel") == kernel and ent.get("kernel_sha") == kernel_source_hash(kernel):
+                return ent
     except Exception:
         pass
     return None
@@ -513,7 +517,9 @@ def time_block(runner, stream, torch, dev, launches: int):
     return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "peak_source": kind, "kernel": "spatial_mix_block",
             "flops_per_launch": flops, "avg_launch_us": us, "launches": launches,
-            "gemm": "library tcgen05 kernel (gemm_tc_kernel), bf16, float32 accumulation in tensor memory",
+            "gemm": ("hand-written tcgen05 kernel, bf16 operands, float32 accumulation in tensor memory: "
+                     + ("gemm_tc_kernel (one CTA per 128x256 tile)" if os.environ.get("VRWKV_GEMM_1CTA") == "1"
+                        else "gemm_tc2_kernel (CTA pairs, cta_group::2, 256x256 tiles)")),
             "timing": "CUDA graphs over the rotating buffer sets"}
 
 
