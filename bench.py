@@ -69,6 +69,7 @@ CSRC = os.path.join(ROOT, "linear_complexity_vision_b200", "csrc")
 # they are unchanged (a change of launch shape comes with a new capture).
 KERNEL_SOURCES = {
     "biwkv_tma_kernel": ("common.cuh", "biwkv_tma.cuh"),
+    "biwkv_tm_kernel": ("common.cuh", "biwkv_tma.cuh", "biwkv_tm.cuh"),
     "biwkv_wide_kernel": ("common.cuh", "biwkv_tma.cuh", "biwkv_wide.cuh"),
     "biwkv_fused_kernel": ("common.cuh", "qshift.cuh", "biwkv.cuh"),
     "channel_mix_vec_kernel": ("common.cuh", "qshift.cuh", "channel_mix.cuh"),

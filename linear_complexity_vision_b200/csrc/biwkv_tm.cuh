@@ -1,0 +1,578 @@
+// Fused Q-Shift -> Bi-WKV -> sigma(R) gate with 32-token thread chunks whose
+// per-token partial sums live in tensor memory (sm_100a).
+//
+// Evaluates Bi-WKV of "Vision-RWKV Backbone", Linear Complexity
+// Bidirectional Attention, eq. 5, on inputs Q-Shifted per Quad-Directional
+// Token Shift, eq. 9, gated per Overall Architecture, eq. 2 -- the same
+// chunked two-sided scan as the 8-channel TMA kernel (biwkv_tma.cuh):
+//
+//   A_t = sum_{i<t} a^{t-1-i} p_i v_i,  B_t = sum_{i>t} a^{i-t-1} p_i v_i,
+//   C_t, D_t with v = 1,  a = e^{-w/T},  p_i = e^{k_i - M},
+//   wkv_t = (A_t + B_t + e^u p_t v_t) / (C_t + D_t + e^u p_t).
+//
+// What changes against that kernel: a thread owns a channel pair and 32
+// tokens (four sub-chunks of 8) instead of 16, so the fixed per-thread cost
+// of the warp, CTA and cluster scans, the exchange and the set-up is spread
+// over twice the tokens.  The 128 per-token partial sums a thread carries
+// from the local pass to the output pass (numerator and denominator of 32
+// tokens x 2 channels) do not fit next to the scan state in registers; they
+// go to the thread's own lane of tensor memory (tcgen05.st, 32 columns per
+// sub-chunk) and come back one sub-chunk at a time (tcgen05.ld).  A CTA holds
+// 128 columns, so four CTAs fill an SM's 512; the host keeps at most four
+// resident (a shared-memory floor) so an allocation never waits.
+//
+// The gate factor e^{-r} of a token is parked in the two tile slots the
+// thread has just read to make r (r's own and shifted r's; without Q-Shift,
+// r's slot and one extra tile), so no shared-memory array of gate factors
+// is needed; the result later goes into the first slot.  Every slot is read
+// and written by the one thread that owns the token.
+//
+// A CTA covers 1024 tokens x 8 channels; longer columns use a cluster of up
+// to 8 CTAs along T (T <= 8192) exchanging their aggregates through
+// asynchronous shared-memory stores, as in the 8-channel kernel.
+#pragma once
+
+#include "biwkv_tma.cuh"
+
+namespace vrwkv {
+namespace tm32 {
+
+using fast::kCS;
+using fast::kKV;
+using fast::kL;
+using fast::kNP;
+using fast::kRKV;
+using fast::kX;
+using fast::bulk_commit_and_wait_read;
+using fast::cluster_arrive_relaxed;
+using fast::cluster_wait_acquire;
+using fast::fence_proxy_async_smem;
+using fast::fma4;
+using fast::hi2;
+using fast::lds_pair;
+using fast::lo2;
+using fast::mapa_u32;
+using fast::mbar_expect_tx;
+using fast::mbar_init;
+using fast::mbar_wait_bounded;
+using fast::mbar_wait_cluster_bounded;
+using fast::shfl_down4;
+using fast::shfl_up4;
+using fast::smem_u32;
+using fast::st_async2;
+using fast::st_async4;
+using fast::tma_load_3d;
+using fast::tma_load_4d;
+using fast::tma_store_3d;
+using fast::zero4;
+
+constexpr int kThreads = 128;              // 4 channel pairs x 32 chunks
+constexpr int kKL = 32;                    // tokens per thread chunk
+constexpr int kH = kKL / kL;               // sub-chunks of 8 per chunk
+constexpr int kNW = kThreads / 32;         // warps
+constexpr int kCPW = 32 / kNP;             // chunks per warp
+constexpr int kTc = kThreads / kNP * kKL;  // tokens per CTA (1024)
+constexpr int kChunks = kTc / kKL;         // chunks per CTA
+constexpr int kWarpTok = kCPW * kKL;       // tokens per warp (256)
+constexpr int kClusterMax = 8;             // CTAs per column: T <= 8192
+constexpr int kTmemCols = kH * 32;         // num, den of 32 tokens x 2 channels
+// Dynamic shared memory of at least this many bytes keeps five CTAs from
+// fitting on an SM (228 KB, 1 KB reserved per CTA): at most four CTAs hold
+// tensor memory at once, 4 x 128 = 512 columns.
+constexpr int kSmemFloor = 46 * 1024;
+
+struct alignas(16) Scratch {
+    float2 tab[kChunks][kNP];  // a^(32 m) per channel pair
+    float2 wmax[kNP][kNW + 1];
+    float2 wsc[kNP][kNW + 1];
+    float4 waggF[kNP][kNW + 1];
+    float4 waggB[kNP][kNW + 1];
+    float4 wcarF[kNP][kNW + 1];
+    float4 wcarB[kNP][kNW + 1];
+    float2 mbM[kClusterMax][kNP + 1];
+    float4 mbF[kClusterMax][kNP + 1];
+    float4 mbG[kClusterMax][kNP + 1];
+    float4 ownF[kNP];
+    float4 ownG[kNP];
+    float2 ownM[kNP];
+    float4 cscale[kCS];
+    float4 ccarry[kCS];
+    unsigned long long bar;
+    unsigned long long xbar;
+    unsigned int tmem;  // base address of this CTA's tensor-memory columns
+};
+
+// 32 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+        "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+        "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+        "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+        : "memory");
+}
+// Load and wait in one statement, so no use of the registers can be
+// scheduled before the data has arrived.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+          "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]),
+          "=f"(v[15]), "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]), "=f"(v[20]), "=f"(v[21]),
+          "=f"(v[22]), "=f"(v[23]), "=f"(v[24]), "=f"(v[25]), "=f"(v[26]), "=f"(v[27]), "=f"(v[28]),
+          "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+// A gate factor's store into a slot depends on the values read from that
+// slot (they make r), and a result's store on the gate factor read from its
+// slot: data dependence alone orders each slot's accesses.
+__device__ __forceinline__ void sts_f32(char* p, float v) { *reinterpret_cast<float*>(p) = v; }
+__device__ __forceinline__ float lds_f32(const char* p) { return *reinterpret_cast<const float*>(p); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+template <typename IO, int LAYOUT, bool QS>
+__global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_constant__ fast::Params p) {
+    constexpr bool GATE = LAYOUT != kKV;
+    constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
+    constexpr int NTILE = NSRC * (QS ? 2 : 1);
+    constexpr int SR = 0;
+    constexpr int SK = LAYOUT == kRKV ? 1 : 0;
+    constexpr int SV = LAYOUT == kKV ? 1 : (LAYOUT == kRKV ? 2 : 0);
+    constexpr int es = Io<IO>::kBytes;
+    constexpr int RB = kCS * es;         // bytes per token row of a tile
+    constexpr int PB = 2 * es;           // bytes per channel pair
+    constexpr int SUB = kTc / kL * RB;   // bytes per sub-tile (128 token rows)
+
+    extern __shared__ __align__(128) char smem_raw[];
+    char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+    // The gate factor's two halves are parked in r's slot and, with Q-Shift,
+    // in shifted r's slot (both read to make r); without Q-Shift in one
+    // extra tile, so no slot another value still needs is overwritten.
+    constexpr int NTA = GATE && !QS ? NTILE + 1 : NTILE;
+    constexpr int G1 = QS ? 2 * SR + 1 : NTILE;  // tile of the second half
+    Scratch& S = *reinterpret_cast<Scratch*>(smem + NTA * p.tile_bytes);
+
+    const int tid = threadIdx.x;
+    const int j = tid % kNP;   // channel pair
+    const int q = tid / kNP;   // chunk within the CTA
+    const int cq = q % kCPW;   // chunk within the warp
+    const int warp = tid >> 5;
+    if (tid == 0) {
+        mbar_init(&S.bar, 1);
+        if (p.ncl > 1) {
+            mbar_init(&S.xbar, 1);
+            mbar_expect_tx(&S.xbar, (unsigned)(p.ncl * kNP * (sizeof(float4) * 2 + sizeof(float2))));
+        }
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (p.ncl > 1) cluster_arrive_relaxed();  // waited for before the first push
+    // this thread's lane of the CTA's columns
+    const uint32_t tmem = S.tmem + ((uint32_t)(warp * 32) << 16);
+
+    const int rank = blockIdx.x, slab = blockIdx.y, b = blockIdx.z;
+    const int c0 = slab * kCS;
+    const int t0 = rank * p.Tc;
+    const int tend = min(p.T, t0 + p.Tc);
+    int grp = QS ? qs_group(c0, p.g) : 4;
+    if (grp >= p.ng) grp = 4;
+    const bool shifted = QS && grp < 4;
+
+    // ---- tile loads: lane i of warp 0 loads sub-tile i of each tile -----------
+    if (warp == 0) {
+        if (tid == 0)
+            mbar_expect_tx(&S.bar, (unsigned)p.box_bytes * (unsigned)(kL * NSRC * (shifted ? 2 : 1)));
+        __syncwarp();
+        if (tid < kL) {
+            const int i = tid, h0 = rank * p.rows;
+            for (int s = 0; s < NSRC; ++s) {
+                char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB;
+                if (!QS) {
+#pragma unroll
+                    for (int h = 0; h < kTc / 256; ++h)
+                        tma_load_3d(plain + h * 32 * RB, &p.map[s], c0, t0 + i + 256 * h, b, &S.bar);
+                } else {
+                    tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar);
+                    if (shifted) {
+                        const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
+                        const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
+                        tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, h0 + dh, b, &S.bar);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- per-thread constants (overlap the copies) -------------------------------
+    const int cA = c0 + 2 * j;
+    const float invT = p.invT;
+    const float2 wv = make_float2(__ldg(p.w + cA), __ldg(p.w + cA + 1));
+    const float2 uv = make_float2(__ldg(p.u + cA), __ldg(p.u + cA + 1));
+    const float2 lam2 = mul2(wv, f2(invT * kLog2e));  // w / T in base-2 units
+    const float2 alpha = ex2c(make_float2(-lam2.x, -lam2.y));
+    const float2 eu = ex2(mul2(uv, f2(kLog2e)));
+    const float2 a8 = ex2c(mul2(lam2, f2(-(float)kL)));  // a^8: across one sub-chunk
+    auto mu_of = [&](const float* m) { return m ? make_float2(__ldg(m + cA), __ldg(m + cA + 1)) : f2(0.0f); };
+    const float2 muk = QS ? mu_of(p.mu[1]) : f2(1.0f);
+    const float2 muv = QS ? mu_of(p.mu[2]) : f2(1.0f);
+    const float2 mur = (QS && GATE) ? mu_of(p.mu[0]) : f2(1.0f);
+    S.tab[q][j] = ex2c(mul2(lam2, f2(-(float)kKL * q)));  // a^(32 q)
+
+    const int nvt = max(0, min(kKL, tend - (t0 + q * kKL)));  // valid tokens of this chunk
+
+    if (tid == 0) mbar_wait_bounded(&S.bar, p.err);
+    __syncthreads();
+
+    // ---- 1-2. per 8-token sub-chunk: load, Q-Shift mix, gate factor (parked in
+    // the token's slots), local maximum, p = 2^(k - M_h), two-sided sums inside
+    // the sub-chunk; the per-token sums go to tensor memory -------------------------
+    const char* tK = smem + (QS ? 2 * SK : SK) * p.tile_bytes;
+    const char* tV = smem + (QS ? 2 * SV : SV) * p.tile_bytes;
+    const char* tR = smem + (QS ? 2 * SR : SR) * p.tile_bytes;
+    const int dsh = shifted ? p.tile_bytes : 0;
+    char* g0 = smem + (QS ? 2 * SR : SR) * p.tile_bytes;  // gate factor, first channel
+    char* g1 = smem + G1 * p.tile_bytes;                 // second channel
+    float4 Fh[kH], Gh[kH];
+    float2 Mh[kH];
+#pragma unroll
+    for (int h = 0; h < kH; ++h) {
+        const int rowoff = (q * kH + h) * RB + j * PB;
+        const int nv = max(0, min(kL, nvt - h * kL));
+        float2 kk[kL], vv[kL];
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            const int o = rowoff + i * SUB;
+            float2 k, v, r;
+            if (QS) {
+                if (LAYOUT == kX) {
+                    const float2 x = lds_pair<IO>(tK, o), xd = lds_pair<IO>(tK + dsh, o);
+                    const float2 d = fma2(xd, f2(-1.0f), x);
+                    k = fma2(muk, d, xd);
+                    v = fma2(muv, d, xd);
+                    r = fma2(mur, d, xd);
+                } else {
+                    const float2 xk = lds_pair<IO>(tK, o), xkd = lds_pair<IO>(tK + dsh, o);
+                    const float2 xv = lds_pair<IO>(tV, o), xvd = lds_pair<IO>(tV + dsh, o);
+                    k = fma2(muk, fma2(xkd, f2(-1.0f), xk), xkd);
+                    v = fma2(muv, fma2(xvd, f2(-1.0f), xv), xvd);
+                    if (GATE) {
+                        const float2 xr = lds_pair<IO>(tR, o), xrd = lds_pair<IO>(tR + dsh, o);
+                        r = fma2(mur, fma2(xrd, f2(-1.0f), xr), xrd);
+                    }
+                }
+            } else {
+                k = lds_pair<IO>(tK, o);
+                v = lds_pair<IO>(tV, o);
+                if (GATE) r = lds_pair<IO>(tR, o);
+            }
+            if (GATE) {
+                const float2 g = ex2(mul2(r, f2(-kLog2e)));
+                sts_f32(g0 + o, g.x);
+                sts_f32(g1 + o, g.y);
+            }
+            kk[i] = k;
+            vv[i] = v;
+        }
+        float2 mx = f2(-INFINITY);
+        if (nv == kL) {
+#pragma unroll
+            for (int i = 0; i < kL; ++i) mx = max2(mx, kk[i]);
+        } else {
+            // tokens past the sequence end: p = 0 and p v = 0
+#pragma unroll
+            for (int i = 0; i < kL; ++i) {
+                kk[i] = (i < nv) ? kk[i] : f2(-INFINITY);
+                vv[i] = (i < nv) ? vv[i] : f2(0.0f);
+                mx = max2(mx, kk[i]);
+            }
+        }
+        Mh[h] = mx;
+        const float2 negM = make_float2(mx.x == -INFINITY ? 0.0f : -mx.x * kLog2e,
+                                        mx.y == -INFINITY ? 0.0f : -mx.y * kLog2e);
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            kk[i] = ex2(fma2(kk[i], f2(kLog2e), negM));  // p_i (0 beyond T)
+            vv[i] = mul2(kk[i], vv[i]);                  // p_i v_i
+        }
+        float nd[32];  // per token i: num.x, num.y, den.x, den.y
+        float2 fa = f2(0.0f), fc = f2(0.0f);
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            nd[4 * i + 0] = fa.x;
+            nd[4 * i + 1] = fa.y;
+            nd[4 * i + 2] = fc.x;
+            nd[4 * i + 3] = fc.y;
+            fa = fma2(alpha, fa, vv[i]);
+            fc = fma2(alpha, fc, kk[i]);
+        }
+        float2 ga = f2(0.0f), gc = f2(0.0f);
+#pragma unroll
+        for (int i = kL - 1; i >= 0; --i) {
+            const float2 n2 = add2(make_float2(nd[4 * i], nd[4 * i + 1]), fma2(eu, vv[i], ga));
+            const float2 d2 = add2(make_float2(nd[4 * i + 2], nd[4 * i + 3]), fma2(eu, kk[i], gc));
+            nd[4 * i + 0] = n2.x;
+            nd[4 * i + 1] = n2.y;
+            nd[4 * i + 2] = d2.x;
+            nd[4 * i + 3] = d2.y;
+            ga = fma2(alpha, ga, vv[i]);
+            gc = fma2(alpha, gc, kk[i]);
+        }
+        tmem_st32(tmem + h * 32, nd);
+        Fh[h] = make_float4(fa.x, fa.y, fc.x, fc.y);
+        Gh[h] = make_float4(ga.x, ga.y, gc.x, gc.y);
+    }
+
+    // ---- 3a. warp maximum (the reference of the warp's sums) and the chunk's
+    // totals on it ---------------------------------------------------------------
+    float2 mx = max2(max2(Mh[0], Mh[1]), max2(Mh[2], Mh[3]));
+#pragma unroll
+    for (int d = kNP; d < 32; d <<= 1) {
+        mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
+        mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, d));
+    }
+    if (cq == 0) S.wmax[j][warp] = mx;  // -inf for a warp wholly past T
+    const float2 mref = make_float2(mx.x == -INFINITY ? 0.0f : mx.x, mx.y == -INFINITY ? 0.0f : mx.y);
+    float2 eh[kH];
+    auto scale4 = [](float2 e, float4 v) { return make_float4(v.x * e.x, v.y * e.y, v.z * e.x, v.w * e.y); };
+#pragma unroll
+    for (int h = 0; h < kH; ++h) {
+        eh[h] = ex2(mul2(add2(Mh[h], make_float2(-mref.x, -mref.y)), f2(kLog2e)));
+        Fh[h] = scale4(eh[h], Fh[h]);  // sub-chunk totals on the warp reference
+        Gh[h] = scale4(eh[h], Gh[h]);
+    }
+    // chunk totals: forward at the chunk's end, backward at its start
+    float4 Fi = Fh[0], Gi = Gh[kH - 1];
+#pragma unroll
+    for (int h = 1; h < kH; ++h) {
+        Fi = fma4(a8, Fi, Fh[h]);
+        Gi = fma4(a8, Gi, Gh[kH - 1 - h]);
+    }
+
+    // ---- 3b. scans: warp, CTA, cluster ------------------------------------------
+#pragma unroll
+    for (int e = 0; (kNP << e) < 32; ++e) {
+        const float2 m = S.tab[1 << e][j];  // a^(32 * 2^e)
+        float4 o = shfl_up4(Fi, kNP << e, 32);
+        if (cq >= (1 << e)) Fi = fma4(m, o, Fi);
+        o = shfl_down4(Gi, kNP << e, 32);
+        if (cq + (1 << e) < kCPW) Gi = fma4(m, o, Gi);
+    }
+    float4 X = shfl_up4(Fi, kNP, 32), Y = shfl_down4(Gi, kNP, 32);
+    if (cq == 0) X = zero4();
+    if (cq == kCPW - 1) Y = zero4();
+    if (cq == kCPW - 1) S.waggF[j][warp] = Fi;
+    if (cq == 0) S.waggB[j][warp] = Gi;
+    __syncthreads();
+    if (warp == 0) {
+        const bool act = tid < kNP * kNW;
+        const int jj = act ? tid / kNW : 0, wi = act ? tid % kNW : 0;
+        const float2 mw = S.wmax[jj][wi];
+        float2 mc = mw;
+#pragma unroll
+        for (int d = 1; d < kNW; d <<= 1) {
+            mc.x = fmaxf(mc.x, __shfl_xor_sync(0xffffffffu, mc.x, d, kNW));
+            mc.y = fmaxf(mc.y, __shfl_xor_sync(0xffffffffu, mc.y, d, kNW));
+        }
+        const float2 ws = ex2(mul2(add2(mw, make_float2(-mc.x, -mc.y)), f2(kLog2e)));
+        float4 f = scale4(ws, S.waggF[jj][wi]);
+        float4 gb = scale4(ws, S.waggB[jj][wi]);
+#pragma unroll
+        for (int d = 1; d < kNW; d <<= 1) {
+            const float2 m = S.tab[kCPW * d][jj];  // across d warps
+            float4 o = shfl_up4(f, d, kNW);
+            if (wi >= d) f = fma4(m, o, f);
+            o = shfl_down4(gb, d, kNW);
+            if (wi + d < kNW) gb = fma4(m, o, gb);
+        }
+        float4 xw = shfl_up4(f, 1, kNW), yw = shfl_down4(gb, 1, kNW);
+        if (wi == 0) xw = zero4();
+        if (wi == kNW - 1) yw = zero4();
+        if (act) {
+            S.wsc[jj][wi] = ws;
+            S.wcarF[jj][wi] = xw;
+            S.wcarB[jj][wi] = yw;
+            if (p.ncl > 1) {
+                if (wi == p.Tc / kWarpTok - 1) S.ownF[jj] = f;
+                if (wi == 0) {
+                    S.ownG[jj] = gb;
+                    S.ownM[jj] = mul2(mc, f2(kLog2e));
+                }
+            }
+        }
+    }
+    // exchange lanes: thread (channel lc, peer rr) in segments of 8 lanes
+    const int lc = tid >> 3, rr = tid & 7;
+    constexpr int nex = kCS * 8;  // 64 threads: warp-uniform
+    float2 cs_sl = f2(1.0f), cs_af = f2(0.0f), cs_cf = f2(0.0f), cs_bb = f2(0.0f), cs_db = f2(0.0f);
+    if (p.ncl > 1) {
+        float mdec[3];
+        if (tid < nex) {
+            const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
+#pragma unroll
+            for (int e = 0; e < 3; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
+        }
+        __syncthreads();
+        cluster_wait_acquire();  // every mailbox barrier is initialised
+        {
+            const int peer = tid / (2 * kNP), jj = (tid >> 1) % kNP;
+            if (peer < p.ncl) {
+                const unsigned rbar = mapa_u32(smem_u32(&S.xbar), peer);
+                if ((tid & 1) == 0) {
+                    st_async4(mapa_u32(smem_u32(&S.mbF[rank][jj]), peer), S.ownF[jj], rbar);
+                } else {
+                    st_async4(mapa_u32(smem_u32(&S.mbG[rank][jj]), peer), S.ownG[jj], rbar);
+                    st_async2(mapa_u32(smem_u32(&S.mbM[rank][jj]), peer), S.ownM[jj], rbar);
+                }
+            }
+        }
+        if (tid == 0) mbar_wait_cluster_bounded(&S.xbar, p.err);
+        __syncthreads();
+        if (tid < nex) {
+            float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
+            if (rr < p.ncl) {
+                const float4 F = S.mbF[rr][lc >> 1], G = S.mbG[rr][lc >> 1];
+                const float2 Mp = S.mbM[rr][lc >> 1];
+                const bool hi = lc & 1;
+                Mr = hi ? Mp.y : Mp.x;
+                fa2 = hi ? F.y : F.x;
+                fc2 = hi ? F.w : F.z;
+                ga2 = hi ? G.y : G.x;
+                gc2 = hi ? G.w : G.z;
+            }
+            float Mc = Mr;
+#pragma unroll
+            for (int d = 4; d >= 1; d >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, 8));
+            const float sc = ex2(Mr - Mc);  // 0 for lanes past the cluster
+            fa2 *= sc;
+            fc2 *= sc;
+            ga2 *= sc;
+            gc2 *= sc;
+#pragma unroll
+            for (int e = 0, d = 1; d < 8; ++e, d <<= 1) {
+                const float m = mdec[e];  // decay across d CTAs
+                const float ua = __shfl_up_sync(0xffffffffu, fa2, d, 8);
+                const float uc = __shfl_up_sync(0xffffffffu, fc2, d, 8);
+                const float da = __shfl_down_sync(0xffffffffu, ga2, d, 8);
+                const float dc = __shfl_down_sync(0xffffffffu, gc2, d, 8);
+                if (rr >= d) {
+                    fa2 = fmaf(m, ua, fa2);
+                    fc2 = fmaf(m, uc, fc2);
+                }
+                if (rr + d < 8) {
+                    ga2 = fmaf(m, da, ga2);
+                    gc2 = fmaf(m, dc, gc2);
+                }
+            }
+            const float Af = __shfl_sync(0xffffffffu, fa2, max(rank - 1, 0), 8);
+            const float Cf = __shfl_sync(0xffffffffu, fc2, max(rank - 1, 0), 8);
+            const float Bb = __shfl_sync(0xffffffffu, ga2, min(rank + 1, 7), 8);
+            const float Db = __shfl_sync(0xffffffffu, gc2, min(rank + 1, 7), 8);
+            const float Mme = __shfl_sync(0xffffffffu, Mr, rank, 8);
+            if (rr == 0) {
+                S.cscale[lc] = make_float4(ex2(Mme - Mc), 0.f, 0.f, 0.f);
+                S.ccarry[lc] = make_float4(rank > 0 ? Af : 0.f, rank > 0 ? Cf : 0.f,
+                                           rank + 1 < p.ncl ? Bb : 0.f, rank + 1 < p.ncl ? Db : 0.f);
+            }
+        }
+        __syncthreads();
+        const float4 s0 = S.cscale[2 * j], s1 = S.cscale[2 * j + 1];
+        const float4 k0 = S.ccarry[2 * j], k1 = S.ccarry[2 * j + 1];
+        cs_sl = make_float2(s0.x, s1.x);
+        cs_af = make_float2(k0.x, k1.x);
+        cs_cf = make_float2(k0.y, k1.y);
+        cs_bb = make_float2(k0.z, k1.z);
+        cs_db = make_float2(k0.w, k1.w);
+    } else {
+        __syncthreads();
+    }
+
+    // ---- 4. carries -> outputs ---------------------------------------------------
+    const float2 sl = cs_sl;
+    const float2 slw = mul2(sl, S.wsc[j][warp]);
+    const float4 XW = S.wcarF[j][warp], YW = S.wcarB[j][warp];
+    const float2 slF = mul2(sl, S.tab[cq][j]), slB = mul2(sl, S.tab[kCPW - 1 - cq][j]);
+    const float2 kf = S.tab[q][j];                          // CTA start -> chunk start
+    const float2 kb = S.tab[max(0, p.Tc / kKL - 1 - q)][j];  // chunk end -> CTA end
+    // carries into the chunk: from the left at its start, from the right at its end
+    float2 Ac = fma2(slw, lo2(X), fma2(slF, lo2(XW), mul2(kf, cs_af)));
+    float2 Cc = fma2(slw, hi2(X), fma2(slF, hi2(XW), mul2(kf, cs_cf)));
+    // carries from the right into each sub-chunk: B_3 = the chunk's, then
+    // B_{h-1} = a^8 B_h + sub-chunk h's backward total
+    float2 Bs[kH], Ds[kH];
+    Bs[kH - 1] = fma2(slw, lo2(Y), fma2(slB, lo2(YW), mul2(kb, cs_bb)));
+    Ds[kH - 1] = fma2(slw, hi2(Y), fma2(slB, hi2(YW), mul2(kb, cs_db)));
+#pragma unroll
+    for (int h = kH - 1; h > 0; --h) {
+        Bs[h - 1] = fma2(slw, lo2(Gh[h]), mul2(a8, Bs[h]));
+        Ds[h - 1] = fma2(slw, hi2(Gh[h]), mul2(a8, Ds[h]));
+    }
+    float2 pw[kL];
+    pw[0] = f2(1.0f);
+#pragma unroll
+    for (int i = 1; i < kL; ++i) pw[i] = min2(mul2(pw[i - 1], alpha), f2(0x1p126f));
+    tmem_wait_st();
+    char* tout = smem;
+#pragma unroll
+    for (int h = 0; h < kH; ++h) {
+        float nd[32];
+        tmem_ld32(tmem + h * 32, nd);
+        const float2 sh = mul2(slw, eh[h]);
+        const int rowoff = (q * kH + h) * RB + j * PB;
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            const int o = rowoff + i * SUB;
+            const float2 nn = make_float2(nd[4 * i], nd[4 * i + 1]);
+            const float2 dd = make_float2(nd[4 * i + 2], nd[4 * i + 3]);
+            const float2 num = fma2(sh, nn, fma2(pw[i], Ac, mul2(pw[kL - 1 - i], Bs[h])));
+            float2 den = fma2(sh, dd, fma2(pw[i], Cc, mul2(pw[kL - 1 - i], Ds[h])));
+            if (GATE) {
+                // read before the result overwrites the first slot
+                const float2 g = make_float2(lds_f32(g0 + o), lds_f32(g1 + o));
+                den = fma2(den, g, den);
+            }
+            Io<IO>::st_pair(tout + o, mul2(num, rcp(den)));
+        }
+        // carry from the left into the next sub-chunk
+        Ac = fma2(slw, lo2(Fh[h]), mul2(a8, Ac));
+        Cc = fma2(slw, hi2(Fh[h]), mul2(a8, Cc));
+    }
+    // results leave by TMA stores: lane i of warp 0 stores sub-tile i in boxes
+    // of 256 strided tokens, clipped at T by the tensor map
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid < kL) {
+        const int nbox = (tend - t0 + 255) / 256;
+        for (int hb = 0; hb < nbox; ++hb)
+            tma_store_3d(&p.omap, tout + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
+        bulk_commit_and_wait_read();
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(S.tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace tm32
+}  // namespace vrwkv

@@ -19,6 +19,7 @@
 #include "vrwkv.h"
 #include "biwkv.cuh"
 #include "biwkv_tma.cuh"
+#include "biwkv_tm.cuh"
 #include "biwkv_wide.cuh"
 #include "qshift.cuh"
 #include "channel_mix.cuh"
@@ -417,7 +418,9 @@ bool tma_chunk8_forced() {
 
 struct FastPlan {
     fast::Params p;
+    bool tm;     // 32-token chunks with tensor-memory partial sums (biwkv_tm_kernel)
     int layout;
+    int ntiles;  // tiles per CTA (sources, doubled with Q-Shift)
     bool qs;
     bool gx;  // exchange through the caller's workspace instead of a cluster
     int nt;   // threads per CTA
@@ -527,6 +530,69 @@ constexpr int kFastThreads8 = 256;
 constexpr int kFastTcMax = fast::Cfg<kFastThreads16, 16>::kTcMax;
 static_assert(kFastTcMax == fast::Cfg<kFastThreads8, 8>::kTcMax, "one tile geometry for both shapes");
 
+// The 32-token tensor-memory kernel: a cluster per column as in the 8-channel
+// kernel.  Sets *fell_back when the shape cannot be co-scheduled or more
+// than four CTAs would share an SM (their tensor memory would not fit).
+template <typename IO, int LAYOUT, bool QS>
+vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
+    auto kern = tm32::biwkv_tm_kernel<IO, LAYOUT, QS>;
+    static std::atomic<int> granted{0};
+    cudaError_t e = ensure_smem(kern, granted, pl.smem);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = pl.grid;
+    cfg.blockDim = dim3(tm32::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.p.ncl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+    cfg.attrs = attr;
+    cfg.numAttrs = pl.p.ncl > 1 ? 2 : 0;
+    // checked once per (cluster size, shared memory)
+    static std::mutex mu;
+    static std::vector<std::array<int, 3>> seen;
+    int okv = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (const auto& a : seen)
+            if (a[0] == pl.p.ncl && a[1] == pl.smem) okv = a[2];
+    }
+    if (okv == 0) {
+        int per_sm = 0, nclu = 1;
+        cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tm32::kThreads, pl.smem);
+        if (oe == cudaSuccess && pl.p.ncl > 1) oe = cudaOccupancyMaxActiveClusters(&nclu, kern, &cfg);
+        if (oe != cudaSuccess) cudaGetLastError();
+        okv = (oe == cudaSuccess && per_sm >= 1 && per_sm * tm32::kTmemCols <= 512 && nclu > 0) ? 1 : -1;
+        std::lock_guard<std::mutex> lk(mu);
+        seen.push_back({pl.p.ncl, pl.smem, okv});
+    }
+    if (okv < 0) {
+        *fell_back = true;
+        return VRWKV_OK;
+    }
+    e = cudaLaunchKernelEx(&cfg, kern, pl.p);
+    if (e != cudaSuccess) return cuda_status(e, "biwkv_tm_kernel launch");
+    g_last_kernel = "biwkv_tm_kernel";
+    return ok();
+}
+
+template <typename IO>
+vrwkv_status dispatch_tm(const FastPlan& pl, cudaStream_t s, bool* fb) {
+    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
+    case fast::kKV * 2 + 0: return launch_tm<IO, fast::kKV, false>(pl, s, fb);
+    case fast::kKV * 2 + 1: return launch_tm<IO, fast::kKV, true>(pl, s, fb);
+    case fast::kRKV * 2 + 0: return launch_tm<IO, fast::kRKV, false>(pl, s, fb);
+    case fast::kRKV * 2 + 1: return launch_tm<IO, fast::kRKV, true>(pl, s, fb);
+    case fast::kX * 2 + 0: return launch_tm<IO, fast::kX, false>(pl, s, fb);
+    default: return launch_tm<IO, fast::kX, true>(pl, s, fb);
+    }
+}
+
 template <typename IO>
 vrwkv_status dispatch_fast(const FastPlan& pl, cudaStream_t s, bool* fb) {
     if (pl.kl == 16)
@@ -543,12 +609,22 @@ int fast_smem(int ntiles, int tile_bytes, int kl) {
     return ntiles * tile_bytes + scratch + 128;  // + alignment slack
 }
 
+// Shared memory of a tensor-memory kernel CTA: its tiles (one extra for the
+// gate factor without Q-Shift), the scratch block, and at least the floor
+// that keeps a fifth CTA off an SM.
+int tm_smem(bool gate, bool qs, int ntiles, int tile_bytes) {
+    const int nta = gate && !qs ? ntiles + 1 : ntiles;
+    return std::max(nta * tile_bytes + (int)sizeof(tm32::Scratch) + 128, tm32::kSmemFloor);
+}
+
 // Plan the TMA path; returns false when the problem is outside its limits
-// (the generic kernel then runs).
+// (the generic kernel then runs).  tmem_chunks plans the 32-token kernel
+// (1024-token CTAs, clusters of up to 8).
 bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void* v, const float* w,
                const float* u, void* out, int B, int T, int C, vrwkv_dtype dtype,
-               const vrwkv_qshift_params* qs, void* ws) {
+               const vrwkv_qshift_params* qs, void* ws, bool tmem_chunks = false) {
     if (tma_disabled()) return false;
+    pl.tm = tmem_chunks;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const int es = elem_bytes(dtype);
@@ -580,8 +656,9 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     p.C = C;
     const int RB = fast::kCS * es;
     const int ntiles = nsrc * (pl.qs ? 2 : 1);
-    const int TcMax = kFastTcMax;
-    pl.kl = tma_chunk8_forced() ? 8 : 16;
+    pl.ntiles = ntiles;
+    const int TcMax = pl.tm ? tm32::kTc : kFastTcMax;
+    pl.kl = pl.tm ? tm32::kKL : (tma_chunk8_forced() ? 8 : 16);
     if (pl.qs) {
         p.H = qs->H;
         p.W = qs->W;
@@ -598,8 +675,10 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
             // 16-token chunks where possible, else 8-token chunks
             int rows = 0;
             for (int kl = pl.kl; kl >= 8 && rows == 0; kl /= 2) {
-                const int warp_tok = kl == 16 ? fast::Cfg<kFastThreads16, 16>::kWarpTok
-                                              : fast::Cfg<kFastThreads8, 8>::kWarpTok;
+                if (pl.tm && kl != tm32::kKL) break;
+                const int warp_tok = kl == 32   ? tm32::kWarpTok
+                                     : kl == 16 ? fast::Cfg<kFastThreads16, 16>::kWarpTok
+                                                : fast::Cfg<kFastThreads8, 8>::kWarpTok;
                 for (int rr = TcMax / p.W; rr >= 1; --rr)
                     if ((rr * p.W) % warp_tok == 0) {
                         rows = rr;
@@ -622,7 +701,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         p.Tc = std::min(T, TcMax);
         p.ncl = (T + p.Tc - 1) / p.Tc;
     }
-    if (p.ncl > fast::kClusterMax) return false;
+    if (p.ncl > (pl.tm ? tm32::kClusterMax : fast::kClusterMax)) return false;
     // 8 sub-tiles of TcMax / 8 token rows; every thread reads its row of
     // each, so a tile always spans TcMax tokens even when the boxes deliver
     // fewer
@@ -631,8 +710,8 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     // and its full TcMax / 8 rows without (boxes of 32 rows; tokens past T
     // arrive as zeros)
     p.box_bytes = (pl.qs ? (p.W / fast::kL) * p.rows : TcMax / fast::kL) * RB;
-    pl.nt = pl.kl == 16 ? kFastThreads16 : kFastThreads8;
-    pl.smem = fast_smem(ntiles, p.tile_bytes, pl.kl);
+    pl.nt = pl.tm ? tm32::kThreads : (pl.kl == 16 ? kFastThreads16 : kFastThreads8);
+    pl.smem = pl.tm ? tm_smem(gate, pl.qs, ntiles, p.tile_bytes) : fast_smem(ntiles, p.tile_bytes, pl.kl);
     if (pl.smem > 227 * 1024) return false;
     const CUtensorMapDataType dt =
         dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -684,6 +763,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     p.nslab = C / fast::kCS;
     p.total = p.ncl * p.nslab * B;
     pl.gx = ws != nullptr && p.ncl > 1;
+    if (pl.tm && (pl.gx || !p.tma_store)) return false;
     if (pl.gx) {
         const WsLayout L = ws_layout(B, C);
         char* base = static_cast<char*>(ws);
@@ -711,6 +791,16 @@ bool wide_disabled() {
 bool wide_preferred() {
     const char* e = getenv("VRWKV_FORWARD");
     return e && e[0] == 'w';
+}
+
+// The 32-token tensor-memory kernel takes columns of 2048 tokens and more
+// (shorter ones leave too many of its threads idle); VRWKV_FORWARD=tm takes
+// it wherever it qualifies, VRWKV_FORWARD=narrow never.
+bool tm_wanted(int T) {
+    const char* e = getenv("VRWKV_FORWARD");
+    if (e && e[0] == 't') return true;
+    if (e && e[0]) return false;
+    return T >= 2048;
 }
 
 struct WidePlan {
@@ -976,6 +1066,16 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
             cudaStream_t ws_ = static_cast<cudaStream_t>(stream);
             vrwkv_status st = dtype == VRWKV_F32 ? dispatch_wide<float>(wp, ws_, &fell_back)
                                                  : dispatch_wide<__nv_bfloat16>(wp, ws_, &fell_back);
+            if (!fell_back) return st;
+        }
+    }
+    if (B <= 65535 && C / vrwkv::fast::kCS <= 65535 && !with_ws && tm_wanted(T)) {
+        FastPlan fp;
+        if (plan_fast(fp, gate, r, k, v, w, u, out, B, T, C, dtype, qs, nullptr, true)) {
+            bool fell_back = false;
+            cudaStream_t fs = static_cast<cudaStream_t>(stream);
+            vrwkv_status st = dtype == VRWKV_F32 ? dispatch_tm<float>(fp, fs, &fell_back)
+                                                 : dispatch_tm<__nv_bfloat16>(fp, fs, &fell_back);
             if (!fell_back) return st;
         }
     }

@@ -175,14 +175,16 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     return (got, err) if return_out else err
 
 
-@pytest.fixture(params=["tma", "wide", "tma8", "gx", "generic"])
+@pytest.fixture(params=["default", "narrow", "tm", "wide", "tma8", "gx", "generic"])
 def kernel_path(request, monkeypatch):
-    """Run a test on the default path (the 8-channel TMA kernel with 16-token
-    thread chunks where the shape and cluster geometry allow), on the
-    16-channel slab kernel where the shape qualifies ("wide"), on the
-    8-channel kernel held to 8-token chunks, on its workspace variant
-    (global-memory exchange instead of clusters) and with the generic kernel
-    forced."""
+    """Run a test on the default path (the 32-token tensor-memory kernel for
+    columns of 2048 tokens and more, else the 8-channel TMA kernel with
+    16-token thread chunks, where the shape and cluster geometry allow), on
+    the latter alone ("narrow"), on the tensor-memory kernel wherever it
+    qualifies ("tm"), on the 16-channel slab kernel where the shape qualifies
+    ("wide"), on the 8-channel kernel held to 8-token chunks, on its
+    workspace variant (global-memory exchange instead of clusters) and with
+    the generic kernel forced."""
     if request.param == "generic":
         monkeypatch.setenv("VRWKV_DISABLE_TMA", "1")
     else:
@@ -191,8 +193,9 @@ def kernel_path(request, monkeypatch):
         monkeypatch.setenv("VRWKV_TMA_CHUNK", "8")
     else:
         monkeypatch.delenv("VRWKV_TMA_CHUNK", raising=False)
-    if request.param == "wide":
-        monkeypatch.setenv("VRWKV_FORWARD", "wide")
+    forward = {"wide": "wide", "tm": "tm", "narrow": "narrow", "tma8": "narrow"}.get(request.param)
+    if forward:
+        monkeypatch.setenv("VRWKV_FORWARD", forward)
     else:
         monkeypatch.delenv("VRWKV_FORWARD", raising=False)
     _GX["on"] = request.param == "gx"
@@ -204,6 +207,14 @@ def kernel_path(request, monkeypatch):
 def test_workload_full_size(vk, oracle_mod, cfg, kernel_path):
     wl = synth.WORKLOADS[cfg]
     run_fused(vk, oracle_mod, wl)
+
+
+@pytest.mark.parametrize("cfg", [4, 5])
+def test_default_forward_is_the_tensor_memory_kernel(vk, oracle_mod, cfg, monkeypatch):
+    monkeypatch.delenv("VRWKV_FORWARD", raising=False)
+    wl = synth.WORKLOADS[cfg]
+    run_fused(vk, oracle_mod, wl)
+    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tm_kernel"
 
 
 @pytest.mark.parametrize("cfg", [4, 5])
@@ -239,6 +250,33 @@ def test_wide_kernel_shapes(vk, oracle_mod, case, monkeypatch):
     run_fused(vk, oracle_mod, wl)
     got = vk.load_library().vrwkv_last_kernel().decode()
     assert (got == "biwkv_wide_kernel") == wide, got
+
+
+# Shapes aimed at the 32-token tensor-memory kernel's geometry: 1024-token
+# CTAs (16 image rows of 64), CTAs of 768 tokens (W = 48, 96), a last CTA
+# holding one token, 8-CTA clusters at T = 8192, float32 tiles (three or one
+# CTA per SM), separate r, k, v with Q-Shift (six tiles) and copied channels.
+TM_CASES = [
+    # call, B, H, W, C, dtype, gamma
+    ("gate_qs_x", 1, 128, 64, 64, "bf16", 0.25),   # T = 8192: 8 CTAs
+    ("biwkv", 2, 1, 8192, 16, "f32", 0.25),        # 8 CTAs, no Q-Shift, float32
+    ("biwkv", 1, 1, 2049, 16, "bf16", 0.25),       # the third CTA holds one token
+    ("gate_qs", 1, 32, 96, 32, "f32", 0.25),       # W = 96: CTAs of 8 rows (768 tokens)
+    ("gate_qs_x", 2, 48, 48, 32, "bf16", 0.25),    # W = 48: CTAs of 16 rows (768 tokens)
+    ("qshift_biwkv", 1, 32, 64, 64, "bf16", 0.25),  # no gate, Q-Shift
+    ("gate_qs_x", 1, 64, 64, 128, "bf16", 0.125),  # copied channels 64..127
+    ("gate_qs", 2, 64, 64, 32, "bf16", 0.25),      # r, k, v with Q-Shift: six tiles
+    ("gate_qs_x", 1, 12, 16, 64, "bf16", 0.25),    # T = 192: one CTA, 6 of 32 chunks used
+]
+
+
+@pytest.mark.parametrize("case", TM_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_tm_kernel_shapes(vk, oracle_mod, case, monkeypatch):
+    monkeypatch.setenv("VRWKV_FORWARD", "tm")
+    call, B, H, W, C, dt, gamma = case
+    wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000, gamma=gamma)
+    run_fused(vk, oracle_mod, wl)
+    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tm_kernel"
 
 
 # Sequences past 4096 tokens: the pages' efficiency comparison runs 2048^2
@@ -452,9 +490,9 @@ def test_workspace_reuse_across_launches(vk, oracle_mod, monkeypatch):
         mus = [vec_f32(inp[n])[0] for n in ("mu_r", "mu_k", "mu_v")]
         qs = vk.QShift(H, W, 1, 0.25, *mus)
         a = vk.spatial_gate(x, x, x, w, u, qs=qs, workspace=ws)
-        monkeypatch.setenv("VRWKV_DISABLE_WIDE", "1")
+        monkeypatch.setenv("VRWKV_FORWARD", "narrow")
         b = vk.spatial_gate(x, x, x, w, u, qs=qs)  # the same kernel's cluster exchange
-        monkeypatch.delenv("VRWKV_DISABLE_WIDE")
+        monkeypatch.delenv("VRWKV_FORWARD")
         vk.device_status()
         assert torch.equal(a, b)
         outs.append(a)
