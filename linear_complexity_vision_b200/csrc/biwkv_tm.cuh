@@ -102,6 +102,15 @@ struct alignas(16) Scratch {
     unsigned int tmem;  // base address of this CTA's tensor-memory columns
 };
 
+// Per-thread sub-chunk values in natural sub-chunk order, for the rotated
+// kernel: entry [h][thread] (threads fastest: conflict-free 16-byte
+// accesses).  Holds the sub-chunk totals after the load pass, then the
+// carries into each sub-chunk for the output pass.
+struct alignas(16) Stash {
+    float4 a[kH][kThreads];  // totals F_h (A.xy, C.xy), then carries from the left
+    float4 b[kH][kThreads];  // totals G_h, then carries from the right
+};
+
 // 32 consecutive 32-bit columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(
@@ -135,6 +144,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // slot: data dependence alone orders each slot's accesses.
 __device__ __forceinline__ void sts_f32(char* p, float v) { *reinterpret_cast<float*>(p) = v; }
 __device__ __forceinline__ float lds_f32(const char* p) { return *reinterpret_cast<const float*>(p); }
+// three-input maximum (one instruction on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -143,7 +158,12 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-template <typename IO, int LAYOUT, bool QS>
+// ROT: lanes take their four sub-chunks in a rotated order (lane pair m of
+// a warp starts at sub-chunk m), so at every step the warp's 32 lanes touch
+// 8 different 16-byte rows of each 128-byte line: conflict-free tile, gate
+// and result accesses for 16-byte token rows.  The sub-chunk values that are
+// needed in natural order pass through a per-thread stash.
+template <typename IO, int LAYOUT, bool QS, bool ROT>
 __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_constant__ fast::Params p) {
     constexpr bool GATE = LAYOUT != kKV;
     constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
@@ -164,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     constexpr int NTA = GATE && !QS ? NTILE + 1 : NTILE;
     constexpr int G1 = QS ? 2 * SR + 1 : NTILE;  // tile of the second half
     Scratch& S = *reinterpret_cast<Scratch*>(smem + NTA * p.tile_bytes);
+    Stash& X2 = *reinterpret_cast<Stash*>(smem + NTA * p.tile_bytes + sizeof(Scratch));  // ROT only
 
     const int tid = threadIdx.x;
     const int j = tid % kNP;   // channel pair
@@ -252,10 +273,12 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     const int dsh = shifted ? p.tile_bytes : 0;
     char* g0 = smem + (QS ? 2 * SR : SR) * p.tile_bytes;  // gate factor, first channel
     char* g1 = smem + G1 * p.tile_bytes;                 // second channel
-    float4 Fh[kH], Gh[kH];
+    const int rot = ROT ? (cq >> 1) & (kH - 1) : 0;
+    float4 Fh[kH], Gh[kH];  // by step: the totals of sub-chunk (step + rot) mod 4
     float2 Mh[kH];
 #pragma unroll
-    for (int h = 0; h < kH; ++h) {
+    for (int st = 0; st < kH; ++st) {
+        const int h = ROT ? (st + rot) & (kH - 1) : st;  // the sub-chunk of this step
         const int rowoff = (q * kH + h) * RB + j * PB;
         const int nv = max(0, min(kL, nvt - h * kL));
         float2 kk[kL], vv[kL];
@@ -293,20 +316,18 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
             kk[i] = k;
             vv[i] = v;
         }
-        float2 mx = f2(-INFINITY);
-        if (nv == kL) {
-#pragma unroll
-            for (int i = 0; i < kL; ++i) mx = max2(mx, kk[i]);
-        } else {
+        if (nv < kL) {
             // tokens past the sequence end: p = 0 and p v = 0
 #pragma unroll
             for (int i = 0; i < kL; ++i) {
                 kk[i] = (i < nv) ? kk[i] : f2(-INFINITY);
                 vv[i] = (i < nv) ? vv[i] : f2(0.0f);
-                mx = max2(mx, kk[i]);
             }
         }
-        Mh[h] = mx;
+        float2 mx;
+        mx.x = max3f(max3f(kk[0].x, kk[1].x, kk[2].x), max3f(kk[3].x, kk[4].x, kk[5].x), fmaxf(kk[6].x, kk[7].x));
+        mx.y = max3f(max3f(kk[0].y, kk[1].y, kk[2].y), max3f(kk[3].y, kk[4].y, kk[5].y), fmaxf(kk[6].y, kk[7].y));
+        Mh[st] = mx;
         const float2 negM = make_float2(mx.x == -INFINITY ? 0.0f : -mx.x * kLog2e,
                                         mx.y == -INFINITY ? 0.0f : -mx.y * kLog2e);
 #pragma unroll
@@ -314,32 +335,46 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
             kk[i] = ex2(fma2(kk[i], f2(kLog2e), negM));  // p_i (0 beyond T)
             vv[i] = mul2(kk[i], vv[i]);                  // p_i v_i
         }
+        // Two-sided sums inside the sub-chunk, both directions in one pass (four
+        // independent recurrences per step): step it adds the forward sum
+        // before token it and the backward sum after token 7 - it; a token's
+        // second contribution also brings its own term e^u p v.
         float nd[32];  // per token i: num.x, num.y, den.x, den.y
-        float2 fa = f2(0.0f), fc = f2(0.0f);
+        float2 fa = f2(0.0f), fc = f2(0.0f), ga = f2(0.0f), gc = f2(0.0f);
 #pragma unroll
-        for (int i = 0; i < kL; ++i) {
-            nd[4 * i + 0] = fa.x;
-            nd[4 * i + 1] = fa.y;
-            nd[4 * i + 2] = fc.x;
-            nd[4 * i + 3] = fc.y;
+        for (int it = 0; it < kL; ++it) {
+            const int i = it, ib = kL - 1 - it;
+            if (it < kL / 2) {
+                nd[4 * i + 0] = fa.x;
+                nd[4 * i + 1] = fa.y;
+                nd[4 * i + 2] = fc.x;
+                nd[4 * i + 3] = fc.y;
+                nd[4 * ib + 0] = ga.x;
+                nd[4 * ib + 1] = ga.y;
+                nd[4 * ib + 2] = gc.x;
+                nd[4 * ib + 3] = gc.y;
+            } else {
+                const float2 n1 = add2(make_float2(nd[4 * i], nd[4 * i + 1]), fma2(eu, vv[i], fa));
+                const float2 d1 = add2(make_float2(nd[4 * i + 2], nd[4 * i + 3]), fma2(eu, kk[i], fc));
+                const float2 n2 = add2(make_float2(nd[4 * ib], nd[4 * ib + 1]), fma2(eu, vv[ib], ga));
+                const float2 d2 = add2(make_float2(nd[4 * ib + 2], nd[4 * ib + 3]), fma2(eu, kk[ib], gc));
+                nd[4 * i + 0] = n1.x;
+                nd[4 * i + 1] = n1.y;
+                nd[4 * i + 2] = d1.x;
+                nd[4 * i + 3] = d1.y;
+                nd[4 * ib + 0] = n2.x;
+                nd[4 * ib + 1] = n2.y;
+                nd[4 * ib + 2] = d2.x;
+                nd[4 * ib + 3] = d2.y;
+            }
             fa = fma2(alpha, fa, vv[i]);
             fc = fma2(alpha, fc, kk[i]);
-        }
-        float2 ga = f2(0.0f), gc = f2(0.0f);
-#pragma unroll
-        for (int i = kL - 1; i >= 0; --i) {
-            const float2 n2 = add2(make_float2(nd[4 * i], nd[4 * i + 1]), fma2(eu, vv[i], ga));
-            const float2 d2 = add2(make_float2(nd[4 * i + 2], nd[4 * i + 3]), fma2(eu, kk[i], gc));
-            nd[4 * i + 0] = n2.x;
-            nd[4 * i + 1] = n2.y;
-            nd[4 * i + 2] = d2.x;
-            nd[4 * i + 3] = d2.y;
-            ga = fma2(alpha, ga, vv[i]);
-            gc = fma2(alpha, gc, kk[i]);
+            ga = fma2(alpha, ga, vv[ib]);
+            gc = fma2(alpha, gc, kk[ib]);
         }
         tmem_st32(tmem + h * 32, nd);
-        Fh[h] = make_float4(fa.x, fa.y, fc.x, fc.y);
-        Gh[h] = make_float4(ga.x, ga.y, gc.x, gc.y);
+        Fh[st] = make_float4(fa.x, fa.y, fc.x, fc.y);
+        Gh[st] = make_float4(ga.x, ga.y, gc.x, gc.y);
     }
 
     // ---- 3a. warp maximum (the reference of the warp's sums) and the chunk's
@@ -353,12 +388,28 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     if (cq == 0) S.wmax[j][warp] = mx;  // -inf for a warp wholly past T
     const float2 mref = make_float2(mx.x == -INFINITY ? 0.0f : mx.x, mx.y == -INFINITY ? 0.0f : mx.y);
     float2 eh[kH];
-    auto scale4 = [](float2 e, float4 v) { return make_float4(v.x * e.x, v.y * e.y, v.z * e.x, v.w * e.y); };
+    auto scale4 = [](float2 e, float4 v) {
+        const float2 a = mul2(e, lo2(v)), c = mul2(e, hi2(v));
+        return make_float4(a.x, a.y, c.x, c.y);
+    };
 #pragma unroll
-    for (int h = 0; h < kH; ++h) {
-        eh[h] = ex2(mul2(add2(Mh[h], make_float2(-mref.x, -mref.y)), f2(kLog2e)));
-        Fh[h] = scale4(eh[h], Fh[h]);  // sub-chunk totals on the warp reference
-        Gh[h] = scale4(eh[h], Gh[h]);
+    for (int st = 0; st < kH; ++st) {
+        eh[st] = ex2(mul2(add2(Mh[st], make_float2(-mref.x, -mref.y)), f2(kLog2e)));
+        Fh[st] = scale4(eh[st], Fh[st]);  // sub-chunk totals on the warp reference
+        Gh[st] = scale4(eh[st], Gh[st]);
+    }
+    if (ROT) {
+        // into natural sub-chunk order (each thread reads back its own entries)
+#pragma unroll
+        for (int st = 0; st < kH; ++st) {
+            X2.a[(st + rot) & (kH - 1)][tid] = Fh[st];
+            X2.b[(st + rot) & (kH - 1)][tid] = Gh[st];
+        }
+#pragma unroll
+        for (int h = 0; h < kH; ++h) {
+            Fh[h] = X2.a[h][tid];
+            Gh[h] = X2.b[h][tid];
+        }
     }
     // chunk totals: forward at the chunk's end, backward at its start
     float4 Fi = Fh[0], Gi = Gh[kH - 1];
@@ -371,11 +422,11 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     // ---- 3b. scans: warp, CTA, cluster ------------------------------------------
 #pragma unroll
     for (int e = 0; (kNP << e) < 32; ++e) {
-        const float2 m = S.tab[1 << e][j];  // a^(32 * 2^e)
-        float4 o = shfl_up4(Fi, kNP << e, 32);
-        if (cq >= (1 << e)) Fi = fma4(m, o, Fi);
-        o = shfl_down4(Gi, kNP << e, 32);
-        if (cq + (1 << e) < kCPW) Gi = fma4(m, o, Gi);
+        // a^(32 * 2^e), zero where the partner lane lies outside the warp's chunks
+        const float2 m = S.tab[1 << e][j];
+        const float2 mf = cq >= (1 << e) ? m : f2(0.0f), mb = cq + (1 << e) < kCPW ? m : f2(0.0f);
+        Fi = fma4(mf, shfl_up4(Fi, kNP << e, 32), Fi);
+        Gi = fma4(mb, shfl_down4(Gi, kNP << e, 32), Gi);
     }
     float4 X = shfl_up4(Fi, kNP, 32), Y = shfl_down4(Gi, kNP, 32);
     if (cq == 0) X = zero4();
@@ -516,15 +567,34 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     // carries into the chunk: from the left at its start, from the right at its end
     float2 Ac = fma2(slw, lo2(X), fma2(slF, lo2(XW), mul2(kf, cs_af)));
     float2 Cc = fma2(slw, hi2(X), fma2(slF, hi2(XW), mul2(kf, cs_cf)));
-    // carries from the right into each sub-chunk: B_3 = the chunk's, then
-    // B_{h-1} = a^8 B_h + sub-chunk h's backward total
-    float2 Bs[kH], Ds[kH];
-    Bs[kH - 1] = fma2(slw, lo2(Y), fma2(slB, lo2(YW), mul2(kb, cs_bb)));
-    Ds[kH - 1] = fma2(slw, hi2(Y), fma2(slB, hi2(YW), mul2(kb, cs_db)));
+    // carries into each sub-chunk, natural order: from the right, B_3 = the
+    // chunk's and B_{h-1} = a^8 B_h + G_h; from the left, A_0 = the chunk's
+    // and A_{h+1} = a^8 A_h + F_h (sub-chunk totals on the column reference)
+    float4 Lc[kH], Rc[kH];  // (A.xy, C.xy), (B.xy, D.xy)
+    {
+        float2 Bq = fma2(slw, lo2(Y), fma2(slB, lo2(YW), mul2(kb, cs_bb)));
+        float2 Dq = fma2(slw, hi2(Y), fma2(slB, hi2(YW), mul2(kb, cs_db)));
 #pragma unroll
-    for (int h = kH - 1; h > 0; --h) {
-        Bs[h - 1] = fma2(slw, lo2(Gh[h]), mul2(a8, Bs[h]));
-        Ds[h - 1] = fma2(slw, hi2(Gh[h]), mul2(a8, Ds[h]));
+        for (int h = kH - 1; h >= 0; --h) {
+            Rc[h] = make_float4(Bq.x, Bq.y, Dq.x, Dq.y);
+            if (h > 0) {
+                Bq = fma2(slw, lo2(Gh[h]), mul2(a8, Bq));
+                Dq = fma2(slw, hi2(Gh[h]), mul2(a8, Dq));
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < kH; ++h) {
+            Lc[h] = make_float4(Ac.x, Ac.y, Cc.x, Cc.y);
+            Ac = fma2(slw, lo2(Fh[h]), mul2(a8, Ac));
+            Cc = fma2(slw, hi2(Fh[h]), mul2(a8, Cc));
+        }
+    }
+    if (ROT) {
+#pragma unroll
+        for (int h = 0; h < kH; ++h) {
+            X2.a[h][tid] = Lc[h];
+            X2.b[h][tid] = Rc[h];
+        }
     }
     float2 pw[kL];
     pw[0] = f2(1.0f);
@@ -533,18 +603,21 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     tmem_wait_st();
     char* tout = smem;
 #pragma unroll
-    for (int h = 0; h < kH; ++h) {
+    for (int st = 0; st < kH; ++st) {
+        const int h = ROT ? (st + rot) & (kH - 1) : st;
         float nd[32];
         tmem_ld32(tmem + h * 32, nd);
-        const float2 sh = mul2(slw, eh[h]);
+        const float2 sh = mul2(slw, eh[st]);
+        const float4 L4 = ROT ? X2.a[h][tid] : Lc[st], R4 = ROT ? X2.b[h][tid] : Rc[st];
+        const float2 Ah = lo2(L4), Ch = hi2(L4), Bh = lo2(R4), Dh = hi2(R4);
         const int rowoff = (q * kH + h) * RB + j * PB;
 #pragma unroll
         for (int i = 0; i < kL; ++i) {
             const int o = rowoff + i * SUB;
             const float2 nn = make_float2(nd[4 * i], nd[4 * i + 1]);
             const float2 dd = make_float2(nd[4 * i + 2], nd[4 * i + 3]);
-            const float2 num = fma2(sh, nn, fma2(pw[i], Ac, mul2(pw[kL - 1 - i], Bs[h])));
-            float2 den = fma2(sh, dd, fma2(pw[i], Cc, mul2(pw[kL - 1 - i], Ds[h])));
+            const float2 num = fma2(sh, nn, fma2(pw[i], Ah, mul2(pw[kL - 1 - i], Bh)));
+            float2 den = fma2(sh, dd, fma2(pw[i], Ch, mul2(pw[kL - 1 - i], Dh)));
             if (GATE) {
                 // read before the result overwrites the first slot
                 const float2 g = make_float2(lds_f32(g0 + o), lds_f32(g1 + o));
@@ -552,9 +625,6 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
             }
             Io<IO>::st_pair(tout + o, mul2(num, rcp(den)));
         }
-        // carry from the left into the next sub-chunk
-        Ac = fma2(slw, lo2(Fh[h]), mul2(a8, Ac));
-        Cc = fma2(slw, hi2(Fh[h]), mul2(a8, Cc));
     }
     // results leave by TMA stores: lane i of warp 0 stores sub-tile i in boxes
     // of 256 strided tokens, clipped at T by the tensor map

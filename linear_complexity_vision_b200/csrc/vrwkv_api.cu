@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <mutex>
 #include <string>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -419,6 +420,7 @@ bool tma_chunk8_forced() {
 struct FastPlan {
     fast::Params p;
     bool tm;     // 32-token chunks with tensor-memory partial sums (biwkv_tm_kernel)
+    bool rot;    // tm: rotated sub-chunk order (conflict-free shared-memory rows)
     int layout;
     int ntiles;  // tiles per CTA (sources, doubled with Q-Shift)
     bool qs;
@@ -533,9 +535,9 @@ static_assert(kFastTcMax == fast::Cfg<kFastThreads8, 8>::kTcMax, "one tile geome
 // The 32-token tensor-memory kernel: a cluster per column as in the 8-channel
 // kernel.  Sets *fell_back when the shape cannot be co-scheduled or more
 // than four CTAs would share an SM (their tensor memory would not fit).
-template <typename IO, int LAYOUT, bool QS>
+template <typename IO, int LAYOUT, bool QS, bool ROT>
 vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
-    auto kern = tm32::biwkv_tm_kernel<IO, LAYOUT, QS>;
+    auto kern = tm32::biwkv_tm_kernel<IO, LAYOUT, QS, ROT>;
     static std::atomic<int> granted{0};
     cudaError_t e = ensure_smem(kern, granted, pl.smem);
     if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
@@ -581,16 +583,25 @@ vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back)
     return ok();
 }
 
+template <typename IO, bool ROT>
+vrwkv_status dispatch_tm_rot(const FastPlan& pl, cudaStream_t s, bool* fb) {
+    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
+    case fast::kKV * 2 + 0: return launch_tm<IO, fast::kKV, false, ROT>(pl, s, fb);
+    case fast::kKV * 2 + 1: return launch_tm<IO, fast::kKV, true, ROT>(pl, s, fb);
+    case fast::kRKV * 2 + 0: return launch_tm<IO, fast::kRKV, false, ROT>(pl, s, fb);
+    case fast::kRKV * 2 + 1: return launch_tm<IO, fast::kRKV, true, ROT>(pl, s, fb);
+    case fast::kX * 2 + 0: return launch_tm<IO, fast::kX, false, ROT>(pl, s, fb);
+    default: return launch_tm<IO, fast::kX, true, ROT>(pl, s, fb);
+    }
+}
+
 template <typename IO>
 vrwkv_status dispatch_tm(const FastPlan& pl, cudaStream_t s, bool* fb) {
-    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
-    case fast::kKV * 2 + 0: return launch_tm<IO, fast::kKV, false>(pl, s, fb);
-    case fast::kKV * 2 + 1: return launch_tm<IO, fast::kKV, true>(pl, s, fb);
-    case fast::kRKV * 2 + 0: return launch_tm<IO, fast::kRKV, false>(pl, s, fb);
-    case fast::kRKV * 2 + 1: return launch_tm<IO, fast::kRKV, true>(pl, s, fb);
-    case fast::kX * 2 + 0: return launch_tm<IO, fast::kX, false>(pl, s, fb);
-    default: return launch_tm<IO, fast::kX, true>(pl, s, fb);
+    // the rotated order is only ever planned for 16-byte rows (bfloat16)
+    if constexpr (std::is_same<IO, __nv_bfloat16>::value) {
+        if (pl.rot) return dispatch_tm_rot<IO, true>(pl, s, fb);
     }
+    return dispatch_tm_rot<IO, false>(pl, s, fb);
 }
 
 template <typename IO>
@@ -612,9 +623,24 @@ int fast_smem(int ntiles, int tile_bytes, int kl) {
 // Shared memory of a tensor-memory kernel CTA: its tiles (one extra for the
 // gate factor without Q-Shift), the scratch block, and at least the floor
 // that keeps a fifth CTA off an SM.
-int tm_smem(bool gate, bool qs, int ntiles, int tile_bytes) {
+int tm_smem(bool gate, bool qs, int ntiles, int tile_bytes, bool rot) {
     const int nta = gate && !qs ? ntiles + 1 : ntiles;
-    return std::max(nta * tile_bytes + (int)sizeof(tm32::Scratch) + 128, tm32::kSmemFloor);
+    const int stash = rot ? (int)sizeof(tm32::Stash) : 0;
+    return std::max(nta * tile_bytes + (int)sizeof(tm32::Scratch) + stash + 128, tm32::kSmemFloor);
+}
+
+// VRWKV_TM_ROT=0 keeps the tensor-memory kernel's sub-chunks in natural order
+// (diagnostics and tests).
+bool tm_rot_disabled() {
+    const char* e = getenv("VRWKV_TM_ROT");
+    return e && e[0] == '0' && e[1] == 0;
+}
+
+// Rotated sub-chunk order where it pays: 16-byte token rows (bfloat16) and
+// a stash that still leaves room for four CTAs per SM.
+bool tm_rot_wanted(bool gate, bool qs, int ntiles, int tile_bytes, int es) {
+    if (tm_rot_disabled() || es != 2) return false;
+    return 4 * (tm_smem(gate, qs, ntiles, tile_bytes, true) + 1024) <= 228 * 1024;
 }
 
 // Plan the TMA path; returns false when the problem is outside its limits
@@ -711,7 +737,8 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     // arrive as zeros)
     p.box_bytes = (pl.qs ? (p.W / fast::kL) * p.rows : TcMax / fast::kL) * RB;
     pl.nt = pl.tm ? tm32::kThreads : (pl.kl == 16 ? kFastThreads16 : kFastThreads8);
-    pl.smem = pl.tm ? tm_smem(gate, pl.qs, ntiles, p.tile_bytes) : fast_smem(ntiles, p.tile_bytes, pl.kl);
+    pl.rot = pl.tm && tm_rot_wanted(gate, pl.qs, ntiles, p.tile_bytes, es);
+    pl.smem = pl.tm ? tm_smem(gate, pl.qs, ntiles, p.tile_bytes, pl.rot) : fast_smem(ntiles, p.tile_bytes, pl.kl);
     if (pl.smem > 227 * 1024) return false;
     const CUtensorMapDataType dt =
         dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;

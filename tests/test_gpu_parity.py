@@ -270,9 +270,13 @@ TM_CASES = [
 ]
 
 
+@pytest.mark.parametrize("rot", ["rot", "natural"])
 @pytest.mark.parametrize("case", TM_CASES, ids=lambda c: "_".join(map(str, c)))
-def test_tm_kernel_shapes(vk, oracle_mod, case, monkeypatch):
+def test_tm_kernel_shapes(vk, oracle_mod, case, rot, monkeypatch):
+    # "rot": the rotated sub-chunk order wherever it is planned (bfloat16
+    # rows, room for the stash); "natural": sub-chunks in order everywhere
     monkeypatch.setenv("VRWKV_FORWARD", "tm")
+    monkeypatch.setenv("VRWKV_TM_ROT", "1" if rot == "rot" else "0")
     call, B, H, W, C, dt, gamma = case
     wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000, gamma=gamma)
     run_fused(vk, oracle_mod, wl)
