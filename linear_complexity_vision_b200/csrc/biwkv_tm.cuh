@@ -21,11 +21,12 @@
 // 128 columns, so four CTAs fill an SM's 512; the host keeps at most four
 // resident (a shared-memory floor) so an allocation never waits.
 //
-// The gate factor e^{-r} of a token is parked in the two tile slots the
-// thread has just read to make r (r's own and shifted r's; without Q-Shift,
-// r's slot and one extra tile), so no shared-memory array of gate factors
-// is needed; the result later goes into the first slot.  Every slot is read
-// and written by the one thread that owns the token.
+// The gate factor e^{-r} of a token is parked in two tile slots the thread
+// has just read (r's own and shifted r's; without Q-Shift, r's and k's, or
+// r's and one extra tile when one x feeds r, k and v), so no shared-memory
+// array of gate factors is needed; the result later goes into the first
+// slot.  Every slot is read and written by the one thread that owns the
+// token.
 //
 // A CTA covers 1024 tokens x 8 channels; longer columns use a cluster of up
 // to 8 CTAs along T (T <= 8192) exchanging their aggregates through
@@ -179,10 +180,12 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     extern __shared__ __align__(128) char smem_raw[];
     char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
     // The gate factor's two halves are parked in r's slot and, with Q-Shift,
-    // in shifted r's slot (both read to make r); without Q-Shift in one
-    // extra tile, so no slot another value still needs is overwritten.
-    constexpr int NTA = GATE && !QS ? NTILE + 1 : NTILE;
-    constexpr int G1 = QS ? 2 * SR + 1 : NTILE;  // tile of the second half
+    // in shifted r's slot (both read to make r); without Q-Shift in k's slot
+    // (separate r, k, v) or in one extra tile (one x), so no slot another
+    // value still needs is overwritten.
+    constexpr bool G1_IN_K = GATE && !QS && LAYOUT == kRKV;
+    constexpr int NTA = GATE && !QS && !G1_IN_K ? NTILE + 1 : NTILE;
+    constexpr int G1 = QS ? 2 * SR + 1 : (G1_IN_K ? SK : NTILE);  // tile of the second half
     Scratch& S = *reinterpret_cast<Scratch*>(smem + NTA * p.tile_bytes);
     Stash& X2 = *reinterpret_cast<Stash*>(smem + NTA * p.tile_bytes + sizeof(Scratch));  // ROT only
 
@@ -309,7 +312,10 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
                 if (GATE) r = lds_pair<IO>(tR, o);
             }
             if (GATE) {
-                const float2 g = ex2(mul2(r, f2(-kLog2e)));
+                float2 g = ex2(mul2(r, f2(-kLog2e)));
+                // in k's slot the second half must follow the read of k, which
+                // it does not depend on: tie it to k (no instruction)
+                if (G1_IN_K) asm volatile("" : "+f"(g.y) : "f"(k.x), "f"(k.y));
                 sts_f32(g0 + o, g.x);
                 sts_f32(g1 + o, g.y);
             }

@@ -138,17 +138,19 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
 
 // 32 consecutive float32 columns of one tensor-memory lane per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    // load and wait in one statement: no use of v can be scheduled between
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
           "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
           "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
           "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        : "r"(taddr)
+        : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ Params p) {
@@ -537,6 +539,362 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 }  // namespace pair
+
+// ---------------------------------------------------------------------------
+// The three token projections of the spatial-mix block with the Q-Shift mix
+// as the A operand's producer ("Vision-RWKV Backbone", Overall Architecture,
+// eq. 1: R, K, V = (mu x + (1 - mu) x-dagger) W, x-dagger per
+// Quad-Directional Token Shift, eq. 9).  Same CTA-pair tiles and pipeline as
+// gemm_tc2_kernel, plus:
+//  * per stage, x and its Q-Shifted copy arrive by TMA from x's image view
+//    (C, W, H, B): the shifted box is the same box displaced by +-s along w
+//    or h, and TMA's zero fill is Q-Shift's border; a 64-channel K block lies
+//    in one channel group, so one displacement serves the whole box;
+//  * four groups of four mix warps, one per stage, turn x into the mix in
+//    place, each thread one 128-byte row (the 128-byte swizzle permutes
+//    16-byte chunks within a row, and the mix is element-wise, so chunk c of
+//    a row pairs with chunk c of the shifted row and with mu of its logical
+//    channels), with the
+//    rounding of the stand-alone mix kernel (mu x and (1 - mu) x-dagger, each
+//    rounded, then their sum): the A operand is the staged mix bit for bit;
+//  * the leader's "full" barrier waits for both CTAs' mixes as well as the
+//    B bytes; tiles run M block by M block over the three projections, so
+//    the x tiles of one M block are read from HBM once.
+// The mixed tokens never go to HBM.
+// ---------------------------------------------------------------------------
+namespace qsmix {
+
+using pair::BM;
+using pair::BN;
+using pair::BK;
+using pair::kHalf;
+constexpr int kStages = 4;
+constexpr int A_BYTES = kHalf * BK * 2;  // 16 KB: 128 rows x 64 channels
+constexpr int B_BYTES = kHalf * BK * 2;
+constexpr int kMixGroups = kStages;          // mix group g owns stage g (stages in flight: all)
+constexpr int kMixGroupThreads = 128;        // one thread per row of a CTA's A tile
+constexpr int kThreadsQ = 192 + kMixGroups * kMixGroupThreads;  // producer, MMA, 4 epilogue, 16 mix warps
+constexpr int kMaxC = 1024;                  // mu of three projections in shared memory
+
+struct Params {
+    CUtensorMap mx;     // x as (C, W, H, B): box (64, bw, bh, 1) = 128 tokens, 128-byte swizzle
+    CUtensorMap mb[3];  // Wt of each projection as (K, N): box (64, 128), 128-byte swizzle
+    const float* mu[3];
+    __nv_bfloat16* d[3];
+    int M, N, K;        // M = B T tokens, N = K = C
+    int T, W;
+    int s;              // shift
+    QsBounds g;
+    int ng;             // shifted groups (4, or 2 for the bidirectional shift)
+    int nproj;
+    unsigned int* err;
+};
+
+struct alignas(1024) Smem {
+    uint8_t a[kStages][A_BYTES];   // x, then the mix in place: the MMA's A operand
+    uint8_t b[kStages][B_BYTES];
+    uint8_t xs[kStages][A_BYTES];  // the Q-Shifted x
+    float mu[3][kMaxC];
+    float om[3][kMaxC];  // 1 - mu, rounded once
+    unsigned long long full[kStages], empty[kStages], xfull[kStages];
+    unsigned long long tfull[kAcc], tempty[kAcc];
+    unsigned long long drain;
+    unsigned tmem_base;
+    int abort;
+    int mixok[kMixGroups];  // each mix group's verdict on its current stage
+};
+
+// The channel group's displacement (dw, dh) of a K block; 4: copied.
+__device__ __forceinline__ int k_group(int k0, const Params& p) {
+    int grp = qs_group(k0, p.g);
+    return grp >= p.ng ? 4 : grp;
+}
+
+__device__ __forceinline__ bool mbar_test_cluster(unsigned long long* bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(fast::smem_u32(bar)), "r"(parity), "r"(100000u)
+        : "memory");
+    return ok != 0;
+}
+// Bounded cluster-scope wait (the leader's full barrier takes the other
+// CTA's release arrivals).
+__device__ __forceinline__ bool wait_phase_cluster(unsigned long long* bar, unsigned parity, volatile int* abort,
+                                                   unsigned* err) {
+    if (mbar_test_cluster(bar, parity)) return true;
+    const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+    while (!mbar_test_cluster(bar, parity)) {
+        if (*abort) return false;
+        if (fast::global_ns() - t0 > lim) {
+            atomicOr(err, kErrFlag);
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+// named barrier 1 + g of mix group g
+__device__ __forceinline__ void group_sync(int g) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(kMixGroupThreads) : "memory");
+}
+
+// (M block, projection, N block) of tile t: the projections of one M block
+// are consecutive, so concurrent clusters share its x tiles through L2.
+struct Tile {
+    int mb, proj, nb;
+};
+__device__ __forceinline__ Tile tile_of(int t, int nt, int nproj) {
+    Tile r;
+    r.mb = t / (nt * nproj);
+    const int rem = t - r.mb * nt * nproj;
+    r.proj = rem / nt;
+    r.nb = rem - r.proj * nt;
+    return r;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsQ, 1)
+    gemm_qs2_kernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(1024) char smem_raw[];
+    Smem& S = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (fast::smem_u32(smem_raw) & 1023u)) & 1023u));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = pair::cluster_rank();
+    const bool leader = rank == 0;
+    const int nt = (p.N + BN - 1) / BN, mt = (p.M + BM - 1) / BM;
+    const int ntiles = nt * mt * p.nproj, nk = (p.K + BK - 1) / BK;
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    volatile int* abort = &S.abort;
+
+    for (int e = tid; e < p.nproj * p.K; e += kThreadsQ) {
+        const int pj = e / p.K, c = e - pj * p.K;
+        const float m = __ldg(p.mu[pj] + c);
+        S.mu[pj][c] = m;
+        S.om[pj][c] = __fsub_rn(1.0f, m);
+    }
+    if (tid == 0) {
+        for (int st = 0; st < kStages; ++st) {
+            // the leader's full barrier: its producer's expect_tx and both mixes
+            fast::mbar_init(&S.full[st], 3);
+            fast::mbar_init(&S.empty[st], 1);
+            fast::mbar_init(&S.xfull[st], 1);
+        }
+        for (int a = 0; a < kAcc; ++a) {
+            fast::mbar_init(&S.tfull[a], 1);
+            fast::mbar_init(&S.tempty[a], 8);  // the epilogue warps of both CTAs
+        }
+        fast::mbar_init(&S.drain, 1);
+        S.abort = 0;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         fast::smem_u32(&S.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    pair::cluster_sync_all();  // both CTAs' barriers exist before any remote signal
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer: x and its shift into this CTA's stage (local barrier),
+            // this CTA's half of Bt (the leader's barrier)
+            int it = 0;
+            int last_par[kStages];
+            for (int st = 0; st < kStages; ++st) last_par[st] = -1;
+            for (int t = cid; t < ntiles && !*abort; t += ncl) {
+                const Tile tl = tile_of(t, nt, p.nproj);
+                const int m_cta = tl.mb * BM + (int)rank * kHalf;  // this CTA's first token
+                const int bidx = m_cta / p.T, tok = m_cta - bidx * p.T;
+                const int hrow = tok / p.W, w0 = tok - hrow * p.W;
+                const int n0 = tl.nb * BN + (int)rank * kHalf;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int st = it % kStages;
+                    const unsigned ph = (it / kStages) & 1;
+                    if (!wait_phase(&S.empty[st], ph ^ 1u, abort, p.err)) break;
+                    const int k0 = kb * BK;
+                    const int grp = k_group(k0, p);
+                    const uint32_t lbar = fast::mapa_u32(fast::smem_u32(&S.full[st]), 0);
+                    if (leader) fast::mbar_expect_tx(&S.full[st], 2 * B_BYTES);
+                    fast::mbar_expect_tx(&S.xfull[st], (unsigned)(grp < 4 ? 2 * A_BYTES : A_BYTES));
+                    fast::tma_load_4d(S.a[st], &p.mx, k0, w0, hrow, bidx, &S.xfull[st]);
+                    if (grp < 4) {
+                        const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
+                        const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
+                        fast::tma_load_4d(S.xs[st], &p.mx, k0, w0 + dw, hrow + dh, bidx, &S.xfull[st]);
+                    }
+                    pair::tma_load_2d_pair(S.b[st], &p.mb[tl.proj], k0, n0, lbar);
+                    last_par[st] = (int)ph;
+                }
+            }
+            if (*abort) {
+                // let this CTA's copies land before it leaves
+                for (int st = 0; st < kStages; ++st) {
+                    if (last_par[st] < 0) continue;
+                    const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+                    while (!mbar_test(&S.xfull[st], (unsigned)last_par[st]) && fast::global_ns() - t0 <= lim) {
+                    }
+                    if (leader)
+                        while (!mbar_test_cluster(&S.full[st], (unsigned)last_par[st]) &&
+                               fast::global_ns() - t0 <= lim) {
+                        }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // MMA issuer (the pair's leader)
+            int it = 0, lt = 0;
+            bool issued = false;
+            for (int t = cid; t < ntiles && !*abort; t += ncl, ++lt) {
+                const int acc = lt & 1;
+                const unsigned aph = (lt >> 1) & 1;
+                if (!wait_phase(&S.tempty[acc], aph ^ 1u, abort, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int st = it % kStages;
+                    const unsigned ph = (it / kStages) & 1;
+                    if (!wait_phase_cluster(&S.full[st], ph, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(fast::smem_u32(S.a[st]));
+                    const uint64_t bd = sw128_desc(fast::smem_u32(S.b[st]));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        pair::mma_pair(d_tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k),
+                                       (kb > 0 || k > 0) ? 1u : 0u);
+                    issued = true;
+                    pair::commit_pair(&S.empty[st]);
+                }
+                if (!ok) break;
+                pair::commit_pair(&S.tfull[acc]);
+            }
+            if (*abort && issued) {
+                tc_commit(&S.drain);
+                const unsigned long long t0 = fast::global_ns(), lim = fast::g_vrwkv_wait_ns;
+                while (!mbar_test(&S.drain, 0) && fast::global_ns() - t0 <= lim) {
+                }
+            }
+        }
+    } else if (warp < 6) {
+        // epilogue: this CTA's 128 rows of the pair's tile
+        const int quad = warp & 3;
+        const uint32_t leader_tempty[2] = {fast::mapa_u32(fast::smem_u32(&S.tempty[0]), 0),
+                                           fast::mapa_u32(fast::smem_u32(&S.tempty[1]), 0)};
+        int lt = 0;
+        for (int t = cid; t < ntiles; t += ncl, ++lt) {
+            const int acc = lt & 1;
+            const unsigned aph = (lt >> 1) & 1;
+            if (!wait_phase(&S.tfull[acc], aph, abort, p.err)) break;
+            tc_fence_after();
+            const Tile tl = tile_of(t, nt, p.nproj);
+            const int m0 = tl.mb * BM, n0 = tl.nb * BN;
+            const int row = m0 + (int)rank * kHalf + quad * 32 + lane;
+            const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+            __nv_bfloat16* D = p.d[tl.proj];
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tbase + (uint32_t)(c * 32), v);
+                const int col = n0 + c * 32;
+                if (row < p.M && col + 32 <= p.N) {
+                    uint32_t w16[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]),
+                                                                       __uint_as_float(v[2 * e + 1]));
+                        w16[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    uint4* d4 = reinterpret_cast<uint4*>(D + (size_t)row * p.N + col);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d4[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) pair::arrive_remote(leader_tempty[acc]);
+        }
+    } else {
+        // mix warps: group g (four warps) mixes every stage-g tile; thread r of
+        // the group owns row r of this CTA's 128-row A tile.  The groups work
+        // on their stages concurrently, so a stage's mix latency overlaps the
+        // MMAs of the others.
+        const int gi = (warp - 6) >> 2;
+        const int r = tid - 192 - gi * kMixGroupThreads;
+        const uint32_t rowoff = (uint32_t)r * 128u;
+        int it = 0;
+        bool go = true;
+        for (int t = cid; t < ntiles && go; t += ncl) {
+            const Tile tl = tile_of(t, nt, p.nproj);
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int st = it % kStages;
+                if (st != gi) continue;
+                const unsigned ph = (it / kStages) & 1;
+                if (r == 0) S.mixok[gi] = wait_phase(&S.xfull[st], ph, abort, p.err) ? 1 : 0;
+                group_sync(gi);
+                if (!S.mixok[gi]) {
+                    go = false;
+                    break;
+                }
+                const int k0 = kb * BK;
+                const bool shifted = k_group(k0, p) < 4;
+                const uint8_t* xa = S.a[st] + rowoff;
+                const uint8_t* xd = (shifted ? S.xs[st] : S.a[st]) + rowoff;
+                const float* mu = &S.mu[tl.proj][k0];
+                const float* om = &S.om[tl.proj][k0];
+#pragma unroll 4
+                for (int c = 0; c < BK / 8; ++c) {
+                    const uint32_t off = (uint32_t)((c ^ (r & 7)) * 16);  // chunk c's place in the swizzled row
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xa + off);
+                    const uint4 dv = *reinterpret_cast<const uint4*>(xd + off);
+                    const float4 m0 = *reinterpret_cast<const float4*>(mu + 8 * c);
+                    const float4 m1 = *reinterpret_cast<const float4*>(mu + 8 * c + 4);
+                    const float4 o0 = *reinterpret_cast<const float4*>(om + 8 * c);
+                    const float4 o1 = *reinterpret_cast<const float4*>(om + 8 * c + 4);
+                    const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                    const float ov[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // mu x + (1 - mu) x-dagger, each operation rounded on its own
+                        // (no contraction into a multiply-add)
+                        const float lo = __fadd_rn(__fmul_rn(mv[2 * e], __uint_as_float(xw[e] << 16)),
+                                                   __fmul_rn(ov[2 * e], __uint_as_float(dw[e] << 16)));
+                        const float hi = __fadd_rn(__fmul_rn(mv[2 * e + 1], __uint_as_float(xw[e] & 0xffff0000u)),
+                                                   __fmul_rn(ov[2 * e + 1], __uint_as_float(dw[e] & 0xffff0000u)));
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+                        ow[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    *reinterpret_cast<uint4*>(const_cast<uint8_t*>(xa) + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+                // the mix is read by the tensor cores (async proxy)
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                group_sync(gi);
+                if (r == 0) pair::arrive_remote(fast::mapa_u32(fast::smem_u32(&S.full[st]), 0));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    pair::cluster_sync_all();  // no CTA leaves while its pair may still signal it
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
+}  // namespace qsmix
 
 // W (K x N, row-major) -> Wt (N x K, row-major), 32 x 32 tiles through
 // shared memory; the GEMM reads its B operand K-major.

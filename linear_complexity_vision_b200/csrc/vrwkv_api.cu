@@ -310,6 +310,101 @@ vrwkv_status gemm_project(const void* X, const void* W, void* D, int M, int N, i
     return cuda_status(cudaGetLastError(), "gemm_tc_kernel launch");
 }
 
+// VRWKV_BLOCK_FUSED=1 projects R, K, V with the fused Q-Shift GEMM instead of
+// staging the three mixes in HBM.  Off by default: measured on the B200 at
+// B = 8, 64 x 64, C = 1024 the fused block takes 585 us against 502 us
+// staged.  The fused A producer mixes every x tile once per N tile (four
+// times per projection at C = 1024), and that element-wise work (about six
+// instructions per element) outgrows what the SM issues beside the MMAs;
+// staged, each element is mixed once per projection.
+bool block_fused_wanted() {
+    const char* e = getenv("VRWKV_BLOCK_FUSED");
+    return e && e[0] == '1';
+}
+
+// R, K, V = mix_{r,k,v}(x) W_{r,k,v} in one launch of the fused Q-Shift GEMM
+// (bfloat16).  Returns false (nothing launched) when the shape is outside its
+// limits: C a multiple of 256 and at most 1024, 64-channel K blocks inside
+// one channel group, 128-token tiles of whole image rows (or whole 128-token
+// pieces of one row) inside one image, all three mu given.
+bool gemm_qs_project(const void* x, const void* const* wts, const float* const* mus, void* const* dst,
+                     int B, int T, int C, const vrwkv_qshift_params* qs, char* wt_slots, size_t wslot,
+                     cudaStream_t s, vrwkv_status* st) {
+    using namespace tcgemm::qsmix;
+    if (!mus[0] || !mus[1] || !mus[2]) return false;
+    if (C % 256 != 0 || C > kMaxC || T % 128 != 0) return false;
+    const int W = qs->W, H = qs->H;
+    if (!((W <= 128 && 128 % W == 0) || W % 128 == 0)) return false;
+    const QsBounds g = qs_bounds(C, qs->gamma);
+    if (!bounds_multiple_of(g, 64)) return false;
+    if (!aligned(x, 16)) return false;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    Params p;
+    {
+        const int bw = W <= 128 ? W : 128, bh = W <= 128 ? 128 / W : 1;
+        const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)B};
+        const cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)T * C * 2};
+        const cuuint32_t box[4] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, 1u};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (enc(&p.mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    for (int i = 0; i < 3; ++i) {
+        void* wt = wt_slots + i * wslot;
+        const dim3 grid((unsigned)((C + 31) / 32), (unsigned)((C + 31) / 32));
+        tcgemm::transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(wts[i]),
+                                                                      static_cast<__nv_bfloat16*>(wt), C, C);
+        const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)C};
+        const cuuint64_t strides[1] = {(cuuint64_t)C * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)tcgemm::BK, (cuuint32_t)tcgemm::pair::kHalf};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&p.mb[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wt, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+            *st = fail(VRWKV_ERR_UNSUPPORTED, "tensor map of a projection's B operand could not be encoded");
+            return true;
+        }
+        p.mu[i] = mus[i];
+        p.d[i] = static_cast<__nv_bfloat16*>(dst[i]);
+    }
+    {
+        vrwkv_status e0 = cuda_status(cudaGetLastError(), "transpose_kernel launch");
+        if (e0 != VRWKV_OK) {
+            *st = e0;
+            return true;
+        }
+    }
+    p.M = B * T;
+    p.N = C;
+    p.K = C;
+    p.T = T;
+    p.W = W;
+    p.s = qs->shift_pixel;
+    p.g = g;
+    p.ng = shifted_groups(qs);
+    p.nproj = 3;
+    p.err = device_error_word();
+    if (!p.err) {
+        *st = fail(VRWKV_ERR_CUDA, "cannot locate the device error word");
+        return true;
+    }
+    const int smem = (int)sizeof(Smem) + 1024;
+    static std::atomic<int> granted{0};
+    cudaError_t e = ensure_smem(gemm_qs2_kernel, granted, smem);
+    if (e != cudaSuccess) {
+        *st = cuda_status(e, "cudaFuncSetAttribute");
+        return true;
+    }
+    const int tiles = ((p.M + BM - 1) / BM) * (C / BN) * 3;
+    const int pairs = std::max(1, std::min(tiles, sm_count() / 2));
+    gemm_qs2_kernel<<<2 * pairs, kThreadsQ, smem, s>>>(p);
+    *st = cuda_status(cudaGetLastError(), "gemm_qs2_kernel launch");
+    return true;
+}
+
 // Workspace of vrwkv_spatial_mix_block: six (B, T, C) token buffers and the
 // four transposed weight matrices, each 256-byte aligned.
 size_t block_wt_slot(int C, vrwkv_dtype dtype) {
@@ -624,7 +719,9 @@ int fast_smem(int ntiles, int tile_bytes, int kl) {
 // gate factor without Q-Shift), the scratch block, and at least the floor
 // that keeps a fifth CTA off an SM.
 int tm_smem(bool gate, bool qs, int ntiles, int tile_bytes, bool rot) {
-    const int nta = gate && !qs ? ntiles + 1 : ntiles;
+    // one extra tile for the gate factor's second half when one x feeds r, k
+    // and v without Q-Shift (one tile); separate r, k, v park it in k's slot
+    const int nta = gate && !qs && ntiles == 1 ? ntiles + 1 : ntiles;
     const int stash = rot ? (int)sizeof(tm32::Stash) : 0;
     return std::max(nta * tile_bytes + (int)sizeof(tm32::Scratch) + stash + 128, tm32::kSmemFloor);
 }
@@ -1535,20 +1632,27 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     const void* wts[3] = {w_r, w_k, w_v};
     void* dst[3] = {bR, bK, bV};
     vrwkv_status qst = VRWKV_OK;
-    const bool walked = mus[0] && mus[1] && mus[2] &&
-                        launch_qs_mix<3>(x, sh, mus, B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
-                                         shifted_groups(qs), dtype, s, &qst);
-    if (walked && qst != VRWKV_OK) return qst;
-    if (!walked) {
+    // bfloat16: the mixes as the projections' A-operand producer (one fused
+    // launch, nothing staged in HBM) where the shape allows
+    const bool fused = dtype == VRWKV_BF16 && block_fused_wanted() && !gemm_single_cta_forced() &&
+                       gemm_qs_project(x, wts, mus, dst, B, T, C, qs, wts_t, wslot, s, &qst);
+    if (fused && qst != VRWKV_OK) return qst;
+    if (!fused) {
+        const bool walked = mus[0] && mus[1] && mus[2] &&
+                            launch_qs_mix<3>(x, sh, mus, B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
+                                             shifted_groups(qs), dtype, s, &qst);
+        if (walked && qst != VRWKV_OK) return qst;
+        if (!walked) {
+            for (int i = 0; i < 3; ++i) {
+                vrwkv_status st = shift_entry(x, sh[i], mus[i], B, qs->H, qs->W, C, qs->shift_pixel,
+                                              qs->gamma, shifted_groups(qs), dtype, stream);
+                if (st != VRWKV_OK) return st;
+            }
+        }
         for (int i = 0; i < 3; ++i) {
-            vrwkv_status st = shift_entry(x, sh[i], mus[i], B, qs->H, qs->W, C, qs->shift_pixel, qs->gamma,
-                                          shifted_groups(qs), dtype, stream);
+            vrwkv_status st = gemm_project(sh[i], wts[i], dst[i], M, C, C, dtype, wts_t + i * wslot, s);
             if (st != VRWKV_OK) return st;
         }
-    }
-    for (int i = 0; i < 3; ++i) {
-        vrwkv_status st = gemm_project(sh[i], wts[i], dst[i], M, C, C, dtype, wts_t + i * wslot, s);
-        if (st != VRWKV_OK) return st;
     }
     // sigma(R) (.) Bi-WKV(K, V) on the projected channels (Q-Shift already
     // applied before the projections), into t0

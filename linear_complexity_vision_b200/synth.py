@@ -108,6 +108,10 @@ class Workload:
             return ["r", "k", "v"]
         if self.call == "gate_qs_x":
             return ["x"]
+        if self.call == "gate":      # sigma(r) * Bi-WKV(k, v), no Q-Shift
+            return ["r", "k", "v"]
+        if self.call == "gate_x":    # one x feeds r, k and v, no Q-Shift
+            return ["x"]
         raise ValueError(self.call)
 
     def generate(self) -> dict:
@@ -118,7 +122,7 @@ class Workload:
                              self.dists[name])
         for name in ("w", "u"):
             out[name] = draw(self.seed, name, (self.C,), self.dists[name])
-        if self.call != "biwkv":
+        if self.call not in ("biwkv", "gate", "gate_x"):
             for name in ("mu_r", "mu_k", "mu_v"):
                 out[name] = draw(self.seed, name, (self.C,), ("uniform", 0.0, 1.0))
         return out

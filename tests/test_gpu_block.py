@@ -92,6 +92,42 @@ def test_block_parity(vk, oracle_mod, dt, B, H, W, C, gemm_path):
     assert vk.load_library().vrwkv_last_kernel().decode() == "spatial_mix_block"
 
 
+# The fused projection (VRWKV_BLOCK_FUSED=1: the Q-Shift mix as the GEMM's
+# A-operand producer, bfloat16) against the default staged path (the mixes
+# written to HBM by the mix kernel, then the plain GEMM): the fused mix
+# rounds like the mix kernel and the GEMM tiles are the same, so the block's
+# output is identical bit for bit.
+FUSED_CASES = [
+    # B, H, W, C, gamma, shift, mode
+    (2, 64, 64, 256, 0.25, 1, 0),    # 128-token tiles of two image rows
+    (1, 24, 16, 512, 0.25, 1, 0),    # M = 384: a half-filled last M block; W = 16: 8 rows per tile
+    (1, 8, 256, 256, 0.25, 1, 0),    # W = 256: a tile is half an image row
+    (2, 16, 8, 256, 0.125, 2, 0),    # copied channels 128..255, shift 2, W = 8
+    (1, 32, 32, 512, 0.25, 1, 1),    # bidirectional shift: the vertical groups pass through
+    (1, 16, 64, 1024, 0.25, 3, 0),   # C = 1024 (the largest fused C), shift 3
+]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_block_fused_projection_equals_staged(vk, case, monkeypatch):
+    import torch
+    B, H, W, C, gamma, shift, mode = case
+    x, mats, w, u, mus, g, b = _case(B, H, W, C, "bf16")
+    xt, _ = to_device(x, "bf16")
+    mt = [to_device(m, "bf16")[0] for m in mats]
+    wt, ut, gt, bt = (vec_f32(a)[0] for a in (w, u, g, b))
+    mut = [vec_f32(m)[0] for m in mus]
+    qs = vk.QShift(H, W, shift, gamma, *mut, mode=mode)
+    monkeypatch.delenv("VRWKV_GEMM_1CTA", raising=False)
+    monkeypatch.setenv("VRWKV_BLOCK_FUSED", "1")
+    fused = vk.spatial_mix_block(xt, mt, wt, ut, gt, bt, qs)
+    monkeypatch.delenv("VRWKV_BLOCK_FUSED")
+    staged = vk.spatial_mix_block(xt, mt, wt, ut, gt, bt, qs)
+    vk.device_status()
+    assert torch.isfinite(fused.float()).all()
+    assert torch.equal(fused, staged)
+
+
 def test_block_identity_weights_equal_layer_norm_of_core(vk):
     # W = I everywhere: the block is LayerNorm of vrwkv_spatial_gate's output
     import torch

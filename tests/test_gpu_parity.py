@@ -134,6 +134,13 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     if wl.call == "biwkv":
         out = vk.biwkv_fwd(dev["k"], dev["v"], dev["w"], dev["u"], workspace=ws)
         ks, vs, rs = ref["k"], ref["v"], None
+    elif wl.call == "gate":
+        out = vk.spatial_gate(dev["r"], dev["k"], dev["v"], dev["w"], dev["u"], workspace=ws)
+        ks, vs, rs = ref["k"], ref["v"], ref["r"]
+    elif wl.call == "gate_x":
+        x = dev["x"]
+        out = vk.spatial_gate(x, x, x, dev["w"], dev["u"], workspace=ws)
+        ks = vs = rs = ref["x"]
     else:
         qs = vk.QShift(H, W, s, g, dev.get("mu_r"), dev.get("mu_k"), dev.get("mu_v"))
         if wl.call == "qshift_biwkv":
@@ -267,6 +274,9 @@ TM_CASES = [
     ("gate_qs_x", 1, 64, 64, 128, "bf16", 0.125),  # copied channels 64..127
     ("gate_qs", 2, 64, 64, 32, "bf16", 0.25),      # r, k, v with Q-Shift: six tiles
     ("gate_qs_x", 1, 12, 16, 64, "bf16", 0.25),    # T = 192: one CTA, 6 of 32 chunks used
+    ("gate", 2, 1, 4096, 64, "bf16", 0.25),        # r, k, v without Q-Shift: gate in k's slots
+    ("gate", 1, 1, 3000, 32, "f32", 0.25),         # the same in float32, ragged last CTA
+    ("gate_x", 2, 1, 4096, 32, "bf16", 0.25),      # one x without Q-Shift: gate in an extra tile
 ]
 
 
@@ -358,6 +368,8 @@ EDGE = [
     ("qshift_biwkv", 2, 24, 24, 64, "f32"),  # W = 24: 8 rows of 24 per CTA
     ("biwkv", 2, 1, 4096, 16, "bf16"),      # 8 CTAs without Q-Shift
     ("biwkv", 3, 1, 257, 32, "f32"),        # one token into a second CTA
+    ("gate", 2, 1, 2048, 16, "bf16"),       # r, k, v without Q-Shift
+    ("gate_x", 1, 1, 700, 24, "f32"),       # one x without Q-Shift, ragged
 ]
 
 
