@@ -148,9 +148,15 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *   qs    NULL, or Q-Shift parameters applied to k (mu_k) and v (mu_v) on
  *         load (mu_r is ignored); T must then equal qs->H * qs->W.
  * Kernels (the same results up to rounding):
- *   - the 8-channel TMA kernel, the default: C % 8 == 0, 16-byte-aligned
- *     inputs and, with qs, group bounds int(C*gamma*j) that are multiples of
- *     8 and W <= 256, T <= 8192;
+ *   - the 32-token tensor-memory kernel, the default for T >= 2048: the
+ *     8-channel kernel's conditions with 1024-token CTAs (with qs, whole
+ *     image rows per CTA, a multiple of 256 tokens when the column needs
+ *     more than one CTA), T <= 8192, and the thread-block cluster and
+ *     tensor memory of four CTAs per SM available; each thread's per-token
+ *     partial sums are kept in tensor memory between its two passes;
+ *   - the 8-channel TMA kernel, the default below 2048 tokens: C % 8 == 0,
+ *     16-byte-aligned inputs and, with qs, group bounds int(C*gamma*j) that
+ *     are multiples of 8 and W <= 256, T <= 8192;
  *   - the 16-channel slab kernel, with VRWKV_FORWARD=wide in the
  *     environment (and for long sequences through the workspace variants):
  *     C % 16 == 0, T % 16 == 0, T <= 4096, 16-byte-aligned tensors and,
@@ -159,9 +165,12 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *     vertical ones;
  *   - a generic kernel for everything else (T <= 4096).
  *   Setting VRWKV_DISABLE_TMA=1 in the environment forces the generic
- *   kernel, VRWKV_DISABLE_WIDE=1 keeps the 16-channel one off, VRWKV_TMA_CHUNK=8 holds
- *   the 8-channel kernel to 8-token thread chunks and VRWKV_NO_TMA_STORE=1
- *   to per-thread stores of its results (diagnostics).
+ *   kernel, VRWKV_FORWARD=tm takes the tensor-memory kernel at any T where it
+ *   qualifies and VRWKV_FORWARD=narrow never, VRWKV_TM_ROT=0 keeps its
+ *   sub-chunks in natural order, VRWKV_DISABLE_WIDE=1 keeps the 16-channel
+ *   one off, VRWKV_TMA_CHUNK=8 holds the 8-channel kernel to 8-token thread
+ *   chunks and VRWKV_NO_TMA_STORE=1 to per-thread stores of its results
+ *   (diagnostics).
  * Limits: T <= 8192 on the 8-channel kernel, 4096 on the others
  *   (UNSUPPORTED above; the workspace variants below reach 32768); on the
  *   generic kernel with qs, a halo of shift_pixel*W tokens must fit its
@@ -322,9 +331,17 @@ vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k,
  * vrwkv_spatial_gate core on the projected R, K, V, the W_O GEMM and a
  * LayerNorm kernel.  The GEMMs are the library's own: for bfloat16 a
  * tcgen05 tensor-core kernel (TMA tiles with the 128-byte swizzle, float32
- * accumulators in tensor memory, results rounded to bfloat16 once) after a
- * transpose of each weight into the workspace; for float32 a kernel on the
- * FP32 pipes.  bfloat16 needs C % 8 == 0.
+ * accumulators in tensor memory, results rounded to bfloat16 once; CTA
+ * pairs with cta_group::2 MMAs, or single CTAs with VRWKV_GEMM_1CTA=1) after
+ * a transpose of each weight into the workspace; for float32 a kernel on the
+ * FP32 pipes.  bfloat16 needs C % 8 == 0.  The sigma(R) gate is applied in
+ * the core's epilogue, so W_O reads the gated result directly.
+ * VRWKV_BLOCK_FUSED=1 projects R, K, V in one launch whose A operand is the
+ * Q-Shift mix made in shared memory from x and its shifted copy (no staging
+ * in HBM; bit-identical to the staged path) where bfloat16, C a multiple of
+ * 256 up to 1024, T % 128 == 0, W dividing 128 (or a multiple of it) and
+ * group bounds that are multiples of 64 allow; off by default (slower on the
+ * B200: it mixes each x tile once per output tile).
  * Errors: INVALID_ARG for bad sizes, NULL or misaligned pointers, overlaps,
  *   bad qs fields or a small workspace; UNSUPPORTED for B*T >= 2^31, a
  *   bfloat16 C that is not a multiple of 8, or the core's limits; CUDA for a
