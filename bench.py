@@ -74,6 +74,7 @@ KERNEL_SOURCES = {
     "biwkv_fused_kernel": ("common.cuh", "qshift.cuh", "biwkv.cuh"),
     "channel_mix_vec_kernel": ("common.cuh", "qshift.cuh", "channel_mix.cuh"),
     "biwkv_bwd_kernel": ("common.cuh", "biwkv_tma.cuh", "biwkv_bwd.cuh"),
+    "biwkv_bwd_tm_kernel": ("common.cuh", "biwkv_tma.cuh", "biwkv_tm.cuh", "biwkv_bwd.cuh", "biwkv_bwd_tm.cuh"),
 }
 
 

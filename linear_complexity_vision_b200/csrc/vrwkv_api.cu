@@ -25,6 +25,7 @@
 #include "qshift.cuh"
 #include "channel_mix.cuh"
 #include "biwkv_bwd.cuh"
+#include "biwkv_bwd_tm.cuh"
 #include "layer_norm.cuh"
 #include "gemm_tc.cuh"
 
@@ -308,6 +309,57 @@ vrwkv_status gemm_project(const void* X, const void* W, void* D, int M, int N, i
     const int grid = std::min(tiles, sm_count());
     tcgemm::gemm_tc_kernel<<<grid, tcgemm::kThreads, smem, s>>>(p);
     return cuda_status(cudaGetLastError(), "gemm_tc_kernel launch");
+}
+
+// VRWKV_BWD_TM=0 keeps the backward on the 8-token kernel (diagnostics and
+// tests).
+bool bwd_tm_disabled() {
+    const char* e = getenv("VRWKV_BWD_TM");
+    return e && e[0] == '0' && e[1] == 0;
+}
+
+// The 16-token tensor-memory backward (bwd2::biwkv_bwd_tm_kernel): sets
+// *fell_back when the shape cannot be co-scheduled or more than four CTAs
+// would share an SM.
+template <typename IO>
+vrwkv_status launch_bwd_tm(const bwd::Params& p, cudaStream_t s, bool* fell_back) {
+    auto kern = bwd2::biwkv_bwd_tm_kernel<IO>;
+    const int smem = std::max((int)bwd2::Layout<IO>::kBytes, bwd2::kSmemFloor);
+    static std::atomic<int> granted{0};
+    cudaError_t e = ensure_smem(kern, granted, smem);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.ncl, (p.C + bwd2::kCS - 1) / bwd2::kCS, p.B);
+    cfg.blockDim = dim3(bwd2::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.ncl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.ncl > 1 ? 2 : 0;
+    static std::atomic<int> checked[bwd2::kClusterMax + 1];
+    int v = checked[p.ncl].load();
+    if (v == 0) {
+        int per_sm = 0, nclu = 1;
+        cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bwd2::kThreads, smem);
+        if (oe == cudaSuccess && p.ncl > 1) oe = cudaOccupancyMaxActiveClusters(&nclu, kern, &cfg);
+        if (oe != cudaSuccess) cudaGetLastError();
+        v = (oe == cudaSuccess && per_sm >= 1 && per_sm * bwd2::kTmemCols <= 512 && nclu > 0) ? 1 : -1;
+        checked[p.ncl].store(v);
+    }
+    if (v < 0) {
+        *fell_back = true;
+        return VRWKV_OK;
+    }
+    e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return cuda_status(e, "biwkv_bwd_tm_kernel launch");
+    g_last_kernel = "biwkv_bwd_tm_kernel";
+    return ok();
 }
 
 // VRWKV_BLOCK_FUSED=1 projects R, K, V with the fused Q-Shift GEMM instead of
@@ -1808,6 +1860,36 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
         }
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the 16-token tensor-memory kernel where the inputs arrive by TMA and gk,
+    // gv can leave by TMA stores
+    if (p.tma && !bwd_tm_disabled() && aligned(gk, 16) && aligned(gv, 16)) {
+        bwd::Params p2 = p;
+        EncodeTiledFn enc = encode_fn();
+        const CUtensorMapDataType tdt =
+            dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+        const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
+        const cuuint32_t box[3] = {(cuuint32_t)bwd::kCS, 256u, 1};
+        const cuuint32_t estr[3] = {1, (cuuint32_t)bwd::kL, 1};
+        void* dsts[2] = {gk, gv};
+        bool oks = enc != nullptr;
+        for (int i = 0; i < 2 && oks; ++i)
+            oks = enc(&p2.omap[i], tdt, 3, dsts[i], dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        if (oks) {
+            bool fell_back = false;
+            vrwkv_status st = dtype == VRWKV_F32 ? launch_bwd_tm<float>(p2, s, &fell_back)
+                                                 : launch_bwd_tm<__nv_bfloat16>(p2, s, &fell_back);
+            if (st != VRWKV_OK) return st;
+            if (!fell_back) {
+                const int blocks = (C + 255) / 256;
+                if (gw_total) bwd::batch_sum_kernel<<<blocks, 256, 0, s>>>(gw, gw_total, B, C);
+                if (gu_total) bwd::batch_sum_kernel<<<blocks, 256, 0, s>>>(gu, gu_total, B, C);
+                return cuda_status(cudaGetLastError(), "batch_sum_kernel launch");
+            }
+        }
+    }
     auto kern = dtype == VRWKV_F32 ? bwd::biwkv_bwd_kernel<float> : bwd::biwkv_bwd_kernel<__nv_bfloat16>;
     {
         static std::atomic<int> granted[2] = {{0}, {0}};

@@ -34,6 +34,18 @@ def vk():
     return vk
 
 
+@pytest.fixture(params=["tm", "8tok"])
+def bwd_path(request, monkeypatch):
+    """The default backward (the 16-token tensor-memory kernel where the
+    inputs arrive by TMA and gk, gv are 16-byte aligned) and the 8-token
+    kernel (VRWKV_BWD_TM=0)."""
+    if request.param == "8tok":
+        monkeypatch.setenv("VRWKV_BWD_TM", "0")
+    else:
+        monkeypatch.delenv("VRWKV_BWD_TM", raising=False)
+    return request.param
+
+
 def _inputs(B, T, C, dt, salt, kstd=1.0, w=("uniform", -5.0, 5.0)):
     seed = 20280000 + zlib.crc32(repr((B, T, C, dt, salt)).encode()) % 100000
     k = synth.draw(seed, "k", (B, T, C), ("normal", kstd))
@@ -107,14 +119,14 @@ SMALL = [
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 @pytest.mark.parametrize("B,T,C", SMALL)
-def test_bwd_parity_small(vk, oracle_mod, dt, B, T, C):
+def test_bwd_parity_small(vk, oracle_mod, dt, B, T, C, bwd_path):
     k, v, g, w, u = _inputs(B, T, C, dt, "small")
     _check(vk, oracle_mod, k, v, g, w, u, dt)
 
 
 @pytest.mark.parametrize("dt,B,T,C", [("bf16", 4, 4096, 768), ("f32", 1, 4096, 64),
                                       ("bf16", 2, 3000, 48), ("f32", 8, 196, 384)])
-def test_bwd_parity_large_sampled(vk, oracle_mod, dt, B, T, C):
+def test_bwd_parity_large_sampled(vk, oracle_mod, dt, B, T, C, bwd_path):
     # the 64 x 64 grid at C = 768 (bf16) is the backward of the
     # biwkv_B4_T4096_C768_bf16 workload; every element of 24 sampled columns
     k, v, g, w, u = _inputs(B, T, C, dt, "large", kstd=2.0, w=("uniform", -8.0, 8.0))
@@ -124,7 +136,7 @@ def test_bwd_parity_large_sampled(vk, oracle_mod, dt, B, T, C):
 
 
 @pytest.mark.parametrize("w_kind", ["zero", "huge_positive", "strong_negative"])
-def test_bwd_decay_extremes(vk, oracle_mod, w_kind):
+def test_bwd_decay_extremes(vk, oracle_mod, w_kind, bwd_path):
     T = 720
     d = {"zero": ("uniform", 0.0, 0.0), "huge_positive": ("uniform", 60.0 * T, 60.0 * T),
          "strong_negative": ("uniform", -20.0, -10.0)}[w_kind]
@@ -132,7 +144,7 @@ def test_bwd_decay_extremes(vk, oracle_mod, w_kind):
     _check(vk, oracle_mod, k, v, g, w, u, "f32")
 
 
-def test_bwd_shift_invariance_in_k(vk, oracle_mod):
+def test_bwd_shift_invariance_in_k(vk, oracle_mod, bwd_path):
     # adding 80 to every k would overflow e^k in float32 without the
     # maximum renormalisation; the gradients must not change
     k, v, g, w, u = _inputs(2, 600, 32, "f32", "shift")
@@ -143,7 +155,7 @@ def test_bwd_shift_invariance_in_k(vk, oracle_mod):
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_bwd_unaligned(vk, oracle_mod, dt):
+def test_bwd_unaligned(vk, oracle_mod, dt, bwd_path):
     # element-aligned tensors that are not pair-aligned take scalar loads
     k, v, g, w, u = _inputs(2, 300, 32, dt, "unaligned")
     _check(vk, oracle_mod, k, v, g, w, u, dt, offset=1)
@@ -155,17 +167,19 @@ def test_bwd_tma_store_path(vk, oracle_mod, monkeypatch, dt, B, T, C):
     # the optional TMA-store output path (VRWKV_BWD_TMA_STORE=1) against the
     # oracle: full CTAs, a ragged last CTA and a single short column
     monkeypatch.setenv("VRWKV_BWD_TMA_STORE", "1")
+    monkeypatch.setenv("VRWKV_BWD_TM", "0")  # an option of the 8-token kernel
     k, v, g, w, u = _inputs(B, T, C, dt, "tma_store")
     _check(vk, oracle_mod, k, v, g, w, u, dt)
 
 
-def test_bwd_deterministic(vk, oracle_mod):
+def test_bwd_deterministic(vk, oracle_mod, bwd_path):
     k, v, g, w, u = _inputs(2, 1024, 64, "bf16", "det")
     a, _, _, _ = _run(vk, k, v, g, w, u, "bf16")
     b, _, _, _ = _run(vk, k, v, g, w, u, "bf16")
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
-    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_bwd_kernel"
+    want = "biwkv_bwd_tm_kernel" if bwd_path == "tm" else "biwkv_bwd_kernel"
+    assert vk.load_library().vrwkv_last_kernel().decode() == want
 
 
 def test_bwd_matches_autograd_of_forward_kernel_shape(vk, oracle_mod):
