@@ -382,9 +382,12 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r,
  * Arithmetic is float32; dw and du are summed in a fixed order, so repeated
  * calls give identical bits.  With C % 8 == 0 and 16-byte-aligned k, v, gy
  * the inputs arrive by TMA, else by direct loads (VRWKV_DISABLE_TMA=1 forces
- * the direct loads; same results); VRWKV_BWD_TMA_STORE=1 also stores gk, gv
- * by TMA from shared memory when the inputs arrive by TMA and gk, gv are
- * 16-byte aligned (same results; measured slower, hence off by default).
+ * the direct loads; same results).  With TMA inputs and 16-byte-aligned gk,
+ * gv the default kernel gives each thread 16 tokens and keeps its per-token
+ * states in tensor memory (VRWKV_BWD_TM=0: the 8-token kernel; the same
+ * results up to rounding); on the 8-token kernel VRWKV_BWD_TMA_STORE=1 also
+ * stores gk, gv by TMA from shared memory (same results; measured slower,
+ * hence off by default).
  * Limits: T <= 4096 (UNSUPPORTED above, or when the GPU cannot co-schedule
  *   the thread-block cluster a column needs); the exponent range is that of
  *   vrwkv_biwkv_fwd.
