@@ -955,7 +955,8 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
 }
 
 // ---------------------------------------------------------------------------
-// 16-channel slab path (biwkv_wide_kernel): the default where it qualifies
+// 16-channel slab path (biwkv_wide_kernel): long sequences through a workspace,
+// and VRWKV_FORWARD=wide
 // ---------------------------------------------------------------------------
 bool wide_disabled() {
     const char* e = getenv("VRWKV_DISABLE_WIDE");
