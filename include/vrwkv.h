@@ -250,7 +250,8 @@ size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C,
  * operations, arguments and results.  Up to 4096 tokens, the CTAs of one
  * (b, 8-channel) column exchange their partial sums through the caller's
  * workspace instead of a thread-block cluster, which frees the kernel from
- * cluster co-scheduling.  Longer sequences (up to T = 32768, e.g. the
+ * cluster co-scheduling (the 32-token tensor-memory kernel from 2048 tokens,
+ * the 8-channel kernel below).  Longer sequences (up to T = 32768, e.g. the
  * 16384 tokens of a 2048^2 image at patch 16) run on the 16-channel kernel
  * when the shape qualifies for it: a column splits into segments of one
  * 8-CTA cluster (4096 tokens); segments take tickets from a counter in the

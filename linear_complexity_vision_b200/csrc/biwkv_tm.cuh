@@ -101,6 +101,8 @@ struct alignas(16) Scratch {
     unsigned long long bar;
     unsigned long long xbar;
     unsigned int tmem;  // base address of this CTA's tensor-memory columns
+    int tk;             // GX: this CTA's ticket
+    unsigned int gen;   // GX: the launch's generation
 };
 
 // Per-thread sub-chunk values in natural sub-chunk order, for the rotated
@@ -164,7 +166,10 @@ __device__ __forceinline__ void tc_fence_after() {
 // 8 different 16-byte rows of each 128-byte line: conflict-free tile, gate
 // and result accesses for 16-byte token rows.  The sub-chunk values that are
 // needed in natural order pass through a per-thread stash.
-template <typename IO, int LAYOUT, bool QS, bool ROT>
+// GX: no cluster; the CTAs of a column take tickets from the caller's
+// workspace and exchange their records through it (the 8-channel kernel's
+// workspace format and protocol: biwkv_tma.cuh).
+template <typename IO, int LAYOUT, bool QS, bool ROT, bool GX>
 __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_constant__ fast::Params p) {
     constexpr bool GATE = LAYOUT != kKV;
     constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
@@ -196,9 +201,22 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     const int warp = tid >> 5;
     if (tid == 0) {
         mbar_init(&S.bar, 1);
-        if (p.ncl > 1) {
+        if (!GX && p.ncl > 1) {
             mbar_init(&S.xbar, 1);
             mbar_expect_tx(&S.xbar, (unsigned)(p.ncl * kNP * (sizeof(float4) * 2 + sizeof(float2))));
+        }
+        if (GX) {
+            S.tk = (int)atomicAdd(p.ws_ctl, 1u);
+            S.gen = *reinterpret_cast<volatile unsigned int*>(p.ws_ctl + 2);
+        }
+    }
+    if (GX) {
+        // a ticket outside the grid means a workspace that was not zero-filled:
+        // leave before any tensor memory is taken
+        __syncthreads();
+        if (S.tk < 0 || S.tk >= p.total) {
+            if (tid == 0) atomicOr(p.err, 4u);
+            return;
         }
     }
     if (warp == 1) {
@@ -210,11 +228,22 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (p.ncl > 1) cluster_arrive_relaxed();  // waited for before the first push
+    if (!GX && p.ncl > 1) cluster_arrive_relaxed();  // waited for before the first push
     // this thread's lane of the CTA's columns
     const uint32_t tmem = S.tmem + ((uint32_t)(warp * 32) << 16);
 
-    const int rank = blockIdx.x, slab = blockIdx.y, b = blockIdx.z;
+    // this CTA's column chunk: the block index, or (GX) the ticket, column by
+    // column so a column's CTAs hold consecutive tickets
+    int rank = blockIdx.x, slab = blockIdx.y, b = blockIdx.z;
+    unsigned int gen = 0;
+    if (GX) {
+        const int t = S.tk;
+        gen = S.gen;
+        rank = t % p.ncl;
+        slab = (t / p.ncl) % p.nslab;
+        b = t / p.ncl / p.nslab;
+    }
+    const int col = b * p.nslab + slab;  // GX: the column's records and flags
     const int c0 = slab * kCS;
     const int t0 = rank * p.Tc;
     const int tend = min(p.T, t0 + p.Tc);
@@ -489,8 +518,46 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
             for (int e = 0; e < 3; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
         }
         __syncthreads();
-        cluster_wait_acquire();  // every mailbox barrier is initialised
-        {
+        if (GX) {
+            // publish the record to the workspace, then the flag (release
+            // after every writer's fence), then wait for the column's flags
+            // and copy the records into the mailbox
+            float4* rec = p.ws_rec + ((size_t)col * fast::kClusterMax + rank) * fast::kRecF4;
+            if (tid < fast::kRecF4) {
+                float4 v;
+                if (tid < kNP) {
+                    v = S.ownF[tid];
+                } else if (tid < 2 * kNP) {
+                    v = S.ownG[tid - kNP];
+                } else {
+                    const int m = 2 * (tid - 2 * kNP);
+                    v = make_float4(S.ownM[m].x, S.ownM[m].y, S.ownM[m + 1].x, S.ownM[m + 1].y);
+                }
+                __stcg(rec + tid, v);
+                __threadfence();
+            }
+            __syncthreads();
+            unsigned int* flags = p.ws_flag + (size_t)col * fast::kClusterMax;
+            if (tid == 0)
+                asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flags + rank), "r"(gen + 1u) : "memory");
+            if (tid < p.ncl) fast::wait_flag(flags + tid, gen + 1u, p.err);
+            __syncthreads();
+            const float4* peers = p.ws_rec + (size_t)col * fast::kClusterMax * fast::kRecF4;
+            for (int e = tid; e < p.ncl * fast::kRecF4; e += kThreads) {
+                const int r = e / fast::kRecF4, k = e - r * fast::kRecF4;
+                const float4 v = __ldcg(peers + e);
+                if (k < kNP) {
+                    S.mbF[r][k] = v;
+                } else if (k < 2 * kNP) {
+                    S.mbG[r][k - kNP] = v;
+                } else {
+                    const int m = 2 * (k - 2 * kNP);
+                    S.mbM[r][m] = make_float2(v.x, v.y);
+                    S.mbM[r][m + 1] = make_float2(v.z, v.w);
+                }
+            }
+        } else {
+            cluster_wait_acquire();  // every mailbox barrier is initialised
             const int peer = tid / (2 * kNP), jj = (tid >> 1) % kNP;
             if (peer < p.ncl) {
                 const unsigned rbar = mapa_u32(smem_u32(&S.xbar), peer);
@@ -501,8 +568,8 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
                     st_async2(mapa_u32(smem_u32(&S.mbM[rank][jj]), peer), S.ownM[jj], rbar);
                 }
             }
+            if (tid == 0) mbar_wait_cluster_bounded(&S.xbar, p.err);
         }
-        if (tid == 0) mbar_wait_cluster_bounded(&S.xbar, p.err);
         __syncthreads();
         if (tid < nex) {
             float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
@@ -647,6 +714,18 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(S.tmem), "r"(kTmemCols)
                      : "memory");
+    }
+    if (GX && tid == 0) {
+        // count the CTA out; the last one resets the counters for the next
+        // launch and advances the generation
+        __threadfence();
+        const unsigned int d = atomicAdd(p.ws_ctl + 1, 1u);
+        if (d == (unsigned int)p.total - 1u) {
+            atomicExch(p.ws_ctl + 0, 0u);
+            atomicExch(p.ws_ctl + 1, 0u);
+            __threadfence();
+            atomicExch(p.ws_ctl + 2, gen + 1u);
+        }
     }
 }
 

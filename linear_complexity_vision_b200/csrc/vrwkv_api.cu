@@ -682,9 +682,9 @@ static_assert(kFastTcMax == fast::Cfg<kFastThreads8, 8>::kTcMax, "one tile geome
 // The 32-token tensor-memory kernel: a cluster per column as in the 8-channel
 // kernel.  Sets *fell_back when the shape cannot be co-scheduled or more
 // than four CTAs would share an SM (their tensor memory would not fit).
-template <typename IO, int LAYOUT, bool QS, bool ROT>
+template <typename IO, int LAYOUT, bool QS, bool ROT, bool GX>
 vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
-    auto kern = tm32::biwkv_tm_kernel<IO, LAYOUT, QS, ROT>;
+    auto kern = tm32::biwkv_tm_kernel<IO, LAYOUT, QS, ROT, GX>;
     static std::atomic<int> granted{0};
     cudaError_t e = ensure_smem(kern, granted, pl.smem);
     if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute");
@@ -701,7 +701,7 @@ vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back)
     attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
     attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
-    cfg.numAttrs = pl.p.ncl > 1 ? 2 : 0;
+    cfg.numAttrs = (!GX && pl.p.ncl > 1) ? 2 : 0;  // GX: a plain 1-D grid of tickets
     // checked once per (cluster size, shared memory)
     static std::mutex mu;
     static std::vector<std::array<int, 3>> seen;
@@ -714,7 +714,7 @@ vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back)
     if (okv == 0) {
         int per_sm = 0, nclu = 1;
         cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tm32::kThreads, pl.smem);
-        if (oe == cudaSuccess && pl.p.ncl > 1) oe = cudaOccupancyMaxActiveClusters(&nclu, kern, &cfg);
+        if (oe == cudaSuccess && !GX && pl.p.ncl > 1) oe = cudaOccupancyMaxActiveClusters(&nclu, kern, &cfg);
         if (oe != cudaSuccess) cudaGetLastError();
         okv = (oe == cudaSuccess && per_sm >= 1 && per_sm * tm32::kTmemCols <= 512 && nclu > 0) ? 1 : -1;
         std::lock_guard<std::mutex> lk(mu);
@@ -730,16 +730,21 @@ vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back)
     return ok();
 }
 
+template <typename IO, bool ROT, bool GX>
+vrwkv_status dispatch_tm_layout(const FastPlan& pl, cudaStream_t s, bool* fb) {
+    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
+    case fast::kKV * 2 + 0: return launch_tm<IO, fast::kKV, false, ROT, GX>(pl, s, fb);
+    case fast::kKV * 2 + 1: return launch_tm<IO, fast::kKV, true, ROT, GX>(pl, s, fb);
+    case fast::kRKV * 2 + 0: return launch_tm<IO, fast::kRKV, false, ROT, GX>(pl, s, fb);
+    case fast::kRKV * 2 + 1: return launch_tm<IO, fast::kRKV, true, ROT, GX>(pl, s, fb);
+    case fast::kX * 2 + 0: return launch_tm<IO, fast::kX, false, ROT, GX>(pl, s, fb);
+    default: return launch_tm<IO, fast::kX, true, ROT, GX>(pl, s, fb);
+    }
+}
+
 template <typename IO, bool ROT>
 vrwkv_status dispatch_tm_rot(const FastPlan& pl, cudaStream_t s, bool* fb) {
-    switch (pl.layout * 2 + (pl.qs ? 1 : 0)) {
-    case fast::kKV * 2 + 0: return launch_tm<IO, fast::kKV, false, ROT>(pl, s, fb);
-    case fast::kKV * 2 + 1: return launch_tm<IO, fast::kKV, true, ROT>(pl, s, fb);
-    case fast::kRKV * 2 + 0: return launch_tm<IO, fast::kRKV, false, ROT>(pl, s, fb);
-    case fast::kRKV * 2 + 1: return launch_tm<IO, fast::kRKV, true, ROT>(pl, s, fb);
-    case fast::kX * 2 + 0: return launch_tm<IO, fast::kX, false, ROT>(pl, s, fb);
-    default: return launch_tm<IO, fast::kX, true, ROT>(pl, s, fb);
-    }
+    return pl.gx ? dispatch_tm_layout<IO, ROT, true>(pl, s, fb) : dispatch_tm_layout<IO, ROT, false>(pl, s, fb);
 }
 
 template <typename IO>
@@ -939,7 +944,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     p.nslab = C / fast::kCS;
     p.total = p.ncl * p.nslab * B;
     pl.gx = ws != nullptr && p.ncl > 1;
-    if (pl.tm && (pl.gx || !p.tma_store)) return false;
+    if (pl.tm && !p.tma_store) return false;
     if (pl.gx) {
         const WsLayout L = ws_layout(B, C);
         char* base = static_cast<char*>(ws);
@@ -1246,9 +1251,11 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
             if (!fell_back) return st;
         }
     }
-    if (B <= 65535 && C / vrwkv::fast::kCS <= 65535 && !with_ws && tm_wanted(T)) {
+    // the 32-token kernel: a cluster per column, or with a workspace (T <= 4096
+    // here; longer ones took the 16-channel segments above) its global exchange
+    if (B <= 65535 && C / vrwkv::fast::kCS <= 65535 && tm_wanted(T)) {
         FastPlan fp;
-        if (plan_fast(fp, gate, r, k, v, w, u, out, B, T, C, dtype, qs, nullptr, true)) {
+        if (plan_fast(fp, gate, r, k, v, w, u, out, B, T, C, dtype, qs, with_ws ? ws : nullptr, true)) {
             bool fell_back = false;
             cudaStream_t fs = static_cast<cudaStream_t>(stream);
             vrwkv_status st = dtype == VRWKV_F32 ? dispatch_tm<float>(fp, fs, &fell_back)

@@ -38,11 +38,15 @@ def _inputs(B, T, C):
     return k, v, w, u
 
 
-def test_workspace_peer_wait_runs_out_and_is_reported(vk, oracle_mod):
+@pytest.mark.parametrize("T,kernel", [(1024, "biwkv_tma_kernel"), (2048, "biwkv_tm_kernel")])
+def test_workspace_peer_wait_runs_out_and_is_reported(vk, oracle_mod, T, kernel):
     import torch
-    # fast path without Q-Shift: one 8-channel slab, 512-token CTAs, so the
-    # grid holds exactly two CTAs, ranks 0 and 1 of one column
-    B, T, C = 1, 1024, 8
+    # fast paths without Q-Shift, one 8-channel slab: 512-token CTAs of the
+    # 8-channel kernel at T = 1024, 1024-token CTAs of the 32-token kernel at
+    # T = 2048, so the grid holds exactly two CTAs, ranks 0 and 1 of one
+    # column (the CTA that finds its ticket past the grid leaves before it
+    # takes any tensor memory)
+    B, C = 1, 8
     k, v, w, u = _inputs(B, T, C)
     kt, kd = to_device(k, "bf16")
     vt, vd = to_device(v, "bf16")
@@ -69,6 +73,7 @@ def test_workspace_peer_wait_runs_out_and_is_reported(vk, oracle_mod):
     # the context is intact: a fresh workspace gives the oracle's result
     out = vk.biwkv_fwd(kt, vt, wt, ut, workspace=vk.fwd_workspace(B, T, C))
     vk.device_status()
+    assert vk.load_library().vrwkv_last_kernel().decode() == kernel
     got = to_numpy(out)
     want = oracle_mod.biwkv_direct(kd, vd, wd, ud)
     err = scaled_error(got, want, biwkv_scale(oracle_mod, kd, vd, wd, ud))
