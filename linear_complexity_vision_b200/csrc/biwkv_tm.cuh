@@ -85,19 +85,14 @@ constexpr int kSmemFloor = 46 * 1024;
 struct alignas(16) Scratch {
     float2 tab[kChunks][kNP];  // a^(32 m) per channel pair
     float2 wmax[kNP][kNW + 1];
-    float2 wsc[kNP][kNW + 1];
     float4 waggF[kNP][kNW + 1];
     float4 waggB[kNP][kNW + 1];
-    float4 wcarF[kNP][kNW + 1];
-    float4 wcarB[kNP][kNW + 1];
     float2 mbM[kClusterMax][kNP + 1];
     float4 mbF[kClusterMax][kNP + 1];
     float4 mbG[kClusterMax][kNP + 1];
     float4 ownF[kNP];
     float4 ownG[kNP];
     float2 ownM[kNP];
-    float4 cscale[kCS];
-    float4 ccarry[kCS];
     unsigned long long bar;
     unsigned long long xbar;
     unsigned int tmem;  // base address of this CTA's tensor-memory columns
@@ -469,59 +464,61 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     if (cq == kCPW - 1) S.waggF[j][warp] = Fi;
     if (cq == 0) S.waggB[j][warp] = Gi;
     __syncthreads();
-    if (warp == 0) {
-        const bool act = tid < kNP * kNW;
-        const int jj = act ? tid / kNW : 0, wi = act ? tid % kNW : 0;
-        const float2 mw = S.wmax[jj][wi];
-        float2 mc = mw;
+    // CTA scan, in every thread for its own pair (no warp waits on another's
+    // serial scan): each warp's scale onto the CTA maximum, the folds of the
+    // warps before and after this one, and the CTA's records for the column
+    float4 XW = zero4(), YW = zero4();  // exclusive carries into this warp (CTA frame)
+    float2 wsw = f2(0.0f);              // this warp's scale onto the CTA reference
+    float4 ownF = zero4(), ownG = zero4();
+    float2 ownM;
+    {
+        float2 mw[kNW];
+        float4 sF[kNW], sB[kNW];
 #pragma unroll
-        for (int d = 1; d < kNW; d <<= 1) {
-            mc.x = fmaxf(mc.x, __shfl_xor_sync(0xffffffffu, mc.x, d, kNW));
-            mc.y = fmaxf(mc.y, __shfl_xor_sync(0xffffffffu, mc.y, d, kNW));
-        }
-        const float2 ws = ex2(mul2(add2(mw, make_float2(-mc.x, -mc.y)), f2(kLog2e)));
-        float4 f = scale4(ws, S.waggF[jj][wi]);
-        float4 gb = scale4(ws, S.waggB[jj][wi]);
+        for (int w = 0; w < kNW; ++w) mw[w] = S.wmax[j][w];
+        const float2 mc = max2(max2(mw[0], mw[1]), max2(mw[2], mw[3]));
+        const float2 a256 = S.tab[kCPW][j];  // across one warp's 256 tokens
 #pragma unroll
-        for (int d = 1; d < kNW; d <<= 1) {
-            const float2 m = S.tab[kCPW * d][jj];  // across d warps
-            float4 o = shfl_up4(f, d, kNW);
-            if (wi >= d) f = fma4(m, o, f);
-            o = shfl_down4(gb, d, kNW);
-            if (wi + d < kNW) gb = fma4(m, o, gb);
+        for (int w = 0; w < kNW; ++w) {
+            // 2^(M_w - M_cta), 0 for a warp wholly past T
+            const float2 sc = ex2(mul2(add2(mw[w], make_float2(-mc.x, -mc.y)), f2(kLog2e)));
+            sF[w] = scale4(sc, S.waggF[j][w]);
+            sB[w] = scale4(sc, S.waggB[j][w]);
+            if (w == warp) wsw = sc;
         }
-        float4 xw = shfl_up4(f, 1, kNW), yw = shfl_down4(gb, 1, kNW);
-        if (wi == 0) xw = zero4();
-        if (wi == kNW - 1) yw = zero4();
-        if (act) {
-            S.wsc[jj][wi] = ws;
-            S.wcarF[jj][wi] = xw;
-            S.wcarB[jj][wi] = yw;
-            if (p.ncl > 1) {
-                if (wi == p.Tc / kWarpTok - 1) S.ownF[jj] = f;
-                if (wi == 0) {
-                    S.ownG[jj] = gb;
-                    S.ownM[jj] = mul2(mc, f2(kLog2e));
-                }
-            }
+        // forward: the CTA's total sits at its last real warp (Tc may be
+        // shorter than the CTA's capacity when the column spans several CTAs)
+        const int wl = p.Tc / kWarpTok - 1;
+        float4 acc = zero4();
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) {
+            if (w == warp) XW = acc;
+            acc = fma4(a256, acc, sF[w]);
+            if (w == wl) ownF = acc;
         }
+        acc = zero4();
+#pragma unroll
+        for (int w = kNW - 1; w >= 0; --w) {
+            if (w == warp) YW = acc;
+            acc = fma4(a256, acc, sB[w]);
+        }
+        ownG = acc;
+        ownM = mul2(mc, f2(kLog2e));  // base 2, the unit of the exponents below
     }
-    // exchange lanes: thread (channel lc, peer rr) in segments of 8 lanes
-    const int lc = tid >> 3, rr = tid & 7;
-    constexpr int nex = kCS * 8;  // 64 threads: warp-uniform
+    // column exchange: every CTA's records reach every CTA of the column;
+    // each thread then folds them for its pair
     float2 cs_sl = f2(1.0f), cs_af = f2(0.0f), cs_cf = f2(0.0f), cs_bb = f2(0.0f), cs_db = f2(0.0f);
     if (p.ncl > 1) {
-        float mdec[3];
-        if (tid < nex) {
-            const float l2 = __ldg(p.w + c0 + lc) * (invT * kLog2e);
-#pragma unroll
-            for (int e = 0; e < 3; ++e) mdec[e] = ex2c(-(float)(p.Tc << e) * l2);
-        }
-        __syncthreads();
         if (GX) {
             // publish the record to the workspace, then the flag (release
             // after every writer's fence), then wait for the column's flags
             // and copy the records into the mailbox
+            if (q == 0) {
+                S.ownF[j] = ownF;
+                S.ownG[j] = ownG;
+                S.ownM[j] = ownM;
+            }
+            __syncthreads();
             float4* rec = p.ws_rec + ((size_t)col * fast::kClusterMax + rank) * fast::kRecF4;
             if (tid < fast::kRecF4) {
                 float4 v;
@@ -556,84 +553,59 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
                     S.mbM[r][m + 1] = make_float2(v.z, v.w);
                 }
             }
+            __syncthreads();
         } else {
+            // asynchronous stores into every CTA's mailbox (its own included):
+            // thread (pair j, chunk q) sends pair j's forward record to peer q
+            // (q < ncl), its backward record and maximum to peer q - ncl
+            // (ncl <= q < 2 ncl); each thread then waits, bounded, until its
+            // CTA's mailbox is full
             cluster_wait_acquire();  // every mailbox barrier is initialised
-            const int peer = tid / (2 * kNP), jj = (tid >> 1) % kNP;
-            if (peer < p.ncl) {
+            if (q < 2 * p.ncl) {
+                const int peer = q < p.ncl ? q : q - p.ncl;
                 const unsigned rbar = mapa_u32(smem_u32(&S.xbar), peer);
-                if ((tid & 1) == 0) {
-                    st_async4(mapa_u32(smem_u32(&S.mbF[rank][jj]), peer), S.ownF[jj], rbar);
+                if (q < p.ncl) {
+                    st_async4(mapa_u32(smem_u32(&S.mbF[rank][j]), peer), ownF, rbar);
                 } else {
-                    st_async4(mapa_u32(smem_u32(&S.mbG[rank][jj]), peer), S.ownG[jj], rbar);
-                    st_async2(mapa_u32(smem_u32(&S.mbM[rank][jj]), peer), S.ownM[jj], rbar);
+                    st_async4(mapa_u32(smem_u32(&S.mbG[rank][j]), peer), ownG, rbar);
+                    st_async2(mapa_u32(smem_u32(&S.mbM[rank][j]), peer), ownM, rbar);
                 }
             }
-            if (tid == 0) mbar_wait_cluster_bounded(&S.xbar, p.err);
+            mbar_wait_cluster_bounded(&S.xbar, p.err);
         }
-        __syncthreads();
-        if (tid < nex) {
-            float Mr = -INFINITY, fa2 = 0.f, fc2 = 0.f, ga2 = 0.f, gc2 = 0.f;
-            if (rr < p.ncl) {
-                const float4 F = S.mbF[rr][lc >> 1], G = S.mbG[rr][lc >> 1];
-                const float2 Mp = S.mbM[rr][lc >> 1];
-                const bool hi = lc & 1;
-                Mr = hi ? Mp.y : Mp.x;
-                fa2 = hi ? F.y : F.x;
-                fc2 = hi ? F.w : F.z;
-                ga2 = hi ? G.y : G.x;
-                gc2 = hi ? G.w : G.z;
-            }
-            float Mc = Mr;
+        // fold the peers' records on the column maximum: the forward ones of
+        // the CTAs before this one, the backward ones of those after it, each
+        // CTA a decay of a^Tc further
+        const float2 aTc = ex2c(mul2(lam2, f2(-(float)p.Tc)));
+        float2 Mc = f2(-INFINITY);
 #pragma unroll
-            for (int d = 4; d >= 1; d >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, d, 8));
-            const float sc = ex2(Mr - Mc);  // 0 for lanes past the cluster
-            fa2 *= sc;
-            fc2 *= sc;
-            ga2 *= sc;
-            gc2 *= sc;
+        for (int r = 0; r < kClusterMax; ++r)
+            if (r < p.ncl) Mc = max2(Mc, S.mbM[r][j]);
+        float4 accF = zero4(), accG = zero4();
 #pragma unroll
-            for (int e = 0, d = 1; d < 8; ++e, d <<= 1) {
-                const float m = mdec[e];  // decay across d CTAs
-                const float ua = __shfl_up_sync(0xffffffffu, fa2, d, 8);
-                const float uc = __shfl_up_sync(0xffffffffu, fc2, d, 8);
-                const float da = __shfl_down_sync(0xffffffffu, ga2, d, 8);
-                const float dc = __shfl_down_sync(0xffffffffu, gc2, d, 8);
-                if (rr >= d) {
-                    fa2 = fmaf(m, ua, fa2);
-                    fc2 = fmaf(m, uc, fc2);
-                }
-                if (rr + d < 8) {
-                    ga2 = fmaf(m, da, ga2);
-                    gc2 = fmaf(m, dc, gc2);
-                }
-            }
-            const float Af = __shfl_sync(0xffffffffu, fa2, max(rank - 1, 0), 8);
-            const float Cf = __shfl_sync(0xffffffffu, fc2, max(rank - 1, 0), 8);
-            const float Bb = __shfl_sync(0xffffffffu, ga2, min(rank + 1, 7), 8);
-            const float Db = __shfl_sync(0xffffffffu, gc2, min(rank + 1, 7), 8);
-            const float Mme = __shfl_sync(0xffffffffu, Mr, rank, 8);
-            if (rr == 0) {
-                S.cscale[lc] = make_float4(ex2(Mme - Mc), 0.f, 0.f, 0.f);
-                S.ccarry[lc] = make_float4(rank > 0 ? Af : 0.f, rank > 0 ? Cf : 0.f,
-                                           rank + 1 < p.ncl ? Bb : 0.f, rank + 1 < p.ncl ? Db : 0.f);
+        for (int r = 0; r < kClusterMax; ++r) {
+            if (r < rank) {
+                const float2 sc = ex2(add2(S.mbM[r][j], make_float2(-Mc.x, -Mc.y)));
+                accF = fma4(aTc, accF, scale4(sc, S.mbF[r][j]));
             }
         }
-        __syncthreads();
-        const float4 s0 = S.cscale[2 * j], s1 = S.cscale[2 * j + 1];
-        const float4 k0 = S.ccarry[2 * j], k1 = S.ccarry[2 * j + 1];
-        cs_sl = make_float2(s0.x, s1.x);
-        cs_af = make_float2(k0.x, k1.x);
-        cs_cf = make_float2(k0.y, k1.y);
-        cs_bb = make_float2(k0.z, k1.z);
-        cs_db = make_float2(k0.w, k1.w);
-    } else {
-        __syncthreads();
+#pragma unroll
+        for (int r = kClusterMax - 1; r >= 0; --r) {
+            if (r > rank && r < p.ncl) {
+                const float2 sc = ex2(add2(S.mbM[r][j], make_float2(-Mc.x, -Mc.y)));
+                accG = fma4(aTc, accG, scale4(sc, S.mbG[r][j]));
+            }
+        }
+        cs_sl = ex2(add2(ownM, make_float2(-Mc.x, -Mc.y)));
+        cs_af = lo2(accF);
+        cs_cf = hi2(accF);
+        cs_bb = lo2(accG);
+        cs_db = hi2(accG);
     }
 
     // ---- 4. carries -> outputs ---------------------------------------------------
     const float2 sl = cs_sl;
-    const float2 slw = mul2(sl, S.wsc[j][warp]);
-    const float4 XW = S.wcarF[j][warp], YW = S.wcarB[j][warp];
+    const float2 slw = mul2(sl, wsw);
     const float2 slF = mul2(sl, S.tab[cq][j]), slB = mul2(sl, S.tab[kCPW - 1 - cq][j]);
     const float2 kf = S.tab[q][j];                          // CTA start -> chunk start
     const float2 kb = S.tab[max(0, p.Tc / kKL - 1 - q)][j];  // chunk end -> CTA end
