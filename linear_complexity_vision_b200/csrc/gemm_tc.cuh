@@ -327,9 +327,15 @@ constexpr int A_BYTES = kHalf * BK * 2;      // 16 KB
 constexpr int B_BYTES = kHalf * BK * 2;      // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 
+// Epilogue staging of one warp: 32 rows x 32 bfloat16 columns, rows 80
+// bytes apart (64 bytes of data + 16 of padding: conflict-free 16-byte
+// accesses in both directions).
+constexpr int kStgRowWords = 20;
+
 struct alignas(1024) Smem {
     uint8_t a[kStages][A_BYTES];
     uint8_t b[kStages][B_BYTES];
+    uint32_t stg[4][32 * kStgRowWords];  // per epilogue warp
     unsigned long long full[kStages], empty[kStages];
     unsigned long long tfull[kAcc], tempty[kAcc];
     unsigned long long drain;
@@ -483,8 +489,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // epilogue: this CTA's 128 rows of the pair's tile
+        // epilogue: this CTA's 128 rows of the pair's tile; a warp's 32 x 32
+        // chunk goes through shared memory so the global stores cover whole
+        // 64-byte row segments (eight rows per instruction) instead of one
+        // 16-byte piece of 32 rows
         const int quad = warp & 3;
+        uint32_t* stg = S.stg[warp - 2];
         const uint32_t leader_tempty[2] = {fast::mapa_u32(fast::smem_u32(&S.tempty[0]), 0),
                                            fast::mapa_u32(fast::smem_u32(&S.tempty[1]), 0)};
         int lt = 0;
@@ -494,14 +504,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!wait_phase(&S.tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
             const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
-            const int row = m0 + (int)rank * kHalf + quad * 32 + lane;
+            const int row0 = m0 + (int)rank * kHalf + quad * 32;  // the warp's first row
+            const int row = row0 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+            const bool whole = row0 + 32 <= p.M && n0 + BN <= p.N && (p.N % 8) == 0;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tbase + (uint32_t)(c * 32), v);
                 const int col = n0 + c * 32;
-                if (row < p.M && col < p.N) {
+                if (whole) {
+                    uint32_t* mine = stg + lane * kStgRowWords;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]),
+                                                                           __uint_as_float(v[8 * q + 2 * e + 1]));
+                            w4[e] = *reinterpret_cast<const uint32_t*>(&h);
+                        }
+                        *reinterpret_cast<uint4*>(mine + 4 * q) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                    __syncwarp();
+                    // lane l: row 8 i + l / 4, 16-byte piece l % 4
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = 8 * i + (lane >> 2), pc = lane & 3;
+                        const uint4 d = *reinterpret_cast<const uint4*>(stg + r * kStgRowWords + 4 * pc);
+                        *reinterpret_cast<uint4*>(p.d + (size_t)(row0 + r) * p.N + col + 8 * pc) = d;
+                    }
+                    __syncwarp();
+                } else if (row < p.M && col < p.N) {
                     uint32_t w16[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
