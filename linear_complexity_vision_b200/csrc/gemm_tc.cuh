@@ -327,10 +327,11 @@ constexpr int A_BYTES = kHalf * BK * 2;      // 16 KB
 constexpr int B_BYTES = kHalf * BK * 2;      // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 
-// Epilogue staging of one warp: 32 rows x 32 bfloat16 columns, rows 80
-// bytes apart (64 bytes of data + 16 of padding: conflict-free 16-byte
-// accesses in both directions).
-constexpr int kStgRowWords = 20;
+// Epilogue staging of one warp: 32 rows x 32 bfloat16 columns, 64 bytes a
+// row; 16-byte piece c of row r sits at piece c ^ ((r >> 1) & 3), which keeps
+// the row-wise writes and the piece-wise reads free of bank conflicts.
+constexpr int kStgRowWords = 16;
+__device__ __forceinline__ int stg_piece(int r, int c) { return c ^ ((r >> 1) & 3); }
 
 struct alignas(1024) Smem {
     uint8_t a[kStages][A_BYTES];
@@ -524,14 +525,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                                            __uint_as_float(v[8 * q + 2 * e + 1]));
                             w4[e] = *reinterpret_cast<const uint32_t*>(&h);
                         }
-                        *reinterpret_cast<uint4*>(mine + 4 * q) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        *reinterpret_cast<uint4*>(mine + 4 * pair::stg_piece(lane, q)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
                     __syncwarp();
                     // lane l: row 8 i + l / 4, 16-byte piece l % 4
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int r = 8 * i + (lane >> 2), pc = lane & 3;
-                        const uint4 d = *reinterpret_cast<const uint4*>(stg + r * kStgRowWords + 4 * pc);
+                        const uint4 d = *reinterpret_cast<const uint4*>(stg + r * kStgRowWords + 4 * stg_piece(r, pc));
                         *reinterpret_cast<uint4*>(p.d + (size_t)(row0 + r) * p.N + col + 8 * pc) = d;
                     }
                     __syncwarp();
@@ -630,6 +631,7 @@ struct alignas(1024) Smem {
     uint8_t xs[kStages][A_BYTES];  // the Q-Shifted x
     float mu[3][kMaxC];
     float om[3][kMaxC];  // 1 - mu, rounded once
+    uint32_t stg[4][32 * pair::kStgRowWords];  // epilogue staging, per epilogue warp
     unsigned long long full[kStages], empty[kStages], xfull[kStages];
     unsigned long long tfull[kAcc], tempty[kAcc];
     unsigned long long drain;
@@ -832,15 +834,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsQ, 1)
             tc_fence_after();
             const Tile tl = tile_of(t, nt, p.nproj);
             const int m0 = tl.mb * BM, n0 = tl.nb * BN;
-            const int row = m0 + (int)rank * kHalf + quad * 32 + lane;
+            const int row0 = m0 + (int)rank * kHalf + quad * 32;
+            const int row = row0 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
             __nv_bfloat16* D = p.d[tl.proj];
+            uint32_t* stg = S.stg[warp - 2];
+            const bool whole = row0 + 32 <= p.M;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tbase + (uint32_t)(c * 32), v);
                 const int col = n0 + c * 32;
-                if (row < p.M && col + 32 <= p.N) {
+                if (whole) {
+                    // through shared memory: whole 64-byte row segments per store
+                    uint32_t* mine = stg + lane * pair::kStgRowWords;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]),
+                                                                           __uint_as_float(v[8 * q + 2 * e + 1]));
+                            w4[e] = *reinterpret_cast<const uint32_t*>(&h);
+                        }
+                        *reinterpret_cast<uint4*>(mine + 4 * pair::stg_piece(lane, q)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = 8 * i + (lane >> 2), pc = lane & 3;
+                        const uint4 d = *reinterpret_cast<const uint4*>(stg + r * pair::kStgRowWords + 4 * pair::stg_piece(r, pc));
+                        *reinterpret_cast<uint4*>(D + (size_t)(row0 + r) * p.N + col + 8 * pc) = d;
+                    }
+                    __syncwarp();
+                } else if (row < p.M && col + 32 <= p.N) {
                     uint32_t w16[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
