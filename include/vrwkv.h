@@ -342,7 +342,8 @@ vrwkv_status vrwkv_spatial_gate_static(const void* r, const void* k,
  * in HBM; bit-identical to the staged path) where bfloat16, C a multiple of
  * 256 up to 1024, T % 128 == 0, W dividing 128 (or a multiple of it) and
  * group bounds that are multiples of 64 allow; off by default (slower on the
- * B200: it mixes each x tile once per output tile).
+ * B200, 521 against 424 us at B = 8, 64 x 64, C = 1024: it mixes each x tile
+ * once per output tile).
  * Errors: INVALID_ARG for bad sizes, NULL or misaligned pointers, overlaps,
  *   bad qs fields or a small workspace; UNSUPPORTED for B*T >= 2^31, a
  *   bfloat16 C that is not a multiple of 8, or the core's limits; CUDA for a

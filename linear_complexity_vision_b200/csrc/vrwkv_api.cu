@@ -364,7 +364,7 @@ vrwkv_status launch_bwd_tm(const bwd::Params& p, cudaStream_t s, bool* fell_back
 
 // VRWKV_BLOCK_FUSED=1 projects R, K, V with the fused Q-Shift GEMM instead of
 // staging the three mixes in HBM.  Off by default: measured on the B200 at
-// B = 8, 64 x 64, C = 1024 the fused block takes 585 us against 502 us
+// B = 8, 64 x 64, C = 1024 the fused block takes 521 us against 424 us
 // staged.  The fused A producer mixes every x tile once per N tile (four
 // times per projection at C = 1024), and that element-wise work (about six
 // instructions per element) outgrows what the SM issues beside the MMAs;
