@@ -52,9 +52,67 @@ struct Params {
     unsigned int* err;
 };
 
+// Epilogue staging of one warp: 32 rows x 32 bfloat16 columns, 64 bytes a
+// row; 16-byte piece c of row r sits at piece c ^ ((r >> 1) & 3), which keeps
+// the row-wise writes and the piece-wise reads free of bank conflicts.
+constexpr int kStgRowWords = 16;
+__device__ __forceinline__ int stg_piece(int r, int c) { return c ^ ((r >> 1) & 3); }
+
+// One warp's 32 x 32 chunk of results (lane = row row0 + lane, 32 float32
+// columns from col), rounded to bfloat16.  A whole chunk passes through the
+// warp's staging buffer so each store instruction covers 64-byte segments of
+// eight rows instead of 16-byte pieces of 32 rows; a ragged one is stored
+// row by row.
+__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], uint32_t* stg, int lane, int row0, int col,
+                                            int M, int N, __nv_bfloat16* d) {
+    const int row = row0 + lane;
+    if (row0 + 32 <= M && col + 32 <= N && (N % 8) == 0) {  // warp-uniform
+        uint32_t* mine = stg + lane * kStgRowWords;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 h =
+                    __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
+                w4[e] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(mine + 4 * stg_piece(lane, q)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // lane l: row 8 i + l / 4, 16-byte piece l % 4
+            const int r = 8 * i + (lane >> 2), pc = lane & 3;
+            const uint4 w = *reinterpret_cast<const uint4*>(stg + r * kStgRowWords + 4 * stg_piece(r, pc));
+            *reinterpret_cast<uint4*>(d + (size_t)(row0 + r) * N + col + 8 * pc) = w;
+        }
+        __syncwarp();
+    } else if (row < M && col < N) {
+        uint32_t w16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            w16[e] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        __nv_bfloat16* dst = d + (size_t)row * N + col;
+        if (col + 32 <= N && (N % 8) == 0) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) d4[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+        } else {
+            for (int e = 0; e < 32 && col + e < N; ++e) {
+                const uint32_t wv = w16[e >> 1];
+                const unsigned short hv = (e & 1) ? (unsigned short)(wv >> 16) : (unsigned short)(wv & 0xffffu);
+                dst[e] = __ushort_as_bfloat16(hv);
+            }
+        }
+    }
+}
+
 struct alignas(1024) Smem {
     uint8_t a[kStages][A_BYTES];
     uint8_t b[kStages][B_BYTES];
+    uint32_t stg[4][32 * kStgRowWords];  // epilogue staging, per epilogue warp
     unsigned long long full[kStages], empty[kStages];
     unsigned long long tfull[kAcc], tempty[kAcc];
     unsigned long long drain;  // completion of every issued MMA (abort path)
@@ -263,35 +321,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             if (!wait_phase(&S.tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
             const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
-            const int row = m0 + quad * 32 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tbase + (uint32_t)(c * 32), v);
-                const int col = n0 + c * 32;
-                if (row < p.M && col < p.N) {
-                    uint32_t w16[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]),
-                                                                       __uint_as_float(v[2 * e + 1]));
-                        w16[e] = *reinterpret_cast<const uint32_t*>(&h);
-                    }
-                    __nv_bfloat16* dst = p.d + (size_t)row * p.N + col;
-                    if (col + 32 <= p.N && (p.N % 8) == 0) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            d4[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
-                    } else {
-                        for (int e = 0; e < 32 && col + e < p.N; ++e) {
-                            const uint32_t wv = w16[e >> 1];
-                            const unsigned short hv = (e & 1) ? (unsigned short)(wv >> 16) : (unsigned short)(wv & 0xffffu);
-                            dst[e] = __ushort_as_bfloat16(hv);
-                        }
-                    }
-                }
+                store_chunk(v, S.stg[warp - 2], lane, m0 + quad * 32, n0 + c * 32, p.M, p.N, p.d);
             }
             tc_fence_before();
             __syncwarp();
@@ -327,16 +362,10 @@ constexpr int A_BYTES = kHalf * BK * 2;      // 16 KB
 constexpr int B_BYTES = kHalf * BK * 2;      // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 
-// Epilogue staging of one warp: 32 rows x 32 bfloat16 columns, 64 bytes a
-// row; 16-byte piece c of row r sits at piece c ^ ((r >> 1) & 3), which keeps
-// the row-wise writes and the piece-wise reads free of bank conflicts.
-constexpr int kStgRowWords = 16;
-__device__ __forceinline__ int stg_piece(int r, int c) { return c ^ ((r >> 1) & 3); }
-
 struct alignas(1024) Smem {
     uint8_t a[kStages][A_BYTES];
     uint8_t b[kStages][B_BYTES];
-    uint32_t stg[4][32 * kStgRowWords];  // per epilogue warp
+    uint32_t stg[4][32 * kStgRowWords];  // epilogue staging, per epilogue warp
     unsigned long long full[kStages], empty[kStages];
     unsigned long long tfull[kAcc], tempty[kAcc];
     unsigned long long drain;
@@ -490,12 +519,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // epilogue: this CTA's 128 rows of the pair's tile; a warp's 32 x 32
-        // chunk goes through shared memory so the global stores cover whole
-        // 64-byte row segments (eight rows per instruction) instead of one
-        // 16-byte piece of 32 rows
+        // epilogue: this CTA's 128 rows of the pair's tile, 32 x 32 chunks per
+        // warp through its staging buffer
         const int quad = warp & 3;
-        uint32_t* stg = S.stg[warp - 2];
         const uint32_t leader_tempty[2] = {fast::mapa_u32(fast::smem_u32(&S.tempty[0]), 0),
                                            fast::mapa_u32(fast::smem_u32(&S.tempty[1]), 0)};
         int lt = 0;
@@ -505,59 +531,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!wait_phase(&S.tfull[acc], aph, abort, p.err)) break;
             tc_fence_after();
             const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
-            const int row0 = m0 + (int)rank * kHalf + quad * 32;  // the warp's first row
-            const int row = row0 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
-            const bool whole = row0 + 32 <= p.M && n0 + BN <= p.N && (p.N % 8) == 0;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tbase + (uint32_t)(c * 32), v);
-                const int col = n0 + c * 32;
-                if (whole) {
-                    uint32_t* mine = stg + lane * kStgRowWords;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]),
-                                                                           __uint_as_float(v[8 * q + 2 * e + 1]));
-                            w4[e] = *reinterpret_cast<const uint32_t*>(&h);
-                        }
-                        *reinterpret_cast<uint4*>(mine + 4 * pair::stg_piece(lane, q)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                    __syncwarp();
-                    // lane l: row 8 i + l / 4, 16-byte piece l % 4
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = 8 * i + (lane >> 2), pc = lane & 3;
-                        const uint4 d = *reinterpret_cast<const uint4*>(stg + r * kStgRowWords + 4 * stg_piece(r, pc));
-                        *reinterpret_cast<uint4*>(p.d + (size_t)(row0 + r) * p.N + col + 8 * pc) = d;
-                    }
-                    __syncwarp();
-                } else if (row < p.M && col < p.N) {
-                    uint32_t w16[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]),
-                                                                       __uint_as_float(v[2 * e + 1]));
-                        w16[e] = *reinterpret_cast<const uint32_t*>(&h);
-                    }
-                    __nv_bfloat16* dst = p.d + (size_t)row * p.N + col;
-                    if (col + 32 <= p.N && (p.N % 8) == 0) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            d4[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
-                    } else {
-                        for (int e = 0; e < 32 && col + e < p.N; ++e) {
-                            const uint32_t wv = w16[e >> 1];
-                            const unsigned short hv = (e & 1) ? (unsigned short)(wv >> 16) : (unsigned short)(wv & 0xffffu);
-                            dst[e] = __ushort_as_bfloat16(hv);
-                        }
-                    }
-                }
+                store_chunk(v, S.stg[warp - 2], lane, m0 + (int)rank * kHalf + quad * 32, n0 + c * 32, p.M, p.N,
+                            p.d);
             }
             tc_fence_before();
             __syncwarp();
@@ -631,7 +611,7 @@ struct alignas(1024) Smem {
     uint8_t xs[kStages][A_BYTES];  // the Q-Shifted x
     float mu[3][kMaxC];
     float om[3][kMaxC];  // 1 - mu, rounded once
-    uint32_t stg[4][32 * pair::kStgRowWords];  // epilogue staging, per epilogue warp
+    uint32_t stg[4][32 * kStgRowWords];  // epilogue staging, per epilogue warp
     unsigned long long full[kStages], empty[kStages], xfull[kStages];
     unsigned long long tfull[kAcc], tempty[kAcc];
     unsigned long long drain;
@@ -834,52 +814,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsQ, 1)
             tc_fence_after();
             const Tile tl = tile_of(t, nt, p.nproj);
             const int m0 = tl.mb * BM, n0 = tl.nb * BN;
-            const int row0 = m0 + (int)rank * kHalf + quad * 32;
-            const int row = row0 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
-            __nv_bfloat16* D = p.d[tl.proj];
-            uint32_t* stg = S.stg[warp - 2];
-            const bool whole = row0 + 32 <= p.M;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tbase + (uint32_t)(c * 32), v);
-                const int col = n0 + c * 32;
-                if (whole) {
-                    // through shared memory: whole 64-byte row segments per store
-                    uint32_t* mine = stg + lane * pair::kStgRowWords;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]),
-                                                                           __uint_as_float(v[8 * q + 2 * e + 1]));
-                            w4[e] = *reinterpret_cast<const uint32_t*>(&h);
-                        }
-                        *reinterpret_cast<uint4*>(mine + 4 * pair::stg_piece(lane, q)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = 8 * i + (lane >> 2), pc = lane & 3;
-                        const uint4 d = *reinterpret_cast<const uint4*>(stg + r * pair::kStgRowWords + 4 * pair::stg_piece(r, pc));
-                        *reinterpret_cast<uint4*>(D + (size_t)(row0 + r) * p.N + col + 8 * pc) = d;
-                    }
-                    __syncwarp();
-                } else if (row < p.M && col + 32 <= p.N) {
-                    uint32_t w16[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]),
-                                                                       __uint_as_float(v[2 * e + 1]));
-                        w16[e] = *reinterpret_cast<const uint32_t*>(&h);
-                    }
-                    uint4* d4 = reinterpret_cast<uint4*>(D + (size_t)row * p.N + col);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        d4[q] = make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
-                }
+                store_chunk(v, S.stg[warp - 2], lane, m0 + (int)rank * kHalf + quad * 32, n0 + c * 32, p.M, p.N,
+                            p.d[tl.proj]);
             }
             tc_fence_before();
             __syncwarp();
