@@ -975,14 +975,16 @@ bool wide_preferred() {
     return e && e[0] == 'w';
 }
 
-// The 32-token tensor-memory kernel takes columns of 2048 tokens and more
-// (shorter ones leave too many of its threads idle); VRWKV_FORWARD=tm takes
-// it wherever it qualifies, VRWKV_FORWARD=narrow never.
+// The 32-token tensor-memory kernel takes columns of 1024 tokens and more
+// (measured on the B200 at C = 1024: 80.5 against 95.8 us at T = 1024, but
+// 130 against 74 us at T = 256, where most of its threads have no token);
+// VRWKV_FORWARD=tm takes it wherever it qualifies, VRWKV_FORWARD=narrow
+// never.
 bool tm_wanted(int T) {
     const char* e = getenv("VRWKV_FORWARD");
     if (e && e[0] == 't') return true;
     if (e && e[0]) return false;
-    return T >= 2048;
+    return T >= 1024;
 }
 
 struct WidePlan {
