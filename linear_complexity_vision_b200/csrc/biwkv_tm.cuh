@@ -50,6 +50,7 @@ using fast::cluster_wait_acquire;
 using fast::fence_proxy_async_smem;
 using fast::fma4;
 using fast::hi2;
+using fast::lds_f32;
 using fast::lds_pair;
 using fast::lo2;
 using fast::mapa_u32;
@@ -62,6 +63,7 @@ using fast::shfl_up4;
 using fast::smem_u32;
 using fast::st_async2;
 using fast::st_async4;
+using fast::sts_f32;
 using fast::tma_load_3d;
 using fast::tma_load_4d;
 using fast::tma_store_3d;
@@ -137,11 +139,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
         : "r"(taddr)
         : "memory");
 }
-// A gate factor's store into a slot depends on the values read from that
-// slot (they make r), and a result's store on the gate factor read from its
-// slot: data dependence alone orders each slot's accesses.
-__device__ __forceinline__ void sts_f32(char* p, float v) { *reinterpret_cast<float*>(p) = v; }
-__device__ __forceinline__ float lds_f32(const char* p) { return *reinterpret_cast<const float*>(p); }
 // three-input maximum (one instruction on sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
@@ -255,10 +252,18 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
             const int i = tid, h0 = rank * p.rows;
             for (int s = 0; s < NSRC; ++s) {
                 char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB;
-                if (!QS) {
+                if (!QS || p.flat) {
 #pragma unroll
                     for (int h = 0; h < kTc / 256; ++h)
                         tma_load_3d(plain + h * 32 * RB, &p.map[s], c0, t0 + i + 256 * h, b, &S.bar);
+                    if (QS && shifted) {
+                        // the flat view: the same boxes displaced by the group's token offset
+                        const int dt = grp == 0 ? -p.s : (grp == 1 ? p.s : (grp == 2 ? -p.s * p.W : p.s * p.W));
+#pragma unroll
+                        for (int h = 0; h < kTc / 256; ++h)
+                            tma_load_3d(plain + p.tile_bytes + h * 32 * RB, &p.map[s], c0, t0 + i + dt + 256 * h, b,
+                                        &S.bar);
+                    }
                 } else {
                     tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar);
                     if (shifted) {
@@ -290,6 +295,10 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
 
     if (tid == 0) mbar_wait_bounded(&S.bar, p.err);
     __syncthreads();
+    if (QS && p.flat && shifted && grp < 2) {
+        fast::zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, tend, p.W, p.s, grp == 0, tid, kThreads);
+        __syncthreads();
+    }
 
     // ---- 1-2. per 8-token sub-chunk: load, Q-Shift mix, gate factor (parked in
     // the token's slots), local maximum, p = 2^(k - M_h), two-sided sums inside

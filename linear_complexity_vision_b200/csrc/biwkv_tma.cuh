@@ -107,6 +107,8 @@ struct alignas(64) Params {
     int tile_bytes;      // bytes per tile: 8 sub-tiles of 32 token rows
     int box_bytes;       // bytes one strided box delivers (zero fill included)
     int tma_store;       // results leave by TMA stores (the CTA's span is whole boxes, or the column's end)
+    int flat;            // Q-Shift through the flat (C, T, B) view: shifted tiles loaded at a token
+                         // offset, row-wrapped tokens of horizontal groups zeroed after the load
     // global-memory exchange (GX kernels only): see the workspace layout below
     unsigned int* ws_ctl;   // [0] ticket counter, [1] finished CTAs, [2] generation
     unsigned int* ws_flag;  // per (column, rank): generation + 1 once its record is out
@@ -147,7 +149,6 @@ struct alignas(16) Scratch {
     float4 ownF[kNP];           // this CTA's inclusive forward aggregate, staged for the push
     float4 ownG[kNP];           // this CTA's inclusive backward aggregate
     float2 ownM[kNP];           // this CTA's max of k (times log2 e)
-    float2 gpark[Cfg<NT, KL>::kTcMax][kNP];  // gate factors, parked between load and output
     float4 cscale[kCS];         // per channel: sl (scale of this CTA's own sums)
     int tk;                     // GX: this CTA's ticket
     unsigned int gen;           // GX: the launch's generation
@@ -155,6 +156,40 @@ struct alignas(16) Scratch {
     unsigned long long bar;     // TMA completion barrier
     unsigned long long xbar;    // mailbox barrier: completes when every peer's record is in
 };
+
+// Q-Shift through the flat token view (any W): a shifted tile loaded at the
+// token offset -s or +s (horizontal groups 0 and 1) holds, at the first or
+// last s columns of every image row, a token of the neighbouring row.  eq. 9
+// wants zeros there; this clears those token rows of each source's shifted
+// tile (tile 2 src + 1) after the load.  Vertical groups need nothing: the
+// offset -s W or +s W leaves [0, T) exactly where the row leaves [0, H), and
+// the TMA's zero fill covers it.  Token tl of the CTA sits at sub-tile tl % 8,
+// row tl / 8.
+template <int RB>
+__device__ __forceinline__ void zero_row_wrap(char* smem, int tile_bytes, int sub_bytes, int nsrc, int t0, int tend,
+                                              int W, int s, bool left, int tid, int nthreads) {
+    const int sw = min(s, W);  // source outside the row: w < s (left) or w >= W - s
+    const int h0 = t0 / W, nrow = (tend - 1) / W - h0 + 1;
+    const int per_src = nrow * sw;
+    for (int e = tid; e < nsrc * per_src; e += nthreads) {
+        const int src = e / per_src, r = e - src * per_src;
+        const int hr = h0 + r / sw, k = r % sw;
+        const int t = hr * W + (left ? k : W - 1 - k);
+        if (t < t0 || t >= tend) continue;
+        const int tl = t - t0;
+        char* dst = smem + (2 * src + 1) * tile_bytes + (tl & (kL - 1)) * sub_bytes + (tl / kL) * RB;
+#pragma unroll
+        for (int o = 0; o < RB; o += 16) *reinterpret_cast<uint4*>(dst + o) = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// One float of a tile slot: the gate factor parked between the load and the
+// output pass (see the kernels).  A gate factor's store into a slot depends
+// on the values read from that slot (they make r), and a result's store on
+// the gate factor read from its slot: data dependence alone orders each
+// slot's accesses.
+__device__ __forceinline__ void sts_f32(char* p, float v) { *reinterpret_cast<float*>(p) = v; }
+__device__ __forceinline__ float lds_f32(const char* p) { return *reinterpret_cast<const float*>(p); }
 
 // ---- PTX wrappers ----------------------------------------------------------
 __device__ __forceinline__ unsigned smem_u32(const void* p) {
@@ -332,7 +367,6 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     constexpr int kNW = C_::kNW;
     constexpr int kTcMax = C_::kTcMax;
     constexpr int kH = C_::kH;          // sub-chunks of 8 tokens per thread chunk
-    constexpr int kChunks = C_::kTab;   // chunks per CTA
     using Scratch = fast::Scratch<NT, KL>;
     constexpr bool GATE = LAYOUT != kKV;
     constexpr int NSRC = LAYOUT == kKV ? 2 : (LAYOUT == kRKV ? 3 : 1);
@@ -348,7 +382,15 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     // destinations; the host adds 128 bytes of slack
     extern __shared__ __align__(128) char smem_raw[];
     char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
-    Scratch& S = *reinterpret_cast<Scratch*>(smem + NTILE * p.tile_bytes);
+    // The gate factor e^{-r} of a token waits for the output pass in two tile
+    // slots its thread has just read: r's own and shifted r's with Q-Shift;
+    // r's and k's for separate r, k, v without; r's and one extra tile when
+    // one x feeds r, k and v without Q-Shift.  The result later goes into the
+    // first slot.
+    constexpr bool G1_IN_K = GATE && !QS && LAYOUT == kRKV;
+    constexpr int NTA = GATE && !QS && !G1_IN_K ? NTILE + 1 : NTILE;
+    constexpr int G1 = QS ? 2 * SR + 1 : (G1_IN_K ? SK : NTILE);  // tile of the second half
+    Scratch& S = *reinterpret_cast<Scratch*>(smem + NTA * p.tile_bytes);
 
     const int tid = threadIdx.x;
     const int j = tid % kNP;     // channel pair
@@ -407,12 +449,20 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
             const int h0 = rank * p.rows;
             for (int s = 0; s < NSRC; ++s) {
                 char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB;
-                if (!QS) {
+                if (!QS || p.flat) {
                     // boxes of 256 strided tokens (32 rows); a box wholly past T
                     // still delivers its zero-filled bytes
 #pragma unroll
                     for (int h = 0; h < kTcMax / 256; ++h)
                         tma_load_3d(plain + h * 32 * RB, &p.map[s], c0, t0 + i + 256 * h, b, &S.bar);
+                    if (QS && shifted) {
+                        // the flat view: the same boxes displaced by the group's token offset
+                        const int dt = grp == 0 ? -p.s : (grp == 1 ? p.s : (grp == 2 ? -p.s * p.W : p.s * p.W));
+#pragma unroll
+                        for (int h = 0; h < kTcMax / 256; ++h)
+                            tma_load_3d(plain + p.tile_bytes + h * 32 * RB, &p.map[s], c0, t0 + i + dt + 256 * h, b,
+                                        &S.bar);
+                    }
                 } else {
                     tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar);
                     if (shifted) {
@@ -455,6 +505,10 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     // one thread waits for the tiles; the others sleep at the CTA barrier
     if (tid == 0) mbar_wait_bounded(&S.bar, p.err);
     __syncthreads();
+    if (QS && p.flat && shifted && grp < 2) {
+        zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, tend, p.W, p.s, grp == 0, tid, kThreads);
+        __syncthreads();
+    }
 
     // ---- 1-2. per 8-token sub-chunk: load, Q-Shift mix, gate factor, local
     // maximum, p = 2^(k - M_h), two-sided sums inside the sub-chunk ----------
@@ -499,8 +553,15 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
                 v = lds_pair<IO>(tV, o);
                 if (GATE) r = lds_pair<IO>(tR, o);
             }
-            // gate factor e^{-r}, parked in shared memory until the output phase
-            if (GATE) S.gpark[(h * kL + i) * kChunks + q][j] = ex2(mul2(r, f2(-kLog2e)));
+            // gate factor e^{-r}, parked in the token's slots until the output pass
+            if (GATE) {
+                float2 g = ex2(mul2(r, f2(-kLog2e)));
+                // in k's slot the second half must follow the read of k, which
+                // it does not depend on: tie it to k (no instruction)
+                if (G1_IN_K) asm volatile("" : "+f"(g.y) : "f"(k.x), "f"(k.y));
+                sts_f32(smem + SR * (QS ? 2 : 1) * p.tile_bytes + o, g.x);
+                sts_f32(smem + G1 * p.tile_bytes + o, g.y);
+            }
             kk[i] = k;
             vv[i] = v;
         }
@@ -818,7 +879,13 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
         for (int i = 0; i < kL; ++i) {
             const float2 num = fma2(sh, n[h][i], fma2(pw[i], Ah, mul2(pw[kL - 1 - i], Bh)));
             float2 den = fma2(sh, dd[h][i], fma2(pw[i], Ch, mul2(pw[kL - 1 - i], Dh)));
-            if (GATE) den = fma2(den, S.gpark[(h * kL + i) * kChunks + q][j], den);
+            if (GATE) {
+                // read before the result overwrites the first slot
+                const int o = rowoff + i * SUB;
+                const float2 g = make_float2(lds_f32(smem + SR * (QS ? 2 : 1) * p.tile_bytes + o),
+                                             lds_f32(smem + G1 * p.tile_bytes + o));
+                den = fma2(den, g, den);
+            }
             Io<IO>::st_pair(tout + rowoff + i * SUB, mul2(num, rcp(den)));
         }
     }

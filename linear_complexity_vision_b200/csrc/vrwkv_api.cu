@@ -670,14 +670,19 @@ vrwkv_status dispatch_fast_nt(const FastPlan& pl, cudaStream_t s, bool* fb) {
     }
 }
 
-// CTA shapes of the fast path, both 512 tokens x 8 channels at four CTAs per
-// SM: 128 threads with 16-token chunks (the default: half the per-thread
+// CTA shapes of the fast path, two of 512 tokens x 8 channels at four CTAs
+// per SM: 128 threads with 16-token chunks (the default: half the per-thread
 // scan and exchange work per token), or 256 threads with 8-token chunks where
-// a cluster's CTAs cannot hold whole 128-token warps.
+// a cluster's CTAs cannot hold whole 128-token warps; and one of 256 tokens
+// (64 threads, 16-token chunks) for columns of at most 256 tokens, so a
+// 14 x 14 grid keeps 13 of 16 chunks busy instead of 13 of 32 and its smaller
+// tiles let twice the CTAs share an SM.
 constexpr int kFastThreads16 = 128;
 constexpr int kFastThreads8 = 256;
+constexpr int kFastThreadsShort = 64;
 constexpr int kFastTcMax = fast::Cfg<kFastThreads16, 16>::kTcMax;
-static_assert(kFastTcMax == fast::Cfg<kFastThreads8, 8>::kTcMax, "one tile geometry for both shapes");
+constexpr int kFastTcShort = fast::Cfg<kFastThreadsShort, 16>::kTcMax;
+static_assert(kFastTcMax == fast::Cfg<kFastThreads8, 8>::kTcMax, "one tile geometry for both long shapes");
 
 // The 32-token tensor-memory kernel: a cluster per column as in the 8-channel
 // kernel.  Sets *fell_back when the shape cannot be co-scheduled or more
@@ -758,6 +763,7 @@ vrwkv_status dispatch_tm(const FastPlan& pl, cudaStream_t s, bool* fb) {
 
 template <typename IO>
 vrwkv_status dispatch_fast(const FastPlan& pl, cudaStream_t s, bool* fb) {
+    if (pl.nt == kFastThreadsShort) return dispatch_fast_nt<IO, kFastThreadsShort, 16, false>(pl, s, fb);
     if (pl.kl == 16)
         return pl.gx ? dispatch_fast_nt<IO, kFastThreads16, 16, true>(pl, s, fb)
                      : dispatch_fast_nt<IO, kFastThreads16, 16, false>(pl, s, fb);
@@ -765,11 +771,31 @@ vrwkv_status dispatch_fast(const FastPlan& pl, cudaStream_t s, bool* fb) {
                  : dispatch_fast_nt<IO, kFastThreads8, 8, false>(pl, s, fb);
 }
 
-// Shared memory of a fast-path CTA: the tiles plus the scratch block.
-int fast_smem(int ntiles, int tile_bytes, int kl) {
-    const int scratch = kl == 16 ? (int)sizeof(fast::Scratch<kFastThreads16, 16>)
-                                 : (int)sizeof(fast::Scratch<kFastThreads8, 8>);
-    return ntiles * tile_bytes + scratch + 128;  // + alignment slack
+// Shared memory of a fast-path CTA: the tiles (one extra for the gate
+// factor when one x feeds r, k and v without Q-Shift) plus the scratch block.
+int fast_smem(bool gate, bool qs, int ntiles, int tile_bytes, int nt) {
+    const int nta = gate && !qs && ntiles == 1 ? ntiles + 1 : ntiles;
+    const int scratch = nt == kFastThreadsShort ? (int)sizeof(fast::Scratch<kFastThreadsShort, 16>)
+                        : nt == kFastThreads16  ? (int)sizeof(fast::Scratch<kFastThreads16, 16>)
+                                                : (int)sizeof(fast::Scratch<kFastThreads8, 8>);
+    return nta * tile_bytes + scratch + 128;  // + alignment slack
+}
+
+// VRWKV_QS_VIEW=flat takes Q-Shift through the flat token view wherever the
+// TMA kernels run it (also where the image view qualifies), =image never
+// (grids whose W is not a multiple of 8 then go to the generic kernel);
+// diagnostics and tests.
+int qs_view_forced() {
+    const char* e = getenv("VRWKV_QS_VIEW");
+    if (!e || !e[0]) return 0;
+    return e[0] == 'f' ? 1 : (e[0] == 'i' ? -1 : 0);
+}
+
+// VRWKV_SHORT_CTA=0 keeps columns of at most 256 tokens on the 512-token CTA
+// shape (diagnostics and tests).
+bool short_cta_disabled() {
+    const char* e = getenv("VRWKV_SHORT_CTA");
+    return e && e[0] == '0' && e[1] == 0;
 }
 
 // Shared memory of a tensor-memory kernel CTA: its tiles (one extra for the
@@ -837,15 +863,24 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     const int RB = fast::kCS * es;
     const int ntiles = nsrc * (pl.qs ? 2 : 1);
     pl.ntiles = ntiles;
-    const int TcMax = pl.tm ? tm32::kTc : kFastTcMax;
+    const bool short_cta = !pl.tm && T <= kFastTcShort && !tma_chunk8_forced() && !short_cta_disabled();
+    const int TcMax = pl.tm ? tm32::kTc : (short_cta ? kFastTcShort : kFastTcMax);
     pl.kl = pl.tm ? tm32::kKL : (tma_chunk8_forced() ? 8 : 16);
+    p.flat = 0;
     if (pl.qs) {
         p.H = qs->H;
         p.W = qs->W;
         p.s = qs->shift_pixel;
         p.g = qs_bounds(C, qs->gamma);
         p.ng = shifted_groups(qs);
-        if (!bounds_multiple_of(p.g, fast::kCS) || p.W > 256 || p.W % fast::kL != 0) return false;
+        if (!bounds_multiple_of(p.g, fast::kCS)) return false;
+        // the image view (C, W, H, B) needs W a multiple of 8 and at most 256
+        // (one box row); any other W takes the flat token view
+        const int view = qs_view_forced();
+        p.flat = (view > 0 || p.W > 256 || p.W % fast::kL != 0) ? 1 : 0;
+        if (p.flat && view < 0) return false;
+    }
+    if (pl.qs && !p.flat) {
         if (T <= TcMax) {
             p.rows = p.H;
             p.Tc = T;
@@ -872,11 +907,13 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
             p.ncl = (p.H + rows - 1) / rows;
         }
     } else {
-        p.H = 1;
-        p.W = T;
-        p.s = 0;
-        p.g = no_shift_bounds();
-        p.ng = 4;
+        if (!pl.qs) {
+            p.H = 1;
+            p.W = T;
+            p.s = 0;
+            p.g = no_shift_bounds();
+            p.ng = 4;
+        }
         p.rows = 1;
         p.Tc = std::min(T, TcMax);
         p.ncl = (T + p.Tc - 1) / p.Tc;
@@ -886,13 +923,13 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     // each, so a tile always spans TcMax tokens even when the boxes deliver
     // fewer
     p.tile_bytes = TcMax * RB;
-    // a sub-tile receives (W / 8) x rows token rows with Q-Shift (one box),
-    // and its full TcMax / 8 rows without (boxes of 32 rows; tokens past T
-    // arrive as zeros)
-    p.box_bytes = (pl.qs ? (p.W / fast::kL) * p.rows : TcMax / fast::kL) * RB;
-    pl.nt = pl.tm ? tm32::kThreads : (pl.kl == 16 ? kFastThreads16 : kFastThreads8);
+    // a sub-tile receives (W / 8) x rows token rows with Q-Shift in the image
+    // view (one box), and its full TcMax / 8 rows in the flat view (boxes of
+    // 32 rows; tokens past T arrive as zeros)
+    p.box_bytes = (pl.qs && !p.flat ? (p.W / fast::kL) * p.rows : TcMax / fast::kL) * RB;
+    pl.nt = pl.tm ? tm32::kThreads : (short_cta ? kFastThreadsShort : (pl.kl == 16 ? kFastThreads16 : kFastThreads8));
     pl.rot = pl.tm && tm_rot_wanted(gate, pl.qs, ntiles, p.tile_bytes, es);
-    pl.smem = pl.tm ? tm_smem(gate, pl.qs, ntiles, p.tile_bytes, pl.rot) : fast_smem(ntiles, p.tile_bytes, pl.kl);
+    pl.smem = pl.tm ? tm_smem(gate, pl.qs, ntiles, p.tile_bytes, pl.rot) : fast_smem(gate, pl.qs, ntiles, p.tile_bytes, pl.nt);
     if (pl.smem > 227 * 1024) return false;
     const CUtensorMapDataType dt =
         dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -900,7 +937,7 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
         CUresult cr;
         // element stride 8 along the token (w) axis: box i holds tokens 8q + i
         const cuuint32_t estr[4] = {1, (cuuint32_t)fast::kL, 1, 1};
-        if (pl.qs) {
+        if (pl.qs && !p.flat) {
             const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)B};
             const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)p.W * C * es,
                                            (cuuint64_t)p.H * p.W * C * es};

@@ -182,16 +182,18 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     return (got, err) if return_out else err
 
 
-@pytest.fixture(params=["default", "narrow", "tm", "wide", "tma8", "gx", "generic"])
+@pytest.fixture(params=["default", "narrow", "flat", "tm", "wide", "tma8", "gx", "generic"])
 def kernel_path(request, monkeypatch):
     """Run a test on the default path (the 32-token tensor-memory kernel for
-    columns of 2048 tokens and more, else the 8-channel TMA kernel with
-    16-token thread chunks, where the shape and cluster geometry allow), on
-    the latter alone ("narrow"), on the tensor-memory kernel wherever it
-    qualifies ("tm"), on the 16-channel slab kernel where the shape qualifies
-    ("wide"), on the 8-channel kernel held to 8-token chunks, on its
-    workspace variant (global-memory exchange instead of clusters) and with
-    the generic kernel forced."""
+    columns of 1024 tokens and more, else the 8-channel TMA kernel with
+    16-token thread chunks, on 256-token CTAs for columns of at most 256
+    tokens, where the shape and cluster geometry allow), on the latter alone
+    ("narrow"), on it with Q-Shift through the flat token view everywhere and
+    512-token CTAs at any length ("flat"), on the tensor-memory kernel
+    wherever it qualifies ("tm"), on the 16-channel slab kernel where the
+    shape qualifies ("wide"), on the 8-channel kernel held to 8-token chunks,
+    on its workspace variant (global-memory exchange instead of clusters) and
+    with the generic kernel forced."""
     if request.param == "generic":
         monkeypatch.setenv("VRWKV_DISABLE_TMA", "1")
     else:
@@ -200,7 +202,14 @@ def kernel_path(request, monkeypatch):
         monkeypatch.setenv("VRWKV_TMA_CHUNK", "8")
     else:
         monkeypatch.delenv("VRWKV_TMA_CHUNK", raising=False)
-    forward = {"wide": "wide", "tm": "tm", "narrow": "narrow", "tma8": "narrow"}.get(request.param)
+    if request.param == "flat":
+        monkeypatch.setenv("VRWKV_QS_VIEW", "flat")
+        monkeypatch.setenv("VRWKV_SHORT_CTA", "0")
+    else:
+        monkeypatch.delenv("VRWKV_QS_VIEW", raising=False)
+        monkeypatch.delenv("VRWKV_SHORT_CTA", raising=False)
+    forward = {"wide": "wide", "tm": "tm", "narrow": "narrow", "tma8": "narrow",
+               "flat": "narrow"}.get(request.param)
     if forward:
         monkeypatch.setenv("VRWKV_FORWARD", forward)
     else:
@@ -222,6 +231,16 @@ def test_default_forward_is_the_tensor_memory_kernel(vk, oracle_mod, cfg, monkey
     wl = synth.WORKLOADS[cfg]
     run_fused(vk, oracle_mod, wl)
     assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tm_kernel"
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_14x14_grids_take_the_8_channel_kernel(vk, oracle_mod, cfg, monkeypatch):
+    # W = 14 is not a multiple of 8: Q-Shift goes through the flat token view
+    for name in ("VRWKV_FORWARD", "VRWKV_QS_VIEW", "VRWKV_SHORT_CTA", "VRWKV_DISABLE_TMA"):
+        monkeypatch.delenv(name, raising=False)
+    wl = synth.WORKLOADS[cfg]
+    run_fused(vk, oracle_mod, wl)
+    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tma_kernel"
 
 
 @pytest.mark.parametrize("cfg", [4, 5])
@@ -277,6 +296,9 @@ TM_CASES = [
     ("gate", 2, 1, 4096, 64, "bf16", 0.25),        # r, k, v without Q-Shift: gate in k's slots
     ("gate", 1, 1, 3000, 32, "f32", 0.25),         # the same in float32, ragged last CTA
     ("gate_x", 2, 1, 4096, 32, "bf16", 0.25),      # one x without Q-Shift: gate in an extra tile
+    ("gate_qs_x", 1, 36, 36, 64, "bf16", 0.25),    # W = 36: flat token view, 2 CTAs
+    ("gate_qs", 1, 45, 50, 32, "f32", 0.25),       # W = 50: flat view in float32, 3 CTAs
+    ("qshift_biwkv", 2, 14, 14, 64, "bf16", 0.25),  # 14 x 14: flat view, one CTA
 ]
 
 
@@ -380,9 +402,11 @@ def test_edge_shapes(vk, oracle_mod, case, kernel_path):
     run_fused(vk, oracle_mod, wl)
 
 
-@pytest.mark.parametrize("s,H,W", [(2, 6, 7), (3, 2, 300), (5, 4, 4), (2, 32, 64), (70, 8, 64)])
+@pytest.mark.parametrize("s,H,W", [(2, 6, 7), (3, 2, 300), (5, 4, 4), (2, 32, 64), (70, 8, 64), (3, 10, 13)])
 def test_large_shifts(vk, oracle_mod, s, H, W, kernel_path):
-    C = 64 if W % 8 == 0 and W <= 256 else 24  # C = 64: the TMA path qualifies
+    # C = 64: group bounds 16, 32, 48, 64, so the TMA kernels qualify (through
+    # the flat token view where W is not a multiple of 8 or exceeds 256)
+    C = 64
     wl = _custom("gate_qs", 1, H, W, C, "bf16", seed=77 + s, s=s)
     run_fused(vk, oracle_mod, wl)
     wl = _custom("gate_qs_x", 1, H, W, C, "f32", seed=78 + s, s=s)
