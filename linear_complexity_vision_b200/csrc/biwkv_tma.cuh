@@ -519,11 +519,18 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     const char* tV = smem + (QS ? 2 * SV : SV) * p.tile_bytes;
     const char* tR = smem + (QS ? 2 * SR : SR) * p.tile_bytes;
     const int dsh = shifted ? p.tile_bytes : 0;  // shifted tile = plain + dsh
+    // With 16-token chunks the lanes of chunks 4..7 of a warp take their two
+    // sub-chunks in the opposite order: at each step the warp's eight chunks
+    // read rows 2 q + (h ^ rot), eight different rows modulo 8, so tile, gate
+    // and result accesses are free of bank conflicts.  Register arrays are
+    // indexed by step; h is the sub-chunk a step works on.
+    const int rot = kH == 2 ? (cq >> 2) & 1 : 0;
     float2 n[kH][kL], dd[kH][kL];
-    float4 Fh[kH], Gh[kH];  // per sub-chunk: forward (A.xy, C.xy) and backward totals
-    float2 Mh[kH];          // per sub-chunk maximum of k (-inf if wholly past T)
+    float4 Fh[kH], Gh[kH];  // per step: forward (A.xy, C.xy) and backward totals of its sub-chunk
+    float2 Mh[kH];          // per step: its sub-chunk's maximum of k (-inf if wholly past T)
 #pragma unroll
-    for (int h = 0; h < kH; ++h) {
+    for (int st = 0; st < kH; ++st) {
+        const int h = st ^ rot;
         const int rowoff = (q * kH + h) * RB + j * PB;
         const int nv = max(0, min(kL, nvt - h * kL));
         float2 kk[kL], vv[kL];
@@ -579,7 +586,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
                 mx = max2(mx, kk[i]);
             }
         }
-        Mh[h] = mx;
+        Mh[st] = mx;
         const float2 negM = make_float2(mx.x == -INFINITY ? 0.0f : -mx.x * kLog2e,
                                         mx.y == -INFINITY ? 0.0f : -mx.y * kLog2e);
 #pragma unroll
@@ -587,31 +594,39 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
             kk[i] = ex2(fma2(kk[i], f2(kLog2e), negM));  // p_i (0 beyond T)
             vv[i] = mul2(kk[i], vv[i]);                  // p_i v_i
         }
-        float2 fa = f2(0.0f), fc = f2(0.0f);
+        // Two-sided sums inside the sub-chunk, both directions in one walk
+        // (four independent recurrences per step): step it adds the forward
+        // sum before token it and the backward sum after token 7 - it; a
+        // token's second contribution also brings its own term e^u p v.
+        float2 fa = f2(0.0f), fc = f2(0.0f), ga = f2(0.0f), gc = f2(0.0f);
 #pragma unroll
-        for (int i = 0; i < kL; ++i) {
-            n[h][i] = fa;
-            dd[h][i] = fc;
+        for (int it = 0; it < kL; ++it) {
+            const int i = it, ib = kL - 1 - it;
+            if (it < kL / 2) {
+                n[st][i] = fa;
+                dd[st][i] = fc;
+                n[st][ib] = ga;
+                dd[st][ib] = gc;
+            } else {
+                n[st][i] = add2(n[st][i], fma2(eu, vv[i], fa));
+                dd[st][i] = add2(dd[st][i], fma2(eu, kk[i], fc));
+                n[st][ib] = add2(n[st][ib], fma2(eu, vv[ib], ga));
+                dd[st][ib] = add2(dd[st][ib], fma2(eu, kk[ib], gc));
+            }
             fa = fma2(alpha, fa, vv[i]);
             fc = fma2(alpha, fc, kk[i]);
+            ga = fma2(alpha, ga, vv[ib]);
+            gc = fma2(alpha, gc, kk[ib]);
         }
-        float2 ga = f2(0.0f), gc = f2(0.0f);
-#pragma unroll
-        for (int i = kL - 1; i >= 0; --i) {
-            n[h][i] = add2(n[h][i], fma2(eu, vv[i], ga));
-            dd[h][i] = add2(dd[h][i], fma2(eu, kk[i], gc));
-            ga = fma2(alpha, ga, vv[i]);
-            gc = fma2(alpha, gc, kk[i]);
-        }
-        Fh[h] = make_float4(fa.x, fa.y, fc.x, fc.y);
-        Gh[h] = make_float4(ga.x, ga.y, gc.x, gc.y);
+        Fh[st] = make_float4(fa.x, fa.y, fc.x, fc.y);
+        Gh[st] = make_float4(ga.x, ga.y, gc.x, gc.y);
     }
 
     // ---- 3a. warp maximum (the reference of the warp's sums) and the chunk's
     // totals on it ---------------------------------------------------------------
     float2 mx = Mh[0];
 #pragma unroll
-    for (int h = 1; h < kH; ++h) mx = max2(mx, Mh[h]);
+    for (int st = 1; st < kH; ++st) mx = max2(mx, Mh[st]);
 #pragma unroll
     for (int d = kNP; d < 32; d <<= 1) {
         mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, d));
@@ -622,18 +637,22 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     const float2 mref = make_float2(mx.x == -INFINITY ? 0.0f : mx.x, mx.y == -INFINITY ? 0.0f : mx.y);
     float2 eh[kH];
 #pragma unroll
-    for (int h = 0; h < kH; ++h) eh[h] = ex2(mul2(add2(Mh[h], make_float2(-mref.x, -mref.y)), f2(kLog2e)));
+    for (int st = 0; st < kH; ++st) eh[st] = ex2(mul2(add2(Mh[st], make_float2(-mref.x, -mref.y)), f2(kLog2e)));
     auto scale4 = [](float2 e, float4 v) { return make_float4(v.x * e.x, v.y * e.y, v.z * e.x, v.w * e.y); };
+    auto sel4 = [](bool c, float4 a, float4 b) { return c ? a : b; };
     float4 Fi, Gi;
     float4 F0s = zero4(), G1s = zero4();  // KL = 16: sub-chunk 0's forward, sub-chunk 1's backward total
     if (kH == 1) {
         Fi = scale4(eh[0], Fh[0]);
         Gi = scale4(eh[0], Gh[0]);
     } else {
-        F0s = scale4(eh[0], Fh[0]);
-        G1s = scale4(eh[kH - 1], Gh[kH - 1]);
-        Fi = fma4(a8, F0s, scale4(eh[kH - 1], Fh[kH - 1]));
-        Gi = fma4(a8, G1s, scale4(eh[0], Gh[0]));
+        // sub-chunk 0 was step rot, sub-chunk 1 step 1 - rot
+        const float4 sF0 = scale4(eh[0], Fh[0]), sF1 = scale4(eh[1], Fh[1]);
+        const float4 sG0 = scale4(eh[0], Gh[0]), sG1 = scale4(eh[1], Gh[1]);
+        F0s = sel4(rot, sF1, sF0);
+        G1s = sel4(rot, sG0, sG1);
+        Fi = fma4(a8, F0s, sel4(rot, sF0, sF1));
+        Gi = fma4(a8, G1s, sel4(rot, sG1, sG0));
     }
 
     // ---- 3b. scans: warp, CTA, cluster -----------------------------------------
@@ -861,24 +880,27 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     // results go to the first input tile (dead since the load phase), at the
     // same conflict-free offsets, then leave as coalesced 16-byte stores
     char* tout = smem;
+    // carries into sub-chunk 1 from the left and into sub-chunk 0 from the
+    // right: the other sub-chunk's total joins them (16-token chunks)
+    const float2 A1 = fma2(slw, lo2(F0s), mul2(a8, As)), C1 = fma2(slw, hi2(F0s), mul2(a8, Cs));
+    const float2 B0 = fma2(slw, lo2(G1s), mul2(a8, Be)), D0 = fma2(slw, hi2(G1s), mul2(a8, De));
 #pragma unroll
-    for (int h = 0; h < kH; ++h) {
-        // carries into sub-chunk h: the other sub-chunk's total joins them
+    for (int st = 0; st < kH; ++st) {
+        const int h = st ^ rot;
         float2 Ah = As, Ch = Cs, Bh = Be, Dh = De;
-        if (kH == 2 && h == 0) {
-            Bh = fma2(slw, lo2(G1s), mul2(a8, Be));
-            Dh = fma2(slw, hi2(G1s), mul2(a8, De));
+        if (kH == 2) {
+            const bool first = h == 0;
+            Ah = first ? As : A1;
+            Ch = first ? Cs : C1;
+            Bh = first ? B0 : Be;
+            Dh = first ? D0 : De;
         }
-        if (kH == 2 && h == 1) {
-            Ah = fma2(slw, lo2(F0s), mul2(a8, As));
-            Ch = fma2(slw, hi2(F0s), mul2(a8, Cs));
-        }
-        const float2 sh = mul2(slw, eh[h]);
+        const float2 sh = mul2(slw, eh[st]);
         const int rowoff = (q * kH + h) * RB + j * PB;
 #pragma unroll
         for (int i = 0; i < kL; ++i) {
-            const float2 num = fma2(sh, n[h][i], fma2(pw[i], Ah, mul2(pw[kL - 1 - i], Bh)));
-            float2 den = fma2(sh, dd[h][i], fma2(pw[i], Ch, mul2(pw[kL - 1 - i], Dh)));
+            const float2 num = fma2(sh, n[st][i], fma2(pw[i], Ah, mul2(pw[kL - 1 - i], Bh)));
+            float2 den = fma2(sh, dd[st][i], fma2(pw[i], Ch, mul2(pw[kL - 1 - i], Dh)));
             if (GATE) {
                 // read before the result overwrites the first slot
                 const int o = rowoff + i * SUB;
