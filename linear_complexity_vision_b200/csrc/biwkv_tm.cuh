@@ -95,7 +95,7 @@ struct alignas(16) Scratch {
     float4 ownF[kNP];
     float4 ownG[kNP];
     float2 ownM[kNP];
-    unsigned long long bar;
+    unsigned long long bar[kNW];  // tile boxes of warp w's 256 tokens
     unsigned long long xbar;
     unsigned int tmem;  // base address of this CTA's tensor-memory columns
     int tk;             // GX: this CTA's ticket
@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     const int cq = q % kCPW;   // chunk within the warp
     const int warp = tid >> 5;
     if (tid == 0) {
-        mbar_init(&S.bar, 1);
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) mbar_init(&S.bar[w], 1);
         if (!GX && p.ncl > 1) {
             mbar_init(&S.xbar, 1);
             mbar_expect_tx(&S.xbar, (unsigned)(p.ncl * kNP * (sizeof(float4) * 2 + sizeof(float2))));
@@ -211,18 +212,6 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
             return;
         }
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (!GX && p.ncl > 1) cluster_arrive_relaxed();  // waited for before the first push
-    // this thread's lane of the CTA's columns
-    const uint32_t tmem = S.tmem + ((uint32_t)(warp * 32) << 16);
 
     // this CTA's column chunk: the block index, or (GX) the ticket, column by
     // column so a column's CTAs hold consecutive tickets
@@ -243,33 +232,43 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     if (grp >= p.ng) grp = 4;
     const bool shifted = QS && grp < 4;
 
-    // ---- tile loads: lane i of warp 0 loads sub-tile i of each tile -----------
+    // ---- tile loads, first of all: lane i of warp 0 loads sub-tile i of each
+    // tile.  In the flat token view (no Q-Shift, or Q-Shift at any W) the
+    // boxes are 256 strided tokens: box h holds warp h's tokens and completes
+    // on that warp's barrier, so a warp starts on its own tokens as soon as
+    // they are in; the shifted tile is the same boxes displaced by the group's
+    // token offset.  In the image view (C, W, H, B) one box holds the CTA's
+    // rows (four times fewer, larger copies; measured faster with Q-Shift at
+    // W = 64), displaced by +-s along w or h, and completes on barrier 0. ----------
+    const bool img = QS && !p.flat;
     if (warp == 0) {
-        if (tid == 0)
-            mbar_expect_tx(&S.bar, (unsigned)p.box_bytes * (unsigned)(kL * NSRC * (shifted ? 2 : 1)));
+        // bytes per lane and source: a box of 32 rows of a sub-tile per warp in
+        // the flat view; the CTA's (W / 8) x rows rows in the image view
+        constexpr unsigned kBoxBytes = 32 * RB;
+        const unsigned copies = (unsigned)(kL * NSRC * (shifted ? 2 : 1));
+        if (tid < kNW && (!img || tid == 0))
+            mbar_expect_tx(&S.bar[tid], (img ? (unsigned)p.box_bytes : kBoxBytes) * copies);
         __syncwarp();
         if (tid < kL) {
-            const int i = tid, h0 = rank * p.rows;
-            for (int s = 0; s < NSRC; ++s) {
-                char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB;
-                if (!QS || p.flat) {
+            const int i = tid;
+            const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
+            const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
+            if (img) {
+                const int h0 = rank * p.rows;
+                for (int s = 0; s < NSRC; ++s) {
+                    char* plain = smem + 2 * s * p.tile_bytes + i * SUB;
+                    tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar[0]);
+                    if (shifted) tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, h0 + dh, b, &S.bar[0]);
+                }
+            } else {
+                const int dt = dw + dh * p.W;
 #pragma unroll
-                    for (int h = 0; h < kTc / 256; ++h)
-                        tma_load_3d(plain + h * 32 * RB, &p.map[s], c0, t0 + i + 256 * h, b, &S.bar);
-                    if (QS && shifted) {
-                        // the flat view: the same boxes displaced by the group's token offset
-                        const int dt = grp == 0 ? -p.s : (grp == 1 ? p.s : (grp == 2 ? -p.s * p.W : p.s * p.W));
-#pragma unroll
-                        for (int h = 0; h < kTc / 256; ++h)
-                            tma_load_3d(plain + p.tile_bytes + h * 32 * RB, &p.map[s], c0, t0 + i + dt + 256 * h, b,
-                                        &S.bar);
-                    }
-                } else {
-                    tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar);
-                    if (shifted) {
-                        const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
-                        const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
-                        tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, h0 + dh, b, &S.bar);
+                for (int h = 0; h < kNW; ++h) {
+                    for (int s = 0; s < NSRC; ++s) {
+                        char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB + h * 32 * RB;
+                        tma_load_3d(plain, &p.map[s], c0, t0 + i + 256 * h, b, &S.bar[h]);
+                        if (QS && shifted)
+                            tma_load_3d(plain + p.tile_bytes, &p.map[s], c0, t0 + i + dt + 256 * h, b, &S.bar[h]);
                     }
                 }
             }
@@ -293,11 +292,30 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
 
     const int nvt = max(0, min(kKL, tend - (t0 + q * kKL)));  // valid tokens of this chunk
 
-    if (tid == 0) mbar_wait_bounded(&S.bar, p.err);
+    // tensor memory; the CTA barrier also publishes the decay table and the
+    // tile barriers' initialisation to every warp
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    if (!GX && p.ncl > 1) cluster_arrive_relaxed();  // waited for before the first push
+    // this thread's lane of the CTA's columns
+    const uint32_t tmem = S.tmem + ((uint32_t)(warp * 32) << 16);
+
+    // this warp's tokens: every lane waits (bounded) for their boxes; with
+    // Q-Shift in a horizontal group the warp then clears its row-wrapped
+    // tokens of the shifted tiles
+    mbar_wait_bounded(&S.bar[img ? 0 : warp], p.err);
     if (QS && p.flat && shifted && grp < 2) {
-        fast::zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, tend, p.W, p.s, grp == 0, tid, kThreads);
-        __syncthreads();
+        const int lo = t0 + warp * kWarpTok;
+        fast::zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, lo, min(tend, lo + kWarpTok), p.W, p.s,
+                                grp == 0, tid & 31, 32);
+        __syncwarp();
     }
 
     // ---- 1-2. per 8-token sub-chunk: load, Q-Shift mix, gate factor (parked in

@@ -165,21 +165,24 @@ struct alignas(16) Scratch {
 // offset -s W or +s W leaves [0, T) exactly where the row leaves [0, H), and
 // the TMA's zero fill covers it.  Token tl of the CTA sits at sub-tile tl % 8,
 // row tl / 8.
+// The tokens cleared are those in [lo, hi); t0 is the CTA's first token.
+// Threads take image rows; one division per thread.
 template <int RB>
-__device__ __forceinline__ void zero_row_wrap(char* smem, int tile_bytes, int sub_bytes, int nsrc, int t0, int tend,
-                                              int W, int s, bool left, int tid, int nthreads) {
+__device__ __forceinline__ void zero_row_wrap(char* smem, int tile_bytes, int sub_bytes, int nsrc, int t0, int lo,
+                                              int hi, int W, int s, bool left, int tid, int nthreads) {
+    if (hi <= lo) return;
     const int sw = min(s, W);  // source outside the row: w < s (left) or w >= W - s
-    const int h0 = t0 / W, nrow = (tend - 1) / W - h0 + 1;
-    const int per_src = nrow * sw;
-    for (int e = tid; e < nsrc * per_src; e += nthreads) {
-        const int src = e / per_src, r = e - src * per_src;
-        const int hr = h0 + r / sw, k = r % sw;
-        const int t = hr * W + (left ? k : W - 1 - k);
-        if (t < t0 || t >= tend) continue;
-        const int tl = t - t0;
-        char* dst = smem + (2 * src + 1) * tile_bytes + (tl & (kL - 1)) * sub_bytes + (tl / kL) * RB;
+    for (int hr = lo / W + tid, t_row = hr * W; t_row < hi; hr += nthreads, t_row += nthreads * W) {
+        for (int k = 0; k < sw; ++k) {
+            const int t = t_row + (left ? k : W - 1 - k);
+            if (t < lo || t >= hi) continue;
+            const int tl = t - t0;
+            for (int src = 0; src < nsrc; ++src) {
+                char* dst = smem + (2 * src + 1) * tile_bytes + (tl & (kL - 1)) * sub_bytes + (tl / kL) * RB;
 #pragma unroll
-        for (int o = 0; o < RB; o += 16) *reinterpret_cast<uint4*>(dst + o) = make_uint4(0u, 0u, 0u, 0u);
+                for (int o = 0; o < RB; o += 16) *reinterpret_cast<uint4*>(dst + o) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
     }
 }
 
@@ -506,7 +509,7 @@ __global__ void __launch_bounds__(NT, Cfg<NT, KL>::kMinBlocks)
     if (tid == 0) mbar_wait_bounded(&S.bar, p.err);
     __syncthreads();
     if (QS && p.flat && shifted && grp < 2) {
-        zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, tend, p.W, p.s, grp == 0, tid, kThreads);
+        zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, t0, tend, p.W, p.s, grp == 0, tid, kThreads);
         __syncthreads();
     }
 
