@@ -233,42 +233,41 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     const bool shifted = QS && grp < 4;
 
     // ---- tile loads, first of all: lane i of warp 0 loads sub-tile i of each
-    // tile.  In the flat token view (no Q-Shift, or Q-Shift at any W) the
-    // boxes are 256 strided tokens: box h holds warp h's tokens and completes
-    // on that warp's barrier, so a warp starts on its own tokens as soon as
-    // they are in; the shifted tile is the same boxes displaced by the group's
-    // token offset.  In the image view (C, W, H, B) one box holds the CTA's
-    // rows (four times fewer, larger copies; measured faster with Q-Shift at
-    // W = 64), displaced by +-s along w or h, and completes on barrier 0. ----------
+    // tile in nbox boxes; box g holds the tokens of warps g * 4 / nbox onwards
+    // and completes on tile barrier g, so warps start on their own tokens as
+    // soon as those are in.  Fewer, larger boxes cost the TMA less per byte
+    // (measured): the host picks nbox per view.  Views: the image (C, W, H, B)
+    // with Q-Shift where W allows (boxes of rows / nbox image rows, the
+    // shifted tile displaced by +-s along w or h); without Q-Shift, when T is
+    // a multiple of 256, tokens folded as (C, 256, T / 256, B) (boxes of 4 /
+    // nbox folds); otherwise the flat (C, T, B) with a box of 256 strided
+    // tokens per warp (the shifted tile displaced by the group's token
+    // offset). ------------------------------------------------------------------------
     const bool img = QS && !p.flat;
+    const int nb = p.nbox, wpb = kNW / nb;  // boxes per lane and tile, warps per box
     if (warp == 0) {
-        // bytes per lane and source: a box of 32 rows of a sub-tile per warp in
-        // the flat view; the CTA's (W / 8) x rows rows in the image view
-        constexpr unsigned kBoxBytes = 32 * RB;
+        // bytes per lane and source: p.box_bytes in all, a share per box
         const unsigned copies = (unsigned)(kL * NSRC * (shifted ? 2 : 1));
-        if (tid < kNW && (!img || tid == 0))
-            mbar_expect_tx(&S.bar[tid], (img ? (unsigned)p.box_bytes : kBoxBytes) * copies);
+        if (tid < nb) mbar_expect_tx(&S.bar[tid], (unsigned)p.box_bytes / (unsigned)nb * copies);
         __syncwarp();
         if (tid < kL) {
             const int i = tid;
             const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
             const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
-            if (img) {
-                const int h0 = rank * p.rows;
+            const int dt = dw + dh * p.W;
+            for (int g = 0; g < nb; ++g) {
                 for (int s = 0; s < NSRC; ++s) {
-                    char* plain = smem + 2 * s * p.tile_bytes + i * SUB;
-                    tma_load_4d(plain, &p.map[s], c0, i, h0, b, &S.bar[0]);
-                    if (shifted) tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, h0 + dh, b, &S.bar[0]);
-                }
-            } else {
-                const int dt = dw + dh * p.W;
-#pragma unroll
-                for (int h = 0; h < kNW; ++h) {
-                    for (int s = 0; s < NSRC; ++s) {
-                        char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB + h * 32 * RB;
-                        tma_load_3d(plain, &p.map[s], c0, t0 + i + 256 * h, b, &S.bar[h]);
+                    char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB + g * wpb * 32 * RB;
+                    if (img) {
+                        const int r0 = rank * p.rows + g * (p.rows / nb);
+                        tma_load_4d(plain, &p.map[s], c0, i, r0, b, &S.bar[g]);
+                        if (shifted) tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, r0 + dh, b, &S.bar[g]);
+                    } else if (!QS && nb < kNW) {
+                        tma_load_4d(plain, &p.map[s], c0, i, t0 / 256 + g * wpb, b, &S.bar[g]);
+                    } else {
+                        tma_load_3d(plain, &p.map[s], c0, t0 + i + 256 * g, b, &S.bar[g]);
                         if (QS && shifted)
-                            tma_load_3d(plain + p.tile_bytes, &p.map[s], c0, t0 + i + dt + 256 * h, b, &S.bar[h]);
+                            tma_load_3d(plain + p.tile_bytes, &p.map[s], c0, t0 + i + dt + 256 * g, b, &S.bar[g]);
                     }
                 }
             }
@@ -310,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     // this warp's tokens: every lane waits (bounded) for their boxes; with
     // Q-Shift in a horizontal group the warp then clears its row-wrapped
     // tokens of the shifted tiles
-    mbar_wait_bounded(&S.bar[img ? 0 : warp], p.err);
+    mbar_wait_bounded(&S.bar[warp / wpb], p.err);
     if (QS && p.flat && shifted && grp < 2) {
         const int lo = t0 + warp * kWarpTok;
         fast::zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, lo, min(tend, lo + kWarpTok), p.W, p.s,
@@ -704,9 +703,13 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
     if (tid < kL) {
-        const int nbox = (tend - t0 + 255) / 256;
-        for (int hb = 0; hb < nbox; ++hb)
-            tma_store_3d(&p.omap, tout + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
+        if (p.ofold) {
+            fast::tma_store_4d(&p.omap, tout + tid * SUB, c0, tid, t0 / 256, b);
+        } else {
+            const int nbox = (tend - t0 + 255) / 256;
+            for (int hb = 0; hb < nbox; ++hb)
+                tma_store_3d(&p.omap, tout + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
+        }
         bulk_commit_and_wait_read();
     }
     if (warp == 1) {

@@ -109,6 +109,10 @@ struct alignas(64) Params {
     int tma_store;       // results leave by TMA stores (the CTA's span is whole boxes, or the column's end)
     int flat;            // Q-Shift through the flat (C, T, B) view: shifted tiles loaded at a token
                          // offset, row-wrapped tokens of horizontal groups zeroed after the load
+    int nbox;            // tensor-memory kernel: boxes per lane and tile (1, 2 or 4); box g holds
+                         // warps g * 4 / nbox onwards and completes on their tile barrier g
+    int ofold;           // tensor-memory kernel: omap is the folded (C, 256, T / 256, B) view and a
+                         // lane stores its sub-tile in one box of four folds
     // global-memory exchange (GX kernels only): see the workspace layout below
     unsigned int* ws_ctl;   // [0] ticket counter, [1] finished CTAs, [2] generation
     unsigned int* ws_flag;  // per (column, rank): generation + 1 once its record is out
@@ -254,6 +258,13 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                      reinterpret_cast<unsigned long long>(map)),
                  "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                             int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                     reinterpret_cast<unsigned long long>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit_and_wait_read() {

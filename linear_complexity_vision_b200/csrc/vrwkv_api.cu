@@ -791,6 +791,22 @@ int qs_view_forced() {
     return e[0] == 'f' ? 1 : (e[0] == 'i' ? -1 : 0);
 }
 
+// VRWKV_TM_NBOX=1, 2 or 4: boxes per lane and tile of the tensor-memory
+// kernel where its view allows that count (diagnostics and tests); 0 = the
+// library's choice.
+int tm_nbox_forced() {
+    const char* e = getenv("VRWKV_TM_NBOX");
+    if (!e || e[1] != 0) return 0;
+    return e[0] == '1' ? 1 : (e[0] == '2' ? 2 : (e[0] == '4' ? 4 : 0));
+}
+
+// VRWKV_TM_OFOLD=0 keeps the tensor-memory kernel's result stores at one
+// 256-token box each (diagnostics and tests).
+bool tm_ofold_disabled() {
+    const char* e = getenv("VRWKV_TM_OFOLD");
+    return e && e[0] == '0' && e[1] == 0;
+}
+
 // VRWKV_SHORT_CTA=0 keeps columns of at most 256 tokens on the 512-token CTA
 // shape (diagnostics and tests).
 bool short_cta_disabled() {
@@ -901,12 +917,18 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
                         break;
                     }
             }
-            if (rows == 0 || rows > 256) return false;
-            p.rows = rows;
-            p.Tc = rows * p.W;
-            p.ncl = (p.H + rows - 1) / rows;
+            if (rows == 0 || rows > 256) {
+                // whole image rows cannot make whole warps: the flat view
+                if (qs_view_forced() < 0) return false;
+                p.flat = 1;
+            } else {
+                p.rows = rows;
+                p.Tc = rows * p.W;
+                p.ncl = (p.H + rows - 1) / rows;
+            }
         }
-    } else {
+    }
+    if (!pl.qs || p.flat) {
         if (!pl.qs) {
             p.H = 1;
             p.W = T;
@@ -933,6 +955,22 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     if (pl.smem > 227 * 1024) return false;
     const CUtensorMapDataType dt =
         dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    // Boxes per lane and tile of the tensor-memory kernel (fewer, larger boxes
+    // cost the TMA less; measured at T = 4096): one image-view box with
+    // Q-Shift, one box of four 256-token folds without it when T is a
+    // multiple of 256, else one 256-token box per warp.  VRWKV_TM_NBOX=1, 2
+    // or 4 asks for another count where the view allows it (diagnostics).
+    p.nbox = tm32::kNW;
+    const bool fold = pl.tm && !pl.qs && T % 256 == 0;  // tokens folded as (C, 256, T / 256, B)
+    if (pl.tm) {
+        const int want = tm_nbox_forced();
+        if (pl.qs && !p.flat) {
+            const int nb = want ? want : 1;
+            p.nbox = (p.rows % nb == 0 && p.rows * p.W == tm32::kTc) ? nb : 1;
+        } else if (fold) {
+            p.nbox = want ? want : 1;
+        }
+    }
     for (int i = 0; i < nsrc; ++i) {
         CUresult cr;
         // element stride 8 along the token (w) axis: box i holds tokens 8q + i
@@ -941,7 +979,15 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
             const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)B};
             const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)p.W * C * es,
                                            (cuuint64_t)p.H * p.W * C * es};
-            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, (cuuint32_t)p.W, (cuuint32_t)p.rows, 1};
+            const cuuint32_t rows = pl.tm ? (cuuint32_t)(p.rows / p.nbox) : (cuuint32_t)p.rows;
+            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, (cuuint32_t)p.W, rows, 1};
+            cr = enc(&p.map[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        } else if (fold && p.nbox < tm32::kNW) {
+            const cuuint64_t dims[4] = {(cuuint64_t)C, 256, (cuuint64_t)T / 256, (cuuint64_t)B};
+            const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)256 * C * es, (cuuint64_t)T * C * es};
+            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, 256u, (cuuint32_t)(tm32::kNW / p.nbox), 1};
             cr = enc(&p.map[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -958,14 +1004,27 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     {
         // the output in the tiles' layout: boxes of 256 strided tokens; a CTA
         // stores by TMA when its span is whole boxes or ends the column, so no
-        // box reaches another CTA's tokens (the tensor bound clips at T)
-        const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
-        const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
-        const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, 256u, 1};
-        const cuuint32_t estr[3] = {1, (cuuint32_t)fast::kL, 1};
-        const CUresult cr = enc(&p.omap, dt, 3, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        // box reaches another CTA's tokens (the tensor bound clips at T).  The
+        // tensor-memory kernel at T a multiple of 256 stores four folds of 256
+        // tokens per box instead (one store per lane), where a CTA spans 1024
+        // tokens or the whole column (a box never reaches another CTA's tokens).
+        p.ofold = pl.tm && T % 256 == 0 && (p.Tc == tm32::kTc || p.ncl == 1) && !tm_ofold_disabled() ? 1 : 0;
+        CUresult cr;
+        if (p.ofold) {
+            const cuuint64_t dims[4] = {(cuuint64_t)C, 256, (cuuint64_t)T / 256, (cuuint64_t)B};
+            const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)256 * C * es, (cuuint64_t)T * C * es};
+            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, 256u, (cuuint32_t)tm32::kNW, 1};
+            const cuuint32_t estr[4] = {1, (cuuint32_t)fast::kL, 1, 1};
+            cr = enc(&p.omap, dt, 4, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        } else {
+            const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+            const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
+            const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, 256u, 1};
+            const cuuint32_t estr[3] = {1, (cuuint32_t)fast::kL, 1};
+            cr = enc(&p.omap, dt, 3, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        }
         p.tma_store = (cr == CUDA_SUCCESS && (p.Tc % 256 == 0 || p.ncl == 1) && !tma_store_disabled()) ? 1 : 0;
     }
     p.invT = (float)(1.0 / (double)T);

@@ -315,6 +315,32 @@ def test_tm_kernel_shapes(vk, oracle_mod, case, rot, monkeypatch):
     assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tm_kernel"
 
 
+# The tensor-memory kernel's copy shapes: 1, 2 or 4 boxes per lane and tile
+# (one per 1024, 512 or 256 tokens) in the image view with Q-Shift and the
+# folded token view without, and the folded result store on and off.
+NBOX_CASES = [
+    # call, B, H, W, C, dtype
+    ("gate_qs_x", 2, 64, 64, 64, "bf16"),     # image view, 16 rows per CTA
+    ("gate_qs", 1, 32, 32, 32, "f32"),        # image view, 32 rows per CTA, float32
+    ("biwkv", 2, 1, 3072, 32, "bf16"),        # folded view, 3 CTAs
+    ("gate_x", 1, 1, 1280, 16, "f32"),        # folded view, a second CTA of one fold
+    ("gate_qs_x", 1, 40, 40, 32, "bf16"),     # flat view (W = 40 does not divide 1024)
+]
+
+
+@pytest.mark.parametrize("ofold", ["1", "0"])
+@pytest.mark.parametrize("nbox", ["1", "2", "4"])
+@pytest.mark.parametrize("case", NBOX_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_tm_box_counts(vk, oracle_mod, case, nbox, ofold, monkeypatch):
+    monkeypatch.setenv("VRWKV_FORWARD", "tm")
+    monkeypatch.setenv("VRWKV_TM_NBOX", nbox)
+    monkeypatch.setenv("VRWKV_TM_OFOLD", ofold)
+    call, B, H, W, C, dt = case
+    wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000)
+    run_fused(vk, oracle_mod, wl)
+    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tm_kernel"
+
+
 # Sequences past 4096 tokens: the pages' efficiency comparison runs 2048^2
 # images at patch 16, T = 16384 ("Vision-RWKV Backbone", Ablation /
 # efficiency analysis, Fig. 3(b)).  With a workspace the 16-channel kernel
