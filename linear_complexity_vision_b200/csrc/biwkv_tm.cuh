@@ -66,6 +66,7 @@ using fast::st_async4;
 using fast::sts_f32;
 using fast::tma_load_3d;
 using fast::tma_load_4d;
+using fast::tma_load_5d;
 using fast::tma_store_3d;
 using fast::zero4;
 
@@ -232,42 +233,67 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     if (grp >= p.ng) grp = 4;
     const bool shifted = QS && grp < 4;
 
-    // ---- tile loads, first of all: lane i of warp 0 loads sub-tile i of each
-    // tile in nbox boxes; box g holds the tokens of warps g * 4 / nbox onwards
-    // and completes on tile barrier g, so warps start on their own tokens as
-    // soon as those are in.  Fewer, larger boxes cost the TMA less per byte
-    // (measured): the host picks nbox per view.  Views: the image (C, W, H, B)
-    // with Q-Shift where W allows (boxes of rows / nbox image rows, the
-    // shifted tile displaced by +-s along w or h); without Q-Shift, when T is
-    // a multiple of 256, tokens folded as (C, 256, T / 256, B) (boxes of 4 /
-    // nbox folds); otherwise the flat (C, T, B) with a box of 256 strided
-    // tokens per warp (the shifted tile displaced by the group's token
-    // offset). ------------------------------------------------------------------------
+    // ---- tile loads, first of all.  Fewer, larger boxes cost the TMA less per
+    // byte (measured), so where the shape allows (imaj) a tile arrives in one
+    // box from a residue-major view that puts token 8 m + i at sub-tile i, row
+    // m: (C, T / 8, 8, B) over the flat tokens, (C, W / 8, H, 8, B) over the
+    // image with Q-Shift.  A vertical shift displaces the image box along h; a
+    // horizontal shift (and any shift in the flat view) has lane i of warp 0
+    // load sub-tile i of the shifted tile from a lane-strided view (xmap):
+    // displaced by +-s along w in the image, by the group's token offset in
+    // the flat tokens.  Elsewhere lane i loads sub-tile i of every tile in
+    // nbox boxes; box g holds the tokens of warps g * 4 / nbox onwards and
+    // completes on tile barrier g. ----------------------------------------------------
     const bool img = QS && !p.flat;
     const int nb = p.nbox, wpb = kNW / nb;  // boxes per lane and tile, warps per box
     if (warp == 0) {
-        // bytes per lane and source: p.box_bytes in all, a share per box
-        const unsigned copies = (unsigned)(kL * NSRC * (shifted ? 2 : 1));
-        if (tid < nb) mbar_expect_tx(&S.bar[tid], (unsigned)p.box_bytes / (unsigned)nb * copies);
-        __syncwarp();
-        if (tid < kL) {
-            const int i = tid;
-            const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
-            const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
-            const int dt = dw + dh * p.W;
-            for (int g = 0; g < nb; ++g) {
-                for (int s = 0; s < NSRC; ++s) {
-                    char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB + g * wpb * 32 * RB;
+        const int dw = grp == 0 ? -p.s : (grp == 1 ? p.s : 0);
+        const int dh = grp == 2 ? -p.s : (grp == 3 ? p.s : 0);
+        const int dt = dw + dh * p.W;
+        const int r0 = rank * p.rows;
+        if (p.imaj) {
+            if (tid == 0) mbar_expect_tx(&S.bar[0], (unsigned)p.tile_bytes * (unsigned)(NSRC * (shifted ? 2 : 1)));
+            __syncwarp();
+            const bool one_shift = img && dh != 0;  // the shifted tile in one box too
+            for (int s = 0; s < NSRC; ++s) {
+                char* tile = smem + (QS ? 2 * s : s) * p.tile_bytes;
+                if (tid == 0) {
                     if (img) {
-                        const int r0 = rank * p.rows + g * (p.rows / nb);
-                        tma_load_4d(plain, &p.map[s], c0, i, r0, b, &S.bar[g]);
-                        if (shifted) tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, r0 + dh, b, &S.bar[g]);
-                    } else if (!QS && nb < kNW) {
-                        tma_load_4d(plain, &p.map[s], c0, i, t0 / 256 + g * wpb, b, &S.bar[g]);
+                        tma_load_5d(tile, &p.map[s], c0, 0, r0, 0, b, &S.bar[0]);
+                        if (shifted && one_shift) tma_load_5d(tile + p.tile_bytes, &p.map[s], c0, 0, r0 + dh, 0, b, &S.bar[0]);
                     } else {
-                        tma_load_3d(plain, &p.map[s], c0, t0 + i + 256 * g, b, &S.bar[g]);
-                        if (QS && shifted)
-                            tma_load_3d(plain + p.tile_bytes, &p.map[s], c0, t0 + i + dt + 256 * g, b, &S.bar[g]);
+                        tma_load_4d(tile, &p.map[s], c0, t0 / kL, 0, b, &S.bar[0]);
+                    }
+                }
+                if (shifted && !one_shift && tid < kL) {
+                    char* sh = tile + p.tile_bytes + tid * SUB;
+                    if (img) {
+                        tma_load_4d(sh, &p.xmap[s], c0, tid + dw, r0, b, &S.bar[0]);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < kNW; ++g)
+                            tma_load_3d(sh + g * 32 * RB, &p.xmap[s], c0, t0 + tid + dt + 256 * g, b, &S.bar[0]);
+                    }
+                }
+            }
+        } else {
+            // bytes per lane and source: p.box_bytes in all, a share per box
+            const unsigned copies = (unsigned)(kL * NSRC * (shifted ? 2 : 1));
+            if (tid < nb) mbar_expect_tx(&S.bar[tid], (unsigned)p.box_bytes / (unsigned)nb * copies);
+            __syncwarp();
+            if (tid < kL) {
+                const int i = tid;
+                for (int g = 0; g < nb; ++g) {
+                    for (int s = 0; s < NSRC; ++s) {
+                        char* plain = smem + (QS ? 2 * s : s) * p.tile_bytes + i * SUB + g * wpb * 32 * RB;
+                        if (img) {
+                            tma_load_4d(plain, &p.map[s], c0, i, r0, b, &S.bar[g]);
+                            if (shifted) tma_load_4d(plain + p.tile_bytes, &p.map[s], c0, i + dw, r0 + dh, b, &S.bar[g]);
+                        } else {
+                            tma_load_3d(plain, &p.map[s], c0, t0 + i + 256 * g, b, &S.bar[g]);
+                            if (QS && shifted)
+                                tma_load_3d(plain + p.tile_bytes, &p.map[s], c0, t0 + i + dt + 256 * g, b, &S.bar[g]);
+                        }
                     }
                 }
             }
@@ -704,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     __syncthreads();
     if (tid < kL) {
         if (p.ofold) {
-            fast::tma_store_4d(&p.omap, tout + tid * SUB, c0, tid, t0 / 256, b);
+            if (tid == 0) fast::tma_store_4d(&p.omap, tout, c0, t0 / kL, 0, b);
         } else {
             const int nbox = (tend - t0 + 255) / 256;
             for (int hb = 0; hb < nbox; ++hb)

@@ -109,10 +109,14 @@ struct alignas(64) Params {
     int tma_store;       // results leave by TMA stores (the CTA's span is whole boxes, or the column's end)
     int flat;            // Q-Shift through the flat (C, T, B) view: shifted tiles loaded at a token
                          // offset, row-wrapped tokens of horizontal groups zeroed after the load
-    int nbox;            // tensor-memory kernel: boxes per lane and tile (1, 2 or 4); box g holds
-                         // warps g * 4 / nbox onwards and completes on their tile barrier g
-    int ofold;           // tensor-memory kernel: omap is the folded (C, 256, T / 256, B) view and a
-                         // lane stores its sub-tile in one box of four folds
+    // tensor-memory kernel only:
+    int nbox;            // boxes per lane and tile (1 or 4); box g holds warps g * 4 / nbox onwards
+                         // and completes on their tile barrier g
+    int imaj;            // map[] are residue-major views (one box fills a whole tile, sub-tile i
+                         // holding the tokens 8 m + i); xmap[] are the lane-strided views of the
+                         // shifted tiles that a single box cannot displace
+    int ofold;           // omap is the residue-major view: one store writes the CTA's results
+    CUtensorMap xmap[3];
     // global-memory exchange (GX kernels only): see the workspace layout below
     unsigned int* ws_ctl;   // [0] ticket counter, [1] finished CTAs, [2] generation
     unsigned int* ws_flag;  // per (column, rank): generation + 1 once its record is out
@@ -259,6 +263,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                      reinterpret_cast<unsigned long long>(map)),
                  "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
                  : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            int c3, int c4, unsigned long long* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+        "r"(smem_u32(bar))
+        : "memory");
 }
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
                                              int c3) {

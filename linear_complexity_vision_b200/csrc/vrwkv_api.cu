@@ -791,19 +791,18 @@ int qs_view_forced() {
     return e[0] == 'f' ? 1 : (e[0] == 'i' ? -1 : 0);
 }
 
-// VRWKV_TM_NBOX=1, 2 or 4: boxes per lane and tile of the tensor-memory
-// kernel where its view allows that count (diagnostics and tests); 0 = the
-// library's choice.
-int tm_nbox_forced() {
-    const char* e = getenv("VRWKV_TM_NBOX");
-    if (!e || e[1] != 0) return 0;
-    return e[0] == '1' ? 1 : (e[0] == '2' ? 2 : (e[0] == '4' ? 4 : 0));
+// VRWKV_TM_IMAJ=0 keeps the tensor-memory kernel's tile loads on
+// lane-strided boxes (eight or more per tile) instead of one residue-major
+// box (diagnostics and tests).
+bool tm_imaj_disabled() {
+    const char* e = getenv("VRWKV_TM_IMAJ");
+    return e && e[0] == '0' && e[1] == 0;
 }
 
-// VRWKV_TM_OFOLD=0 keeps the tensor-memory kernel's result stores at one
-// 256-token box each (diagnostics and tests).
+// VRWKV_TM_OSTORE=0 keeps the tensor-memory kernel's result stores at one
+// lane-strided 256-token box each (diagnostics and tests).
 bool tm_ofold_disabled() {
-    const char* e = getenv("VRWKV_TM_OFOLD");
+    const char* e = getenv("VRWKV_TM_OSTORE");
     return e && e[0] == '0' && e[1] == 0;
 }
 
@@ -955,78 +954,82 @@ bool plan_fast(FastPlan& pl, bool gate, const void* r, const void* k, const void
     if (pl.smem > 227 * 1024) return false;
     const CUtensorMapDataType dt =
         dtype == VRWKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    // Boxes per lane and tile of the tensor-memory kernel (fewer, larger boxes
-    // cost the TMA less; measured at T = 4096): one image-view box with
-    // Q-Shift, one box of four 256-token folds without it when T is a
-    // multiple of 256, else one 256-token box per warp.  VRWKV_TM_NBOX=1, 2
-    // or 4 asks for another count where the view allows it (diagnostics).
-    p.nbox = tm32::kNW;
-    const bool fold = pl.tm && !pl.qs && T % 256 == 0;  // tokens folded as (C, 256, T / 256, B)
-    if (pl.tm) {
-        const int want = tm_nbox_forced();
-        if (pl.qs && !p.flat) {
-            const int nb = want ? want : 1;
-            p.nbox = (p.rows % nb == 0 && p.rows * p.W == tm32::kTc) ? nb : 1;
-        } else if (fold) {
-            p.nbox = want ? want : 1;
-        }
-    }
-    for (int i = 0; i < nsrc; ++i) {
-        CUresult cr;
-        // element stride 8 along the token (w) axis: box i holds tokens 8q + i
+    const cuuint64_t ces = (cuuint64_t)C * es;  // bytes per token
+    auto encode = [&](CUtensorMap* m, const void* src, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                      const cuuint32_t* box, const cuuint32_t* estr, CUtensorMapL2promotion l2) {
+        return enc(m, dt, rank, const_cast<void*>(src), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    const auto l2_in = CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+    const auto l2_out = CU_TENSOR_MAP_L2_PROMOTION_NONE;
+    // Lane-strided views (element stride 8 along the tokens: lane i's box
+    // holds tokens 8 m + i): the image (C, W, H, B) with boxes of `rows` image
+    // rows, and the flat tokens (C, T, B) with boxes of 256 tokens.
+    auto image_strided = [&](CUtensorMap* m, const void* src, int rows) {
+        const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)B};
+        const cuuint64_t strides[3] = {ces, (cuuint64_t)p.W * ces, (cuuint64_t)p.H * p.W * ces};
+        const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, (cuuint32_t)p.W, (cuuint32_t)rows, 1};
         const cuuint32_t estr[4] = {1, (cuuint32_t)fast::kL, 1, 1};
-        if (pl.qs && !p.flat) {
-            const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)B};
-            const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)p.W * C * es,
-                                           (cuuint64_t)p.H * p.W * C * es};
-            const cuuint32_t rows = pl.tm ? (cuuint32_t)(p.rows / p.nbox) : (cuuint32_t)p.rows;
-            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, (cuuint32_t)p.W, rows, 1};
-            cr = enc(&p.map[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        } else if (fold && p.nbox < tm32::kNW) {
-            const cuuint64_t dims[4] = {(cuuint64_t)C, 256, (cuuint64_t)T / 256, (cuuint64_t)B};
-            const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)256 * C * es, (cuuint64_t)T * C * es};
-            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, 256u, (cuuint32_t)(tm32::kNW / p.nbox), 1};
-            cr = enc(&p.map[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        } else {
-            const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
-            const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
-            const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, 256u, 1};  // 32 strided rows
-            cr = enc(&p.map[i], dt, 3, const_cast<void*>(srcs[i]), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        return encode(m, src, 4, dims, strides, box, estr, l2_in);
+    };
+    auto flat_strided = [&](CUtensorMap* m, const void* src, CUtensorMapL2promotion l2) {
+        const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+        const cuuint64_t strides[2] = {ces, (cuuint64_t)T * ces};
+        const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, 256u, 1};
+        const cuuint32_t estr[3] = {1, (cuuint32_t)fast::kL, 1};
+        return encode(m, src, 3, dims, strides, box, estr, l2);
+    };
+    // Residue-major views for the tensor-memory kernel (T a multiple of 8):
+    // the tokens as (C, T / 8, 8, B), token 8 m + i at (m, i), and the image
+    // as (C, W / 8, H, 8, B); the residue axis is outermost in the box, so one
+    // box fills all eight sub-tiles of a tile (128 rows each).
+    auto flat_residue = [&](CUtensorMap* m, const void* src, CUtensorMapL2promotion l2) {
+        const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)T / 8, 8, (cuuint64_t)B};
+        const cuuint64_t strides[3] = {8 * ces, ces, (cuuint64_t)T * ces};
+        const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, (cuuint32_t)(tm32::kTc / 8), 8, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        return encode(m, src, 4, dims, strides, box, estr, l2);
+    };
+    auto image_residue = [&](CUtensorMap* m, const void* src) {
+        const cuuint64_t dims[5] = {(cuuint64_t)C, (cuuint64_t)p.W / 8, (cuuint64_t)p.H, 8, (cuuint64_t)B};
+        const cuuint64_t strides[4] = {8 * ces, (cuuint64_t)p.W * ces, ces, (cuuint64_t)p.H * p.W * ces};
+        const cuuint32_t box[5] = {(cuuint32_t)fast::kCS, (cuuint32_t)(p.W / 8), (cuuint32_t)p.rows, 8, 1};
+        const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+        return encode(m, src, 5, dims, strides, box, estr, l2_in);
+    };
+    const bool img = pl.qs && !p.flat;
+    p.imaj = 0;
+    p.nbox = pl.tm && !img ? tm32::kNW : 1;
+    if (pl.tm && !tm_imaj_disabled() && T % 8 == 0 && (!img || p.rows * p.W == tm32::kTc)) {
+        bool okm = true;
+        for (int i = 0; i < nsrc && okm; ++i) {
+            okm = img ? image_residue(&p.map[i], srcs[i]) : flat_residue(&p.map[i], srcs[i], l2_in);
+            if (okm && pl.qs) okm = img ? image_strided(&p.xmap[i], srcs[i], p.rows) : flat_strided(&p.xmap[i], srcs[i], l2_in);
         }
-        if (cr != CUDA_SUCCESS) return false;
-    }
-    {
-        // the output in the tiles' layout: boxes of 256 strided tokens; a CTA
-        // stores by TMA when its span is whole boxes or ends the column, so no
-        // box reaches another CTA's tokens (the tensor bound clips at T).  The
-        // tensor-memory kernel at T a multiple of 256 stores four folds of 256
-        // tokens per box instead (one store per lane), where a CTA spans 1024
-        // tokens or the whole column (a box never reaches another CTA's tokens).
-        p.ofold = pl.tm && T % 256 == 0 && (p.Tc == tm32::kTc || p.ncl == 1) && !tm_ofold_disabled() ? 1 : 0;
-        CUresult cr;
-        if (p.ofold) {
-            const cuuint64_t dims[4] = {(cuuint64_t)C, 256, (cuuint64_t)T / 256, (cuuint64_t)B};
-            const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)256 * C * es, (cuuint64_t)T * C * es};
-            const cuuint32_t box[4] = {(cuuint32_t)fast::kCS, 256u, (cuuint32_t)tm32::kNW, 1};
-            const cuuint32_t estr[4] = {1, (cuuint32_t)fast::kL, 1, 1};
-            cr = enc(&p.omap, dt, 4, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        } else {
-            const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
-            const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
-            const cuuint32_t box[3] = {(cuuint32_t)fast::kCS, 256u, 1};
-            const cuuint32_t estr[3] = {1, (cuuint32_t)fast::kL, 1};
-            cr = enc(&p.omap, dt, 3, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (okm) {
+            p.imaj = 1;
+            p.nbox = 1;
         }
-        p.tma_store = (cr == CUDA_SUCCESS && (p.Tc % 256 == 0 || p.ncl == 1) && !tma_store_disabled()) ? 1 : 0;
     }
+    if (!p.imaj) {
+        for (int i = 0; i < nsrc; ++i) {
+            const bool okm = img ? image_strided(&p.map[i], srcs[i], p.rows) : flat_strided(&p.map[i], srcs[i], l2_in);
+            if (!okm) return false;
+        }
+    }
+    // The output in the tiles' layout: lane-strided boxes of 256 tokens; a
+    // CTA stores by TMA when its span is whole boxes or ends the column, so no
+    // box reaches another CTA's tokens (the tensor bound clips at T).  The
+    // tensor-memory kernel stores through the residue-major view instead, one
+    // box for its 1024 tokens, where T is a multiple of 8 and a CTA spans 1024
+    // tokens or the whole column.
+    p.ofold = pl.tm && T % 8 == 0 && (p.Tc == tm32::kTc || p.ncl == 1) && !tm_ofold_disabled() ? 1 : 0;
+    bool okout = p.ofold ? flat_residue(&p.omap, out, l2_out) : flat_strided(&p.omap, out, l2_out);
+    if (!okout && p.ofold) {
+        p.ofold = 0;
+        okout = flat_strided(&p.omap, out, l2_out);
+    }
+    p.tma_store = (okout && (p.Tc % 256 == 0 || p.ncl == 1) && !tma_store_disabled()) ? 1 : 0;
     p.invT = (float)(1.0 / (double)T);
     p.err = device_error_word();
     if (!p.err) return false;

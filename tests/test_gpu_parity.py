@@ -315,26 +315,29 @@ def test_tm_kernel_shapes(vk, oracle_mod, case, rot, monkeypatch):
     assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tm_kernel"
 
 
-# The tensor-memory kernel's copy shapes: 1, 2 or 4 boxes per lane and tile
-# (one per 1024, 512 or 256 tokens) in the image view with Q-Shift and the
-# folded token view without, and the folded result store on and off.
-NBOX_CASES = [
+# The tensor-memory kernel's copy shapes: each tile in one residue-major box
+# (image view with Q-Shift, flat tokens without or at any W) or in
+# lane-strided boxes, and results stored in one residue-major box or in
+# lane-strided 256-token boxes.
+COPY_CASES = [
     # call, B, H, W, C, dtype
     ("gate_qs_x", 2, 64, 64, 64, "bf16"),     # image view, 16 rows per CTA
     ("gate_qs", 1, 32, 32, 32, "f32"),        # image view, 32 rows per CTA, float32
-    ("biwkv", 2, 1, 3072, 32, "bf16"),        # folded view, 3 CTAs
-    ("gate_x", 1, 1, 1280, 16, "f32"),        # folded view, a second CTA of one fold
-    ("gate_qs_x", 1, 40, 40, 32, "bf16"),     # flat view (W = 40 does not divide 1024)
+    ("qshift_biwkv", 1, 48, 96, 32, "bf16"),  # W = 96: 768-token CTAs (lane-strided loads only)
+    ("biwkv", 2, 1, 3072, 32, "bf16"),        # flat tokens, 3 CTAs
+    ("gate_x", 1, 1, 1288, 16, "f32"),        # flat tokens, a second CTA of 264 tokens
+    ("gate_qs_x", 1, 40, 40, 32, "bf16"),     # W = 40: flat view, shifted tiles lane-strided
+    ("gate", 1, 1, 1000, 16, "bf16"),         # one CTA of 1000 tokens
 ]
 
 
-@pytest.mark.parametrize("ofold", ["1", "0"])
-@pytest.mark.parametrize("nbox", ["1", "2", "4"])
-@pytest.mark.parametrize("case", NBOX_CASES, ids=lambda c: "_".join(map(str, c)))
-def test_tm_box_counts(vk, oracle_mod, case, nbox, ofold, monkeypatch):
+@pytest.mark.parametrize("ostore", ["1", "0"])
+@pytest.mark.parametrize("imaj", ["1", "0"])
+@pytest.mark.parametrize("case", COPY_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_tm_copy_shapes(vk, oracle_mod, case, imaj, ostore, monkeypatch):
     monkeypatch.setenv("VRWKV_FORWARD", "tm")
-    monkeypatch.setenv("VRWKV_TM_NBOX", nbox)
-    monkeypatch.setenv("VRWKV_TM_OFOLD", ofold)
+    monkeypatch.setenv("VRWKV_TM_IMAJ", imaj)
+    monkeypatch.setenv("VRWKV_TM_OSTORE", ostore)
     call, B, H, W, C, dt = case
     wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000)
     run_fused(vk, oracle_mod, wl)
