@@ -69,6 +69,8 @@ struct alignas(64) Params {
     unsigned int* err;   // device error word (bounded TMA wait)
     int tma;             // inputs arrive by TMA
     int tma_store;       // gk, gv leave by TMA stores from shared memory
+    int imaj;            // tensor-memory kernel: map[] and omap[] are residue-major views (one box
+                         // per tile; sub-tile i holds the tokens 8 m + i)
     const char* k;
     const char* v;
     const char* g;  // upstream gradient dL/dy

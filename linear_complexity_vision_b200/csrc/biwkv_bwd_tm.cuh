@@ -150,11 +150,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtas<IO>) biwkv_bwd_tm_kernel(co
     if (multi) fast::cluster_arrive_relaxed();
     const uint32_t tmem = S.tmem + ((uint32_t)(warp * 32) << 16);
 
-    // ---- TMA: lane i of warp 0 loads sub-tile i of k, v and g -------------------
+    // ---- TMA: each of k, v and g in one box from a residue-major view (token
+    // 8 m + i at sub-tile i, row m), or lane i of warp 0 loads sub-tile i in
+    // boxes of 256 strided tokens -------------------------------------------------
     if (warp == 0) {
         if (tid == 0) fast::mbar_expect_tx(&S.tma_bar, (unsigned)(3 * TILE));
         __syncwarp();
-        if (tid < kHL) {
+        if (p.imaj) {
+            if (tid == 0) {
+#pragma unroll
+                for (int s3 = 0; s3 < 3; ++s3)
+                    fast::tma_load_4d(tiles + s3 * TILE, &p.map[s3], c0, t0 / kHL, 0, b, &S.tma_bar);
+            }
+        } else if (tid < kHL) {
 #pragma unroll
             for (int s3 = 0; s3 < 3; ++s3)
 #pragma unroll
@@ -573,10 +581,17 @@ __global__ void __launch_bounds__(kThreads, kMinCtas<IO>) biwkv_bwd_tm_kernel(co
     tm32::tc_fence_before();
     __syncthreads();
     if (tid < kHL) {
-        const int nbox = (tend - t0 + 255) / 256;
-        for (int hb = 0; hb < nbox; ++hb) {
-            fast::tma_store_3d(&p.omap[0], tk + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
-            fast::tma_store_3d(&p.omap[1], tg + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
+        if (p.imaj) {
+            if (tid == 0) {
+                fast::tma_store_4d(&p.omap[0], tk, c0, t0 / kHL, 0, b);
+                fast::tma_store_4d(&p.omap[1], tg, c0, t0 / kHL, 0, b);
+            }
+        } else {
+            const int nbox = (tend - t0 + 255) / 256;
+            for (int hb = 0; hb < nbox; ++hb) {
+                fast::tma_store_3d(&p.omap[0], tk + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
+                fast::tma_store_3d(&p.omap[1], tg + tid * SUB + hb * 32 * RB, c0, t0 + tid + 256 * hb, b);
+            }
         }
         fast::bulk_commit_and_wait_read();
     }

@@ -1917,6 +1917,7 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
                 return fail(VRWKV_ERR_INVALID_ARG, "outputs overlap");
     }
     bwd::Params p;
+    p.imaj = 0;
     p.k = static_cast<const char*>(k);
     p.v = static_cast<const char*>(v);
     p.g = static_cast<const char*>(gy);
@@ -1982,7 +1983,34 @@ vrwkv_status vrwkv_biwkv_bwd(const void* k, const void* v, const float* w, const
         const cuuint32_t estr[3] = {1, (cuuint32_t)bwd::kL, 1};
         void* dsts[2] = {gk, gv};
         bool oks = enc != nullptr;
-        for (int i = 0; i < 2 && oks; ++i)
+        // residue-major views (tokens as (C, T / 8, 8, B), one box per 512-token
+        // tile) where T is a multiple of 8: a CTA's boxes are then one load per
+        // input and one store per output instead of sixteen each
+        p2.imaj = 0;
+        if (oks && T % 8 == 0 && !tm_imaj_disabled()) {
+            const void* srcs[3] = {k, v, gy};
+            const cuuint64_t rdims[4] = {(cuuint64_t)C, (cuuint64_t)T / 8, 8, (cuuint64_t)B};
+            const cuuint64_t rstrides[3] = {(cuuint64_t)8 * C * es, (cuuint64_t)C * es, (cuuint64_t)T * C * es};
+            const cuuint32_t rbox[4] = {(cuuint32_t)bwd::kCS, (cuuint32_t)(bwd2::kTc / 8), 8, 1};
+            const cuuint32_t restr[4] = {1, 1, 1, 1};
+            bool okr = true;
+            for (int i = 0; i < 3 && okr; ++i)
+                okr = enc(&p2.map[i], tdt, 4, const_cast<void*>(srcs[i]), rdims, rstrides, rbox, restr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            for (int i = 0; i < 2 && okr; ++i)
+                okr = enc(&p2.omap[i], tdt, 4, dsts[i], rdims, rstrides, rbox, restr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            if (okr) {
+                p2.imaj = 1;
+            } else {
+                p2.map[0] = p.map[0];
+                p2.map[1] = p.map[1];
+                p2.map[2] = p.map[2];
+            }
+        }
+        for (int i = 0; i < 2 && oks && !p2.imaj; ++i)
             oks = enc(&p2.omap[i], tdt, 3, dsts[i], dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                       CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
