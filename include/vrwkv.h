@@ -149,14 +149,18 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *         load (mu_r is ignored); T must then equal qs->H * qs->W.
  * Kernels (the same results up to rounding):
  *   - the 32-token tensor-memory kernel, the default for T >= 1024: the
- *     8-channel kernel's conditions with 1024-token CTAs (with qs, whole
- *     image rows per CTA, a multiple of 256 tokens when the column needs
- *     more than one CTA), T <= 8192, and the thread-block cluster and
- *     tensor memory of four CTAs per SM available; each thread's per-token
- *     partial sums are kept in tensor memory between its two passes;
- *   - the 8-channel TMA kernel, the default below 1024 tokens: C % 8 == 0,
- *     16-byte-aligned inputs and, with qs, group bounds int(C*gamma*j) that
- *     are multiples of 8 and W <= 256, T <= 8192;
+ *     8-channel kernel's conditions with 1024-token CTAs, T <= 8192, and
+ *     the thread-block cluster and tensor memory of four CTAs per SM
+ *     available; each thread's per-token partial sums are kept in tensor
+ *     memory between its two passes.  Where T is a multiple of 8 a tile
+ *     arrives in one TMA box and the results leave in one;
+ *   - the 8-channel TMA kernel, the default below 1024 tokens (256-token
+ *     CTAs for T <= 256): C % 8 == 0, 16-byte-aligned inputs and, with qs,
+ *     group bounds int(C*gamma*j) that are multiples of 8, T <= 8192.
+ *     Q-Shift reads the image (C, W, H, B) where W % 8 == 0, W <= 256 and
+ *     whole image rows make whole warps, else the flat tokens with the
+ *     shifted tiles displaced by the group's token offset (row-wrapped
+ *     tokens cleared after the load);
  *   - the 16-channel slab kernel, with VRWKV_FORWARD=wide in the
  *     environment (and for long sequences through the workspace variants):
  *     C % 16 == 0, T % 16 == 0, T <= 4096, 16-byte-aligned tensors and,
@@ -167,10 +171,13 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *   Setting VRWKV_DISABLE_TMA=1 in the environment forces the generic
  *   kernel, VRWKV_FORWARD=tm takes the tensor-memory kernel at any T where it
  *   qualifies and VRWKV_FORWARD=narrow never, VRWKV_TM_ROT=0 keeps its
- *   sub-chunks in natural order, VRWKV_DISABLE_WIDE=1 keeps the 16-channel
- *   one off, VRWKV_TMA_CHUNK=8 holds the 8-channel kernel to 8-token thread
- *   chunks and VRWKV_NO_TMA_STORE=1 to per-thread stores of its results
- *   (diagnostics).
+ *   sub-chunks in natural order, VRWKV_TM_IMAJ=0 and VRWKV_TM_OSTORE=0 keep
+ *   its loads and stores on lane-strided boxes, VRWKV_QS_VIEW=flat (image)
+ *   takes Q-Shift through the flat token view wherever it can (never),
+ *   VRWKV_SHORT_CTA=0 keeps short columns on 512-token CTAs,
+ *   VRWKV_DISABLE_WIDE=1 keeps the 16-channel one off, VRWKV_TMA_CHUNK=8
+ *   holds the 8-channel kernel to 8-token thread chunks and
+ *   VRWKV_NO_TMA_STORE=1 to per-thread stores of its results (diagnostics).
  * Limits: T <= 8192 on the 8-channel kernel, 4096 on the others
  *   (UNSUPPORTED above; the workspace variants below reach 32768); on the
  *   generic kernel with qs, a halo of shift_pixel*W tokens must fit its
