@@ -332,10 +332,16 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     // this thread's lane of the CTA's columns
     const uint32_t tmem = S.tmem + ((uint32_t)(warp * 32) << 16);
 
-    // this warp's tokens: every lane waits (bounded) for their boxes; with
-    // Q-Shift in a horizontal group the warp then clears its row-wrapped
-    // tokens of the shifted tiles
-    mbar_wait_bounded(&S.bar[warp / wpb], p.err);
+    // this warp's tokens: with a barrier per warp every lane waits (bounded)
+    // for its boxes; with Q-Shift in a horizontal group the warp then clears
+    // its row-wrapped tokens of the shifted tiles
+    if (nb == 1) {
+        // one barrier: one thread waits, the others sleep at the CTA barrier
+        if (tid == 0) mbar_wait_bounded(&S.bar[0], p.err);
+        __syncthreads();
+    } else {
+        mbar_wait_bounded(&S.bar[warp / wpb], p.err);
+    }
     if (QS && p.flat && shifted && grp < 2) {
         const int lo = t0 + warp * kWarpTok;
         fast::zero_row_wrap<RB>(smem, p.tile_bytes, SUB, NSRC, t0, lo, min(tend, lo + kWarpTok), p.W, p.s,

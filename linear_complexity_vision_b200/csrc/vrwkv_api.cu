@@ -321,6 +321,20 @@ bool bwd_tm_disabled() {
 // The 16-token tensor-memory backward (bwd2::biwkv_bwd_tm_kernel): sets
 // *fell_back when the shape cannot be co-scheduled or more than four CTAs
 // would share an SM.
+// Cluster scheduling policy of the clustered kernels: spread by default
+// (measured on the B200 with the tensor-memory forward at B=8, T=4096,
+// C=1024: 83.0 us against 84.9 us with load balancing);
+// VRWKV_CLUSTER_POLICY=l(oad balancing) or d(efault) for comparisons, and
+// VRWKV_CLUSTER_POLICY_BWD / _NARROW for the backward and 8-channel kernels
+// alone.
+cudaClusterSchedulingPolicy cluster_policy(const char* var) {
+    const char* e = getenv(var);
+    if (!e || !e[0]) e = getenv("VRWKV_CLUSTER_POLICY");
+    if (e && e[0] == 'l') return cudaClusterSchedulingPolicyLoadBalancing;
+    if (e && e[0] == 'd') return cudaClusterSchedulingPolicyDefault;
+    return cudaClusterSchedulingPolicySpread;
+}
+
 template <typename IO>
 vrwkv_status launch_bwd_tm(const bwd::Params& p, cudaStream_t s, bool* fell_back) {
     auto kern = bwd2::biwkv_bwd_tm_kernel<IO>;
@@ -339,7 +353,7 @@ vrwkv_status launch_bwd_tm(const bwd::Params& p, cudaStream_t s, bool* fell_back
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
-    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+    attr[1].val.clusterSchedulingPolicyPreference = cluster_policy("VRWKV_CLUSTER_POLICY_BWD");
     cfg.attrs = attr;
     cfg.numAttrs = p.ncl > 1 ? 2 : 0;
     static std::atomic<int> checked[bwd2::kClusterMax + 1];
@@ -633,7 +647,7 @@ vrwkv_status launch_fast(const FastPlan& pl, cudaStream_t stream, bool* fell_bac
     // let the hardware balance a cluster's CTAs over the SMs (measured with
     // 16-CTA clusters on the B200: 33 instead of 31 co-resident, 3 % faster)
     attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
-    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+    attr[1].val.clusterSchedulingPolicyPreference = cluster_policy("VRWKV_CLUSTER_POLICY_NARROW");
     cfg.attrs = attr;
     cfg.numAttrs = pl.p.ncl > 1 ? 2 : 0;
     if (pl.p.ncl > 1) {
@@ -687,17 +701,6 @@ static_assert(kFastTcMax == fast::Cfg<kFastThreads8, 8>::kTcMax, "one tile geome
 // The 32-token tensor-memory kernel: a cluster per column as in the 8-channel
 // kernel.  Sets *fell_back when the shape cannot be co-scheduled or more
 // than four CTAs would share an SM (their tensor memory would not fit).
-// Cluster scheduling policy of the tensor-memory kernel: spread (measured on
-// the B200 at B=8, T=4096, C=1024: 83.0 us against 84.9 us with load
-// balancing); VRWKV_CLUSTER_POLICY=l(oad balancing) or d(efault) for
-// comparisons.
-cudaClusterSchedulingPolicy tm_cluster_policy() {
-    const char* e = getenv("VRWKV_CLUSTER_POLICY");
-    if (e && e[0] == 'l') return cudaClusterSchedulingPolicyLoadBalancing;
-    if (e && e[0] == 'd') return cudaClusterSchedulingPolicyDefault;
-    return cudaClusterSchedulingPolicySpread;
-}
-
 template <typename IO, int LAYOUT, bool QS, bool ROT, bool GX>
 vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back) {
     auto kern = tm32::biwkv_tm_kernel<IO, LAYOUT, QS, ROT, GX>;
@@ -715,7 +718,7 @@ vrwkv_status launch_tm(const FastPlan& pl, cudaStream_t stream, bool* fell_back)
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
-    attr[1].val.clusterSchedulingPolicyPreference = tm_cluster_policy();
+    attr[1].val.clusterSchedulingPolicyPreference = cluster_policy("VRWKV_CLUSTER_POLICY_TM");
     cfg.attrs = attr;
     cfg.numAttrs = (!GX && pl.p.ncl > 1) ? 2 : 0;  // GX: a plain 1-D grid of tickets
     // checked once per (cluster size, shared memory)
