@@ -30,10 +30,10 @@
  *   vrwkv_spatial_gate_static.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *   default stream).  Work is enqueued asynchronously; the caller
- *   synchronises.  vrwkv_spatial_gate, vrwkv_channel_mix and
- *   vrwkv_spatial_mix_block enqueue kernel launches only and are replayed
- *   from CUDA graphs by the benchmark; capture of the other calls has not
- *   been tested.
+ *   synchronises.  vrwkv_spatial_gate (and its _ws variant),
+ *   vrwkv_channel_mix, vrwkv_spatial_mix_block and vrwkv_biwkv_bwd enqueue
+ *   kernel launches only and are replayed from CUDA graphs by the benchmark;
+ *   capture of the other calls has not been tested.
  * Dtypes.  VRWKV_F32 or VRWKV_BF16 select the storage type of the token
  *   tensors (inputs and output alike).  Arithmetic is float32 throughout;
  *   bfloat16 outputs are rounded to nearest even once, at the store.

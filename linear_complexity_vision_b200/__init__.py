@@ -422,18 +422,27 @@ def spatial_mix_block(x, weights, w, u, ln_gamma, ln_beta, qs: QShift, ln_eps: f
     return out
 
 
-def biwkv_bwd(k, v, w, u, gy, totals: bool = True):
+def biwkv_bwd(k, v, w, u, gy, totals: bool = True, out=None):
     """Gradients of eq. 5 for the upstream gradient gy: gk, gv (B, T, C) in
     the input dtype, gw, gu float32 (B, C) per batch row and, if totals, their
-    sums over the batch (float32 (C,)); otherwise those two are None."""
+    sums over the batch (float32 (C,)); otherwise those two are None.
+    out: optional (gk, gv, gw, gu) to write instead of allocating them."""
     import torch
     _require_tokens(("k", k), ("v", v), ("gy", gy))
     B, T, C = k.shape
     for t, name in ((w, "w"), (u, "u")):
         _require_vec(t, C, k.device, name)
-    gk, gv = torch.empty_like(k), torch.empty_like(k)
-    gw = torch.empty((B, C), dtype=torch.float32, device=k.device)
-    gu = torch.empty((B, C), dtype=torch.float32, device=k.device)
+    if out is None:
+        gk, gv = torch.empty_like(k), torch.empty_like(k)
+        gw = torch.empty((B, C), dtype=torch.float32, device=k.device)
+        gu = torch.empty((B, C), dtype=torch.float32, device=k.device)
+    else:
+        gk, gv, gw, gu = out
+        _require_tokens(("k", k), ("gk", gk), ("gv", gv))
+        for t, name in ((gw, "gw"), (gu, "gu")):
+            if (t.dtype != torch.float32 or t.device != k.device or not t.is_contiguous()
+                    or t.numel() != B * C):
+                raise ValueError(f"{name} must be a contiguous float32 tensor of B*C elements on {k.device}")
     gwt = torch.empty(C, dtype=torch.float32, device=k.device) if totals else None
     gut = torch.empty(C, dtype=torch.float32, device=k.device) if totals else None
     _check(load_library().vrwkv_biwkv_bwd(

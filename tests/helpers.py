@@ -42,3 +42,9 @@ def scaled_error(got, want, scale):
 def biwkv_scale(oracle, k, v, w, u):
     """S_t: the eq. 5 weighted mean of |v| (computed by the RNN form)."""
     return oracle.biwkv_rnn(k, np.abs(v), w, u)
+
+
+def plain_relative_error(got, want, floor=1e-6):
+    """max |got - want| / max(|want|, floor): the plain relative error, for
+    information (outputs that cancel to ~0 inflate it)."""
+    return float(np.max(np.abs(got - want) / np.maximum(np.abs(want), floor)))

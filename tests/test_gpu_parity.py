@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 from linear_complexity_vision_b200 import synth
-from helpers import (TOL, biwkv_scale, scaled_error, to_device, to_numpy, torch_dtype,
+from helpers import (TOL, plain_relative_error, biwkv_scale, scaled_error, to_device, to_numpy, torch_dtype,
                      vec_f32)
 
 pytestmark = pytest.mark.gpu
@@ -99,6 +99,10 @@ def _custom(call, B, H, W, C, dt, seed, s=1, gamma=0.25, **d):
                           shift_pixel=s, gamma=gamma, seed=seed)
 
 
+# The last run_fused call's error figures (for tests that report them).
+_LAST = {}
+
+
 # Workspace of the global-exchange kernels, shared by every "gx" test on the
 # one stream (the kernels leave it ready for the next call).
 _GX = {"on": False, "ws": None}
@@ -171,6 +175,15 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
     tol = TOL[dt]
     err = scaled_error(got, want, scale)
     assert err <= tol, f"{wl.name}: scaled error {err:.3e} > {tol}"
+    # the plain relative error where the weighted mean does not cancel
+    # (|wkv| at least half the weighted mean of |v|): bounded by 2 tol
+    well = np.abs(want) >= 0.5 * scale
+    if well.any():
+        plain = plain_relative_error(got[well], want[well])
+        assert plain <= 2 * tol, f"{wl.name}: plain relative error {plain:.3e} > {2 * tol}"
+    _LAST["plain_all"] = plain_relative_error(got, want)
+    _LAST["plain_well"] = plain_relative_error(got[well], want[well]) if well.any() else 0.0
+    _LAST["scaled"] = err
     if not small:
         rng = np.random.default_rng(wl.seed)
         idx = rng.choice(got.size, size=min(got.size, 3000), replace=False)
@@ -223,6 +236,22 @@ def kernel_path(request, monkeypatch):
 def test_workload_full_size(vk, oracle_mod, cfg, kernel_path):
     wl = synth.WORKLOADS[cfg]
     run_fused(vk, oracle_mod, wl)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+def test_plain_relative_error_reported(vk, oracle_mod, cfg, record_property, monkeypatch, capsys):
+    # The parity bar is the scaled error (|delta| / S_t, S_t the eq. 5-weighted
+    # mean of |v|); the plain max |delta| / max(|wkv|, 1e-6) is reported beside
+    # it, over all outputs and over those where |wkv| >= S_t / 2.
+    for name in ("VRWKV_FORWARD", "VRWKV_QS_VIEW", "VRWKV_SHORT_CTA", "VRWKV_DISABLE_TMA"):
+        monkeypatch.delenv(name, raising=False)
+    wl = synth.WORKLOADS[cfg]
+    run_fused(vk, oracle_mod, wl)
+    for k in ("scaled", "plain_all", "plain_well"):
+        record_property(k, _LAST[k])
+    with capsys.disabled():
+        print(f"\n{wl.name}: scaled {_LAST['scaled']:.3e}, plain (all) {_LAST['plain_all']:.3e}, "
+              f"plain (|wkv| >= S/2) {_LAST['plain_well']:.3e}")
 
 
 @pytest.mark.parametrize("cfg", [4, 5])
