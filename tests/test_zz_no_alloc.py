@@ -35,11 +35,12 @@ def _inputs(B, H, W, C, dt, seed):
 
 
 @pytest.mark.parametrize("dt,B,H,W,C", [
-    ("bf16", 2, 64, 64, 64),    # 8 CTAs of 512 tokens per column: the exchange runs in the static workspace
-    ("f32", 1, 40, 40, 64),     # 8-token chunks, 8 rows of 40 per CTA: 5 CTAs per column
-    ("bf16", 1, 128, 64, 64),   # 16 CTAs per column: every flag and record slot of a column
+    ("bf16", 2, 64, 64, 64),    # tensor-memory kernel, 4 CTAs of 1024 tokens per column exchanging in the static workspace
+    ("f32", 1, 40, 40, 64),     # W = 40: flat-view Q-Shift, CTAs of 1024 and 576 tokens
+    ("bf16", 1, 128, 64, 64),   # T = 8192: 16-channel kernel, two 4096-token segments meeting in the static workspace
     ("bf16", 8, 64, 64, 1024),  # 1024 columns: the full-size workload
-    ("bf16", 2, 14, 14, 96),    # one CTA per column: no exchange
+    ("bf16", 2, 14, 14, 96),    # one 256-token CTA per column: no exchange
+    ("bf16", 2, 25, 40, 64),    # T = 1000: 8-channel kernel, 4 CTAs of 8 image rows exchanging in the static workspace
 ])
 def test_static_matches_spatial_gate_twice(vk, oracle_mod, dt, B, H, W, C):
     import torch
