@@ -89,3 +89,15 @@ def test_public_calls_refuse_before_launch():
     w4 = tuple(FakeCuda((C, C)) for _ in range(3)) + (FakeCuda((C, C + 1)),)
     with pytest.raises(ValueError, match=r"weights\[3\]"):
         vk.spatial_mix_block(tok(), w4, vec(), vec(), vec(), vec(), vk.QShift(14, 14))
+
+
+def test_backward_outputs_are_checked():
+    k, v, g = tok(), tok(), tok()
+    good_rows = FakeCuda((B, C), dtype=torch.float32)
+    with pytest.raises(ValueError, match="gv must match"):
+        vk.biwkv_bwd(k, v, vec(), vec(), g, out=(tok(), FakeCuda((B, T, C + 8)), good_rows, good_rows))
+    with pytest.raises(ValueError, match="gw must be a contiguous float32"):
+        vk.biwkv_bwd(k, v, vec(), vec(), g, out=(tok(), tok(), FakeCuda((B, C)), good_rows))
+    with pytest.raises(ValueError, match="gu must be a contiguous float32"):
+        vk.biwkv_bwd(k, v, vec(), vec(), g, out=(tok(), tok(), good_rows, FakeCuda((B, C + 1), dtype=torch.float32)))
+
