@@ -216,9 +216,10 @@ vrwkv_status vrwkv_spatial_gate(const void* r, const void* k, const void* v,
  * with the host <-> device traffic overlapped with the computation.  The
  * batch is cut into slices of slice_b rows (each (b, c) column is
  * independent and Q-Shift mixes tokens of one batch row only, so a slice is
- * an exact sub-problem); slice i is copied host -> device into slot i % 2 of
- * dev_buf on a library copy stream, computed on `stream`, and copied back on
- * a second copy stream, so both copy directions and the kernels overlap.
+ * an exact sub-problem); slice i is copied host -> device into slot i % n of
+ * dev_buf (n = 3 slots, or 2 when dev_buf holds only two) on a library copy
+ * stream, computed on `stream`, and copied back on a second copy stream, so
+ * both copy directions and the kernels overlap.
  * Results equal vrwkv_spatial_gate's bit for bit.
  *   r, k, v   (B, T, C) inputs in page-locked host memory (cudaHostAlloc or
  *             cudaHostRegister); they may be the same buffer, copied once.
@@ -246,9 +247,9 @@ vrwkv_status vrwkv_spatial_gate_host(const void* r, const void* k,
                                      int slice_b, void* dev_buf,
                                      size_t dev_buf_bytes, void* stream);
 
-/* Device staging bytes vrwkv_spatial_gate_host needs for slices of slice_b
- * batch rows with `inputs` (1 to 3) distinct input buffers; 0 for invalid
- * arguments. */
+/* Device staging bytes vrwkv_spatial_gate_host uses for slices of slice_b
+ * batch rows with `inputs` (1 to 3) distinct input buffers (three slots; two
+ * thirds of it is the minimum it accepts); 0 for invalid arguments. */
 size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C,
                                             vrwkv_dtype dtype, int inputs);
 

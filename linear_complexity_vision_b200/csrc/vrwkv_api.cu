@@ -1471,6 +1471,9 @@ vrwkv_status fused_entry(bool gate, const void* r, const void* k, const void* v,
 // ---------------------------------------------------------------------------
 size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
 
+// Device slots of the host pipeline (staging for one slice each).
+constexpr int kHostSlots = 3;
+
 size_t host_slot_bytes(int slice_b, int T, int C, int es, int inputs) {
     const size_t tensor = (size_t)slice_b * T * C * es;
     return (size_t)(inputs + 1) * round256(tensor);
@@ -1482,7 +1485,7 @@ size_t host_slot_bytes(int slice_b, int T, int C, int es, int inputs) {
 // threads onto them.
 struct HostPipe {
     cudaStream_t in = nullptr, outs = nullptr;
-    cudaEvent_t start = nullptr, loaded[2] = {}, done[2] = {}, freed[2] = {};
+    cudaEvent_t start = nullptr, loaded[kHostSlots] = {}, done[kHostSlots] = {}, freed[kHostSlots] = {};
     bool ok = false;
 };
 
@@ -1496,7 +1499,7 @@ HostPipe* host_pipe(int dev) {
         bool good = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
                     cudaStreamCreateWithFlags(&p.outs, cudaStreamNonBlocking) == cudaSuccess &&
                     cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess;
-        for (int i = 0; i < 2 && good; ++i)
+        for (int i = 0; i < kHostSlots && good; ++i)
             good = cudaEventCreateWithFlags(&p.loaded[i], cudaEventDisableTiming) == cudaSuccess &&
                    cudaEventCreateWithFlags(&p.done[i], cudaEventDisableTiming) == cudaSuccess &&
                    cudaEventCreateWithFlags(&p.freed[i], cudaEventDisableTiming) == cudaSuccess;
@@ -1550,6 +1553,9 @@ vrwkv_status host_pipeline(const void* r, const void* k, const void* v, const fl
     if (dev_buf_bytes < 2 * slot)
         return fail(VRWKV_ERR_INVALID_ARG, "device buffer holds %zu bytes; slices of %d rows need %zu",
                     dev_buf_bytes, slice_b, 2 * slot);
+    // as many slots as the buffer holds, up to three: with three, a slice's
+    // copy in never waits for the copy out of the slice two before it
+    const int nslots = (int)std::min<size_t>(kHostSlots, dev_buf_bytes / slot);
     if (!aligned(dev_buf, 256)) return fail(VRWKV_ERR_INVALID_ARG, "device buffer must be 256-byte aligned");
     for (const void* p : {r, k, v, (const void*)out})
         if (!host_pinned(p))
@@ -1577,10 +1583,11 @@ vrwkv_status host_pipeline(const void* r, const void* k, const void* v, const fl
         return VRWKV_ERR_CUDA;
     const int nslices = (B + slice_b - 1) / slice_b;
     for (int i = 0; i < nslices; ++i) {
-        const int sl = i & 1;
+        const int sl = i % nslots;
         const int b0 = i * slice_b, nb = std::min(slice_b, B - b0);
         const size_t off = (size_t)b0 * row, n = (size_t)nb * row;
-        if (i >= 2 && !check(cudaStreamWaitEvent(hp->in, hp->freed[sl], 0), "stream wait")) return VRWKV_ERR_CUDA;
+        if (i >= nslots && !check(cudaStreamWaitEvent(hp->in, hp->freed[sl], 0), "stream wait"))
+            return VRWKV_ERR_CUDA;
         for (int j = 0; j < inputs; ++j) {
             int src = 0;
             while (slot_of[src] != j) ++src;
@@ -2103,7 +2110,7 @@ size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C, vrwkv_dty
     if (slice_b <= 0 || T <= 0 || C <= 0 || inputs < 1 || inputs > 3 ||
         (dtype != VRWKV_F32 && dtype != VRWKV_BF16))
         return 0;
-    return 2 * host_slot_bytes(slice_b, T, C, elem_bytes(dtype), inputs);
+    return kHostSlots * host_slot_bytes(slice_b, T, C, elem_bytes(dtype), inputs);
 }
 
 vrwkv_status vrwkv_spatial_gate_host(const void* r, const void* k, const void* v, const float* w,

@@ -226,10 +226,10 @@ def test_host_buffer_bytes(lib):
     f = lib.vrwkv_spatial_gate_host_buffer_bytes
     f.argtypes = [ctypes.c_int] * 5
     f.restype = ctypes.c_size_t
-    # two slots of (inputs + 1) tensors of slice_b * T * C elements, 256-byte rounded
-    assert f(1, 4096, 1024, 1, 1) == 2 * 2 * 4096 * 1024 * 2
-    assert f(2, 196, 768, 0, 3) == 2 * 4 * ((2 * 196 * 768 * 4 + 255) // 256 * 256)
-    assert f(1, 3, 5, 1, 1) == 2 * 2 * 256
+    # three slots of (inputs + 1) tensors of slice_b * T * C elements, 256-byte rounded
+    assert f(1, 4096, 1024, 1, 1) == 3 * 2 * 4096 * 1024 * 2
+    assert f(2, 196, 768, 0, 3) == 3 * 4 * ((2 * 196 * 768 * 4 + 255) // 256 * 256)
+    assert f(1, 3, 5, 1, 1) == 3 * 2 * 256
     for bad in ((0, 16, 16, 1, 1), (1, 16, 16, 1, 0), (1, 16, 16, 1, 4), (1, 16, 16, 7, 1)):
         assert f(*bad) == 0
 

@@ -59,6 +59,22 @@ def test_host_pipeline_equals_device_call(vk, dt, B, H, W, C, distinct, slice_b)
         assert torch.equal(out, want)
 
 
+def test_host_pipeline_with_two_slots(vk):
+    # a staging buffer of two slots (the minimum) gives the same results
+    import torch
+    B, H, W, C = 5, 32, 32, 256
+    r, k, v, w, u, mus = _setup(B, H, W, C, "bf16", False, seed=4321)
+    qs = vk.QShift(H, W, 1, 0.25, *mus)
+    want = vk.spatial_gate(r.cuda(), k.cuda(), v.cuda(), w, u, qs=qs).cpu()
+    full = vk.spatial_gate_host_buffer(r, k, v, 1)
+    two = full[: full.numel() * 2 // 3]
+    out = torch.full_like(k, float("nan")).pin_memory()
+    vk.spatial_gate_host(r, k, v, w, u, qs=qs, out=out, slice_b=1, dev_buf=two)
+    torch.cuda.current_stream().synchronize()
+    vk.device_status()
+    assert torch.equal(out, want)
+
+
 def test_host_pipeline_rejects_pageable_memory(vk):
     import torch
     x = torch.zeros(2, 16, 32, dtype=torch.bfloat16)  # not page-locked
