@@ -916,6 +916,41 @@ __global__ void __launch_bounds__(256) transpose_kernel(const T* __restrict__ w,
     }
 }
 
+// The same transpose for 16-bit elements two at a time: 64 x 64 tiles, each
+// thread moving 4-byte pairs (rows of a warp access are 128 bytes instead of
+// 64), the tile's rows padded to 33 words (at most 2-way bank conflicts when
+// a warp reads a column of pairs).  Needs K and N even and every pointer
+// 4-byte aligned.
+// Up to four matrices in one launch: blockIdx.z picks the pair (w, wt).
+template <typename T>
+struct TransposeBatch {
+    const T* w[4];
+    T* wt[4];
+};
+template <typename T>
+__global__ void __launch_bounds__(256) transpose2_kernel(const __grid_constant__ TransposeBatch<T> tb, int K, int N) {
+    static_assert(sizeof(T) == 2, "16-bit elements");
+    __shared__ uint32_t tile[64][33];  // [k][pair of n]
+    const T* __restrict__ w = tb.w[blockIdx.z];
+    T* __restrict__ wt = tb.wt[blockIdx.z];
+    const int k0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    for (int r = ty; r < 64; r += 8) {
+        const int k = k0 + r, n = n0 + 2 * tx;
+        tile[r][tx] = (k < K && n < N) ? *reinterpret_cast<const uint32_t*>(w + (size_t)k * N + n) : 0u;
+    }
+    __syncthreads();
+    for (int c = ty; c < 64; c += 8) {
+        const int n = n0 + c, k = k0 + 2 * tx;
+        if (n < N && k < K) {
+            const uint32_t a = tile[2 * tx][c >> 1], b = tile[2 * tx + 1][c >> 1];
+            const uint32_t lo = (c & 1) ? (a >> 16) : (a & 0xffffu);
+            const uint32_t hi = (c & 1) ? (b >> 16) : (b & 0xffffu);
+            *reinterpret_cast<uint32_t*>(wt + (size_t)n * K + k) = lo | (hi << 16);
+        }
+    }
+}
+
 // float32 projections on the FP32 pipes (the bfloat16 path above is the
 // tensor-core one): D = A W with W (K x N) row-major, 64 x 64 tiles, 4 x 4
 // results per thread.

@@ -234,8 +234,35 @@ int sm_count() {
 // D (M x N) = X (M x K) * W (K x N), all row-major.  bfloat16: W is first
 // transposed into wt (N x K, the K-major B operand) and the product runs on
 // the tensor cores with float32 accumulation; float32: on the FP32 pipes.
+// n matrices W[i] (K x N, bfloat16, row-major) -> wt[i] (N x K) in one
+// launch, two elements per thread access; false (nothing launched) unless
+// the sizes are even and every pointer 4-byte aligned.
+bool launch_transpose_pairs(const void* const* W, void* const* wt, int n, int K, int N, cudaStream_t s) {
+    if (n < 1 || n > 4 || K % 2 != 0 || N % 2 != 0) return false;
+    tcgemm::TransposeBatch<__nv_bfloat16> tb{};
+    for (int i = 0; i < n; ++i) {
+        if (!aligned(W[i], 4) || !aligned(wt[i], 4)) return false;
+        tb.w[i] = static_cast<const __nv_bfloat16*>(W[i]);
+        tb.wt[i] = static_cast<__nv_bfloat16*>(wt[i]);
+    }
+    const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((K + 63) / 64), (unsigned)n);
+    tcgemm::transpose2_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(tb, K, N);
+    return true;
+}
+
+// W (K x N, bfloat16, row-major) -> wt (N x K): pairs of elements per thread
+// where the sizes are even and the pointers 4-byte aligned, else one.
+vrwkv_status launch_transpose(const void* W, void* wt, int K, int N, cudaStream_t s) {
+    if (!launch_transpose_pairs(&W, &wt, 1, K, N, s)) {
+        const dim3 grid((unsigned)((N + 31) / 32), (unsigned)((K + 31) / 32));
+        tcgemm::transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(W),
+                                                                      static_cast<__nv_bfloat16*>(wt), K, N);
+    }
+    return cuda_status(cudaGetLastError(), "transpose launch");
+}
+
 vrwkv_status gemm_project(const void* X, const void* W, void* D, int M, int N, int K, vrwkv_dtype dtype,
-                          void* wt, cudaStream_t s) {
+                          void* wt, cudaStream_t s, bool wt_ready = false) {
     if (dtype == VRWKV_F32) {
         const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64));
         tcgemm::gemm_f32_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(X), static_cast<const float*>(W),
@@ -243,11 +270,8 @@ vrwkv_status gemm_project(const void* X, const void* W, void* D, int M, int N, i
         return cuda_status(cudaGetLastError(), "gemm_f32_kernel launch");
     }
     if (K % 8 != 0) return fail(VRWKV_ERR_UNSUPPORTED, "bfloat16 projections need C %% 8 == 0");
-    {
-        const dim3 grid((unsigned)((N + 31) / 32), (unsigned)((K + 31) / 32));
-        tcgemm::transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(W),
-                                                                      static_cast<__nv_bfloat16*>(wt), K, N);
-        vrwkv_status st = cuda_status(cudaGetLastError(), "transpose_kernel launch");
+    if (!wt_ready) {  // else the caller transposed W into wt already
+        vrwkv_status st = launch_transpose(W, wt, K, N, s);
         if (st != VRWKV_OK) return st;
     }
     EncodeTiledFn enc = encode_fn();
@@ -420,9 +444,13 @@ bool gemm_qs_project(const void* x, const void* const* wts, const float* const* 
     }
     for (int i = 0; i < 3; ++i) {
         void* wt = wt_slots + i * wslot;
-        const dim3 grid((unsigned)((C + 31) / 32), (unsigned)((C + 31) / 32));
-        tcgemm::transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(wts[i]),
-                                                                      static_cast<__nv_bfloat16*>(wt), C, C);
+        {
+            const vrwkv_status e = launch_transpose(wts[i], wt, C, C, s);
+            if (e != VRWKV_OK) {
+                *st = e;
+                return true;
+            }
+        }
         const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)C};
         const cuuint64_t strides[1] = {(cuuint64_t)C * 2};
         const cuuint32_t box[2] = {(cuuint32_t)tcgemm::BK, (cuuint32_t)tcgemm::pair::kHalf};
@@ -1814,6 +1842,7 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     const void* wts[3] = {w_r, w_k, w_v};
     void* dst[3] = {bR, bK, bV};
     vrwkv_status qst = VRWKV_OK;
+    bool wo_ready = false;  // W_O already transposed (with the other three)
     // bfloat16: the mixes as the projections' A-operand producer (one fused
     // launch, nothing staged in HBM) where the shape allows
     const bool fused = dtype == VRWKV_BF16 && block_fused_wanted() && !gemm_single_cta_forced() &&
@@ -1831,8 +1860,12 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
                 if (st != VRWKV_OK) return st;
             }
         }
+        // the four weights transposed in one launch where it applies
+        const void* w4[4] = {w_r, w_k, w_v, w_o};
+        void* wt4[4] = {wts_t, wts_t + wslot, wts_t + 2 * wslot, wts_t + 3 * wslot};
+        wo_ready = dtype == VRWKV_BF16 && launch_transpose_pairs(w4, wt4, 4, C, C, s);
         for (int i = 0; i < 3; ++i) {
-            vrwkv_status st = gemm_project(sh[i], wts[i], dst[i], M, C, C, dtype, wts_t + i * wslot, s);
+            vrwkv_status st = gemm_project(sh[i], wts[i], dst[i], M, C, C, dtype, wts_t + i * wslot, s, wo_ready);
             if (st != VRWKV_OK) return st;
         }
     }
@@ -1841,7 +1874,7 @@ vrwkv_status vrwkv_spatial_mix_block(const void* x, const void* w_r, const void*
     vrwkv_status st = vrwkv_spatial_gate(bR, bK, bV, w, u, t0, B, T, C, dtype, nullptr, stream);
     if (st != VRWKV_OK) return st;
     // W_O into the R buffer (dead after the gate), then LayerNorm into out
-    st = gemm_project(t0, w_o, bR, M, C, C, dtype, wts_t + 3 * wslot, s);
+    st = gemm_project(t0, w_o, bR, M, C, C, dtype, wts_t + 3 * wslot, s, wo_ready);
     if (st != VRWKV_OK) return st;
     LayerNormParams lp;
     lp.x = static_cast<const char*>(bR);
