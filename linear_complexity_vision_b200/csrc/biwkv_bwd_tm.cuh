@@ -263,9 +263,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtas<IO>) biwkv_bwd_tm_kernel(co
     __syncthreads();
     {
         // CTA scan, in every thread for its own pair (no warp waits for a
-        // serial scan in warp 0; measured 6.3 us of a 20 us CTA that way):
-        // the exclusive carries into this thread's warp, and the CTA's
-        // records from the lanes of chunk 0
+        // serial scan in warp 0): the exclusive carries into this thread's
+        // warp, and the CTA's records from the lanes of chunk 0
         const float L = (float)kWarpTok;
         const float2 aW = decay(lam2, L);  // across one warp's tokens
         R1 acc = r1_zero(), xw = r1_zero();
