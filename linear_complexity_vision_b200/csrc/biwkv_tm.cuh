@@ -31,6 +31,13 @@
 // A CTA covers 1024 tokens x 8 channels; longer columns use a cluster of up
 // to 8 CTAs along T (T <= 8192) exchanging their aggregates through
 // asynchronous shared-memory stores, as in the 8-channel kernel.
+//
+// Copies: the TMA's cost grows with the number of boxes, so where T is a
+// multiple of 8 a whole tile arrives in one box from a residue-major view
+// (token 8 m + i lands at sub-tile i, row m) and the CTA's results leave in
+// one store; elsewhere lane i of warp 0 moves sub-tile i in lane-strided
+// boxes.  Q-Shift reads the image view where W allows and the flat token
+// view otherwise (see the loads below).
 #pragma once
 
 #include "biwkv_tma.cuh"

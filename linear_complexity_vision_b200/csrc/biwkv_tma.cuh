@@ -24,12 +24,17 @@
 //    16-token chunks), and every address is a compile-time offset from one
 //    base register.
 //  * With Q-Shift the (B, T, C) tensor is described as the 4-D image
-//    (C, W, H, B) (W a multiple of 8); the shifted tile x_shift is the same
-//    set of boxes displaced by +-s along w or h.  TMA fills out-of-image
-//    elements with zeros, which is exactly Q-Shift's zero border, so no
-//    per-token shift arithmetic remains: token t of both tiles sits at the
-//    same shared-memory offset.  A CTA's kCS channels lie in one channel
-//    group (the host requires the group size to be a multiple of kCS).
+//    (C, W, H, B) (W a multiple of 8, at most 256); the shifted tile x_shift
+//    is the same set of boxes displaced by +-s along w or h.  TMA fills
+//    out-of-image elements with zeros, which is exactly Q-Shift's zero
+//    border, so no per-token shift arithmetic remains: token t of both tiles
+//    sits at the same shared-memory offset.  Any other W takes the flat
+//    token view: the shifted tile is displaced by the group's token offset
+//    and its row-wrapped tokens are cleared after the load (zero_row_wrap).
+//    A CTA's kCS channels lie in one channel group (the host requires the
+//    group bounds to be multiples of kCS).
+//  * Columns of at most 256 tokens (a 14 x 14 grid: 196) run 64-thread CTAs
+//    of 256 tokens; longer ones 128-thread CTAs of 512.
 //  * Four CTAs per SM (128 threads at <= 128 registers, or 256 at 64), so
 //    one CTA's barriers and scans overlap another's arithmetic.  Sequences
 //    longer than 512 tokens split over a thread-block cluster along T (8
