@@ -148,13 +148,13 @@ vrwkv_status vrwkv_bishift(const void* x, void* out, const float* mu, int B,
  *   qs    NULL, or Q-Shift parameters applied to k (mu_k) and v (mu_v) on
  *         load (mu_r is ignored); T must then equal qs->H * qs->W.
  * Kernels (the same results up to rounding):
- *   - the 32-token tensor-memory kernel, the default for T >= 1024: the
+ *   - the 32-token tensor-memory kernel, the default for T > 512: the
  *     8-channel kernel's conditions with 1024-token CTAs, T <= 8192, and
  *     the thread-block cluster and tensor memory of four CTAs per SM
  *     available; each thread's per-token partial sums are kept in tensor
  *     memory between its two passes.  Where T is a multiple of 8 a tile
  *     arrives in one TMA box and the results leave in one;
- *   - the 8-channel TMA kernel, the default below 1024 tokens (256-token
+ *   - the 8-channel TMA kernel, the default up to 512 tokens (256-token
  *     CTAs for T <= 256): C % 8 == 0, 16-byte-aligned inputs and, with qs,
  *     group bounds int(C*gamma*j) that are multiples of 8, T <= 8192.
  *     Q-Shift reads the image (C, W, H, B) where W % 8 == 0, W <= 256 and
@@ -258,8 +258,8 @@ size_t vrwkv_spatial_gate_host_buffer_bytes(int slice_b, int T, int C,
  * operations, arguments and results.  Up to 4096 tokens, the CTAs of one
  * (b, 8-channel) column exchange their partial sums through the caller's
  * workspace instead of a thread-block cluster, which frees the kernel from
- * cluster co-scheduling (the 32-token tensor-memory kernel from 1024 tokens,
- * the 8-channel kernel below).  Longer sequences (up to T = 32768, e.g. the
+ * cluster co-scheduling (the 32-token tensor-memory kernel above 512 tokens,
+ * the 8-channel kernel up to 512).  Longer sequences (up to T = 32768, e.g. the
  * 16384 tokens of a 2048^2 image at patch 16) run on the 16-channel kernel
  * when the shape qualifies for it: a column splits into segments of one
  * 8-CTA cluster (4096 tokens); segments take tickets from a counter in the

@@ -1116,16 +1116,18 @@ bool wide_preferred() {
     return e && e[0] == 'w';
 }
 
-// The 32-token tensor-memory kernel takes columns of 1024 tokens and more
-// (measured on the B200 at C = 1024: 80.5 against 95.8 us at T = 1024, but
-// 130 against 74 us at T = 256, where most of its threads have no token);
+// The 32-token tensor-memory kernel takes columns of more than 512 tokens,
+// which the 8-channel kernel would split over a cluster (measured on the
+// B200 at C = 1024: 91.0 against 112.2 us at T = 768, 76.2 against 94.4 us
+// at T = 1024, but 105.3 against 64.0 us at T = 512, where the 8-channel
+// kernel needs one CTA and most tensor-memory threads have no token);
 // VRWKV_FORWARD=tm takes it wherever it qualifies, VRWKV_FORWARD=narrow
 // never.
 bool tm_wanted(int T) {
     const char* e = getenv("VRWKV_FORWARD");
     if (e && e[0] == 't') return true;
     if (e && e[0]) return false;
-    return T >= 1024;
+    return T > 512;
 }
 
 struct WidePlan {

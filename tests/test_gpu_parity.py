@@ -198,7 +198,7 @@ def run_fused(vk, oracle, wl, mu_none=False, kshift=0.0, return_out=False):
 @pytest.fixture(params=["default", "narrow", "flat", "tm", "wide", "tma8", "gx", "generic"])
 def kernel_path(request, monkeypatch):
     """Run a test on the default path (the 32-token tensor-memory kernel for
-    columns of 1024 tokens and more, else the 8-channel TMA kernel with
+    columns of more than 512 tokens, else the 8-channel TMA kernel with
     16-token thread chunks, on 256-token CTAs for columns of at most 256
     tokens, where the shape and cluster geometry allow), on the latter alone
     ("narrow"), on it with Q-Shift through the flat token view everywhere and

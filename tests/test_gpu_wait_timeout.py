@@ -38,14 +38,20 @@ def _inputs(B, T, C):
     return k, v, w, u
 
 
-@pytest.mark.parametrize("T,kernel", [(1000, "biwkv_tma_kernel"), (2048, "biwkv_tm_kernel")])
-def test_workspace_peer_wait_runs_out_and_is_reported(vk, oracle_mod, T, kernel):
+@pytest.mark.parametrize("T,kernel,forward", [(1000, "biwkv_tma_kernel", "narrow"),
+                                              (2048, "biwkv_tm_kernel", None)])
+def test_workspace_peer_wait_runs_out_and_is_reported(vk, oracle_mod, T, kernel, forward, monkeypatch):
     import torch
     # fast paths without Q-Shift, one 8-channel slab: 512-token CTAs of the
-    # 8-channel kernel at T = 1000, 1024-token CTAs of the 32-token kernel at
-    # T = 2048, so the grid holds exactly two CTAs, ranks 0 and 1 of one
-    # column (the CTA that finds its ticket past the grid leaves before it
-    # takes any tensor memory)
+    # 8-channel kernel at T = 1000 (held to it: the default there is the
+    # 32-token kernel), 1024-token CTAs of the 32-token kernel at T = 2048, so
+    # the grid holds exactly two CTAs, ranks 0 and 1 of one column (the CTA
+    # that finds its ticket past the grid leaves before it takes any tensor
+    # memory)
+    if forward:
+        monkeypatch.setenv("VRWKV_FORWARD", forward)
+    else:
+        monkeypatch.delenv("VRWKV_FORWARD", raising=False)
     B, C = 1, 8
     k, v, w, u = _inputs(B, T, C)
     kt, kd = to_device(k, "bf16")

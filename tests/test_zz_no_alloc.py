@@ -40,7 +40,7 @@ def _inputs(B, H, W, C, dt, seed):
     ("bf16", 1, 128, 64, 64),   # T = 8192: 16-channel kernel, two 4096-token segments meeting in the static workspace
     ("bf16", 8, 64, 64, 1024),  # 1024 columns: the full-size workload
     ("bf16", 2, 14, 14, 96),    # one 256-token CTA per column: no exchange
-    ("bf16", 2, 25, 40, 64),    # T = 1000: 8-channel kernel, 4 CTAs of 8 image rows exchanging in the static workspace
+    ("bf16", 2, 25, 40, 64),    # T = 1000: one tensor-memory CTA per column (flat view: W = 40)
 ])
 def test_static_matches_spatial_gate_twice(vk, oracle_mod, dt, B, H, W, C):
     import torch
@@ -56,6 +56,23 @@ def test_static_matches_spatial_gate_twice(vk, oracle_mod, dt, B, H, W, C):
         assert torch.equal(got, want)
         err = scaled_error(got.double().cpu().numpy(), want_default.double().cpu().numpy(), scale)
         assert err <= TOL[dt], err
+
+
+def test_static_8_channel_exchange(vk, oracle_mod, monkeypatch):
+    # the 8-channel kernel held to (the default at T = 1000 is the 32-token
+    # kernel): 8-token chunks, 4 CTAs of 8 image rows per column exchanging in
+    # the static workspace, twice in a row, bit-equal to the workspace call
+    import torch
+    monkeypatch.setenv("VRWKV_FORWARD", "narrow")
+    B, H, W, C = 2, 25, 40, 64
+    x, _, (w, u, *mus), _ = _inputs(B, H, W, C, "bf16", seed=1000)
+    qs = vk.QShift(H, W, 1, 0.25, *mus)
+    want = vk.spatial_gate(x, x, x, w, u, qs=qs, workspace=vk.fwd_workspace(B, H * W, C))
+    assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tma_kernel"
+    for _ in range(2):
+        got = vk.spatial_gate_static(x, x, x, w, u, qs=qs, out=torch.empty_like(x))
+        vk.device_status()
+        assert torch.equal(got, want)
 
 
 def test_static_long_sequence_matches_workspace_call(vk):
