@@ -344,6 +344,28 @@ def test_tm_kernel_shapes(vk, oracle_mod, case, rot, monkeypatch):
     assert vk.load_library().vrwkv_last_kernel().decode() == "biwkv_tm_kernel"
 
 
+# The default selection on both sides of its switch: the 8-channel kernel up
+# to 512 tokens, the tensor-memory kernel (one CTA per column) above.
+SWITCH_CASES = [
+    # call, B, H, W, C, dtype, kernel
+    ("gate_qs_x", 2, 16, 32, 64, "bf16", "biwkv_tma_kernel"),   # T = 512
+    ("biwkv", 2, 1, 512, 16, "f32", "biwkv_tma_kernel"),         # T = 512, no Q-Shift
+    ("biwkv", 2, 1, 513, 16, "bf16", "biwkv_tm_kernel"),         # T = 513: 17 chunks, one holding a token
+    ("gate_qs_x", 2, 24, 32, 64, "bf16", "biwkv_tm_kernel"),    # T = 768, image view
+    ("gate_qs", 1, 25, 40, 32, "f32", "biwkv_tm_kernel"),       # T = 1000, W = 40: flat view
+]
+
+
+@pytest.mark.parametrize("case", SWITCH_CASES, ids=lambda c: "_".join(map(str, c[:6])))
+def test_default_forward_switch(vk, oracle_mod, case, monkeypatch):
+    for name in ("VRWKV_FORWARD", "VRWKV_QS_VIEW", "VRWKV_SHORT_CTA", "VRWKV_DISABLE_TMA", "VRWKV_TM_ROT"):
+        monkeypatch.delenv(name, raising=False)
+    call, B, H, W, C, dt, kernel = case
+    wl = _custom(call, B, H, W, C, dt, seed=zlib.crc32(repr(case).encode()) % 100000)
+    run_fused(vk, oracle_mod, wl)
+    assert vk.load_library().vrwkv_last_kernel().decode() == kernel
+
+
 # The tensor-memory kernel's copy shapes: each tile in one residue-major box
 # (image view with Q-Shift, flat tokens without or at any W) or in
 # lane-strided boxes, and results stored in one residue-major box or in
