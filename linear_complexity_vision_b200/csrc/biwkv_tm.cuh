@@ -467,7 +467,9 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
             ga = fma2(alpha, ga, vv[ib]);
             gc = fma2(alpha, gc, kk[ib]);
         }
-        tmem_st32(tmem + h * 32, nd);
+        // columns by step, not by sub-chunk: tcgen05.st takes one address for
+        // the warp, and the output pass reads step st back at step st
+        tmem_st32(tmem + st * 32, nd);
         Fh[st] = make_float4(fa.x, fa.y, fc.x, fc.y);
         Gh[st] = make_float4(ga.x, ga.y, gc.x, gc.y);
     }
@@ -716,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
     for (int st = 0; st < kH; ++st) {
         const int h = ROT ? (st + rot) & (kH - 1) : st;
         float nd[32];
-        tmem_ld32(tmem + h * 32, nd);
+        tmem_ld32(tmem + st * 32, nd);  // the sums of sub-chunk h, stored at this step
         const float2 sh = mul2(slw, eh[st]);
         const float4 L4 = ROT ? X2.a[h][tid] : Lc[st], R4 = ROT ? X2.b[h][tid] : Rc[st];
         const float2 Ah = lo2(L4), Ch = hi2(L4), Bh = lo2(R4), Dh = hi2(R4);
