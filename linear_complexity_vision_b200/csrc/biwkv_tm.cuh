@@ -644,24 +644,21 @@ __global__ void __launch_bounds__(kThreads, 4) biwkv_tm_kernel(const __grid_cons
         // the CTAs before this one, the backward ones of those after it, each
         // CTA a decay of a^Tc further
         const float2 aTc = ex2c(mul2(lam2, f2(-(float)p.Tc)));
+        // (loops of exactly the peers' count: rank and ncl are the same in
+        // every thread of the CTA)
         float2 Mc = f2(-INFINITY);
-#pragma unroll
-        for (int r = 0; r < kClusterMax; ++r)
-            if (r < p.ncl) Mc = max2(Mc, S.mbM[r][j]);
+#pragma unroll 1
+        for (int r = 0; r < p.ncl; ++r) Mc = max2(Mc, S.mbM[r][j]);
         float4 accF = zero4(), accG = zero4();
-#pragma unroll
-        for (int r = 0; r < kClusterMax; ++r) {
-            if (r < rank) {
-                const float2 sc = ex2(add2(S.mbM[r][j], make_float2(-Mc.x, -Mc.y)));
-                accF = fma4(aTc, accF, scale4(sc, S.mbF[r][j]));
-            }
+#pragma unroll 1
+        for (int r = 0; r < rank; ++r) {
+            const float2 sc = ex2(add2(S.mbM[r][j], make_float2(-Mc.x, -Mc.y)));
+            accF = fma4(aTc, accF, scale4(sc, S.mbF[r][j]));
         }
-#pragma unroll
-        for (int r = kClusterMax - 1; r >= 0; --r) {
-            if (r > rank && r < p.ncl) {
-                const float2 sc = ex2(add2(S.mbM[r][j], make_float2(-Mc.x, -Mc.y)));
-                accG = fma4(aTc, accG, scale4(sc, S.mbG[r][j]));
-            }
+#pragma unroll 1
+        for (int r = p.ncl - 1; r > rank; --r) {
+            const float2 sc = ex2(add2(S.mbM[r][j], make_float2(-Mc.x, -Mc.y)));
+            accG = fma4(aTc, accG, scale4(sc, S.mbG[r][j]));
         }
         cs_sl = ex2(add2(ownM, make_float2(-Mc.x, -Mc.y)));
         cs_af = lo2(accF);
