@@ -155,8 +155,10 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x2: "applications_clocks_setting", 0x10: "sync_boost", 0x1: "gpu_idle"}
 
-    def __init__(self, local_rank: int, period_s: float = 0.01):
+    def __init__(self, local_rank: int, period_s: float = 0.01,
+                 window: str = "pre-roll of the same launches (~0.3 s) + the timed region"):
         self.samples, self.reasons = [], 0
+        self.window = window
         self.max_mhz = None
         self.ok = False
         self.period = period_s
@@ -209,8 +211,16 @@ class ClockSampler:
             return None
         return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "samples": len(self.samples),
-                "window": "pre-roll of the same launches (~0.3 s) + the timed region",
+                "window": self.window,
                 "reasons": sorted(n for b, n in self.REASONS.items() if self.reasons & b)}
+
+
+def row_clocks(dev) -> ClockSampler:
+    """SM clocks sampled every 2 ms over one row's timed region (a row times
+    tens of milliseconds, after other rows that may have heated the GPU)."""
+    c = ClockSampler(dev.index or 0, period_s=0.002, window="the row's timed region")
+    c.start()
+    return c
 
 
 # ---------------------------------------------------------------------------
@@ -383,12 +393,14 @@ def time_channel_mix(runner, stream, torch, dev, launches: int, peak: float):
     reps = max(1, launches // G)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
+    row_clk = row_clocks(dev)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(reps):
             graph.replay()
         e1.record(stream)
     torch.cuda.synchronize(dev)
+    row_clk.stop()
     del graph
     us = e0.elapsed_time(e1) * 1e3 / (reps * G)
     es = 4 if wl.dtype == "f32" else 2
@@ -399,7 +411,7 @@ def time_channel_mix(runner, stream, torch, dev, launches: int, peak: float):
             "traffic": committed_traffic("channel_mix/" + wl.name, runner.kernel_name),
             "kernel": runner.kernel_name,
             "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
-            "launches": reps * G}
+            "launches": reps * G, "clocks": row_clk.summary()}
 
 
 def time_fused_ws(runner, stream, torch, dev, launches: int, peak: float):
@@ -437,12 +449,14 @@ def time_fused_ws(runner, stream, torch, dev, launches: int, peak: float):
     reps = max(1, launches // G)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
+    row_clk = row_clocks(dev)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(reps):
             graph.replay()
         e1.record(stream)
     torch.cuda.synchronize(dev)
+    row_clk.stop()
     del graph
     vk.device_status()
     us = e0.elapsed_time(e1) * 1e3 / (reps * G)
@@ -451,7 +465,7 @@ def time_fused_ws(runner, stream, torch, dev, launches: int, peak: float):
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "kernel": runner.kernel_name,
             "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us, "launches": reps * G,
-            "exchange": "global-memory workspace (no clusters)"}
+            "exchange": "global-memory workspace (no clusters)", "clocks": row_clk.summary()}
 
 
 def measured_tensor_peak():
@@ -503,12 +517,14 @@ def time_block(runner, stream, torch, dev, launches: int):
     reps = max(1, launches // G)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
+    row_clk = row_clocks(dev)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(reps):
             graph.replay()
         e1.record(stream)
     torch.cuda.synchronize(dev)
+    row_clk.stop()
     del graph
     vk.device_status()
     us = e0.elapsed_time(e1) * 1e3 / (reps * G)
@@ -522,7 +538,7 @@ def time_block(runner, stream, torch, dev, launches: int):
             "gemm": ("hand-written tcgen05 kernel, bf16 operands, float32 accumulation in tensor memory: "
                      + ("gemm_tc_kernel (one CTA per 128x256 tile)" if os.environ.get("VRWKV_GEMM_1CTA") == "1"
                         else "gemm_tc2_kernel (CTA pairs, cta_group::2, 256x256 tiles)")),
-            "timing": "CUDA graphs over the rotating buffer sets"}
+            "timing": "CUDA graphs over the rotating buffer sets", "clocks": row_clk.summary()}
 
 
 def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float, sm_mhz=None):
@@ -564,11 +580,13 @@ def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float, sm_mh
                 launch(i)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    row_clk = row_clocks(dev)
     with torch.cuda.stream(stream):
         e0.record(stream)
         graph.replay()
         e1.record(stream)
     torch.cuda.synchronize(dev)
+    row_clk.stop()
     del graph
     us = e0.elapsed_time(e1) * 1e3 / launches
     es = 4 if wl.dtype == "f32" else 2
@@ -581,7 +599,8 @@ def time_biwkv_bwd(runner, stream, torch, dev, launches: int, peak: float, sm_mh
             "frac": achieved / peak, "traffic": committed_traffic("biwkv_bwd/" + wl.name, kname),
             "kernel": kname, "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": us,
             "issue_roofline": issue,
-            "launches": launches, "timing": "one CUDA graph of the launches (preallocated outputs)"}
+            "launches": launches, "timing": "one CUDA graph of the launches (preallocated outputs)",
+            "clocks": row_clk.summary()}
 
 
 def parity_sample(runner, out_dev, oracle, npts=128):
